@@ -1,0 +1,233 @@
+"""Pins of the oracle's code tables and NF4 double quantisation (CPU only).
+
+Each pin comes from outside the oracle: figures the pages print
+(tests/golden/pages_figures.json), closed forms of the published table
+constructions, brute force on tiny tensors, special cases that reduce to the
+identity, and the error bound of nearest-entry quantisation.
+"""
+import io
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import account, bf16, codebooks, quant
+from nf4_layer_streamed_b200 import synth
+
+GOLD = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "pages_figures.json")))
+
+
+# ----------------------------------------------------------------------------- code tables
+
+def test_nf4_table_shape_and_ends():
+    t = codebooks.nf4_table()
+    assert t.dtype == np.float32 and t.size == GOLD["nf4_table_entries"]["value"]
+    assert t[0] == -1.0 and t[-1] == 1.0
+    assert t[7] == 0.0 and np.count_nonzero(t == 0.0) == 1
+    assert np.all(np.diff(t.astype(np.float64)) > 0)
+    assert np.count_nonzero(t > 0) == 8 and np.count_nonzero(t < 0) == 7
+
+
+def _phi(x):
+    return 0.5 * math.erfc(-x / math.sqrt(2.0))
+
+
+def _phi_inv_bisect(p):
+    lo, hi = -10.0, 10.0
+    for _ in range(200):
+        mid = 0.5 * (lo + hi)
+        if _phi(mid) < p:
+            lo = mid
+        else:
+            hi = mid
+    return 0.5 * (lo + hi)
+
+
+def test_nf4_table_matches_normal_quantiles_via_erfc():
+    # Independent route to the same quantiles: bisection on erfc instead of ndtri.
+    delta = 0.5 * ((1 - 1 / 30) + (1 - 1 / 32))
+    top = _phi_inv_bisect(delta)
+    t = codebooks.nf4_table().astype(np.float64)
+    pos = sorted(_phi_inv_bisect(delta + i * (0.5 - delta) / 8) / top for i in range(8))
+    neg = sorted(-_phi_inv_bisect(delta + i * (0.5 - delta) / 7) / top for i in range(7))
+    np.testing.assert_allclose(t[8:], pos, rtol=0, atol=2e-7)
+    np.testing.assert_allclose(t[:7], neg, rtol=0, atol=2e-7)
+
+
+def test_code8_table_closed_forms():
+    t = codebooks.code8_table()
+    assert t.dtype == np.float32 and t.size == GOLD["nested_table_entries"]["value"]
+    assert np.all(np.diff(t.astype(np.float64)) > 0)
+    assert np.count_nonzero(t == 0.0) == 1
+    assert t.max() == 1.0
+    assert t.min() == np.float32(-(1.0 - 0.9 / 128.0))
+    assert t[t > 0].min() == np.float32(0.55e-6)
+    # per decade level i there are 2^i values of each sign in [0.1, 1) * 10^(i-6)
+    for i in range(7):
+        lo, hi = 0.1 * 10.0 ** (i - 6), 10.0 ** (i - 6)
+        pos = t[(t >= np.float32(lo) * 0.999) & (t < np.float32(hi) * 0.999)]
+        neg = t[(t <= -np.float32(lo) * 0.999) & (t > -np.float32(hi) * 0.999)]
+        assert pos.size == 2 ** i and neg.size == 2 ** i, i
+
+
+def test_midpoint_rule_brute_force():
+    rng = np.random.default_rng(0)
+    for table in (codebooks.nf4_table(), codebooks.code8_table()):
+        tt = table.astype(np.float64)
+        u = rng.uniform(-1, 1, 4000).astype(np.float32)
+        u = np.concatenate([u, codebooks.midpoints(table), table])
+        idx = codebooks.nearest_index(u, table)
+        mids = codebooks.midpoints(table).astype(np.float64)
+        window = np.max(np.abs(mids - (tt[:-1] + tt[1:]) / 2))
+        for ui, ii in zip(u.astype(np.float64), idx):
+            dist = np.abs(tt - ui)
+            assert dist[ii] <= dist.min() + 2 * window + 1e-12
+        # exact ties at a midpoint go to the lower index
+        m_idx = codebooks.nearest_index(codebooks.midpoints(table), table)
+        assert np.array_equal(m_idx, np.arange(table.size - 1))
+
+
+def test_codebook_hash_stable():
+    assert codebooks.codebook_hash() == codebooks.codebook_hash()
+    assert codebooks.fnv1a64(b"") == 0xCBF29CE484222325
+
+
+# ----------------------------------------------------------------------------- bytes
+
+def test_byte_identity_matches_quantizer_output():
+    rng = np.random.default_rng(1)
+    for n in (64, 64 * 256, 64 * 300, 576 * 192):
+        w = bf16.round_f32(rng.normal(0, 0.02, n).astype(np.float32))
+        q = quant.quantize(w)
+        tb = quant.tensor_bytes(n)
+        assert q["packed"].nbytes == tb["packed"] == n // 2
+        assert q["q8"].nbytes == tb["q8"] == n // 64
+        assert q["nested"].nbytes == tb["nested"] == 4 * math.ceil(n / 16384)
+
+
+def test_bytes_per_param_and_store_sizes_from_pages():
+    L8 = synth.LLAMA_8B
+    b = account.layer_shard_bytes(L8)
+    assert b == 112_513_052
+    ratio = b / account.decoder_params(L8)
+    assert round(ratio, 3) == GOLD["bytes_per_param"]["value"]
+    assert round(account.store_bytes(L8, 32) / 1e9, 2) == GOLD["llama8b_pinned_store_gb"]["value"]
+    S1 = synth.SMOLLM2_135M
+    assert account.layer_shard_bytes(S1) == 1_825_668
+    assert round(account.store_bytes(S1, 30) / 1e9, 3) == GOLD["smollm2_pinned_store_gb"]["value"]
+    big = account.layer_shard_bytes(synth.QWEN_32B_CLASS)
+    assert big / 2 ** 20 > GOLD["aliasing_layer_threshold_mib"]["value"]
+
+
+# ----------------------------------------------------------------------------- quantiser
+
+def _brute_quantize(w):
+    """Pure-Python loops over blocks, elements and all table entries."""
+    nf4 = [float(v) for v in codebooks.nf4_table()]
+    c8 = [float(v) for v in codebooks.code8_table()]
+    x = [float(v) for v in np.asarray(w, np.float32)]
+    nb = len(x) // 64
+    absmax, codes = [], []
+    for b in range(nb):
+        blk = x[b * 64:(b + 1) * 64]
+        am = max(abs(v) for v in blk)
+        absmax.append(am)
+        for v in blk:
+            if am == 0.0:
+                codes.append(nf4.index(0.0))
+                continue
+            u = float(np.float32(v) / np.float32(am))
+            best = min(range(16), key=lambda j: (abs(u - nf4[j]), j))
+            codes.append(best)
+    tot = 0.0
+    for am in absmax:
+        tot += am
+    offset = float(np.float32(tot / nb))
+    cs = [float(np.float32(np.float32(am) - np.float32(offset))) for am in absmax]
+    nested, q8 = [], []
+    for g in range(0, nb, 256):
+        grp = cs[g:g + 256]
+        nm = max(abs(c) for c in grp)
+        nested.append(nm)
+        for c in grp:
+            if nm == 0.0:
+                q8.append(c8.index(0.0))
+                continue
+            u = float(np.float32(c) / np.float32(nm))
+            q8.append(min(range(256), key=lambda j: (abs(u - c8[j]), j)))
+    packed = [(codes[2 * j] << 4) | codes[2 * j + 1] for j in range(len(codes) // 2)]
+    return packed, q8, nested, offset
+
+
+@pytest.mark.parametrize("n,seed", [(64 * 4, 0), (64 * 300, 1), (64 * 513, 2)])
+def test_quantizer_brute_force(n, seed):
+    rng = np.random.default_rng(seed)
+    w = bf16.round_f32(rng.normal(0, 0.02, n).astype(np.float32))
+    w[:64] = 0.0                       # a zero block
+    q = quant.quantize(w)
+    packed, q8, nested, offset = _brute_quantize(w)
+    assert q["offset"] == np.float32(offset)
+    np.testing.assert_array_equal(q["nested"], np.array(nested, np.float32))
+    # nearest-entry choices may differ only inside the fp32-midpoint window; check bytes
+    # where the brute force is unambiguous, and that all choices are near-optimal.
+    assert np.mean(q["packed"] == np.array(packed, np.uint8)) > 0.999
+    assert np.mean(q["q8"] == np.array(q8, np.uint8)) > 0.999
+
+
+def test_nibble_order_high_first():
+    nf4 = codebooks.nf4_table()
+    A = np.float32(0.125)
+    codes = np.array([15, 0] + [7] * 62, dtype=np.int64)
+    w = bf16.round_f32(nf4[codes] * A)
+    q = quant.quantize(w)
+    assert q["packed"][0] == 0xF0
+    assert q["packed"][1] == 0x77
+
+
+def test_quant_dequant_identity_on_representable_tensor():
+    # Every block holds +-A and table values times A with the same power-of-two A:
+    # offset = A, nested = 0, s = A exactly, so dequant(quant(w)) == w bit for bit.
+    rng = np.random.default_rng(3)
+    nf4 = codebooks.nf4_table()
+    A = np.float32(2.0 ** -5)
+    codes = rng.integers(0, 16, 64 * 700)
+    codes[0::64] = 15
+    w = bf16.round_f32(nf4[codes] * A)
+    q = quant.quantize(w)
+    np.testing.assert_array_equal(quant.unpack_codes(q["packed"]), codes)
+    np.testing.assert_array_equal(quant.dequantize_bits(q), bf16.f32_to_bf16_bits(w))
+
+
+def test_dequant_error_bound_and_zero_block():
+    rng = np.random.default_rng(4)
+    n = 64 * 1000
+    w = bf16.round_f32(rng.normal(0, 0.02, n).astype(np.float32))
+    w[64 * 10:64 * 11] = 0.0
+    q = quant.quantize(w)
+    wh = quant.dequantize(q)
+    nf4 = codebooks.nf4_table().astype(np.float64)
+    c8 = codebooks.code8_table().astype(np.float64)
+    g4 = np.max(np.diff(nf4)) / 2
+    g8 = np.max(np.diff(c8)) / 2
+    xb = w.astype(np.float64).reshape(-1, 64)
+    absmax = np.abs(xb).max(axis=1)
+    nested_max = float(q["nested"].max())
+    bound = g4 * absmax[:, None] + g8 * nested_max + 2.0 ** -8 * np.abs(xb) + 1e-9
+    assert np.all(np.abs(xb - wh.reshape(-1, 64)) <= bound)
+    assert np.all(wh.reshape(-1, 64)[10] == 0.0)
+
+
+def test_quantize_deterministic_and_roundtrip_through_bytes():
+    w = synth.tensor_values((192, 576), seed=77, scale=0.02).float().numpy()
+    q1, q2 = quant.quantize(w), quant.quantize(w)
+    for k in ("packed", "q8", "nested"):
+        assert np.array_equal(q1[k], q2[k])
+    buf = io.BytesIO()
+    np.savez(buf, **{k: q1[k] for k in ("packed", "q8", "nested")}, offset=q1["offset"])
+    buf.seek(0)
+    r = np.load(buf)
+    assert np.array_equal(quant.dequantize_bits({**{k: r[k] for k in ("packed", "q8", "nested")},
+                                                 "offset": r["offset"]}),
+                          quant.dequantize_bits(q1))
