@@ -1,0 +1,373 @@
+"""Python face of libnf4ls: the C-ABI calls with torch tensors as buffers.
+
+Marshalling only: torch allocates device and pinned memory and supplies streams;
+every computation is a call into libnf4ls.so (binding.py).  Function names follow
+the C ABI (include/nf4ls.h): nf4_quantize_shard, layer_forward, layer_backward,
+stream_prefetch and the pool, model and building-block calls.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+from . import binding as B
+from .synth import LayerShape, Workload
+
+LAYER_TENSORS = ("q", "k", "v", "o", "gate", "up", "down", "norm_in", "norm_post")
+
+
+def _p(t) -> ctypes.c_void_p:
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _s(stream=None) -> ctypes.c_void_p:
+    st = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(st.cuda_stream)
+
+
+def _aligned(t: torch.Tensor, a: int = 256) -> torch.Tensor:
+    assert t.data_ptr() % a == 0, "buffer is not aligned"
+    return t
+
+
+def _buffer(nbytes: int, device="cuda") -> torch.Tensor:
+    return _aligned(torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device))
+
+
+def layer_cfg(shape: LayerShape, batch: int, seq: int) -> B.LayerCfg:
+    return B.LayerCfg(shape.hidden, shape.inter, shape.n_q, shape.n_kv, shape.head_dim, batch, seq,
+                      shape.rope_theta, shape.rms_eps, shape.lora_r, shape.lora_alpha)
+
+
+def codebooks():
+    nf4 = np.zeros(16, np.float32)
+    c8 = np.zeros(256, np.float32)
+    h = ctypes.c_uint64()
+    B.call("nf4ls_codebooks", nf4.ctypes.data, c8.ctypes.data, ctypes.byref(h))
+    return nf4, c8, h.value
+
+
+def set_gemm_path(path: int) -> None:
+    B.call("nf4ls_set_gemm_path", path)
+
+
+def device_error():
+    out = (ctypes.c_int32 * 4)()
+    st = B.call_status("nf4ls_device_error", ctypes.cast(out, ctypes.c_void_p))
+    return st, list(out)
+
+
+# ----------------------------------------------------------------------------- NF4 tensors
+
+def nf4_quantize_tensor(w: torch.Tensor, stream=None) -> dict:
+    """bf16 device tensor -> dict(packed, q8, nested, offset) of device tensors."""
+    assert w.dtype == torch.bfloat16 and w.is_cuda and w.is_contiguous()
+    n = w.numel()
+    dev = w.device
+    packed = _buffer(n // 2, dev)[: n // 2]
+    q8 = _buffer(n // 64, dev)[: n // 64]
+    nested = torch.empty((n // 64 + 255) // 256, dtype=torch.float32, device=dev)
+    offset = torch.empty(1, dtype=torch.float32, device=dev)
+    scratch_bytes = B.lib().nf4ls_quantize_scratch_bytes(n)
+    scratch = _buffer(scratch_bytes, dev)
+    B.call("nf4_quantize_tensor", _p(w), n, _p(packed), _p(q8), _p(nested), _p(offset), _p(scratch),
+           scratch_bytes, _s(stream))
+    return {"packed": packed, "q8": q8, "nested": nested, "offset": offset, "n": n, "_scratch": scratch}
+
+
+def nf4_dequantize_tensor(q: dict, stream=None) -> torch.Tensor:
+    n = q["n"]
+    out = torch.empty(n, dtype=torch.bfloat16, device=q["packed"].device)
+    B.call("nf4_dequantize_tensor", _p(q["packed"]), _p(q["q8"]), _p(q["nested"]), _p(q["offset"]), n, _p(out),
+           _s(stream))
+    return out
+
+
+# ----------------------------------------------------------------------------- shards
+
+def shard_bytes(cfg: B.LayerCfg) -> int:
+    return B.lib().nf4ls_shard_bytes(ctypes.byref(cfg))
+
+
+def shard_quantized_bytes(cfg: B.LayerCfg) -> int:
+    return B.lib().nf4ls_shard_quantized_bytes(ctypes.byref(cfg))
+
+
+def nf4_quantize_shard(cfg: B.LayerCfg, weights: dict, fingerprint: int = 0, out: torch.Tensor | None = None,
+                       stream=None) -> torch.Tensor:
+    """Quantises one layer (dict of bf16 device tensors) into a device shard (uint8)."""
+    nbytes = shard_bytes(cfg)
+    dev = weights["q"].device
+    shard = out if out is not None else _buffer(nbytes, dev)
+    ptrs = (ctypes.c_void_p * 9)(*[weights[n].contiguous().data_ptr() for n in LAYER_TENSORS])
+    sb = B.lib().nf4ls_shard_scratch_bytes(ctypes.byref(cfg))
+    scratch = _buffer(sb, dev)
+    used = ctypes.c_size_t()
+    B.call("nf4_quantize_shard", ctypes.byref(cfg), ctypes.cast(ptrs, ctypes.c_void_p), fingerprint, _p(shard),
+           shard.numel(), ctypes.byref(used), _p(scratch), sb, _s(stream))
+    return shard[:nbytes] if out is None else shard
+
+
+def shard_check(header: torch.Tensor, cfg: B.LayerCfg | None, fingerprint: int = 0) -> int:
+    h = header[:1024].cpu().contiguous()
+    return B.call_status("nf4ls_shard_check", _p(h), ctypes.byref(cfg) if cfg is not None else None, fingerprint)
+
+
+# ----------------------------------------------------------------------------- layer calls
+
+def _lora_struct(lora: dict | None):
+    if lora is None:
+        return None
+    return B.Lora(lora["A_q"].data_ptr(), lora["B_q"].data_ptr(), lora["A_v"].data_ptr(), lora["B_v"].data_ptr())
+
+
+class LayerWorkspace:
+    def __init__(self, cfg: B.LayerCfg, device="cuda"):
+        self.nbytes = B.lib().nf4ls_workspace_bytes(ctypes.byref(cfg))
+        self.buf = _buffer(self.nbytes, device)
+
+
+def layer_forward(cfg: B.LayerCfg, shard: torch.Tensor, lora: dict | None, x: torch.Tensor,
+                  ws: LayerWorkspace | None = None, y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    ws = ws or LayerWorkspace(cfg, x.device)
+    y = torch.empty_like(x) if y is None else y
+    lo = _lora_struct(lora)
+    B.call("layer_forward", ctypes.byref(cfg), _p(shard), ctypes.byref(lo) if lo else None, _p(x), _p(y),
+           _p(ws.buf), ws.nbytes, _s(stream))
+    return y
+
+
+def layer_backward(cfg: B.LayerCfg, shard: torch.Tensor, lora: dict | None, x: torch.Tensor, dy: torch.Tensor,
+                   ws: LayerWorkspace | None = None, dx: torch.Tensor | None = None, grads: dict | None = None,
+                   stream=None):
+    ws = ws or LayerWorkspace(cfg, x.device)
+    dx = torch.empty_like(x) if dx is None else dx
+    lo = _lora_struct(lora)
+    gs = None
+    if lora is not None:
+        if grads is None:
+            grads = {"dA_q": torch.empty_like(lora["A_q"]), "dB_q": torch.empty_like(lora["B_q"]),
+                     "dA_v": torch.empty_like(lora["A_v"]), "dB_v": torch.empty_like(lora["B_v"])}
+        gs = B.LoraGrads(grads["dA_q"].data_ptr(), grads["dB_q"].data_ptr(), grads["dA_v"].data_ptr(),
+                         grads["dB_v"].data_ptr())
+    B.call("layer_backward", ctypes.byref(cfg), _p(shard), ctypes.byref(lo) if lo else None, _p(x), _p(dy), _p(dx),
+           ctypes.byref(gs) if gs else None, _p(ws.buf), ws.nbytes, _s(stream))
+    return dx, grads
+
+
+def mse_loss(out: torch.Tensor, stream=None):
+    """loss = mean(out^2) (fp32 device scalar), dout = bf16(2 out / n)."""
+    n = out.numel()
+    dout = torch.empty_like(out)
+    loss = torch.empty(1, dtype=torch.float32, device=out.device)
+    npart = 256
+    partial = torch.empty(npart, dtype=torch.float32, device=out.device)
+    B.call("nf4ls_mse_loss", _p(out), n, _p(dout), _p(loss), _p(partial), npart, _s(stream))
+    return loss, dout
+
+
+def gemm_bf16(A: torch.Tensor, Bm: torch.Tensor, b_trans: bool = False, stream=None) -> torch.Tensor:
+    """out = A B^T (B [N, K]) or, with b_trans, out = A B (B [K, N]); tcgen05 kernel."""
+    M, K = A.shape
+    N = Bm.shape[1] if b_trans else Bm.shape[0]
+    out = torch.empty(M, N, dtype=torch.bfloat16, device=A.device)
+    B.call("nf4ls_gemm_bf16", _p(A), _p(Bm), _p(out), M, N, K, int(b_trans), N, _s(stream))
+    return out
+
+
+def gemm_nf4(A: torch.Tensor, q: dict, rows: int, cols: int, dgrad: bool = False, stream=None) -> torch.Tensor:
+    """out = A W^T (forward) or A W (dgrad) with W [rows, cols] given as an NF4 tensor dict."""
+    M = A.shape[0]
+    N = cols if dgrad else rows
+    out = torch.empty(M, N, dtype=torch.bfloat16, device=A.device)
+    B.call("nf4ls_gemm_nf4", _p(A), A.stride(0), M, _p(q["packed"]), _p(q["q8"]), _p(q["nested"]),
+           _p(q["offset"]), rows, cols, int(dgrad), _p(out), N, _s(stream))
+    return out
+
+
+def attention_fwd(cfg: B.LayerCfg, q, k, v, ld_q: int, ld_kv: int, stream=None):
+    M = cfg.batch * cfg.seq
+    o = torch.empty(M, cfg.n_q * cfg.head_dim, dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty(cfg.batch, cfg.n_q, cfg.seq, dtype=torch.float32, device=q.device)
+    B.call("nf4ls_attention_fwd", ctypes.byref(cfg), _p(q), _p(k), _p(v), ld_q, ld_kv, _p(o), _p(lse), _s(stream))
+    return o, lse
+
+
+# ----------------------------------------------------------------------------- streaming pool
+
+class Pool:
+    """n-deep HBM slot pool filled from a pinned host store (nf4ls_pool_*)."""
+
+    def __init__(self, store: torch.Tensor, offsets, sizes, depth: int, slot_bytes: int | None = None,
+                 device="cuda"):
+        assert store.is_pinned(), "the host store must be page-locked"
+        self.store = store
+        n = len(offsets)
+        self.offsets = (ctypes.c_size_t * n)(*offsets)
+        self.sizes = (ctypes.c_size_t * n)(*sizes)
+        self.slot_bytes = slot_bytes or (max(sizes) + 255) // 256 * 256
+        self.slots = _buffer(depth * self.slot_bytes, device)
+        self.handle = ctypes.c_void_p()
+        B.call("nf4ls_pool_create", _p(store), ctypes.cast(self.offsets, ctypes.c_void_p),
+               ctypes.cast(self.sizes, ctypes.c_void_p), n, depth, _p(self.slots), self.slot_bytes,
+               ctypes.byref(self.handle))
+
+    def prefetch(self, layer: int) -> int:
+        return B.call_status("nf4ls_pool_prefetch", self.handle, layer)
+
+    def stream_prefetch(self, layer: int, stream=None) -> int:
+        out = ctypes.c_void_p()
+        B.call("stream_prefetch", self.handle, layer, _s(stream), ctypes.byref(out))
+        return out.value
+
+    def release(self, layer: int, stream=None) -> None:
+        B.call("nf4ls_pool_release", self.handle, layer, _s(stream))
+
+    def wait(self, layer: int, timeout_ms: int) -> int:
+        return B.call_status("nf4ls_wait", self.handle, layer, timeout_ms)
+
+    def set_poison(self, on: bool) -> None:
+        B.call("nf4ls_pool_set_poison", self.handle, int(on))
+
+    def stats(self) -> dict:
+        s = B.PoolStats()
+        B.call("nf4ls_pool_get_stats", self.handle, ctypes.byref(s))
+        return {"bytes_copied": s.bytes_copied, "copies": s.copies, "hits": s.hits, "acquisitions": s.acquisitions}
+
+    def synchronize(self) -> None:
+        B.call("nf4ls_pool_synchronize", self.handle)
+
+    def destroy(self) -> None:
+        if self.handle:
+            B.call("nf4ls_pool_destroy", self.handle)
+            self.handle = ctypes.c_void_p()
+
+    def view(self, ptr: int, nbytes: int) -> torch.Tensor:
+        """A uint8 view of the slot at device address ptr (for reading a streamed shard)."""
+        off = ptr - self.slots.data_ptr()
+        return self.slots[off: off + nbytes]
+
+
+# ----------------------------------------------------------------------------- whole model
+
+@dataclass
+class TrainConfig:
+    lr: float = 2e-4
+    beta1: float = 0.9
+    beta2: float = 0.999
+    eps: float = 1e-8
+    weight_decay: float = 0.0
+
+
+class StreamedModel:
+    """All buffers of one n-layer model: pinned NF4 store (or resident shards), the
+    resident bf16 embedding / lm_head, LoRA masters, gradients and AdamW moments, and
+    the step workspace.  Quantisation runs through nf4_quantize_shard on the GPU."""
+
+    def __init__(self, wl: Workload, depth: int = 2, resident: bool = False, b_random: bool = False,
+                 train: TrainConfig = TrainConfig(), device="cuda", weights_device=None, fingerprint: int = 1234):
+        self.wl = wl
+        shape = wl.shape
+        self.cfg = B.ModelCfg(layer_cfg(shape, wl.batch, wl.seq), wl.n_layers, wl.vocab, int(wl.tied), train.lr,
+                              train.beta1, train.beta2, train.eps, train.weight_decay)
+        lc = self.cfg.layer
+        from . import synth
+        wdev = weights_device or device
+        self.shard_nbytes = shard_bytes(lc)
+        self.slot_bytes = (self.shard_nbytes + 255) // 256 * 256
+        L = wl.n_layers
+        self.resident = resident
+        self.pool = None
+        shards = []
+        if resident:
+            self.shard_buf = _buffer(L * self.slot_bytes, device)
+        else:
+            self.store = torch.empty(L * self.slot_bytes, dtype=torch.uint8).pin_memory()
+        tmp = _buffer(self.slot_bytes, device)
+        for i in range(L):
+            w = synth.layer_weights(shape, i, wl.seed, device=wdev)
+            w = {k: v.to(device) for k, v in w.items()}
+            if resident:
+                dst = self.shard_buf[i * self.slot_bytes:(i + 1) * self.slot_bytes]
+                nf4_quantize_shard(lc, w, fingerprint, out=dst)
+                shards.append(dst.data_ptr())
+            else:
+                nf4_quantize_shard(lc, w, fingerprint, out=tmp)
+                torch.cuda.synchronize()
+                self.store[i * self.slot_bytes:(i + 1) * self.slot_bytes].copy_(tmp)
+            del w
+        del tmp
+        if resident:
+            self.shard_ptrs = (ctypes.c_void_p * L)(*shards)
+        else:
+            offs = [i * self.slot_bytes for i in range(L)]
+            self.pool = Pool(self.store, offs, [self.shard_nbytes] * L, depth, self.slot_bytes, device)
+        self.embed = synth.embedding(wl.vocab, shape.hidden, wl.seed, 0, device=wdev).to(device)
+        self.lm_head = None if wl.tied else synth.embedding(wl.vocab, shape.hidden, wl.seed, 1, device=wdev).to(device)
+        self.norm_final = torch.ones(shape.hidden, dtype=torch.bfloat16, device=device)
+        self.stride = B.lib().nf4ls_lora_stride(ctypes.byref(lc))
+        self.lora = torch.zeros(L * self.stride, dtype=torch.float32, device=device)
+        for i in range(L):
+            lp = synth.lora_params(shape, i, wl.seed, b_random=b_random, device="cpu")
+            flat = torch.cat([lp["A_q"].reshape(-1), lp["B_q"].reshape(-1), lp["A_v"].reshape(-1),
+                              lp["B_v"].reshape(-1)])
+            self.lora[i * self.stride:(i + 1) * self.stride].copy_(flat)
+        self.grads = torch.zeros_like(self.lora)
+        self.adam_m = torch.zeros_like(self.lora)
+        self.adam_v = torch.zeros_like(self.lora)
+        self.ws_bytes = B.lib().nf4ls_model_workspace_bytes(ctypes.byref(self.cfg))
+        self.ws = _buffer(self.ws_bytes, device)
+        self.loss = torch.zeros(1, dtype=torch.float32, device=device)
+        self.model = B.Model(self.embed.data_ptr(), 0 if self.lm_head is None else self.lm_head.data_ptr(),
+                             self.norm_final.data_ptr(), self.lora.data_ptr(), self.grads.data_ptr(),
+                             self.adam_m.data_ptr(), self.adam_v.data_ptr(),
+                             self.pool.handle.value if self.pool else None,
+                             ctypes.cast(self.shard_ptrs, ctypes.c_void_p) if resident else None,
+                             self.ws.data_ptr(), self.ws_bytes)
+        self.step_count = 0
+
+    def lora_views(self, layer: int) -> dict:
+        sh = self.wl.shape
+        r, H = sh.lora_r, sh.hidden
+        base = self.lora[layer * self.stride:(layer + 1) * self.stride]
+        a = r * H
+        bq = sh.q_dim * r
+        return {"A_q": base[:a].view(r, H), "B_q": base[a:a + bq].view(sh.q_dim, r),
+                "A_v": base[a + bq:2 * a + bq].view(r, H), "B_v": base[2 * a + bq:].view(sh.kv_dim, r)}
+
+    def grad_views(self, layer: int) -> dict:
+        sh = self.wl.shape
+        r, H = sh.lora_r, sh.hidden
+        base = self.grads[layer * self.stride:(layer + 1) * self.stride]
+        a = r * H
+        bq = sh.q_dim * r
+        return {"dA_q": base[:a].view(r, H), "dB_q": base[a:a + bq].view(sh.q_dim, r),
+                "dA_v": base[a + bq:2 * a + bq].view(r, H), "dB_v": base[2 * a + bq:].view(sh.kv_dim, r)}
+
+    def train_step(self, ids: torch.Tensor, stream=None) -> torch.Tensor:
+        self.step_count += 1
+        B.call("nf4ls_train_step", ctypes.byref(self.cfg), ctypes.byref(self.model), _p(ids), self.step_count,
+               _p(self.loss), _s(stream))
+        return self.loss
+
+    def forward_backward(self, ids: torch.Tensor, stream=None) -> torch.Tensor:
+        B.call("nf4ls_forward_backward", ctypes.byref(self.cfg), ctypes.byref(self.model), _p(ids), _p(self.loss),
+               _s(stream))
+        return self.loss
+
+    def adamw_step(self, stream=None) -> None:
+        self.step_count += 1
+        B.call("nf4ls_adamw_step", ctypes.byref(self.cfg), ctypes.byref(self.model), self.step_count, _s(stream))
+
+    def forward_loss(self, ids: torch.Tensor, lora_on: bool = True, stream=None) -> torch.Tensor:
+        B.call("nf4ls_forward_loss", ctypes.byref(self.cfg), ctypes.byref(self.model), _p(ids), int(lora_on),
+               _p(self.loss), _s(stream))
+        return self.loss
+
+    def close(self) -> None:
+        if self.pool is not None:
+            self.pool.destroy()
+            self.pool = None

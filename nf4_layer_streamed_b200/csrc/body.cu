@@ -1,0 +1,478 @@
+// Layer-body and model-end kernels around the tcgen05 GEMMs: RMSNorm forward and
+// backward (K8), RoPE tables and the RoPE transpose for dL/dq, dL/dk (K9), the LoRA
+// down-projection, its gradient products and the padded adapter operands (K6/K7),
+// embedding gather (K13), causal-LM cross-entropy with its gradient (K12), the
+// single-layer mean-square loss, and AdamW (K14).
+//
+// The layer body is the HF Llama decoder layer the pages' system runs ("Soup
+// layer-streamed NF4 gate record" §2.1); LoRA r=16 / alpha=32 on q_proj and v_proj
+// trained with AdamW (the SFT configuration of "Soup v0.72.4 技术解析", §4.2).
+// All reductions run in a fixed order (no atomics), so every result is
+// bit-reproducible from run to run and independent of buffer addresses.
+#include <algorithm>
+#include <cmath>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace nf4ls {
+
+namespace {
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    f[2 * j] = bf16_lo(w[j]);
+    f[2 * j + 1] = bf16_hi(w[j]);
+  }
+}
+__device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
+  return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                    pack_bf16x2(f[6], f[7]));
+}
+
+// ------------------------------------------------------------------ RMSNorm (one warp per row)
+__global__ void k_rmsnorm_fwd(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ w,
+                              __nv_bfloat16* __restrict__ y, int M, int H, float eps) {
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)row * H);
+  const uint4* wr = reinterpret_cast<const uint4*>(w);
+  uint4* yr = reinterpret_cast<uint4*>(y + (size_t)row * H);
+  const int nv = H / 8;
+  float ss = 0.f;
+  for (int i = lane; i < nv; i += 32) {
+    float f[8];
+    unpack8(xr[i], f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) ss += f[j] * f[j];
+  }
+  ss = warp_sum(ss);
+  const float r = 1.0f / sqrtf(ss / (float)H + eps);
+  for (int i = lane; i < nv; i += 32) {
+    float f[8], g[8];
+    unpack8(xr[i], f);
+    unpack8(wr[i], g);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) f[j] = f[j] * r * g[j];
+    yr[i] = pack8(f);
+  }
+}
+
+// dx = resid + r w dy - x r^3 sum(w dy x) / H
+__global__ void k_rmsnorm_bwd(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ w,
+                              const __nv_bfloat16* __restrict__ dy, const __nv_bfloat16* __restrict__ resid,
+                              __nv_bfloat16* __restrict__ dx, int M, int H, float eps) {
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)row * H);
+  const uint4* wr = reinterpret_cast<const uint4*>(w);
+  const uint4* dr = reinterpret_cast<const uint4*>(dy + (size_t)row * H);
+  const uint4* rr = resid ? reinterpret_cast<const uint4*>(resid + (size_t)row * H) : nullptr;
+  uint4* out = reinterpret_cast<uint4*>(dx + (size_t)row * H);
+  const int nv = H / 8;
+  float ss = 0.f, dot = 0.f;
+  for (int i = lane; i < nv; i += 32) {
+    float a[8], b[8], c[8];
+    unpack8(xr[i], a);
+    unpack8(wr[i], b);
+    unpack8(dr[i], c);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      ss += a[j] * a[j];
+      dot += b[j] * c[j] * a[j];
+    }
+  }
+  ss = warp_sum(ss);
+  dot = warp_sum(dot);
+  const float r = 1.0f / sqrtf(ss / (float)H + eps);
+  const float k = r * r * r * dot / (float)H;
+  for (int i = lane; i < nv; i += 32) {
+    float a[8], b[8], c[8], e[8];
+    unpack8(xr[i], a);
+    unpack8(wr[i], b);
+    unpack8(dr[i], c);
+    if (rr)
+      unpack8(rr[i], e);
+    else
+#pragma unroll
+      for (int j = 0; j < 8; ++j) e[j] = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) e[j] += r * b[j] * c[j] - a[j] * k;
+    out[i] = pack8(e);
+  }
+}
+
+// ------------------------------------------------------------------ RoPE
+__global__ void k_rope_tables(float* cos_t, float* sin_t, int seq, int d, double theta) {
+  const int half = d / 2;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= seq * half) return;
+  const int p = i / half, j = i % half;
+  const double inv = pow(theta, -(2.0 * j) / (double)d);
+  const double a = (double)p * inv;
+  cos_t[i] = (float)cos(a);
+  sin_t[i] = (float)sin(a);
+}
+
+// In place: (x1, x2) -> (x1 c + x2 s, x2 c - x1 s), the transpose of the rotation.
+__global__ void k_rope_bwd(__nv_bfloat16* __restrict__ x, int ld, int M, int cols, int seq, int d,
+                           const float* __restrict__ cos_t, const float* __restrict__ sin_t) {
+  const int half = d / 2;
+  const size_t per_row = (size_t)cols / 2;
+  const size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
+  if (i >= per_row * M) return;
+  const int m = (int)(i / per_row);
+  const int r = (int)(i % per_row);
+  const int head = r / half, j = r % half;
+  const int pos = m % seq;
+  __nv_bfloat16* p = x + (size_t)m * ld + head * d;
+  const float c = cos_t[pos * half + j], s = sin_t[pos * half + j];
+  const float a = __bfloat162float(p[j]), b = __bfloat162float(p[j + half]);
+  p[j] = __float2bfloat16_rn(a * c + b * s);
+  p[j + half] = __float2bfloat16_rn(b * c - a * s);
+}
+
+// ------------------------------------------------------------------ LoRA
+// out[m, oc + r] = scale * sum_k X[m, k] * bf16(W(r, k)) for r < 16 (fixed k order),
+// W(r, k) = W[r * sr + k * sk] fp32.  Writes fp32 (out_f, ld 16) and/or bf16
+// (out_b at column offset oc, ld ldb).  64 rows per block, 256 threads, 8 outputs each.
+__global__ void __launch_bounds__(256) k_skinny(const __nv_bfloat16* __restrict__ X, int ldx, int M, int K,
+                                                const float* __restrict__ W, int sr, int sk, float scale,
+                                                float* __restrict__ out_f, __nv_bfloat16* __restrict__ out_b, int ldb,
+                                                int oc) {
+  __shared__ float xs[64][65];
+  __shared__ float ws[16][65];
+  const int t = threadIdx.x;
+  const int row = t >> 2, r0 = (t & 3) * 4;
+  const int m0 = blockIdx.x * 64;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int k0 = 0; k0 < K; k0 += 64) {
+    for (int i = t; i < 64 * 64; i += 256) {
+      const int rr = i >> 6, kk = i & 63;
+      const int m = m0 + rr;
+      xs[rr][kk] = (m < M) ? __bfloat162float(X[(size_t)m * ldx + k0 + kk]) : 0.f;
+    }
+    for (int i = t; i < 16 * 64; i += 256) {
+      const int rr = i >> 6, kk = i & 63;
+      ws[rr][kk] = __bfloat162float(__float2bfloat16_rn(W[(size_t)rr * sr + (size_t)(k0 + kk) * sk]));
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < 64; ++kk) {
+      const float xv = xs[row][kk];
+#pragma unroll
+      for (int o = 0; o < 4; ++o) acc[o] += xv * ws[r0 + o][kk];
+    }
+    __syncthreads();
+  }
+  const int m = m0 + row;
+  if (m >= M) return;
+#pragma unroll
+  for (int o = 0; o < 4; ++o) {
+    const float v = acc[o] * scale;
+    if (out_f) out_f[(size_t)m * 16 + r0 + o] = v;
+    if (out_b) out_b[(size_t)m * ldb + oc + r0 + o] = __float2bfloat16_rn(v);
+  }
+}
+
+// out(n, r) = scale * sum_m X[m, n] * Y[m, r] (fixed m order); X bf16 [M, ldx],
+// Y fp32 (y_f) or bf16 (y_b) [M, ldy] from column yc; out(n, r) at out[n * so_n + r * so_r].
+// Block: 64 columns n, 256 threads, 4 outputs each.
+__global__ void __launch_bounds__(256) k_grad_reduce(const __nv_bfloat16* __restrict__ X, int ldx, int M, int N,
+                                                     const float* __restrict__ y_f, const __nv_bfloat16* __restrict__ y_b,
+                                                     int ldy, int yc, float scale, float* __restrict__ out, int so_n,
+                                                     int so_r) {
+  __shared__ float xs[64][65];
+  __shared__ float ys[64][17];
+  const int t = threadIdx.x;
+  const int n_l = t >> 2, r0 = (t & 3) * 4;
+  const int n0 = blockIdx.x * 64;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int mb = 0; mb < M; mb += 64) {
+    for (int i = t; i < 64 * 64; i += 256) {
+      const int mm = i >> 6, nn = i & 63;
+      const int m = mb + mm, n = n0 + nn;
+      xs[mm][nn] = (m < M && n < N) ? __bfloat162float(X[(size_t)m * ldx + n]) : 0.f;
+    }
+    for (int i = t; i < 64 * 16; i += 256) {
+      const int mm = i >> 4, rr = i & 15;
+      const int m = mb + mm;
+      float v = 0.f;
+      if (m < M) v = y_f ? y_f[(size_t)m * ldy + yc + rr] : __bfloat162float(y_b[(size_t)m * ldy + yc + rr]);
+      ys[mm][rr] = v;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int mm = 0; mm < 64; ++mm) {
+      const float xv = xs[mm][n_l];
+#pragma unroll
+      for (int o = 0; o < 4; ++o) acc[o] += xv * ys[mm][r0 + o];
+    }
+    __syncthreads();
+  }
+  const int n = n0 + n_l;
+  if (n >= N) return;
+#pragma unroll
+  for (int o = 0; o < 4; ++o) out[(size_t)n * so_n + (size_t)(r0 + o) * so_r] = acc[o] * scale;
+}
+
+// Padded bf16 adapter operands of the GEMM extra block:
+//   bup [Nqkv, 64]: row n of q -> scale*B_q[n, :] in cols 0-15; row of v -> scale*B_v in 16-31; k rows 0.
+//   adn [64, H]   : rows 0-15 = A_q, rows 16-31 = A_v, other rows 0.
+__global__ void k_lora_pack(const float* __restrict__ Aq, const float* __restrict__ Bq, const float* __restrict__ Av,
+                            const float* __restrict__ Bv, int H, int qd, int kvd, float scale,
+                            __nv_bfloat16* __restrict__ bup, __nv_bfloat16* __restrict__ adn) {
+  const int nq = qd + 2 * kvd;
+  const size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
+  const size_t n_bup = (size_t)nq * 64, n_adn = (size_t)64 * H;
+  if (i < n_bup) {
+    const int n = (int)(i / 64), c = (int)(i % 64);
+    float v = 0.f;
+    if (n < qd && c < 16)
+      v = scale * __bfloat162float(__float2bfloat16_rn(Bq[(size_t)n * 16 + c]));
+    else if (n >= qd + kvd && c >= 16 && c < 32)
+      v = scale * __bfloat162float(__float2bfloat16_rn(Bv[(size_t)(n - qd - kvd) * 16 + c - 16]));
+    bup[i] = __float2bfloat16_rn(v);
+  } else if (i < n_bup + n_adn) {
+    const size_t j = i - n_bup;
+    const int r = (int)(j / H), k = (int)(j % H);
+    float v = 0.f;
+    if (r < 16)
+      v = Aq[(size_t)r * H + k];
+    else if (r < 32)
+      v = Av[(size_t)(r - 16) * H + k];
+    adn[j] = __float2bfloat16_rn(v);
+  }
+}
+
+__global__ void k_zero_cols(__nv_bfloat16* __restrict__ x, int ld, int M, int c0, int c1) {
+  const int w = c1 - c0;
+  const size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
+  if (i >= (size_t)M * w) return;
+  x[(i / w) * ld + c0 + (i % w)] = __float2bfloat16_rn(0.f);
+}
+
+// ------------------------------------------------------------------ embedding, CE, losses, AdamW
+__global__ void k_embed(const int32_t* __restrict__ ids, const __nv_bfloat16* __restrict__ E, __nv_bfloat16* __restrict__ h,
+                        int M, int H) {
+  const int m = blockIdx.x;
+  if (m >= M) return;
+  const uint4* src = reinterpret_cast<const uint4*>(E + (size_t)ids[m] * H);
+  uint4* dst = reinterpret_cast<uint4*>(h + (size_t)m * H);
+  for (int i = threadIdx.x; i < H / 8; i += blockDim.x) dst[i] = src[i];
+}
+
+// One block per token row: loss_row = logsumexp(logits) - logits[target], and
+// dlogits = (softmax - onehot) * inv_count, for rows with a target (t < seq-1);
+// other rows get zero loss and zero gradient.
+// logits and dlogits may be the same buffer (the gradient overwrites the logits).
+__global__ void __launch_bounds__(256) k_ce(const __nv_bfloat16* logits, const int32_t* __restrict__ ids, int V,
+                                            int seq, float inv_count, float* __restrict__ row_loss,
+                                            __nv_bfloat16* dlogits) {
+  __shared__ float red[8];
+  __shared__ float bval[2];
+  const int m = blockIdx.x;
+  const int t = threadIdx.x, lane = t & 31, wid = t >> 5;
+  const __nv_bfloat16* row = logits + (size_t)m * V;
+  __nv_bfloat16* drow = dlogits + (size_t)m * V;
+  const bool has_target = (m % seq) != seq - 1;
+  if (!has_target) {
+    for (int j = t; j < V; j += blockDim.x) drow[j] = __float2bfloat16_rn(0.f);
+    if (t == 0) row_loss[m] = 0.f;
+    return;
+  }
+  const int tgt = ids[m + 1];
+  float mx = -INFINITY;
+  for (int j = t; j < V; j += blockDim.x) mx = fmaxf(mx, __bfloat162float(row[j]));
+  mx = warp_max(mx);
+  if (lane == 0) red[wid] = mx;
+  __syncthreads();
+  if (t == 0) {
+    float v = red[0];
+    for (int i = 1; i < 8; ++i) v = fmaxf(v, red[i]);
+    bval[0] = v;
+  }
+  __syncthreads();
+  mx = bval[0];
+  float s = 0.f;
+  for (int j = t; j < V; j += blockDim.x) s += expf(__bfloat162float(row[j]) - mx);
+  s = warp_sum(s);
+  __syncthreads();
+  if (lane == 0) red[wid] = s;
+  __syncthreads();
+  if (t == 0) {
+    float v = 0.f;
+    for (int i = 0; i < 8; ++i) v += red[i];
+    bval[1] = v;
+  }
+  __syncthreads();
+  const float sum = bval[1];
+  const float lse = mx + logf(sum);
+  const float inv_sum = 1.0f / sum;
+  const float lt = __bfloat162float(row[tgt]);  // read before the row may be overwritten in place
+  __syncthreads();
+  for (int j = t; j < V; j += blockDim.x) {
+    float p = expf(__bfloat162float(row[j]) - mx) * inv_sum;
+    if (j == tgt) p -= 1.0f;
+    drow[j] = __float2bfloat16_rn(p * inv_count);
+  }
+  if (t == 0) row_loss[m] = lse - lt;
+}
+
+// Deterministic mean: one block sums n values in a fixed pattern, then scales.
+__global__ void k_sum_scale(const float* __restrict__ v, int n, float scale, float* __restrict__ out) {
+  __shared__ double red[256];
+  double s = 0.0;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) s += (double)v[i];
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int o = blockDim.x / 2; o > 0; o >>= 1) {
+    if ((int)threadIdx.x < o) red[threadIdx.x] += red[threadIdx.x + o];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *out = (float)(red[0] * (double)scale);
+}
+
+// Single-layer loss of the one-layer workloads: L = mean(out^2), dL/dout = 2 out / n.
+__global__ void k_mse(const __nv_bfloat16* __restrict__ out, size_t n, float* __restrict__ partial,
+                      __nv_bfloat16* __restrict__ dout) {
+  __shared__ float red[8];
+  float s = 0.f;
+  const float g = 2.0f / (float)n;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+    const float v = __bfloat162float(out[i]);
+    s += v * v;
+    dout[i] = __float2bfloat16_rn(g * v);
+  }
+  s = warp_sum(s);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float v = 0.f;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) v += red[i];
+    partial[blockIdx.x] = v;
+  }
+}
+
+__global__ void k_adamw(float* __restrict__ p, const float* __restrict__ g, float* __restrict__ m, float* __restrict__ v,
+                        size_t n, float lr, float b1, float b2, float eps, float wd, float bc1, float bc2) {
+  const size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const float gi = g[i];
+  const float mi = b1 * m[i] + (1.0f - b1) * gi;
+  const float vi = b2 * v[i] + (1.0f - b2) * gi * gi;
+  m[i] = mi;
+  v[i] = vi;
+  const float mh = mi / bc1, vh = vi / bc2;
+  p[i] = p[i] - lr * (mh / (sqrtf(vh) + eps) + wd * p[i]);
+}
+
+inline unsigned blocks_for(size_t n, int threads) { return (unsigned)((n + threads - 1) / threads); }
+
+}  // namespace
+
+int rmsnorm_fwd(const __nv_bfloat16* x, const __nv_bfloat16* w, __nv_bfloat16* y, int M, int H, float eps,
+                cudaStream_t s) {
+  if (H % 8) return fail(NF4LS_SHAPE, "rmsnorm: H %% 8");
+  k_rmsnorm_fwd<<<(M + 7) / 8, 256, 0, s>>>(x, w, y, M, H, eps);
+  NF4_CUDA_TRY(cudaGetLastError());
+  return NF4LS_OK;
+}
+
+int rmsnorm_bwd(const __nv_bfloat16* x, const __nv_bfloat16* w, const __nv_bfloat16* dy, const __nv_bfloat16* resid,
+                __nv_bfloat16* dx, int M, int H, float eps, cudaStream_t s) {
+  k_rmsnorm_bwd<<<(M + 7) / 8, 256, 0, s>>>(x, w, dy, resid, dx, M, H, eps);
+  NF4_CUDA_TRY(cudaGetLastError());
+  return NF4LS_OK;
+}
+
+int rope_tables(float* cos_t, float* sin_t, int seq, int d, float theta, cudaStream_t s) {
+  k_rope_tables<<<blocks_for((size_t)seq * d / 2, 256), 256, 0, s>>>(cos_t, sin_t, seq, d, (double)theta);
+  NF4_CUDA_TRY(cudaGetLastError());
+  return NF4LS_OK;
+}
+
+int rope_bwd(__nv_bfloat16* x, int ld, int M, int cols, int seq, int d, const float* cos_t, const float* sin_t,
+             cudaStream_t s) {
+  k_rope_bwd<<<blocks_for((size_t)M * cols / 2, 256), 256, 0, s>>>(x, ld, M, cols, seq, d, cos_t, sin_t);
+  NF4_CUDA_TRY(cudaGetLastError());
+  return NF4LS_OK;
+}
+
+int lora_skinny(const __nv_bfloat16* X, int ldx, int M, int K, const float* W, int sr, int sk, float scale,
+                float* out_f, __nv_bfloat16* out_b, int ldb, int oc, cudaStream_t s) {
+  if (K % 64) return fail(NF4LS_SHAPE, "lora: K %% 64");
+  k_skinny<<<(M + 63) / 64, 256, 0, s>>>(X, ldx, M, K, W, sr, sk, scale, out_f, out_b, ldb, oc);
+  NF4_CUDA_TRY(cudaGetLastError());
+  return NF4LS_OK;
+}
+
+int lora_grad_reduce(const __nv_bfloat16* X, int ldx, int M, int N, const float* y_f, const __nv_bfloat16* y_b, int ldy,
+                     int yc, float scale, float* out, int so_n, int so_r, cudaStream_t s) {
+  k_grad_reduce<<<(N + 63) / 64, 256, 0, s>>>(X, ldx, M, N, y_f, y_b, ldy, yc, scale, out, so_n, so_r);
+  NF4_CUDA_TRY(cudaGetLastError());
+  return NF4LS_OK;
+}
+
+int lora_pack(const nf4ls_lora* l, int H, int qd, int kvd, float scale, __nv_bfloat16* bup, __nv_bfloat16* adn,
+              cudaStream_t s) {
+  const size_t n = (size_t)(qd + 2 * kvd) * 64 + (size_t)64 * H;
+  k_lora_pack<<<blocks_for(n, 256), 256, 0, s>>>(l->A_q, l->B_q, l->A_v, l->B_v, H, qd, kvd, scale, bup, adn);
+  NF4_CUDA_TRY(cudaGetLastError());
+  return NF4LS_OK;
+}
+
+int zero_cols(__nv_bfloat16* x, int ld, int M, int c0, int c1, cudaStream_t s) {
+  k_zero_cols<<<blocks_for((size_t)M * (c1 - c0), 256), 256, 0, s>>>(x, ld, M, c0, c1);
+  NF4_CUDA_TRY(cudaGetLastError());
+  return NF4LS_OK;
+}
+
+int embed(const int32_t* ids, const __nv_bfloat16* E, __nv_bfloat16* h, int M, int H, cudaStream_t s) {
+  k_embed<<<M, 128, 0, s>>>(ids, E, h, M, H);
+  NF4_CUDA_TRY(cudaGetLastError());
+  return NF4LS_OK;
+}
+
+int cross_entropy(const __nv_bfloat16* logits, const int32_t* ids, int M, int V, int batch, int seq, float* row_loss,
+                  __nv_bfloat16* dlogits, float* loss, cudaStream_t s) {
+  const int count = batch * (seq - 1);
+  k_ce<<<M, 256, 0, s>>>(logits, ids, V, seq, 1.0f / (float)count, row_loss, dlogits);
+  k_sum_scale<<<1, 256, 0, s>>>(row_loss, M, 1.0f / (float)count, loss);
+  NF4_CUDA_TRY(cudaGetLastError());
+  return NF4LS_OK;
+}
+
+int mse_loss(const __nv_bfloat16* out, size_t n, float* partial, int n_partial, __nv_bfloat16* dout, float* loss,
+             cudaStream_t s) {
+  k_mse<<<n_partial, 256, 0, s>>>(out, n, partial, dout);
+  k_sum_scale<<<1, 256, 0, s>>>(partial, n_partial, 1.0f / (float)n, loss);
+  NF4_CUDA_TRY(cudaGetLastError());
+  return NF4LS_OK;
+}
+
+int adamw(float* p, const float* g, float* m, float* v, size_t n, int step, float lr, float b1, float b2, float eps,
+          float wd, cudaStream_t s) {
+  const float bc1 = (float)(1.0 - std::pow((double)b1, step));
+  const float bc2 = (float)(1.0 - std::pow((double)b2, step));
+  k_adamw<<<blocks_for(n, 256), 256, 0, s>>>(p, g, m, v, n, lr, b1, b2, eps, wd, bc1, bc2);
+  NF4_CUDA_TRY(cudaGetLastError());
+  return NF4LS_OK;
+}
+
+}  // namespace nf4ls

@@ -1,0 +1,632 @@
+// K3/K4/K5: tcgen05 GEMMs for the frozen base linears, with the NF4 weights
+// decoded inside the mainloop, and the dense bf16 variant (lm_head, and the
+// dequantise-then-multiply path).
+//
+// The products come from the layer-streaming pages: the frozen base linears run
+// for the forward, for the checkpoint recompute and for dL/dx = W^T dL/dy
+// ("4GB 显存微调 8B 模型是真的", mechanism section; "Soup layer-streamed NF4 gate
+// record" §4.4: C = 6, no dL/dW), on NF4 weights with double-quantised absmax
+// (§2.1, §2.4).  The decode is the dequantisation of §2.4 exactly:
+// w^ = bf16_rne(fp32(nf4[code] * fp32(fp32(code8[q8] * nested) + offset))).
+//
+// Tile: 256 tokens x 256 output features per CTA, 64-deep reduction stages,
+// 3 stages.  The 256 tokens are two 128-row MMAs (M = 128, N = 256, K = 16) that
+// share one B tile, so each decoded weight is used by 256 tokens; the two fp32
+// accumulators take all 512 TMEM columns.
+//
+// Warp roles (one CTA per SM):
+//   warp 0      TMA producer: A tiles (128-byte swizzle), dense B tiles or the packed
+//               NF4 code tiles, the LoRA extra block.
+//   warp 1      TMEM allocation and the MMA issuer (one elected thread).
+//   warps 2-5   epilogue: tcgen05.ld of the accumulators, fused epilogue, bf16 stores.
+//   warps 6-13  NF4 decoders (decode variant only): each thread turns one 64-weight
+//               block (32 code bytes + its two-level scale) into 128 bytes of bf16 in
+//               the swizzled layout the MMA reads, K-major for the forward, N-major
+//               for dL/dx.
+//
+// The decode builds, per block, the 16 possible bf16 outputs nf4[j] * s (16 fp32
+// multiplies, 8 packed conversions) as byte tables and looks codes up with byte
+// permutes (prmt), four codes per permute.
+//
+// Every wait on an mbarrier is bounded (common.cuh); on expiry the kernel records
+// the site in the device error record, all roles leave their loops, and TMEM is
+// released before exit.
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace nf4ls {
+
+namespace {
+
+constexpr int BM = 256, BN = 256, BK = 64, STAGES = 3;
+constexpr int A_BYTES = BM * BK * 2;  // 32 KB
+constexpr int B_BYTES = BN * BK * 2;  // 32 KB
+constexpr int C_BYTES = BN * BK / 2;  // 8 KB of packed codes
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + C_BYTES;
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256 + 1024;
+constexpr int NUM_DECODERS = 256;
+
+struct GemmParams {
+  CUtensorMap tmA, tmAx, tmB, tmBx;
+  CUtensorMap tmC[4];
+  int M, N, K, num_kb, has_extra, n_mt;
+  int n_seg, swiglu, dense_swiglu_rows;
+  int seg_start[5];
+  const uint8_t* q8[4];
+  const float* nested[4];
+  const float* offset[4];
+  int seg_cols;
+  // epilogue
+  int epi;
+  __nv_bfloat16* out;
+  int ldo;
+  const __nv_bfloat16* aux0;
+  int ld_aux0;
+  __nv_bfloat16* aux_out;
+  int ld_aux_out, inter;
+  const float* rope_cos;
+  const float* rope_sin;
+  int seq, head_dim, rope_cols;
+  float nf4[16];
+  float code8[256];
+  int* err;
+};
+
+// ------------------------------------------------------------------------------ decode
+__device__ __forceinline__ void decode_block(uint32_t row_addr, int row_in_atom, const uint32_t (&w)[8], float s,
+                                             const float (&nf4)[16]) {
+  uint32_t p[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) p[j] = pack_bf16x2(__fmul_rn(nf4[2 * j], s), __fmul_rn(nf4[2 * j + 1], s));
+  // hi/lo bytes of entries 0-3, 4-7, 8-11, 12-15
+  const uint32_t th0 = prmt(p[0], p[1], 0x7531u), th1 = prmt(p[2], p[3], 0x7531u);
+  const uint32_t th2 = prmt(p[4], p[5], 0x7531u), th3 = prmt(p[6], p[7], 0x7531u);
+  const uint32_t tl0 = prmt(p[0], p[1], 0x6420u), tl1 = prmt(p[2], p[3], 0x6420u);
+  const uint32_t tl2 = prmt(p[4], p[5], 0x6420u), tl3 = prmt(p[6], p[7], 0x6420u);
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    uint32_t o[4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      // nibbles of x (low 16 bits) hold the codes of elements 1,0,3,2 of this quad
+      const uint32_t x = h ? (w[c] >> 16) : w[c];
+      const uint32_t sel = x & 0x7777u;
+      const uint32_t m = prmt(0x0000FF00u, 0u, (x >> 3) & 0x1111u);  // 0xFF where code >= 8
+      const uint32_t hA = prmt(th0, th1, sel), hB = prmt(th2, th3, sel);
+      const uint32_t lA = prmt(tl0, tl1, sel), lB = prmt(tl2, tl3, sel);
+      const uint32_t hi = (hA & ~m) | (hB & m);
+      const uint32_t lo = (lA & ~m) | (lB & m);
+      o[2 * h] = prmt(lo, hi, 0x4051u);      // elements 0,1
+      o[2 * h + 1] = prmt(lo, hi, 0x6273u);  // elements 2,3
+    }
+    st_shared_v4(row_addr + ((uint32_t)(c ^ row_in_atom) << 4), o[0], o[1], o[2], o[3]);
+  }
+}
+
+__device__ __forceinline__ void zero_block(uint32_t row_addr) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c) st_shared_v4(row_addr + (c << 4), 0u, 0u, 0u, 0u);
+}
+
+__device__ __forceinline__ int find_seg(const GemmParams& p, int row) {
+  int s = 0;
+#pragma unroll
+  for (int i = 1; i < 4; ++i)
+    if (i < p.n_seg && row >= p.seg_start[i]) s = i;
+  return s;
+}
+
+__device__ __forceinline__ float silu_f(float x) { return x / (1.0f + expf(-x)); }
+__device__ __forceinline__ float round_bf16(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
+
+__device__ __forceinline__ void store32(__nv_bfloat16* dst, const float (&v)[32]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    d[i] = make_uint4(pack_bf16x2(v[8 * i + 0], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                      pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+}
+
+__device__ __forceinline__ void load32_bf16(const __nv_bfloat16* src, float (&v)[32]) {
+  const uint4* s = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 u = s[i];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[8 * i + 2 * j] = bf16_lo(w[j]);
+      v[8 * i + 2 * j + 1] = bf16_hi(w[j]);
+    }
+  }
+}
+
+__device__ __forceinline__ void ld_acc(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  tmem_ld32(taddr, r);
+  tmem_wait_ld();
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// ------------------------------------------------------------------------------ kernel
+template <bool DECODE, bool BMN>
+__global__ void __launch_bounds__(DECODE ? 448 : 192, 1) k_gemm(const __grid_constant__ GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* misc = base + STAGES * STAGE_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(misc);
+  uint64_t* empty = full + STAGES;
+  uint64_t* codes_full = empty + STAGES;
+  uint64_t* accum_full = codes_full + STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum_full + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* code8_s = reinterpret_cast<float*>(misc + 256);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int mt = blockIdx.x % p.n_mt, nt = blockIdx.x / p.n_mt;
+  const int m0 = mt * BM;
+  const int total_kb = p.num_kb + p.has_extra;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], DECODE ? 1 + NUM_DECODERS : 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&codes_full[s], 1);
+    }
+    mbar_init(accum_full, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&p.tmA);
+    if (p.has_extra) {
+      tma_prefetch_desc(&p.tmAx);
+      tma_prefetch_desc(&p.tmBx);
+    }
+    if (!DECODE) tma_prefetch_desc(&p.tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  if (DECODE && warp >= 6)
+    for (int i = threadIdx.x - 192; i < 256; i += NUM_DECODERS) code8_s[i] = p.code8[i];
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      for (int kb = 0; kb < total_kb; ++kb) {
+        const int s = kb % STAGES;
+        const uint32_t ph = (kb / STAGES) & 1;
+        if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, p.err, KID_GEMM, 1)) break;
+        uint8_t* sA = base + s * STAGE_BYTES;
+        uint8_t* sB = sA + A_BYTES;
+        uint8_t* sC = sB + B_BYTES;
+        if (kb < p.num_kb) {
+          mbar_arrive_expect_tx(&full[s], A_BYTES + (DECODE ? 0 : B_BYTES));
+          tma_load_2d(sA, &p.tmA, &full[s], kb * BK, m0);
+          if (!DECODE) {
+            if (BMN) {
+              for (int j = 0; j < 4; ++j) tma_load_2d(sB + j * 8192, &p.tmB, &full[s], nt * BN + 64 * j, kb * BK);
+            } else if (p.dense_swiglu_rows) {
+              tma_load_2d(sB, &p.tmB, &full[s], kb * BK, nt * 128);
+              tma_load_2d(sB + 16384, &p.tmB, &full[s], kb * BK, p.dense_swiglu_rows + nt * 128);
+            } else {
+              tma_load_2d(sB, &p.tmB, &full[s], kb * BK, nt * BN);
+            }
+          } else {
+            // packed codes of this stage
+            if (BMN) {
+              const int row = kb * BK;
+              const int sg = find_seg(p, row);
+              mbar_arrive_expect_tx(&codes_full[s], C_BYTES);
+              tma_load_2d(sC, &p.tmC[sg], &codes_full[s], nt * (BN / 2), row - p.seg_start[sg]);
+            } else {
+              int nbox = 0;
+              int sg[4], lr[4];
+              for (int rb = 0; rb < 4; ++rb) {
+                if (p.swiglu) {
+                  sg[rb] = rb >> 1;
+                  lr[rb] = nt * 128 + 64 * (rb & 1);
+                } else {
+                  const int row = nt * BN + 64 * rb;
+                  sg[rb] = row < p.N ? find_seg(p, row) : -1;
+                  lr[rb] = row < p.N ? row - p.seg_start[sg[rb]] : 0;
+                }
+                if (sg[rb] >= 0) ++nbox;
+              }
+              if (nbox) {
+                mbar_arrive_expect_tx(&codes_full[s], nbox * 2048);
+                for (int rb = 0; rb < 4; ++rb)
+                  if (sg[rb] >= 0) tma_load_2d(sC + rb * 2048, &p.tmC[sg[rb]], &codes_full[s], kb * (BK / 2), lr[rb]);
+              } else {
+                mbar_arrive(&codes_full[s]);
+              }
+            }
+          }
+        } else {
+          // LoRA extra block: A from the extra activations, B from the padded adapter
+          mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES);
+          tma_load_2d(sA, &p.tmAx, &full[s], 0, m0);
+          if (BMN) {
+            for (int j = 0; j < 4; ++j) tma_load_2d(sB + j * 8192, &p.tmBx, &full[s], nt * BN + 64 * j, 0);
+          } else {
+            tma_load_2d(sB, &p.tmBx, &full[s], 0, nt * BN);
+          }
+          if (DECODE) mbar_arrive(&codes_full[s]);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    constexpr uint32_t idesc = idesc_bf16(128, BN, BMN);
+    for (int kb = 0; kb < total_kb; ++kb) {
+      const int s = kb % STAGES;
+      const uint32_t ph = (kb / STAGES) & 1;
+      if (!mbar_wait(&full[s], ph, abort_flag, p.err, KID_GEMM, 2)) break;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t aA = smem_u32(base + s * STAGE_BYTES);
+        const uint32_t aB = aA + A_BYTES;
+#pragma unroll
+        for (int ks = 0; ks < BK / 16; ++ks) {
+          const uint64_t bdesc = BMN ? sdesc_sw128(aB + ks * 2048, 8192, 1024) : sdesc_sw128(aB + ks * 32, 16, 1024);
+#pragma unroll
+          for (int a = 0; a < 2; ++a) {
+            const uint64_t adesc = sdesc_sw128(aA + a * 16384 + ks * 32, 16, 1024);
+            umma_bf16(tmem + a * 256, adesc, bdesc, idesc, (kb | ks) != 0 ? 1u : 0u);
+          }
+        }
+        umma_commit(&empty[s]);
+      }
+      __syncwarp();
+    }
+    if (lane == 0) umma_commit(accum_full);
+    __syncwarp();
+  } else if (warp < 6) {
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp & 3;
+    if (mbar_wait(accum_full, 0, abort_flag, p.err, KID_GEMM, 3)) {
+      tc_fence_after();
+      for (int a = 0; a < 2; ++a) {
+        const int m = m0 + a * 128 + q * 32 + lane;
+        const bool mv = m < p.M;
+        const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + a * 256;
+        float v[32], w[32];
+        if (p.epi == EPI_SWIGLU) {
+          for (int c = 0; c < 4; ++c) {
+            ld_acc(tb + c * 32, v);
+            ld_acc(tb + 128 + c * 32, w);
+            if (!mv) continue;
+            const int col = nt * 128 + c * 32;
+            float o[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              v[i] = round_bf16(v[i]);
+              w[i] = round_bf16(w[i]);
+              o[i] = silu_f(v[i]) * w[i];
+            }
+            store32(p.out + (size_t)m * p.ldo + col, o);
+            if (p.aux_out) {
+              store32(p.aux_out + (size_t)m * p.ld_aux_out + col, v);
+              store32(p.aux_out + (size_t)m * p.ld_aux_out + p.inter + col, w);
+            }
+          }
+        } else if (p.epi == EPI_ROPE) {
+          const int d = p.head_dim, half = d / 2;
+          const int pos = m % p.seq;
+          for (int h = 0; h < BN / d; ++h) {
+            const int hc = nt * BN + h * d;
+            if (hc >= p.N) break;
+            if (hc < p.rope_cols) {
+              for (int i = 0; i < half / 32; ++i) {
+                ld_acc(tb + h * d + i * 32, v);
+                ld_acc(tb + h * d + half + i * 32, w);
+                if (!mv) continue;
+                const float* cs = p.rope_cos + (size_t)pos * half + i * 32;
+                const float* sn = p.rope_sin + (size_t)pos * half + i * 32;
+                float o1[32], o2[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                  const float c_ = cs[j], s_ = sn[j];
+                  o1[j] = v[j] * c_ - w[j] * s_;
+                  o2[j] = w[j] * c_ + v[j] * s_;
+                }
+                store32(p.out + (size_t)m * p.ldo + hc + i * 32, o1);
+                store32(p.out + (size_t)m * p.ldo + hc + half + i * 32, o2);
+              }
+            } else {
+              for (int c = 0; c < d / 32; ++c) {
+                ld_acc(tb + h * d + c * 32, v);
+                if (mv) store32(p.out + (size_t)m * p.ldo + hc + c * 32, v);
+              }
+            }
+          }
+        } else {
+          for (int c = 0; c < BN / 32; ++c) {
+            const int col = nt * BN + c * 32;
+            if (col >= p.N) break;
+            ld_acc(tb + c * 32, v);
+            if (!mv) continue;
+            if (p.epi == EPI_RESID) {
+              load32_bf16(p.aux0 + (size_t)m * p.ld_aux0 + col, w);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) v[i] += w[i];
+              store32(p.out + (size_t)m * p.ldo + col, v);
+            } else if (p.epi == EPI_DSWIGLU) {
+              float g[32], u[32], dg[32], du[32];
+              load32_bf16(p.aux0 + (size_t)m * p.ld_aux0 + col, g);
+              load32_bf16(p.aux0 + (size_t)m * p.ld_aux0 + p.inter + col, u);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const float sg = 1.0f / (1.0f + expf(-g[i]));
+                dg[i] = v[i] * u[i] * sg * (1.0f + g[i] * (1.0f - sg));
+                du[i] = v[i] * g[i] * sg;
+              }
+              store32(p.out + (size_t)m * p.ldo + col, dg);
+              store32(p.out + (size_t)m * p.ldo + p.inter + col, du);
+            } else {
+              store32(p.out + (size_t)m * p.ldo + col, v);
+            }
+          }
+        }
+      }
+    }
+  } else if (DECODE) {
+    // ---------------------------------------------------------------- NF4 decoders
+    const int d = threadIdx.x - 192;  // 0..255
+    float nf4[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) nf4[i] = p.nf4[i];
+    // forward: one B row per thread, constant over the reduction
+    int f_seg = 0, f_row = 0;
+    bool f_valid = true;
+    float f_off = 0.f;
+    if (!BMN) {
+      if (p.swiglu) {
+        f_seg = d >> 7;
+        f_row = nt * 128 + (d & 127);
+      } else {
+        const int row = nt * BN + d;
+        f_valid = row < p.N;
+        f_seg = f_valid ? find_seg(p, row) : 0;
+        f_row = f_valid ? row - p.seg_start[f_seg] : 0;
+      }
+      f_off = *p.offset[f_seg];
+    }
+    const int rr = d & 63, jj = d >> 6;          // dL/dx: reduction row and column block
+    const int dg_col = nt * BN + 64 * jj;         // first weight column of this thread's block
+    const int blocks_per_row = p.seg_cols / 64;
+    for (int kb = 0; kb < total_kb; ++kb) {
+      const int s = kb % STAGES;
+      const uint32_t ph = (kb / STAGES) & 1;
+      // scale inputs are independent of the code tile: fetch them before waiting
+      bool valid = false;
+      int b = 0, sg = 0;
+      uint32_t q8 = 0;
+      float nested = 0.f, off = 0.f;
+      if (kb < p.num_kb) {
+        if (BMN) {
+          const int row = kb * BK + rr;
+          sg = find_seg(p, kb * BK);
+          valid = dg_col < p.seg_cols;
+          b = (row - p.seg_start[sg]) * blocks_per_row + (dg_col >> 6);
+          if (valid) off = *p.offset[sg];
+        } else {
+          sg = f_seg;
+          valid = f_valid;
+          b = f_row * blocks_per_row + kb;
+          off = f_off;
+        }
+        if (valid) {
+          q8 = p.q8[sg][b];
+          nested = p.nested[sg][b >> 8];
+        }
+      }
+      if (!mbar_wait(&codes_full[s], ph, abort_flag, p.err, KID_GEMM, 4)) break;
+      if (kb < p.num_kb) {
+        const uint32_t sB = smem_u32(base + s * STAGE_BYTES + A_BYTES);
+        const uint32_t sC = sB + B_BYTES;
+        const uint32_t row_addr = BMN ? sB + jj * 8192 + rr * 128 : sB + d * 128;
+        const int row_in_atom = (BMN ? rr : d) & 7;
+        if (valid) {
+          const uint32_t caddr = BMN ? sC + rr * 128 + jj * 32 : sC + d * 32;
+          const uint4 c0 = ld_shared_v4(caddr), c1 = ld_shared_v4(caddr + 16);
+          const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+          const float sc = __fadd_rn(__fmul_rn(code8_s[q8], nested), off);
+          decode_block(row_addr, row_in_atom, w, sc, nf4);
+        } else {
+          zero_block(row_addr);
+        }
+        fence_proxy_async_smem();
+      }
+      mbar_arrive(&full[s]);
+    }
+  }
+
+  // On an aborted run the MMAs already issued must finish before TMEM is freed.
+  if (warp == 1 && *abort_flag) mbar_wait_drain(accum_full, 0);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+int make_map(CUtensorMap* map, CUtensorMapDataType dt, int esize, const void* ptr, uint64_t inner, uint64_t outer,
+             uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(NF4LS_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  if (!aligned(ptr, 16) || row_bytes % 16) return fail(NF4LS_ALIGN, "TMA operand base/row stride not 16-byte aligned");
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t es[2] = {1, 1};
+  (void)esize;
+  const CUresult r = fn(map, dt, 2, const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(NF4LS_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return NF4LS_OK;
+}
+
+template <bool DECODE, bool BMN>
+int launch(const GemmParams& p, int grid, cudaStream_t s) {
+  static int configured[16] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 16 && !configured[dev]) {
+    NF4_CUDA_TRY(cudaFuncSetAttribute(k_gemm<DECODE, BMN>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
+    configured[dev] = 1;
+  }
+  k_gemm<DECODE, BMN><<<grid, DECODE ? 448 : 192, SMEM_BYTES, s>>>(p);
+  NF4_CUDA_TRY(cudaGetLastError());
+  return NF4LS_OK;
+}
+
+}  // namespace
+
+int gemm(const __nv_bfloat16* A, int lda, int M, int N, int K, const GemmWeights& W, bool dgrad,
+         const GemmExtra& extra, const GemmEpilogue& epi, cudaStream_t s) {
+  if (!A || !epi.out) return fail(NF4LS_INVALID_ARG, "gemm: null operand");
+  if (M <= 0 || N <= 0 || K <= 0 || K % 64 || N % 64) return fail(NF4LS_SHAPE, "gemm: M=%d N=%d K=%d (K, N % 64)", M, N, K);
+  const bool decode = W.dense == nullptr;
+  const bool swiglu = epi.kind == EPI_SWIGLU;
+  if (decode && (W.n_seg < 1 || W.n_seg > 4)) return fail(NF4LS_INVALID_ARG, "gemm: 1-4 weight segments");
+  if (swiglu && (dgrad || epi.inter <= 0 || epi.inter % 128 || N != 2 * epi.inter))
+    return fail(NF4LS_SHAPE, "gemm: SwiGLU epilogue needs N = 2*I with I % 128 == 0");
+  if (epi.kind == EPI_ROPE && (epi.head_dim <= 0 || BN % epi.head_dim || epi.seq <= 0))
+    return fail(NF4LS_SHAPE, "gemm: RoPE epilogue head_dim");
+  static_assert(sizeof(GemmParams) <= 4096, "kernel parameters exceed 4 KB");
+
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.num_kb = K / 64;
+  p.has_extra = extra.a != nullptr;
+  p.n_mt = (M + BM - 1) / BM;
+  const int n_nt = swiglu ? epi.inter / 128 : (N + BN - 1) / BN;
+  NF4_TRY(make_map(&p.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A, K, M, (uint64_t)lda * 2, 64, 256, true));
+  if (p.has_extra) {
+    if (!extra.b) return fail(NF4LS_INVALID_ARG, "gemm: extra block needs both operands");
+    NF4_TRY(make_map(&p.tmAx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, extra.a, 64, M, 128, 64, 256, true));
+    if (dgrad)
+      NF4_TRY(make_map(&p.tmBx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, extra.b, N, 64, (uint64_t)N * 2, 64, 64, true));
+    else
+      NF4_TRY(make_map(&p.tmBx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, extra.b, 64, N, 128, 64, 256, true));
+  }
+  if (!decode) {
+    if (dgrad)  // W [K, N]
+      NF4_TRY(make_map(&p.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W.dense, N, K, (uint64_t)N * 2, 64, 64, true));
+    else if (swiglu) {  // W [2I, K]: gate rows then up rows
+      NF4_TRY(make_map(&p.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W.dense, K, N, (uint64_t)K * 2, 64, 128, true));
+      p.dense_swiglu_rows = epi.inter;
+    } else
+      NF4_TRY(make_map(&p.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W.dense, K, N, (uint64_t)K * 2, 64, 256, true));
+  } else {
+    p.n_seg = W.n_seg;
+    p.swiglu = swiglu;
+    int start = 0;
+    const int cols = W.seg[0].cols;
+    for (int i = 0; i < W.n_seg; ++i) {
+      const NF4Tensor& t = W.seg[i];
+      if (t.cols != cols || t.rows % 64) return fail(NF4LS_SHAPE, "gemm: segment %d shape", i);
+      p.seg_start[i] = start;
+      start += t.rows;
+      p.q8[i] = t.q8;
+      p.nested[i] = t.nested;
+      p.offset[i] = t.offset;
+      if (dgrad)  // codes [rows, N/2] bytes; box 128 B x 64 rows
+        NF4_TRY(make_map(&p.tmC[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, t.packed, cols / 2, t.rows, cols / 2, 128, 64, false));
+      else  // codes [rows, K/2] bytes; box 32 B x 64 rows
+        NF4_TRY(make_map(&p.tmC[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, t.packed, cols / 2, t.rows, cols / 2, 32, 64, false));
+    }
+    p.seg_start[W.n_seg] = start;
+    p.seg_cols = cols;
+    if (dgrad && (start != K || cols != N)) return fail(NF4LS_SHAPE, "gemm: dL/dx segments do not match K x N");
+    if (!dgrad && (start != N || cols != K)) return fail(NF4LS_SHAPE, "gemm: forward segments do not match N x K");
+    if (swiglu && (W.n_seg != 2 || W.seg[0].rows != epi.inter || W.seg[1].rows != epi.inter))
+      return fail(NF4LS_SHAPE, "gemm: SwiGLU needs gate and up segments of I rows");
+    const Codebooks& cb = codebooks();
+    std::memcpy(p.nf4, cb.nf4, sizeof(p.nf4));
+    std::memcpy(p.code8, cb.code8, sizeof(p.code8));
+  }
+  p.epi = epi.kind;
+  p.out = epi.out;
+  p.ldo = epi.ldo;
+  p.aux0 = epi.aux0;
+  p.ld_aux0 = epi.ld_aux0;
+  p.aux_out = epi.aux_out;
+  p.ld_aux_out = epi.ld_aux_out;
+  p.inter = epi.inter;
+  p.rope_cos = epi.rope_cos;
+  p.rope_sin = epi.rope_sin;
+  p.seq = epi.seq;
+  p.head_dim = epi.head_dim;
+  p.rope_cols = epi.rope_cols;
+  p.err = device_error_ptr();
+  const int grid = p.n_mt * n_nt;
+  if (decode) return dgrad ? launch<true, true>(p, grid, s) : launch<true, false>(p, grid, s);
+  return dgrad ? launch<false, true>(p, grid, s) : launch<false, false>(p, grid, s);
+}
+
+}  // namespace nf4ls
+
+extern "C" int nf4ls_gemm_bf16(const void* A_dev, const void* B_dev, void* out_dev, int M, int N, int K, int b_trans,
+                               int ldo, nf4ls_stream stream) {
+  nf4ls::clear_error();
+  nf4ls::GemmWeights W;
+  W.dense = static_cast<const __nv_bfloat16*>(B_dev);
+  if (!W.dense) return nf4ls::fail(NF4LS_INVALID_ARG, "nf4ls_gemm_bf16: null B");
+  nf4ls::GemmEpilogue e;
+  e.out = static_cast<__nv_bfloat16*>(out_dev);
+  e.ldo = ldo;
+  return nf4ls::gemm(static_cast<const __nv_bfloat16*>(A_dev), K, M, N, K, W, b_trans != 0, nf4ls::GemmExtra(), e,
+                     static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int nf4ls_gemm_nf4(const void* A_dev, int lda, int M, const uint8_t* packed_dev, const uint8_t* q8_dev,
+                              const float* nested_dev, const float* offset_dev, int rows, int cols, int dgrad,
+                              void* out_dev, int ldo, nf4ls_stream stream) {
+  nf4ls::clear_error();
+  nf4ls::GemmWeights W;
+  W.n_seg = 1;
+  W.seg[0] = nf4ls::NF4Tensor{packed_dev, q8_dev, nested_dev, offset_dev, rows, cols};
+  nf4ls::GemmEpilogue e;
+  e.out = static_cast<__nv_bfloat16*>(out_dev);
+  e.ldo = ldo;
+  const int N = dgrad ? cols : rows, K = dgrad ? rows : cols;
+  return nf4ls::gemm(static_cast<const __nv_bfloat16*>(A_dev), lda, M, N, K, W, dgrad != 0, nf4ls::GemmExtra(), e,
+                     static_cast<cudaStream_t>(stream));
+}

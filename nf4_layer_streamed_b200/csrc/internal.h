@@ -1,0 +1,164 @@
+// Host-side internals of libnf4ls shared between translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/nf4ls.h"
+
+namespace nf4ls {
+
+// ----------------------------------------------------------------------------- status
+int fail(int status, const char* fmt, ...);
+void clear_error();
+
+#define NF4_CUDA_TRY(expr)                                                                             \
+  do {                                                                                                 \
+    cudaError_t e_ = (expr);                                                                           \
+    if (e_ != cudaSuccess)                                                                             \
+      return ::nf4ls::fail(NF4LS_CUDA, "%s failed: %s (%s:%d)", #expr, cudaGetErrorString(e_), __FILE__, \
+                           __LINE__);                                                                  \
+  } while (0)
+
+#define NF4_TRY(expr)         \
+  do {                        \
+    int s_ = (expr);          \
+    if (s_ != NF4LS_OK) return s_; \
+  } while (0)
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ----------------------------------------------------------------------------- code tables
+struct Codebooks {
+  float nf4[16];
+  float code8[256];
+  float mid4[15];   // fp32 midpoints between neighbouring NF4 entries
+  float mid8[255];  // fp32 midpoints between neighbouring code8 entries
+  int zero4;        // index of the exact 0 in nf4
+  int zero8;        // index of the exact 0 in code8
+  uint64_t hash;
+};
+const Codebooks& codebooks();
+
+// ----------------------------------------------------------------------------- quantiser
+int quantize_tensor(const void* w, size_t n, uint8_t* packed, uint8_t* q8, float* nested, float* offset,
+                    void* scratch, size_t scratch_bytes, cudaStream_t s);
+int dequantize_tensor(const uint8_t* packed, const uint8_t* q8, const float* nested, const float* offset,
+                      size_t n, void* out, cudaStream_t s);
+
+// ----------------------------------------------------------------------------- shard view
+struct NF4Tensor {
+  const uint8_t* packed;
+  const uint8_t* q8;
+  const float* nested;
+  const float* offset;
+  int rows, cols;
+};
+struct ShardView {
+  NF4Tensor t[7];
+  const __nv_bfloat16* norm_in;
+  const __nv_bfloat16* norm_post;
+};
+// Builds device pointers into a shard at shard_dev from the layout that cfg implies.
+void shard_view(const nf4ls_layer_cfg* cfg, const void* shard_dev, ShardView* v);
+struct ShardLayout {
+  uint64_t off_packed[7], off_q8[7], off_nested[7], off_offset[7];
+  uint64_t off_norm_in, off_norm_post;
+  uint64_t total, quantized;
+  int rows[7], cols[7];
+};
+void shard_layout(const nf4ls_layer_cfg* cfg, ShardLayout* L);
+
+// ----------------------------------------------------------------------------- GEMM
+// Output epilogues of the tcgen05 GEMM (accumulator fp32 -> bf16 stores).
+enum Epilogue : int {
+  EPI_STORE = 0,    // out = acc
+  EPI_RESID = 1,    // out = acc + aux0[m, n]
+  EPI_ROPE = 2,     // out = rope(acc) on columns < rope_cols, acc elsewhere
+  EPI_SWIGLU = 3,   // columns [0,128) gate, [128,256) up of block i: out[m, i] = silu(g) * u; aux_out g,u
+  EPI_DSWIGLU = 4,  // acc = da[m, i]; aux0 = [g | u] -> out = [dg | du]
+};
+
+struct GemmEpilogue {
+  int kind = EPI_STORE;
+  __nv_bfloat16* out = nullptr;
+  int ldo = 0;
+  const __nv_bfloat16* aux0 = nullptr;  // residual / g,u source
+  int ld_aux0 = 0;
+  __nv_bfloat16* aux_out = nullptr;     // g,u store of EPI_SWIGLU (may be null)
+  int ld_aux_out = 0;
+  int inter = 0;                        // I for the SwiGLU layouts
+  const float* rope_cos = nullptr;      // [seq, d/2]
+  const float* rope_sin = nullptr;
+  int seq = 0, head_dim = 0, rope_cols = 0;
+};
+
+// Weights of a GEMM: either one dense bf16 matrix, or up to four NF4 tensors that
+// are concatenated along the weight's rows (its output features).
+struct GemmWeights {
+  const __nv_bfloat16* dense = nullptr;  // [rows, cols] row-major
+  int n_seg = 0;
+  NF4Tensor seg[4];
+};
+
+struct GemmExtra {
+  // One extra 64-wide reduction block appended after the main reduction: the LoRA
+  // up-projection (forward) or the LoRA A^T product (dL/dx).  a: bf16 [M, 64];
+  // b: bf16 [N, 64] (forward, K-major) or [64, N] (dL/dx, N-major).
+  const __nv_bfloat16* a = nullptr;
+  const __nv_bfloat16* b = nullptr;
+};
+
+// Forward product out[M, N] = A[M, K] W^T, W [N, K] (weights rows = N).
+// dL/dx product out[M, N] = A[M, K] W, W [K, N] (weights rows = K, the reduction).
+int gemm(const __nv_bfloat16* A, int lda, int M, int N, int K, const GemmWeights& W, bool dgrad,
+         const GemmExtra& extra, const GemmEpilogue& epi, cudaStream_t s);
+
+int gemm_path();
+int check_cfg(const nf4ls_layer_cfg* c);
+int* device_error_ptr();
+
+// ----------------------------------------------------------------------------- body kernels
+int rmsnorm_fwd(const __nv_bfloat16* x, const __nv_bfloat16* w, __nv_bfloat16* y, int M, int H, float eps,
+                cudaStream_t s);
+// dx = resid + rmsnorm_bwd(x, w, dy); resid may be null.
+int rmsnorm_bwd(const __nv_bfloat16* x, const __nv_bfloat16* w, const __nv_bfloat16* dy,
+                const __nv_bfloat16* resid, __nv_bfloat16* dx, int M, int H, float eps, cudaStream_t s);
+int rope_tables(float* cos_t, float* sin_t, int seq, int d, float theta, cudaStream_t s);
+int rope_bwd(__nv_bfloat16* x, int ld, int M, int cols, int seq, int d, const float* cos_t,
+             const float* sin_t, cudaStream_t s);
+int attention_fwd(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, int ldq, int ldkv,
+                  __nv_bfloat16* o, int ldo, float* lse, int batch, int seq, int nq, int nkv, int d,
+                  cudaStream_t s);
+int attention_bwd(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, int ldq, int ldkv,
+                  const __nv_bfloat16* o, const __nv_bfloat16* dout, int ldo, const float* lse, float* delta,
+                  __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv, int ld_dq, int ld_dkv, int batch,
+                  int seq, int nq, int nkv, int d, cudaStream_t s);
+
+int lora_skinny(const __nv_bfloat16* X, int ldx, int M, int K, const float* W, int sr, int sk, float scale,
+                float* out_f, __nv_bfloat16* out_b, int ldb, int oc, cudaStream_t s);
+int lora_grad_reduce(const __nv_bfloat16* X, int ldx, int M, int N, const float* y_f, const __nv_bfloat16* y_b, int ldy,
+                     int yc, float scale, float* out, int so_n, int so_r, cudaStream_t s);
+int lora_pack(const nf4ls_lora* l, int H, int qd, int kvd, float scale, __nv_bfloat16* bup, __nv_bfloat16* adn,
+              cudaStream_t s);
+int zero_cols(__nv_bfloat16* x, int ld, int M, int c0, int c1, cudaStream_t s);
+int embed(const int32_t* ids, const __nv_bfloat16* E, __nv_bfloat16* h, int M, int H, cudaStream_t s);
+int cross_entropy(const __nv_bfloat16* logits, const int32_t* ids, int M, int V, int batch, int seq, float* row_loss,
+                  __nv_bfloat16* dlogits, float* loss, cudaStream_t s);
+int mse_loss(const __nv_bfloat16* out, size_t n, float* partial, int n_partial, __nv_bfloat16* dout, float* loss,
+             cudaStream_t s);
+int adamw(float* p, const float* g, float* m, float* v, size_t n, int step, float lr, float b1, float b2, float eps,
+          float wd, cudaStream_t s);
+
+// ----------------------------------------------------------------------------- layer
+int layer_fwd_impl(const nf4ls_layer_cfg* cfg, const void* shard, const nf4ls_lora* lora, const __nv_bfloat16* x,
+                   __nv_bfloat16* y, void* ws, size_t ws_bytes, cudaStream_t s);
+int layer_bwd_impl(const nf4ls_layer_cfg* cfg, const void* shard, const nf4ls_lora* lora, const __nv_bfloat16* x,
+                   const __nv_bfloat16* dy, __nv_bfloat16* dx, const nf4ls_lora_grads* g, void* ws, size_t ws_bytes,
+                   cudaStream_t s);
+size_t layer_ws_bytes(const nf4ls_layer_cfg* cfg);
+
+}  // namespace nf4ls

@@ -1,0 +1,228 @@
+// One SFT step of the whole stack: embedding -> streamed decoder layers (forward,
+// saving each layer input) -> final RMSNorm -> lm_head -> causal-LM cross-entropy ->
+// lm_head and final-norm backward -> streamed decoder layers in reverse (checkpoint
+// recompute + dL/dx + LoRA gradients) -> AdamW on the LoRA tensors.
+//
+// From the layer-streaming review ("4GB 显存微调 8B 模型是真的", mechanism section):
+// only the adapter, its gradients and its optimiser state stay resident, together with
+// the unquantised embedding and lm_head; the frozen layers are prefetched one step
+// ahead on a side stream, i+1 in the forward and i-1 in the backward.  From the gate
+// record §4.4: lm_head sits outside the checkpointed layers (2 forward + 2 dL/dx FLOP
+// per parameter and token).  The DPO/KTO write-up ("Soup v0.72.4 技术解析" §3.1) reuses
+// the same streamed base with the adapter switched off as the reference model, which
+// nf4ls_forward_loss(lora_on = 0) provides.
+#include "common.cuh"
+#include "internal.h"
+
+namespace nf4ls {
+
+namespace {
+
+struct ModelWs {
+  size_t xs, hf, logits, row_loss, dh, dhf, layer, total;
+};
+
+ModelWs model_ws(const nf4ls_model_cfg* c) {
+  const size_t M = (size_t)c->layer.batch * c->layer.seq, H = c->layer.hidden;
+  ModelWs L;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = round_up(off + bytes, 256);
+    return o;
+  };
+  L.xs = take((size_t)(c->n_layers + 1) * M * H * 2);
+  L.hf = take(M * H * 2);
+  L.logits = take(M * (size_t)c->vocab * 2);
+  L.row_loss = take(M * 4);
+  L.dh = take(M * H * 2);
+  L.dhf = take(M * H * 2);
+  L.layer = take(layer_ws_bytes(&c->layer));
+  L.total = off;
+  return L;
+}
+
+size_t stride_of(const nf4ls_layer_cfg* c) {
+  const size_t r = c->lora_r, H = c->hidden;
+  return r * H + (size_t)c->n_q * c->head_dim * r + r * H + (size_t)c->n_kv * c->head_dim * r;
+}
+
+void lora_views(const nf4ls_layer_cfg* c, float* base, nf4ls_lora* l, nf4ls_lora_grads* g, float* gbase) {
+  const size_t r = c->lora_r, H = c->hidden, qd = (size_t)c->n_q * c->head_dim;
+  l->A_q = base;
+  l->B_q = base + r * H;
+  l->A_v = base + r * H + qd * r;
+  l->B_v = base + 2 * r * H + qd * r;
+  if (g) {
+    g->dA_q = gbase;
+    g->dB_q = gbase + r * H;
+    g->dA_v = gbase + r * H + qd * r;
+    g->dB_v = gbase + 2 * r * H + qd * r;
+  }
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+int acquire(const nf4ls_model* m, int layer, int dir, cudaStream_t s, const void** shard) {
+  if (!m->pool) {
+    *shard = m->shards_dev[layer];
+    return NF4LS_OK;
+  }
+  NF4_TRY(stream_prefetch(m->pool, layer, s, shard));
+  return NF4LS_OK;
+}
+
+int lookahead(const nf4ls_model* m, const nf4ls_model_cfg* c, int layer, int dir, int depth) {
+  if (!m->pool) return NF4LS_OK;
+  for (int k = 1; k < depth; ++k) {
+    const int j = layer + dir * k;
+    if (j < 0 || j >= c->n_layers) break;
+    const int st = nf4ls_pool_prefetch(m->pool, j);
+    if (st == NF4LS_BUFFER_BUSY) break;  // no free slot yet: the next acquire copies it
+    NF4_TRY(st);
+  }
+  return NF4LS_OK;
+}
+
+int release(const nf4ls_model* m, int layer, cudaStream_t s) {
+  if (!m->pool) return NF4LS_OK;
+  return nf4ls_pool_release(m->pool, layer, s);
+}
+
+int check_model(const nf4ls_model_cfg* c, const nf4ls_model* m) {
+  if (!c || !m) return fail(NF4LS_INVALID_ARG, "model: null config or model");
+  NF4_TRY(check_cfg(&c->layer));
+  if (c->n_layers <= 0 || c->vocab <= 0 || c->vocab % 64) return fail(NF4LS_SHAPE, "model: vocab must be a multiple of 64");
+  if (!m->embed_dev || !m->norm_final_dev || !m->lora_dev || !m->ws_dev) return fail(NF4LS_INVALID_ARG, "model: null buffer");
+  if (!c->tied && !m->lm_head_dev) return fail(NF4LS_INVALID_ARG, "model: untied model needs lm_head");
+  if (!m->pool && !m->shards_dev) return fail(NF4LS_INVALID_ARG, "model: needs a pool or resident shards");
+  if (!aligned(m->ws_dev, 256)) return fail(NF4LS_ALIGN, "model: workspace must be 256-byte aligned");
+  if (m->ws_bytes < model_ws(c).total) return fail(NF4LS_INVALID_ARG, "model: workspace too small");
+  return NF4LS_OK;
+}
+
+int pool_depth(const nf4ls_model* m) {
+  if (!m->pool) return 1;
+  return 2;  // prefetch one layer ahead, as the pages do
+}
+
+// Forward through embedding, layers, final norm, lm_head and the loss.
+int forward_to_loss(const nf4ls_model_cfg* c, const nf4ls_model* m, const int32_t* ids, bool lora_on, float* loss,
+                    cudaStream_t s, const ModelWs& L) {
+  const nf4ls_layer_cfg* lc = &c->layer;
+  const int M = lc->batch * lc->seq, H = lc->hidden, V = c->vocab;
+  void* ws = m->ws_dev;
+  auto* xs = at<__nv_bfloat16>(ws, L.xs);
+  const size_t act = (size_t)M * H;
+  const size_t stride = stride_of(lc);
+  NF4_TRY(embed(ids, static_cast<const __nv_bfloat16*>(m->embed_dev), xs, M, H, s));
+  const int depth = pool_depth(m);
+  for (int i = 0; i < c->n_layers; ++i) {
+    const void* shard;
+    NF4_TRY(acquire(m, i, +1, s, &shard));
+    NF4_TRY(lookahead(m, c, i, +1, depth));
+    nf4ls_lora l;
+    lora_views(lc, m->lora_dev + (size_t)i * stride, &l, nullptr, nullptr);
+    NF4_TRY(layer_fwd_impl(lc, shard, lora_on ? &l : nullptr, xs + (size_t)i * act, xs + (size_t)(i + 1) * act,
+                           at<void>(ws, L.layer), L.total - L.layer, s));
+    NF4_TRY(release(m, i, s));
+  }
+  auto* hf = at<__nv_bfloat16>(ws, L.hf);
+  auto* logits = at<__nv_bfloat16>(ws, L.logits);
+  const auto* lm = static_cast<const __nv_bfloat16*>(c->tied ? m->embed_dev : m->lm_head_dev);
+  NF4_TRY(rmsnorm_fwd(xs + (size_t)c->n_layers * act, static_cast<const __nv_bfloat16*>(m->norm_final_dev), hf, M, H,
+                      lc->rms_eps, s));
+  GemmWeights w;
+  w.dense = lm;
+  GemmEpilogue e;
+  e.out = logits;
+  e.ldo = V;
+  NF4_TRY(gemm(hf, H, M, V, H, w, false, GemmExtra(), e, s));
+  // dlogits overwrite the logits in place
+  return cross_entropy(logits, ids, M, V, lc->batch, lc->seq, at<float>(ws, L.row_loss), logits, loss, s);
+}
+
+}  // namespace
+
+}  // namespace nf4ls
+
+using namespace nf4ls;
+
+extern "C" size_t nf4ls_lora_stride(const nf4ls_layer_cfg* cfg) { return cfg ? stride_of(cfg) : 0; }
+
+extern "C" size_t nf4ls_model_workspace_bytes(const nf4ls_model_cfg* cfg) { return cfg ? model_ws(cfg).total : 0; }
+
+extern "C" int nf4ls_forward_loss(const nf4ls_model_cfg* cfg, const nf4ls_model* m, const int32_t* ids_dev,
+                                  int32_t lora_on, float* loss_dev, nf4ls_stream stream) {
+  clear_error();
+  NF4_TRY(check_model(cfg, m));
+  if (!ids_dev || !loss_dev) return fail(NF4LS_INVALID_ARG, "nf4ls_forward_loss: null ids or loss");
+  return forward_to_loss(cfg, m, ids_dev, lora_on != 0, loss_dev, static_cast<cudaStream_t>(stream), model_ws(cfg));
+}
+
+extern "C" int nf4ls_forward_backward(const nf4ls_model_cfg* cfg, const nf4ls_model* m, const int32_t* ids_dev,
+                                      float* loss_dev, nf4ls_stream stream) {
+  clear_error();
+  NF4_TRY(check_model(cfg, m));
+  if (!ids_dev || !loss_dev || !m->grads_dev) return fail(NF4LS_INVALID_ARG, "nf4ls_forward_backward: null argument");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const ModelWs L = model_ws(cfg);
+  NF4_TRY(forward_to_loss(cfg, m, ids_dev, true, loss_dev, s, L));
+  const nf4ls_layer_cfg* lc = &cfg->layer;
+  const int M = lc->batch * lc->seq, H = lc->hidden, V = cfg->vocab;
+  void* ws = m->ws_dev;
+  auto* xs = at<__nv_bfloat16>(ws, L.xs);
+  const size_t act = (size_t)M * H;
+  auto* logits = at<__nv_bfloat16>(ws, L.logits);  // now dlogits
+  auto* dhf = at<__nv_bfloat16>(ws, L.dhf);
+  auto* dh = at<__nv_bfloat16>(ws, L.dh);
+  const auto* lm = static_cast<const __nv_bfloat16*>(cfg->tied ? m->embed_dev : m->lm_head_dev);
+  GemmWeights w;
+  w.dense = lm;
+  GemmEpilogue e;
+  e.out = dhf;
+  e.ldo = H;
+  NF4_TRY(gemm(logits, V, M, H, V, w, true, GemmExtra(), e, s));
+  NF4_TRY(rmsnorm_bwd(xs + (size_t)cfg->n_layers * act, static_cast<const __nv_bfloat16*>(m->norm_final_dev), dhf,
+                      nullptr, dh, M, H, lc->rms_eps, s));
+  const size_t stride = stride_of(lc);
+  const int depth = pool_depth(m);
+  for (int i = cfg->n_layers - 1; i >= 0; --i) {
+    const void* shard;
+    NF4_TRY(acquire(m, i, -1, s, &shard));
+    NF4_TRY(lookahead(m, cfg, i, -1, depth));
+    nf4ls_lora l;
+    nf4ls_lora_grads g;
+    lora_views(lc, m->lora_dev + (size_t)i * stride, &l, &g, m->grads_dev + (size_t)i * stride);
+    NF4_TRY(layer_bwd_impl(lc, shard, &l, xs + (size_t)i * act, dh, dh, &g, at<void>(ws, L.layer), L.total - L.layer, s));
+    NF4_TRY(release(m, i, s));
+  }
+  return NF4LS_OK;
+}
+
+extern "C" int nf4ls_adamw_step(const nf4ls_model_cfg* cfg, const nf4ls_model* m, int32_t step, nf4ls_stream stream) {
+  clear_error();
+  if (!cfg || !m || !m->lora_dev || !m->grads_dev || !m->adam_m_dev || !m->adam_v_dev || step < 1)
+    return fail(NF4LS_INVALID_ARG, "nf4ls_adamw_step: bad argument");
+  const size_t n = (size_t)cfg->n_layers * stride_of(&cfg->layer);
+  return adamw(m->lora_dev, m->grads_dev, m->adam_m_dev, m->adam_v_dev, n, step, cfg->lr, cfg->beta1, cfg->beta2,
+               cfg->adam_eps, cfg->weight_decay, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int nf4ls_train_step(const nf4ls_model_cfg* cfg, const nf4ls_model* m, const int32_t* ids_dev, int32_t step,
+                                float* loss_dev, nf4ls_stream stream) {
+  NF4_TRY(nf4ls_forward_backward(cfg, m, ids_dev, loss_dev, stream));
+  return nf4ls_adamw_step(cfg, m, step, stream);
+}
+
+extern "C" int nf4ls_mse_loss(const void* out_dev, size_t n, void* dout_dev, float* loss_dev, float* partial_dev,
+                              int n_partial, nf4ls_stream stream) {
+  clear_error();
+  if (!out_dev || !dout_dev || !loss_dev || !partial_dev || n_partial <= 0 || n_partial > 4096)
+    return fail(NF4LS_INVALID_ARG, "nf4ls_mse_loss: bad argument");
+  return mse_loss(static_cast<const __nv_bfloat16*>(out_dev), n, partial_dev, n_partial,
+                  static_cast<__nv_bfloat16*>(dout_dev), loss_dev, static_cast<cudaStream_t>(stream));
+}

@@ -1,0 +1,108 @@
+"""C-ABI library checks that need no GPU: the library loads, exports every symbol the
+header declares, builds code tables equal to the oracle's, sizes shards by the byte
+identity, and refuses bad headers, sizes and pool depths on the host."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from nf4_layer_streamed_b200 import api, binding as B, synth
+from oracle import account, codebooks
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "nf4ls.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b([A-Za-z_][A-Za-z0-9_]*)\s*\([^;{]*\)\s*;", text)
+    return sorted(set(n for n in names if n not in ("defined",)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = B.lib()
+    declared = _declared_functions()
+    assert len(declared) >= 30
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(declared) == set(B.SIGNATURES), set(declared) ^ set(B.SIGNATURES)
+
+
+def test_code_tables_equal_oracle_bit_for_bit():
+    nf4, c8, h = api.codebooks()
+    assert np.array_equal(nf4.view(np.uint32), codebooks.nf4_table().view(np.uint32))
+    assert np.array_equal(c8.view(np.uint32), codebooks.code8_table().view(np.uint32))
+    assert h == codebooks.codebook_hash()
+
+
+@pytest.mark.parametrize("shape", [synth.SMOLLM2_135M, synth.LLAMA_8B, synth.QWEN_32B_CLASS])
+def test_shard_sizes_follow_byte_identity(shape):
+    cfg = api.layer_cfg(shape, 1, 512)
+    assert api.shard_quantized_bytes(cfg) == account.layer_shard_bytes(shape)
+    total = api.shard_bytes(cfg)
+    # header + descriptors + 256-byte alignment of 30 regions + two bf16 norm vectors
+    assert account.layer_shard_bytes(shape) < total <= account.layer_shard_bytes(shape) + 1024 + 30 * 256 + \
+        4 * shape.hidden + 512
+
+
+def _header(cfg, fp=7, magic=0x5334464E, version=1, chash=None):
+    h = np.zeros(1024, np.uint8)
+    u32 = h[:48].view(np.uint32)
+    u32[:] = [magic, version, 1, 64, 256, 9, cfg.hidden, cfg.inter, cfg.n_q, cfg.n_kv, cfg.head_dim, 0]
+    u64 = h[48:80].view(np.uint64)
+    u64[0] = codebooks.codebook_hash() if chash is None else chash
+    u64[1] = fp
+    u64[2] = api.shard_bytes(cfg)
+    return h
+
+
+def test_shard_header_checks():
+    cfg = api.layer_cfg(synth.SMOLLM2_135M, 1, 512)
+    ok = _header(cfg)
+    st = B.call_status("nf4ls_shard_check", ok.ctypes.data, ctypes.byref(cfg), 7)
+    assert st == B.OK, B.last_error()
+    assert B.call_status("nf4ls_shard_check", ok.ctypes.data, ctypes.byref(cfg), 8) == -5   # fingerprint
+    bad = _header(cfg, chash=123)
+    assert B.call_status("nf4ls_shard_check", bad.ctypes.data, ctypes.byref(cfg), 0) == -4  # code tables
+    bad = _header(cfg, magic=0)
+    assert B.call_status("nf4ls_shard_check", bad.ctypes.data, ctypes.byref(cfg), 0) == -1
+    other = api.layer_cfg(synth.LLAMA_8B, 1, 512)
+    assert B.call_status("nf4ls_shard_check", ok.ctypes.data, ctypes.byref(other), 0) == -2  # shape
+
+
+def test_pool_rejects_bad_depth_and_sizes_without_touching_a_gpu():
+    store = np.zeros(4096, np.uint8)
+    offs = (ctypes.c_size_t * 2)(0, 2048)
+    sizes = (ctypes.c_size_t * 2)(1024, 1024)
+    out = ctypes.c_void_p()
+    fake_dev = ctypes.c_void_p(1 << 20)  # never dereferenced: arguments are rejected first
+    for depth in (1, 9):
+        st = B.call_status("nf4ls_pool_create", store.ctypes.data, ctypes.cast(offs, ctypes.c_void_p),
+                           ctypes.cast(sizes, ctypes.c_void_p), 2, depth, fake_dev, 2048, ctypes.byref(out))
+        assert st == -1 and "depth" in B.last_error()
+    st = B.call_status("nf4ls_pool_create", store.ctypes.data, ctypes.cast(offs, ctypes.c_void_p),
+                       ctypes.cast(sizes, ctypes.c_void_p), 2, 2, fake_dev, 512, ctypes.byref(out))
+    assert st == -1 and "exceeds slot" in B.last_error()
+    st = B.call_status("nf4ls_pool_create", store.ctypes.data, ctypes.cast(offs, ctypes.c_void_p),
+                       ctypes.cast(sizes, ctypes.c_void_p), 2, 2, ctypes.c_void_p((1 << 20) + 8), 2048,
+                       ctypes.byref(out))
+    assert st == -3
+
+
+def test_workspace_queries_and_options():
+    cfg = api.layer_cfg(synth.LLAMA_8B, 4, 512)
+    assert B.lib().nf4ls_workspace_bytes(ctypes.byref(cfg)) > 0
+    assert B.lib().nf4ls_lora_stride(ctypes.byref(cfg)) == 16 * (2 * 4096 + 4096 + 1024)
+    assert B.call_status("nf4ls_set_gemm_path", 3) == -1
+    assert B.call_status("nf4ls_set_gemm_path", 0) == 0
+    assert B.lib().nf4ls_quantize_scratch_bytes(64 * 1000) >= 4000
+
+
+def test_layer_calls_validate_config_on_host():
+    cfg = api.layer_cfg(synth.SMOLLM2_135M, 1, 512)
+    cfg.head_dim = 96
+    st = B.call_status("layer_forward", ctypes.byref(cfg), ctypes.c_void_p(256), None, ctypes.c_void_p(256),
+                       ctypes.c_void_p(256), ctypes.c_void_p(256), 1 << 30, None)
+    assert st == -2

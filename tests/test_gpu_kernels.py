@@ -1,0 +1,134 @@
+"""Parity of the individual CUDA kernels against the oracle (GPU).
+
+Quantiser and dequantiser: bit-exact bytes and bf16 values, including zero blocks,
+partial nested groups, one-block tensors and the full Llama-8B q_proj.  GEMMs: the
+tcgen05 kernel against a float64 product of the same bf16 operands; the in-mainloop
+NF4 decode against the dense kernel on the oracle's dequantised weights, bit for bit.
+Attention forward against the oracle's causal GQA attention.
+"""
+import numpy as np
+import pytest
+import torch
+
+from nf4_layer_streamed_b200 import api, synth
+from oracle import bf16 as obf16, layer as olayer, quant
+from tests.helpers import TOL, close, f64
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _q_to_np(q):
+    return {"packed": q["packed"].cpu().numpy(), "q8": q["q8"].cpu().numpy(), "nested": q["nested"].cpu().numpy(),
+            "offset": np.float32(q["offset"].cpu().numpy()[0])}
+
+
+@pytest.mark.parametrize("shape,seed", [((1, 64), 1), ((257, 64), 2), ((192, 576), 3),
+                                        ((1536, 576), 4), ((4096, 4096), 5)])
+def test_quantize_bit_exact_against_oracle(shape, seed):
+    w = synth.tensor_values(shape, seed=seed, scale=0.02)
+    if w.numel() >= 256:
+        w.view(-1)[64:128] = 0                     # a zero block
+    q = api.nf4_quantize_tensor(w.to(DEV))
+    torch.cuda.synchronize()
+    ref = quant.quantize(w.float().numpy().reshape(-1))
+    got = _q_to_np(q)
+    assert got["offset"] == ref["offset"]
+    np.testing.assert_array_equal(got["nested"], ref["nested"])
+    np.testing.assert_array_equal(got["q8"], ref["q8"])
+    np.testing.assert_array_equal(got["packed"], ref["packed"])
+    deq = api.nf4_dequantize_tensor(q)
+    np.testing.assert_array_equal(deq.view(torch.int16).cpu().numpy().view(np.uint16), quant.dequantize_bits(ref))
+
+
+def test_quantize_deterministic_across_calls():
+    w = synth.tensor_values((1024, 4096), seed=11, scale=0.02).to(DEV)
+    a, b = api.nf4_quantize_tensor(w), api.nf4_quantize_tensor(w)
+    for k in ("packed", "q8", "nested", "offset"):
+        assert torch.equal(a[k], b[k])
+
+
+def test_quantize_extreme_values():
+    # one huge block and tiny blocks: nested range and offset far from most absmax values
+    w = synth.tensor_values((64, 256), seed=12, scale=1e-3)
+    w.view(-1)[:64] = 30.0
+    w.view(-1)[64:128] = -1e-30
+    q = api.nf4_quantize_tensor(w.to(DEV))
+    ref = quant.quantize(w.float().numpy().reshape(-1))
+    got = _q_to_np(q)
+    np.testing.assert_array_equal(got["packed"], ref["packed"])
+    np.testing.assert_array_equal(got["q8"], ref["q8"])
+    assert got["offset"] == ref["offset"]
+
+
+def test_shard_regions_match_oracle_and_header():
+    shape = synth.SMOLLM2_135M
+    cfg = api.layer_cfg(shape, 1, 512)
+    w = synth.layer_weights(shape, 0, 1234, device=DEV)
+    shard = api.nf4_quantize_shard(cfg, w, fingerprint=42)
+    torch.cuda.synchronize()
+    host = shard.cpu().numpy()
+    assert api.shard_check(shard, cfg, 42) == 0
+    assert api.shard_check(shard, cfg, 43) == -5
+    desc = host[256:256 + 9 * 64].view(np.uint64).reshape(9, 8)
+    for t, name in enumerate(("q", "k", "v", "o", "gate", "up", "down")):
+        rows, cols = int(desc[t, 1]), int(desc[t, 2])
+        assert (rows, cols) == tuple(w[name].shape)
+        n = rows * cols
+        ref = quant.quantize(w[name].float().cpu().numpy().reshape(-1))
+        op, oq, on, oo = (int(x) for x in desc[t, 3:7])
+        np.testing.assert_array_equal(host[op:op + n // 2], ref["packed"])
+        np.testing.assert_array_equal(host[oq:oq + n // 64], ref["q8"])
+        np.testing.assert_array_equal(host[on:on + ref["nested"].nbytes].view(np.float32), ref["nested"])
+        assert host[oo:oo + 4].view(np.float32)[0] == ref["offset"]
+
+
+@pytest.mark.parametrize("M,N,K", [(256, 256, 64), (300, 576, 576), (1, 960, 576), (512, 4096, 4096),
+                                   (2048, 1536, 1024)])
+def test_dense_gemm_forward_and_transposed(M, N, K):
+    A = synth.tensor_values((M, K), seed=M + N, scale=1.0).to(DEV)
+    Bm = synth.tensor_values((N, K), seed=K, scale=0.05).to(DEV)
+    out = api.gemm_bf16(A, Bm)
+    ref = f64(A) @ f64(Bm).T
+    close(out, ref, tol=1e-2, what="A B^T")
+    Bt = synth.tensor_values((K, N), seed=K + 1, scale=0.05).to(DEV)
+    out2 = api.gemm_bf16(A, Bt, b_trans=True)
+    close(out2, f64(A) @ f64(Bt), tol=1e-2, what="A B")
+
+
+@pytest.mark.parametrize("M,rows,cols", [(512, 576, 576), (300, 192, 576), (2048, 4096, 4096), (64, 1536, 576)])
+def test_nf4_gemm_bit_exact_against_dense_on_dequantised(M, rows, cols):
+    w = synth.tensor_values((rows, cols), seed=rows + cols, scale=0.02).to(DEV)
+    q = api.nf4_quantize_tensor(w)
+    deq = api.nf4_dequantize_tensor(q).view(rows, cols)
+    # dequantised weights equal the oracle's
+    ref = quant.quantize(w.float().cpu().numpy().reshape(-1))
+    np.testing.assert_array_equal(deq.view(torch.int16).cpu().numpy().view(np.uint16).reshape(-1),
+                                  quant.dequantize_bits(ref))
+    A = synth.tensor_values((M, cols), seed=M, scale=1.0).to(DEV)
+    fused = api.gemm_nf4(A, q, rows, cols, dgrad=False)
+    dense = api.gemm_bf16(A, deq)
+    assert torch.equal(fused, dense)
+    close(fused, f64(A) @ f64(deq).T, tol=1e-2, what="NF4 forward")
+    G = synth.tensor_values((M, rows), seed=M + 7, scale=1.0).to(DEV)
+    fused_t = api.gemm_nf4(G, q, rows, cols, dgrad=True)
+    dense_t = api.gemm_bf16(G, deq, b_trans=True)
+    assert torch.equal(fused_t, dense_t)
+    close(fused_t, f64(G) @ f64(deq), tol=1e-2, what="NF4 dL/dx")
+    st, err = api.device_error()
+    assert st == 0, err
+
+
+@pytest.mark.parametrize("shape,batch,seq", [(synth.SMOLLM2_135M, 1, 512), (synth.LLAMA_8B, 2, 128)])
+def test_attention_forward_against_oracle(shape, batch, seq):
+    cfg = api.layer_cfg(shape, batch, seq)
+    M = batch * seq
+    qd, kvd = shape.q_dim, shape.kv_dim
+    qkv = synth.tensor_values((M, qd + 2 * kvd), seed=seq, scale=1.0).to(DEV)
+    o, lse = api.attention_fwd(cfg, qkv, qkv[:, qd:], qkv[:, qd + kvd:], qd + 2 * kvd, qd + 2 * kvd)
+    x = f64(qkv)
+    q = x[:, :qd].reshape(batch, seq, shape.n_q, shape.head_dim)
+    k = x[:, qd:qd + kvd].reshape(batch, seq, shape.n_kv, shape.head_dim)
+    v = x[:, qd + kvd:].reshape(batch, seq, shape.n_kv, shape.head_dim)
+    ref, P = olayer.attention(q, k, v)
+    close(o, ref.reshape(M, qd), what="attention out")

@@ -1,0 +1,200 @@
+"""Streaming checks (GPU): the pool's copy / reuse bookkeeping, the 30-layer
+SmolLM2-shaped training run streamed at depth 2 and 3 against the HBM-resident run
+(25 AdamW steps, loss curves and adapters bit-equal; first step against the oracle),
+the poisoned-pool run, and the 32B-class layers above the 165 MiB aliasing threshold
+whose LoRA gradients after buffer reuse must equal the resident gradients exactly.
+These are the gate-record checks of "Soup layer-streamed NF4 gate record" §2.2 (streamed
+= resident, n=2 = n=3, same-seed reruns, nonzero LoRA gradients in every layer) and the
+Issue #331 scenario of the layer-streaming review's bug history."""
+import numpy as np
+import pytest
+import torch
+
+from nf4_layer_streamed_b200 import api, synth
+from oracle import model as omodel
+from tests.helpers import LOSS_RTOL, close, f64, oracle_lora, oracle_weights
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def test_pool_copies_hits_and_slot_contents():
+    shape = synth.SMOLLM2_135M
+    cfg = api.layer_cfg(shape, 1, 512)
+    nb = api.shard_bytes(cfg)
+    slot = (nb + 255) // 256 * 256
+    store = torch.empty(3 * slot, dtype=torch.uint8).pin_memory()
+    for i in range(3):
+        w = synth.layer_weights(shape, i, 1234, device=DEV)
+        store[i * slot:i * slot + nb].copy_(api.nf4_quantize_shard(cfg, w).cpu())
+    pool = api.Pool(store, [0, slot, 2 * slot], [nb] * 3, depth=2)
+    try:
+        seen = {}
+        for i in range(3):                          # forward order
+            p = pool.stream_prefetch(i)
+            if i + 1 < 3:
+                pool.prefetch(i + 1)
+            seen[i] = pool.view(p, nb).clone()
+            pool.release(i)
+        for i in (2, 1, 0):                         # backward order
+            p = pool.stream_prefetch(i)
+            if i - 1 >= 0:
+                pool.prefetch(i - 1)
+            assert torch.equal(pool.view(p, nb).cpu(), store[i * slot:i * slot + nb])
+            pool.release(i)
+        torch.cuda.synchronize()
+        for i in range(3):
+            assert torch.equal(seen[i].cpu(), store[i * slot:i * slot + nb])
+        assert pool.wait(0, 1000) == 0
+        s = pool.stats()
+        assert s["copies"] == 4 and s["bytes_copied"] == 4 * nb
+        assert s["acquisitions"] == 6 and s["hits"] == 5
+    finally:
+        pool.destroy()
+
+
+def _train(wl, depth, resident, steps, poison=False, b_random=False):
+    m = api.StreamedModel(wl, depth=depth, resident=resident, b_random=b_random)
+    if poison and m.pool is not None:
+        m.pool.set_poison(True)
+    losses, first_grads = [], None
+    try:
+        for s in range(steps):
+            ids = synth.token_ids(wl.vocab, wl.batch, wl.seq, wl.seed, step=s, device=DEV)
+            m.forward_backward(ids)
+            if s == 0:
+                first_grads = m.grads.clone()
+            losses.append(m.loss.clone())
+            m.adamw_step()
+        torch.cuda.synchronize()
+        st, err = api.device_error()
+        assert st == 0, err
+        stats = m.pool.stats() if m.pool is not None else None
+        return torch.cat(losses), m.lora.clone(), first_grads, m, stats
+    finally:
+        m.close()
+
+
+def test_smollm2_30_layers_streamed_equals_resident_and_depths():
+    wl = synth.WORKLOADS["smollm2_30L_tied_b1s512"]
+    steps = wl.steps
+    l_res, p_res, g_res, m, _ = _train(wl, 2, True, steps)
+    l_2, p_2, g_2, _, st2 = _train(wl, 2, False, steps)
+    l_3, p_3, g_3, _, _ = _train(wl, 3, False, steps)
+    assert torch.equal(l_res, l_2) and torch.equal(l_2, l_3)
+    assert torch.equal(p_res, p_2) and torch.equal(p_2, p_3)
+    assert torch.equal(g_res, g_2) and torch.equal(g_2, g_3)
+    l_again, p_again, _, _, _ = _train(wl, 2, False, steps)
+    assert torch.equal(l_again, l_2) and torch.equal(p_again, p_2)
+    # every layer is read twice per step, minus the layers the backward finds resident
+    assert st2["copies"] <= 2 * wl.n_layers * steps
+    assert torch.all(torch.isfinite(l_2))
+    assert float(l_2[-1]) < float(l_2[0])
+
+
+def test_smollm2_30_layers_first_step_against_oracle():
+    wl = synth.WORKLOADS["smollm2_30L_tied_b1s512"]
+    shape = wl.shape
+    m = api.StreamedModel(wl, depth=2, resident=False)
+    try:
+        ids = synth.token_ids(wl.vocab, wl.batch, wl.seq, wl.seed, step=0, device=DEV)
+        m.forward_backward(ids)
+        torch.cuda.synchronize()
+        loss_gpu = float(m.loss.item())
+        grads = [m.grad_views(i) for i in range(wl.n_layers)]
+        # B = 0 at initialisation: dB is nonzero in every layer, dA is exactly zero
+        for g in grads:
+            assert torch.count_nonzero(g["dB_q"]) > 0 and torch.count_nonzero(g["dB_v"]) > 0
+            assert torch.count_nonzero(g["dA_q"]) == 0
+        layers = [oracle_weights(synth.layer_weights(shape, i, wl.seed, device="cpu")) for i in range(wl.n_layers)]
+        loras = [oracle_lora(synth.lora_params(shape, i, wl.seed)) for i in range(wl.n_layers)]
+        emb = f64(m.embed)
+        loss, og, _ = omodel.forward_backward(ids.cpu().numpy(), layers, loras, emb, None,
+                                              np.ones(shape.hidden), shape, wl.batch, wl.seq, rnd=True)
+        assert abs(loss_gpu - loss) <= LOSS_RTOL * abs(loss), (loss_gpu, loss)
+        for i in (0, wl.n_layers - 1):
+            close(grads[i]["dB_q"], og[i]["dB_q"], what=f"layer {i} dB_q")
+            close(grads[i]["dB_v"], og[i]["dB_v"], what=f"layer {i} dB_v")
+        # second step: B is now nonzero, so dA is nonzero in every layer
+        m.adamw_step()
+        ids2 = synth.token_ids(wl.vocab, wl.batch, wl.seq, wl.seed, step=1, device=DEV)
+        m.forward_backward(ids2)
+        torch.cuda.synchronize()
+        for i in range(wl.n_layers):
+            assert torch.count_nonzero(m.grad_views(i)["dA_q"]) > 0, i
+    finally:
+        m.close()
+
+
+def test_poisoned_pool_still_equals_resident():
+    wl = synth.Workload("smollm2_6L_tied", synth.SMOLLM2_135M, 6, 1, 512, vocab=49152, tied=True)
+    l_res, p_res, _, _, _ = _train(wl, 2, True, 3, b_random=True)
+    l_poi, p_poi, _, _, _ = _train(wl, 2, False, 3, poison=True, b_random=True)
+    assert torch.equal(l_res, l_poi) and torch.equal(p_res, p_poi)
+
+
+def _stack_grads(shape, n_layers, batch, seq, depth, resident, poison=False):
+    cfg = api.layer_cfg(shape, batch, seq)
+    nb = api.shard_bytes(cfg)
+    slot = (nb + 255) // 256 * 256
+    shards = []
+    if resident:
+        buf = torch.empty(n_layers * slot, dtype=torch.uint8, device=DEV)
+    else:
+        store = torch.empty(n_layers * slot, dtype=torch.uint8).pin_memory()
+    for i in range(n_layers):
+        w = synth.layer_weights(shape, i, 1234, device=DEV)
+        if resident:
+            api.nf4_quantize_shard(cfg, w, out=buf[i * slot:(i + 1) * slot])
+            shards.append(buf[i * slot:(i + 1) * slot])
+        else:
+            store[i * slot:i * slot + nb].copy_(api.nf4_quantize_shard(cfg, w).cpu())
+        del w
+    pool = None if resident else api.Pool(store, [i * slot for i in range(n_layers)], [nb] * n_layers, depth)
+    if pool is not None and poison:
+        pool.set_poison(True)
+
+    def get(i, nxt):
+        if resident:
+            return shards[i]
+        p = pool.stream_prefetch(i)
+        if 0 <= nxt < n_layers:
+            pool.prefetch(nxt)
+        return pool.view(p, nb)
+
+    try:
+        ws = api.LayerWorkspace(cfg)
+        loras = [synth.lora_params(shape, i, 1234, b_random=True, device=DEV) for i in range(n_layers)]
+        xs = [synth.hidden_states(shape, batch, seq, 1234, device=DEV).view(batch * seq, shape.hidden)]
+        for i in range(n_layers):
+            s = get(i, i + 1)
+            xs.append(api.layer_forward(cfg, s, loras[i], xs[-1], ws))
+            if pool:
+                pool.release(i)
+        _, dy = api.mse_loss(xs[-1])
+        grads = [None] * n_layers
+        for i in range(n_layers - 1, -1, -1):
+            s = get(i, i - 1)
+            dy, grads[i] = api.layer_backward(cfg, s, loras[i], xs[i], dy, ws)
+            if pool:
+                pool.release(i)
+        torch.cuda.synchronize()
+        return grads, dy
+    finally:
+        if pool is not None:
+            pool.destroy()
+
+
+def test_32b_class_layers_over_165mib_gradients_after_reuse_equal_resident():
+    wl = synth.WORKLOADS["qwen32b_4L_b1s1024"]
+    shape = wl.shape
+    assert api.shard_bytes(api.layer_cfg(shape, 1, 1024)) > 165 * 2 ** 20
+    g_res, dx_res = _stack_grads(shape, wl.n_layers, wl.batch, wl.seq, 2, True)
+    g_str, dx_str = _stack_grads(shape, wl.n_layers, wl.batch, wl.seq, 2, False, poison=True)
+    assert torch.equal(dx_res, dx_str)
+    for i in range(wl.n_layers):
+        for k in g_res[i]:
+            assert torch.equal(g_res[i][k], g_str[i][k]), (i, k)
+            assert torch.count_nonzero(g_res[i][k]) > 0
+    st, err = api.device_error()
+    assert st == 0, err
