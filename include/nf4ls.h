@@ -60,6 +60,17 @@ typedef void* nf4ls_stream; /* cudaStream_t */
 const char* nf4ls_last_error(void);
 int nf4ls_version(void);
 
+/* Number of kernels the library has launched in this process (all devices). */
+uint64_t nf4ls_launch_count(void);
+
+/* Per-launch timing of the GEMM kernels with CUDA events recorded on the launching
+ * stream (off by default).  nf4ls_profile_read(kind, out) waits for the recorded
+ * launches of that kind (0 dense bf16 GEMM, 1 NF4-decode GEMM), returns out[0] =
+ * launches, out[1] = total milliseconds, out[2] = total algorithmic FLOPs
+ * (2 M N K per launch), and forgets them. */
+int nf4ls_profile(int on);
+int nf4ls_profile_read(int kind, double out[3]);
+
 /* Reads and clears the device error flag of the current device: out[0] = code
  * (0 none, 1 barrier timeout), out[1] = kernel id, out[2] = block, out[3] = site.
  * Synchronises the device. */

@@ -54,6 +54,21 @@ def set_gemm_path(path: int) -> None:
     B.call("nf4ls_set_gemm_path", path)
 
 
+def launch_count() -> int:
+    return int(B.lib().nf4ls_launch_count())
+
+
+def profile(on: bool) -> None:
+    B.call("nf4ls_profile", int(on))
+
+
+def profile_read(kind: int) -> dict:
+    """kind 0: dense GEMM launches, 1: NF4-decode GEMM launches since the last read."""
+    out = (ctypes.c_double * 3)()
+    B.call("nf4ls_profile_read", kind, ctypes.cast(out, ctypes.c_void_p))
+    return {"launches": int(out[0]), "ms": float(out[1]), "flops": float(out[2])}
+
+
 def device_error():
     out = (ctypes.c_int32 * 4)()
     st = B.call_status("nf4ls_device_error", ctypes.cast(out, ctypes.c_void_p))

@@ -70,6 +70,9 @@ SIGNATURES = {
     "nf4ls_last_error": (ctypes.c_char_p, []),
     "nf4ls_version": (ctypes.c_int, []),
     "nf4ls_device_error": (ctypes.c_int, [P]),
+    "nf4ls_launch_count": (U64, []),
+    "nf4ls_profile": (ctypes.c_int, [ctypes.c_int]),
+    "nf4ls_profile_read": (ctypes.c_int, [ctypes.c_int, P]),
     "nf4ls_codebooks": (ctypes.c_int, [P, P, ctypes.POINTER(U64)]),
     "nf4ls_quantize_scratch_bytes": (SZ, [SZ]),
     "nf4_quantize_tensor": (ctypes.c_int, [P, SZ, P, P, P, P, P, SZ, P]),

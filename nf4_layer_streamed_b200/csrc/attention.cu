@@ -444,10 +444,12 @@ int attention_fwd(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfl
     const int sm = 3 * Tile<128>::BYTES;
     NF4_TRY(set_smem(k_attn_fwd<128>, sm));
     k_attn_fwd<128><<<grid, 128, sm, s>>>(q, k, v, ldq, ldkv, o, ldo, lse, seq, nq, nkv, scale_log2);
+    note_launch();
   } else {
     const int sm = 3 * Tile<64>::BYTES;
     NF4_TRY(set_smem(k_attn_fwd<64>, sm));
     k_attn_fwd<64><<<grid, 128, sm, s>>>(q, k, v, ldq, ldkv, o, ldo, lse, seq, nq, nkv, scale_log2);
+    note_launch();
   }
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;
@@ -461,19 +463,24 @@ int attention_bwd(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfl
   const int M = batch * seq;
   const float scale = 1.0f / sqrtf((float)d);
   k_attn_delta<<<(M * nq + 7) / 8, 256, 0, s>>>(o, dout, ldo, M, seq, nq, d, delta);
+  note_launch();
   dim3 gq(seq / TQ, nq, batch), gk(seq / TK, nkv, batch);
   if (d == 128) {
     const int sq = 4 * Tile<128>::BYTES, sk = 4 * Tile<128>::BYTES + 512;
     NF4_TRY(set_smem(k_attn_dq<128>, sq));
     NF4_TRY(set_smem(k_attn_dkv<128>, sk));
     k_attn_dq<128><<<gq, 128, sq, s>>>(q, k, v, ldq, ldkv, dout, ldo, lse, delta, dq, ld_dq, seq, nq, nkv, scale);
+    note_launch();
     k_attn_dkv<128><<<gk, 128, sk, s>>>(q, k, v, ldq, ldkv, dout, ldo, lse, delta, dk, dv, ld_dkv, seq, nq, nkv, scale);
+    note_launch();
   } else {
     const int sq = 4 * Tile<64>::BYTES, sk = 4 * Tile<64>::BYTES + 512;
     NF4_TRY(set_smem(k_attn_dq<64>, sq));
     NF4_TRY(set_smem(k_attn_dkv<64>, sk));
     k_attn_dq<64><<<gq, 128, sq, s>>>(q, k, v, ldq, ldkv, dout, ldo, lse, delta, dq, ld_dq, seq, nq, nkv, scale);
+    note_launch();
     k_attn_dkv<64><<<gk, 128, sk, s>>>(q, k, v, ldq, ldkv, dout, ldo, lse, delta, dk, dv, ld_dkv, seq, nq, nkv, scale);
+    note_launch();
   }
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;

@@ -390,6 +390,7 @@ int rmsnorm_fwd(const __nv_bfloat16* x, const __nv_bfloat16* w, __nv_bfloat16* y
                 cudaStream_t s) {
   if (H % 8) return fail(NF4LS_SHAPE, "rmsnorm: H %% 8");
   k_rmsnorm_fwd<<<(M + 7) / 8, 256, 0, s>>>(x, w, y, M, H, eps);
+  note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;
 }
@@ -397,12 +398,14 @@ int rmsnorm_fwd(const __nv_bfloat16* x, const __nv_bfloat16* w, __nv_bfloat16* y
 int rmsnorm_bwd(const __nv_bfloat16* x, const __nv_bfloat16* w, const __nv_bfloat16* dy, const __nv_bfloat16* resid,
                 __nv_bfloat16* dx, int M, int H, float eps, cudaStream_t s) {
   k_rmsnorm_bwd<<<(M + 7) / 8, 256, 0, s>>>(x, w, dy, resid, dx, M, H, eps);
+  note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;
 }
 
 int rope_tables(float* cos_t, float* sin_t, int seq, int d, float theta, cudaStream_t s) {
   k_rope_tables<<<blocks_for((size_t)seq * d / 2, 256), 256, 0, s>>>(cos_t, sin_t, seq, d, (double)theta);
+  note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;
 }
@@ -410,6 +413,7 @@ int rope_tables(float* cos_t, float* sin_t, int seq, int d, float theta, cudaStr
 int rope_bwd(__nv_bfloat16* x, int ld, int M, int cols, int seq, int d, const float* cos_t, const float* sin_t,
              cudaStream_t s) {
   k_rope_bwd<<<blocks_for((size_t)M * cols / 2, 256), 256, 0, s>>>(x, ld, M, cols, seq, d, cos_t, sin_t);
+  note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;
 }
@@ -418,6 +422,7 @@ int lora_skinny(const __nv_bfloat16* X, int ldx, int M, int K, const float* W, i
                 float* out_f, __nv_bfloat16* out_b, int ldb, int oc, cudaStream_t s) {
   if (K % 64) return fail(NF4LS_SHAPE, "lora: K %% 64");
   k_skinny<<<(M + 63) / 64, 256, 0, s>>>(X, ldx, M, K, W, sr, sk, scale, out_f, out_b, ldb, oc);
+  note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;
 }
@@ -425,6 +430,7 @@ int lora_skinny(const __nv_bfloat16* X, int ldx, int M, int K, const float* W, i
 int lora_grad_reduce(const __nv_bfloat16* X, int ldx, int M, int N, const float* y_f, const __nv_bfloat16* y_b, int ldy,
                      int yc, float scale, float* out, int so_n, int so_r, cudaStream_t s) {
   k_grad_reduce<<<(N + 63) / 64, 256, 0, s>>>(X, ldx, M, N, y_f, y_b, ldy, yc, scale, out, so_n, so_r);
+  note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;
 }
@@ -433,18 +439,21 @@ int lora_pack(const nf4ls_lora* l, int H, int qd, int kvd, float scale, __nv_bfl
               cudaStream_t s) {
   const size_t n = (size_t)(qd + 2 * kvd) * 64 + (size_t)64 * H;
   k_lora_pack<<<blocks_for(n, 256), 256, 0, s>>>(l->A_q, l->B_q, l->A_v, l->B_v, H, qd, kvd, scale, bup, adn);
+  note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;
 }
 
 int zero_cols(__nv_bfloat16* x, int ld, int M, int c0, int c1, cudaStream_t s) {
   k_zero_cols<<<blocks_for((size_t)M * (c1 - c0), 256), 256, 0, s>>>(x, ld, M, c0, c1);
+  note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;
 }
 
 int embed(const int32_t* ids, const __nv_bfloat16* E, __nv_bfloat16* h, int M, int H, cudaStream_t s) {
   k_embed<<<M, 128, 0, s>>>(ids, E, h, M, H);
+  note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;
 }
@@ -453,7 +462,9 @@ int cross_entropy(const __nv_bfloat16* logits, const int32_t* ids, int M, int V,
                   __nv_bfloat16* dlogits, float* loss, cudaStream_t s) {
   const int count = batch * (seq - 1);
   k_ce<<<M, 256, 0, s>>>(logits, ids, V, seq, 1.0f / (float)count, row_loss, dlogits);
+  note_launch();
   k_sum_scale<<<1, 256, 0, s>>>(row_loss, M, 1.0f / (float)count, loss);
+  note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;
 }
@@ -461,7 +472,9 @@ int cross_entropy(const __nv_bfloat16* logits, const int32_t* ids, int M, int V,
 int mse_loss(const __nv_bfloat16* out, size_t n, float* partial, int n_partial, __nv_bfloat16* dout, float* loss,
              cudaStream_t s) {
   k_mse<<<n_partial, 256, 0, s>>>(out, n, partial, dout);
+  note_launch();
   k_sum_scale<<<1, 256, 0, s>>>(partial, n_partial, 1.0f / (float)n, loss);
+  note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;
 }
@@ -471,6 +484,7 @@ int adamw(float* p, const float* g, float* m, float* v, size_t n, int step, floa
   const float bc1 = (float)(1.0 - std::pow((double)b1, step));
   const float bc2 = (float)(1.0 - std::pow((double)b2, step));
   k_adamw<<<blocks_for(n, 256), 256, 0, s>>>(p, g, m, v, n, lr, b1, b2, eps, wd, bc1, bc2);
+  note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;
 }

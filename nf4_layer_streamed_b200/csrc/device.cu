@@ -3,7 +3,9 @@
 // clears it through nf4ls_device_error().  The record is a file-scope __device__
 // array, so every device that loads the library holds its own copy; its address is
 // looked up once per device with cudaGetSymbolAddress.
+#include <atomic>
 #include <mutex>
+#include <vector>
 
 #include "internal.h"
 
@@ -25,7 +27,83 @@ int* device_error_ptr() {
   return ptrs[dev];
 }
 
+namespace {
+std::atomic<uint64_t> g_launches{0};
+std::atomic<int> g_profile{0};
+struct Rec {
+  int kind;
+  double flops;
+  cudaEvent_t e0, e1;
+};
+std::mutex g_prof_mu;
+std::vector<Rec> g_recs;
+std::vector<cudaEvent_t> g_free_events;
+
+cudaEvent_t take_event() {
+  if (!g_free_events.empty()) {
+    cudaEvent_t e = g_free_events.back();
+    g_free_events.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+}  // namespace
+
+void note_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+bool profiling() { return g_profile.load(std::memory_order_relaxed) != 0; }
+
+void profile_begin(cudaStream_t s, cudaEvent_t* e0) {
+  std::lock_guard<std::mutex> g(g_prof_mu);
+  *e0 = take_event();
+  if (*e0) cudaEventRecord(*e0, s);
+}
+
+void profile_end(cudaStream_t s, cudaEvent_t e0, int kind, double flops) {
+  std::lock_guard<std::mutex> g(g_prof_mu);
+  cudaEvent_t e1 = take_event();
+  if (!e0 || !e1) return;
+  cudaEventRecord(e1, s);
+  g_recs.push_back(Rec{kind, flops, e0, e1});
+}
+
 }  // namespace nf4ls
+
+extern "C" uint64_t nf4ls_launch_count(void) { return nf4ls::g_launches.load(); }
+
+extern "C" int nf4ls_profile(int on) {
+  nf4ls::g_profile.store(on ? 1 : 0);
+  return NF4LS_OK;
+}
+
+extern "C" int nf4ls_profile_read(int kind, double out[3]) {
+  nf4ls::clear_error();
+  if (!out) return nf4ls::fail(NF4LS_INVALID_ARG, "nf4ls_profile_read: null output");
+  std::lock_guard<std::mutex> g(nf4ls::g_prof_mu);
+  double n = 0, ms = 0, flops = 0;
+  std::vector<nf4ls::Rec> keep;
+  for (auto& r : nf4ls::g_recs) {
+    if (r.kind != kind) {
+      keep.push_back(r);
+      continue;
+    }
+    NF4_CUDA_TRY(cudaEventSynchronize(r.e1));
+    float t = 0.f;
+    NF4_CUDA_TRY(cudaEventElapsedTime(&t, r.e0, r.e1));
+    n += 1;
+    ms += t;
+    flops += r.flops;
+    nf4ls::g_free_events.push_back(r.e0);
+    nf4ls::g_free_events.push_back(r.e1);
+  }
+  nf4ls::g_recs.swap(keep);
+  out[0] = n;
+  out[1] = ms;
+  out[2] = flops;
+  return NF4LS_OK;
+}
 
 extern "C" int nf4ls_device_error(int32_t out[4]) {
   nf4ls::clear_error();

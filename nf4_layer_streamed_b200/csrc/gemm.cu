@@ -509,6 +509,7 @@ int launch(const GemmParams& p, int grid, cudaStream_t s) {
     configured[dev] = 1;
   }
   k_gemm<DECODE, BMN><<<grid, DECODE ? 448 : 192, SMEM_BYTES, s>>>(p);
+  note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;
 }
@@ -597,8 +598,16 @@ int gemm(const __nv_bfloat16* A, int lda, int M, int N, int K, const GemmWeights
   p.rope_cols = epi.rope_cols;
   p.err = device_error_ptr();
   const int grid = p.n_mt * n_nt;
-  if (decode) return dgrad ? launch<true, true>(p, grid, s) : launch<true, false>(p, grid, s);
-  return dgrad ? launch<false, true>(p, grid, s) : launch<false, false>(p, grid, s);
+  cudaEvent_t e0 = nullptr;
+  if (profiling()) profile_begin(s, &e0);
+  int st;
+  if (decode)
+    st = dgrad ? launch<true, true>(p, grid, s) : launch<true, false>(p, grid, s);
+  else
+    st = dgrad ? launch<false, true>(p, grid, s) : launch<false, false>(p, grid, s);
+  // algorithmic work: 2 M N K, plus the 64-wide LoRA block when present
+  if (e0) profile_end(s, e0, decode ? 1 : 0, 2.0 * M * (double)N * (K + (p.has_extra ? 64 : 0)));
+  return st;
 }
 
 }  // namespace nf4ls

@@ -181,9 +181,12 @@ int quantize_tensor(const void* w, size_t n, uint8_t* packed, uint8_t* q8, float
   const size_t chunks = (nb + 3) / 4;
   const size_t blocks = std::min<size_t>((chunks + 7) / 8, (size_t)sm_count() * 16);
   k_absmax_codes<<<(unsigned)blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(w), nb, packed, am, tab);
+  note_launch();
   k_offset_seq<<<1, 32, 0, s>>>(am, nb, offset);
+  note_launch();
   const size_t groups = (nb + 255) / 256;
   k_nested_q8<<<(unsigned)groups, 256, 0, s>>>(am, nb, offset, nested, q8, tab);
+  note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;
 }
@@ -200,6 +203,7 @@ int dequantize_tensor(const uint8_t* packed, const uint8_t* q8, const float* nes
   const size_t n8 = n / 8;
   const size_t blocks = std::min<size_t>((n8 + 255) / 256, (size_t)sm_count() * 8);
   k_dequant<<<(unsigned)blocks, 256, 0, s>>>(packed, q8, nested, offset, n8, static_cast<__nv_bfloat16*>(out), tab);
+  note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;
 }
