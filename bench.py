@@ -45,7 +45,7 @@ def peaks():
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama8b_32L_b4s512")
@@ -251,6 +251,19 @@ def main():
         raise RuntimeError(f"device error record: {err}")
     loss = float(m.loss.item())
 
+    # raw host-to-device link rate from pinned memory (one 1 GiB copy, best of 3)
+    probe_h = torch.empty(1 << 30, dtype=torch.uint8).pin_memory()
+    probe_d = torch.empty(1 << 30, dtype=torch.uint8, device="cuda")
+    best = 0.0
+    for _ in range(3):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        probe_d.copy_(probe_h, non_blocking=True)
+        b.record()
+        torch.cuda.synchronize()
+        best = max(best, (1 << 30) / (a.elapsed_time(b) / 1000.0) / 1e9)
+    del probe_h, probe_d
+
     pk, pk_kind = peaks()
     peak = float(pk.get("bf16_tflops_sustained", FALLBACK["bf16_tflops_sustained"]))
     achieved = nf4["flops"] / (nf4["ms"] / 1000.0) / 1e12 if nf4["ms"] > 0 else 0.0
@@ -311,6 +324,8 @@ def main():
                            "tflops": dense["flops"] / (dense["ms"] / 1000.0) / 1e12 if dense["ms"] > 0 else 0.0},
             "stream": {"h2d_bytes_per_step": copy_bytes,
                        "h2d_gbs_over_step": copy_bytes / (ms_max / 1000.0) / 1e9,
+                       "h2d_link_gbs": best,
+                       "copy_ms_per_step_at_link_rate": copy_bytes / best / 1e6 if best else None,
                        "copies_per_step": (st1["copies"] - st0["copies"]) / args.steps},
             "loss_last": loss,
             "gpu_launches": int(launches),

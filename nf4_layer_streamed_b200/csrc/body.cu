@@ -147,119 +147,6 @@ __global__ void k_rope_bwd(__nv_bfloat16* __restrict__ x, int ld, int M, int col
   p[j + half] = __float2bfloat16_rn(b * c - a * s);
 }
 
-// ------------------------------------------------------------------ LoRA
-// out[m, oc + r] = scale * sum_k X[m, k] * bf16(W(r, k)) for r < 16 (fixed k order),
-// W(r, k) = W[r * sr + k * sk] fp32.  Writes fp32 (out_f, ld 16) and/or bf16
-// (out_b at column offset oc, ld ldb).  64 rows per block, 256 threads, 8 outputs each.
-__global__ void __launch_bounds__(256) k_skinny(const __nv_bfloat16* __restrict__ X, int ldx, int M, int K,
-                                                const float* __restrict__ W, int sr, int sk, float scale,
-                                                float* __restrict__ out_f, __nv_bfloat16* __restrict__ out_b, int ldb,
-                                                int oc) {
-  __shared__ float xs[64][65];
-  __shared__ float ws[16][65];
-  const int t = threadIdx.x;
-  const int row = t >> 2, r0 = (t & 3) * 4;
-  const int m0 = blockIdx.x * 64;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int k0 = 0; k0 < K; k0 += 64) {
-    for (int i = t; i < 64 * 64; i += 256) {
-      const int rr = i >> 6, kk = i & 63;
-      const int m = m0 + rr;
-      xs[rr][kk] = (m < M) ? __bfloat162float(X[(size_t)m * ldx + k0 + kk]) : 0.f;
-    }
-    for (int i = t; i < 16 * 64; i += 256) {
-      const int rr = i >> 6, kk = i & 63;
-      ws[rr][kk] = __bfloat162float(__float2bfloat16_rn(W[(size_t)rr * sr + (size_t)(k0 + kk) * sk]));
-    }
-    __syncthreads();
-#pragma unroll 8
-    for (int kk = 0; kk < 64; ++kk) {
-      const float xv = xs[row][kk];
-#pragma unroll
-      for (int o = 0; o < 4; ++o) acc[o] += xv * ws[r0 + o][kk];
-    }
-    __syncthreads();
-  }
-  const int m = m0 + row;
-  if (m >= M) return;
-#pragma unroll
-  for (int o = 0; o < 4; ++o) {
-    const float v = acc[o] * scale;
-    if (out_f) out_f[(size_t)m * 16 + r0 + o] = v;
-    if (out_b) out_b[(size_t)m * ldb + oc + r0 + o] = __float2bfloat16_rn(v);
-  }
-}
-
-// out(n, r) = scale * sum_m X[m, n] * Y[m, r] (fixed m order); X bf16 [M, ldx],
-// Y fp32 (y_f) or bf16 (y_b) [M, ldy] from column yc; out(n, r) at out[n * so_n + r * so_r].
-// Block: 64 columns n, 256 threads, 4 outputs each.
-__global__ void __launch_bounds__(256) k_grad_reduce(const __nv_bfloat16* __restrict__ X, int ldx, int M, int N,
-                                                     const float* __restrict__ y_f, const __nv_bfloat16* __restrict__ y_b,
-                                                     int ldy, int yc, float scale, float* __restrict__ out, int so_n,
-                                                     int so_r) {
-  __shared__ float xs[64][65];
-  __shared__ float ys[64][17];
-  const int t = threadIdx.x;
-  const int n_l = t >> 2, r0 = (t & 3) * 4;
-  const int n0 = blockIdx.x * 64;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int mb = 0; mb < M; mb += 64) {
-    for (int i = t; i < 64 * 64; i += 256) {
-      const int mm = i >> 6, nn = i & 63;
-      const int m = mb + mm, n = n0 + nn;
-      xs[mm][nn] = (m < M && n < N) ? __bfloat162float(X[(size_t)m * ldx + n]) : 0.f;
-    }
-    for (int i = t; i < 64 * 16; i += 256) {
-      const int mm = i >> 4, rr = i & 15;
-      const int m = mb + mm;
-      float v = 0.f;
-      if (m < M) v = y_f ? y_f[(size_t)m * ldy + yc + rr] : __bfloat162float(y_b[(size_t)m * ldy + yc + rr]);
-      ys[mm][rr] = v;
-    }
-    __syncthreads();
-#pragma unroll 8
-    for (int mm = 0; mm < 64; ++mm) {
-      const float xv = xs[mm][n_l];
-#pragma unroll
-      for (int o = 0; o < 4; ++o) acc[o] += xv * ys[mm][r0 + o];
-    }
-    __syncthreads();
-  }
-  const int n = n0 + n_l;
-  if (n >= N) return;
-#pragma unroll
-  for (int o = 0; o < 4; ++o) out[(size_t)n * so_n + (size_t)(r0 + o) * so_r] = acc[o] * scale;
-}
-
-// Padded bf16 adapter operands of the GEMM extra block:
-//   bup [Nqkv, 64]: row n of q -> scale*B_q[n, :] in cols 0-15; row of v -> scale*B_v in 16-31; k rows 0.
-//   adn [64, H]   : rows 0-15 = A_q, rows 16-31 = A_v, other rows 0.
-__global__ void k_lora_pack(const float* __restrict__ Aq, const float* __restrict__ Bq, const float* __restrict__ Av,
-                            const float* __restrict__ Bv, int H, int qd, int kvd, float scale,
-                            __nv_bfloat16* __restrict__ bup, __nv_bfloat16* __restrict__ adn) {
-  const int nq = qd + 2 * kvd;
-  const size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
-  const size_t n_bup = (size_t)nq * 64, n_adn = (size_t)64 * H;
-  if (i < n_bup) {
-    const int n = (int)(i / 64), c = (int)(i % 64);
-    float v = 0.f;
-    if (n < qd && c < 16)
-      v = scale * __bfloat162float(__float2bfloat16_rn(Bq[(size_t)n * 16 + c]));
-    else if (n >= qd + kvd && c >= 16 && c < 32)
-      v = scale * __bfloat162float(__float2bfloat16_rn(Bv[(size_t)(n - qd - kvd) * 16 + c - 16]));
-    bup[i] = __float2bfloat16_rn(v);
-  } else if (i < n_bup + n_adn) {
-    const size_t j = i - n_bup;
-    const int r = (int)(j / H), k = (int)(j % H);
-    float v = 0.f;
-    if (r < 16)
-      v = Aq[(size_t)r * H + k];
-    else if (r < 32)
-      v = Av[(size_t)(r - 16) * H + k];
-    adn[j] = __float2bfloat16_rn(v);
-  }
-}
-
 __global__ void k_zero_cols(__nv_bfloat16* __restrict__ x, int ld, int M, int c0, int c1) {
   const int w = c1 - c0;
   const size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
@@ -413,32 +300,6 @@ int rope_tables(float* cos_t, float* sin_t, int seq, int d, float theta, cudaStr
 int rope_bwd(__nv_bfloat16* x, int ld, int M, int cols, int seq, int d, const float* cos_t, const float* sin_t,
              cudaStream_t s) {
   k_rope_bwd<<<blocks_for((size_t)M * cols / 2, 256), 256, 0, s>>>(x, ld, M, cols, seq, d, cos_t, sin_t);
-  note_launch();
-  NF4_CUDA_TRY(cudaGetLastError());
-  return NF4LS_OK;
-}
-
-int lora_skinny(const __nv_bfloat16* X, int ldx, int M, int K, const float* W, int sr, int sk, float scale,
-                float* out_f, __nv_bfloat16* out_b, int ldb, int oc, cudaStream_t s) {
-  if (K % 64) return fail(NF4LS_SHAPE, "lora: K %% 64");
-  k_skinny<<<(M + 63) / 64, 256, 0, s>>>(X, ldx, M, K, W, sr, sk, scale, out_f, out_b, ldb, oc);
-  note_launch();
-  NF4_CUDA_TRY(cudaGetLastError());
-  return NF4LS_OK;
-}
-
-int lora_grad_reduce(const __nv_bfloat16* X, int ldx, int M, int N, const float* y_f, const __nv_bfloat16* y_b, int ldy,
-                     int yc, float scale, float* out, int so_n, int so_r, cudaStream_t s) {
-  k_grad_reduce<<<(N + 63) / 64, 256, 0, s>>>(X, ldx, M, N, y_f, y_b, ldy, yc, scale, out, so_n, so_r);
-  note_launch();
-  NF4_CUDA_TRY(cudaGetLastError());
-  return NF4LS_OK;
-}
-
-int lora_pack(const nf4ls_lora* l, int H, int qd, int kvd, float scale, __nv_bfloat16* bup, __nv_bfloat16* adn,
-              cudaStream_t s) {
-  const size_t n = (size_t)(qd + 2 * kvd) * 64 + (size_t)64 * H;
-  k_lora_pack<<<blocks_for(n, 256), 256, 0, s>>>(l->A_q, l->B_q, l->A_v, l->B_v, H, qd, kvd, scale, bup, adn);
   note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;

@@ -146,12 +146,14 @@ int attention_bwd(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfl
                   __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv, int ld_dq, int ld_dkv, int batch,
                   int seq, int nq, int nkv, int d, cudaStream_t s);
 
-int lora_skinny(const __nv_bfloat16* X, int ldx, int M, int K, const float* W, int sr, int sk, float scale,
-                float* out_f, __nv_bfloat16* out_b, int ldb, int oc, cudaStream_t s);
-int lora_grad_reduce(const __nv_bfloat16* X, int ldx, int M, int N, const float* y_f, const __nv_bfloat16* y_b, int ldy,
-                     int yc, float scale, float* out, int so_n, int so_r, cudaStream_t s);
-int lora_pack(const nf4ls_lora* l, int H, int qd, int kvd, float scale, __nv_bfloat16* bup, __nv_bfloat16* adn,
-              cudaStream_t s);
+size_t lora_partial_bytes(int M, int Nmax);
+int lora_pack2(const nf4ls_lora* l, int H, int qd, int kvd, float scale, __nv_bfloat16* bup, __nv_bfloat16* adn,
+               __nv_bfloat16* bqt, __nv_bfloat16* bvt, cudaStream_t s);
+int lora_rows(const __nv_bfloat16* X, int ldx, int M, int nseg, const int* xcol, const int* K,
+              const __nv_bfloat16* const* W, const int* ldw, float scale, float* part, __nv_bfloat16* out_b, int ldb,
+              int oc, cudaStream_t s);
+int lora_cols(const __nv_bfloat16* X, int ldx, int xcol, int N, int M, const __nv_bfloat16* Y, int ldy, int ycol,
+              int NR, float scale, float* part, float* out0, float* out1, int so_n, int so_r, cudaStream_t s);
 int zero_cols(__nv_bfloat16* x, int ld, int M, int c0, int c1, cudaStream_t s);
 int embed(const int32_t* ids, const __nv_bfloat16* E, __nv_bfloat16* h, int M, int H, cudaStream_t s);
 int cross_entropy(const __nv_bfloat16* logits, const int32_t* ids, int M, int V, int batch, int seq, float* row_loss,

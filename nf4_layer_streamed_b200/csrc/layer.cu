@@ -23,6 +23,8 @@
 //   do  = dh Wo;  dq, dk, dv = attention_bwd;  RoPE^T on dq, dk
 //   dB = s dq^T t, dt = s dq B, dA = dt^T h1                  (q and v adapters)
 //   dx  = dh + rmsnorm_bwd(x, [dq|dk|dv] [Wq;Wk;Wv] + dt [A_q; A_v])
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -31,8 +33,8 @@ namespace nf4ls {
 namespace {
 
 struct WsLayout {
-  size_t cos, sin, h1, qkv, tpad, bup, adn, o, lse, h, h2, gu, act, dgu, dh2, dh, dO, dqkv, delta, dt, dtpad, dh1, dense,
-      total;
+  size_t cos, sin, h1, qkv, tpad, bup, adn, o, lse, h, h2, gu, act, dgu, dh2, dh, dO, dqkv, delta, bqt, bvt, part,
+      dtpad, dh1, dense, total;
 };
 
 WsLayout ws_layout(const nf4ls_layer_cfg* c) {
@@ -64,7 +66,9 @@ WsLayout ws_layout(const nf4ls_layer_cfg* c) {
   L.dO = take(M * qd * 2);
   L.dqkv = take(M * nqkv * 2);
   L.delta = take((size_t)c->batch * c->n_q * c->seq * 4);
-  L.dt = take(M * 32 * 4);
+  L.bqt = take(16 * qd * 2);
+  L.bvt = take(16 * kvd * 2);
+  L.part = take(lora_partial_bytes((int)M, (int)std::max(H, qd)));
   L.dtpad = take(M * 64 * 2);
   L.dh1 = take(M * H * 2);
   // bf16 copy of the layer's seven linears for the dequantise-then-multiply path
@@ -158,10 +162,13 @@ int forward_body(LayerCtx& x, const nf4ls_lora* lora, const __nv_bfloat16* X, __
   if (lora) {
     auto* bup = at<__nv_bfloat16>(ws, x.L.bup);
     auto* adn = at<__nv_bfloat16>(ws, x.L.adn);
-    NF4_TRY(lora_pack(lora, H, x.qd, x.kvd, x.scale, bup, adn, s));
+    NF4_TRY(lora_pack2(lora, H, x.qd, x.kvd, x.scale, bup, adn, at<__nv_bfloat16>(ws, x.L.bqt),
+                       at<__nv_bfloat16>(ws, x.L.bvt), s));
     NF4_TRY(zero_cols(tpad, 64, M, 32, 64, s));
-    NF4_TRY(lora_skinny(h1, H, M, H, lora->A_q, H, 1, 1.0f, nullptr, tpad, 64, 0, s));
-    NF4_TRY(lora_skinny(h1, H, M, H, lora->A_v, H, 1, 1.0f, nullptr, tpad, 64, 16, s));
+    // t = [h1 A_q^T | h1 A_v^T] into columns 0-31 of the padded extra operand
+    const int xcol[2] = {0, 0}, K[2] = {H, H}, ldw[2] = {H, H};
+    const __nv_bfloat16* Wd[2] = {adn, adn + (size_t)16 * H};
+    NF4_TRY(lora_rows(h1, H, M, 2, xcol, K, Wd, ldw, 1.0f, at<float>(ws, x.L.part), tpad, 64, 0, s));
     ex.a = tpad;
     ex.b = bup;
   }
@@ -269,18 +276,18 @@ int layer_bwd_impl(const nf4ls_layer_cfg* c, const void* shard, const nf4ls_lora
   if (lora) {
     auto* tpad = at<__nv_bfloat16>(ws, x.L.tpad);
     auto* dtpad = at<__nv_bfloat16>(ws, x.L.dtpad);
-    float* dt = at<float>(ws, x.L.dt);
-    float* dt_q = dt;
-    float* dt_v = dt + (size_t)M * 16;
-    __nv_bfloat16* dq = dqkv;
-    __nv_bfloat16* dv = dqkv + x.qd + x.kvd;
-    NF4_TRY(lora_grad_reduce(dq, x.nqkv, M, x.qd, nullptr, tpad, 64, 0, x.scale, g->dB_q, 16, 1, s));
-    NF4_TRY(lora_grad_reduce(dv, x.nqkv, M, x.kvd, nullptr, tpad, 64, 16, x.scale, g->dB_v, 16, 1, s));
+    float* part = at<float>(ws, x.L.part);
+    const int vcol = x.qd + x.kvd;
+    // dB = s dq^T t_q, s dv^T t_v
+    NF4_TRY(lora_cols(dqkv, x.nqkv, 0, x.qd, M, tpad, 64, 0, 16, x.scale, part, g->dB_q, nullptr, 16, 1, s));
+    NF4_TRY(lora_cols(dqkv, x.nqkv, vcol, x.kvd, M, tpad, 64, 16, 16, x.scale, part, g->dB_v, nullptr, 16, 1, s));
+    // dt = s [dq B_q | dv B_v] (bf16, the extra operand of the dL/dx GEMM)
     NF4_TRY(zero_cols(dtpad, 64, M, 32, 64, s));
-    NF4_TRY(lora_skinny(dq, x.nqkv, M, x.qd, lora->B_q, 1, 16, x.scale, dt_q, dtpad, 64, 0, s));
-    NF4_TRY(lora_skinny(dv, x.nqkv, M, x.kvd, lora->B_v, 1, 16, x.scale, dt_v, dtpad, 64, 16, s));
-    NF4_TRY(lora_grad_reduce(h1, H, M, H, dt_q, nullptr, 16, 0, 1.0f, g->dA_q, 1, H, s));
-    NF4_TRY(lora_grad_reduce(h1, H, M, H, dt_v, nullptr, 16, 0, 1.0f, g->dA_v, 1, H, s));
+    const int xcol[2] = {0, vcol}, K[2] = {x.qd, x.kvd}, ldw[2] = {x.qd, x.kvd};
+    const __nv_bfloat16* Wt[2] = {at<__nv_bfloat16>(ws, x.L.bqt), at<__nv_bfloat16>(ws, x.L.bvt)};
+    NF4_TRY(lora_rows(dqkv, x.nqkv, M, 2, xcol, K, Wt, ldw, x.scale, part, dtpad, 64, 0, s));
+    // dA = dt^T h1 for q (dt columns 0-15) and v (16-31)
+    NF4_TRY(lora_cols(h1, H, 0, H, M, dtpad, 64, 0, 32, 1.0f, part, g->dA_q, g->dA_v, 1, H, s));
     ex.a = dtpad;
     ex.b = at<__nv_bfloat16>(ws, x.L.adn);
   }

@@ -1,0 +1,85 @@
+"""Shape-matched GEMM throughput of the tcgen05 kernels (NF4 decode in the mainloop,
+and the dense bf16 kernel on the same dequantised weights).
+
+The shapes are the Llama-3.1-8B projections the gate record's §4.4 table measures
+("Soup layer-streamed NF4 gate record": q/o 4096x4096, k/v 1024x4096, gate/up
+14336x4096, down 4096x14336), at M = batch x 512 tokens, both for the forward
+product out = x W^T and the dL/dx product out = dy W.
+
+    python -m nf4_layer_streamed_b200.gemm_bench [--M 2048] [--shapes gateup,down] [--iters 20]
+    python -m nf4_layer_streamed_b200.gemm_bench --once --shapes gateup   (one launch each: for ncu)
+
+Prints one JSON object per (shape, direction, kernel) with the mean launch time
+(CUDA events on the launching stream, after warm-up) and TFLOP/s = 2 M N K / time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+
+import torch
+
+from . import api, synth
+
+SHAPES = {  # name: (rows = out features, cols = in features) of W
+    "qo": (4096, 4096),
+    "kv": (1024, 4096),
+    "gateup": (28672, 4096),   # gate and up stacked, as the fused GEMM runs them
+    "down": (4096, 14336),
+}
+
+
+def run(M: int, names, iters: int, once: bool):
+    out = []
+    for name in names:
+        rows, cols = SHAPES[name]
+        w = synth.tensor_values((rows, cols), seed=rows + cols, scale=0.02, device="cuda")
+        q = api.nf4_quantize_tensor(w)
+        deq = api.nf4_dequantize_tensor(q).view(rows, cols)
+        del w
+        for dgrad in (False, True):
+            K = rows if dgrad else cols
+            N = cols if dgrad else rows
+            A = synth.tensor_values((M, K), seed=M + K, scale=1.0, device="cuda")
+            for kind in ("nf4", "dense"):
+                def f():
+                    if kind == "nf4":
+                        return api.gemm_nf4(A, q, rows, cols, dgrad=dgrad)
+                    return api.gemm_bf16(A, deq, b_trans=dgrad)
+                if once:
+                    f()
+                    torch.cuda.synchronize()
+                    continue
+                for _ in range(3):
+                    f()
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                for _ in range(iters):
+                    f()
+                e1.record()
+                torch.cuda.synchronize()
+                ms = e0.elapsed_time(e1) / iters
+                tf = 2.0 * M * N * K / (ms / 1000.0) / 1e12
+                rec = {"shape": name, "M": M, "N": N, "K": K, "product": "dL/dx" if dgrad else "forward",
+                       "kernel": kind, "ms": ms, "tflops": tf}
+                out.append(rec)
+                print(json.dumps(rec), flush=True)
+    return out
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--M", type=int, default=2048)
+    ap.add_argument("--shapes", default="qo,kv,gateup,down")
+    ap.add_argument("--iters", type=int, default=20)
+    ap.add_argument("--once", action="store_true")
+    a = ap.parse_args(argv)
+    run(a.M, a.shapes.split(","), a.iters, a.once)
+    st, err = api.device_error()
+    if st != 0:
+        raise RuntimeError(f"device error record {err}")
+
+
+if __name__ == "__main__":
+    main()

@@ -88,8 +88,9 @@ def test_smollm2_30_layers_streamed_equals_resident_and_depths():
     assert torch.equal(l_again, l_2) and torch.equal(p_again, p_2)
     # every layer is read twice per step, minus the layers the backward finds resident
     assert st2["copies"] <= 2 * wl.n_layers * steps
+    # uniform random targets: the loss stays near ln V (nothing to learn), finite throughout
     assert torch.all(torch.isfinite(l_2))
-    assert float(l_2[-1]) < float(l_2[0])
+    assert torch.all(torch.abs(l_2 - np.log(wl.vocab)) < 1.0)
 
 
 def test_smollm2_30_layers_first_step_against_oracle():
@@ -106,7 +107,8 @@ def test_smollm2_30_layers_first_step_against_oracle():
         for g in grads:
             assert torch.count_nonzero(g["dB_q"]) > 0 and torch.count_nonzero(g["dB_v"]) > 0
             assert torch.count_nonzero(g["dA_q"]) == 0
-        layers = [oracle_weights(synth.layer_weights(shape, i, wl.seed, device="cpu")) for i in range(wl.n_layers)]
+        # the model drew its weights on the GPU: regenerate them there, then hand them to the oracle
+        layers = [oracle_weights(synth.layer_weights(shape, i, wl.seed, device=DEV)) for i in range(wl.n_layers)]
         loras = [oracle_lora(synth.lora_params(shape, i, wl.seed)) for i in range(wl.n_layers)]
         emb = f64(m.embed)
         loss, og, _ = omodel.forward_backward(ids.cpu().numpy(), layers, loras, emb, None,
