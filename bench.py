@@ -216,6 +216,7 @@ def main():
         else:
             m.train_step(ids[i])
 
+    api.profile(True)  # warm the profiler's event pool during the warm-up steps
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()

@@ -260,7 +260,9 @@ int lora_rows(const __nv_bfloat16* X, int ldx, int M, int nseg, const int* xcol,
     kmin = std::min(kmin, K[j] / 64);
   }
   const int mb = (M + 63) / 64;
-  const int S = splits_for(kmin, mb * nseg);
+  // The split of K depends on K only, so a row's sum is grouped the same way for any
+  // M: a token's result does not depend on how many tokens share the launch.
+  const int S = std::min(8, kmin);
   k_lora_rows<<<dim3(mb, S, nseg), 128, 0, s>>>(X, ldx, M, sg, nseg, S, part);
   note_launch();
   const int n = M * 16 * nseg;
