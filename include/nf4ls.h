@@ -141,6 +141,23 @@ int nf4_quantize_tensor(const void* w_dev, size_t n, uint8_t* packed_dev, uint8_
 int nf4_dequantize_tensor(const uint8_t* packed_dev, const uint8_t* q8_dev, const float* nested_dev,
                           const float* offset_dev, size_t n, void* out_dev, nf4ls_stream stream);
 
+/* nf4_quantize_tensor without a scratch argument, for callers that cannot allocate
+ * device memory (code inside another framework's memory pool, host callbacks that
+ * must not allocate, processes whose device memory belongs to a pool they do not
+ * control).  The pages have no counterpart: their quantiser runs through PyTorch and
+ * may allocate freely.
+ * The scratch lives in a fixed file-scope device array for tensors of up to
+ * nf4ls_quantize_noalloc_max_elems() weights (2^28, 16 MiB of device memory held by
+ * every GPU that loads the library until the process exits).  Larger n returns
+ * NF4LS_INVALID_ARG.  The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress); make it before any stream capture.  All calls share the
+ * array, so calls that overlap on the GPU race; serialise them on one stream.  No
+ * part of the array needs to start at zero.  Allocates nothing; results are the same
+ * bytes nf4_quantize_tensor produces. */
+size_t nf4ls_quantize_noalloc_max_elems(void);
+int nf4_quantize_tensor_noalloc(const void* w_dev, size_t n, uint8_t* packed_dev, uint8_t* q8_dev,
+                                float* nested_dev, float* offset_dev, nf4ls_stream stream);
+
 /* ------------------------------------------------------------------ layer shards
  * A shard is one decoder layer as one contiguous byte range, the unit that streams
  * ([gate] §2.1: offline per-layer shards; [review]: the cache key carries the

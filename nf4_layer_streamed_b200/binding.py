@@ -77,6 +77,8 @@ SIGNATURES = {
     "nf4ls_quantize_scratch_bytes": (SZ, [SZ]),
     "nf4_quantize_tensor": (ctypes.c_int, [P, SZ, P, P, P, P, P, SZ, P]),
     "nf4_dequantize_tensor": (ctypes.c_int, [P, P, P, P, SZ, P, P]),
+    "nf4ls_quantize_noalloc_max_elems": (SZ, []),
+    "nf4_quantize_tensor_noalloc": (ctypes.c_int, [P, SZ, P, P, P, P, P]),
     "nf4ls_shard_bytes": (SZ, [ctypes.POINTER(LayerCfg)]),
     "nf4ls_shard_quantized_bytes": (SZ, [ctypes.POINTER(LayerCfg)]),
     "nf4ls_shard_scratch_bytes": (SZ, [ctypes.POINTER(LayerCfg)]),
