@@ -257,6 +257,11 @@ int layer_backward(const nf4ls_layer_cfg* cfg, const void* shard_dev, const nf4l
  * Both give bit-identical results (same decoded values, same MMA order). */
 int nf4ls_set_gemm_path(int path);
 
+/* CTA-pair GEMMs (process-wide; default 1): products with more than 256 tokens run
+ * on clusters of two CTAs sharing one 2-SM tcgen05 MMA (512 tokens x 256 features per
+ * pair); 0 keeps one CTA per 256 x 256 tile.  For testing and comparison. */
+int nf4ls_set_gemm_pair(int on);
+
 /* ------------------------------------------------------------------ streaming pool
  * [review] mechanism section: the frozen base lives in pinned host memory; 2-8
  * preallocated HBM buffers (double by default) are filled on a dedicated CUDA

@@ -54,6 +54,10 @@ def set_gemm_path(path: int) -> None:
     B.call("nf4ls_set_gemm_path", path)
 
 
+def set_gemm_pair(on: bool) -> None:
+    B.call("nf4ls_set_gemm_pair", int(on))
+
+
 def launch_count() -> int:
     return int(B.lib().nf4ls_launch_count())
 

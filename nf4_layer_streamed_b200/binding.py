@@ -89,6 +89,7 @@ SIGNATURES = {
     "layer_backward": (ctypes.c_int, [ctypes.POINTER(LayerCfg), P, ctypes.POINTER(Lora), P, P, P,
                                       ctypes.POINTER(LoraGrads), P, SZ, P]),
     "nf4ls_set_gemm_path": (ctypes.c_int, [ctypes.c_int]),
+    "nf4ls_set_gemm_pair": (ctypes.c_int, [ctypes.c_int]),
     "nf4ls_pool_create": (ctypes.c_int, [P, P, P, ctypes.c_int, ctypes.c_int, P, SZ, ctypes.POINTER(P)]),
     "nf4ls_pool_prefetch": (ctypes.c_int, [P, ctypes.c_int]),
     "stream_prefetch": (ctypes.c_int, [P, ctypes.c_int, P, ctypes.POINTER(P)]),

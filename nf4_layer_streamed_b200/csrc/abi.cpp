@@ -19,6 +19,7 @@ namespace nf4ls {
 namespace {
 thread_local char g_msg[1024] = "";
 int g_gemm_path = 0;
+int g_gemm_pair = 1;
 }  // namespace
 
 int fail(int status, const char* fmt, ...) {
@@ -32,6 +33,7 @@ int fail(int status, const char* fmt, ...) {
 void clear_error() { g_msg[0] = 0; }
 
 int gemm_path() { return g_gemm_path; }
+int gemm_pair() { return g_gemm_pair; }
 
 void shard_layout(const nf4ls_layer_cfg* c, ShardLayout* L) {
   const int qd = c->n_q * c->head_dim, kvd = c->n_kv * c->head_dim;
@@ -101,6 +103,11 @@ extern "C" int nf4ls_version(void) { return 1; }
 extern "C" int nf4ls_set_gemm_path(int path) {
   if (path != 0 && path != 1) return fail(NF4LS_INVALID_ARG, "gemm path must be 0 or 1");
   g_gemm_path = path;
+  return NF4LS_OK;
+}
+
+extern "C" int nf4ls_set_gemm_pair(int on) {
+  g_gemm_pair = on ? 1 : 0;
   return NF4LS_OK;
 }
 

@@ -153,6 +153,95 @@ __device__ __forceinline__ void ld_acc(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// ------------------------------------------------------------------------------ epilogue
+// One epilogue warp (TMEM lane quarter q) turns the two 128 x 256 fp32 accumulators of
+// its CTA (tokens m0 + [0, 256), output features of tile nt) into bf16 results.
+__device__ __forceinline__ void epilogue_rows(const GemmParams& p, uint32_t tmem, int m0, int nt, int q, int lane) {
+  for (int a = 0; a < 2; ++a) {
+    const int m = m0 + a * 128 + q * 32 + lane;
+    const bool mv = m < p.M;
+    const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + a * 256;
+    float v[32], w[32];
+    if (p.epi == EPI_SWIGLU) {
+      for (int c = 0; c < 4; ++c) {
+        ld_acc(tb + c * 32, v);
+        ld_acc(tb + 128 + c * 32, w);
+        if (!mv) continue;
+        const int col = nt * 128 + c * 32;
+        float o[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          v[i] = round_bf16(v[i]);
+          w[i] = round_bf16(w[i]);
+          o[i] = silu_f(v[i]) * w[i];
+        }
+        store32(p.out + (size_t)m * p.ldo + col, o);
+        if (p.aux_out) {
+          store32(p.aux_out + (size_t)m * p.ld_aux_out + col, v);
+          store32(p.aux_out + (size_t)m * p.ld_aux_out + p.inter + col, w);
+        }
+      }
+    } else if (p.epi == EPI_ROPE) {
+      const int d = p.head_dim, half = d / 2;
+      const int pos = m % p.seq;
+      for (int h = 0; h < BN / d; ++h) {
+        const int hc = nt * BN + h * d;
+        if (hc >= p.N) break;
+        if (hc < p.rope_cols) {
+          for (int i = 0; i < half / 32; ++i) {
+            ld_acc(tb + h * d + i * 32, v);
+            ld_acc(tb + h * d + half + i * 32, w);
+            if (!mv) continue;
+            const float* cs = p.rope_cos + (size_t)pos * half + i * 32;
+            const float* sn = p.rope_sin + (size_t)pos * half + i * 32;
+            float o1[32], o2[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float c_ = cs[j], s_ = sn[j];
+              o1[j] = v[j] * c_ - w[j] * s_;
+              o2[j] = w[j] * c_ + v[j] * s_;
+            }
+            store32(p.out + (size_t)m * p.ldo + hc + i * 32, o1);
+            store32(p.out + (size_t)m * p.ldo + hc + half + i * 32, o2);
+          }
+        } else {
+          for (int c = 0; c < d / 32; ++c) {
+            ld_acc(tb + h * d + c * 32, v);
+            if (mv) store32(p.out + (size_t)m * p.ldo + hc + c * 32, v);
+          }
+        }
+      }
+    } else {
+      for (int c = 0; c < BN / 32; ++c) {
+        const int col = nt * BN + c * 32;
+        if (col >= p.N) break;
+        ld_acc(tb + c * 32, v);
+        if (!mv) continue;
+        if (p.epi == EPI_RESID) {
+          load32_bf16(p.aux0 + (size_t)m * p.ld_aux0 + col, w);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] += w[i];
+          store32(p.out + (size_t)m * p.ldo + col, v);
+        } else if (p.epi == EPI_DSWIGLU) {
+          float g[32], u[32], dg[32], du[32];
+          load32_bf16(p.aux0 + (size_t)m * p.ld_aux0 + col, g);
+          load32_bf16(p.aux0 + (size_t)m * p.ld_aux0 + p.inter + col, u);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float sg = 1.0f / (1.0f + expf(-g[i]));
+            dg[i] = v[i] * u[i] * sg * (1.0f + g[i] * (1.0f - sg));
+            du[i] = v[i] * g[i] * sg;
+          }
+          store32(p.out + (size_t)m * p.ldo + col, dg);
+          store32(p.out + (size_t)m * p.ldo + p.inter + col, du);
+        } else {
+          store32(p.out + (size_t)m * p.ldo + col, v);
+        }
+      }
+    }
+  }
+}
+
 // ------------------------------------------------------------------------------ kernel
 template <bool DECODE, bool BMN>
 __global__ void __launch_bounds__(DECODE ? 448 : 192, 1) k_gemm(const __grid_constant__ GemmParams p) {
@@ -298,89 +387,7 @@ __global__ void __launch_bounds__(DECODE ? 448 : 192, 1) k_gemm(const __grid_con
     const int q = warp & 3;
     if (mbar_wait(accum_full, 0, abort_flag, p.err, KID_GEMM, 3)) {
       tc_fence_after();
-      for (int a = 0; a < 2; ++a) {
-        const int m = m0 + a * 128 + q * 32 + lane;
-        const bool mv = m < p.M;
-        const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + a * 256;
-        float v[32], w[32];
-        if (p.epi == EPI_SWIGLU) {
-          for (int c = 0; c < 4; ++c) {
-            ld_acc(tb + c * 32, v);
-            ld_acc(tb + 128 + c * 32, w);
-            if (!mv) continue;
-            const int col = nt * 128 + c * 32;
-            float o[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              v[i] = round_bf16(v[i]);
-              w[i] = round_bf16(w[i]);
-              o[i] = silu_f(v[i]) * w[i];
-            }
-            store32(p.out + (size_t)m * p.ldo + col, o);
-            if (p.aux_out) {
-              store32(p.aux_out + (size_t)m * p.ld_aux_out + col, v);
-              store32(p.aux_out + (size_t)m * p.ld_aux_out + p.inter + col, w);
-            }
-          }
-        } else if (p.epi == EPI_ROPE) {
-          const int d = p.head_dim, half = d / 2;
-          const int pos = m % p.seq;
-          for (int h = 0; h < BN / d; ++h) {
-            const int hc = nt * BN + h * d;
-            if (hc >= p.N) break;
-            if (hc < p.rope_cols) {
-              for (int i = 0; i < half / 32; ++i) {
-                ld_acc(tb + h * d + i * 32, v);
-                ld_acc(tb + h * d + half + i * 32, w);
-                if (!mv) continue;
-                const float* cs = p.rope_cos + (size_t)pos * half + i * 32;
-                const float* sn = p.rope_sin + (size_t)pos * half + i * 32;
-                float o1[32], o2[32];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                  const float c_ = cs[j], s_ = sn[j];
-                  o1[j] = v[j] * c_ - w[j] * s_;
-                  o2[j] = w[j] * c_ + v[j] * s_;
-                }
-                store32(p.out + (size_t)m * p.ldo + hc + i * 32, o1);
-                store32(p.out + (size_t)m * p.ldo + hc + half + i * 32, o2);
-              }
-            } else {
-              for (int c = 0; c < d / 32; ++c) {
-                ld_acc(tb + h * d + c * 32, v);
-                if (mv) store32(p.out + (size_t)m * p.ldo + hc + c * 32, v);
-              }
-            }
-          }
-        } else {
-          for (int c = 0; c < BN / 32; ++c) {
-            const int col = nt * BN + c * 32;
-            if (col >= p.N) break;
-            ld_acc(tb + c * 32, v);
-            if (!mv) continue;
-            if (p.epi == EPI_RESID) {
-              load32_bf16(p.aux0 + (size_t)m * p.ld_aux0 + col, w);
-#pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] += w[i];
-              store32(p.out + (size_t)m * p.ldo + col, v);
-            } else if (p.epi == EPI_DSWIGLU) {
-              float g[32], u[32], dg[32], du[32];
-              load32_bf16(p.aux0 + (size_t)m * p.ld_aux0 + col, g);
-              load32_bf16(p.aux0 + (size_t)m * p.ld_aux0 + p.inter + col, u);
-#pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const float sg = 1.0f / (1.0f + expf(-g[i]));
-                dg[i] = v[i] * u[i] * sg * (1.0f + g[i] * (1.0f - sg));
-                du[i] = v[i] * g[i] * sg;
-              }
-              store32(p.out + (size_t)m * p.ldo + col, dg);
-              store32(p.out + (size_t)m * p.ldo + p.inter + col, du);
-            } else {
-              store32(p.out + (size_t)m * p.ldo + col, v);
-            }
-          }
-        }
-      }
+      epilogue_rows(p, tmem, m0, nt, q, lane);
     }
   } else if (DECODE) {
     // ---------------------------------------------------------------- NF4 decoders
@@ -440,8 +447,18 @@ __global__ void __launch_bounds__(DECODE ? 448 : 192, 1) k_gemm(const __grid_con
         const uint32_t row_addr = BMN ? sB + jj * 8192 + rr * 128 : sB + d * 128;
         const int row_in_atom = (BMN ? rr : d) & 7;
         if (valid) {
-          const uint32_t caddr = BMN ? sC + rr * 128 + jj * 32 : sC + d * 32;
-          const uint4 c0 = ld_shared_v4(caddr), c1 = ld_shared_v4(caddr + 16);
+          // code tiles arrive swizzled (128-byte rows for dL/dx, 32-byte rows forward),
+          // so the 16-byte reads of eight neighbouring rows hit distinct banks
+          uint32_t a0, a1;
+          if (BMN) {
+            a0 = sC + rr * 128 + ((uint32_t)((2 * jj) ^ (rr & 7)) << 4);
+            a1 = sC + rr * 128 + ((uint32_t)((2 * jj + 1) ^ (rr & 7)) << 4);
+          } else {
+            const uint32_t flip = (uint32_t)((d >> 2) & 1) << 4;
+            a0 = sC + d * 32 + flip;
+            a1 = sC + d * 32 + (16u ^ flip);
+          }
+          const uint4 c0 = ld_shared_v4(a0), c1 = ld_shared_v4(a1);
           const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
           const float sc = __fadd_rn(__fmul_rn(code8_s[q8], nested), off);
           decode_block(row_addr, row_in_atom, w, sc, nf4);
@@ -464,6 +481,265 @@ __global__ void __launch_bounds__(DECODE ? 448 : 192, 1) k_gemm(const __grid_con
   }
 }
 
+// ------------------------------------------------------------------------------ CTA-pair kernel
+// The same product with two CTAs per tile (a cluster of 2) and the 2-CTA tcgen05 MMA:
+// the pair computes 512 tokens x 256 output features, CTA r holds tokens
+// m0 + 256 r + [0, 256) (two 128-row accumulators, as above) and supplies B rows
+// 128 r + [0, 128) of the 256-wide tile.  Each decoded weight still meets 256 tokens
+// per MMA, but every SM now decodes (or loads) only half a B tile per stage, which
+// halves the decode ALU work and the B-operand shared-memory traffic per SM.
+// CTA 0 issues every MMA; both CTAs' operand loads and decoders arrive on CTA 0's
+// stage barrier, and the MMA completion is multicast to both CTAs' barriers.
+constexpr int P_STAGES = 4;
+constexpr int PB_BYTES = 128 * BK * 2;  // 16 KB: this CTA's half of the B tile
+constexpr int PC_BYTES = 4096;          // its packed codes
+constexpr int P_STAGE_BYTES = A_BYTES + PB_BYTES + PC_BYTES;
+constexpr int P_SMEM_BYTES = 1024 + P_STAGES * P_STAGE_BYTES + 256 + 1024;
+// Two groups of 4 decoder warps per CTA take alternate k-blocks: each block row of
+// a stage is one thread's work, and a thread has two stages' time to finish it.
+constexpr int P_DECODERS = 256;
+constexpr int P_GROUP = 128;
+
+template <bool DECODE, bool BMN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DECODE ? 448 : 192, 1)
+    k_gemm_pair(const __grid_constant__ GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* misc = base + P_STAGES * P_STAGE_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(misc);
+  uint64_t* empty = full + P_STAGES;
+  uint64_t* codes_full = empty + P_STAGES;
+  uint64_t* accum_full = codes_full + P_STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum_full + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* code8_s = reinterpret_cast<float*>(misc + 256);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1;
+  const int mt = pair % p.n_mt, nt = pair / p.n_mt;
+  const int m0 = mt * 512 + (int)rank * 256;
+  const int total_kb = p.num_kb + p.has_extra;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P_STAGES; ++s) {
+      mbar_init(&full[s], DECODE ? 1 + 2 * (P_GROUP / 32) : 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&codes_full[s], 1);
+    }
+    mbar_init(accum_full, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&p.tmA);
+    if (p.has_extra) {
+      tma_prefetch_desc(&p.tmAx);
+      tma_prefetch_desc(&p.tmBx);
+    }
+    if (!DECODE) tma_prefetch_desc(&p.tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
+  }
+  if (DECODE && warp >= 6)
+    for (int i = threadIdx.x - 192; i < 256; i += P_DECODERS) code8_s[i] = p.code8[i];
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer (both CTAs)
+    if (lane == 0) {
+      for (int kb = 0; kb < total_kb; ++kb) {
+        const int s = kb % P_STAGES;
+        const uint32_t ph = (kb / P_STAGES) & 1;
+        if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, p.err, KID_GEMM, 11)) break;
+        const uint32_t lead = mapa_shared(smem_u32(&full[s]), 0);
+        uint8_t* sA = base + s * P_STAGE_BYTES;
+        uint8_t* sB = sA + A_BYTES;
+        uint8_t* sC = sB + PB_BYTES;
+        const int bcol = nt * BN + (int)rank * 128;  // this CTA's first B row (forward) or column (dL/dx)
+        if (kb < p.num_kb) {
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * A_BYTES + (DECODE ? 0 : 2 * PB_BYTES));
+          tma_load_2d_pair(sA, &p.tmA, lead, kb * BK, m0);
+          if (!DECODE) {
+            if (BMN) {
+              for (int j = 0; j < 2; ++j) tma_load_2d_pair(sB + j * 8192, &p.tmB, lead, bcol + 64 * j, kb * BK);
+            } else if (p.dense_swiglu_rows) {
+              tma_load_2d_pair(sB, &p.tmB, lead, kb * BK, (int)rank * p.dense_swiglu_rows + nt * 128);
+            } else {
+              tma_load_2d_pair(sB, &p.tmB, lead, kb * BK, bcol);
+            }
+          } else if (BMN) {
+            const int row = kb * BK;
+            const int sg = find_seg(p, row);
+            mbar_arrive_expect_tx(&codes_full[s], PC_BYTES);
+            tma_load_2d(sC, &p.tmC[sg], &codes_full[s], bcol / 2, row - p.seg_start[sg]);
+          } else {
+            int nbox = 0, sg[2], lr[2];
+            for (int rb = 0; rb < 2; ++rb) {
+              if (p.swiglu) {
+                sg[rb] = (int)rank;
+                lr[rb] = nt * 128 + 64 * rb;
+              } else {
+                const int row = bcol + 64 * rb;
+                sg[rb] = row < p.N ? find_seg(p, row) : -1;
+                lr[rb] = row < p.N ? row - p.seg_start[sg[rb]] : 0;
+              }
+              if (sg[rb] >= 0) ++nbox;
+            }
+            if (nbox) {
+              mbar_arrive_expect_tx(&codes_full[s], nbox * 2048);
+              for (int rb = 0; rb < 2; ++rb)
+                if (sg[rb] >= 0) tma_load_2d(sC + rb * 2048, &p.tmC[sg[rb]], &codes_full[s], kb * (BK / 2), lr[rb]);
+            } else {
+              mbar_arrive(&codes_full[s]);
+            }
+          }
+        } else {
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * A_BYTES + 2 * PB_BYTES);
+          tma_load_2d_pair(sA, &p.tmAx, lead, 0, m0);
+          if (BMN) {
+            for (int j = 0; j < 2; ++j) tma_load_2d_pair(sB + j * 8192, &p.tmBx, lead, bcol + 64 * j, 0);
+          } else {
+            tma_load_2d_pair(sB, &p.tmBx, lead, 0, bcol);
+          }
+          if (DECODE) mbar_arrive(&codes_full[s]);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer (CTA 0)
+    if (rank == 0) {
+      constexpr uint32_t idesc = idesc_bf16(256, BN, BMN);
+      for (int kb = 0; kb < total_kb; ++kb) {
+        const int s = kb % P_STAGES;
+        const uint32_t ph = (kb / P_STAGES) & 1;
+        if (!mbar_wait(&full[s], ph, abort_flag, p.err, KID_GEMM, 12)) break;
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t aA = smem_u32(base + s * P_STAGE_BYTES);
+          const uint32_t aB = aA + A_BYTES;
+#pragma unroll
+          for (int ks = 0; ks < BK / 16; ++ks) {
+            const uint64_t bdesc =
+                BMN ? sdesc_sw128(aB + ks * 2048, 8192, 1024) : sdesc_sw128(aB + ks * 32, 16, 1024);
+#pragma unroll
+            for (int a = 0; a < 2; ++a) {
+              const uint64_t adesc = sdesc_sw128(aA + a * 16384 + ks * 32, 16, 1024);
+              umma_bf16_pair(tmem + a * 256, adesc, bdesc, idesc, (kb | ks) != 0 ? 1u : 0u);
+            }
+          }
+          umma_commit_pair(&empty[s]);
+        }
+        __syncwarp();
+      }
+      if (lane == 0) umma_commit_pair(accum_full);
+      __syncwarp();
+    }
+  } else if (warp < 6) {
+    // ---------------------------------------------------------------- epilogue (both CTAs)
+    const int q = warp & 3;
+    if (mbar_wait(accum_full, 0, abort_flag, p.err, KID_GEMM, 13)) {
+      tc_fence_after();
+      epilogue_rows(p, tmem, m0, nt, q, lane);
+    }
+  } else if (DECODE) {
+    // ---------------------------------------------------------------- NF4 decoders (both CTAs)
+    const int grp = (threadIdx.x - 192) / P_GROUP;  // which k-blocks: kb = grp, grp + 2, ...
+    const int d = (threadIdx.x - 192) % P_GROUP;    // 0..127
+    float nf4[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) nf4[i] = p.nf4[i];
+    const int bcol = nt * BN + (int)rank * 128;
+    int f_seg = 0, f_row = 0;
+    bool f_valid = true;
+    float f_off = 0.f;
+    if (!BMN) {
+      if (p.swiglu) {
+        f_seg = (int)rank;
+        f_row = nt * 128 + d;
+      } else {
+        const int row = bcol + d;
+        f_valid = row < p.N;
+        f_seg = f_valid ? find_seg(p, row) : 0;
+        f_row = f_valid ? row - p.seg_start[f_seg] : 0;
+      }
+      f_off = *p.offset[f_seg];
+    }
+    const int rr = d & 63, jj = d >> 6;
+    const int dg_col = bcol + 64 * jj;
+    const int blocks_per_row = p.seg_cols / 64;
+    for (int kb = grp; kb < total_kb; kb += 2) {
+      const int s = kb % P_STAGES;
+      const uint32_t ph = (kb / P_STAGES) & 1;
+      bool valid = false;
+      int b = 0, sg = 0;
+      uint32_t q8 = 0;
+      float nested = 0.f, off = 0.f;
+      if (kb < p.num_kb) {
+        if (BMN) {
+          const int row = kb * BK + rr;
+          sg = find_seg(p, kb * BK);
+          valid = dg_col < p.seg_cols;
+          b = (row - p.seg_start[sg]) * blocks_per_row + (dg_col >> 6);
+          if (valid) off = *p.offset[sg];
+        } else {
+          sg = f_seg;
+          valid = f_valid;
+          b = f_row * blocks_per_row + kb;
+          off = f_off;
+        }
+        if (valid) {
+          q8 = p.q8[sg][b];
+          nested = p.nested[sg][b >> 8];
+        }
+      }
+      if (!mbar_wait(&codes_full[s], ph, abort_flag, p.err, KID_GEMM, 14)) break;
+      if (kb < p.num_kb) {
+        const uint32_t sB = smem_u32(base + s * P_STAGE_BYTES + A_BYTES);
+        const uint32_t sC = sB + PB_BYTES;
+        const uint32_t row_addr = BMN ? sB + jj * 8192 + rr * 128 : sB + d * 128;
+        const int row_in_atom = (BMN ? rr : d) & 7;
+        if (valid) {
+          // swizzled code tiles: 64-byte rows (dL/dx) or 32-byte rows (forward)
+          uint32_t a0, a1;
+          if (BMN) {
+            const int x = (rr >> 1) & 3;
+            a0 = sC + rr * 64 + ((uint32_t)((2 * jj) ^ x) << 4);
+            a1 = sC + rr * 64 + ((uint32_t)((2 * jj + 1) ^ x) << 4);
+          } else {
+            const uint32_t flip = (uint32_t)((d >> 2) & 1) << 4;
+            a0 = sC + d * 32 + flip;
+            a1 = sC + d * 32 + (16u ^ flip);
+          }
+          const uint4 c0 = ld_shared_v4(a0), c1 = ld_shared_v4(a1);
+          const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+          const float sc = __fadd_rn(__fmul_rn(code8_s[q8], nested), off);
+          decode_block(row_addr, row_in_atom, w, sc, nf4);
+        } else {
+          zero_block(row_addr);
+        }
+        fence_proxy_async_smem();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&full[s]), 0));
+    }
+  }
+
+  if (rank == 0 && warp == 1 && *abort_flag) mbar_wait_drain(accum_full, 0);
+  tc_fence_before();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, 512);
+  }
+}
+
 // ------------------------------------------------------------------------------ host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -483,7 +759,7 @@ EncodeTiledFn encode_fn() {
 }
 
 int make_map(CUtensorMap* map, CUtensorMapDataType dt, int esize, const void* ptr, uint64_t inner, uint64_t outer,
-             uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+             uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(NF4LS_CUDA, "cuTensorMapEncodeTiled is unavailable");
   if (!aligned(ptr, 16) || row_bytes % 16) return fail(NF4LS_ALIGN, "TMA operand base/row stride not 16-byte aligned");
@@ -493,7 +769,7 @@ int make_map(CUtensorMap* map, CUtensorMapDataType dt, int esize, const void* pt
   const cuuint32_t es[2] = {1, 1};
   (void)esize;
   const CUresult r = fn(map, dt, 2, const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        swz,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(NF4LS_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return NF4LS_OK;
@@ -509,6 +785,22 @@ int launch(const GemmParams& p, int grid, cudaStream_t s) {
     configured[dev] = 1;
   }
   k_gemm<DECODE, BMN><<<grid, DECODE ? 448 : 192, SMEM_BYTES, s>>>(p);
+  note_launch();
+  NF4_CUDA_TRY(cudaGetLastError());
+  return NF4LS_OK;
+}
+
+template <bool DECODE, bool BMN>
+int launch_pair(const GemmParams& p, int grid, cudaStream_t s) {
+  static int configured[16] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 16 && !configured[dev]) {
+    NF4_CUDA_TRY(cudaFuncSetAttribute(k_gemm_pair<DECODE, BMN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      P_SMEM_BYTES));
+    configured[dev] = 1;
+  }
+  k_gemm_pair<DECODE, BMN><<<grid, DECODE ? 448 : 192, P_SMEM_BYTES, s>>>(p);
   note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;
@@ -536,25 +828,28 @@ int gemm(const __nv_bfloat16* A, int lda, int M, int N, int K, const GemmWeights
   p.K = K;
   p.num_kb = K / 64;
   p.has_extra = extra.a != nullptr;
-  p.n_mt = (M + BM - 1) / BM;
+  // CTA pairs for every product with more than one 256-token tile; single CTAs below.
+  const bool pair = gemm_pair() && M > BM;
+  const uint32_t bbox = pair ? 128 : 256;  // B rows one CTA loads (forward, K-major)
+  p.n_mt = pair ? (M + 511) / 512 : (M + BM - 1) / BM;
   const int n_nt = swiglu ? epi.inter / 128 : (N + BN - 1) / BN;
-  NF4_TRY(make_map(&p.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A, K, M, (uint64_t)lda * 2, 64, 256, true));
+  NF4_TRY(make_map(&p.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A, K, M, (uint64_t)lda * 2, 64, 256, CU_TENSOR_MAP_SWIZZLE_128B));
   if (p.has_extra) {
     if (!extra.b) return fail(NF4LS_INVALID_ARG, "gemm: extra block needs both operands");
-    NF4_TRY(make_map(&p.tmAx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, extra.a, 64, M, 128, 64, 256, true));
+    NF4_TRY(make_map(&p.tmAx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, extra.a, 64, M, 128, 64, 256, CU_TENSOR_MAP_SWIZZLE_128B));
     if (dgrad)
-      NF4_TRY(make_map(&p.tmBx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, extra.b, N, 64, (uint64_t)N * 2, 64, 64, true));
+      NF4_TRY(make_map(&p.tmBx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, extra.b, N, 64, (uint64_t)N * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B));
     else
-      NF4_TRY(make_map(&p.tmBx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, extra.b, 64, N, 128, 64, 256, true));
+      NF4_TRY(make_map(&p.tmBx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, extra.b, 64, N, 128, 64, bbox, CU_TENSOR_MAP_SWIZZLE_128B));
   }
   if (!decode) {
     if (dgrad)  // W [K, N]
-      NF4_TRY(make_map(&p.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W.dense, N, K, (uint64_t)N * 2, 64, 64, true));
+      NF4_TRY(make_map(&p.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W.dense, N, K, (uint64_t)N * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B));
     else if (swiglu) {  // W [2I, K]: gate rows then up rows
-      NF4_TRY(make_map(&p.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W.dense, K, N, (uint64_t)K * 2, 64, 128, true));
+      NF4_TRY(make_map(&p.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W.dense, K, N, (uint64_t)K * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B));
       p.dense_swiglu_rows = epi.inter;
     } else
-      NF4_TRY(make_map(&p.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W.dense, K, N, (uint64_t)K * 2, 64, 256, true));
+      NF4_TRY(make_map(&p.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W.dense, K, N, (uint64_t)K * 2, 64, bbox, CU_TENSOR_MAP_SWIZZLE_128B));
   } else {
     p.n_seg = W.n_seg;
     p.swiglu = swiglu;
@@ -568,10 +863,15 @@ int gemm(const __nv_bfloat16* A, int lda, int M, int N, int K, const GemmWeights
       p.q8[i] = t.q8;
       p.nested[i] = t.nested;
       p.offset[i] = t.offset;
-      if (dgrad)  // codes [rows, N/2] bytes; box 128 B x 64 rows
-        NF4_TRY(make_map(&p.tmC[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, t.packed, cols / 2, t.rows, cols / 2, 128, 64, false));
+      if (dgrad && pair)  // codes [rows, N/2] bytes; box 64 B x 64 rows (one CTA's 128 columns)
+        NF4_TRY(make_map(&p.tmC[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, t.packed, cols / 2, t.rows, cols / 2, 64, 64,
+                         CU_TENSOR_MAP_SWIZZLE_64B));
+      else if (dgrad)  // codes [rows, N/2] bytes; box 128 B x 64 rows
+        NF4_TRY(make_map(&p.tmC[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, t.packed, cols / 2, t.rows, cols / 2, 128, 64,
+                                 CU_TENSOR_MAP_SWIZZLE_128B));
       else  // codes [rows, K/2] bytes; box 32 B x 64 rows
-        NF4_TRY(make_map(&p.tmC[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, t.packed, cols / 2, t.rows, cols / 2, 32, 64, false));
+        NF4_TRY(make_map(&p.tmC[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, t.packed, cols / 2, t.rows, cols / 2, 32, 64,
+                                 CU_TENSOR_MAP_SWIZZLE_32B));
     }
     p.seg_start[W.n_seg] = start;
     p.seg_cols = cols;
@@ -597,14 +897,20 @@ int gemm(const __nv_bfloat16* A, int lda, int M, int N, int K, const GemmWeights
   p.head_dim = epi.head_dim;
   p.rope_cols = epi.rope_cols;
   p.err = device_error_ptr();
-  const int grid = p.n_mt * n_nt;
+  const int grid = p.n_mt * n_nt * (pair ? 2 : 1);
   cudaEvent_t e0 = nullptr;
   if (profiling()) profile_begin(s, &e0);
   int st;
-  if (decode)
+  if (pair) {
+    if (decode)
+      st = dgrad ? launch_pair<true, true>(p, grid, s) : launch_pair<true, false>(p, grid, s);
+    else
+      st = dgrad ? launch_pair<false, true>(p, grid, s) : launch_pair<false, false>(p, grid, s);
+  } else if (decode) {
     st = dgrad ? launch<true, true>(p, grid, s) : launch<true, false>(p, grid, s);
-  else
+  } else {
     st = dgrad ? launch<false, true>(p, grid, s) : launch<false, false>(p, grid, s);
+  }
   // algorithmic work: 2 M N K, plus the 64-wide LoRA block when present
   if (e0) profile_end(s, e0, decode ? 1 : 0, 2.0 * M * (double)N * (K + (p.has_extra ? 64 : 0)));
   return st;

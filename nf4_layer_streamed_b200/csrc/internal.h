@@ -118,6 +118,7 @@ int gemm(const __nv_bfloat16* A, int lda, int M, int N, int K, const GemmWeights
          const GemmExtra& extra, const GemmEpilogue& epi, cudaStream_t s);
 
 int gemm_path();
+int gemm_pair();
 int check_cfg(const nf4ls_layer_cfg* c);
 int* device_error_ptr();
 

@@ -74,7 +74,9 @@ def main(argv=None):
     ap.add_argument("--shapes", default="qo,kv,gateup,down")
     ap.add_argument("--iters", type=int, default=20)
     ap.add_argument("--once", action="store_true")
+    ap.add_argument("--single", action="store_true", help="one CTA per tile instead of CTA pairs")
     a = ap.parse_args(argv)
+    api.set_gemm_pair(not a.single)
     run(a.M, a.shapes.split(","), a.iters, a.once)
     st, err = api.device_error()
     if st != 0:

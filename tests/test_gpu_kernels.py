@@ -119,6 +119,29 @@ def test_nf4_gemm_bit_exact_against_dense_on_dequantised(M, rows, cols):
     assert st == 0, err
 
 
+@pytest.mark.parametrize("M,rows,cols", [(512, 576, 576), (600, 960, 576), (2048, 4096, 4096)])
+def test_cta_pair_gemm_equals_single_cta(M, rows, cols):
+    w = synth.tensor_values((rows, cols), seed=3 * rows + cols, scale=0.02).to(DEV)
+    q = api.nf4_quantize_tensor(w)
+    deq = api.nf4_dequantize_tensor(q).view(rows, cols)
+    A = synth.tensor_values((M, cols), seed=M + 1, scale=1.0).to(DEV)
+    G = synth.tensor_values((M, rows), seed=M + 2, scale=1.0).to(DEV)
+    outs = {}
+    try:
+        for pair in (False, True):
+            api.set_gemm_pair(pair)
+            outs[pair] = [api.gemm_nf4(A, q, rows, cols), api.gemm_nf4(G, q, rows, cols, dgrad=True),
+                          api.gemm_bf16(A, deq), api.gemm_bf16(G, deq, b_trans=True)]
+    finally:
+        api.set_gemm_pair(True)
+    for a, b in zip(outs[False], outs[True]):
+        assert torch.equal(a, b)
+    close(outs[True][0], f64(A) @ f64(deq).T, tol=1e-2, what="pair forward")
+    close(outs[True][1], f64(G) @ f64(deq), tol=1e-2, what="pair dL/dx")
+    st, err = api.device_error()
+    assert st == 0, err
+
+
 @pytest.mark.parametrize("shape,batch,seq", [(synth.SMOLLM2_135M, 1, 512), (synth.LLAMA_8B, 2, 128)])
 def test_attention_forward_against_oracle(shape, batch, seq):
     cfg = api.layer_cfg(shape, batch, seq)
