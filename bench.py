@@ -223,7 +223,7 @@ def main():
     barrier()
     st0 = m.pool.stats()
     launches0 = api.launch_count()
-    api.profile_read(0), api.profile_read(1)
+    api.profile_reset()
     api.profile(True)
     clocks = Clocks(local)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -247,6 +247,15 @@ def main():
     value = tok * world / (ms_max / 1000.0)
     nf4 = api.profile_read(1)
     dense = api.profile_read(0)
+    breakdown = {}
+    for code, name in list(api.GEMM_DETAILS.items()) + list(api.PHASES.items()):
+        r = api.profile_read(code)
+        if r["launches"]:
+            e = {"ms_per_step": r["ms"] / args.steps, "launches_per_step": r["launches"] / args.steps}
+            if r["flops"]:
+                e["tflops"] = r["flops"] / (r["ms"] / 1000.0) / 1e12
+            breakdown[name] = e
+    api.profile_reset()
     st, err = api.device_error()
     if st != 0:
         raise RuntimeError(f"device error record: {err}")
@@ -328,6 +337,7 @@ def main():
                        "h2d_link_gbs": best,
                        "copy_ms_per_step_at_link_rate": copy_bytes / best / 1e6 if best else None,
                        "copies_per_step": (st1["copies"] - st0["copies"]) / args.steps},
+            "breakdown": breakdown,
             "loss_last": loss,
             "gpu_launches": int(launches),
             "clocks": ck,

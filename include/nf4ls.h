@@ -63,13 +63,18 @@ int nf4ls_version(void);
 /* Number of kernels the library has launched in this process (all devices). */
 uint64_t nf4ls_launch_count(void);
 
-/* Per-launch timing of the GEMM kernels with CUDA events recorded on the launching
- * stream (off by default).  nf4ls_profile_read(kind, out) waits for the recorded
- * launches of that kind (0 dense bf16 GEMM, 1 NF4-decode GEMM), returns out[0] =
- * launches, out[1] = total milliseconds, out[2] = total algorithmic FLOPs
- * (2 M N K per launch), and forgets them. */
+/* Per-launch timing with CUDA events recorded on the launching stream (off by
+ * default): every GEMM launch and the phases of the model step.  nf4ls_profile_read
+ * waits for the matching records and returns out[0] = count, out[1] = total ms,
+ * out[2] = total algorithmic FLOPs (2 M N K per GEMM launch).  sel < 1000 selects a
+ * kind (0 dense bf16 GEMM, 1 NF4-decode GEMM, 2 step phase); sel >= 1000 a detail:
+ * 1000 + 100 * (NF4 decode) + 10 * (dL/dx product) + epilogue (0 store, 1 residual,
+ * 2 RoPE, 3 SwiGLU, 4 SwiGLU backward) for GEMMs, and 2000 layer forwards, 2001
+ * final norm + lm_head + loss, 2002 lm_head dL/dx + final-norm backward, 2003 layer
+ * backwards for phases.  nf4ls_profile_reset forgets every record. */
 int nf4ls_profile(int on);
-int nf4ls_profile_read(int kind, double out[3]);
+int nf4ls_profile_read(int sel, double out[3]);
+int nf4ls_profile_reset(void);
 
 /* Reads and clears the device error flag of the current device: out[0] = code
  * (0 none, 1 barrier timeout), out[1] = kernel id, out[2] = block, out[3] = site.

@@ -66,11 +66,24 @@ def profile(on: bool) -> None:
     B.call("nf4ls_profile", int(on))
 
 
-def profile_read(kind: int) -> dict:
-    """kind 0: dense GEMM launches, 1: NF4-decode GEMM launches since the last read."""
+def profile_read(sel: int) -> dict:
+    """Aggregate of the timed records since the last reset: sel 0 dense GEMMs, 1 NF4-decode
+    GEMMs, 2 step phases; sel >= 1000 one detail (see nf4ls_profile_read in the header)."""
     out = (ctypes.c_double * 3)()
-    B.call("nf4ls_profile_read", kind, ctypes.cast(out, ctypes.c_void_p))
+    B.call("nf4ls_profile_read", sel, ctypes.cast(out, ctypes.c_void_p))
     return {"launches": int(out[0]), "ms": float(out[1]), "flops": float(out[2])}
+
+
+def profile_reset() -> None:
+    B.call("nf4ls_profile_reset")
+
+
+GEMM_DETAILS = {}
+for _dec, _dn in ((0, "dense"), (1, "nf4")):
+    for _dg, _gn in ((0, "fwd"), (1, "dgrad")):
+        for _e, _en in enumerate(("store", "resid", "rope", "swiglu", "dswiglu")):
+            GEMM_DETAILS[1000 + 100 * _dec + 10 * _dg + _e] = f"{_dn}_{_gn}_{_en}"
+PHASES = {2000: "layers_forward", 2001: "head_forward_loss", 2002: "head_backward", 2003: "layers_backward"}
 
 
 def device_error():

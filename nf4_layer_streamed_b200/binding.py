@@ -73,6 +73,7 @@ SIGNATURES = {
     "nf4ls_launch_count": (U64, []),
     "nf4ls_profile": (ctypes.c_int, [ctypes.c_int]),
     "nf4ls_profile_read": (ctypes.c_int, [ctypes.c_int, P]),
+    "nf4ls_profile_reset": (ctypes.c_int, []),
     "nf4ls_codebooks": (ctypes.c_int, [P, P, ctypes.POINTER(U64)]),
     "nf4ls_quantize_scratch_bytes": (SZ, [SZ]),
     "nf4_quantize_tensor": (ctypes.c_int, [P, SZ, P, P, P, P, P, SZ, P]),

@@ -31,7 +31,7 @@ namespace {
 std::atomic<uint64_t> g_launches{0};
 std::atomic<int> g_profile{0};
 struct Rec {
-  int kind;
+  int kind, detail;
   double flops;
   cudaEvent_t e0, e1;
 };
@@ -61,12 +61,12 @@ void profile_begin(cudaStream_t s, cudaEvent_t* e0) {
   if (*e0) cudaEventRecord(*e0, s);
 }
 
-void profile_end(cudaStream_t s, cudaEvent_t e0, int kind, double flops) {
+void profile_end(cudaStream_t s, cudaEvent_t e0, int kind, int detail, double flops) {
   std::lock_guard<std::mutex> g(g_prof_mu);
   cudaEvent_t e1 = take_event();
   if (!e0 || !e1) return;
   cudaEventRecord(e1, s);
-  g_recs.push_back(Rec{kind, flops, e0, e1});
+  g_recs.push_back(Rec{kind, detail, flops, e0, e1});
 }
 
 }  // namespace nf4ls
@@ -74,34 +74,48 @@ void profile_end(cudaStream_t s, cudaEvent_t e0, int kind, double flops) {
 extern "C" uint64_t nf4ls_launch_count(void) { return nf4ls::g_launches.load(); }
 
 extern "C" int nf4ls_profile(int on) {
+  if (on) {
+    // create the events up front so that recording stays cheap inside a timed region
+    std::lock_guard<std::mutex> g(nf4ls::g_prof_mu);
+    while (nf4ls::g_free_events.size() + 2 * nf4ls::g_recs.size() < 16384) {
+      cudaEvent_t e = nullptr;
+      if (cudaEventCreate(&e) != cudaSuccess) break;
+      nf4ls::g_free_events.push_back(e);
+    }
+  }
   nf4ls::g_profile.store(on ? 1 : 0);
   return NF4LS_OK;
 }
 
-extern "C" int nf4ls_profile_read(int kind, double out[3]) {
+extern "C" int nf4ls_profile_read(int sel, double out[3]) {
   nf4ls::clear_error();
   if (!out) return nf4ls::fail(NF4LS_INVALID_ARG, "nf4ls_profile_read: null output");
   std::lock_guard<std::mutex> g(nf4ls::g_prof_mu);
   double n = 0, ms = 0, flops = 0;
-  std::vector<nf4ls::Rec> keep;
   for (auto& r : nf4ls::g_recs) {
-    if (r.kind != kind) {
-      keep.push_back(r);
-      continue;
-    }
+    if ((sel < 1000 ? r.kind : r.detail) != sel) continue;
     NF4_CUDA_TRY(cudaEventSynchronize(r.e1));
     float t = 0.f;
     NF4_CUDA_TRY(cudaEventElapsedTime(&t, r.e0, r.e1));
     n += 1;
     ms += t;
     flops += r.flops;
-    nf4ls::g_free_events.push_back(r.e0);
-    nf4ls::g_free_events.push_back(r.e1);
   }
-  nf4ls::g_recs.swap(keep);
   out[0] = n;
   out[1] = ms;
   out[2] = flops;
+  return NF4LS_OK;
+}
+
+extern "C" int nf4ls_profile_reset(void) {
+  nf4ls::clear_error();
+  std::lock_guard<std::mutex> g(nf4ls::g_prof_mu);
+  for (auto& r : nf4ls::g_recs) {
+    NF4_CUDA_TRY(cudaEventSynchronize(r.e1));
+    nf4ls::g_free_events.push_back(r.e0);
+    nf4ls::g_free_events.push_back(r.e1);
+  }
+  nf4ls::g_recs.clear();
   return NF4LS_OK;
 }
 

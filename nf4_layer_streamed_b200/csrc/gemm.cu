@@ -154,31 +154,68 @@ __device__ __forceinline__ void ld_acc(uint32_t taddr, float (&v)[32]) {
 }
 
 // ------------------------------------------------------------------------------ epilogue
-// One epilogue warp (TMEM lane quarter q) turns the two 128 x 256 fp32 accumulators of
-// its CTA (tokens m0 + [0, 256), output features of tile nt) into bf16 results.
-__device__ __forceinline__ void epilogue_rows(const GemmParams& p, uint32_t tmem, int m0, int nt, int q, int lane) {
+// The epilogue warps of TMEM lane quarter q turn the two 128 x 256 fp32 accumulators of
+// their CTA (tokens m0 + [0, 256), output features of tile nt) into bf16 results.
+// The work of a quarter is a list of 16-column items (per accumulator: 16 column
+// chunks, 8 gate/up chunk pairs for SwiGLU, or per head the RoPE half-chunk pairs);
+// warp `part` of the `nparts` warps that share the quarter takes every nparts-th item.
+__device__ __forceinline__ void ld_acc16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  tmem_ld16(taddr, r);
+  tmem_wait_ld();
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void store16(__nv_bfloat16* dst, const float (&v)[16]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+    d[i] = make_uint4(pack_bf16x2(v[8 * i + 0], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                      pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+}
+
+__device__ __forceinline__ void load16_bf16(const __nv_bfloat16* src, float (&v)[16]) {
+  const uint4* s = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const uint4 u = s[i];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[8 * i + 2 * j] = bf16_lo(w[j]);
+      v[8 * i + 2 * j + 1] = bf16_hi(w[j]);
+    }
+  }
+}
+
+__device__ __forceinline__ void epilogue_rows(const GemmParams& p, uint32_t tmem, int m0, int nt, int q, int lane,
+                                              int part = 0, int nparts = 1) {
+  constexpr int CW = 16;
+  int item = 0;
   for (int a = 0; a < 2; ++a) {
     const int m = m0 + a * 128 + q * 32 + lane;
     const bool mv = m < p.M;
     const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + a * 256;
-    float v[32], w[32];
+    float v[CW], w[CW];
     if (p.epi == EPI_SWIGLU) {
-      for (int c = 0; c < 4; ++c) {
-        ld_acc(tb + c * 32, v);
-        ld_acc(tb + 128 + c * 32, w);
+      for (int c = 0; c < 128 / CW; ++c) {
+        if ((item++ % nparts) != part) continue;
+        ld_acc16(tb + c * CW, v);
+        ld_acc16(tb + 128 + c * CW, w);
         if (!mv) continue;
-        const int col = nt * 128 + c * 32;
-        float o[32];
+        const int col = nt * 128 + c * CW;
+        float o[CW];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
+        for (int i = 0; i < CW; ++i) {
           v[i] = round_bf16(v[i]);
           w[i] = round_bf16(w[i]);
           o[i] = silu_f(v[i]) * w[i];
         }
-        store32(p.out + (size_t)m * p.ldo + col, o);
+        store16(p.out + (size_t)m * p.ldo + col, o);
         if (p.aux_out) {
-          store32(p.aux_out + (size_t)m * p.ld_aux_out + col, v);
-          store32(p.aux_out + (size_t)m * p.ld_aux_out + p.inter + col, w);
+          store16(p.aux_out + (size_t)m * p.ld_aux_out + col, v);
+          store16(p.aux_out + (size_t)m * p.ld_aux_out + p.inter + col, w);
         }
       }
     } else if (p.epi == EPI_ROPE) {
@@ -188,54 +225,62 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, uint32_t tmem
         const int hc = nt * BN + h * d;
         if (hc >= p.N) break;
         if (hc < p.rope_cols) {
-          for (int i = 0; i < half / 32; ++i) {
-            ld_acc(tb + h * d + i * 32, v);
-            ld_acc(tb + h * d + half + i * 32, w);
+          for (int i = 0; i < half / CW; ++i) {
+            if ((item++ % nparts) != part) continue;
+            ld_acc16(tb + h * d + i * CW, v);
+            ld_acc16(tb + h * d + half + i * CW, w);
             if (!mv) continue;
-            const float* cs = p.rope_cos + (size_t)pos * half + i * 32;
-            const float* sn = p.rope_sin + (size_t)pos * half + i * 32;
-            float o1[32], o2[32];
+            const float* cs = p.rope_cos + (size_t)pos * half + i * CW;
+            const float* sn = p.rope_sin + (size_t)pos * half + i * CW;
+            float o1[CW], o2[CW];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
+            for (int j = 0; j < CW; ++j) {
               const float c_ = cs[j], s_ = sn[j];
               o1[j] = v[j] * c_ - w[j] * s_;
               o2[j] = w[j] * c_ + v[j] * s_;
             }
-            store32(p.out + (size_t)m * p.ldo + hc + i * 32, o1);
-            store32(p.out + (size_t)m * p.ldo + hc + half + i * 32, o2);
+            store16(p.out + (size_t)m * p.ldo + hc + i * CW, o1);
+            store16(p.out + (size_t)m * p.ldo + hc + half + i * CW, o2);
           }
         } else {
-          for (int c = 0; c < d / 32; ++c) {
-            ld_acc(tb + h * d + c * 32, v);
-            if (mv) store32(p.out + (size_t)m * p.ldo + hc + c * 32, v);
+          for (int c = 0; c < d / CW; ++c) {
+            if ((item++ % nparts) != part) continue;
+            ld_acc16(tb + h * d + c * CW, v);
+            if (mv) store16(p.out + (size_t)m * p.ldo + hc + c * CW, v);
           }
         }
       }
     } else {
-      for (int c = 0; c < BN / 32; ++c) {
-        const int col = nt * BN + c * 32;
+      for (int c = 0; c < BN / CW; ++c) {
+        const int col = nt * BN + c * CW;
         if (col >= p.N) break;
-        ld_acc(tb + c * 32, v);
-        if (!mv) continue;
+        if ((item++ % nparts) != part) continue;
         if (p.epi == EPI_RESID) {
-          load32_bf16(p.aux0 + (size_t)m * p.ld_aux0 + col, w);
+          if (mv) load16_bf16(p.aux0 + (size_t)m * p.ld_aux0 + col, w);  // in flight during the TMEM load
+          ld_acc16(tb + c * CW, v);
+          if (!mv) continue;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] += w[i];
-          store32(p.out + (size_t)m * p.ldo + col, v);
+          for (int i = 0; i < CW; ++i) v[i] += w[i];
+          store16(p.out + (size_t)m * p.ldo + col, v);
         } else if (p.epi == EPI_DSWIGLU) {
-          float g[32], u[32], dg[32], du[32];
-          load32_bf16(p.aux0 + (size_t)m * p.ld_aux0 + col, g);
-          load32_bf16(p.aux0 + (size_t)m * p.ld_aux0 + p.inter + col, u);
+          float g[CW], u[CW], dg[CW], du[CW];
+          if (mv) {
+            load16_bf16(p.aux0 + (size_t)m * p.ld_aux0 + col, g);
+            load16_bf16(p.aux0 + (size_t)m * p.ld_aux0 + p.inter + col, u);
+          }
+          ld_acc16(tb + c * CW, v);
+          if (!mv) continue;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
+          for (int i = 0; i < CW; ++i) {
             const float sg = 1.0f / (1.0f + expf(-g[i]));
             dg[i] = v[i] * u[i] * sg * (1.0f + g[i] * (1.0f - sg));
             du[i] = v[i] * g[i] * sg;
           }
-          store32(p.out + (size_t)m * p.ldo + col, dg);
-          store32(p.out + (size_t)m * p.ldo + p.inter + col, du);
+          store16(p.out + (size_t)m * p.ldo + col, dg);
+          store16(p.out + (size_t)m * p.ldo + p.inter + col, du);
         } else {
-          store32(p.out + (size_t)m * p.ldo + col, v);
+          ld_acc16(tb + c * CW, v);
+          if (mv) store16(p.out + (size_t)m * p.ldo + col, v);
         }
       }
     }
@@ -387,7 +432,7 @@ __global__ void __launch_bounds__(DECODE ? 448 : 192, 1) k_gemm(const __grid_con
     const int q = warp & 3;
     if (mbar_wait(accum_full, 0, abort_flag, p.err, KID_GEMM, 3)) {
       tc_fence_after();
-      epilogue_rows(p, tmem, m0, nt, q, lane);
+      epilogue_rows(p, tmem, m0, nt, q, lane, 0, DECODE ? 3 : 1);
     }
   } else if (DECODE) {
     // ---------------------------------------------------------------- NF4 decoders
@@ -468,6 +513,11 @@ __global__ void __launch_bounds__(DECODE ? 448 : 192, 1) k_gemm(const __grid_con
         fence_proxy_async_smem();
       }
       mbar_arrive(&full[s]);
+    }
+    // then share the epilogue: 3 warps per TMEM lane quarter
+    if (mbar_wait(accum_full, 0, abort_flag, p.err, KID_GEMM, 5)) {
+      tc_fence_after();
+      epilogue_rows(p, tmem, m0, nt, warp & 3, lane, (warp - 2) / 4, 3);
     }
   }
 
@@ -646,7 +696,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DECODE ? 448 : 192, 
     const int q = warp & 3;
     if (mbar_wait(accum_full, 0, abort_flag, p.err, KID_GEMM, 13)) {
       tc_fence_after();
-      epilogue_rows(p, tmem, m0, nt, q, lane);
+      epilogue_rows(p, tmem, m0, nt, q, lane, 0, DECODE ? 3 : 1);
     }
   } else if (DECODE) {
     // ---------------------------------------------------------------- NF4 decoders (both CTAs)
@@ -728,6 +778,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DECODE ? 448 : 192, 
       }
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&full[s]), 0));
+    }
+    // then share the epilogue: 3 warps per TMEM lane quarter
+    if (mbar_wait(accum_full, 0, abort_flag, p.err, KID_GEMM, 15)) {
+      tc_fence_after();
+      epilogue_rows(p, tmem, m0, nt, warp & 3, lane, (warp - 2) / 4, 3);
     }
   }
 
@@ -912,7 +967,10 @@ int gemm(const __nv_bfloat16* A, int lda, int M, int N, int K, const GemmWeights
     st = dgrad ? launch<false, true>(p, grid, s) : launch<false, false>(p, grid, s);
   }
   // algorithmic work: 2 M N K, plus the 64-wide LoRA block when present
-  if (e0) profile_end(s, e0, decode ? 1 : 0, 2.0 * M * (double)N * (K + (p.has_extra ? 64 : 0)));
+  // kind 0/1 (dense / NF4 decode); detail 1000 + 100 decode + 10 dL/dx + epilogue
+  if (e0)
+    profile_end(s, e0, decode ? 1 : 0, 1000 + (decode ? 100 : 0) + (dgrad ? 10 : 0) + epi.kind,
+                2.0 * M * (double)N * (K + (p.has_extra ? 64 : 0)));
   return st;
 }
 

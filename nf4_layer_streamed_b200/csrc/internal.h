@@ -128,7 +128,7 @@ void note_launch(int n = 1);
 // Optional per-launch CUDA-event timing of the GEMMs (kind 0 dense, 1 NF4 decode).
 bool profiling();
 void profile_begin(cudaStream_t s, cudaEvent_t* e0);
-void profile_end(cudaStream_t s, cudaEvent_t e0, int kind, double flops);
+void profile_end(cudaStream_t s, cudaEvent_t e0, int kind, int detail, double flops);
 
 // ----------------------------------------------------------------------------- body kernels
 int rmsnorm_fwd(const __nv_bfloat16* x, const __nv_bfloat16* w, __nv_bfloat16* y, int M, int H, float eps,

@@ -66,6 +66,20 @@ T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
 }
 
+// Phase timing (when profiling is on): detail 2000 layer forwards, 2001 final norm +
+// lm_head + loss, 2002 lm_head dL/dx + final-norm backward, 2003 layer backwards.
+struct Phase {
+  cudaStream_t s;
+  cudaEvent_t e = nullptr;
+  int detail;
+  Phase(cudaStream_t s_, int d) : s(s_), detail(d) {
+    if (profiling()) profile_begin(s, &e);
+  }
+  ~Phase() {
+    if (e) profile_end(s, e, 2, detail, 0.0);
+  }
+};
+
 int acquire(const nf4ls_model* m, int layer, int dir, cudaStream_t s, const void** shard) {
   if (!m->pool) {
     *shard = m->shards_dev[layer];
@@ -120,6 +134,8 @@ int forward_to_loss(const nf4ls_model_cfg* c, const nf4ls_model* m, const int32_
   const size_t stride = stride_of(lc);
   NF4_TRY(embed(ids, static_cast<const __nv_bfloat16*>(m->embed_dev), xs, M, H, s));
   const int depth = pool_depth(m);
+  {
+  Phase fwd_phase(s, 2000);
   for (int i = 0; i < c->n_layers; ++i) {
     const void* shard;
     NF4_TRY(acquire(m, i, +1, s, &shard));
@@ -130,6 +146,8 @@ int forward_to_loss(const nf4ls_model_cfg* c, const nf4ls_model* m, const int32_
                            at<void>(ws, L.layer), L.total - L.layer, s));
     NF4_TRY(release(m, i, s));
   }
+  }
+  Phase head(s, 2001);
   auto* hf = at<__nv_bfloat16>(ws, L.hf);
   auto* logits = at<__nv_bfloat16>(ws, L.logits);
   const auto* lm = static_cast<const __nv_bfloat16*>(c->tied ? m->embed_dev : m->lm_head_dev);
@@ -180,16 +198,20 @@ extern "C" int nf4ls_forward_backward(const nf4ls_model_cfg* cfg, const nf4ls_mo
   auto* dhf = at<__nv_bfloat16>(ws, L.dhf);
   auto* dh = at<__nv_bfloat16>(ws, L.dh);
   const auto* lm = static_cast<const __nv_bfloat16*>(cfg->tied ? m->embed_dev : m->lm_head_dev);
-  GemmWeights w;
-  w.dense = lm;
-  GemmEpilogue e;
-  e.out = dhf;
-  e.ldo = H;
-  NF4_TRY(gemm(logits, V, M, H, V, w, true, GemmExtra(), e, s));
-  NF4_TRY(rmsnorm_bwd(xs + (size_t)cfg->n_layers * act, static_cast<const __nv_bfloat16*>(m->norm_final_dev), dhf,
-                      nullptr, dh, M, H, lc->rms_eps, s));
+  {
+    Phase head_bwd(s, 2002);
+    GemmWeights w;
+    w.dense = lm;
+    GemmEpilogue e;
+    e.out = dhf;
+    e.ldo = H;
+    NF4_TRY(gemm(logits, V, M, H, V, w, true, GemmExtra(), e, s));
+    NF4_TRY(rmsnorm_bwd(xs + (size_t)cfg->n_layers * act, static_cast<const __nv_bfloat16*>(m->norm_final_dev), dhf,
+                        nullptr, dh, M, H, lc->rms_eps, s));
+  }
   const size_t stride = stride_of(lc);
   const int depth = pool_depth(m);
+  Phase bwd_phase(s, 2003);
   for (int i = cfg->n_layers - 1; i >= 0; --i) {
     const void* shard;
     NF4_TRY(acquire(m, i, -1, s, &shard));
