@@ -53,6 +53,30 @@ def test_pool_copies_hits_and_slot_contents():
         pool.destroy()
 
 
+def test_pool_wait_times_out_while_the_slot_is_still_read():
+    """A copy into a slot waits for the release event of the slot's last reader; a
+    bounded host wait on that copy returns TIMEOUT while the reader is still busy
+    (a GPU spin of about a second, which ends by itself) and OK afterwards."""
+    shape = synth.SMOLLM2_135M
+    cfg = api.layer_cfg(shape, 1, 512)
+    nb = api.shard_bytes(cfg)
+    slot = (nb + 255) // 256 * 256
+    store = torch.zeros(3 * slot, dtype=torch.uint8).pin_memory()
+    pool = api.Pool(store, [0, slot, 2 * slot], [nb] * 3, depth=2)
+    try:
+        pool.stream_prefetch(0)
+        torch.cuda._sleep(2_000_000_000)      # the reader of layer 0 stays busy ~1 s
+        pool.release(0)
+        pool.stream_prefetch(1)
+        pool.release(1)
+        assert pool.prefetch(2) == 0          # goes into layer 0's slot, after its release
+        assert pool.wait(2, 20) == -7         # TIMEOUT
+        assert pool.wait(2, 10000) == 0
+        torch.cuda.synchronize()
+    finally:
+        pool.destroy()
+
+
 def _train(wl, depth, resident, steps, poison=False, b_random=False):
     m = api.StreamedModel(wl, depth=depth, resident=resident, b_random=b_random)
     if poison and m.pool is not None:
@@ -126,6 +150,32 @@ def test_smollm2_30_layers_first_step_against_oracle():
             assert torch.count_nonzero(m.grad_views(i)["dA_q"]) > 0, i
     finally:
         m.close()
+
+
+def test_adapter_off_reference_pass():
+    """The DPO/KTO reference model is the same streamed base with the adapter off
+    ("Soup v0.72.4 技术解析" §3.1): nf4ls_forward_loss(lora_on = 0) over the streamed
+    layers equals the resident run bit for bit, differs from the adapter-on loss when
+    B is nonzero, and matches the oracle's adapter-free forward."""
+    wl = synth.Workload("smollm2_4L_tied", synth.SMOLLM2_135M, 4, 1, 512, vocab=49152, tied=True)
+    m_res = api.StreamedModel(wl, resident=True, b_random=True)
+    m_str = api.StreamedModel(wl, depth=2, resident=False, b_random=True)
+    try:
+        ids = synth.token_ids(wl.vocab, wl.batch, wl.seq, wl.seed, step=0, device=DEV)
+        off_res = m_res.forward_loss(ids, lora_on=False).clone()
+        off_str = m_str.forward_loss(ids, lora_on=False).clone()
+        on_str = m_str.forward_loss(ids, lora_on=True).clone()
+        torch.cuda.synchronize()
+        assert torch.equal(off_res, off_str)
+        assert not torch.equal(off_str, on_str)
+        shape = wl.shape
+        layers = [oracle_weights(synth.layer_weights(shape, i, wl.seed, device=DEV)) for i in range(wl.n_layers)]
+        loss, _, _ = omodel.forward_backward(ids.cpu().numpy(), layers, [None] * wl.n_layers, f64(m_str.embed), None,
+                                             np.ones(shape.hidden), shape, wl.batch, wl.seq, rnd=True)
+        assert abs(float(off_str.item()) - loss) <= LOSS_RTOL * abs(loss)
+    finally:
+        m_res.close()
+        m_str.close()
 
 
 def test_poisoned_pool_still_equals_resident():
