@@ -118,15 +118,22 @@ __global__ void k_rmsnorm_bwd(const __nv_bfloat16* __restrict__ x, const __nv_bf
 }
 
 // ------------------------------------------------------------------ RoPE
-__global__ void k_rope_tables(float* cos_t, float* sin_t, int seq, int d, double theta) {
+// cos/sin of position p and frequency j, twice: [seq, d/2] (row per position) for
+// k_rope_bwd and [d/2, seq] (row per frequency) for the GEMM epilogue, whose lanes hold
+// consecutive positions.
+__global__ void k_rope_tables(float* cos_t, float* sin_t, float* cos_tt, float* sin_tt, int seq, int d,
+                              double theta) {
   const int half = d / 2;
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= seq * half) return;
   const int p = i / half, j = i % half;
   const double inv = pow(theta, -(2.0 * j) / (double)d);
   const double a = (double)p * inv;
-  cos_t[i] = (float)cos(a);
-  sin_t[i] = (float)sin(a);
+  const float c = (float)cos(a), sn = (float)sin(a);
+  cos_t[i] = c;
+  sin_t[i] = sn;
+  cos_tt[(size_t)j * seq + p] = c;
+  sin_tt[(size_t)j * seq + p] = sn;
 }
 
 // In place: (x1, x2) -> (x1 c + x2 s, x2 c - x1 s), the transpose of the rotation.
@@ -290,8 +297,9 @@ int rmsnorm_bwd(const __nv_bfloat16* x, const __nv_bfloat16* w, const __nv_bfloa
   return NF4LS_OK;
 }
 
-int rope_tables(float* cos_t, float* sin_t, int seq, int d, float theta, cudaStream_t s) {
-  k_rope_tables<<<blocks_for((size_t)seq * d / 2, 256), 256, 0, s>>>(cos_t, sin_t, seq, d, (double)theta);
+int rope_tables(float* cos_t, float* sin_t, float* cos_tt, float* sin_tt, int seq, int d, float theta, cudaStream_t s) {
+  k_rope_tables<<<blocks_for((size_t)seq * d / 2, 256), 256, 0, s>>>(cos_t, sin_t, cos_tt, sin_tt, seq, d,
+                                                                     (double)theta);
   note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;

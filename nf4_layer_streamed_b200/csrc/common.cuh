@@ -281,9 +281,13 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t a, uint32_t rank) {
   return r;
 }
 
-// Arrive (release, cluster scope) on an mbarrier given by its shared::cluster address.
+// Arrive on an mbarrier given by its shared::cluster address (possibly the other CTA's).
+// Release at CTA scope: what the arrival publishes is this thread's own CTA's shared
+// memory, already handed to the async proxy by fence.proxy.async, and CTA scope orders
+// those writes before the arrive.  A cluster-scope release adds a cluster-wide fence
+// on every arrival, which cost the pair GEMMs a quarter of their throughput.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // TMA tile load into this CTA's shared memory whose transaction bytes complete on the

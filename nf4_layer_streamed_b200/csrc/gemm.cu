@@ -120,7 +120,10 @@ __device__ __forceinline__ int find_seg(const GemmParams& p, int row) {
   return s;
 }
 
-__device__ __forceinline__ float silu_f(float x) { return x / (1.0f + expf(-x)); }
+// x * sigmoid(x) and sigmoid(x) with the fast exponential and divide: the results are
+// rounded to bf16, far coarser than either approximation.
+__device__ __forceinline__ float sigmoid_f(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
+__device__ __forceinline__ float silu_f(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
 __device__ __forceinline__ float round_bf16(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
 
 __device__ __forceinline__ void store32(__nv_bfloat16* dst, const float (&v)[32]) {
@@ -189,6 +192,27 @@ __device__ __forceinline__ void load16_bf16(const __nv_bfloat16* src, float (&v)
   }
 }
 
+// Pulls the rows of the epilogue's bf16 side input (the residual, or g and u) that this
+// CTA will read into L2 while the mainloop runs: threads t of nthreads, one 128-byte
+// line per prefetch.  A hint only; nothing waits for it.
+__device__ __forceinline__ void prefetch_aux(const GemmParams& p, int m0, int nt, int t, int nthreads) {
+  if (p.epi != EPI_RESID && p.epi != EPI_DSWIGLU) return;
+  const int col = nt * BN;
+  if (col >= p.N) return;
+  const int span = min(BN, p.N - col) * 2;  // bytes of one row segment
+  const int lines = (span + 127) / 128;
+  const int segs = p.epi == EPI_DSWIGLU ? 2 : 1;
+  const int total = 256 * segs * lines;
+  for (int i = t; i < total; i += nthreads) {
+    const int r = i / (segs * lines), rest = i % (segs * lines);
+    const int m = m0 + r;
+    if (m >= p.M) continue;
+    const int sgi = rest / lines, ln = rest % lines;
+    const char* a = reinterpret_cast<const char*>(p.aux0 + (size_t)m * p.ld_aux0 + col + (sgi ? p.inter : 0)) + ln * 128;
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
+  }
+}
+
 __device__ __forceinline__ void epilogue_rows(const GemmParams& p, uint32_t tmem, int m0, int nt, int q, int lane,
                                               int part = 0, int nparts = 1) {
   constexpr int CW = 16;
@@ -230,12 +254,13 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, uint32_t tmem
             ld_acc16(tb + h * d + i * CW, v);
             ld_acc16(tb + h * d + half + i * CW, w);
             if (!mv) continue;
-            const float* cs = p.rope_cos + (size_t)pos * half + i * CW;
-            const float* sn = p.rope_sin + (size_t)pos * half + i * CW;
+            // frequency-major tables: the 32 lanes (consecutive positions) read one line
+            const float* cs = p.rope_cos + (size_t)(i * CW) * p.seq + pos;
+            const float* sn = p.rope_sin + (size_t)(i * CW) * p.seq + pos;
             float o1[CW], o2[CW];
 #pragma unroll
             for (int j = 0; j < CW; ++j) {
-              const float c_ = cs[j], s_ = sn[j];
+              const float c_ = cs[(size_t)j * p.seq], s_ = sn[(size_t)j * p.seq];
               o1[j] = v[j] * c_ - w[j] * s_;
               o2[j] = w[j] * c_ + v[j] * s_;
             }
@@ -272,7 +297,7 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, uint32_t tmem
           if (!mv) continue;
 #pragma unroll
           for (int i = 0; i < CW; ++i) {
-            const float sg = 1.0f / (1.0f + expf(-g[i]));
+            const float sg = sigmoid_f(g[i]);
             dg[i] = v[i] * u[i] * sg * (1.0f + g[i] * (1.0f - sg));
             du[i] = v[i] * g[i] * sg;
           }
@@ -430,6 +455,7 @@ __global__ void __launch_bounds__(DECODE ? 448 : 192, 1) k_gemm(const __grid_con
   } else if (warp < 6) {
     // ---------------------------------------------------------------- epilogue
     const int q = warp & 3;
+    prefetch_aux(p, m0, nt, threadIdx.x - 64, 128);
     if (mbar_wait(accum_full, 0, abort_flag, p.err, KID_GEMM, 3)) {
       tc_fence_after();
       epilogue_rows(p, tmem, m0, nt, q, lane, 0, DECODE ? 3 : 1);
@@ -546,7 +572,8 @@ constexpr int PC_BYTES = 4096;          // its packed codes
 constexpr int P_STAGE_BYTES = A_BYTES + PB_BYTES + PC_BYTES;
 constexpr int P_SMEM_BYTES = 1024 + P_STAGES * P_STAGE_BYTES + 256 + 1024;
 // Two groups of 4 decoder warps per CTA take alternate k-blocks: each block row of
-// a stage is one thread's work, and a thread has two stages' time to finish it.
+// a stage is one thread's work, and a thread has two stages' time to finish it.  (All
+// 8 warps on every k-block, half a block row each, measured 10-25% slower.)
 constexpr int P_DECODERS = 256;
 constexpr int P_GROUP = 128;
 
@@ -669,6 +696,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DECODE ? 448 : 192, 
       for (int kb = 0; kb < total_kb; ++kb) {
         const int s = kb % P_STAGES;
         const uint32_t ph = (kb / P_STAGES) & 1;
+        // Completes on both CTAs' A/B bytes and on the decoders of both CTAs, whose
+        // tiles sit in their own CTA's shared memory behind fence.proxy.async and a
+        // release arrive; the tensor core reads them after the fence below.
         if (!mbar_wait(&full[s], ph, abort_flag, p.err, KID_GEMM, 12)) break;
         tc_fence_after();
         if (lane == 0) {
@@ -694,6 +724,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DECODE ? 448 : 192, 
   } else if (warp < 6) {
     // ---------------------------------------------------------------- epilogue (both CTAs)
     const int q = warp & 3;
+    prefetch_aux(p, m0, nt, threadIdx.x - 64, 128);
     if (mbar_wait(accum_full, 0, abort_flag, p.err, KID_GEMM, 13)) {
       tc_fence_after();
       epilogue_rows(p, tmem, m0, nt, q, lane, 0, DECODE ? 3 : 1);

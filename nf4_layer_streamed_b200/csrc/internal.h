@@ -91,7 +91,7 @@ struct GemmEpilogue {
   __nv_bfloat16* aux_out = nullptr;     // g,u store of EPI_SWIGLU (may be null)
   int ld_aux_out = 0;
   int inter = 0;                        // I for the SwiGLU layouts
-  const float* rope_cos = nullptr;      // [seq, d/2]
+  const float* rope_cos = nullptr;      // [d/2, seq] (row per frequency)
   const float* rope_sin = nullptr;
   int seq = 0, head_dim = 0, rope_cols = 0;
 };
@@ -136,7 +136,7 @@ int rmsnorm_fwd(const __nv_bfloat16* x, const __nv_bfloat16* w, __nv_bfloat16* y
 // dx = resid + rmsnorm_bwd(x, w, dy); resid may be null.
 int rmsnorm_bwd(const __nv_bfloat16* x, const __nv_bfloat16* w, const __nv_bfloat16* dy,
                 const __nv_bfloat16* resid, __nv_bfloat16* dx, int M, int H, float eps, cudaStream_t s);
-int rope_tables(float* cos_t, float* sin_t, int seq, int d, float theta, cudaStream_t s);
+int rope_tables(float* cos_t, float* sin_t, float* cos_tt, float* sin_tt, int seq, int d, float theta, cudaStream_t s);
 int rope_bwd(__nv_bfloat16* x, int ld, int M, int cols, int seq, int d, const float* cos_t,
              const float* sin_t, cudaStream_t s);
 int attention_fwd(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, int ldq, int ldkv,

@@ -33,7 +33,7 @@ namespace nf4ls {
 namespace {
 
 struct WsLayout {
-  size_t cos, sin, h1, qkv, tpad, bup, adn, o, lse, h, h2, gu, act, dgu, dh2, dh, dO, dqkv, delta, bqt, bvt, part,
+  size_t cos, sin, cos_t, sin_t, h1, qkv, tpad, bup, adn, o, lse, h, h2, gu, act, dgu, dh2, dh, dO, dqkv, delta, bqt, bvt, part,
       dtpad, dh1, dense, total;
 };
 
@@ -49,6 +49,8 @@ WsLayout ws_layout(const nf4ls_layer_cfg* c) {
   };
   L.cos = take((size_t)c->seq * c->head_dim / 2 * 4);
   L.sin = take((size_t)c->seq * c->head_dim / 2 * 4);
+  L.cos_t = take((size_t)c->seq * c->head_dim / 2 * 4);
+  L.sin_t = take((size_t)c->seq * c->head_dim / 2 * 4);
   L.h1 = take(M * H * 2);
   L.qkv = take(M * nqkv * 2);
   L.tpad = take(M * 64 * 2);
@@ -141,7 +143,8 @@ int prepare(LayerCtx& x, const nf4ls_layer_cfg* c, const void* shard, void* ws, 
     x.w_down.n_seg = 1;
     x.w_down.seg[0] = x.v.t[6];
   }
-  return rope_tables(at<float>(ws, x.L.cos), at<float>(ws, x.L.sin), c->seq, c->head_dim, c->rope_theta, s);
+  return rope_tables(at<float>(ws, x.L.cos), at<float>(ws, x.L.sin), at<float>(ws, x.L.cos_t),
+                     at<float>(ws, x.L.sin_t), c->seq, c->head_dim, c->rope_theta, s);
 }
 
 // Forward body up to the SwiGLU activation; y (optional) gets the layer output.
@@ -176,8 +179,8 @@ int forward_body(LayerCtx& x, const nf4ls_lora* lora, const __nv_bfloat16* X, __
   e.kind = EPI_ROPE;
   e.out = qkv;
   e.ldo = x.nqkv;
-  e.rope_cos = at<float>(ws, x.L.cos);
-  e.rope_sin = at<float>(ws, x.L.sin);
+  e.rope_cos = at<float>(ws, x.L.cos_t);
+  e.rope_sin = at<float>(ws, x.L.sin_t);
   e.seq = c->seq;
   e.head_dim = c->head_dim;
   e.rope_cols = x.qd + x.kvd;
