@@ -213,6 +213,15 @@ __device__ __forceinline__ void prefetch_aux(const GemmParams& p, int m0, int nt
   }
 }
 
+__device__ __forceinline__ void unpack16(uint4 a, uint4 b, float (&v)[16]) {
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    v[2 * j] = bf16_lo(w[j]);
+    v[2 * j + 1] = bf16_hi(w[j]);
+  }
+}
+
 __device__ __forceinline__ void epilogue_rows(const GemmParams& p, uint32_t tmem, int m0, int nt, int q, int lane,
                                               int part = 0, int nparts = 1) {
   constexpr int CW = 16;
@@ -251,18 +260,24 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, uint32_t tmem
         if (hc < p.rope_cols) {
           for (int i = 0; i < half / CW; ++i) {
             if ((item++ % nparts) != part) continue;
+            // frequency-major tables: the 32 lanes (consecutive positions) read one line;
+            // the loads are in flight during the TMEM loads
+            const float* cs = p.rope_cos + (size_t)(i * CW) * p.seq + pos;
+            const float* sn = p.rope_sin + (size_t)(i * CW) * p.seq + pos;
+            float c_[CW], s_[CW];
+#pragma unroll
+            for (int j = 0; j < CW; ++j) {
+              c_[j] = cs[(size_t)j * p.seq];
+              s_[j] = sn[(size_t)j * p.seq];
+            }
             ld_acc16(tb + h * d + i * CW, v);
             ld_acc16(tb + h * d + half + i * CW, w);
             if (!mv) continue;
-            // frequency-major tables: the 32 lanes (consecutive positions) read one line
-            const float* cs = p.rope_cos + (size_t)(i * CW) * p.seq + pos;
-            const float* sn = p.rope_sin + (size_t)(i * CW) * p.seq + pos;
             float o1[CW], o2[CW];
 #pragma unroll
             for (int j = 0; j < CW; ++j) {
-              const float c_ = cs[(size_t)j * p.seq], s_ = sn[(size_t)j * p.seq];
-              o1[j] = v[j] * c_ - w[j] * s_;
-              o2[j] = w[j] * c_ + v[j] * s_;
+              o1[j] = v[j] * c_[j] - w[j] * s_[j];
+              o2[j] = w[j] * c_[j] + v[j] * s_[j];
             }
             store16(p.out + (size_t)m * p.ldo + hc + i * CW, o1);
             store16(p.out + (size_t)m * p.ldo + hc + half + i * CW, o2);
@@ -275,39 +290,63 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, uint32_t tmem
           }
         }
       }
-    } else {
+    } else if (p.epi == EPI_STORE) {
       for (int c = 0; c < BN / CW; ++c) {
         const int col = nt * BN + c * CW;
         if (col >= p.N) break;
         if ((item++ % nparts) != part) continue;
-        if (p.epi == EPI_RESID) {
-          if (mv) load16_bf16(p.aux0 + (size_t)m * p.ld_aux0 + col, w);  // in flight during the TMEM load
-          ld_acc16(tb + c * CW, v);
-          if (!mv) continue;
-#pragma unroll
-          for (int i = 0; i < CW; ++i) v[i] += w[i];
-          store16(p.out + (size_t)m * p.ldo + col, v);
-        } else if (p.epi == EPI_DSWIGLU) {
-          float g[CW], u[CW], dg[CW], du[CW];
-          if (mv) {
-            load16_bf16(p.aux0 + (size_t)m * p.ld_aux0 + col, g);
-            load16_bf16(p.aux0 + (size_t)m * p.ld_aux0 + p.inter + col, u);
-          }
-          ld_acc16(tb + c * CW, v);
-          if (!mv) continue;
-#pragma unroll
-          for (int i = 0; i < CW; ++i) {
-            const float sg = sigmoid_f(g[i]);
-            dg[i] = v[i] * u[i] * sg * (1.0f + g[i] * (1.0f - sg));
-            du[i] = v[i] * g[i] * sg;
-          }
-          store16(p.out + (size_t)m * p.ldo + col, dg);
-          store16(p.out + (size_t)m * p.ldo + p.inter + col, du);
-        } else {
-          ld_acc16(tb + c * CW, v);
-          if (mv) store16(p.out + (size_t)m * p.ldo + col, v);
-        }
+        ld_acc16(tb + c * CW, v);
+        if (mv) store16(p.out + (size_t)m * p.ldo + col, v);
       }
+    }
+  }
+  if (p.epi != EPI_RESID && p.epi != EPI_DSWIGLU) return;
+  // Residual / dSwiGLU: this warp's items k = part, part + nparts, ... over both
+  // accumulators (item k: accumulator k / nch, chunk k % nch), with the bf16 side input
+  // of the next item loaded while the current one is processed.
+  const int nch = min(BN, p.N - nt * BN) / CW;
+  const int total = 2 * nch;
+  const bool dsw = p.epi == EPI_DSWIGLU;
+  uint4 nx[4];
+  auto load_side = [&](int k) {
+    const int a = k / nch, c = k - a * nch;
+    const int m = m0 + a * 128 + q * 32 + lane;
+    if (m >= p.M) return;
+    const uint4* src = reinterpret_cast<const uint4*>(p.aux0 + (size_t)m * p.ld_aux0 + nt * BN + c * CW);
+    nx[0] = src[0];
+    nx[1] = src[1];
+    if (dsw) {
+      const uint4* su = reinterpret_cast<const uint4*>(p.aux0 + (size_t)m * p.ld_aux0 + p.inter + nt * BN + c * CW);
+      nx[2] = su[0];
+      nx[3] = su[1];
+    }
+  };
+  if (part < total) load_side(part);
+  for (int k = part; k < total; k += nparts) {
+    const uint4 cur[4] = {nx[0], nx[1], nx[2], nx[3]};
+    if (k + nparts < total) load_side(k + nparts);
+    const int a = k / nch, c = k - a * nch;
+    const int m = m0 + a * 128 + q * 32 + lane;
+    const int col = nt * BN + c * CW;
+    float v[CW], g[CW];
+    ld_acc16(tmem + ((uint32_t)(q * 32) << 16) + a * 256 + c * CW, v);
+    if (m >= p.M) continue;
+    unpack16(cur[0], cur[1], g);
+    if (!dsw) {
+#pragma unroll
+      for (int i = 0; i < CW; ++i) v[i] += g[i];
+      store16(p.out + (size_t)m * p.ldo + col, v);
+    } else {
+      float u[CW], du[CW];
+      unpack16(cur[2], cur[3], u);
+#pragma unroll
+      for (int i = 0; i < CW; ++i) {
+        const float sg = sigmoid_f(g[i]);
+        du[i] = v[i] * g[i] * sg;
+        v[i] = v[i] * u[i] * sg * (1.0f + g[i] * (1.0f - sg));
+      }
+      store16(p.out + (size_t)m * p.ldo + col, v);
+      store16(p.out + (size_t)m * p.ldo + p.inter + col, du);
     }
   }
 }
