@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=128)
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the resident (compute-only) timing and the batch-16 compute-bound point")
     return ap.parse_args()
 
 
@@ -177,6 +179,59 @@ def run_reference(args, wl):
 
 
 # ----------------------------------------------------------------------------- ours
+def time_steps(m, ids, warmup: int, steps: int) -> float:
+    """ms per training step of model m (CUDA events on the current stream)."""
+    import torch
+    for i in range(warmup):
+        m.train_step(ids[i % len(ids)])
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(steps):
+        m.train_step(ids[(warmup + i) % len(ids)])
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / steps
+
+
+def extra_points(args, wl, ms_step: float, copy_ms: float) -> dict:
+    """Single-GPU context for the headline: the same steps with every shard resident in
+    HBM (compute only), the copy/compute overlap, and the batch-16 point where the step
+    is compute-bound."""
+    import torch
+
+    from nf4_layer_streamed_b200 import api, dp, synth
+    out = {}
+    ids = [dp.rank_token_ids(wl, 0, s) for s in range(4)]
+    m = api.StreamedModel(wl, resident=True)
+    t_comp = time_steps(m, ids, 2, max(3, args.steps // 2))
+    m.close()
+    del m
+    out["resident"] = {"ms_per_step": t_comp, "tokens_per_s": wl.tokens / (t_comp / 1000.0)}
+    if copy_ms:
+        out["overlap"] = {"t_copy_ms": copy_ms, "t_compute_ms": t_comp, "t_step_ms": ms_step,
+                          "value": (copy_ms + t_comp - ms_step) / min(copy_ms, t_comp),
+                          "definition": "(T_copy + T_compute - T_step) / min(T_copy, T_compute)"}
+    wl16 = synth.WORKLOADS["llama8b_32L_b16s512"]
+    ids16 = [dp.rank_token_ids(wl16, 0, s) for s in range(3)]
+    m = api.StreamedModel(wl16, depth=args.depth)
+    t16 = time_steps(m, ids16, 1, 2)
+    api.profile(True)
+    api.profile_reset()
+    m.train_step(ids16[0])
+    torch.cuda.synchronize()
+    api.profile(False)
+    r = api.profile_read(1)
+    api.profile_reset()
+    m.close()
+    del m
+    out["batch16"] = {"workload": wl16.name, "ms_per_step": t16, "tokens_per_s": wl16.tokens / (t16 / 1000.0),
+                      "nf4_gemm_tflops": r["flops"] / (r["ms"] / 1000.0) / 1e12 if r["ms"] else None,
+                      "note": "out-of-config point (batch 16 x 512), streamed at the same depth"}
+    torch.cuda.empty_cache()
+    return out
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -323,6 +378,10 @@ def main():
                           f"on {args.cpu_sample_tokens} tokens ({tl:.2f} s + {th:.2f} s), scaled to "
                           f"{wl.n_layers} layers")}
 
+    extra = None
+    if rank == 0 and world == 1 and not args.no_extra:
+        extra = extra_points(args, wl, ms_max, copy_bytes / best / 1e6 if best else 0.0)
+
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -347,6 +406,7 @@ def main():
                        "copy_ms_per_step_at_link_rate": copy_bytes / best / 1e6 if best else None,
                        "copies_per_step": (st1["copies"] - st0["copies"]) / args.steps},
             "breakdown": breakdown,
+            "single_gpu_context": extra,
             "loss_last": loss,
             "gpu_launches": int(launches),
             "clocks": ck,

@@ -175,57 +175,110 @@ __global__ void k_embed(const int32_t* __restrict__ ids, const __nv_bfloat16* __
 // dlogits = (softmax - onehot) * inv_count, for rows with a target (t < seq-1);
 // other rows get zero loss and zero gradient.
 // logits and dlogits may be the same buffer (the gradient overwrites the logits).
+// One row of logits per block: an online (max, sum of exp) pass, then the gradient pass
+// (softmax - onehot) / count in place of the logits.  Rows are read 8 bf16 at a time
+// when V % 8 == 0 (every row then starts 16-byte aligned); the reductions run in a fixed
+// order (each thread's sequential chunks, then a fixed tree), so reruns are bit-exact.
+__device__ __forceinline__ void online_add(float& m, float& s, float x) {
+  if (x > m) {
+    s = s * expf(m - x) + 1.0f;
+    m = x;
+  } else {
+    s += expf(x - m);
+  }
+}
+
+__device__ __forceinline__ void online_merge(float& m, float& s, float m2, float s2) {
+  if (m2 > m) {
+    s = s * expf(m - m2) + s2;
+    m = m2;
+  } else if (m2 > -INFINITY) {
+    s += s2 * expf(m2 - m);
+  }
+}
+
 __global__ void __launch_bounds__(256) k_ce(const __nv_bfloat16* logits, const int32_t* __restrict__ ids, int V,
                                             int seq, float inv_count, float* __restrict__ row_loss,
                                             __nv_bfloat16* dlogits) {
-  __shared__ float red[8];
-  __shared__ float bval[2];
+  __shared__ float red_m[8], red_s[8];
+  __shared__ float bval[3];
   const int m = blockIdx.x;
   const int t = threadIdx.x, lane = t & 31, wid = t >> 5;
   const __nv_bfloat16* row = logits + (size_t)m * V;
   __nv_bfloat16* drow = dlogits + (size_t)m * V;
+  const bool vec = (V & 7) == 0;
+  const int nv = vec ? V >> 3 : 0;  // 16-byte chunks
   const bool has_target = (m % seq) != seq - 1;
   if (!has_target) {
-    for (int j = t; j < V; j += blockDim.x) drow[j] = __float2bfloat16_rn(0.f);
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    for (int j = t; j < nv; j += blockDim.x) reinterpret_cast<uint4*>(drow)[j] = z;
+    for (int j = nv * 8 + t; j < V; j += blockDim.x) drow[j] = __float2bfloat16_rn(0.f);
     if (t == 0) row_loss[m] = 0.f;
     return;
   }
   const int tgt = ids[m + 1];
-  float mx = -INFINITY;
-  for (int j = t; j < V; j += blockDim.x) mx = fmaxf(mx, __bfloat162float(row[j]));
-  mx = warp_max(mx);
-  if (lane == 0) red[wid] = mx;
+  float mx = -INFINITY, sm = 0.f;
+  for (int j = t; j < nv; j += blockDim.x) {
+    const uint4 u = reinterpret_cast<const uint4*>(row)[j];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    float x[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      x[2 * k] = __uint_as_float(w[k] << 16);
+      x[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+    }
+    float cm = x[0];
+#pragma unroll
+    for (int k = 1; k < 8; ++k) cm = fmaxf(cm, x[k]);
+    float cs = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) cs += expf(x[k] - cm);
+    online_merge(mx, sm, cm, cs);
+  }
+  for (int j = nv * 8 + t; j < V; j += blockDim.x) online_add(mx, sm, __bfloat162float(row[j]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, mx, o), s2 = __shfl_xor_sync(0xffffffffu, sm, o);
+    online_merge(mx, sm, m2, s2);
+  }
+  if (lane == 0) {
+    red_m[wid] = mx;
+    red_s[wid] = sm;
+  }
   __syncthreads();
   if (t == 0) {
-    float v = red[0];
-    for (int i = 1; i < 8; ++i) v = fmaxf(v, red[i]);
-    bval[0] = v;
+    float a = red_m[0], b = red_s[0];
+    for (int i = 1; i < 8; ++i) online_merge(a, b, red_m[i], red_s[i]);
+    bval[0] = a;
+    bval[1] = b;
+    bval[2] = __bfloat162float(row[tgt]);  // read before the row is overwritten in place
   }
   __syncthreads();
   mx = bval[0];
-  float s = 0.f;
-  for (int j = t; j < V; j += blockDim.x) s += expf(__bfloat162float(row[j]) - mx);
-  s = warp_sum(s);
-  __syncthreads();
-  if (lane == 0) red[wid] = s;
-  __syncthreads();
-  if (t == 0) {
-    float v = 0.f;
-    for (int i = 0; i < 8; ++i) v += red[i];
-    bval[1] = v;
-  }
-  __syncthreads();
   const float sum = bval[1];
   const float lse = mx + logf(sum);
-  const float inv_sum = 1.0f / sum;
-  const float lt = __bfloat162float(row[tgt]);  // read before the row may be overwritten in place
-  __syncthreads();
-  for (int j = t; j < V; j += blockDim.x) {
-    float p = expf(__bfloat162float(row[j]) - mx) * inv_sum;
-    if (j == tgt) p -= 1.0f;
-    drow[j] = __float2bfloat16_rn(p * inv_count);
+  const float scale = inv_count / sum;
+  for (int j = t; j < nv; j += blockDim.x) {
+    const uint4 u = reinterpret_cast<const uint4*>(row)[j];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float p0 = expf(__uint_as_float(w[k] << 16) - mx) * scale;
+      float p1 = expf(__uint_as_float(w[k] & 0xFFFF0000u) - mx) * scale;
+      const int e = j * 8 + 2 * k;
+      if (e == tgt) p0 -= inv_count;
+      if (e + 1 == tgt) p1 -= inv_count;
+      o[k] = pack_bf16x2(p0, p1);
+    }
+    reinterpret_cast<uint4*>(drow)[j] = make_uint4(o[0], o[1], o[2], o[3]);
   }
-  if (t == 0) row_loss[m] = lse - lt;
+  for (int j = nv * 8 + t; j < V; j += blockDim.x) {
+    float p = expf(__bfloat162float(row[j]) - mx) * scale;
+    if (j == tgt) p -= inv_count;
+    drow[j] = __float2bfloat16_rn(p);
+  }
+  if (t == 0) row_loss[m] = lse - bval[2];
 }
 
 // Deterministic mean: one block sums n values in a fixed pattern, then scales.

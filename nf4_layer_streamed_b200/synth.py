@@ -93,6 +93,9 @@ WORKLOADS = {
     "llama8b_32L_b4s512": Workload("llama8b_32L_b4s512", LLAMA_8B, 32, 4, 512,
                                     vocab=128256, tied=False, steps=10),
     "qwen32b_4L_b1s1024": Workload("qwen32b_4L_b1s1024", QWEN_32B_CLASS, 4, 1, 1024),
+    # out-of-config point: the same stack at batch 16, where the step is compute-bound
+    "llama8b_32L_b16s512": Workload("llama8b_32L_b16s512", LLAMA_8B, 32, 16, 512,
+                                     vocab=128256, tied=False, steps=3),
 }
 
 
