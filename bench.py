@@ -212,6 +212,23 @@ def extra_points(args, wl, ms_step: float, copy_ms: float) -> dict:
         out["overlap"] = {"t_copy_ms": copy_ms, "t_compute_ms": t_comp, "t_step_ms": ms_step,
                           "value": (copy_ms + t_comp - ms_step) / min(copy_ms, t_comp),
                           "definition": "(T_copy + T_compute - T_step) / min(T_copy, T_compute)"}
+    # streamed head: embedding and lm_head in pinned host memory, lm_head in 16384-row chunks
+    m = api.StreamedModel(wl, depth=args.depth, head_chunk_rows=16384)
+    t_sh = time_steps(m, ids, 2, 3)
+    api.profile(True)
+    api.profile_reset()
+    m.train_step(ids[0])
+    torch.cuda.synchronize()
+    api.profile(False)
+    head_ms = api.profile_read(2001)["ms"] + api.profile_read(2002)["ms"]
+    api.profile_reset()
+    m.close()
+    del m
+    out["streamed_head"] = {"ms_per_step": t_sh, "tokens_per_s": wl.tokens / (t_sh / 1000.0),
+                            "head_ms_per_step": head_ms, "head_chunk_rows": 16384,
+                            "hbm_bytes_saved": 2 * wl.vocab * wl.shape.hidden * 2,
+                            "note": "lm_head and embedding stay in pinned host memory; one pass over the "
+                                    "vocab chunks gives loss and dL/dh"}
     wl16 = synth.WORKLOADS["llama8b_32L_b16s512"]
     ids16 = [dp.rank_token_ids(wl16, 0, s) for s in range(3)]
     m = api.StreamedModel(wl16, depth=args.depth)

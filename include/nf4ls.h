@@ -326,6 +326,16 @@ typedef struct {
     int32_t vocab;
     int32_t tied;            /* 1: lm_head is the embedding table      */
     float lr, beta1, beta2, adam_eps, weight_decay;
+    /* 0: embedding and lm_head resident in HBM (embed_dev, lm_head_dev).
+     * > 0: the streamed head ([gate] §4.3 lists streaming the unquantised embedding and
+     * lm_head "as a large layer" as the next step): the output matrix (lm_head, or the
+     * embedding when tied) is read in vocab chunks of head_chunk_rows rows (a multiple
+     * of 64) through head_pool, and the embedding rows of the batch are gathered from
+     * embed_host when embed_dev is NULL.  The loss and dL/dh come from one pass over
+     * the chunks: per row a running max and sum of exp, and the sum of
+     * exp(logit - max) * lm_head row rescaled whenever the max grows, so the [M, V]
+     * logits are never stored. */
+    int32_t head_chunk_rows;
 } nf4ls_model_cfg;
 
 typedef struct {
@@ -340,6 +350,11 @@ typedef struct {
     const void* const* shards_dev;/* ... resident shard pointers        */
     void* ws_dev;
     size_t ws_bytes;
+    /* streamed head only (head_chunk_rows > 0), else NULL: */
+    nf4ls_pool* head_pool;        /* layer i = bf16 rows [i c, min(V, (i+1) c)) x H of
+                                     the output matrix, c = head_chunk_rows            */
+    const void* embed_host;       /* bf16 [V, H] in pinned host memory the device can
+                                     read (mapped), used when embed_dev is NULL         */
 } nf4ls_model;
 
 size_t nf4ls_lora_stride(const nf4ls_layer_cfg* cfg);

@@ -300,11 +300,14 @@ class StreamedModel:
     the step workspace.  Quantisation runs through nf4_quantize_shard on the GPU."""
 
     def __init__(self, wl: Workload, depth: int = 2, resident: bool = False, b_random: bool = False,
-                 train: TrainConfig = TrainConfig(), device="cuda", weights_device=None, fingerprint: int = 1234):
+                 train: TrainConfig = TrainConfig(), device="cuda", weights_device=None, fingerprint: int = 1234,
+                 head_chunk_rows: int = 0):
+        """head_chunk_rows > 0: the embedding and lm_head stay in pinned host memory; the
+        output matrix streams through a depth-2 pool in chunks of that many vocab rows."""
         self.wl = wl
         shape = wl.shape
         self.cfg = B.ModelCfg(layer_cfg(shape, wl.batch, wl.seq), wl.n_layers, wl.vocab, int(wl.tied), train.lr,
-                              train.beta1, train.beta2, train.eps, train.weight_decay)
+                              train.beta1, train.beta2, train.eps, train.weight_decay, head_chunk_rows)
         lc = self.cfg.layer
         from . import synth
         wdev = weights_device or device
@@ -337,8 +340,21 @@ class StreamedModel:
         else:
             offs = [i * self.slot_bytes for i in range(L)]
             self.pool = Pool(self.store, offs, [self.shard_nbytes] * L, depth, self.slot_bytes, device)
-        self.embed = synth.embedding(wl.vocab, shape.hidden, wl.seed, 0, device=wdev).to(device)
-        self.lm_head = None if wl.tied else synth.embedding(wl.vocab, shape.hidden, wl.seed, 1, device=wdev).to(device)
+        self.head_pool = None
+        if head_chunk_rows > 0:
+            self.embed = synth.embedding(wl.vocab, shape.hidden, wl.seed, 0, device=wdev).cpu().pin_memory()
+            self.lm_head = None if wl.tied else \
+                synth.embedding(wl.vocab, shape.hidden, wl.seed, 1, device=wdev).cpu().pin_memory()
+            out = self.embed if wl.tied else self.lm_head
+            row_bytes = shape.hidden * 2
+            n_chunks = (wl.vocab + head_chunk_rows - 1) // head_chunk_rows
+            offs = [i * head_chunk_rows * row_bytes for i in range(n_chunks)]
+            sizes = [min(head_chunk_rows, wl.vocab - i * head_chunk_rows) * row_bytes for i in range(n_chunks)]
+            self.head_pool = Pool(out, offs, sizes, 2, None, device)
+        else:
+            self.embed = synth.embedding(wl.vocab, shape.hidden, wl.seed, 0, device=wdev).to(device)
+            self.lm_head = None if wl.tied else \
+                synth.embedding(wl.vocab, shape.hidden, wl.seed, 1, device=wdev).to(device)
         self.norm_final = torch.ones(shape.hidden, dtype=torch.bfloat16, device=device)
         self.stride = B.lib().nf4ls_lora_stride(ctypes.byref(lc))
         self.lora = torch.zeros(L * self.stride, dtype=torch.float32, device=device)
@@ -353,12 +369,16 @@ class StreamedModel:
         self.ws_bytes = B.lib().nf4ls_model_workspace_bytes(ctypes.byref(self.cfg))
         self.ws = _buffer(self.ws_bytes, device)
         self.loss = torch.zeros(1, dtype=torch.float32, device=device)
-        self.model = B.Model(self.embed.data_ptr(), 0 if self.lm_head is None else self.lm_head.data_ptr(),
+        streamed = self.head_pool is not None
+        self.model = B.Model(None if streamed else self.embed.data_ptr(),
+                             None if (streamed or self.lm_head is None) else self.lm_head.data_ptr(),
                              self.norm_final.data_ptr(), self.lora.data_ptr(), self.grads.data_ptr(),
                              self.adam_m.data_ptr(), self.adam_v.data_ptr(),
                              self.pool.handle.value if self.pool else None,
                              ctypes.cast(self.shard_ptrs, ctypes.c_void_p) if resident else None,
-                             self.ws.data_ptr(), self.ws_bytes)
+                             self.ws.data_ptr(), self.ws_bytes,
+                             self.head_pool.handle.value if streamed else None,
+                             self.embed.data_ptr() if streamed else None)
         self.step_count = 0
 
     def lora_views(self, layer: int) -> dict:
@@ -403,3 +423,6 @@ class StreamedModel:
         if self.pool is not None:
             self.pool.destroy()
             self.pool = None
+        if self.head_pool is not None:
+            self.head_pool.destroy()
+            self.head_pool = None

@@ -44,7 +44,8 @@ class LoraGrads(ctypes.Structure):
 class ModelCfg(ctypes.Structure):
     _fields_ = [("layer", LayerCfg), ("n_layers", ctypes.c_int32), ("vocab", ctypes.c_int32),
                 ("tied", ctypes.c_int32), ("lr", ctypes.c_float), ("beta1", ctypes.c_float),
-                ("beta2", ctypes.c_float), ("adam_eps", ctypes.c_float), ("weight_decay", ctypes.c_float)]
+                ("beta2", ctypes.c_float), ("adam_eps", ctypes.c_float), ("weight_decay", ctypes.c_float),
+                ("head_chunk_rows", ctypes.c_int32)]
 
 
 class Model(ctypes.Structure):
@@ -52,7 +53,8 @@ class Model(ctypes.Structure):
                 ("norm_final_dev", ctypes.c_void_p), ("lora_dev", ctypes.c_void_p),
                 ("grads_dev", ctypes.c_void_p), ("adam_m_dev", ctypes.c_void_p),
                 ("adam_v_dev", ctypes.c_void_p), ("pool", ctypes.c_void_p),
-                ("shards_dev", ctypes.c_void_p), ("ws_dev", ctypes.c_void_p), ("ws_bytes", ctypes.c_size_t)]
+                ("shards_dev", ctypes.c_void_p), ("ws_dev", ctypes.c_void_p), ("ws_bytes", ctypes.c_size_t),
+                ("head_pool", ctypes.c_void_p), ("embed_host", ctypes.c_void_p)]
 
 
 class PoolStats(ctypes.Structure):

@@ -281,6 +281,114 @@ __global__ void __launch_bounds__(256) k_ce(const __nv_bfloat16* logits, const i
   if (t == 0) row_loss[m] = lse - bval[2];
 }
 
+// ------------------------------------------------------------------ streamed head
+// One block per row of a vocab chunk; see ce_chunk in internal.h.
+__global__ void __launch_bounds__(256) k_ce_chunk(__nv_bfloat16* logits, int n, int v0,
+                                                  const __nv_bfloat16* __restrict__ Wc,
+                                                  const int32_t* __restrict__ ids, int H, int seq, int first,
+                                                  float* __restrict__ mx, float* __restrict__ sm,
+                                                  float* __restrict__ alpha, float* __restrict__ lt,
+                                                  __nv_bfloat16* __restrict__ wt) {
+  __shared__ float red[8];
+  __shared__ float bval;
+  const int m = blockIdx.x;
+  const int t = threadIdx.x, lane = t & 31, wid = t >> 5;
+  __nv_bfloat16* row = logits + (size_t)m * n;
+  const int nv = n >> 3;  // n % 64 == 0
+  if ((m % seq) == seq - 1) {  // no target: P = 0 keeps this row of the sum at 0
+    for (int j = t; j < nv; j += blockDim.x) reinterpret_cast<uint4*>(row)[j] = make_uint4(0u, 0u, 0u, 0u);
+    if (t == 0) {
+      alpha[m] = 1.0f;
+      if (first) {
+        mx[m] = 0.0f;
+        sm[m] = 1.0f;
+        lt[m] = 0.0f;
+      }
+    }
+    return;
+  }
+  const int tgt = ids[m + 1] - v0;
+  if (tgt >= 0 && tgt < n) {
+    if (t == 0) lt[m] = __bfloat162float(row[tgt]);  // before the row is overwritten
+    const uint4* src = reinterpret_cast<const uint4*>(Wc + (size_t)tgt * H);
+    uint4* dst = reinterpret_cast<uint4*>(wt + (size_t)m * H);
+    for (int j = t; j < H / 8; j += blockDim.x) dst[j] = src[j];
+  }
+  float cm = -INFINITY;
+  for (int j = t; j < nv; j += blockDim.x) {
+    const uint4 u = reinterpret_cast<const uint4*>(row)[j];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      cm = fmaxf(cm, fmaxf(__uint_as_float(w[k] << 16), __uint_as_float(w[k] & 0xFFFF0000u)));
+  }
+  cm = warp_max(cm);
+  if (lane == 0) red[wid] = cm;
+  __syncthreads();
+  if (t == 0) {
+    float v = red[0];
+    for (int i = 1; i < 8; ++i) v = fmaxf(v, red[i]);
+    const float old = first ? -INFINITY : mx[m];
+    bval = fmaxf(old, v);
+  }
+  __syncthreads();
+  const float mnew = bval;
+  float ssum = 0.f;
+  for (int j = t; j < nv; j += blockDim.x) {
+    const uint4 u = reinterpret_cast<const uint4*>(row)[j];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float p0 = expf(__uint_as_float(w[k] << 16) - mnew);
+      const float p1 = expf(__uint_as_float(w[k] & 0xFFFF0000u) - mnew);
+      ssum += p0 + p1;
+      o[k] = pack_bf16x2(p0, p1);
+    }
+    reinterpret_cast<uint4*>(row)[j] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  ssum = warp_sum(ssum);
+  __syncthreads();
+  if (lane == 0) red[wid] = ssum;
+  __syncthreads();
+  if (t == 0) {
+    float v = 0.f;
+    for (int i = 0; i < 8; ++i) v += red[i];
+    if (first) {
+      sm[m] = v;
+      alpha[m] = 0.0f;
+    } else {
+      const float a = expf(mx[m] - mnew);
+      sm[m] = sm[m] * a + v;
+      alpha[m] = a;
+    }
+    mx[m] = mnew;
+  }
+}
+
+__global__ void __launch_bounds__(256) k_ce_finish(const float* __restrict__ mx, const float* __restrict__ sm,
+                                                   const float* __restrict__ lt, const float* __restrict__ acc,
+                                                   const __nv_bfloat16* __restrict__ wt, int H, int seq,
+                                                   float inv_count, float* __restrict__ row_loss,
+                                                   __nv_bfloat16* __restrict__ dh) {
+  const int m = blockIdx.x, t = threadIdx.x;
+  const bool has_target = (m % seq) != seq - 1;
+  if (t == 0) row_loss[m] = has_target ? mx[m] + logf(sm[m]) - lt[m] : 0.0f;
+  if (!acc) return;
+  const float inv_s = has_target ? 1.0f / sm[m] : 0.0f;
+  const float wscale = has_target ? inv_count : 0.0f;
+  const float4* a = reinterpret_cast<const float4*>(acc + (size_t)m * H);
+  const uint2* w = reinterpret_cast<const uint2*>(wt + (size_t)m * H);
+  uint2* d = reinterpret_cast<uint2*>(dh + (size_t)m * H);
+  for (int j = t; j < H / 4; j += blockDim.x) {
+    const float4 v = a[j];
+    const uint2 ww = has_target ? w[j] : make_uint2(0u, 0u);
+    const float r0 = (v.x * inv_s - bf16_lo(ww.x)) * wscale, r1 = (v.y * inv_s - bf16_hi(ww.x)) * wscale;
+    const float r2 = (v.z * inv_s - bf16_lo(ww.y)) * wscale, r3 = (v.w * inv_s - bf16_hi(ww.y)) * wscale;
+    d[j] = make_uint2(pack_bf16x2(r0, r1), pack_bf16x2(r2, r3));
+  }
+}
+
 // Deterministic mean: one block sums n values in a fixed pattern, then scales.
 __global__ void k_sum_scale(const float* __restrict__ v, int n, float scale, float* __restrict__ out) {
   __shared__ double red[256];
@@ -384,6 +492,26 @@ int cross_entropy(const __nv_bfloat16* logits, const int32_t* ids, int M, int V,
                   __nv_bfloat16* dlogits, float* loss, cudaStream_t s) {
   const int count = batch * (seq - 1);
   k_ce<<<M, 256, 0, s>>>(logits, ids, V, seq, 1.0f / (float)count, row_loss, dlogits);
+  note_launch();
+  k_sum_scale<<<1, 256, 0, s>>>(row_loss, M, 1.0f / (float)count, loss);
+  note_launch();
+  NF4_CUDA_TRY(cudaGetLastError());
+  return NF4LS_OK;
+}
+
+int ce_chunk(__nv_bfloat16* logits, int n, int v0, const __nv_bfloat16* Wc, const int32_t* ids, int M, int H,
+             int seq, int first, float* mx, float* sm, float* alpha, float* lt, __nv_bfloat16* wt, cudaStream_t s) {
+  if (n % 64 || H % 8) return fail(NF4LS_SHAPE, "ce_chunk: chunk rows %% 64 and H %% 8");
+  k_ce_chunk<<<M, 256, 0, s>>>(logits, n, v0, Wc, ids, H, seq, first, mx, sm, alpha, lt, wt);
+  note_launch();
+  NF4_CUDA_TRY(cudaGetLastError());
+  return NF4LS_OK;
+}
+
+int ce_finish(const float* mx, const float* sm, const float* lt, const float* acc, const __nv_bfloat16* wt, int M,
+              int H, int batch, int seq, float* row_loss, float* loss, __nv_bfloat16* dh, cudaStream_t s) {
+  const int count = batch * (seq - 1);
+  k_ce_finish<<<M, 256, 0, s>>>(mx, sm, lt, acc, wt, H, seq, 1.0f / (float)count, row_loss, dh);
   note_launch();
   k_sum_scale<<<1, 256, 0, s>>>(row_loss, M, 1.0f / (float)count, loss);
   note_launch();

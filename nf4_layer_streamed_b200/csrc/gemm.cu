@@ -71,6 +71,9 @@ struct GemmParams {
   const float* rope_cos;
   const float* rope_sin;
   int seq, head_dim, rope_cols;
+  float* out_f32;
+  const float* alpha;
+  int accumulate;
   float nf4[16];
   float code8[256];
   int* err;
@@ -297,6 +300,32 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, uint32_t tmem
         if ((item++ % nparts) != part) continue;
         ld_acc16(tb + c * CW, v);
         if (mv) store16(p.out + (size_t)m * p.ldo + col, v);
+      }
+    } else if (p.epi == EPI_ACC_F32) {
+      for (int c = 0; c < BN / CW; ++c) {
+        const int col = nt * BN + c * CW;
+        if (col >= p.N) break;
+        if ((item++ % nparts) != part) continue;
+        float4* dst = reinterpret_cast<float4*>(p.out_f32 + (size_t)m * p.ldo + col);
+        float4 old[CW / 4];
+        if (mv && p.accumulate) {
+#pragma unroll
+          for (int i = 0; i < CW / 4; ++i) old[i] = dst[i];
+        }
+        ld_acc16(tb + c * CW, v);
+        if (!mv) continue;
+        if (p.accumulate) {
+          const float al = p.alpha[m];
+#pragma unroll
+          for (int i = 0; i < CW / 4; ++i) {
+            v[4 * i + 0] += al * old[i].x;
+            v[4 * i + 1] += al * old[i].y;
+            v[4 * i + 2] += al * old[i].z;
+            v[4 * i + 3] += al * old[i].w;
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < CW / 4; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
       }
     }
   }
@@ -935,7 +964,8 @@ int launch_pair(const GemmParams& p, int grid, cudaStream_t s) {
 
 int gemm(const __nv_bfloat16* A, int lda, int M, int N, int K, const GemmWeights& W, bool dgrad,
          const GemmExtra& extra, const GemmEpilogue& epi, cudaStream_t s) {
-  if (!A || !epi.out) return fail(NF4LS_INVALID_ARG, "gemm: null operand");
+  if (!A || (epi.kind == EPI_ACC_F32 ? !epi.out_f32 || (epi.accumulate && !epi.alpha) : !epi.out))
+    return fail(NF4LS_INVALID_ARG, "gemm: null operand");
   if (M <= 0 || N <= 0 || K <= 0 || K % 64 || N % 64) return fail(NF4LS_SHAPE, "gemm: M=%d N=%d K=%d (K, N % 64)", M, N, K);
   const bool decode = W.dense == nullptr;
   const bool swiglu = epi.kind == EPI_SWIGLU;
@@ -1021,6 +1051,11 @@ int gemm(const __nv_bfloat16* A, int lda, int M, int N, int K, const GemmWeights
   p.seq = epi.seq;
   p.head_dim = epi.head_dim;
   p.rope_cols = epi.rope_cols;
+  p.out_f32 = epi.out_f32;
+  p.alpha = epi.alpha;
+  p.accumulate = epi.accumulate;
+  if (epi.kind == EPI_ACC_F32 && (epi.ldo % 4 || !aligned(epi.out_f32, 16)))
+    return fail(NF4LS_ALIGN, "gemm: fp32 output needs 16-byte rows");
   p.err = device_error_ptr();
   const int grid = p.n_mt * n_nt * (pair ? 2 : 1);
   cudaEvent_t e0 = nullptr;

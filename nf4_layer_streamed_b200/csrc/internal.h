@@ -80,6 +80,7 @@ enum Epilogue : int {
   EPI_ROPE = 2,     // out = rope(acc) on columns < rope_cols, acc elsewhere
   EPI_SWIGLU = 3,   // columns [0,128) gate, [128,256) up of block i: out[m, i] = silu(g) * u; aux_out g,u
   EPI_DSWIGLU = 4,  // acc = da[m, i]; aux0 = [g | u] -> out = [dg | du]
+  EPI_ACC_F32 = 5,  // out_f32[m, n] = acc + (accumulate ? alpha[m] * out_f32[m, n] : 0)
 };
 
 struct GemmEpilogue {
@@ -94,6 +95,9 @@ struct GemmEpilogue {
   const float* rope_cos = nullptr;      // [d/2, seq] (row per frequency)
   const float* rope_sin = nullptr;
   int seq = 0, head_dim = 0, rope_cols = 0;
+  float* out_f32 = nullptr;             // EPI_ACC_F32 output (and input when accumulate)
+  const float* alpha = nullptr;         // EPI_ACC_F32 per-row scale of the old value
+  int accumulate = 0;
 };
 
 // Weights of a GEMM: either one dense bf16 matrix, or up to four NF4 tensors that
@@ -157,6 +161,18 @@ int lora_cols(const __nv_bfloat16* X, int ldx, int xcol, int N, int M, const __n
               int NR, float scale, float* part, float* out0, float* out1, int so_n, int so_r, cudaStream_t s);
 int zero_cols(__nv_bfloat16* x, int ld, int M, int c0, int c1, cudaStream_t s);
 int embed(const int32_t* ids, const __nv_bfloat16* E, __nv_bfloat16* h, int M, int H, cudaStream_t s);
+// Streamed head, per vocab chunk [v0, v0 + n) of the output matrix (rows Wc in HBM):
+// logits [M, n] (bf16, from the GEMM) are folded into the per-row running max mx, sum
+// sm (first chunk: first = 1 starts them) and overwritten in place by
+// P = bf16(exp(logit - mx_new)); alpha[m] = exp(mx_old - mx_new) rescales the running
+// sum of P Wc (the next GEMM's EPI_ACC_F32).  A row whose target id falls in the chunk
+// records the target logit and copies that row of Wc into wt.
+int ce_chunk(__nv_bfloat16* logits, int n, int v0, const __nv_bfloat16* Wc, const int32_t* ids, int M, int H,
+             int seq, int first, float* mx, float* sm, float* alpha, float* lt, __nv_bfloat16* wt, cudaStream_t s);
+// After the last chunk: per-row loss mx + log(sm) - lt (0 for rows without a target),
+// the mean into loss, and (acc != null) dh = bf16((acc / sm - wt) / count).
+int ce_finish(const float* mx, const float* sm, const float* lt, const float* acc, const __nv_bfloat16* wt,
+              int M, int H, int batch, int seq, float* row_loss, float* loss, __nv_bfloat16* dh, cudaStream_t s);
 int cross_entropy(const __nv_bfloat16* logits, const int32_t* ids, int M, int V, int batch, int seq, float* row_loss,
                   __nv_bfloat16* dlogits, float* loss, cudaStream_t s);
 int mse_loss(const __nv_bfloat16* out, size_t n, float* partial, int n_partial, __nv_bfloat16* dout, float* loss,

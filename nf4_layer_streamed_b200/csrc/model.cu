@@ -11,6 +11,8 @@
 // per parameter and token).  The DPO/KTO write-up ("Soup v0.72.4 技术解析" §3.1) reuses
 // the same streamed base with the adapter switched off as the reference model, which
 // nf4ls_forward_loss(lora_on = 0) provides.
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -20,7 +22,10 @@ namespace {
 
 struct ModelWs {
   size_t xs, hf, logits, row_loss, dh, dhf, layer, total;
+  size_t acc = 0, wt = 0, mx = 0, sm = 0, alpha = 0, lt = 0;  // streamed head
 };
+
+bool streamed_head(const nf4ls_model_cfg* c) { return c->head_chunk_rows > 0; }
 
 ModelWs model_ws(const nf4ls_model_cfg* c) {
   const size_t M = (size_t)c->layer.batch * c->layer.seq, H = c->layer.hidden;
@@ -33,8 +38,17 @@ ModelWs model_ws(const nf4ls_model_cfg* c) {
   };
   L.xs = take((size_t)(c->n_layers + 1) * M * H * 2);
   L.hf = take(M * H * 2);
-  L.logits = take(M * (size_t)c->vocab * 2);
+  // resident head: the whole [M, V] logits; streamed head: one vocab chunk of them
+  L.logits = take(M * (size_t)(streamed_head(c) ? std::min(c->head_chunk_rows, c->vocab) : c->vocab) * 2);
   L.row_loss = take(M * 4);
+  if (streamed_head(c)) {
+    L.acc = take(M * H * 4);
+    L.wt = take(M * H * 2);
+    L.mx = take(M * 4);
+    L.sm = take(M * 4);
+    L.alpha = take(M * 4);
+    L.lt = take(M * 4);
+  }
   L.dh = take(M * H * 2);
   L.dhf = take(M * H * 2);
   L.layer = take(layer_ws_bytes(&c->layer));
@@ -110,8 +124,16 @@ int check_model(const nf4ls_model_cfg* c, const nf4ls_model* m) {
   if (!c || !m) return fail(NF4LS_INVALID_ARG, "model: null config or model");
   NF4_TRY(check_cfg(&c->layer));
   if (c->n_layers <= 0 || c->vocab <= 0 || c->vocab % 64) return fail(NF4LS_SHAPE, "model: vocab must be a multiple of 64");
-  if (!m->embed_dev || !m->norm_final_dev || !m->lora_dev || !m->ws_dev) return fail(NF4LS_INVALID_ARG, "model: null buffer");
-  if (!c->tied && !m->lm_head_dev) return fail(NF4LS_INVALID_ARG, "model: untied model needs lm_head");
+  if (!m->norm_final_dev || !m->lora_dev || !m->ws_dev) return fail(NF4LS_INVALID_ARG, "model: null buffer");
+  if (streamed_head(c)) {
+    if (c->head_chunk_rows % 64) return fail(NF4LS_SHAPE, "model: head_chunk_rows must be a multiple of 64");
+    if (!m->head_pool) return fail(NF4LS_INVALID_ARG, "model: streamed head needs head_pool");
+    if (!m->embed_dev && !m->embed_host) return fail(NF4LS_INVALID_ARG, "model: no embedding");
+  } else {
+    if (c->head_chunk_rows < 0) return fail(NF4LS_INVALID_ARG, "model: head_chunk_rows < 0");
+    if (!m->embed_dev) return fail(NF4LS_INVALID_ARG, "model: null embedding");
+    if (!c->tied && !m->lm_head_dev) return fail(NF4LS_INVALID_ARG, "model: untied model needs lm_head");
+  }
   if (!m->pool && !m->shards_dev) return fail(NF4LS_INVALID_ARG, "model: needs a pool or resident shards");
   if (!aligned(m->ws_dev, 256)) return fail(NF4LS_ALIGN, "model: workspace must be 256-byte aligned");
   if (m->ws_bytes < model_ws(c).total) return fail(NF4LS_INVALID_ARG, "model: workspace too small");
@@ -123,16 +145,73 @@ int pool_depth(const nf4ls_model* m) {
   return 2;  // prefetch one layer ahead, as the pages do
 }
 
-// Forward through embedding, layers, final norm, lm_head and the loss.
+// The streamed head: logits, loss and (need_grad) dL/dhf in one pass over the vocab
+// chunks of the output matrix, each chunk used by two GEMMs while it is in its slot:
+// logits_c = hf Wc^T, then (after ce_chunk folded them into the running max / sum and
+// turned them into P = exp(logit - max)) acc = alpha acc + P Wc in fp32.
+int head_streamed(const nf4ls_model_cfg* c, const nf4ls_model* m, const int32_t* ids, const __nv_bfloat16* hf,
+                  bool need_grad, float* loss, __nv_bfloat16* dhf, cudaStream_t s, const ModelWs& L) {
+  const nf4ls_layer_cfg* lc = &c->layer;
+  const int M = lc->batch * lc->seq, H = lc->hidden, V = c->vocab, C = c->head_chunk_rows;
+  void* ws = m->ws_dev;
+  auto* lg = at<__nv_bfloat16>(ws, L.logits);
+  auto* acc = at<float>(ws, L.acc);
+  auto* wt = at<__nv_bfloat16>(ws, L.wt);
+  auto* mx = at<float>(ws, L.mx);
+  auto* sm = at<float>(ws, L.sm);
+  auto* alpha = at<float>(ws, L.alpha);
+  auto* lt = at<float>(ws, L.lt);
+  const int nch = (V + C - 1) / C;
+  for (int k = 0; k < nch; ++k) {
+    const void* slot;
+    NF4_TRY(stream_prefetch(m->head_pool, k, s, &slot));
+    if (k + 1 < nch) {
+      const int st = nf4ls_pool_prefetch(m->head_pool, k + 1);
+      if (st != NF4LS_BUFFER_BUSY) NF4_TRY(st);
+    }
+    const int v0 = k * C, n = std::min(C, V - v0);
+    GemmWeights w;
+    w.dense = static_cast<const __nv_bfloat16*>(slot);
+    GemmEpilogue e;
+    e.out = lg;
+    e.ldo = n;
+    NF4_TRY(gemm(hf, H, M, n, H, w, false, GemmExtra(), e, s));
+    NF4_TRY(ce_chunk(lg, n, v0, w.dense, ids, M, H, lc->seq, k == 0, mx, sm, alpha, lt, wt, s));
+    if (need_grad) {
+      GemmEpilogue ea;
+      ea.kind = EPI_ACC_F32;
+      ea.out_f32 = acc;
+      ea.ldo = H;
+      ea.alpha = alpha;
+      ea.accumulate = k > 0;
+      NF4_TRY(gemm(lg, n, M, H, n, w, true, GemmExtra(), ea, s));
+    }
+    NF4_TRY(nf4ls_pool_release(m->head_pool, k, s));
+  }
+  return ce_finish(mx, sm, lt, need_grad ? acc : nullptr, wt, M, H, lc->batch, lc->seq, at<float>(ws, L.row_loss),
+                   loss, dhf, s);
+}
+
+// Forward through embedding, layers, final norm, lm_head and the loss (and, for the
+// streamed head with need_grad, dL/dhf).
 int forward_to_loss(const nf4ls_model_cfg* c, const nf4ls_model* m, const int32_t* ids, bool lora_on, float* loss,
-                    cudaStream_t s, const ModelWs& L) {
+                    cudaStream_t s, const ModelWs& L, bool need_grad) {
   const nf4ls_layer_cfg* lc = &c->layer;
   const int M = lc->batch * lc->seq, H = lc->hidden, V = c->vocab;
   void* ws = m->ws_dev;
   auto* xs = at<__nv_bfloat16>(ws, L.xs);
   const size_t act = (size_t)M * H;
   const size_t stride = stride_of(lc);
-  NF4_TRY(embed(ids, static_cast<const __nv_bfloat16*>(m->embed_dev), xs, M, H, s));
+  const void* E = m->embed_dev;
+  if (!E) {  // rows gathered straight from pinned host memory
+    void* d = nullptr;
+    if (cudaHostGetDevicePointer(&d, const_cast<void*>(m->embed_host), 0) != cudaSuccess) {
+      cudaGetLastError();
+      return fail(NF4LS_INVALID_ARG, "model: embed_host is not pinned, device-mapped host memory");
+    }
+    E = d;
+  }
+  NF4_TRY(embed(ids, static_cast<const __nv_bfloat16*>(E), xs, M, H, s));
   const int depth = pool_depth(m);
   {
   Phase fwd_phase(s, 2000);
@@ -153,6 +232,8 @@ int forward_to_loss(const nf4ls_model_cfg* c, const nf4ls_model* m, const int32_
   const auto* lm = static_cast<const __nv_bfloat16*>(c->tied ? m->embed_dev : m->lm_head_dev);
   NF4_TRY(rmsnorm_fwd(xs + (size_t)c->n_layers * act, static_cast<const __nv_bfloat16*>(m->norm_final_dev), hf, M, H,
                       lc->rms_eps, s));
+  if (streamed_head(c))
+    return head_streamed(c, m, ids, hf, need_grad, loss, at<__nv_bfloat16>(ws, L.dhf), s, L);
   GemmWeights w;
   w.dense = lm;
   GemmEpilogue e;
@@ -178,7 +259,8 @@ extern "C" int nf4ls_forward_loss(const nf4ls_model_cfg* cfg, const nf4ls_model*
   clear_error();
   NF4_TRY(check_model(cfg, m));
   if (!ids_dev || !loss_dev) return fail(NF4LS_INVALID_ARG, "nf4ls_forward_loss: null ids or loss");
-  return forward_to_loss(cfg, m, ids_dev, lora_on != 0, loss_dev, static_cast<cudaStream_t>(stream), model_ws(cfg));
+  return forward_to_loss(cfg, m, ids_dev, lora_on != 0, loss_dev, static_cast<cudaStream_t>(stream), model_ws(cfg),
+                         false);
 }
 
 extern "C" int nf4ls_forward_backward(const nf4ls_model_cfg* cfg, const nf4ls_model* m, const int32_t* ids_dev,
@@ -188,7 +270,7 @@ extern "C" int nf4ls_forward_backward(const nf4ls_model_cfg* cfg, const nf4ls_mo
   if (!ids_dev || !loss_dev || !m->grads_dev) return fail(NF4LS_INVALID_ARG, "nf4ls_forward_backward: null argument");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const ModelWs L = model_ws(cfg);
-  NF4_TRY(forward_to_loss(cfg, m, ids_dev, true, loss_dev, s, L));
+  NF4_TRY(forward_to_loss(cfg, m, ids_dev, true, loss_dev, s, L, true));
   const nf4ls_layer_cfg* lc = &cfg->layer;
   const int M = lc->batch * lc->seq, H = lc->hidden, V = cfg->vocab;
   void* ws = m->ws_dev;
@@ -200,12 +282,14 @@ extern "C" int nf4ls_forward_backward(const nf4ls_model_cfg* cfg, const nf4ls_mo
   const auto* lm = static_cast<const __nv_bfloat16*>(cfg->tied ? m->embed_dev : m->lm_head_dev);
   {
     Phase head_bwd(s, 2002);
-    GemmWeights w;
-    w.dense = lm;
-    GemmEpilogue e;
-    e.out = dhf;
-    e.ldo = H;
-    NF4_TRY(gemm(logits, V, M, H, V, w, true, GemmExtra(), e, s));
+    if (!streamed_head(cfg)) {  // the streamed head has produced dhf already
+      GemmWeights w;
+      w.dense = lm;
+      GemmEpilogue e;
+      e.out = dhf;
+      e.ldo = H;
+      NF4_TRY(gemm(logits, V, M, H, V, w, true, GemmExtra(), e, s));
+    }
     NF4_TRY(rmsnorm_bwd(xs + (size_t)cfg->n_layers * act, static_cast<const __nv_bfloat16*>(m->norm_final_dev), dhf,
                         nullptr, dh, M, H, lc->rms_eps, s));
   }

@@ -106,3 +106,25 @@ def test_layer_calls_validate_config_on_host():
     st = B.call_status("layer_forward", ctypes.byref(cfg), ctypes.c_void_p(256), None, ctypes.c_void_p(256),
                        ctypes.c_void_p(256), ctypes.c_void_p(256), 1 << 30, None)
     assert st == -2
+
+
+def test_streamed_head_config_checked_on_host():
+    """The model refuses a streamed head whose chunk is not a multiple of 64 rows, or
+    that has no head pool, before it touches any buffer."""
+    wl = synth.WORKLOADS["smollm2_30L_tied_b1s512"]
+    fake = ctypes.c_void_p(256)
+    for rows, pool, want in ((100, fake, -2), (8192, None, -1)):
+        cfg = B.ModelCfg(api.layer_cfg(wl.shape, wl.batch, wl.seq), wl.n_layers, wl.vocab, 1, 2e-4, 0.9, 0.999,
+                         1e-8, 0.0, rows)
+        ws = B.lib().nf4ls_model_workspace_bytes(ctypes.byref(cfg))
+        m = B.Model(None, None, 256, 256, 256, 256, 256, 256, None, 256, ws, pool, 256)
+        st = B.call_status("nf4ls_forward_loss", ctypes.byref(cfg), ctypes.byref(m), fake, 1, fake, None)
+        assert st == want, (rows, st)
+    # the streamed head needs one vocab chunk of logits, not all of them
+    cfg_res = B.ModelCfg(api.layer_cfg(wl.shape, wl.batch, wl.seq), wl.n_layers, wl.vocab, 1, 2e-4, 0.9, 0.999,
+                         1e-8, 0.0, 0)
+    cfg_str = B.ModelCfg(api.layer_cfg(wl.shape, wl.batch, wl.seq), wl.n_layers, wl.vocab, 1, 2e-4, 0.9, 0.999,
+                         1e-8, 0.0, 8192)
+    res = B.lib().nf4ls_model_workspace_bytes(ctypes.byref(cfg_res))
+    strm = B.lib().nf4ls_model_workspace_bytes(ctypes.byref(cfg_str))
+    assert strm < res
