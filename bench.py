@@ -229,6 +229,26 @@ def extra_points(args, wl, ms_step: float, copy_ms: float) -> dict:
                             "hbm_bytes_saved": 2 * wl.vocab * wl.shape.hidden * 2,
                             "note": "lm_head and embedding stay in pinned host memory; one pass over the "
                                     "vocab chunks gives loss and dL/dh"}
+    # disk stream source: the shard set written once to a file, read back every step
+    import tempfile
+    d = tempfile.mkdtemp(dir=os.environ.get("NF4LS_DISK_DIR") or None)
+    path = os.path.join(d, "llama8b_store.bin")
+    try:
+        m = api.StreamedModel(wl, depth=args.depth, source="disk", store_path=path)
+        probe = api.disk_probe(path, 2 << 30)
+        accepted = api.disk_accept(probe, 1.5) == 0
+        t_disk = time_steps(m, ids, 1, 2)
+        st = m.pool.stats()
+        m.close()
+        del m
+        out["disk_source"] = {"ms_per_step": t_disk, "tokens_per_s": wl.tokens / (t_disk / 1000.0),
+                              "probe": probe, "accepted_at_1.5_gbs": accepted,
+                              "read_gbs_over_step": (st["bytes_copied"] / 3) / (t_disk / 1000.0) / 1e9,
+                              "note": "same workload, layers read from a file by the pool's reader thread"}
+    finally:
+        if os.path.exists(path):
+            os.unlink(path)
+        os.rmdir(d)
     wl16 = synth.WORKLOADS["llama8b_32L_b16s512"]
     ids16 = [dp.rank_token_ids(wl16, 0, s) for s in range(3)]
     m = api.StreamedModel(wl16, depth=args.depth)

@@ -54,6 +54,9 @@ extern "C" {
 #define NF4LS_TIMEOUT              -7  /* a bounded host wait expired                 */
 #define NF4LS_CUDA                 -8  /* a CUDA runtime call failed                  */
 #define NF4LS_DEVICE_FAULT         -9  /* a kernel's bounded wait expired             */
+#define NF4LS_SOURCE_REFUSED      -10  /* a stream source too slow, or a SATA / spinning
+                                          disk ([review] mechanism: refused outright)   */
+#define NF4LS_IO                  -11  /* a file read failed                          */
 
 typedef void* nf4ls_stream; /* cudaStream_t */
 
@@ -309,6 +312,45 @@ int nf4ls_pool_set_poison(nf4ls_pool* pool, int on);
 int nf4ls_pool_get_stats(nf4ls_pool* pool, nf4ls_pool_stats* out);
 int nf4ls_pool_synchronize(nf4ls_pool* pool);
 int nf4ls_pool_destroy(nf4ls_pool* pool);
+
+/* ------------------------------------------------------------------ disk stream source
+ * [review] mechanism section: the frozen base lives in (pinned) host memory and falls
+ * back to an NVMe disk when memory is short; SATA and spinning disks are refused
+ * outright; the config key stream_source: auto takes memory when the store fits and
+ * NVMe otherwise.
+ *
+ * nf4ls_disk_probe: classifies the device under `path` (sysfs: block device or not,
+ * NVMe, rotational) and times a sequential read of up to probe_bytes of the file
+ * (O_DIRECT when the file system allows it, so the page cache does not answer).
+ * nf4ls_disk_accept: NF4LS_OK for a non-rotational device that is NVMe or not a block
+ * device at all (memory-backed) and reads at >= min_gbs; NF4LS_SOURCE_REFUSED
+ * otherwise (the message says why).
+ * nf4ls_choose_source: *use_disk = 0 when store_bytes + reserve_bytes fit in the
+ * host's available memory (MemAvailable), else 1. */
+typedef struct {
+    double read_gbs;        /* measured sequential read, GB/s (1e9 B/s)        */
+    int32_t block_device;   /* 1: the file sits on a block device              */
+    int32_t nvme;           /* 1: ... and that device is NVMe                  */
+    int32_t rotational;     /* 1: ... and it is a spinning disk                */
+    int32_t direct_io;      /* 1: the probe read with O_DIRECT                 */
+} nf4ls_disk_info;
+
+int nf4ls_disk_probe(const char* path, size_t probe_bytes, nf4ls_disk_info* out);
+int nf4ls_disk_accept(const nf4ls_disk_info* info, double min_gbs);
+int nf4ls_choose_source(size_t store_bytes, size_t reserve_bytes, int32_t* use_disk);
+
+/* A pool whose store is a file: layer i is bytes [layer_off[i], + layer_bytes[i]) of
+ * `path` (layer_off[i] a multiple of 4096, so reads can bypass the page cache).  A
+ * reader thread reads each requested layer into one of two pinned staging buffers
+ * (staging_host: caller's pinned memory, 4096-byte aligned, >= 2 x the largest layer
+ * rounded up to 4096; nf4ls_pool_file_staging_bytes) and issues its host-to-device
+ * copy on the pool's copy stream; stream_prefetch then returns once that copy is
+ * enqueued (a host wait of at most 60 s, NF4LS_TIMEOUT after).  Every other pool call
+ * behaves as for a pinned store, and the bytes that reach a slot are the same. */
+size_t nf4ls_pool_file_staging_bytes(const size_t* layer_bytes, int n_layers);
+int nf4ls_pool_create_file(const char* path, const size_t* layer_off, const size_t* layer_bytes, int n_layers,
+                           int depth, void* slots_dev, size_t slot_bytes, void* staging_host, size_t staging_bytes,
+                           nf4ls_pool** out);
 
 /* ------------------------------------------------------------------ model step
  * One SFT step of the whole stack ([review]: embeddings and lm_head stay resident

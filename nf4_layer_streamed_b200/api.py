@@ -247,6 +247,27 @@ class Pool:
                ctypes.cast(self.sizes, ctypes.c_void_p), n, depth, _p(self.slots), self.slot_bytes,
                ctypes.byref(self.handle))
 
+    @classmethod
+    def from_file(cls, path: str, offsets, sizes, depth: int, slot_bytes: int | None = None, device="cuda"):
+        """A pool whose store is a file (the disk stream source): a library thread reads
+        each layer into pinned staging and copies it into its slot."""
+        self = cls.__new__(cls)
+        self.store = None
+        n = len(offsets)
+        self.offsets = (ctypes.c_size_t * n)(*offsets)
+        self.sizes = (ctypes.c_size_t * n)(*sizes)
+        self.slot_bytes = slot_bytes or (max(sizes) + 255) // 256 * 256
+        self.slots = _buffer(depth * self.slot_bytes, device)
+        nst = B.lib().nf4ls_pool_file_staging_bytes(ctypes.cast(self.sizes, ctypes.c_void_p), n)
+        raw = torch.empty(nst + 4096, dtype=torch.uint8).pin_memory()
+        skip = (-raw.data_ptr()) % 4096
+        self.staging = raw[skip:skip + nst]
+        self.handle = ctypes.c_void_p()
+        B.call("nf4ls_pool_create_file", path.encode(), ctypes.cast(self.offsets, ctypes.c_void_p),
+               ctypes.cast(self.sizes, ctypes.c_void_p), n, depth, _p(self.slots), self.slot_bytes,
+               _p(self.staging), nst, ctypes.byref(self.handle))
+        return self
+
     def prefetch(self, layer: int) -> int:
         return B.call_status("nf4ls_pool_prefetch", self.handle, layer)
 
@@ -283,6 +304,27 @@ class Pool:
         return self.slots[off: off + nbytes]
 
 
+def disk_probe(path: str, probe_bytes: int = 1 << 30) -> dict:
+    info = B.DiskInfo()
+    B.call("nf4ls_disk_probe", path.encode(), probe_bytes, ctypes.byref(info))
+    return {"read_gbs": info.read_gbs, "block_device": bool(info.block_device), "nvme": bool(info.nvme),
+            "rotational": bool(info.rotational), "direct_io": bool(info.direct_io)}
+
+
+def disk_accept(info: dict, min_gbs: float = 1.5) -> int:
+    """NF4LS_OK, or NF4LS_SOURCE_REFUSED for a spinning / non-NVMe / slow device."""
+    d = B.DiskInfo(info["read_gbs"], int(info["block_device"]), int(info["nvme"]), int(info["rotational"]),
+                   int(info.get("direct_io", False)))
+    return B.call_status("nf4ls_disk_accept", ctypes.byref(d), float(min_gbs))
+
+
+def choose_source(store_bytes: int, reserve_bytes: int = 8 << 30) -> str:
+    """stream_source: auto -- 'ram' when the store fits in available host memory."""
+    out = ctypes.c_int32()
+    B.call("nf4ls_choose_source", store_bytes, reserve_bytes, ctypes.byref(out))
+    return "disk" if out.value else "ram"
+
+
 # ----------------------------------------------------------------------------- whole model
 
 @dataclass
@@ -301,9 +343,14 @@ class StreamedModel:
 
     def __init__(self, wl: Workload, depth: int = 2, resident: bool = False, b_random: bool = False,
                  train: TrainConfig = TrainConfig(), device="cuda", weights_device=None, fingerprint: int = 1234,
-                 head_chunk_rows: int = 0):
+                 head_chunk_rows: int = 0, source: str = "ram", store_path: str | None = None,
+                 min_disk_gbs: float | None = None):
         """head_chunk_rows > 0: the embedding and lm_head stay in pinned host memory; the
-        output matrix streams through a depth-2 pool in chunks of that many vocab rows."""
+        output matrix streams through a depth-2 pool in chunks of that many vocab rows.
+        source: 'ram' (pinned store), 'disk' (the shard set written once to store_path and
+        read back by the pool's reader thread; with min_disk_gbs set, the device is probed
+        first and a spinning, non-NVMe or slower device is refused) or 'auto' (RAM when the
+        store fits in available memory)."""
         self.wl = wl
         shape = wl.shape
         self.cfg = B.ModelCfg(layer_cfg(shape, wl.batch, wl.seq), wl.n_layers, wl.vocab, int(wl.tied), train.lr,
@@ -317,8 +364,18 @@ class StreamedModel:
         self.resident = resident
         self.pool = None
         shards = []
+        file_stride = (self.slot_bytes + 4095) // 4096 * 4096
+        if source == "auto":
+            source = choose_source(L * self.slot_bytes)
+        self.source = "resident" if resident else source
         if resident:
             self.shard_buf = _buffer(L * self.slot_bytes, device)
+        elif source == "disk":
+            if not store_path:
+                raise ValueError("the disk stream source needs store_path")
+            fh = open(store_path, "wb")
+            fh.truncate(L * file_stride)
+            host = torch.empty(self.slot_bytes, dtype=torch.uint8).pin_memory()
         else:
             self.store = torch.empty(L * self.slot_bytes, dtype=torch.uint8).pin_memory()
         tmp = _buffer(self.slot_bytes, device)
@@ -332,11 +389,27 @@ class StreamedModel:
             else:
                 nf4_quantize_shard(lc, w, fingerprint, out=tmp)
                 torch.cuda.synchronize()
-                self.store[i * self.slot_bytes:(i + 1) * self.slot_bytes].copy_(tmp)
+                if source == "disk":
+                    host.copy_(tmp)
+                    fh.seek(i * file_stride)
+                    fh.write(host.numpy().tobytes())
+                else:
+                    self.store[i * self.slot_bytes:(i + 1) * self.slot_bytes].copy_(tmp)
             del w
         del tmp
         if resident:
             self.shard_ptrs = (ctypes.c_void_p * L)(*shards)
+        elif source == "disk":
+            fh.close()
+            del host
+            self.disk = None
+            if min_disk_gbs is not None:
+                self.disk = disk_probe(store_path)
+                st = disk_accept(self.disk, min_disk_gbs)
+                if st != 0:
+                    raise B.NF4LSError(st, B.lib().nf4ls_last_error().decode())
+            offs = [i * file_stride for i in range(L)]
+            self.pool = Pool.from_file(store_path, offs, [self.shard_nbytes] * L, depth, self.slot_bytes, device)
         else:
             offs = [i * self.slot_bytes for i in range(L)]
             self.pool = Pool(self.store, offs, [self.shard_nbytes] * L, depth, self.slot_bytes, device)

@@ -15,7 +15,8 @@ LIB_PATH = os.path.join(PKG, "libnf4ls.so")
 
 OK = 0
 STATUS = {0: "OK", -1: "INVALID_ARG", -2: "SHAPE", -3: "ALIGN", -4: "CODEBOOK_MISMATCH",
-          -5: "FINGERPRINT_MISMATCH", -6: "BUFFER_BUSY", -7: "TIMEOUT", -8: "CUDA", -9: "DEVICE_FAULT"}
+          -5: "FINGERPRINT_MISMATCH", -6: "BUFFER_BUSY", -7: "TIMEOUT", -8: "CUDA", -9: "DEVICE_FAULT",
+          -10: "SOURCE_REFUSED", -11: "IO"}
 
 
 class NF4LSError(RuntimeError):
@@ -62,6 +63,11 @@ class PoolStats(ctypes.Structure):
                 ("acquisitions", ctypes.c_uint64)]
 
 
+class DiskInfo(ctypes.Structure):
+    _fields_ = [("read_gbs", ctypes.c_double), ("block_device", ctypes.c_int32), ("nvme", ctypes.c_int32),
+                ("rotational", ctypes.c_int32), ("direct_io", ctypes.c_int32)]
+
+
 P = ctypes.c_void_p
 I32 = ctypes.c_int32
 SZ = ctypes.c_size_t
@@ -102,6 +108,12 @@ SIGNATURES = {
     "nf4ls_pool_get_stats": (ctypes.c_int, [P, ctypes.POINTER(PoolStats)]),
     "nf4ls_pool_synchronize": (ctypes.c_int, [P]),
     "nf4ls_pool_destroy": (ctypes.c_int, [P]),
+    "nf4ls_disk_probe": (ctypes.c_int, [ctypes.c_char_p, SZ, ctypes.POINTER(DiskInfo)]),
+    "nf4ls_disk_accept": (ctypes.c_int, [ctypes.POINTER(DiskInfo), ctypes.c_double]),
+    "nf4ls_choose_source": (ctypes.c_int, [SZ, SZ, ctypes.POINTER(ctypes.c_int32)]),
+    "nf4ls_pool_file_staging_bytes": (SZ, [P, ctypes.c_int]),
+    "nf4ls_pool_create_file": (ctypes.c_int, [ctypes.c_char_p, P, P, ctypes.c_int, ctypes.c_int, P, SZ, P, SZ,
+                                              ctypes.POINTER(P)]),
     "nf4ls_lora_stride": (SZ, [ctypes.POINTER(LayerCfg)]),
     "nf4ls_model_workspace_bytes": (SZ, [ctypes.POINTER(ModelCfg)]),
     "nf4ls_train_step": (ctypes.c_int, [ctypes.POINTER(ModelCfg), ctypes.POINTER(Model), P, I32, P, P]),

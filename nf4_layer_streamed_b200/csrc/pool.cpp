@@ -14,15 +14,79 @@
 // slot -- has completed.  The copy stream waits on that event; nothing else orders
 // the reuse.  A layer still held by a slot is served without a new copy, which lets
 // the backward start on the layers the forward left behind.
+//
+// Disk source (same pages, mechanism section: the base falls back from pinned memory
+// to an NVMe disk when memory is short; SATA and spinning disks are refused): the
+// store is a file, a reader thread reads each requested layer into one of two
+// caller-owned pinned staging buffers and enqueues its copy into the slot on the copy
+// stream; the slot rules above are unchanged.
+#include <fcntl.h>
+#include <sys/stat.h>
+#include <sys/sysmacros.h>
+#include <unistd.h>
+
 #include <algorithm>
 #include <chrono>
+#include <climits>
+#include <condition_variable>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <deque>
 #include <mutex>
+#include <string>
 #include <thread>
 #include <vector>
 
 #include "internal.h"
 
 using namespace nf4ls;
+
+namespace {
+
+constexpr size_t kIoAlign = 4096;
+constexpr int kFillWaitMs = 60000;  // host bound on waiting for a layer's file read
+
+size_t io_round(size_t b) { return (b + kIoAlign - 1) / kIoAlign * kIoAlign; }
+
+// Reads [off, off + need) of fd into dst (need <= cap, cap a multiple of 4096 when
+// direct); returns 0 or errno-like failure.
+int read_range(int fd, bool direct, uint8_t* dst, size_t cap, size_t off, size_t need) {
+  size_t done = 0;
+  const size_t want = direct ? std::min(cap, io_round(need)) : need;
+  while (done < need) {
+    const ssize_t r = pread(fd, dst + done, want - done, (off_t)(off + done));
+    if (r < 0) {
+      if (errno == EINTR) continue;
+      return errno ? errno : EIO;
+    }
+    if (r == 0) return EIO;  // the file ends before the layer does
+    done += (size_t)r;
+  }
+  return 0;
+}
+
+}  // namespace
+
+struct FileSource {
+  int fd = -1;
+  bool direct = false;
+  uint8_t* staging[2] = {nullptr, nullptr};
+  size_t staging_each = 0;
+  cudaEvent_t staged[2] = {nullptr, nullptr};  // the copy out of staging buffer b is done
+  bool staged_recorded[2] = {false, false};
+  uint64_t seq = 0;
+  struct Job {
+    int layer, slot;
+    bool wait_freed;
+  };
+  std::deque<Job> jobs;
+  std::condition_variable cv_job, cv_done;
+  bool stop = false;
+  int error = NF4LS_OK;
+  std::string error_msg;
+  std::thread reader;
+};
 
 struct nf4ls_pool {
   int device = 0;
@@ -37,6 +101,7 @@ struct nf4ls_pool {
     bool acquired = false;
     bool pending = false;  // filled by a prefetch and not yet acquired
     bool freed_recorded = false;
+    bool filling = false;  // disk source: the reader has not enqueued this slot's copy yet
     uint64_t release_tick = 0;
     cudaEvent_t ready = nullptr, freed = nullptr;
   };
@@ -45,6 +110,7 @@ struct nf4ls_pool {
   bool poison = false;
   nf4ls_pool_stats stats{};
   std::mutex mu;
+  FileSource* file = nullptr;
 
   int find(int layer) const {
     for (int i = 0; i < depth; ++i)
@@ -73,6 +139,18 @@ struct nf4ls_pool {
     if (i < 0) return fail(NF4LS_BUFFER_BUSY, "pool: every slot is acquired or pending (depth %d)", depth);
     Slot& s = slot[i];
     uint8_t* dst = slots + (size_t)i * slot_bytes;
+    if (file) {  // the reader thread reads the layer and enqueues the copy
+      if (file->error) return fail(file->error, "pool: disk source failed earlier: %s", file->error_msg.c_str());
+      file->jobs.push_back(FileSource::Job{layer, i, s.freed_recorded});
+      file->cv_job.notify_one();
+      s.layer = layer;
+      s.pending = true;
+      s.filling = true;
+      stats.bytes_copied += bytes[layer];
+      stats.copies += 1;
+      *out_idx = i;
+      return NF4LS_OK;
+    }
     if (s.freed_recorded) NF4_CUDA_TRY(cudaStreamWaitEvent(copy, s.freed, 0));
     if (poison) NF4_CUDA_TRY(cudaMemsetAsync(dst, 0xFF, slot_bytes, copy));
     NF4_CUDA_TRY(cudaMemcpyAsync(dst, store + off[layer], bytes[layer], cudaMemcpyHostToDevice, copy));
@@ -84,25 +162,103 @@ struct nf4ls_pool {
     *out_idx = i;
     return NF4LS_OK;
   }
+
+  // Disk source: waits (lk held on mu) until slot idx's copy has been enqueued.
+  int wait_filled(std::unique_lock<std::mutex>& lk, int idx) {
+    if (!file) return NF4LS_OK;
+    const bool ok = file->cv_done.wait_for(lk, std::chrono::milliseconds(kFillWaitMs),
+                                           [&] { return !slot[idx].filling || file->error != NF4LS_OK; });
+    if (file->error) return fail(file->error, "pool: disk source: %s", file->error_msg.c_str());
+    if (!ok) return fail(NF4LS_TIMEOUT, "pool: layer %d not read from disk after %d ms", slot[idx].layer, kFillWaitMs);
+    return NF4LS_OK;
+  }
+
+  void reader_loop() {
+    cudaSetDevice(device);
+    FileSource& f = *file;
+    while (true) {
+      FileSource::Job j;
+      {
+        std::unique_lock<std::mutex> lk(mu);
+        f.cv_job.wait(lk, [&] { return f.stop || !f.jobs.empty(); });
+        if (f.jobs.empty()) return;  // stop requested and nothing left
+        j = f.jobs.front();
+      }
+      const int b = (int)(f.seq++ & 1);
+      int err = NF4LS_OK;
+      std::string msg;
+      if (f.staged_recorded[b]) {  // the previous copy out of this staging buffer must be done
+        const auto t0 = std::chrono::steady_clock::now();
+        while (true) {
+          const cudaError_t e = cudaEventQuery(f.staged[b]);
+          if (e == cudaSuccess) break;
+          if (e != cudaErrorNotReady) {
+            err = NF4LS_CUDA;
+            msg = cudaGetErrorString(e);
+            break;
+          }
+          if (std::chrono::steady_clock::now() - t0 > std::chrono::milliseconds(kFillWaitMs)) {
+            err = NF4LS_TIMEOUT;
+            msg = "staging buffer copy did not finish";
+            break;
+          }
+          std::this_thread::sleep_for(std::chrono::microseconds(20));
+        }
+      }
+      if (!err) {
+        const int r = read_range(f.fd, f.direct, f.staging[b], f.staging_each, off[j.layer], bytes[j.layer]);
+        if (r) {
+          err = NF4LS_IO;
+          msg = std::string("read of layer ") + std::to_string(j.layer) + ": " + strerror(r);
+        }
+      }
+      std::lock_guard<std::mutex> g(mu);
+      f.jobs.pop_front();
+      Slot& s = slot[j.slot];
+      if (!err) {
+        uint8_t* dst = slots + (size_t)j.slot * slot_bytes;
+        cudaError_t e = cudaSuccess;
+        if (j.wait_freed) e = cudaStreamWaitEvent(copy, s.freed, 0);
+        if (e == cudaSuccess && poison) e = cudaMemsetAsync(dst, 0xFF, slot_bytes, copy);
+        if (e == cudaSuccess) e = cudaMemcpyAsync(dst, f.staging[b], bytes[j.layer], cudaMemcpyHostToDevice, copy);
+        if (e == cudaSuccess) e = cudaEventRecord(f.staged[b], copy);
+        if (e == cudaSuccess) e = cudaEventRecord(s.ready, copy);
+        if (e != cudaSuccess) {
+          err = NF4LS_CUDA;
+          msg = cudaGetErrorString(e);
+        }
+        f.staged_recorded[b] = true;
+      }
+      if (err && !f.error) {
+        f.error = err;
+        f.error_msg = msg;
+      }
+      s.filling = false;
+      f.cv_done.notify_all();
+    }
+  }
 };
 
-extern "C" int nf4ls_pool_create(const void* pinned_host, const size_t* layer_off, const size_t* layer_bytes,
-                                 int n_layers, int depth, void* slots_dev, size_t slot_bytes, nf4ls_pool** out) {
-  clear_error();
-  if (!pinned_host || !layer_off || !layer_bytes || !slots_dev || !out)
-    return fail(NF4LS_INVALID_ARG, "nf4ls_pool_create: null pointer");
-  if (n_layers <= 0) return fail(NF4LS_INVALID_ARG, "nf4ls_pool_create: n_layers must be positive");
-  if (depth < 2 || depth > 8) return fail(NF4LS_INVALID_ARG, "nf4ls_pool_create: depth %d not in [2, 8]", depth);
+namespace {
+
+int check_pool_args(const size_t* layer_off, const size_t* layer_bytes, int n_layers, int depth, void* slots_dev,
+                    size_t slot_bytes, size_t off_align, const char* who) {
+  if (!layer_off || !layer_bytes || !slots_dev) return fail(NF4LS_INVALID_ARG, "%s: null pointer", who);
+  if (n_layers <= 0) return fail(NF4LS_INVALID_ARG, "%s: n_layers must be positive", who);
+  if (depth < 2 || depth > 8) return fail(NF4LS_INVALID_ARG, "%s: depth %d not in [2, 8]", who, depth);
   if (!aligned(slots_dev, 256) || slot_bytes % 256)
-    return fail(NF4LS_ALIGN, "nf4ls_pool_create: slots must be 256-byte aligned and sized");
+    return fail(NF4LS_ALIGN, "%s: slots must be 256-byte aligned and sized", who);
   for (int i = 0; i < n_layers; ++i) {
     if (layer_bytes[i] > slot_bytes)
-      return fail(NF4LS_INVALID_ARG, "nf4ls_pool_create: layer %d (%zu B) exceeds slot (%zu B)", i, layer_bytes[i],
-                  slot_bytes);
-    if (layer_off[i] % 256) return fail(NF4LS_ALIGN, "nf4ls_pool_create: layer %d offset not 256-aligned", i);
+      return fail(NF4LS_INVALID_ARG, "%s: layer %d (%zu B) exceeds slot (%zu B)", who, i, layer_bytes[i], slot_bytes);
+    if (layer_off[i] % off_align) return fail(NF4LS_ALIGN, "%s: layer %d offset not %zu-aligned", who, i, off_align);
   }
+  return NF4LS_OK;
+}
+
+int make_pool(const size_t* layer_off, const size_t* layer_bytes, int n_layers, int depth, void* slots_dev,
+              size_t slot_bytes, nf4ls_pool** out) {
   nf4ls_pool* p = new nf4ls_pool();
-  p->store = static_cast<const uint8_t*>(pinned_host);
   p->off.assign(layer_off, layer_off + n_layers);
   p->bytes.assign(layer_bytes, layer_bytes + n_layers);
   p->n_layers = n_layers;
@@ -118,9 +274,171 @@ extern "C" int nf4ls_pool_create(const void* pinned_host, const size_t* layer_of
   }
   if (e != cudaSuccess) {
     nf4ls_pool_destroy(p);
-    return fail(NF4LS_CUDA, "nf4ls_pool_create: %s", cudaGetErrorString(e));
+    return fail(NF4LS_CUDA, "pool create: %s", cudaGetErrorString(e));
   }
   *out = p;
+  return NF4LS_OK;
+}
+
+// sysfs path of the block device holding st_dev, or "" (not a block device).
+std::string block_sysfs(dev_t dev) {
+  char link[64], real[PATH_MAX];
+  std::snprintf(link, sizeof(link), "/sys/dev/block/%u:%u", major(dev), minor(dev));
+  if (!realpath(link, real)) return "";
+  return real;
+}
+
+int read_flag(const std::string& path, int* v) {
+  FILE* f = std::fopen(path.c_str(), "r");
+  if (!f) return -1;
+  const int n = std::fscanf(f, "%d", v);
+  std::fclose(f);
+  return n == 1 ? 0 : -1;
+}
+
+}  // namespace
+
+extern "C" int nf4ls_pool_create(const void* pinned_host, const size_t* layer_off, const size_t* layer_bytes,
+                                 int n_layers, int depth, void* slots_dev, size_t slot_bytes, nf4ls_pool** out) {
+  clear_error();
+  if (!pinned_host || !out) return fail(NF4LS_INVALID_ARG, "nf4ls_pool_create: null pointer");
+  NF4_TRY(check_pool_args(layer_off, layer_bytes, n_layers, depth, slots_dev, slot_bytes, 256, "nf4ls_pool_create"));
+  NF4_TRY(make_pool(layer_off, layer_bytes, n_layers, depth, slots_dev, slot_bytes, out));
+  (*out)->store = static_cast<const uint8_t*>(pinned_host);
+  return NF4LS_OK;
+}
+
+extern "C" size_t nf4ls_pool_file_staging_bytes(const size_t* layer_bytes, int n_layers) {
+  if (!layer_bytes || n_layers <= 0) return 0;
+  size_t mx = 0;
+  for (int i = 0; i < n_layers; ++i) mx = std::max(mx, layer_bytes[i]);
+  return 2 * io_round(mx);
+}
+
+extern "C" int nf4ls_pool_create_file(const char* path, const size_t* layer_off, const size_t* layer_bytes,
+                                      int n_layers, int depth, void* slots_dev, size_t slot_bytes,
+                                      void* staging_host, size_t staging_bytes, nf4ls_pool** out) {
+  clear_error();
+  if (!path || !staging_host || !out) return fail(NF4LS_INVALID_ARG, "nf4ls_pool_create_file: null pointer");
+  NF4_TRY(check_pool_args(layer_off, layer_bytes, n_layers, depth, slots_dev, slot_bytes, kIoAlign,
+                          "nf4ls_pool_create_file"));
+  const size_t need = nf4ls_pool_file_staging_bytes(layer_bytes, n_layers);
+  if (!aligned(staging_host, kIoAlign) || staging_bytes < need)
+    return fail(NF4LS_ALIGN, "nf4ls_pool_create_file: staging must be 4096-byte aligned and >= %zu B", need);
+  int fd = open(path, O_RDONLY | O_DIRECT);
+  bool direct = fd >= 0;
+  if (fd < 0) fd = open(path, O_RDONLY);
+  if (fd < 0) return fail(NF4LS_IO, "nf4ls_pool_create_file: cannot open %s: %s", path, strerror(errno));
+  struct stat st;
+  if (fstat(fd, &st) != 0) {
+    close(fd);
+    return fail(NF4LS_IO, "nf4ls_pool_create_file: fstat failed");
+  }
+  for (int i = 0; i < n_layers; ++i)
+    if (layer_off[i] + layer_bytes[i] > (size_t)st.st_size) {
+      close(fd);
+      return fail(NF4LS_INVALID_ARG, "nf4ls_pool_create_file: layer %d ends past the end of %s", i, path);
+    }
+  nf4ls_pool* p = nullptr;
+  const int r = make_pool(layer_off, layer_bytes, n_layers, depth, slots_dev, slot_bytes, &p);
+  if (r) {
+    close(fd);
+    return r;
+  }
+  FileSource* f = new FileSource();
+  f->fd = fd;
+  f->direct = direct;
+  f->staging_each = need / 2;
+  f->staging[0] = static_cast<uint8_t*>(staging_host);
+  f->staging[1] = f->staging[0] + f->staging_each;
+  cudaError_t e = cudaEventCreateWithFlags(&f->staged[0], cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&f->staged[1], cudaEventDisableTiming);
+  p->file = f;
+  if (e != cudaSuccess) {
+    nf4ls_pool_destroy(p);
+    return fail(NF4LS_CUDA, "nf4ls_pool_create_file: %s", cudaGetErrorString(e));
+  }
+  f->reader = std::thread([p] { p->reader_loop(); });
+  *out = p;
+  return NF4LS_OK;
+}
+
+extern "C" int nf4ls_disk_probe(const char* path, size_t probe_bytes, nf4ls_disk_info* out) {
+  clear_error();
+  if (!path || !out || probe_bytes == 0) return fail(NF4LS_INVALID_ARG, "nf4ls_disk_probe: bad argument");
+  std::memset(out, 0, sizeof(*out));
+  struct stat st;
+  if (stat(path, &st) != 0) return fail(NF4LS_IO, "nf4ls_disk_probe: cannot stat %s: %s", path, strerror(errno));
+  const std::string sys = block_sysfs(st.st_dev);
+  if (!sys.empty()) {
+    out->block_device = 1;
+    out->nvme = sys.find("/nvme") != std::string::npos ? 1 : 0;
+    int rot = 0;
+    if (read_flag(sys + "/queue/rotational", &rot) != 0) read_flag(sys + "/../queue/rotational", &rot);
+    out->rotational = rot ? 1 : 0;
+  }
+  int fd = open(path, O_RDONLY | O_DIRECT);
+  out->direct_io = fd >= 0;
+  if (fd < 0) {
+    fd = open(path, O_RDONLY);
+    if (fd >= 0) posix_fadvise(fd, 0, 0, POSIX_FADV_DONTNEED);  // best effort: start cold
+  }
+  if (fd < 0) return fail(NF4LS_IO, "nf4ls_disk_probe: cannot open %s: %s", path, strerror(errno));
+  const size_t chunk = 16u << 20;
+  void* buf = nullptr;
+  if (posix_memalign(&buf, kIoAlign, chunk) != 0) {
+    close(fd);
+    return fail(NF4LS_INVALID_ARG, "nf4ls_disk_probe: no host memory for the probe buffer");
+  }
+  const size_t total = std::min(probe_bytes, (size_t)st.st_size);
+  size_t done = 0;
+  int err = 0;
+  const auto t0 = std::chrono::steady_clock::now();
+  while (done < total) {
+    const ssize_t r = pread(fd, buf, chunk, (off_t)done);
+    if (r < 0) {
+      if (errno == EINTR) continue;
+      err = errno;
+      break;
+    }
+    if (r == 0) break;
+    done += (size_t)r;
+  }
+  const double secs = std::chrono::duration<double>(std::chrono::steady_clock::now() - t0).count();
+  std::free(buf);
+  close(fd);
+  if (err) return fail(NF4LS_IO, "nf4ls_disk_probe: read failed: %s", strerror(err));
+  out->read_gbs = secs > 0 ? (double)done / secs / 1e9 : 0.0;
+  return NF4LS_OK;
+}
+
+extern "C" int nf4ls_disk_accept(const nf4ls_disk_info* info, double min_gbs) {
+  clear_error();
+  if (!info) return fail(NF4LS_INVALID_ARG, "nf4ls_disk_accept: null info");
+  if (info->rotational) return fail(NF4LS_SOURCE_REFUSED, "stream source refused: spinning disk");
+  if (info->block_device && !info->nvme) return fail(NF4LS_SOURCE_REFUSED, "stream source refused: not an NVMe device");
+  if (info->read_gbs < min_gbs)
+    return fail(NF4LS_SOURCE_REFUSED, "stream source refused: reads at %.2f GB/s < %.2f GB/s", info->read_gbs, min_gbs);
+  return NF4LS_OK;
+}
+
+extern "C" int nf4ls_choose_source(size_t store_bytes, size_t reserve_bytes, int32_t* use_disk) {
+  clear_error();
+  if (!use_disk) return fail(NF4LS_INVALID_ARG, "nf4ls_choose_source: null output");
+  *use_disk = 0;
+  FILE* f = std::fopen("/proc/meminfo", "r");
+  if (!f) return NF4LS_OK;  // unknown: memory
+  char key[64];
+  unsigned long long kb = 0;
+  bool found = false;
+  while (std::fscanf(f, "%63s %llu kB\n", key, &kb) == 2) {
+    if (std::strcmp(key, "MemAvailable:") == 0) {
+      found = true;
+      break;
+    }
+  }
+  std::fclose(f);
+  if (found && (unsigned long long)(store_bytes + reserve_bytes) > kb * 1024ull) *use_disk = 1;
   return NF4LS_OK;
 }
 
@@ -136,12 +454,13 @@ extern "C" int stream_prefetch(nf4ls_pool* p, int layer, nf4ls_stream compute, c
   clear_error();
   if (!p || layer < 0 || layer >= p->n_layers || !slot_dev)
     return fail(NF4LS_INVALID_ARG, "stream_prefetch: bad argument");
-  std::lock_guard<std::mutex> g(p->mu);
+  std::unique_lock<std::mutex> lk(p->mu);
   const bool hit = p->find(layer) >= 0;  // resident or already prefetched: this call copies nothing
   int idx;
   NF4_TRY(p->issue(layer, &idx));
   nf4ls_pool::Slot& s = p->slot[idx];
   if (s.acquired) return fail(NF4LS_BUFFER_BUSY, "stream_prefetch: layer %d is already acquired", layer);
+  NF4_TRY(p->wait_filled(lk, idx));
   NF4_CUDA_TRY(cudaStreamWaitEvent(static_cast<cudaStream_t>(compute), s.ready, 0));
   s.acquired = true;
   s.pending = false;
@@ -170,9 +489,10 @@ extern "C" int nf4ls_wait(nf4ls_pool* p, int layer, int timeout_ms) {
   if (!p || layer < 0 || layer >= p->n_layers) return fail(NF4LS_INVALID_ARG, "nf4ls_wait: bad argument");
   cudaEvent_t ev;
   {
-    std::lock_guard<std::mutex> g(p->mu);
+    std::unique_lock<std::mutex> lk(p->mu);
     const int idx = p->find(layer);
     if (idx < 0) return fail(NF4LS_INVALID_ARG, "nf4ls_wait: layer %d has no slot", layer);
+    NF4_TRY(p->wait_filled(lk, idx));
     ev = p->slot[idx].ready;
   }
   const auto t0 = std::chrono::steady_clock::now();
@@ -202,13 +522,34 @@ extern "C" int nf4ls_pool_get_stats(nf4ls_pool* p, nf4ls_pool_stats* out) {
 
 extern "C" int nf4ls_pool_synchronize(nf4ls_pool* p) {
   if (!p) return fail(NF4LS_INVALID_ARG, "null pool");
+  if (p->file) {
+    std::unique_lock<std::mutex> lk(p->mu);
+    p->file->cv_done.wait_for(lk, std::chrono::milliseconds(kFillWaitMs),
+                              [&] { return p->file->jobs.empty() || p->file->error != NF4LS_OK; });
+    if (p->file->error) return fail(p->file->error, "pool: disk source: %s", p->file->error_msg.c_str());
+  }
   NF4_CUDA_TRY(cudaStreamSynchronize(p->copy));
   return NF4LS_OK;
 }
 
 extern "C" int nf4ls_pool_destroy(nf4ls_pool* p) {
   if (!p) return NF4LS_OK;
+  if (p->file) {
+    {
+      std::lock_guard<std::mutex> g(p->mu);
+      p->file->stop = true;
+      p->file->cv_job.notify_all();
+    }
+    if (p->file->reader.joinable()) p->file->reader.join();
+  }
   if (p->copy) cudaStreamSynchronize(p->copy);
+  if (p->file) {
+    for (int b = 0; b < 2; ++b)
+      if (p->file->staged[b]) cudaEventDestroy(p->file->staged[b]);
+    if (p->file->fd >= 0) close(p->file->fd);
+    delete p->file;
+    p->file = nullptr;
+  }
   for (auto& s : p->slot) {
     if (s.ready) cudaEventDestroy(s.ready);
     if (s.freed) cudaEventDestroy(s.freed);
