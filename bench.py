@@ -53,6 +53,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=128)
+    ap.add_argument("--shard-fetch", action="store_true",
+                    help="N > 1: each rank copies only the layers it owns (l %% N) over PCIe and the pools "
+                         "broadcast them to the other ranks over NVLink (NCCL)")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the resident (compute-only) timing and the batch-16 compute-bound point")
     return ap.parse_args()
@@ -295,6 +298,8 @@ def main():
             dist.barrier()
 
     m = api.StreamedModel(wl, depth=args.depth, resident=False)
+    if world > 1 and args.shard_fetch:
+        dp.share_layer_fetch(m)
     tok = wl.batch * wl.seq
     n_steps = args.warmup + args.steps
     ids = [dp.rank_token_ids(wl, rank, s) for s in range(n_steps)]
@@ -427,6 +432,7 @@ def main():
             "config": {"workload": wl.name, "global_batch": wl.batch * world, "seq_len": wl.seq,
                        "layers": wl.n_layers, "vocab": wl.vocab, "pool_depth": args.depth,
                        "parallelism": f"dp{world}", "l2": "inputs larger than L2 (3.6 GB streamed per pass)",
+                       "layer_fetch": "sharded (NCCL broadcast)" if (world > 1 and args.shard_fetch) else "per rank",
                        "gemm_path": "nf4 decode in the tcgen05 mainloop"},
             "roofline": {"bound": "tensor", "kernel": "k_gemm<decode> (NF4-decode tcgen05 GEMM, all launches)",
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
@@ -438,6 +444,7 @@ def main():
             "dense_gemm": {"launches_per_step": dense["launches"] / args.steps, "ms_per_step": dense["ms"] / args.steps,
                            "tflops": dense["flops"] / (dense["ms"] / 1000.0) / 1e12 if dense["ms"] > 0 else 0.0},
             "stream": {"h2d_bytes_per_step": copy_bytes,
+                       "peer_bytes_per_step": (st1["peer_bytes"] - st0["peer_bytes"]) / args.steps,
                        "h2d_gbs_over_step": copy_bytes / (ms_max / 1000.0) / 1e9,
                        "h2d_link_gbs": best,
                        "copy_ms_per_step_at_link_rate": copy_bytes / best / 1e6 if best else None,

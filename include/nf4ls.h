@@ -290,6 +290,7 @@ typedef struct {
     uint64_t copies;         /* layer copies issued                  */
     uint64_t hits;           /* acquisitions served without a copy   */
     uint64_t acquisitions;
+    uint64_t peer_bytes;     /* bytes received from other GPUs (shared fetch) */
 } nf4ls_pool_stats;
 
 int nf4ls_pool_create(const void* pinned_host, const size_t* layer_off, const size_t* layer_bytes,
@@ -312,6 +313,20 @@ int nf4ls_pool_set_poison(nf4ls_pool* pool, int on);
 int nf4ls_pool_get_stats(nf4ls_pool* pool, nf4ls_pool_stats* out);
 int nf4ls_pool_synchronize(nf4ls_pool* pool);
 int nf4ls_pool_destroy(nf4ls_pool* pool);
+
+/* ------------------------------------------------------------------ layer-sharded fetch
+ * Data-parallel ranks stream the same shards; since the step is bound by each GPU's
+ * host-to-device link, ranks can split the fetch: rank r's pool copies from its host
+ * store only the layers it owns (layer % world == r) and every slot fill becomes an
+ * NCCL broadcast of the layer from its owner's slot into the other ranks' slots, over
+ * NVLink, on the pool's copy stream.  The bytes in every slot are those a private
+ * copy would have brought, so results are unchanged.  Every rank's pool must see the
+ * same sequence of prefetch / stream_prefetch / release calls (a data-parallel step
+ * does), so that the broadcasts pair up; a pool with a file store cannot be shared.
+ * nf4ls_nccl_unique_id: rank 0 makes the id, the caller distributes it;
+ * nf4ls_pool_share: called by every rank at the same time (NCCL communicator set-up). */
+int nf4ls_nccl_unique_id(uint8_t id_out[128]);
+int nf4ls_pool_share(nf4ls_pool* pool, int rank, int world, const uint8_t id[128]);
 
 /* ------------------------------------------------------------------ disk stream source
  * [review] mechanism section: the frozen base lives in (pinned) host memory and falls

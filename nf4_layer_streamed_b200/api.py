@@ -288,7 +288,13 @@ class Pool:
     def stats(self) -> dict:
         s = B.PoolStats()
         B.call("nf4ls_pool_get_stats", self.handle, ctypes.byref(s))
-        return {"bytes_copied": s.bytes_copied, "copies": s.copies, "hits": s.hits, "acquisitions": s.acquisitions}
+        return {"bytes_copied": s.bytes_copied, "copies": s.copies, "hits": s.hits, "acquisitions": s.acquisitions,
+                "peer_bytes": s.peer_bytes}
+
+    def share(self, rank: int, world: int, nccl_id: bytes) -> None:
+        """Layer-sharded fetch across ranks (every rank calls this at the same time)."""
+        buf = (ctypes.c_uint8 * 128).from_buffer_copy(nccl_id)
+        B.call("nf4ls_pool_share", self.handle, rank, world, ctypes.cast(buf, ctypes.c_void_p))
 
     def synchronize(self) -> None:
         B.call("nf4ls_pool_synchronize", self.handle)
@@ -302,6 +308,12 @@ class Pool:
         """A uint8 view of the slot at device address ptr (for reading a streamed shard)."""
         off = ptr - self.slots.data_ptr()
         return self.slots[off: off + nbytes]
+
+
+def nccl_unique_id() -> bytes:
+    buf = (ctypes.c_uint8 * 128)()
+    B.call("nf4ls_nccl_unique_id", ctypes.cast(buf, ctypes.c_void_p))
+    return bytes(buf)
 
 
 def disk_probe(path: str, probe_bytes: int = 1 << 30) -> dict:

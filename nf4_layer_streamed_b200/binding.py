@@ -60,7 +60,7 @@ class Model(ctypes.Structure):
 
 class PoolStats(ctypes.Structure):
     _fields_ = [("bytes_copied", ctypes.c_uint64), ("copies", ctypes.c_uint64), ("hits", ctypes.c_uint64),
-                ("acquisitions", ctypes.c_uint64)]
+                ("acquisitions", ctypes.c_uint64), ("peer_bytes", ctypes.c_uint64)]
 
 
 class DiskInfo(ctypes.Structure):
@@ -108,6 +108,8 @@ SIGNATURES = {
     "nf4ls_pool_get_stats": (ctypes.c_int, [P, ctypes.POINTER(PoolStats)]),
     "nf4ls_pool_synchronize": (ctypes.c_int, [P]),
     "nf4ls_pool_destroy": (ctypes.c_int, [P]),
+    "nf4ls_nccl_unique_id": (ctypes.c_int, [P]),
+    "nf4ls_pool_share": (ctypes.c_int, [P, ctypes.c_int, ctypes.c_int, P]),
     "nf4ls_disk_probe": (ctypes.c_int, [ctypes.c_char_p, SZ, ctypes.POINTER(DiskInfo)]),
     "nf4ls_disk_accept": (ctypes.c_int, [ctypes.POINTER(DiskInfo), ctypes.c_double]),
     "nf4ls_choose_source": (ctypes.c_int, [SZ, SZ, ctypes.POINTER(ctypes.c_int32)]),

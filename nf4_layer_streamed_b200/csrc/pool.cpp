@@ -20,7 +20,9 @@
 // store is a file, a reader thread reads each requested layer into one of two
 // caller-owned pinned staging buffers and enqueues its copy into the slot on the copy
 // stream; the slot rules above are unchanged.
+#include <dlfcn.h>
 #include <fcntl.h>
+#include <nccl.h>
 #include <sys/stat.h>
 #include <sys/sysmacros.h>
 #include <unistd.h>
@@ -68,6 +70,34 @@ int read_range(int fd, bool direct, uint8_t* dst, size_t cap, size_t off, size_t
 
 }  // namespace
 
+// NCCL, resolved at run time from the copy already in the process (the one torch
+// loaded) or else from the system's libnccl.so.2.
+struct NcclApi {
+  ncclResult_t (*get_unique_id)(ncclUniqueId*) = nullptr;
+  ncclResult_t (*comm_init_rank)(ncclComm_t*, int, ncclUniqueId, int) = nullptr;
+  ncclResult_t (*broadcast)(const void*, void*, size_t, ncclDataType_t, int, ncclComm_t, cudaStream_t) = nullptr;
+  ncclResult_t (*comm_destroy)(ncclComm_t) = nullptr;
+  const char* (*error_string)(ncclResult_t) = nullptr;
+  bool ok = false;
+};
+
+const NcclApi& nccl_api() {
+  static NcclApi a = [] {
+    NcclApi r;
+    void* h = dlopen("libnccl.so.2", RTLD_NOW | RTLD_NOLOAD);
+    if (!h) h = dlopen("libnccl.so.2", RTLD_NOW);
+    if (!h) return r;
+    r.get_unique_id = reinterpret_cast<decltype(r.get_unique_id)>(dlsym(h, "ncclGetUniqueId"));
+    r.comm_init_rank = reinterpret_cast<decltype(r.comm_init_rank)>(dlsym(h, "ncclCommInitRank"));
+    r.broadcast = reinterpret_cast<decltype(r.broadcast)>(dlsym(h, "ncclBroadcast"));
+    r.comm_destroy = reinterpret_cast<decltype(r.comm_destroy)>(dlsym(h, "ncclCommDestroy"));
+    r.error_string = reinterpret_cast<decltype(r.error_string)>(dlsym(h, "ncclGetErrorString"));
+    r.ok = r.get_unique_id && r.comm_init_rank && r.broadcast && r.comm_destroy && r.error_string;
+    return r;
+  }();
+  return a;
+}
+
 struct FileSource {
   int fd = -1;
   bool direct = false;
@@ -111,6 +141,9 @@ struct nf4ls_pool {
   nf4ls_pool_stats stats{};
   std::mutex mu;
   FileSource* file = nullptr;
+  // layer-sharded fetch: the owner of layer l is rank l % world
+  ncclComm_t comm = nullptr;
+  int rank = 0, world = 1;
 
   int find(int layer) const {
     for (int i = 0; i < depth; ++i)
@@ -153,12 +186,21 @@ struct nf4ls_pool {
     }
     if (s.freed_recorded) NF4_CUDA_TRY(cudaStreamWaitEvent(copy, s.freed, 0));
     if (poison) NF4_CUDA_TRY(cudaMemsetAsync(dst, 0xFF, slot_bytes, copy));
-    NF4_CUDA_TRY(cudaMemcpyAsync(dst, store + off[layer], bytes[layer], cudaMemcpyHostToDevice, copy));
+    const int owner = layer % world;
+    if (owner == rank) {
+      NF4_CUDA_TRY(cudaMemcpyAsync(dst, store + off[layer], bytes[layer], cudaMemcpyHostToDevice, copy));
+      stats.bytes_copied += bytes[layer];
+      stats.copies += 1;
+    }
+    if (comm) {  // from the owner's slot into every other rank's slot, in place
+      const ncclResult_t r = nccl_api().broadcast(dst, dst, bytes[layer], ncclUint8, owner, comm, copy);
+      if (r != ncclSuccess) return fail(NF4LS_CUDA, "pool: NCCL broadcast of layer %d: %s", layer,
+                                        nccl_api().error_string(r));
+      if (owner != rank) stats.peer_bytes += bytes[layer];
+    }
     NF4_CUDA_TRY(cudaEventRecord(s.ready, copy));
     s.layer = layer;
     s.pending = true;
-    stats.bytes_copied += bytes[layer];
-    stats.copies += 1;
     *out_idx = i;
     return NF4LS_OK;
   }
@@ -363,6 +405,42 @@ extern "C" int nf4ls_pool_create_file(const char* path, const size_t* layer_off,
   return NF4LS_OK;
 }
 
+extern "C" int nf4ls_nccl_unique_id(uint8_t id_out[128]) {
+  clear_error();
+  if (!id_out) return fail(NF4LS_INVALID_ARG, "nf4ls_nccl_unique_id: null output");
+  const NcclApi& n = nccl_api();
+  if (!n.ok) return fail(NF4LS_CUDA, "nf4ls_nccl_unique_id: libnccl.so.2 not found");
+  ncclUniqueId id;
+  const ncclResult_t r = n.get_unique_id(&id);
+  if (r != ncclSuccess) return fail(NF4LS_CUDA, "ncclGetUniqueId: %s", n.error_string(r));
+  static_assert(sizeof(id) == 128, "NCCL unique id size");
+  std::memcpy(id_out, &id, sizeof(id));
+  return NF4LS_OK;
+}
+
+extern "C" int nf4ls_pool_share(nf4ls_pool* p, int rank, int world, const uint8_t id[128]) {
+  clear_error();
+  if (!p || !id || world < 1 || rank < 0 || rank >= world)
+    return fail(NF4LS_INVALID_ARG, "nf4ls_pool_share: bad argument (rank %d, world %d)", rank, world);
+  std::lock_guard<std::mutex> g(p->mu);
+  if (p->file) return fail(NF4LS_INVALID_ARG, "nf4ls_pool_share: a pool with a file store cannot be shared");
+  if (p->comm) return fail(NF4LS_INVALID_ARG, "nf4ls_pool_share: already shared");
+  for (const auto& s : p->slot)
+    if (s.layer >= 0) return fail(NF4LS_INVALID_ARG, "nf4ls_pool_share: the pool must not hold a layer yet");
+  const NcclApi& n = nccl_api();
+  if (!n.ok) return fail(NF4LS_CUDA, "nf4ls_pool_share: libnccl.so.2 not found");
+  NF4_CUDA_TRY(cudaSetDevice(p->device));
+  ncclUniqueId uid;
+  std::memcpy(&uid, id, sizeof(uid));
+  ncclComm_t comm = nullptr;
+  const ncclResult_t r = n.comm_init_rank(&comm, world, uid, rank);
+  if (r != ncclSuccess) return fail(NF4LS_CUDA, "ncclCommInitRank: %s", n.error_string(r));
+  p->comm = comm;
+  p->rank = rank;
+  p->world = world;
+  return NF4LS_OK;
+}
+
 extern "C" int nf4ls_disk_probe(const char* path, size_t probe_bytes, nf4ls_disk_info* out) {
   clear_error();
   if (!path || !out || probe_bytes == 0) return fail(NF4LS_INVALID_ARG, "nf4ls_disk_probe: bad argument");
@@ -543,6 +621,7 @@ extern "C" int nf4ls_pool_destroy(nf4ls_pool* p) {
     if (p->file->reader.joinable()) p->file->reader.join();
   }
   if (p->copy) cudaStreamSynchronize(p->copy);
+  if (p->comm) nccl_api().comm_destroy(p->comm);
   if (p->file) {
     for (int b = 0; b < 2; ++b)
       if (p->file->staged[b]) cudaEventDestroy(p->file->staged[b]);

@@ -8,6 +8,14 @@ itself stays per rank and needs no collective.
 
 The model object needs ``forward_backward(ids) -> loss``, a flat fp32 ``grads``
 tensor and ``adamw_step()``; ``api.StreamedModel`` provides them.
+
+Layer-sharded fetch (optional, ``share_layer_fetch``): the step is bound by each
+GPU's host-to-device link, so the ranks can split the layer stream -- the owner of
+layer l (rank l % world) copies it from its host store and the library's pool
+broadcasts it from the owner's slot into the other ranks' slots with NCCL over
+NVLink.  Each rank then moves 1/world of the bytes over PCIe; the slot contents,
+hence the results, do not change.  ``emulate_sharded_fetch`` runs the same schedule
+on host byte arrays with any torch.distributed backend (the CPU tests use gloo).
 """
 from __future__ import annotations
 
@@ -39,3 +47,42 @@ class DataParallelStep:
                 m.grads.mul_(1.0 / self.world)
         m.adamw_step()
         return loss
+
+
+def owner(layer: int, world: int) -> int:
+    """The rank that copies `layer` from its host store in the layer-sharded fetch."""
+    return layer % world
+
+
+def share_layer_fetch(model, group=None, share=None) -> bytes:
+    """Switch every rank's layer pool to the sharded fetch.  Rank 0 makes the NCCL id,
+    the process group carries it to the others, then all ranks call the pool's share
+    (NCCL communicator set-up) together.  `share(rank, world, nccl_id)` defaults to
+    model.pool.share.  Returns the id."""
+    from . import api
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    box = [api.nccl_unique_id() if rank == 0 else None]
+    dist.broadcast_object_list(box, src=0, group=group)
+    nccl_id = box[0]
+    (share or model.pool.share)(rank, world, nccl_id)
+    return nccl_id
+
+
+def emulate_sharded_fetch(store: torch.Tensor, offsets, sizes, order, group=None):
+    """Host model of the pool's sharded fetch: for each layer in `order` (the sequence of
+    slot fills, identical on every rank) the owner takes the bytes from its store and
+    broadcasts them; the others receive.  Returns (the bytes every rank ended with per
+    layer, the layers this rank read from its own store)."""
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    got, own_reads = {}, []
+    for layer in order:
+        src = owner(layer, world)
+        buf = torch.empty(sizes[layer], dtype=torch.uint8)
+        if rank == src:
+            buf.copy_(store[offsets[layer]:offsets[layer] + sizes[layer]])
+            own_reads.append(layer)
+        dist.broadcast(buf, src=src, group=group)
+        got[layer] = buf
+    return got, own_reads

@@ -128,3 +128,13 @@ def test_streamed_head_config_checked_on_host():
     res = B.lib().nf4ls_model_workspace_bytes(ctypes.byref(cfg_res))
     strm = B.lib().nf4ls_model_workspace_bytes(ctypes.byref(cfg_str))
     assert strm < res
+
+
+def test_layer_sharded_fetch_arguments_on_host():
+    nid = api.nccl_unique_id()
+    assert len(nid) == 128 and any(nid)
+    buf = (ctypes.c_uint8 * 128).from_buffer_copy(nid)
+    idp = ctypes.cast(buf, ctypes.c_void_p)
+    assert B.call_status("nf4ls_pool_share", None, 0, 2, idp) == -1
+    assert B.call_status("nf4ls_pool_share", ctypes.c_void_p(256), 2, 2, idp) == -1
+    assert B.call_status("nf4ls_pool_share", ctypes.c_void_p(256), 0, 0, idp) == -1

@@ -93,3 +93,51 @@ def test_data_parallel_step_two_ranks_gloo():
         ref.grads.copy_(sum(gs) / world)
         ref.adamw_step()
     np.testing.assert_allclose(res[0][0], ref.lora.numpy(), rtol=0, atol=1e-15)
+
+
+def _fetch_worker(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        n_layers, size = 7, 4096
+        g = torch.Generator().manual_seed(11)
+        store = torch.randint(0, 256, (n_layers * size,), generator=g, dtype=torch.uint8)  # same on all ranks
+        offs = [i * size for i in range(n_layers)]
+        sizes = [size - 17 * i for i in range(n_layers)]
+        # the fill order of a 7-layer step at depth 2: forward 0..6, backward 4..0
+        order = list(range(n_layers)) + list(range(n_layers - 3, -1, -1))
+        got, reads = dp.emulate_sharded_fetch(store, offs, sizes, order)
+        ok = all(torch.equal(got[l], store[offs[l]:offs[l] + sizes[l]]) for l in got)
+        ids = []
+        dp.share_layer_fetch(None, share=lambda r, w, i: ids.append((r, w, i)))
+        q.put((rank, ok, reads, ids[0]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_layer_sharded_fetch_two_ranks_gloo():
+    """Every rank ends with every layer's bytes while reading only the layers it owns
+    (l % world == rank) from its own store, and all ranks get the same NCCL id."""
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_fetch_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = {}
+    for _ in range(world):
+        r, ok, reads, share_args = q.get(timeout=120)
+        res[r] = (ok, reads, share_args)
+    for p in procs:
+        p.join(30)
+        assert p.exitcode == 0
+    for r in range(world):
+        ok, reads, (rr, w, nccl_id) = res[r]
+        assert ok
+        assert all(l % world == r for l in reads) and reads
+        assert rr == r and w == world and len(nccl_id) == 128
+    assert res[0][2][2] == res[1][2][2]
+    # the fetch is split: together the ranks read each of the 12 fills exactly once
+    assert len(res[0][1]) + len(res[1][1]) == 7 + 5
