@@ -42,6 +42,23 @@ __device__ __forceinline__ void load_tile(uint32_t dst, const __nv_bfloat16* src
   }
 }
 
+// Group-local cp.async tile load: threads t of n.
+template <int D>
+__device__ __forceinline__ void load_tile_part(uint32_t dst, const __nv_bfloat16* src, int ld, int t, int n) {
+  constexpr int CH = D / 8;
+  for (int i = t; i < 64 * CH; i += n) {
+    const int r = i / CH, c = i % CH;
+    cp_async16(dst + (r * Tile<D>::RS + c * 8) * 2, src + (size_t)r * ld + c * 8);
+  }
+}
+
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bar_group(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+
 // A fragment (16x16 at row0, col0) of a row-major tile.
 template <int D>
 __device__ __forceinline__ void frag_a(uint32_t tile, int row0, int col0, uint32_t (&a)[4]) {
@@ -71,21 +88,31 @@ __global__ void __launch_bounds__(128) k_attn_fwd(const __nv_bfloat16* __restric
                                                   __nv_bfloat16* __restrict__ o, int ldo, float* __restrict__ lse,
                                                   int seq, int nq, int nkv, float scale_log2) {
   extern __shared__ __align__(16) uint8_t sm[];
-  const uint32_t sQ = smem_u32(sm), sK = sQ + Tile<D>::BYTES, sV = sK + Tile<D>::BYTES;
-  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  // Q, then two K/V buffers: the next key tile loads while this one is used
+  const uint32_t sQ = smem_u32(sm);
+  const int qt = gridDim.x - 1 - blockIdx.x, h = blockIdx.y, b = blockIdx.z;  // longest rows first
   const int kvh = h / (nq / nkv);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c2 = (lane & 3) * 2;
   const size_t row0 = (size_t)b * seq;
   load_tile<D>(sQ, q + (row0 + qt * TQ) * ldq + h * D, ldq);
+  load_tile<D>(sQ + Tile<D>::BYTES, k + row0 * ldkv + kvh * D, ldkv);
+  load_tile<D>(sQ + 2 * Tile<D>::BYTES, v + row0 * ldkv + kvh * D, ldkv);
+  cp_commit();
   float acc[D / 8][4];
 #pragma unroll
   for (int i = 0; i < D / 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
   float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
   for (int kt = 0; kt <= qt; ++kt) {
-    __syncthreads();
-    load_tile<D>(sK, k + (row0 + kt * TK) * ldkv + kvh * D, ldkv);
-    load_tile<D>(sV, v + (row0 + kt * TK) * ldkv + kvh * D, ldkv);
-    cp_async_wait_all();
+    const uint32_t sK = sQ + (1 + 2 * (kt & 1)) * Tile<D>::BYTES, sV = sK + Tile<D>::BYTES;
+    if (kt < qt) {  // the buffer of tile kt + 1 was last read in iteration kt - 1 (barrier below)
+      const uint32_t nK = sQ + (1 + 2 * ((kt + 1) & 1)) * Tile<D>::BYTES;
+      load_tile<D>(nK, k + (row0 + (kt + 1) * TK) * ldkv + kvh * D, ldkv);
+      load_tile<D>(nK + Tile<D>::BYTES, v + (row0 + (kt + 1) * TK) * ldkv + kvh * D, ldkv);
+      cp_commit();
+      cp_wait<1>();
+    } else {
+      cp_wait<0>();
+    }
     __syncthreads();
     float s[8][4];
 #pragma unroll
@@ -156,6 +183,7 @@ __global__ void __launch_bounds__(128) k_attn_fwd(const __nv_bfloat16* __restric
         mma16816(acc[2 * n2 + 1], a0, a1, a2, a3, bb[2], bb[3]);
       }
     }
+    __syncthreads();
   }
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
@@ -207,14 +235,18 @@ __global__ void __launch_bounds__(128) k_attn_dq(const __nv_bfloat16* __restrict
                                                  __nv_bfloat16* __restrict__ dq, int ld_dq, int seq, int nq, int nkv,
                                                  float scale) {
   extern __shared__ __align__(16) uint8_t sm[];
-  const uint32_t sQ = smem_u32(sm), sO = sQ + Tile<D>::BYTES, sK = sO + Tile<D>::BYTES, sV = sK + Tile<D>::BYTES;
-  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  // Q, dO, then two K/V buffers: the next key tile loads while this one is used
+  const uint32_t sQ = smem_u32(sm), sO = sQ + Tile<D>::BYTES;
+  const int qt = gridDim.x - 1 - blockIdx.x, h = blockIdx.y, b = blockIdx.z;  // longest rows first
   const int kvh = h / (nq / nkv);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c2 = (lane & 3) * 2;
   const size_t row0 = (size_t)b * seq;
   const float scale_log2 = scale * kLog2e;
   load_tile<D>(sQ, q + (row0 + qt * TQ) * ldq + h * D, ldq);
   load_tile<D>(sO, dout + (row0 + qt * TQ) * ldo + h * D, ldo);
+  load_tile<D>(sQ + 2 * Tile<D>::BYTES, k + row0 * ldkv + kvh * D, ldkv);
+  load_tile<D>(sQ + 3 * Tile<D>::BYTES, v + row0 * ldkv + kvh * D, ldkv);
+  cp_commit();
   const int qr = qt * TQ + warp * 16 + g;
   const float* Lh = lse + ((size_t)b * nq + h) * seq;
   const float* Dh = delta + ((size_t)b * nq + h) * seq;
@@ -224,10 +256,16 @@ __global__ void __launch_bounds__(128) k_attn_dq(const __nv_bfloat16* __restrict
 #pragma unroll
   for (int i = 0; i < D / 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
   for (int kt = 0; kt <= qt; ++kt) {
-    __syncthreads();
-    load_tile<D>(sK, k + (row0 + kt * TK) * ldkv + kvh * D, ldkv);
-    load_tile<D>(sV, v + (row0 + kt * TK) * ldkv + kvh * D, ldkv);
-    cp_async_wait_all();
+    const uint32_t sK = sQ + (2 + 2 * (kt & 1)) * Tile<D>::BYTES, sV = sK + Tile<D>::BYTES;
+    if (kt < qt) {
+      const uint32_t nK = sQ + (2 + 2 * ((kt + 1) & 1)) * Tile<D>::BYTES;
+      load_tile<D>(nK, k + (row0 + (kt + 1) * TK) * ldkv + kvh * D, ldkv);
+      load_tile<D>(nK + Tile<D>::BYTES, v + (row0 + (kt + 1) * TK) * ldkv + kvh * D, ldkv);
+      cp_commit();
+      cp_wait<1>();
+    } else {
+      cp_wait<0>();
+    }
     __syncthreads();
     float s[8][4], dp[8][4];
 #pragma unroll
@@ -274,6 +312,7 @@ __global__ void __launch_bounds__(128) k_attn_dq(const __nv_bfloat16* __restrict
         mma16816(acc[2 * n2 + 1], a0, a1, a2, a3, bb[2], bb[3]);
       }
     }
+    __syncthreads();
   }
   __nv_bfloat16* o0 = dq + (row0 + qr) * ld_dq + h * D;
   __nv_bfloat16* o1 = o0 + 8 * (size_t)ld_dq;
@@ -284,102 +323,145 @@ __global__ void __launch_bounds__(128) k_attn_dq(const __nv_bfloat16* __restrict
   }
 }
 
+// dK, dV of one 64-key tile of one kv head: two groups of 4 warps split the work
+// (query heads of the group x query tiles at or after the key tile; group w takes the
+// tiles kt + w, kt + w + 2, ...), each group double-buffers its Q / dO tiles so the
+// next pair loads while this one is used, and the two partial sums are added in a
+// fixed order (group 0 + group 1) at the end.
 template <int D>
-__global__ void __launch_bounds__(128, 1) k_attn_dkv(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+__global__ void __launch_bounds__(256, 1) k_attn_dkv(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                                                      const __nv_bfloat16* __restrict__ v, int ldq, int ldkv,
                                                      const __nv_bfloat16* __restrict__ dout, int ldo,
                                                      const float* __restrict__ lse, const float* __restrict__ delta,
                                                      __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
                                                      int ld_dkv, int seq, int nq, int nkv, float scale) {
+  constexpr int T = Tile<D>::BYTES;
   extern __shared__ __align__(16) uint8_t sm[];
-  const uint32_t sK = smem_u32(sm), sV = sK + Tile<D>::BYTES, sQ = sV + Tile<D>::BYTES, sO = sQ + Tile<D>::BYTES;
-  float* sL = reinterpret_cast<float*>(sm + 4 * Tile<D>::BYTES);
-  float* sD = sL + 64;
-  const int kt = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const uint32_t sK = smem_u32(sm), sV = sK + T;
+  const int kvh = blockIdx.x, b = blockIdx.y, kt = blockIdx.z;  // z slowest: the longest key tiles start first
   const int grp = nq / nkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c2 = (lane & 3) * 2;
+  const int wg = warp >> 2, wq = warp & 3, tg = threadIdx.x & 127;
   const size_t row0 = (size_t)b * seq;
   const float scale_log2 = scale * kLog2e;
   const int n_qt = seq / TQ;
+  const int per_head = (n_qt - kt - wg + 1) / 2;  // query tiles kt + wg + 2j of this group
+  const int n_it = per_head > 0 ? grp * per_head : 0;
+  // buffer j of this group: Q, dO tiles and the 64 lse / delta values
+  auto buf_q = [&](int j) { return sK + (2 + wg * 4 + j * 2) * T; };
+  float* ld_base = reinterpret_cast<float*>(sm + 10 * T) + (wg * 2) * 128;
+  auto load_item = [&](int i, int j) {
+    const int hh = i / per_head, qt = kt + wg + 2 * (i % per_head);
+    const int h = kvh * grp + hh;
+    const uint32_t bq = buf_q(j);
+    load_tile_part<D>(bq, q + (row0 + qt * TQ) * ldq + h * D, ldq, tg, 128);
+    load_tile_part<D>(bq + T, dout + (row0 + qt * TQ) * ldo + h * D, ldo, tg, 128);
+    if (tg < 32) {  // 64 lse then 64 delta values, 16 bytes per thread
+      const float* src = (tg < 16 ? lse : delta) + ((size_t)b * nq + h) * seq + qt * TQ + (tg & 15) * 4;
+      cp_async16(smem_u32(ld_base + j * 128 + (tg < 16 ? 0 : 64) + (tg & 15) * 4), src);
+    }
+  };
   load_tile<D>(sK, k + (row0 + kt * TK) * ldkv + kvh * D, ldkv);
   load_tile<D>(sV, v + (row0 + kt * TK) * ldkv + kvh * D, ldkv);
+  if (n_it > 0) load_item(0, 0);
+  cp_commit();
+  cp_wait<0>();
+  __syncthreads();
   float dK[D / 8][4], dV[D / 8][4];
 #pragma unroll
   for (int i = 0; i < D / 8; ++i)
 #pragma unroll
     for (int e = 0; e < 4; ++e) dK[i][e] = dV[i][e] = 0.f;
-  for (int hh = 0; hh < grp; ++hh) {
-    const int h = kvh * grp + hh;
-    const float* Lh = lse + ((size_t)b * nq + h) * seq;
-    const float* Dh = delta + ((size_t)b * nq + h) * seq;
-    for (int qt = kt; qt < n_qt; ++qt) {
-      __syncthreads();
-      load_tile<D>(sQ, q + (row0 + qt * TQ) * ldq + h * D, ldq);
-      load_tile<D>(sO, dout + (row0 + qt * TQ) * ldo + h * D, ldo);
-      if (threadIdx.x < 64) {
-        sL[threadIdx.x] = Lh[qt * TQ + threadIdx.x] * kLog2e;
-        sD[threadIdx.x] = Dh[qt * TQ + threadIdx.x];
-      }
-      cp_async_wait_all();
-      __syncthreads();
-      // S^T = K Q^T and dP^T = V dO^T for this warp's 16 keys x 64 queries
-      float s[8][4], dp[8][4];
+  for (int it = 0; it < n_it; ++it) {
+    const int j = it & 1;
+    if (it + 1 < n_it) {
+      load_item(it + 1, j ^ 1);
+      cp_commit();
+    }
+    const int qt = kt + wg + 2 * (it % per_head);
+    const uint32_t sQ = buf_q(j), sO = sQ + T;
+    const float* sL = ld_base + j * 128;
+    const float* sD = sL + 64;
+    // S^T = K Q^T and dP^T = V dO^T for this warp's 16 keys x 64 queries
+    float s[8][4], dp[8][4];
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) s[i][e] = dp[i][e] = 0.f;
+      for (int e = 0; e < 4; ++e) s[i][e] = dp[i][e] = 0.f;
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        uint32_t ak[4], av[4];
-        frag_a<D>(sK, warp * 16, kk * 16, ak);
-        frag_a<D>(sV, warp * 16, kk * 16, av);
+    for (int kk = 0; kk < D / 16; ++kk) {
+      uint32_t ak[4], av[4];
+      frag_a<D>(sK, wq * 16, kk * 16, ak);
+      frag_a<D>(sV, wq * 16, kk * 16, av);
 #pragma unroll
-        for (int n2 = 0; n2 < 4; ++n2) {
-          uint32_t bq[4], bo[4];
-          frag_b_rows_n<D>(sQ, n2 * 16, kk * 16, bq);
-          frag_b_rows_n<D>(sO, n2 * 16, kk * 16, bo);
-          mma16816(s[2 * n2], ak[0], ak[1], ak[2], ak[3], bq[0], bq[1]);
-          mma16816(s[2 * n2 + 1], ak[0], ak[1], ak[2], ak[3], bq[2], bq[3]);
-          mma16816(dp[2 * n2], av[0], av[1], av[2], av[3], bo[0], bo[1]);
-          mma16816(dp[2 * n2 + 1], av[0], av[1], av[2], av[3], bo[2], bo[3]);
-        }
-      }
-      // P^T and dS^T; column e&1 of n-tile nt is query nt*8 + c2 + (e&1)
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int qj = nt * 8 + c2 + (e & 1);
-          float p = exp2f(s[nt][e] * scale_log2 - sL[qj]);
-          if (qt == kt) {
-            const int ki = warp * 16 + g + (e >> 1) * 8;
-            if (ki > qj) p = 0.f;
-          }
-          s[nt][e] = p;
-          dp[nt][e] = p * (dp[nt][e] - sD[qj]);
-        }
-#pragma unroll
-      for (int kb = 0; kb < 4; ++kb) {
-        const uint32_t p0 = pack_bf16x2(s[2 * kb][0], s[2 * kb][1]), p1 = pack_bf16x2(s[2 * kb][2], s[2 * kb][3]);
-        const uint32_t p2 = pack_bf16x2(s[2 * kb + 1][0], s[2 * kb + 1][1]),
-                       p3 = pack_bf16x2(s[2 * kb + 1][2], s[2 * kb + 1][3]);
-        const uint32_t d0 = pack_bf16x2(dp[2 * kb][0], dp[2 * kb][1]), d1 = pack_bf16x2(dp[2 * kb][2], dp[2 * kb][3]);
-        const uint32_t d2 = pack_bf16x2(dp[2 * kb + 1][0], dp[2 * kb + 1][1]),
-                       d3 = pack_bf16x2(dp[2 * kb + 1][2], dp[2 * kb + 1][3]);
-#pragma unroll
-        for (int n2 = 0; n2 < D / 16; ++n2) {
-          uint32_t bo[4], bq[4];
-          frag_b_rows_k<D>(sO, kb * 16, n2 * 16, bo);
-          frag_b_rows_k<D>(sQ, kb * 16, n2 * 16, bq);
-          mma16816(dV[2 * n2], p0, p1, p2, p3, bo[0], bo[1]);
-          mma16816(dV[2 * n2 + 1], p0, p1, p2, p3, bo[2], bo[3]);
-          mma16816(dK[2 * n2], d0, d1, d2, d3, bq[0], bq[1]);
-          mma16816(dK[2 * n2 + 1], d0, d1, d2, d3, bq[2], bq[3]);
-        }
+      for (int n2 = 0; n2 < 4; ++n2) {
+        uint32_t bq[4], bo[4];
+        frag_b_rows_n<D>(sQ, n2 * 16, kk * 16, bq);
+        frag_b_rows_n<D>(sO, n2 * 16, kk * 16, bo);
+        mma16816(s[2 * n2], ak[0], ak[1], ak[2], ak[3], bq[0], bq[1]);
+        mma16816(s[2 * n2 + 1], ak[0], ak[1], ak[2], ak[3], bq[2], bq[3]);
+        mma16816(dp[2 * n2], av[0], av[1], av[2], av[3], bo[0], bo[1]);
+        mma16816(dp[2 * n2 + 1], av[0], av[1], av[2], av[3], bo[2], bo[3]);
       }
     }
+    // P^T and dS^T; column e&1 of n-tile nt is query nt*8 + c2 + (e&1)
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int qj = nt * 8 + c2 + (e & 1);
+        float p = exp2f(s[nt][e] * scale_log2 - sL[qj] * kLog2e);
+        if (qt == kt) {
+          const int ki = wq * 16 + g + (e >> 1) * 8;
+          if (ki > qj) p = 0.f;
+        }
+        s[nt][e] = p;
+        dp[nt][e] = p * (dp[nt][e] - sD[qj]);
+      }
+#pragma unroll
+    for (int kb = 0; kb < 4; ++kb) {
+      const uint32_t p0 = pack_bf16x2(s[2 * kb][0], s[2 * kb][1]), p1 = pack_bf16x2(s[2 * kb][2], s[2 * kb][3]);
+      const uint32_t p2 = pack_bf16x2(s[2 * kb + 1][0], s[2 * kb + 1][1]),
+                     p3 = pack_bf16x2(s[2 * kb + 1][2], s[2 * kb + 1][3]);
+      const uint32_t d0 = pack_bf16x2(dp[2 * kb][0], dp[2 * kb][1]), d1 = pack_bf16x2(dp[2 * kb][2], dp[2 * kb][3]);
+      const uint32_t d2 = pack_bf16x2(dp[2 * kb + 1][0], dp[2 * kb + 1][1]),
+                     d3 = pack_bf16x2(dp[2 * kb + 1][2], dp[2 * kb + 1][3]);
+#pragma unroll
+      for (int n2 = 0; n2 < D / 16; ++n2) {
+        uint32_t bo[4], bq[4];
+        frag_b_rows_k<D>(sO, kb * 16, n2 * 16, bo);
+        frag_b_rows_k<D>(sQ, kb * 16, n2 * 16, bq);
+        mma16816(dV[2 * n2], p0, p1, p2, p3, bo[0], bo[1]);
+        mma16816(dV[2 * n2 + 1], p0, p1, p2, p3, bo[2], bo[3]);
+        mma16816(dK[2 * n2], d0, d1, d2, d3, bq[0], bq[1]);
+        mma16816(dK[2 * n2 + 1], d0, d1, d2, d3, bq[2], bq[3]);
+      }
+    }
+    if (it + 1 < n_it) cp_wait<0>();
+    bar_group(1 + wg, 128);  // the next item is in; nobody still reads this buffer
   }
-  const int kr = kt * TK + warp * 16 + g;
+  // group 1 hands its partial sums to group 0 through the (now free) tile memory
+  __syncthreads();
+  float* red = reinterpret_cast<float*>(sm + 2 * T);  // [D/8 * 4 * 2][128], thread-major
+  if (wg == 1) {
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        red[((i * 4 + e) * 2 + 0) * 128 + tg] = dK[i][e];
+        red[((i * 4 + e) * 2 + 1) * 128 + tg] = dV[i][e];
+      }
+  }
+  __syncthreads();
+  if (wg == 1) return;
+#pragma unroll
+  for (int i = 0; i < D / 8; ++i)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      dK[i][e] += red[((i * 4 + e) * 2 + 0) * 128 + tg];
+      dV[i][e] += red[((i * 4 + e) * 2 + 1) * 128 + tg];
+    }
+  const int kr = kt * TK + wq * 16 + g;
   __nv_bfloat16* k0 = dk + (row0 + kr) * ld_dkv + kvh * D;
   __nv_bfloat16* v0 = dv + (row0 + kr) * ld_dkv + kvh * D;
   const size_t step = 8 * (size_t)ld_dkv;
@@ -414,12 +496,12 @@ int attention_fwd(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfl
   const float scale_log2 = (1.0f / sqrtf((float)d)) * kLog2e;
   dim3 grid(seq / TQ, nq, batch);
   if (d == 128) {
-    const int sm = 3 * Tile<128>::BYTES;
+    const int sm = 5 * Tile<128>::BYTES;
     NF4_TRY(set_smem(k_attn_fwd<128>, sm));
     k_attn_fwd<128><<<grid, 128, sm, s>>>(q, k, v, ldq, ldkv, o, ldo, lse, seq, nq, nkv, scale_log2);
     note_launch();
   } else {
-    const int sm = 3 * Tile<64>::BYTES;
+    const int sm = 5 * Tile<64>::BYTES;
     NF4_TRY(set_smem(k_attn_fwd<64>, sm));
     k_attn_fwd<64><<<grid, 128, sm, s>>>(q, k, v, ldq, ldkv, o, ldo, lse, seq, nq, nkv, scale_log2);
     note_launch();
@@ -437,22 +519,22 @@ int attention_bwd(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfl
   const float scale = 1.0f / sqrtf((float)d);
   k_attn_delta<<<(M * nq + 7) / 8, 256, 0, s>>>(o, dout, ldo, M, seq, nq, d, delta);
   note_launch();
-  dim3 gq(seq / TQ, nq, batch), gk(seq / TK, nkv, batch);
+  dim3 gq(seq / TQ, nq, batch), gk(nkv, batch, seq / TK);
   if (d == 128) {
-    const int sq = 4 * Tile<128>::BYTES, sk = 4 * Tile<128>::BYTES + 512;
+    const int sq = 6 * Tile<128>::BYTES, sk = 10 * Tile<128>::BYTES + 2048;
     NF4_TRY(set_smem(k_attn_dq<128>, sq));
     NF4_TRY(set_smem(k_attn_dkv<128>, sk));
     k_attn_dq<128><<<gq, 128, sq, s>>>(q, k, v, ldq, ldkv, dout, ldo, lse, delta, dq, ld_dq, seq, nq, nkv, scale);
     note_launch();
-    k_attn_dkv<128><<<gk, 128, sk, s>>>(q, k, v, ldq, ldkv, dout, ldo, lse, delta, dk, dv, ld_dkv, seq, nq, nkv, scale);
+    k_attn_dkv<128><<<gk, 256, sk, s>>>(q, k, v, ldq, ldkv, dout, ldo, lse, delta, dk, dv, ld_dkv, seq, nq, nkv, scale);
     note_launch();
   } else {
-    const int sq = 4 * Tile<64>::BYTES, sk = 4 * Tile<64>::BYTES + 512;
+    const int sq = 6 * Tile<64>::BYTES, sk = 10 * Tile<64>::BYTES + 2048;
     NF4_TRY(set_smem(k_attn_dq<64>, sq));
     NF4_TRY(set_smem(k_attn_dkv<64>, sk));
     k_attn_dq<64><<<gq, 128, sq, s>>>(q, k, v, ldq, ldkv, dout, ldo, lse, delta, dq, ld_dq, seq, nq, nkv, scale);
     note_launch();
-    k_attn_dkv<64><<<gk, 128, sk, s>>>(q, k, v, ldq, ldkv, dout, ldo, lse, delta, dk, dv, ld_dkv, seq, nq, nkv, scale);
+    k_attn_dkv<64><<<gk, 256, sk, s>>>(q, k, v, ldq, ldkv, dout, ldo, lse, delta, dk, dv, ld_dkv, seq, nq, nkv, scale);
     note_launch();
   }
   NF4_CUDA_TRY(cudaGetLastError());
