@@ -2,7 +2,8 @@
 // device memory.
 //
 // nf4_quantize_tensor needs a scratch buffer of n/64 floats (the per-block absmax
-// values between the quantiser's passes), which its caller allocates.  Some callers
+// values between the quantiser's passes) plus 8 KB for its offset pass, which its
+// caller allocates.  Some callers
 // cannot: code running where the CUDA allocator is off limits (inside another
 // framework's memory pool or a host callback that must not allocate), or a process
 // that has handed all device memory to a pool it does not control.  This entry point
@@ -10,7 +11,7 @@
 // passes its input and output buffers.
 //
 // The array holds the absmax values of tensors up to kMaxElems weights (16 MiB of
-// device memory), and every GPU that loads the library holds its own copy until the
+// device memory, plus the offset pass's 8 KB), and every GPU that loads the library holds its own copy until the
 // process exits.  Host code cannot use the array's name as a device address; the
 // address is looked up once per device with cudaGetSymbolAddress, on the first call
 // made with that device current.  Make that first call before any stream capture.
@@ -26,7 +27,8 @@ namespace nf4ls {
 namespace {
 
 constexpr size_t kMaxElems = 1ull << 28;  // 268,435,456 weights
-static __device__ __align__(256) float g_quant_scratch[kMaxElems / 64];
+constexpr size_t kScratchFloats = kMaxElems / 64 + 2048;  // absmax values + the offset pass's 8 KB
+static __device__ __align__(256) float g_quant_scratch[kScratchFloats];
 
 std::mutex g_mu;
 float* g_ptr[64] = {nullptr};
@@ -64,5 +66,5 @@ extern "C" int nf4_quantize_tensor_noalloc(const void* w_dev, size_t n, uint8_t*
   float* scratch = nullptr;
   NF4_TRY(nf4ls::scratch_address(&scratch));
   return nf4ls::quantize_tensor(w_dev, n, packed_dev, q8_dev, nested_dev, offset_dev, scratch,
-                                (nf4ls::kMaxElems / 64) * sizeof(float), static_cast<cudaStream_t>(stream));
+                                nf4ls::kScratchFloats * sizeof(float), static_cast<cudaStream_t>(stream));
 }

@@ -9,9 +9,14 @@
 //   1. absmax_codes: a warp covers 4 blocks per iteration (8 lanes x 8 values per
 //      block); absmax by shuffle; code = number of NF4 midpoints below fp32(x/absmax);
 //      two codes per byte, the even element in the high nibble.
-//   2. offset_seq: one thread sums the fp32 absmax values in block order in double
-//      precision and divides by nb (a sequential sum, so the result does not depend
-//      on the launch shape).
+//   2. offset: the mean of the fp32 absmax values, defined as their sequential sum in
+//      block order in double precision, divided by nb.  A parallel pass sums them in
+//      a tree and also finds the smallest unit in the last place among the nonzero
+//      values; when the total stays below 2^52 of those units, every partial sum of
+//      any order is exact in double precision, so the tree's sum is the sequential
+//      sum and it is used.  Otherwise one thread repeats the sequential sum.
+//      (Weights of one tensor have absmax values within a factor of a few hundred of
+//      each other, so the parallel sum is the one that runs.)
 //   3. nested_q8: one 256-thread block per group of 256 blocks: nested = max |absmax -
 //      offset|, q8 = number of code8 midpoints below fp32((absmax - offset) / nested).
 #include <algorithm>
@@ -79,8 +84,73 @@ __global__ void __launch_bounds__(256) k_absmax_codes(const __nv_bfloat16* __res
   }
 }
 
-__global__ void k_offset_seq(const float* __restrict__ absmax, size_t nb, float* __restrict__ offset) {
-  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+constexpr int kOffsetBlocks = 256;
+constexpr size_t kOffsetScratch = 8192;  // after the absmax values: partials and the flag
+
+struct OffsetPart {
+  double sum;
+  int min_ulp;  // smallest exponent of the unit in the last place among nonzero values
+  int pad;
+};
+
+__device__ __forceinline__ int ulp_exponent(float x) {
+  const int e = (int)((__float_as_uint(x) >> 23) & 0xFF);
+  return (e > 0 ? e : 1) - 150;
+}
+
+__global__ void __launch_bounds__(256) k_offset_partial(const float* __restrict__ absmax, size_t nb,
+                                                        OffsetPart* __restrict__ part) {
+  __shared__ double ssum[256];
+  __shared__ int sulp[256];
+  double acc = 0.0;
+  int mu = 1 << 20;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < nb; i += (size_t)gridDim.x * blockDim.x) {
+    const float v = absmax[i];
+    acc += (double)v;
+    if (v != 0.f) mu = min(mu, ulp_exponent(v));
+  }
+  ssum[threadIdx.x] = acc;
+  sulp[threadIdx.x] = mu;
+  __syncthreads();
+  for (int o = 128; o > 0; o >>= 1) {
+    if (threadIdx.x < o) {
+      ssum[threadIdx.x] += ssum[threadIdx.x + o];
+      sulp[threadIdx.x] = min(sulp[threadIdx.x], sulp[threadIdx.x + o]);
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) part[blockIdx.x] = OffsetPart{ssum[0], sulp[0], 0};
+}
+
+// Combines the partials; writes the offset and flag = 1 when the sum is provably exact
+// (then equal to the sequential sum), flag = 0 otherwise.
+__global__ void __launch_bounds__(256) k_offset_final(const OffsetPart* __restrict__ part, size_t nb,
+                                                      float* __restrict__ offset, int* __restrict__ flag) {
+  __shared__ double ssum[kOffsetBlocks];
+  __shared__ int sulp[kOffsetBlocks];
+  ssum[threadIdx.x] = part[threadIdx.x].sum;
+  sulp[threadIdx.x] = part[threadIdx.x].min_ulp;
+  __syncthreads();
+  for (int o = kOffsetBlocks / 2; o > 0; o >>= 1) {
+    if (threadIdx.x < o) {
+      ssum[threadIdx.x] += ssum[threadIdx.x + o];
+      sulp[threadIdx.x] = min(sulp[threadIdx.x], sulp[threadIdx.x + o]);
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    const double S = ssum[0];
+    // every value is a multiple of 2^u and >= 0: if some partial sum had rounded, it
+    // (and so S) would be at least 2^(u + 53)
+    const bool exact = sulp[0] > 1000 || S < ldexp(1.0, sulp[0] + 52);
+    if (exact) *offset = (float)(S / (double)nb);
+    *flag = exact ? 1 : 0;
+  }
+}
+
+__global__ void k_offset_seq(const float* __restrict__ absmax, size_t nb, float* __restrict__ offset,
+                             const int* __restrict__ flag) {
+  if (threadIdx.x != 0 || blockIdx.x != 0 || *flag) return;
   double acc = 0.0;
   size_t i = 0;
   for (; i + 8 <= nb; i += 8) {
@@ -168,9 +238,10 @@ int quantize_tensor(const void* w, size_t n, uint8_t* packed, uint8_t* q8, float
   if (!aligned(w, 16) || !aligned(packed, 16) || !aligned(scratch, 16))
     return fail(NF4LS_ALIGN, "nf4_quantize_tensor: pointers must be 16-byte aligned");
   const size_t nb = n / 64;
-  if (scratch_bytes < nb * sizeof(float))
+  const size_t am_bytes = round_up(nb * sizeof(float), 256);
+  if (scratch_bytes < am_bytes + kOffsetScratch)
     return fail(NF4LS_INVALID_ARG, "nf4_quantize_tensor: scratch too small (%zu < %zu)", scratch_bytes,
-                nb * sizeof(float));
+                am_bytes + kOffsetScratch);
   const Codebooks& cb = codebooks();
   QuantTables tab;
   std::memcpy(tab.mid4, cb.mid4, sizeof(tab.mid4));
@@ -182,8 +253,13 @@ int quantize_tensor(const void* w, size_t n, uint8_t* packed, uint8_t* q8, float
   const size_t blocks = std::min<size_t>((chunks + 7) / 8, (size_t)sm_count() * 16);
   k_absmax_codes<<<(unsigned)blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(w), nb, packed, am, tab);
   note_launch();
-  k_offset_seq<<<1, 32, 0, s>>>(am, nb, offset);
-  note_launch();
+  auto* part = reinterpret_cast<OffsetPart*>(static_cast<uint8_t*>(scratch) + am_bytes);
+  int* flag = reinterpret_cast<int*>(part + kOffsetBlocks);
+  static_assert(kOffsetBlocks * sizeof(OffsetPart) + sizeof(int) <= kOffsetScratch, "offset scratch");
+  k_offset_partial<<<kOffsetBlocks, 256, 0, s>>>(am, nb, part);
+  k_offset_final<<<1, kOffsetBlocks, 0, s>>>(part, nb, offset, flag);
+  k_offset_seq<<<1, 32, 0, s>>>(am, nb, offset, flag);
+  note_launch(3);
   const size_t groups = (nb + 255) / 256;
   k_nested_q8<<<(unsigned)groups, 256, 0, s>>>(am, nb, offset, nested, q8, tab);
   note_launch();
@@ -210,7 +286,9 @@ int dequantize_tensor(const uint8_t* packed, const uint8_t* q8, const float* nes
 
 }  // namespace nf4ls
 
-extern "C" size_t nf4ls_quantize_scratch_bytes(size_t n) { return nf4ls::round_up((n / 64) * sizeof(float), 256); }
+extern "C" size_t nf4ls_quantize_scratch_bytes(size_t n) {
+  return nf4ls::round_up((n / 64) * sizeof(float), 256) + nf4ls::kOffsetScratch;
+}
 
 extern "C" int nf4_quantize_tensor(const void* w_dev, size_t n, uint8_t* packed_dev, uint8_t* q8_dev,
                                    float* nested_dev, float* offset_dev, void* scratch_dev, size_t scratch_bytes,

@@ -68,6 +68,34 @@ def run(M: int, names, iters: int, once: bool):
     return out
 
 
+def run_quant(iters: int = 10):
+    """HBM throughput of the quantiser (reads 2 B, writes 0.516 B per weight) and the
+    dequantiser (reads 0.516 B, writes 2 B per weight) on the stacked gate/up matrix."""
+    rows, cols = SHAPES["gateup"]
+    w = synth.tensor_values((rows, cols), seed=rows + cols, scale=0.02, device="cuda")
+    n = rows * cols
+    qb = n // 2 + n // 64 + 4 * ((n // 64 + 255) // 256) + 4
+    q = api.nf4_quantize_tensor(w)
+    out = []
+    for name, f, nbytes in (("quantize", lambda: api.nf4_quantize_tensor(w), 2 * n + qb),
+                            ("dequantize", lambda: api.nf4_dequantize_tensor(q), qb + 2 * n)):
+        for _ in range(3):
+            f()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(iters):
+            f()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / iters
+        rec = {"kernel": name, "weights": n, "ms": ms, "algorithmic_bytes": nbytes,
+               "gbs": nbytes / (ms / 1000.0) / 1e9}
+        out.append(rec)
+        print(json.dumps(rec), flush=True)
+    return out
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--M", type=int, default=2048)
@@ -75,9 +103,12 @@ def main(argv=None):
     ap.add_argument("--iters", type=int, default=20)
     ap.add_argument("--once", action="store_true")
     ap.add_argument("--single", action="store_true", help="one CTA per tile instead of CTA pairs")
+    ap.add_argument("--quant", action="store_true", help="also time the quantiser and dequantiser")
     a = ap.parse_args(argv)
     api.set_gemm_pair(not a.single)
     run(a.M, a.shapes.split(","), a.iters, a.once)
+    if a.quant:
+        run_quant()
     st, err = api.device_error()
     if st != 0:
         raise RuntimeError(f"device error record {err}")

@@ -58,6 +58,27 @@ def test_quantize_extreme_values():
     got = _q_to_np(q)
     np.testing.assert_array_equal(got["packed"], ref["packed"])
     np.testing.assert_array_equal(got["q8"], ref["q8"])
+    # absmax values from 1e-30 to 30: a double sum of them rounds, so the offset comes
+    # from the sequential pass, and must still equal the oracle's
+    assert got["offset"] == ref["offset"]
+    np.testing.assert_array_equal(got["nested"], ref["nested"])
+
+
+def test_quantize_offset_sum_rounding_cases():
+    """The mean absmax takes the parallel sum only when it is provably the sequential
+    one: a tensor whose absmax values span 2^-30 .. 2^1 (the double sum rounds) and one
+    with 2^18 blocks of ordinary weights (it does not) both give the oracle's bytes."""
+    g = torch.Generator().manual_seed(21)
+    w1 = (torch.rand(4096, 64, generator=g) * 2 - 1)
+    w1 = w1 * torch.pow(2.0, torch.randint(-30, 2, (4096, 1), generator=g).float())
+    w2 = synth.tensor_values((1 << 18, 64), seed=22, scale=0.02)
+    for w in (w1.to(torch.bfloat16), w2):
+        q = api.nf4_quantize_tensor(w.to(DEV))
+        ref = quant.quantize(w.float().numpy().reshape(-1))
+        got = _q_to_np(q)
+        assert got["offset"] == ref["offset"]
+        np.testing.assert_array_equal(got["nested"], ref["nested"])
+        np.testing.assert_array_equal(got["q8"], ref["q8"])
     assert got["offset"] == ref["offset"]
 
 
