@@ -270,6 +270,13 @@ int nf4ls_set_gemm_path(int path);
  * pair); 0 keeps one CTA per 256 x 256 tile.  For testing and comparison. */
 int nf4ls_set_gemm_pair(int on);
 
+/* Token height of the CTA-pair tiles (process-wide; default 0): 0 = choose per launch,
+ * taking 256-token pair tiles (128 per CTA, one accumulator) when the launch's tile
+ * count would leave the last wave of 512-token tiles mostly empty; 1 = always 512;
+ * 2 = always 256.  Results do not depend on it (same reduction order per output).
+ * For testing and comparison. */
+int nf4ls_set_gemm_half(int mode);
+
 /* ------------------------------------------------------------------ streaming pool
  * [review] mechanism section: the frozen base lives in pinned host memory; 2-8
  * preallocated HBM buffers (double by default) are filled on a dedicated CUDA

@@ -58,6 +58,11 @@ def set_gemm_pair(on: bool) -> None:
     B.call("nf4ls_set_gemm_pair", int(on))
 
 
+def set_gemm_half(mode: int) -> None:
+    """0: per-launch choice of 512- or 256-token pair tiles; 1: always 512; 2: always 256."""
+    B.call("nf4ls_set_gemm_half", int(mode))
+
+
 def launch_count() -> int:
     return int(B.lib().nf4ls_launch_count())
 

@@ -20,6 +20,7 @@ namespace {
 thread_local char g_msg[1024] = "";
 int g_gemm_path = 0;
 int g_gemm_pair = 1;
+int g_gemm_half = 0;  // 0 auto, 1 never, 2 always
 }  // namespace
 
 int fail(int status, const char* fmt, ...) {
@@ -34,6 +35,7 @@ void clear_error() { g_msg[0] = 0; }
 
 int gemm_path() { return g_gemm_path; }
 int gemm_pair() { return g_gemm_pair; }
+int gemm_half_mode() { return g_gemm_half; }
 
 void shard_layout(const nf4ls_layer_cfg* c, ShardLayout* L) {
   const int qd = c->n_q * c->head_dim, kvd = c->n_kv * c->head_dim;
@@ -108,6 +110,13 @@ extern "C" int nf4ls_set_gemm_path(int path) {
 
 extern "C" int nf4ls_set_gemm_pair(int on) {
   g_gemm_pair = on ? 1 : 0;
+  return NF4LS_OK;
+}
+
+extern "C" int nf4ls_set_gemm_half(int mode) {
+  clear_error();
+  if (mode < 0 || mode > 2) return fail(NF4LS_INVALID_ARG, "nf4ls_set_gemm_half: mode %d not in 0..2", mode);
+  g_gemm_half = mode;
   return NF4LS_OK;
 }
 

@@ -74,6 +74,7 @@ struct GemmParams {
   float* out_f32;
   const float* alpha;
   int accumulate;
+  int half;  // CTA-pair kernel: 256-token pair tiles (one 128-row accumulator per CTA)
   float nf4[16];
   float code8[256];
   int* err;
@@ -198,14 +199,14 @@ __device__ __forceinline__ void load16_bf16(const __nv_bfloat16* src, float (&v)
 // Pulls the rows of the epilogue's bf16 side input (the residual, or g and u) that this
 // CTA will read into L2 while the mainloop runs: threads t of nthreads, one 128-byte
 // line per prefetch.  A hint only; nothing waits for it.
-__device__ __forceinline__ void prefetch_aux(const GemmParams& p, int m0, int nt, int t, int nthreads) {
+__device__ __forceinline__ void prefetch_aux(const GemmParams& p, int m0, int nt, int t, int nthreads, int rows = 256) {
   if (p.epi != EPI_RESID && p.epi != EPI_DSWIGLU) return;
   const int col = nt * BN;
   if (col >= p.N) return;
   const int span = min(BN, p.N - col) * 2;  // bytes of one row segment
   const int lines = (span + 127) / 128;
   const int segs = p.epi == EPI_DSWIGLU ? 2 : 1;
-  const int total = 256 * segs * lines;
+  const int total = rows * segs * lines;
   for (int i = t; i < total; i += nthreads) {
     const int r = i / (segs * lines), rest = i % (segs * lines);
     const int m = m0 + r;
@@ -225,11 +226,14 @@ __device__ __forceinline__ void unpack16(uint4 a, uint4 b, float (&v)[16]) {
   }
 }
 
+// WITH_F32: whether the fp32 accumulate epilogue (used only by dense products) is
+// compiled in; the NF4-decode kernels leave it out, which keeps them free of spills.
+template <int n_acc = 2, bool WITH_F32 = true>
 __device__ __forceinline__ void epilogue_rows(const GemmParams& p, uint32_t tmem, int m0, int nt, int q, int lane,
                                               int part = 0, int nparts = 1) {
   constexpr int CW = 16;
   int item = 0;
-  for (int a = 0; a < 2; ++a) {
+  for (int a = 0; a < n_acc; ++a) {
     const int m = m0 + a * 128 + q * 32 + lane;
     const bool mv = m < p.M;
     const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + a * 256;
@@ -301,7 +305,7 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, uint32_t tmem
         ld_acc16(tb + c * CW, v);
         if (mv) store16(p.out + (size_t)m * p.ldo + col, v);
       }
-    } else if (p.epi == EPI_ACC_F32) {
+    } else if (WITH_F32 && p.epi == EPI_ACC_F32) {
       for (int c = 0; c < BN / CW; ++c) {
         const int col = nt * BN + c * CW;
         if (col >= p.N) break;
@@ -334,7 +338,7 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, uint32_t tmem
   // accumulators (item k: accumulator k / nch, chunk k % nch), with the bf16 side input
   // of the next item loaded while the current one is processed.
   const int nch = min(BN, p.N - nt * BN) / CW;
-  const int total = 2 * nch;
+  const int total = n_acc * nch;
   const bool dsw = p.epi == EPI_DSWIGLU;
   uint4 nx[4];
   auto load_side = [&](int k) {
@@ -383,6 +387,7 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, uint32_t tmem
 // ------------------------------------------------------------------------------ kernel
 template <bool DECODE, bool BMN>
 __global__ void __launch_bounds__(DECODE ? 448 : 192, 1) k_gemm(const __grid_constant__ GemmParams p) {
+  constexpr int NACC = 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* misc = base + STAGES * STAGE_BYTES;
@@ -526,7 +531,7 @@ __global__ void __launch_bounds__(DECODE ? 448 : 192, 1) k_gemm(const __grid_con
     prefetch_aux(p, m0, nt, threadIdx.x - 64, 128);
     if (mbar_wait(accum_full, 0, abort_flag, p.err, KID_GEMM, 3)) {
       tc_fence_after();
-      epilogue_rows(p, tmem, m0, nt, q, lane, 0, DECODE ? 3 : 1);
+      epilogue_rows<NACC, !DECODE>(p, tmem, m0, nt, q, lane, 0, DECODE ? 3 : 1);
     }
   } else if (DECODE) {
     // ---------------------------------------------------------------- NF4 decoders
@@ -611,7 +616,7 @@ __global__ void __launch_bounds__(DECODE ? 448 : 192, 1) k_gemm(const __grid_con
     // then share the epilogue: 3 warps per TMEM lane quarter
     if (mbar_wait(accum_full, 0, abort_flag, p.err, KID_GEMM, 5)) {
       tc_fence_after();
-      epilogue_rows(p, tmem, m0, nt, warp & 3, lane, (warp - 2) / 4, 3);
+      epilogue_rows<NACC, !DECODE>(p, tmem, m0, nt, warp & 3, lane, (warp - 2) / 4, 3);
     }
   }
 
@@ -645,9 +650,10 @@ constexpr int P_SMEM_BYTES = 1024 + P_STAGES * P_STAGE_BYTES + 256 + 1024;
 constexpr int P_DECODERS = 256;
 constexpr int P_GROUP = 128;
 
-template <bool DECODE, bool BMN>
+template <bool DECODE, bool BMN, bool HALF>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DECODE ? 448 : 192, 1)
     k_gemm_pair(const __grid_constant__ GemmParams p) {
+  constexpr int NACC = HALF ? 1 : 2;  // 128-row accumulators per CTA (256- or 512-token pair tiles)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* misc = base + P_STAGES * P_STAGE_BYTES;
@@ -663,7 +669,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DECODE ? 448 : 192, 
   const uint32_t rank = cluster_ctarank();
   const int pair = blockIdx.x >> 1;
   const int mt = pair % p.n_mt, nt = pair / p.n_mt;
-  const int m0 = mt * 512 + (int)rank * 256;
+  const int m0 = HALF ? mt * 256 + (int)rank * 128 : mt * 512 + (int)rank * 256;
   const int total_kb = p.num_kb + p.has_extra;
 
   if (threadIdx.x == 0) {
@@ -709,7 +715,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DECODE ? 448 : 192, 
         uint8_t* sC = sB + PB_BYTES;
         const int bcol = nt * BN + (int)rank * 128;  // this CTA's first B row (forward) or column (dL/dx)
         if (kb < p.num_kb) {
-          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * A_BYTES + (DECODE ? 0 : 2 * PB_BYTES));
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], (HALF ? A_BYTES : 2 * A_BYTES) + (DECODE ? 0 : 2 * PB_BYTES));
           tma_load_2d_pair(sA, &p.tmA, lead, kb * BK, m0);
           if (!DECODE) {
             if (BMN) {
@@ -746,7 +752,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DECODE ? 448 : 192, 
             }
           }
         } else {
-          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * A_BYTES + 2 * PB_BYTES);
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], (HALF ? A_BYTES : 2 * A_BYTES) + 2 * PB_BYTES);
           tma_load_2d_pair(sA, &p.tmAx, lead, 0, m0);
           if (BMN) {
             for (int j = 0; j < 2; ++j) tma_load_2d_pair(sB + j * 8192, &p.tmBx, lead, bcol + 64 * j, 0);
@@ -778,6 +784,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DECODE ? 448 : 192, 
                 BMN ? sdesc_sw128(aB + ks * 2048, 8192, 1024) : sdesc_sw128(aB + ks * 32, 16, 1024);
 #pragma unroll
             for (int a = 0; a < 2; ++a) {
+              if (a >= NACC) break;
               const uint64_t adesc = sdesc_sw128(aA + a * 16384 + ks * 32, 16, 1024);
               umma_bf16_pair(tmem + a * 256, adesc, bdesc, idesc, (kb | ks) != 0 ? 1u : 0u);
             }
@@ -792,10 +799,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DECODE ? 448 : 192, 
   } else if (warp < 6) {
     // ---------------------------------------------------------------- epilogue (both CTAs)
     const int q = warp & 3;
-    prefetch_aux(p, m0, nt, threadIdx.x - 64, 128);
+    prefetch_aux(p, m0, nt, threadIdx.x - 64, 128, 128 * NACC);
     if (mbar_wait(accum_full, 0, abort_flag, p.err, KID_GEMM, 13)) {
       tc_fence_after();
-      epilogue_rows(p, tmem, m0, nt, q, lane, 0, DECODE ? 3 : 1);
+      epilogue_rows<NACC, !DECODE>(p, tmem, m0, nt, q, lane, 0, DECODE ? 3 : 1);
     }
   } else if (DECODE) {
     // ---------------------------------------------------------------- NF4 decoders (both CTAs)
@@ -881,7 +888,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DECODE ? 448 : 192, 
     // then share the epilogue: 3 warps per TMEM lane quarter
     if (mbar_wait(accum_full, 0, abort_flag, p.err, KID_GEMM, 15)) {
       tc_fence_after();
-      epilogue_rows(p, tmem, m0, nt, warp & 3, lane, (warp - 2) / 4, 3);
+      epilogue_rows<NACC, !DECODE>(p, tmem, m0, nt, warp & 3, lane, (warp - 2) / 4, 3);
     }
   }
 
@@ -944,20 +951,51 @@ int launch(const GemmParams& p, int grid, cudaStream_t s) {
   return NF4LS_OK;
 }
 
+// CTA pairs that can be resident at once (the width of one wave).
 template <bool DECODE, bool BMN>
-int launch_pair(const GemmParams& p, int grid, cudaStream_t s) {
+int pair_slots() {
+  static int cached[16] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 16 && cached[dev]) return cached[dev];
+  int n = 0;
+  if (cudaFuncSetAttribute(k_gemm_pair<DECODE, BMN, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           P_SMEM_BYTES) == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * 1024);
+    cfg.blockDim = dim3(DECODE ? 448 : 192);
+    cfg.dynamicSmemBytes = P_SMEM_BYTES;
+    if (cudaOccupancyMaxActiveClusters(&n, (const void*)k_gemm_pair<DECODE, BMN, false>, &cfg) != cudaSuccess) n = 0;
+  }
+  cudaGetLastError();
+  if (n <= 0) {
+    int sms = 148;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    n = sms / 2;
+  }
+  if (dev < 16) cached[dev] = n;
+  return n;
+}
+
+template <bool DECODE, bool BMN, bool HALF>
+int launch_pair_t(const GemmParams& p, int grid, cudaStream_t s) {
   static int configured[16] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 16 && !configured[dev]) {
-    NF4_CUDA_TRY(cudaFuncSetAttribute(k_gemm_pair<DECODE, BMN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    NF4_CUDA_TRY(cudaFuncSetAttribute(k_gemm_pair<DECODE, BMN, HALF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       P_SMEM_BYTES));
     configured[dev] = 1;
   }
-  k_gemm_pair<DECODE, BMN><<<grid, DECODE ? 448 : 192, P_SMEM_BYTES, s>>>(p);
+  k_gemm_pair<DECODE, BMN, HALF><<<grid, DECODE ? 448 : 192, P_SMEM_BYTES, s>>>(p);
   note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;
+}
+
+template <bool DECODE, bool BMN>
+int launch_pair(const GemmParams& p, int grid, cudaStream_t s) {
+  return p.half ? launch_pair_t<DECODE, BMN, true>(p, grid, s) : launch_pair_t<DECODE, BMN, false>(p, grid, s);
 }
 
 }  // namespace
@@ -972,6 +1010,7 @@ int gemm(const __nv_bfloat16* A, int lda, int M, int N, int K, const GemmWeights
   if (decode && (W.n_seg < 1 || W.n_seg > 4)) return fail(NF4LS_INVALID_ARG, "gemm: 1-4 weight segments");
   if (swiglu && (dgrad || epi.inter <= 0 || epi.inter % 128 || N != 2 * epi.inter))
     return fail(NF4LS_SHAPE, "gemm: SwiGLU epilogue needs N = 2*I with I % 128 == 0");
+  if (epi.kind == EPI_ACC_F32 && decode) return fail(NF4LS_INVALID_ARG, "gemm: the fp32 epilogue takes dense weights");
   if (epi.kind == EPI_ROPE && (epi.head_dim <= 0 || BN % epi.head_dim || epi.seq <= 0))
     return fail(NF4LS_SHAPE, "gemm: RoPE epilogue head_dim");
   static_assert(sizeof(GemmParams) <= 4096, "kernel parameters exceed 4 KB");
@@ -986,12 +1025,31 @@ int gemm(const __nv_bfloat16* A, int lda, int M, int N, int K, const GemmWeights
   // CTA pairs for every product with more than one 256-token tile; single CTAs below.
   const bool pair = gemm_pair() && M > BM;
   const uint32_t bbox = pair ? 128 : 256;  // B rows one CTA loads (forward, K-major)
-  p.n_mt = pair ? (M + 511) / 512 : (M + BM - 1) / BM;
   const int n_nt = swiglu ? epi.inter / 128 : (N + BN - 1) / BN;
-  NF4_TRY(make_map(&p.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A, K, M, (uint64_t)lda * 2, 64, 256, CU_TENSOR_MAP_SWIZZLE_128B));
+  // Pair tiles of 512 tokens (two 128-row accumulators per CTA), or of 256 when that
+  // takes fewer tile-times.  A 256-token tile decodes each weight for half as many
+  // tokens, so it runs 0.78 as long as a 512-token one (measured on the 8B products at
+  // full waves): it pays off when the 512-token tiles leave most pairs idle, e.g. the
+  // 16-48 tiles of a 512-token batch.
+  p.half = 0;
+  if (pair) {
+    const int mode = gemm_half_mode();
+    if (mode == 2) {
+      p.half = 1;
+    } else if (mode == 0) {
+      const int P = decode ? (dgrad ? pair_slots<true, true>() : pair_slots<true, false>())
+                           : (dgrad ? pair_slots<false, true>() : pair_slots<false, false>());
+      const int t_full = (M + 511) / 512 * n_nt, t_half = (M + 255) / 256 * n_nt;
+      const double w_full = (double)((t_full + P - 1) / P), w_half = 0.8 * ((t_half + P - 1) / P);
+      p.half = w_half < w_full ? 1 : 0;
+    }
+  }
+  p.n_mt = pair ? (p.half ? (M + 255) / 256 : (M + 511) / 512) : (M + BM - 1) / BM;
+  const uint32_t abox = pair && p.half ? 128 : 256;  // A rows one CTA loads
+  NF4_TRY(make_map(&p.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A, K, M, (uint64_t)lda * 2, 64, abox, CU_TENSOR_MAP_SWIZZLE_128B));
   if (p.has_extra) {
     if (!extra.b) return fail(NF4LS_INVALID_ARG, "gemm: extra block needs both operands");
-    NF4_TRY(make_map(&p.tmAx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, extra.a, 64, M, 128, 64, 256, CU_TENSOR_MAP_SWIZZLE_128B));
+    NF4_TRY(make_map(&p.tmAx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, extra.a, 64, M, 128, 64, abox, CU_TENSOR_MAP_SWIZZLE_128B));
     if (dgrad)
       NF4_TRY(make_map(&p.tmBx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, extra.b, N, 64, (uint64_t)N * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B));
     else

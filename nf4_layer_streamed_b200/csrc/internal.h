@@ -123,6 +123,7 @@ int gemm(const __nv_bfloat16* A, int lda, int M, int N, int K, const GemmWeights
 
 int gemm_path();
 int gemm_pair();
+int gemm_half_mode();
 int check_cfg(const nf4ls_layer_cfg* c);
 int* device_error_ptr();
 

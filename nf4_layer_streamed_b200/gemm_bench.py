@@ -104,8 +104,10 @@ def main(argv=None):
     ap.add_argument("--once", action="store_true")
     ap.add_argument("--single", action="store_true", help="one CTA per tile instead of CTA pairs")
     ap.add_argument("--quant", action="store_true", help="also time the quantiser and dequantiser")
+    ap.add_argument("--half", type=int, default=0, help="pair tile height: 0 auto, 1 512 tokens, 2 256 tokens")
     a = ap.parse_args(argv)
     api.set_gemm_pair(not a.single)
+    api.set_gemm_half(a.half)
     run(a.M, a.shapes.split(","), a.iters, a.once)
     if a.quant:
         run_quant()
