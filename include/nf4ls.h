@@ -277,6 +277,12 @@ int nf4ls_set_gemm_pair(int on);
  * For testing and comparison. */
 int nf4ls_set_gemm_half(int mode);
 
+/* Attention forward (process-wide; default 1): 1 = the tcgen05 kernel (scores and
+ * output accumulated in TMEM) where head_dim is 128 and seq a multiple of 128 up to
+ * 512, the mma.sync kernel elsewhere; 0 = always the mma.sync kernel.  The two agree
+ * up to fp32 summation order.  For testing and comparison. */
+int nf4ls_set_attention_path(int tc);
+
 /* ------------------------------------------------------------------ streaming pool
  * [review] mechanism section: the frozen base lives in pinned host memory; 2-8
  * preallocated HBM buffers (double by default) are filled on a dedicated CUDA

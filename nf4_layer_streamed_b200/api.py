@@ -58,6 +58,11 @@ def set_gemm_pair(on: bool) -> None:
     B.call("nf4ls_set_gemm_pair", int(on))
 
 
+def set_attention_path(tc: bool) -> None:
+    """True: tcgen05 attention forward where the shape allows; False: the mma.sync kernel."""
+    B.call("nf4ls_set_attention_path", int(tc))
+
+
 def set_gemm_half(mode: int) -> None:
     """0: per-launch choice of 512- or 256-token pair tiles; 1: always 512; 2: always 256."""
     B.call("nf4ls_set_gemm_half", int(mode))

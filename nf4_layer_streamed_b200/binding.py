@@ -100,6 +100,7 @@ SIGNATURES = {
     "nf4ls_set_gemm_path": (ctypes.c_int, [ctypes.c_int]),
     "nf4ls_set_gemm_pair": (ctypes.c_int, [ctypes.c_int]),
     "nf4ls_set_gemm_half": (ctypes.c_int, [ctypes.c_int]),
+    "nf4ls_set_attention_path": (ctypes.c_int, [ctypes.c_int]),
     "nf4ls_pool_create": (ctypes.c_int, [P, P, P, ctypes.c_int, ctypes.c_int, P, SZ, ctypes.POINTER(P)]),
     "nf4ls_pool_prefetch": (ctypes.c_int, [P, ctypes.c_int]),
     "stream_prefetch": (ctypes.c_int, [P, ctypes.c_int, P, ctypes.POINTER(P)]),

@@ -21,6 +21,7 @@ thread_local char g_msg[1024] = "";
 int g_gemm_path = 0;
 int g_gemm_pair = 1;
 int g_gemm_half = 0;  // 0 auto, 1 never, 2 always
+int g_attn_tc = 1;    // attention forward on tcgen05 where the shape allows
 }  // namespace
 
 int fail(int status, const char* fmt, ...) {
@@ -36,6 +37,7 @@ void clear_error() { g_msg[0] = 0; }
 int gemm_path() { return g_gemm_path; }
 int gemm_pair() { return g_gemm_pair; }
 int gemm_half_mode() { return g_gemm_half; }
+int attention_tc() { return g_attn_tc; }
 
 void shard_layout(const nf4ls_layer_cfg* c, ShardLayout* L) {
   const int qd = c->n_q * c->head_dim, kvd = c->n_kv * c->head_dim;
@@ -110,6 +112,11 @@ extern "C" int nf4ls_set_gemm_path(int path) {
 
 extern "C" int nf4ls_set_gemm_pair(int on) {
   g_gemm_pair = on ? 1 : 0;
+  return NF4LS_OK;
+}
+
+extern "C" int nf4ls_set_attention_path(int tc) {
+  g_attn_tc = tc ? 1 : 0;
   return NF4LS_OK;
 }
 

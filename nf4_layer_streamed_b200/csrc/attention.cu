@@ -493,6 +493,8 @@ int check_attn(int seq, int nq, int nkv, int d, int ldq, int ldkv) {
 int attention_fwd(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, int ldq, int ldkv,
                   __nv_bfloat16* o, int ldo, float* lse, int batch, int seq, int nq, int nkv, int d, cudaStream_t s) {
   NF4_TRY(check_attn(seq, nq, nkv, d, ldq, ldkv));
+  if (attention_tc() && attention_fwd_tc_supported(seq, d, nq, nkv, ldq, ldkv, ldo))
+    return attention_fwd_tc(q, k, v, ldq, ldkv, o, ldo, lse, batch, seq, nq, nkv, s);
   const float scale_log2 = (1.0f / sqrtf((float)d)) * kLog2e;
   dim3 grid(seq / TQ, nq, batch);
   if (d == 128) {

@@ -1000,6 +1000,12 @@ int launch_pair(const GemmParams& p, int grid, cudaStream_t s) {
 
 }  // namespace
 
+int tma_map_bf16(CUtensorMap* map, const void* ptr, uint64_t cols, uint64_t rows, uint64_t row_bytes,
+                 uint32_t box_cols, uint32_t box_rows) {
+  return make_map(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, cols, rows, row_bytes, box_cols, box_rows,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
 int gemm(const __nv_bfloat16* A, int lda, int M, int N, int K, const GemmWeights& W, bool dgrad,
          const GemmExtra& extra, const GemmEpilogue& epi, cudaStream_t s) {
   if (!A || (epi.kind == EPI_ACC_F32 ? !epi.out_f32 || (epi.accumulate && !epi.alpha) : !epi.out))

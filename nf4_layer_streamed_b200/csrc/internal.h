@@ -124,6 +124,7 @@ int gemm(const __nv_bfloat16* A, int lda, int M, int N, int K, const GemmWeights
 int gemm_path();
 int gemm_pair();
 int gemm_half_mode();
+int attention_tc();
 int check_cfg(const nf4ls_layer_cfg* c);
 int* device_error_ptr();
 
@@ -144,6 +145,14 @@ int rmsnorm_bwd(const __nv_bfloat16* x, const __nv_bfloat16* w, const __nv_bfloa
 int rope_tables(float* cos_t, float* sin_t, float* cos_tt, float* sin_tt, int seq, int d, float theta, cudaStream_t s);
 int rope_bwd(__nv_bfloat16* x, int ld, int M, int cols, int seq, int d, const float* cos_t,
              const float* sin_t, cudaStream_t s);
+// 2D bf16 tensor map, 128-byte swizzle: [rows, cols] with row stride row_bytes, box
+// box_cols x box_rows.
+int tma_map_bf16(CUtensorMap* map, const void* ptr, uint64_t cols, uint64_t rows, uint64_t row_bytes,
+                 uint32_t box_cols, uint32_t box_rows);
+// The tcgen05 attention forward (head_dim 128, seq a multiple of 128 up to 512).
+bool attention_fwd_tc_supported(int seq, int d, int nq, int nkv, int ldq, int ldkv, int ldo);
+int attention_fwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, int ldq, int ldkv,
+                     __nv_bfloat16* o, int ldo, float* lse, int batch, int seq, int nq, int nkv, cudaStream_t s);
 int attention_fwd(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, int ldq, int ldkv,
                   __nv_bfloat16* o, int ldo, float* lse, int batch, int seq, int nq, int nkv, int d,
                   cudaStream_t s);

@@ -187,7 +187,8 @@ def test_pair_tile_heights_give_identical_results(M, rows, cols):
     assert st == 0, err
 
 
-@pytest.mark.parametrize("shape,batch,seq", [(synth.SMOLLM2_135M, 1, 512), (synth.LLAMA_8B, 2, 128)])
+@pytest.mark.parametrize("shape,batch,seq", [(synth.SMOLLM2_135M, 1, 512), (synth.LLAMA_8B, 2, 128),
+                                             (synth.LLAMA_8B, 1, 512)])
 def test_attention_forward_against_oracle(shape, batch, seq):
     cfg = api.layer_cfg(shape, batch, seq)
     M = batch * seq
@@ -200,3 +201,31 @@ def test_attention_forward_against_oracle(shape, batch, seq):
     v = x[:, qd + kvd:].reshape(batch, seq, shape.n_kv, shape.head_dim)
     ref, P = olayer.attention(q, k, v)
     close(o, ref.reshape(M, qd), what="attention out")
+
+
+@pytest.mark.parametrize("seq", [128, 384, 512])
+def test_tcgen05_attention_matches_mma_sync_attention(seq):
+    """The tcgen05 forward (head_dim 128, whole-row softmax in TMEM) against the
+    mma.sync forward on the same GQA inputs: outputs within 1e-2 max|ref|, the
+    log-sum-exp within 1e-4, and bit-exact across reruns."""
+    shape = synth.LLAMA_8B
+    batch = 2
+    cfg = api.layer_cfg(shape, batch, seq)
+    qd, kvd = shape.q_dim, shape.kv_dim
+    ld = qd + 2 * kvd
+    qkv = synth.tensor_values((batch * seq, ld), seed=seq + 7, scale=1.0).to(DEV)
+    args = (cfg, qkv, qkv[:, qd:], qkv[:, qd + kvd:], ld, ld)
+    try:
+        api.set_attention_path(False)
+        o_ref, lse_ref = api.attention_fwd(*args)
+        api.set_attention_path(True)
+        o1, lse1 = api.attention_fwd(*args)
+        o2, lse2 = api.attention_fwd(*args)
+    finally:
+        api.set_attention_path(True)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(lse1, lse2)
+    close(o1, f64(o_ref), tol=1e-2, what="tcgen05 attention")
+    close(lse1, f64(lse_ref), tol=1e-4, what="log-sum-exp")
+    st, err = api.device_error()
+    assert st == 0, err
