@@ -8,6 +8,7 @@ product out = x W^T and the dL/dx product out = dy W.
 
     python -m nf4_layer_streamed_b200.gemm_bench [--M 2048] [--shapes gateup,down] [--iters 20]
     python -m nf4_layer_streamed_b200.gemm_bench --once --shapes gateup   (one launch each: for ncu)
+    python -m nf4_layer_streamed_b200.gemm_bench --attention 4 [--once]      (attention forward, batch 4)
 
 Prints one JSON object per (shape, direction, kernel) with the mean launch time
 (CUDA events on the launching stream, after warm-up) and TFLOP/s = 2 M N K / time.
@@ -96,6 +97,43 @@ def run_quant(iters: int = 10):
     return out
 
 
+def run_attention(batch: int, once: bool, iters: int = 20):
+    """Causal GQA attention forward of the Llama-8B layer (32 query heads, 8 kv heads,
+    d 128) at seq 512: the tcgen05 kernel and the mma.sync kernel."""
+    shape = synth.LLAMA_8B
+    seq = 512
+    cfg = api.layer_cfg(shape, batch, seq)
+    qd, kvd = shape.q_dim, shape.kv_dim
+    ld = qd + 2 * kvd
+    qkv = synth.tensor_values((batch * seq, ld), seed=3, scale=1.0, device="cuda")
+    out = []
+    for tc in ((True,) if once else (True, False)):
+        api.set_attention_path(tc)
+        f = lambda: api.attention_fwd(cfg, qkv, qkv[:, qd:], qkv[:, qd + kvd:], ld, ld)
+        if once:
+            f()
+            f()
+            torch.cuda.synchronize()
+            continue
+        for _ in range(3):
+            f()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(iters):
+            f()
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) / iters * 1000.0
+        flops = 4.0 * seq * seq * shape.head_dim * shape.n_q * batch / 2
+        rec = {"kernel": "attention_fwd_tcgen05" if tc else "attention_fwd_mma_sync", "batch": batch, "seq": seq,
+               "us": us, "tflops": flops / us / 1e6}
+        out.append(rec)
+        print(json.dumps(rec), flush=True)
+    api.set_attention_path(True)
+    return out
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--M", type=int, default=2048)
@@ -105,9 +143,14 @@ def main(argv=None):
     ap.add_argument("--single", action="store_true", help="one CTA per tile instead of CTA pairs")
     ap.add_argument("--quant", action="store_true", help="also time the quantiser and dequantiser")
     ap.add_argument("--half", type=int, default=0, help="pair tile height: 0 auto, 1 512 tokens, 2 256 tokens")
+    ap.add_argument("--attention", type=int, default=0, metavar="BATCH",
+                    help="time the attention forward of the 8B layer at this batch (seq 512) instead")
     a = ap.parse_args(argv)
     api.set_gemm_pair(not a.single)
     api.set_gemm_half(a.half)
+    if a.attention:
+        run_attention(a.attention, a.once)
+        return
     run(a.M, a.shapes.split(","), a.iters, a.once)
     if a.quant:
         run_quant()
