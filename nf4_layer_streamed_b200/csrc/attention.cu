@@ -521,6 +521,10 @@ int attention_bwd(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfl
   const float scale = 1.0f / sqrtf((float)d);
   k_attn_delta<<<(M * nq + 7) / 8, 256, 0, s>>>(o, dout, ldo, M, seq, nq, d, delta);
   note_launch();
+  if (attention_tc() && attention_fwd_tc_supported(seq, d, nq, nkv, ldq, ldkv, ldo) && ld_dq % 8 == 0 &&
+      ld_dkv % 8 == 0)
+    return attention_bwd_tc(q, k, v, ldq, ldkv, dout, ldo, lse, delta, dq, dk, dv, ld_dq, ld_dkv, batch, seq, nq, nkv,
+                            s);
   dim3 gq(seq / TQ, nq, batch), gk(nkv, batch, seq / TK);
   if (d == 128) {
     const int sq = 6 * Tile<128>::BYTES, sk = 10 * Tile<128>::BYTES + 2048;

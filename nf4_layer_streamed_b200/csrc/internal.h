@@ -153,6 +153,10 @@ int tma_map_bf16(CUtensorMap* map, const void* ptr, uint64_t cols, uint64_t rows
 bool attention_fwd_tc_supported(int seq, int d, int nq, int nkv, int ldq, int ldkv, int ldo);
 int attention_fwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, int ldq, int ldkv,
                      __nv_bfloat16* o, int ldo, float* lse, int batch, int seq, int nq, int nkv, cudaStream_t s);
+int attention_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, int ldq, int ldkv,
+                     const __nv_bfloat16* dout, int ldo, const float* lse, const float* delta, __nv_bfloat16* dq,
+                     __nv_bfloat16* dk, __nv_bfloat16* dv, int ld_dq, int ld_dkv, int batch, int seq, int nq, int nkv,
+                     cudaStream_t s);
 int attention_fwd(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, int ldq, int ldkv,
                   __nv_bfloat16* o, int ldo, float* lse, int batch, int seq, int nq, int nkv, int d,
                   cudaStream_t s);

@@ -119,3 +119,33 @@ def test_llama8b_batch4_rows_equal_batch1_rows():
         assert torch.equal(dx1, dx4[sl])
     st, err = api.device_error()
     assert st == 0, err
+
+
+def test_llama8b_layer_tcgen05_attention_matches_mma_sync_attention():
+    """Forward and backward of an 8B layer (batch 2 x 512) with the tcgen05 attention
+    (forward, dQ, dK/dV) against the same layer with the mma.sync attention: outputs,
+    dL/dx and LoRA gradients within 1e-2 max|ref|."""
+    shape = synth.LLAMA_8B
+    cfg = api.layer_cfg(shape, 2, 512)
+    w = synth.layer_weights(shape, 0, 77, device=DEV)
+    shard = api.nf4_quantize_shard(cfg, w, fingerprint=1)
+    lo = synth.lora_params(shape, 0, 77, b_random=True, device=DEV)
+    x = synth.hidden_states(shape, 2, 512, 77, device=DEV).view(1024, shape.hidden)
+    res = {}
+    try:
+        for tc in (False, True):
+            api.set_attention_path(tc)
+            ws = api.LayerWorkspace(cfg)
+            y = api.layer_forward(cfg, shard, lo, x, ws)
+            _, dy = api.mse_loss(y)
+            dx, g = api.layer_backward(cfg, shard, lo, x, dy, ws)
+            torch.cuda.synchronize()
+            res[tc] = (y, dx, g)
+    finally:
+        api.set_attention_path(True)
+    close(res[True][0], f64(res[False][0]), 1e-2, "y")
+    close(res[True][1], f64(res[False][1]), 1e-2, "dx")
+    for k in res[False][2]:
+        close(res[True][2][k], f64(res[False][2][k]), 1e-2, k)
+    st, err = api.device_error()
+    assert st == 0, err
