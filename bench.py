@@ -34,7 +34,7 @@ METRIC = "trained tok/s per step (8B-shaped NF4+LoRA, streamed); GEMM % bf16 TC 
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # dram__bytes_read.sum + dram__bytes_write.sum per NF4-decode GEMM launch, averaged over
 # the 352 launches of one step of this workload (one ncu capture of the current kernel)
-NF4_GEMM_DRAM_BYTES_PER_LAUNCH = 102.9e6
+NF4_GEMM_DRAM_BYTES_PER_LAUNCH = 102.3e6
 
 
 def peaks():
