@@ -443,6 +443,40 @@ int nf4ls_forward_backward(const nf4ls_model_cfg* cfg, const nf4ls_model* model,
                            float* loss_dev, nf4ls_stream stream);
 int nf4ls_adamw_step(const nf4ls_model_cfg* cfg, const nf4ls_model* model, int32_t step, nf4ls_stream stream);
 
+/* ------------------------------------------------------------------ adapter checkpoint
+ * Save / resume of the trainable state: the LoRA parameters and both AdamW moments
+ * (model->lora_dev, adam_m_dev, adam_v_dev, n_layers * nf4ls_lora_stride floats
+ * each) and the number of AdamW steps taken.  [gate] §3.2: a release's adapters
+ * were trained correctly but reloaded as empty, unseen because no test saved and
+ * reloaded one; loading here either restores the exact bytes or fails.
+ *
+ * File: a 64-byte header (magic NF4LS_ADAPTER_MAGIC, version, H, I, n_q, n_kv,
+ * head_dim, lora_r, n_layers, lora_alpha, step, floats per array, FNV-1a 64
+ * checksum of the arrays) then the three fp32 arrays, little-endian, in the device
+ * layout.  nf4ls_adapter_file_bytes gives its size (0 for a NULL or empty config).
+ *
+ * nf4ls_adapter_save: copies the three arrays to the host on `stream` (ordered after
+ * the steps already queued there), writes path + ".tmp", fsyncs it and renames it to
+ * path, so an interrupted save leaves an older file at path intact.  step >= 0 is
+ * stored as given: pass the count of AdamW steps applied so far.  NF4LS_IO on a
+ * failed open / write / rename (the temporary file is removed).
+ *
+ * nf4ls_adapter_load: reads and checks the whole file first; NF4LS_INVALID_ARG for a
+ * wrong magic or version, NF4LS_SHAPE when H, I, heads, head_dim, lora_r, lora_alpha,
+ * n_layers or the array size differ from cfg (batch and seq may differ), NF4LS_IO
+ * for a short, over-long or checksum-failing file.  Only then are the three device
+ * arrays overwritten (on `stream`, synchronised before return) and *step set; on any
+ * failure the model is left as it was.  The next nf4ls_train_step / adamw_step of
+ * the resumed run passes *step + 1.  The gradient buffer is not saved: every step
+ * rewrites it. */
+#define NF4LS_ADAPTER_MAGIC   0x41344E46u /* "FN4A" little-endian */
+#define NF4LS_ADAPTER_VERSION 1u
+size_t nf4ls_adapter_file_bytes(const nf4ls_model_cfg* cfg);
+int nf4ls_adapter_save(const char* path, const nf4ls_model_cfg* cfg, const nf4ls_model* model, int32_t step,
+                       nf4ls_stream stream);
+int nf4ls_adapter_load(const char* path, const nf4ls_model_cfg* cfg, const nf4ls_model* model, int32_t* step,
+                       nf4ls_stream stream);
+
 /* Loss of the single-layer workloads: loss = mean(out^2) over n values and
  * dout = bf16(2 out / n).  partial_dev: n_partial (1..4096) floats of scratch. */
 int nf4ls_mse_loss(const void* out_dev, size_t n, void* dout_dev, float* loss_dev, float* partial_dev,

@@ -8,6 +8,7 @@ stream_prefetch and the pool, model and building-block calls.
 from __future__ import annotations
 
 import ctypes
+import os
 from dataclasses import dataclass
 
 import numpy as np
@@ -508,6 +509,20 @@ class StreamedModel:
     def adamw_step(self, stream=None) -> None:
         self.step_count += 1
         B.call("nf4ls_adamw_step", ctypes.byref(self.cfg), ctypes.byref(self.model), self.step_count, _s(stream))
+
+    def save_adapter(self, path: str, stream=None) -> None:
+        """Writes the LoRA parameters, both AdamW moments and step_count to path."""
+        B.call("nf4ls_adapter_save", os.fsencode(path), ctypes.byref(self.cfg), ctypes.byref(self.model),
+               self.step_count, _s(stream))
+
+    def load_adapter(self, path: str, stream=None) -> int:
+        """Restores what save_adapter wrote (the same model shape is required) and
+        step_count, so the next train_step continues the saved run."""
+        step = ctypes.c_int32(0)
+        B.call("nf4ls_adapter_load", os.fsencode(path), ctypes.byref(self.cfg), ctypes.byref(self.model),
+               ctypes.byref(step), _s(stream))
+        self.step_count = step.value
+        return self.step_count
 
     def forward_loss(self, ids: torch.Tensor, lora_on: bool = True, stream=None) -> torch.Tensor:
         B.call("nf4ls_forward_loss", ctypes.byref(self.cfg), ctypes.byref(self.model), _p(ids), int(lora_on),

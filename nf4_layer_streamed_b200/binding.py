@@ -124,6 +124,10 @@ SIGNATURES = {
     "nf4ls_forward_loss": (ctypes.c_int, [ctypes.POINTER(ModelCfg), ctypes.POINTER(Model), P, I32, P, P]),
     "nf4ls_forward_backward": (ctypes.c_int, [ctypes.POINTER(ModelCfg), ctypes.POINTER(Model), P, P, P]),
     "nf4ls_adamw_step": (ctypes.c_int, [ctypes.POINTER(ModelCfg), ctypes.POINTER(Model), I32, P]),
+    "nf4ls_adapter_file_bytes": (SZ, [ctypes.POINTER(ModelCfg)]),
+    "nf4ls_adapter_save": (ctypes.c_int, [ctypes.c_char_p, ctypes.POINTER(ModelCfg), ctypes.POINTER(Model), I32, P]),
+    "nf4ls_adapter_load": (ctypes.c_int, [ctypes.c_char_p, ctypes.POINTER(ModelCfg), ctypes.POINTER(Model),
+                                          ctypes.POINTER(ctypes.c_int32), P]),
     "nf4ls_mse_loss": (ctypes.c_int, [P, SZ, P, P, P, ctypes.c_int, P]),
     "nf4ls_gemm_bf16": (ctypes.c_int, [P, P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                        ctypes.c_int, P]),

@@ -138,3 +138,75 @@ def test_layer_sharded_fetch_arguments_on_host():
     assert B.call_status("nf4ls_pool_share", None, 0, 2, idp) == -1
     assert B.call_status("nf4ls_pool_share", ctypes.c_void_p(256), 2, 2, idp) == -1
     assert B.call_status("nf4ls_pool_share", ctypes.c_void_p(256), 0, 0, idp) == -1
+
+
+def _fnv1a64(data: bytes) -> int:
+    h = 0xCBF29CE484222325
+    for b in data:
+        h = ((h ^ b) * 0x100000001B3) & 0xFFFFFFFFFFFFFFFF
+    return h
+
+
+def test_adapter_load_refuses_bad_files_before_touching_the_device(tmp_path):
+    """An adapter file that is not exactly what this model saved is refused on the
+    host, before any copy to the (here fake) device pointers: wrong magic or version,
+    another shape or alpha, a short, over-long or corrupted body, a missing file."""
+    import struct
+    wl = synth.WORKLOADS["smollm2_30L_tied_b1s512"]
+    lc = api.layer_cfg(wl.shape, wl.batch, wl.seq)
+    n_layers = 2
+    cfg = B.ModelCfg(lc, n_layers, wl.vocab, 1, 2e-4, 0.9, 0.999, 1e-8, 0.0, 0)
+    stride = B.lib().nf4ls_lora_stride(ctypes.byref(lc))
+    n = n_layers * stride
+    assert B.lib().nf4ls_adapter_file_bytes(ctypes.byref(cfg)) == 64 + 12 * n
+    assert B.lib().nf4ls_adapter_file_bytes(None) == 0
+    m = B.Model(256, None, 256, 256, 256, 256, 256, 256, None, 256, 0, None, None)
+    body = np.arange(3 * n, dtype=np.float32).tobytes()
+    csum = _fnv1a64(body)
+
+    def header(**kw):
+        f = dict(magic=0x41344E46, version=1, hidden=lc.hidden, inter=lc.inter, n_q=lc.n_q, n_kv=lc.n_kv,
+                 head_dim=lc.head_dim, r=lc.lora_r, layers=n_layers, alpha=lc.lora_alpha, step=7, n=n,
+                 csum=csum)
+        f.update(kw)
+        return struct.pack("<IIiiiiiiifiIQQ", f["magic"], f["version"], f["hidden"], f["inter"], f["n_q"],
+                           f["n_kv"], f["head_dim"], f["r"], f["layers"], f["alpha"], f["step"], 0, f["n"],
+                           f["csum"])
+
+    assert len(header()) == 64
+    step = ctypes.c_int32(-1)
+    cases = [
+        ("magic", header(magic=0x12345678) + body, -1),
+        ("version", header(version=2) + body, -1),
+        ("hidden", header(hidden=lc.hidden * 2) + body, -2),
+        ("rank", header(r=lc.lora_r * 2) + body, -2),
+        ("alpha", header(alpha=lc.lora_alpha + 1) + body, -2),
+        ("layers", header(layers=n_layers + 1) + body, -2),
+        ("count", header(n=n - 1) + body, -2),
+        ("short_header", header()[:40], -11),
+        ("truncated", header() + body[:-4], -11),
+        ("trailing", header() + body + b"\0", -11),
+        ("corrupt", header() + body[:-1] + bytes([body[-1] ^ 1]), -11),
+        ("checksum", header(csum=csum ^ 1) + body, -11),
+    ]
+    for name, blob, want in cases:
+        p = tmp_path / f"{name}.adapter"
+        p.write_bytes(blob)
+        st = B.call_status("nf4ls_adapter_load", os.fsencode(str(p)), ctypes.byref(cfg), ctypes.byref(m),
+                           ctypes.byref(step), None)
+        assert st == want, (name, st, B.last_error())
+        assert step.value == -1, name
+    missing = os.fsencode(str(tmp_path / "missing.adapter"))
+    assert B.call_status("nf4ls_adapter_load", missing, ctypes.byref(cfg), ctypes.byref(m), ctypes.byref(step),
+                         None) == -11
+    # null arguments
+    good = tmp_path / "good.adapter"
+    good.write_bytes(header() + body)
+    g = os.fsencode(str(good))
+    assert B.call_status("nf4ls_adapter_load", g, ctypes.byref(cfg), ctypes.byref(m), None, None) == -1
+    assert B.call_status("nf4ls_adapter_load", None, ctypes.byref(cfg), ctypes.byref(m), ctypes.byref(step),
+                         None) == -1
+    no_moments = B.Model(256, None, 256, 256, 256, None, 256, 256, None, 256, 0, None, None)
+    assert B.call_status("nf4ls_adapter_load", g, ctypes.byref(cfg), ctypes.byref(no_moments), ctypes.byref(step),
+                         None) == -1
+    assert B.call_status("nf4ls_adapter_save", g, ctypes.byref(cfg), ctypes.byref(m), -1, None) == -1

@@ -6,11 +6,14 @@ whose LoRA gradients after buffer reuse must equal the resident gradients exactl
 These are the gate-record checks of "Soup layer-streamed NF4 gate record" §2.2 (streamed
 = resident, n=2 = n=3, same-seed reruns, nonzero LoRA gradients in every layer) and the
 Issue #331 scenario of the layer-streaming review's bug history."""
+import ctypes
+import os
+
 import numpy as np
 import pytest
 import torch
 
-from nf4_layer_streamed_b200 import api, synth
+from nf4_layer_streamed_b200 import api, binding as B, synth
 from oracle import model as omodel
 from tests.helpers import LOSS_RTOL, close, f64, oracle_lora, oracle_weights
 
@@ -250,3 +253,53 @@ def test_32b_class_layers_over_165mib_gradients_after_reuse_equal_resident():
             assert torch.count_nonzero(g_res[i][k]) > 0
     st, err = api.device_error()
     assert st == 0, err
+
+
+def test_adapter_checkpoint_resume_is_bit_exact(tmp_path):
+    """Six streamed steps in one run equal three steps, a save, a new model that
+    loads the file and three more steps: losses, adapter and both AdamW moments
+    bit-equal ("Soup layer-streamed NF4 gate record" §3.2: an adapter that was
+    saved must come back, not load as a no-op)."""
+    wl = synth.WORKLOADS["smollm2_30L_tied_b1s512"]
+    ids = [synth.token_ids(wl.vocab, wl.batch, wl.seq, wl.seed, step=s, device=DEV) for s in range(6)]
+
+    def run(m, steps):
+        out = []
+        for s in steps:
+            out.append(m.train_step(ids[s]).clone())
+        torch.cuda.synchronize()
+        return out
+
+    m = api.StreamedModel(wl, depth=2, resident=False, b_random=True)
+    try:
+        l_full = run(m, range(6))
+        full = (m.lora.clone(), m.adam_m.clone(), m.adam_v.clone(), m.step_count)
+    finally:
+        m.close()
+
+    path = str(tmp_path / "adapter.bin")
+    m = api.StreamedModel(wl, depth=2, resident=False, b_random=True)
+    try:
+        l_a = run(m, range(3))
+        m.save_adapter(path)
+        saved = m.lora.clone()
+    finally:
+        m.close()
+    assert os.path.getsize(path) == B.lib().nf4ls_adapter_file_bytes(ctypes.byref(m.cfg))
+
+    m = api.StreamedModel(wl, depth=2, resident=False, b_random=True)
+    try:
+        assert not torch.equal(m.lora, saved)   # a fresh adapter: loading must change it
+        assert m.load_adapter(path) == 3
+        assert torch.equal(m.lora, saved)
+        l_b = run(m, range(3, 6))
+        resumed = (m.lora.clone(), m.adam_m.clone(), m.adam_v.clone(), m.step_count)
+        st, err = api.device_error()
+        assert st == 0, err
+    finally:
+        m.close()
+    assert torch.equal(torch.cat(l_full), torch.cat(l_a + l_b))
+    for a, b in zip(full[:3], resumed[:3]):
+        assert torch.equal(a, b)
+    assert full[3] == resumed[3] == 6
+    assert torch.count_nonzero(full[2]) > 0
