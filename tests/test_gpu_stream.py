@@ -303,3 +303,35 @@ def test_adapter_checkpoint_resume_is_bit_exact(tmp_path):
         assert torch.equal(a, b)
     assert full[3] == resumed[3] == 6
     assert torch.count_nonzero(full[2]) > 0
+
+
+def test_step_log_on_the_streamed_run(tmp_path):
+    """The per-step log of a streamed run: one line per step, the step's copies
+    (every layer read, some backward reads served by the slot still holding it), the
+    loss the step returned, the event time and phases with library profiling on."""
+    import json
+    from nf4_layer_streamed_b200 import steplog
+    wl = synth.WORKLOADS["smollm2_30L_tied_b1s512"]
+    m = api.StreamedModel(wl, depth=2, resident=False)
+    path = str(tmp_path / "steps.jsonl")
+    api.profile(True)
+    try:
+        log = steplog.StepLog(m, path, tokens_per_step=wl.batch * wl.seq)
+        losses = []
+        for s in range(2):
+            ids = synth.token_ids(wl.vocab, wl.batch, wl.seq, wl.seed, step=s, device=DEV)
+            losses.append(log.step(ids)["loss"])
+        log.close()
+    finally:
+        api.profile(False)
+        api.profile_reset()
+        m.close()
+    recs = [json.loads(l) for l in open(path)]
+    assert [r["step"] for r in recs] == [1, 2]
+    for r, l in zip(recs, losses):
+        assert r["loss"] == l and np.isfinite(l)
+        assert r["step_ms"] > 0 and r["peak_mem_bytes"] > 0
+        assert wl.n_layers <= r["copies"] <= 2 * wl.n_layers
+        assert 0 < r["hits"] <= 2 * wl.n_layers   # prefetched or still-resident layers
+        assert r["h2d_bytes"] >= r["copies"] * api.shard_bytes(m.cfg.layer)
+        assert set(r["phases_ms"]) >= {"layers_forward", "layers_backward"}
