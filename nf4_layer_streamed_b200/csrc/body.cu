@@ -54,6 +54,7 @@ __global__ void k_rmsnorm_fwd(const __nv_bfloat16* __restrict__ x, const __nv_bf
   uint4* yr = reinterpret_cast<uint4*>(y + (size_t)row * H);
   const int nv = H / 8;
   float ss = 0.f;
+#pragma unroll 4
   for (int i = lane; i < nv; i += 32) {
     float f[8];
     unpack8(xr[i], f);
@@ -62,6 +63,7 @@ __global__ void k_rmsnorm_fwd(const __nv_bfloat16* __restrict__ x, const __nv_bf
   }
   ss = warp_sum(ss);
   const float r = 1.0f / sqrtf(ss / (float)H + eps);
+#pragma unroll 4
   for (int i = lane; i < nv; i += 32) {
     float f[8], g[8];
     unpack8(xr[i], f);
@@ -86,6 +88,7 @@ __global__ void k_rmsnorm_bwd(const __nv_bfloat16* __restrict__ x, const __nv_bf
   uint4* out = reinterpret_cast<uint4*>(dx + (size_t)row * H);
   const int nv = H / 8;
   float ss = 0.f, dot = 0.f;
+#pragma unroll 4
   for (int i = lane; i < nv; i += 32) {
     float a[8], b[8], c[8];
     unpack8(xr[i], a);
@@ -101,6 +104,7 @@ __global__ void k_rmsnorm_bwd(const __nv_bfloat16* __restrict__ x, const __nv_bf
   dot = warp_sum(dot);
   const float r = 1.0f / sqrtf(ss / (float)H + eps);
   const float k = r * r * r * dot / (float)H;
+#pragma unroll 4
   for (int i = lane; i < nv; i += 32) {
     float a[8], b[8], c[8], e[8];
     unpack8(xr[i], a);
@@ -152,6 +156,35 @@ __global__ void k_rope_bwd(__nv_bfloat16* __restrict__ x, int ld, int M, int col
   const float a = __bfloat162float(p[j]), b = __bfloat162float(p[j + half]);
   p[j] = __float2bfloat16_rn(a * c + b * s);
   p[j + half] = __float2bfloat16_rn(b * c - a * s);
+}
+
+// The same, eight frequencies per thread: one 16-byte load and store of each half and
+// two float4 reads of each table (rows of 16-byte-aligned bf16, d / 2 a multiple of 8).
+// Block (x, row): threads over the row's 8-pair groups.
+__global__ void k_rope_bwd8(__nv_bfloat16* __restrict__ x, int ld, int cols, int seq, int d,
+                            const float* __restrict__ cos_t, const float* __restrict__ sin_t) {
+  const int half = d / 2, groups_per_head = half / 8;
+  const int gi = blockIdx.x * blockDim.x + threadIdx.x;
+  if (gi >= cols / 16) return;
+  const int m = blockIdx.y;
+  const int head = gi / groups_per_head, j0 = (gi - head * groups_per_head) * 8;
+  const int pos = m % seq;
+  __nv_bfloat16* p = x + (size_t)m * ld + head * d + j0;
+  const float4* cr = reinterpret_cast<const float4*>(cos_t + (size_t)pos * half + j0);
+  const float4* sr = reinterpret_cast<const float4*>(sin_t + (size_t)pos * half + j0);
+  const float4 c0 = cr[0], c1 = cr[1], s0 = sr[0], s1 = sr[1];
+  const float c[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+  const float sn[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+  float a[8], b[8], o1[8], o2[8];
+  unpack8(*reinterpret_cast<const uint4*>(p), a);
+  unpack8(*reinterpret_cast<const uint4*>(p + half), b);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    o1[j] = a[j] * c[j] + b[j] * sn[j];
+    o2[j] = b[j] * c[j] - a[j] * sn[j];
+  }
+  *reinterpret_cast<uint4*>(p) = pack8(o1);
+  *reinterpret_cast<uint4*>(p + half) = pack8(o2);
 }
 
 __global__ void k_zero_cols(__nv_bfloat16* __restrict__ x, int ld, int M, int c0, int c1) {
@@ -468,7 +501,12 @@ int rope_tables(float* cos_t, float* sin_t, float* cos_tt, float* sin_tt, int se
 
 int rope_bwd(__nv_bfloat16* x, int ld, int M, int cols, int seq, int d, const float* cos_t, const float* sin_t,
              cudaStream_t s) {
-  k_rope_bwd<<<blocks_for((size_t)M * cols / 2, 256), 256, 0, s>>>(x, ld, M, cols, seq, d, cos_t, sin_t);
+  const bool vec = (d / 2) % 8 == 0 && ld % 8 == 0 && cols % d == 0 && aligned(x, 16) && aligned(cos_t, 16) &&
+                   aligned(sin_t, 16) && M <= 65535;
+  if (vec)
+    k_rope_bwd8<<<dim3(blocks_for((size_t)cols / 16, 128), M), 128, 0, s>>>(x, ld, cols, seq, d, cos_t, sin_t);
+  else
+    k_rope_bwd<<<blocks_for((size_t)M * cols / 2, 256), 256, 0, s>>>(x, ld, M, cols, seq, d, cos_t, sin_t);
   note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;
