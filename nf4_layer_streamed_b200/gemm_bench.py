@@ -9,6 +9,7 @@ product out = x W^T and the dL/dx product out = dy W.
     python -m nf4_layer_streamed_b200.gemm_bench [--M 2048] [--shapes gateup,down] [--iters 20]
     python -m nf4_layer_streamed_b200.gemm_bench --once --shapes gateup   (one launch each: for ncu)
     python -m nf4_layer_streamed_b200.gemm_bench --attention 4 [--once]      (attention forward, batch 4)
+    python -m nf4_layer_streamed_b200.gemm_bench --layer 4 [--once]   (quantise + one 8B layer fwd/bwd)
 
 Prints one JSON object per (shape, direction, kernel) with the mean launch time
 (CUDA events on the launching stream, after warm-up) and TFLOP/s = 2 M N K / time.
@@ -134,6 +135,49 @@ def run_attention(batch: int, once: bool, iters: int = 20):
     return out
 
 
+def run_layer(batch: int, once: bool, iters: int = 10):
+    """One Llama-8B-shaped layer at batch x 512: the shard quantiser, then layer_forward
+    and layer_backward (recompute + dL/dx + LoRA gradients) with random LoRA B.  With
+    --once each runs once (a small case for ncu: every kernel of the layer appears)."""
+    shape = synth.LLAMA_8B
+    seq = 512
+    cfg = api.layer_cfg(shape, batch, seq)
+    w = synth.layer_weights(shape, 0, 1234, device="cuda")
+    lo = synth.lora_params(shape, 0, 1234, b_random=True, device="cuda")
+    x = synth.hidden_states(shape, batch, seq, 7, device="cuda").view(batch * seq, shape.hidden)
+    dy = synth.tensor_values((batch * seq, shape.hidden), seed=5, scale=1e-3, device="cuda")
+    ws = api.LayerWorkspace(cfg)
+    shard = api.nf4_quantize_shard(cfg, w, fingerprint=1)
+    fwd = lambda: api.layer_forward(cfg, shard, lo, x, ws)
+    bwd = lambda: api.layer_backward(cfg, shard, lo, x, dy, ws)
+    if once:
+        fwd()
+        bwd()
+        torch.cuda.synchronize()
+        return []
+    out = []
+    for name, f in (("quantize_shard", lambda: api.nf4_quantize_shard(cfg, w, fingerprint=1, out=shard)),
+                    ("layer_forward", fwd), ("layer_backward", bwd)):
+        ms = _time(f, iters)
+        rec = {"step": name, "batch": batch, "seq": seq, "ms": ms}
+        out.append(rec)
+        print(json.dumps(rec), flush=True)
+    return out
+
+
+def _time(f, iters):
+    for _ in range(3):
+        f()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(iters):
+        f()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / iters
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--M", type=int, default=2048)
@@ -143,6 +187,8 @@ def main(argv=None):
     ap.add_argument("--single", action="store_true", help="one CTA per tile instead of CTA pairs")
     ap.add_argument("--quant", action="store_true", help="also time the quantiser and dequantiser")
     ap.add_argument("--half", type=int, default=0, help="pair tile height: 0 auto, 1 512 tokens, 2 256 tokens")
+    ap.add_argument("--layer", type=int, default=0, metavar="BATCH",
+                    help="time the shard quantiser and one 8B layer forward / backward at this batch instead")
     ap.add_argument("--attention", type=int, default=0, metavar="BATCH",
                     help="time the attention forward of the 8B layer at this batch (seq 512) instead")
     a = ap.parse_args(argv)
@@ -150,6 +196,12 @@ def main(argv=None):
     api.set_gemm_half(a.half)
     if a.attention:
         run_attention(a.attention, a.once)
+        return
+    if a.layer:
+        run_layer(a.layer, a.once)
+        st, err = api.device_error()
+        if st != 0:
+            raise RuntimeError(f"device error record {err}")
         return
     run(a.M, a.shapes.split(","), a.iters, a.once)
     if a.quant:
