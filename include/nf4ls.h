@@ -270,11 +270,12 @@ int nf4ls_set_gemm_path(int path);
  * pair); 0 keeps one CTA per 256 x 256 tile.  For testing and comparison. */
 int nf4ls_set_gemm_pair(int on);
 
-/* Token height of the CTA-pair tiles (process-wide; default 0): 0 = choose per launch,
- * taking 256-token pair tiles (128 per CTA, one accumulator) when the launch's tile
- * count would leave the last wave of 512-token tiles mostly empty; 1 = always 512;
- * 2 = always 256.  Results do not depend on it (same reduction order per output).
- * For testing and comparison. */
+/* Token height of the CTA-pair tiles (process-wide; default 0): 0 = choose per launch
+ * between 512 and 256 by their tile-times; 1 = always 512; 2 = always 256
+ * (128 per CTA, one accumulator); 3 = 512-token tiles for the whole waves and the tiles
+ * of the last, partial wave as 256-token tiles in a second launch (where every
+ * 512-token tile is two 256-token tiles, else as 1).  Results do not depend on it (same
+ * reduction order per output).  For testing and comparison. */
 int nf4ls_set_gemm_half(int mode);
 
 /* Attention forward (process-wide; default 1): 1 = the tcgen05 kernel (scores and

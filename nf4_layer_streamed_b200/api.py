@@ -65,7 +65,8 @@ def set_attention_path(tc: bool) -> None:
 
 
 def set_gemm_half(mode: int) -> None:
-    """0: per-launch choice of 512- or 256-token pair tiles; 1: always 512; 2: always 256."""
+    """0: per-launch choice of the pair-tile schedule; 1: always 512 tokens; 2: always 256;
+    3: 512 for the whole waves, 256 for the last partial wave (nf4ls_set_gemm_half)."""
     B.call("nf4ls_set_gemm_half", int(mode))
 
 

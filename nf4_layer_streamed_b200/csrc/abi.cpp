@@ -20,7 +20,7 @@ namespace {
 thread_local char g_msg[1024] = "";
 int g_gemm_path = 0;
 int g_gemm_pair = 1;
-int g_gemm_half = 0;  // 0 auto, 1 never, 2 always
+int g_gemm_half = 0;  // 0 auto, 1 never, 2 always, 3 the last partial wave only
 int g_attn_tc = 1;    // attention forward on tcgen05 where the shape allows
 }  // namespace
 
@@ -122,7 +122,7 @@ extern "C" int nf4ls_set_attention_path(int tc) {
 
 extern "C" int nf4ls_set_gemm_half(int mode) {
   clear_error();
-  if (mode < 0 || mode > 2) return fail(NF4LS_INVALID_ARG, "nf4ls_set_gemm_half: mode %d not in 0..2", mode);
+  if (mode < 0 || mode > 3) return fail(NF4LS_INVALID_ARG, "nf4ls_set_gemm_half: mode %d not in 0..3", mode);
   g_gemm_half = mode;
   return NF4LS_OK;
 }

@@ -74,7 +74,8 @@ struct GemmParams {
   float* out_f32;
   const float* alpha;
   int accumulate;
-  int half;  // CTA-pair kernel: 256-token pair tiles (one 128-row accumulator per CTA)
+  int half;   // CTA-pair kernel: 256-token pair tiles (one 128-row accumulator per CTA)
+  int tile0;  // CTA-pair kernel: tile index of the launch's first pair (mt fastest)
   float nf4[16];
   float code8[256];
   int* err;
@@ -667,8 +668,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DECODE ? 448 : 192, 
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
-  const int pair = blockIdx.x >> 1;
-  const int mt = pair % p.n_mt, nt = pair / p.n_mt;
+  const int tile = (blockIdx.x >> 1) + p.tile0;
+  const int mt = tile % p.n_mt, nt = tile / p.n_mt;
   const int m0 = HALF ? mt * 256 + (int)rank * 128 : mt * 512 + (int)rank * 256;
   const int total_kb = p.num_kb + p.has_extra;
 
@@ -1036,26 +1037,47 @@ int gemm(const __nv_bfloat16* A, int lda, int M, int N, int K, const GemmWeights
   // takes fewer tile-times.  A 256-token tile decodes each weight for half as many
   // tokens, so it runs 0.78 as long as a 512-token one (measured on the 8B products at
   // full waves): it pays off when the 512-token tiles leave most pairs idle, e.g. the
-  // 16-48 tiles of a 512-token batch.
+  // 16-48 tiles of a 512-token batch.  Or, on request only (mode 3), split: the whole
+  // waves of 512-token tiles in one launch and the tiles of the last, partial wave as
+  // twice as many 256-token tiles in a second launch.  Measured on the 8B products of
+  // a 2048-token batch, whose last waves hold 22, 2 and 4 of 74 tiles (q/k/v forward,
+  // down dL/dx, gate/up forward), it changed them by -1%, -3% and +1%: a partial last
+  // wave of 512-token tiles already runs faster than a full one, so the automatic
+  // choice leaves it out.  All three schedules reduce every output in the same order.
   p.half = 0;
+  int split_full = 0;  // tiles of the 512-token launch when the tail is split off
+  const int t_full = (M + 511) / 512 * n_nt, t_half = (M + 255) / 256 * n_nt;
+  // the split needs every 512-token tile to be exactly two 256-token tiles
+  const bool can_split = pair && (M + 255) / 256 == 2 * ((M + 511) / 512);
   if (pair) {
     const int mode = gemm_half_mode();
+    const int P = decode ? (dgrad ? pair_slots<true, true>() : pair_slots<true, false>())
+                         : (dgrad ? pair_slots<false, true>() : pair_slots<false, false>());
+    const int waves = t_full / P;
     if (mode == 2) {
       p.half = 1;
+    } else if (mode == 3 && can_split) {
+      split_full = waves * P;
     } else if (mode == 0) {
-      const int P = decode ? (dgrad ? pair_slots<true, true>() : pair_slots<true, false>())
-                           : (dgrad ? pair_slots<false, true>() : pair_slots<false, false>());
-      const int t_full = (M + 511) / 512 * n_nt, t_half = (M + 255) / 256 * n_nt;
       const double w_full = (double)((t_full + P - 1) / P), w_half = 0.8 * ((t_half + P - 1) / P);
       p.half = w_half < w_full ? 1 : 0;
     }
   }
+  const bool split = pair && gemm_half_mode() == 3 && can_split;
   p.n_mt = pair ? (p.half ? (M + 255) / 256 : (M + 511) / 512) : (M + BM - 1) / BM;
-  const uint32_t abox = pair && p.half ? 128 : 256;  // A rows one CTA loads
-  NF4_TRY(make_map(&p.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A, K, M, (uint64_t)lda * 2, 64, abox, CU_TENSOR_MAP_SWIZZLE_128B));
+  // A rows one CTA loads: 128 for 256-token pair tiles, else 256
+  auto map_a = [&](bool half_rows) -> int {
+    const uint32_t abox = pair && half_rows ? 128 : 256;
+    NF4_TRY(make_map(&p.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A, K, M, (uint64_t)lda * 2, 64, abox,
+                     CU_TENSOR_MAP_SWIZZLE_128B));
+    if (p.has_extra)
+      NF4_TRY(make_map(&p.tmAx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, extra.a, 64, M, 128, 64, abox,
+                       CU_TENSOR_MAP_SWIZZLE_128B));
+    return NF4LS_OK;
+  };
+  if (p.has_extra && !extra.b) return fail(NF4LS_INVALID_ARG, "gemm: extra block needs both operands");
+  NF4_TRY(map_a(p.half != 0));
   if (p.has_extra) {
-    if (!extra.b) return fail(NF4LS_INVALID_ARG, "gemm: extra block needs both operands");
-    NF4_TRY(make_map(&p.tmAx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, extra.a, 64, M, 128, 64, abox, CU_TENSOR_MAP_SWIZZLE_128B));
     if (dgrad)
       NF4_TRY(make_map(&p.tmBx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, extra.b, N, 64, (uint64_t)N * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B));
     else
@@ -1121,15 +1143,29 @@ int gemm(const __nv_bfloat16* A, int lda, int M, int N, int K, const GemmWeights
   if (epi.kind == EPI_ACC_F32 && (epi.ldo % 4 || !aligned(epi.out_f32, 16)))
     return fail(NF4LS_ALIGN, "gemm: fp32 output needs 16-byte rows");
   p.err = device_error_ptr();
+  p.tile0 = 0;
   const int grid = p.n_mt * n_nt * (pair ? 2 : 1);
   cudaEvent_t e0 = nullptr;
   if (profiling()) profile_begin(s, &e0);
-  int st;
-  if (pair) {
+  auto run_pair = [&](int pairs) {
     if (decode)
-      st = dgrad ? launch_pair<true, true>(p, grid, s) : launch_pair<true, false>(p, grid, s);
-    else
-      st = dgrad ? launch_pair<false, true>(p, grid, s) : launch_pair<false, false>(p, grid, s);
+      return dgrad ? launch_pair<true, true>(p, 2 * pairs, s) : launch_pair<true, false>(p, 2 * pairs, s);
+    return dgrad ? launch_pair<false, true>(p, 2 * pairs, s) : launch_pair<false, false>(p, 2 * pairs, s);
+  };
+  int st;
+  if (split) {
+    // 512-token tiles [0, split_full), then 256-token tiles [2 split_full, 2 t_full):
+    // with mt fastest, 512-token tile t is 256-token tiles 2t and 2t + 1.
+    st = split_full > 0 ? run_pair(split_full) : NF4LS_OK;
+    if (st == NF4LS_OK) {
+      p.half = 1;
+      p.n_mt = (M + 255) / 256;
+      p.tile0 = 2 * split_full;
+      st = map_a(true);
+      if (st == NF4LS_OK) st = run_pair(t_half - 2 * split_full);
+    }
+  } else if (pair) {
+    st = run_pair(grid / 2);
   } else if (decode) {
     st = dgrad ? launch<true, true>(p, grid, s) : launch<true, false>(p, grid, s);
   } else {

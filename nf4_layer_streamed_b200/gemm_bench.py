@@ -24,6 +24,7 @@ import torch
 from . import api, synth
 
 SHAPES = {  # name: (rows = out features, cols = in features) of W
+    "qkv": (6144, 4096),       # q, k and v stacked, as the fused GEMM runs them
     "qo": (4096, 4096),
     "kv": (1024, 4096),
     "gateup": (28672, 4096),   # gate and up stacked, as the fused GEMM runs them
@@ -186,7 +187,8 @@ def main(argv=None):
     ap.add_argument("--once", action="store_true")
     ap.add_argument("--single", action="store_true", help="one CTA per tile instead of CTA pairs")
     ap.add_argument("--quant", action="store_true", help="also time the quantiser and dequantiser")
-    ap.add_argument("--half", type=int, default=0, help="pair tile height: 0 auto, 1 512 tokens, 2 256 tokens")
+    ap.add_argument("--half", type=int, default=0,
+                    help="pair tile height: 0 auto, 1 512 tokens, 2 256 tokens, 3 last partial wave as 256")
     ap.add_argument("--layer", type=int, default=0, metavar="BATCH",
                     help="time the shard quantiser and one 8B layer forward / backward at this batch instead")
     ap.add_argument("--attention", type=int, default=0, metavar="BATCH",

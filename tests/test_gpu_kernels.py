@@ -163,10 +163,13 @@ def test_cta_pair_gemm_equals_single_cta(M, rows, cols):
     assert st == 0, err
 
 
-@pytest.mark.parametrize("M,rows,cols", [(1280, 576, 1536), (2048, 6144, 4096)])
+@pytest.mark.parametrize("M,rows,cols", [(1280, 576, 1536), (2048, 6144, 4096), (2048, 14336, 4096),
+                                         (1536, 28672, 4096)])
 def test_pair_tile_heights_give_identical_results(M, rows, cols):
-    """256- and 512-token pair tiles reduce every output in the same order: equal bits,
-    forward and dL/dx, NF4 decode and dense, including a ragged last token tile."""
+    """256- and 512-token pair tiles, and the split schedule (whole waves of 512-token
+    tiles, the last partial wave as 256-token tiles in a second launch), reduce every
+    output in the same order: equal bits, forward and dL/dx, NF4 decode and dense,
+    including a ragged last token tile."""
     w = synth.tensor_values((rows, cols), seed=5 * rows + cols, scale=0.02).to(DEV)
     q = api.nf4_quantize_tensor(w)
     deq = api.nf4_dequantize_tensor(q).view(rows, cols)
@@ -174,14 +177,15 @@ def test_pair_tile_heights_give_identical_results(M, rows, cols):
     G = synth.tensor_values((M, rows), seed=M + 4, scale=1.0).to(DEV)
     outs = {}
     try:
-        for mode in (1, 2):
+        for mode in (1, 2, 3):
             api.set_gemm_half(mode)
             outs[mode] = [api.gemm_nf4(A, q, rows, cols), api.gemm_nf4(G, q, rows, cols, dgrad=True),
                           api.gemm_bf16(A, deq), api.gemm_bf16(G, deq, b_trans=True)]
     finally:
         api.set_gemm_half(0)
-    for a, b in zip(outs[1], outs[2]):
-        assert torch.equal(a, b)
+    for mode in (2, 3):
+        for a, b in zip(outs[1], outs[mode]):
+            assert torch.equal(a, b), mode
     close(outs[2][0], f64(A) @ f64(deq).T, tol=1e-2, what="half-height forward")
     st, err = api.device_error()
     assert st == 0, err
