@@ -59,6 +59,8 @@ def parse():
     ap.add_argument("--shard-fetch", action="store_true",
                     help="N > 1: each rank copies only the layers it owns (l %% N) over PCIe and the pools "
                          "broadcast them to the other ranks over NVLink (NCCL)")
+    ap.add_argument("--oracle-configs", action="store_true",
+                    help="time the CPU oracle on the small configurations (1 and all BLAS threads) and exit")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the resident (compute-only) timing and the batch-16 compute-bound point")
     return ap.parse_args()
@@ -184,6 +186,75 @@ def run_reference(args, wl):
     print(json.dumps(line), flush=True)
 
 
+def run_oracle_configs(args):
+    """The oracle, as it stands, on the small configurations, with the BLAS pool at one
+    thread and at every core: one SmolLM2-shaped layer and one Llama-8B-shaped layer at
+    1 x 512 tokens (forward, checkpoint recompute, backward with LoRA gradients), and
+    one training step of the 30-layer SmolLM2-shaped stack (batch 1 x 512: forward,
+    recompute + backward per layer, tied-head cross-entropy, AdamW on every adapter).
+    Weight generation and oracle quantisation happen before the clock starts.  Prints
+    one JSON line with `"impl": "oracle_configs"`; the default run does not do this."""
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+
+    from nf4_layer_streamed_b200 import synth
+    from oracle import layer as olayer, model as omodel, quant
+
+    def dequant_layer(w):
+        out = {}
+        for n in ("q", "k", "v", "o", "gate", "up", "down"):
+            q = quant.quantize(w[n].float().numpy().reshape(-1))
+            out[n] = quant.dequantize(q).reshape(w[n].shape)
+        out["norm_in"] = w["norm_in"].double().numpy()
+        out["norm_post"] = w["norm_post"].double().numpy()
+        return out
+
+    def layer_case(shape, tokens):
+        W = dequant_layer(synth.layer_weights(shape, 0, 1234))
+        lo = {k: v.double().numpy() for k, v in synth.lora_params(shape, 0, 1234, b_random=True).items()}
+        x = synth.hidden_states(shape, 1, tokens, 1234).double().numpy().reshape(tokens, shape.hidden)
+
+        def run():
+            out, sv = olayer.forward(x, W, lo, shape, 1, tokens)
+            _, sv = olayer.forward(x, W, lo, shape, 1, tokens)
+            olayer.backward(out * 1e-3, W, lo, shape, 1, tokens, sv)
+        return run
+
+    def step_case(wl):
+        shape = wl.shape
+        layers = [dequant_layer(synth.layer_weights(shape, i, wl.seed)) for i in range(wl.n_layers)]
+        loras = [{k: v.double().numpy() for k, v in synth.lora_params(shape, i, wl.seed).items()}
+                 for i in range(wl.n_layers)]
+        moments = [({k: np.zeros_like(v) for k, v in lo.items()}, {k: np.zeros_like(v) for k, v in lo.items()})
+                   for lo in loras]
+        emb = synth.embedding(wl.vocab, shape.hidden, wl.seed).double().numpy()
+        ids = synth.token_ids(wl.vocab, wl.batch, wl.seq, wl.seed).numpy()
+
+        def run():
+            _, grads, _ = omodel.forward_backward(ids, layers, loras, emb, None, np.ones(shape.hidden), shape,
+                                                  wl.batch, wl.seq)
+            for lo, g, (m, v) in zip(loras, grads, moments):
+                for k in lo:
+                    lo[k], m[k], v[k] = omodel.adamw(lo[k], g["d" + k], m[k], v[k], 1)
+        return run
+
+    cases = [("smollm2_layer_b1s512", layer_case(synth.SMOLLM2_135M, 512), 512),
+             ("llama8b_layer_b1s512", layer_case(synth.LLAMA_8B, 512), 512),
+             ("smollm2_30L_step_b1s512", step_case(synth.WORKLOADS["smollm2_30L_tied_b1s512"]), 512)]
+    cores = os.cpu_count() or 1
+    res = {}
+    for name, run, tokens in cases:
+        for threads in (1, cores):
+            with threadpool_limits(limits=threads, user_api="blas"):
+                t0 = time.perf_counter()
+                run()
+                dt = time.perf_counter() - t0
+            res[f"{name}_threads{threads}"] = {"seconds": dt, "tokens_per_s": tokens / dt, "threads": threads}
+    print(json.dumps({"impl": "oracle_configs", "kind": "oracle", "host_cores": cores, "dtype": "f64",
+                      "note": "one run each, after weight generation and oracle quantisation",
+                      "results": res}), flush=True)
+
+
 # ----------------------------------------------------------------------------- ours
 def time_steps(m, ids, warmup: int, steps: int) -> float:
     """ms per training step of model m (CUDA events on the current stream)."""
@@ -286,6 +357,10 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             run_reference(args, wl)
+        return 0
+    if args.oracle_configs:
+        if rank == 0:
+            run_oracle_configs(args)
         return 0
 
     import torch
