@@ -316,6 +316,12 @@ class Pool:
             B.call("nf4ls_pool_destroy", self.handle)
             self.handle = ctypes.c_void_p()
 
+    def __enter__(self) -> "Pool":
+        return self
+
+    def __exit__(self, *exc) -> None:
+        self.destroy()
+
     def view(self, ptr: int, nbytes: int) -> torch.Tensor:
         """A uint8 view of the slot at device address ptr (for reading a streamed shard)."""
         off = ptr - self.slots.data_ptr()
@@ -537,3 +543,9 @@ class StreamedModel:
         if self.head_pool is not None:
             self.head_pool.destroy()
             self.head_pool = None
+
+    def __enter__(self) -> "StreamedModel":
+        return self
+
+    def __exit__(self, *exc) -> None:
+        self.close()
