@@ -335,3 +335,31 @@ def test_step_log_on_the_streamed_run(tmp_path):
         assert 0 < r["hits"] <= 2 * wl.n_layers   # prefetched or still-resident layers
         assert r["h2d_bytes"] >= r["copies"] * api.shard_bytes(m.cfg.layer)
         assert set(r["phases_ms"]) >= {"layers_forward", "layers_backward"}
+
+
+def test_llama8b_32_layers_b4s512_streamed_equals_resident():
+    """The bench workload at full size (32 Llama-8B-shaped layers, untied vocab 128256,
+    batch 4 x 512), streamed at depth 2 as the bench times it, against every shard
+    resident in HBM: two AdamW steps with bit-equal losses, LoRA gradients and adapters;
+    the loss at initialisation sits near ln V (uniform targets)."""
+    wl = synth.WORKLOADS["llama8b_32L_b4s512"]
+    out = {}
+    for resident in (False, True):
+        m = api.StreamedModel(wl, depth=2, resident=resident)
+        try:
+            losses = []
+            for s in range(2):
+                ids = synth.token_ids(wl.vocab, wl.batch, wl.seq, wl.seed, step=s, device=DEV)
+                m.forward_backward(ids)
+                losses.append(m.loss.clone())
+                m.adamw_step()
+            torch.cuda.synchronize()
+            st, err = api.device_error()
+            assert st == 0, err
+            out[resident] = (torch.cat(losses), m.grads.clone(), m.lora.clone())
+        finally:
+            m.close()
+    for a, b in zip(out[False], out[True]):
+        assert torch.equal(a, b)
+    l0 = float(out[False][0][0])
+    assert np.isfinite(l0) and abs(l0 - np.log(wl.vocab)) < 1.0
