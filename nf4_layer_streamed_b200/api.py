@@ -38,6 +38,54 @@ def _buffer(nbytes: int, device="cuda") -> torch.Tensor:
     return _aligned(torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device))
 
 
+# The library takes raw device pointers and cannot see a wrong dtype, size, layout or
+# device itself, so each call below first checks every tensor's dtype, size and layout,
+# then that all of them live on a CUDA device, and only then passes the pointers.
+def _need(t, name: str, dtype, numel: int | None = None, contiguous: bool = True) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if numel is not None and t.numel() != numel:
+        raise ValueError(f"{name}: {t.numel()} elements, expected {numel}")
+    if contiguous and not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    return t
+
+
+def _need_rows(t, name: str, rows: int, ld: int, width: int) -> torch.Tensor:
+    """A bf16 row-major view of `rows` rows of `width` elements, `ld` elements apart."""
+    if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or t.dim() != 2:
+        raise ValueError(f"{name}: expected a 2-D bf16 tensor")
+    if t.shape[0] < rows or t.shape[1] < width or t.stride(1) != 1 or (rows > 1 and t.stride(0) != ld):
+        raise ValueError(f"{name}: shape {tuple(t.shape)} / strides {t.stride()} do not hold {rows} rows "
+                         f"of {width} elements {ld} apart")
+    return t
+
+
+def _need_cuda(**tensors) -> None:
+    for name, t in tensors.items():
+        if t is not None and not t.is_cuda:
+            raise ValueError(f"{name}: must be a CUDA tensor")
+
+
+def _need_shard(shard, cfg: B.LayerCfg) -> None:
+    if not isinstance(shard, torch.Tensor):
+        raise TypeError("shard: expected a torch.Tensor")
+    if shard.numel() * shard.element_size() < shard_bytes(cfg):
+        raise ValueError(f"shard: {shard.numel() * shard.element_size()} bytes, the layer needs {shard_bytes(cfg)}")
+
+
+def _need_lora(lora: dict | None, cfg: B.LayerCfg, grads: bool = False) -> dict:
+    if lora is None:
+        return {}
+    r, H, qd, kvd = cfg.lora_r, cfg.hidden, cfg.n_q * cfg.head_dim, cfg.n_kv * cfg.head_dim
+    p = "d" if grads else ""
+    for k, n in (("A_q", r * H), ("B_q", qd * r), ("A_v", r * H), ("B_v", kvd * r)):
+        _need(lora[p + k], p + k, torch.float32, n)
+    return {p + k: lora[p + k] for k in ("A_q", "B_q", "A_v", "B_v")}
+
+
 def layer_cfg(shape: LayerShape, batch: int, seq: int) -> B.LayerCfg:
     return B.LayerCfg(shape.hidden, shape.inter, shape.n_q, shape.n_kv, shape.head_dim, batch, seq,
                       shape.rope_theta, shape.rms_eps, shape.lora_r, shape.lora_alpha)
@@ -176,6 +224,13 @@ class LayerWorkspace:
 
 def layer_forward(cfg: B.LayerCfg, shard: torch.Tensor, lora: dict | None, x: torch.Tensor,
                   ws: LayerWorkspace | None = None, y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    MH = cfg.batch * cfg.seq * cfg.hidden
+    _need(x, "x", torch.bfloat16, MH)
+    _need_shard(shard, cfg)
+    lt = _need_lora(lora, cfg)
+    if y is not None:
+        _need(y, "y", torch.bfloat16, MH)
+    _need_cuda(x=x, shard=shard, y=y, **lt)
     ws = ws or LayerWorkspace(cfg, x.device)
     y = torch.empty_like(x) if y is None else y
     lo = _lora_struct(lora)
@@ -187,6 +242,15 @@ def layer_forward(cfg: B.LayerCfg, shard: torch.Tensor, lora: dict | None, x: to
 def layer_backward(cfg: B.LayerCfg, shard: torch.Tensor, lora: dict | None, x: torch.Tensor, dy: torch.Tensor,
                    ws: LayerWorkspace | None = None, dx: torch.Tensor | None = None, grads: dict | None = None,
                    stream=None):
+    MH = cfg.batch * cfg.seq * cfg.hidden
+    _need(x, "x", torch.bfloat16, MH)
+    _need(dy, "dy", torch.bfloat16, MH)
+    _need_shard(shard, cfg)
+    lt = _need_lora(lora, cfg)
+    if dx is not None:
+        _need(dx, "dx", torch.bfloat16, MH)
+    gt = _need_lora(grads, cfg, grads=True) if (lora is not None and grads is not None) else {}
+    _need_cuda(x=x, dy=dy, shard=shard, dx=dx, **lt, **gt)
     ws = ws or LayerWorkspace(cfg, x.device)
     dx = torch.empty_like(x) if dx is None else dx
     lo = _lora_struct(lora)
@@ -204,6 +268,8 @@ def layer_backward(cfg: B.LayerCfg, shard: torch.Tensor, lora: dict | None, x: t
 
 def mse_loss(out: torch.Tensor, stream=None):
     """loss = mean(out^2) (fp32 device scalar), dout = bf16(2 out / n)."""
+    _need(out, "out", torch.bfloat16)
+    _need_cuda(out=out)
     n = out.numel()
     dout = torch.empty_like(out)
     loss = torch.empty(1, dtype=torch.float32, device=out.device)
@@ -215,6 +281,11 @@ def mse_loss(out: torch.Tensor, stream=None):
 
 def gemm_bf16(A: torch.Tensor, Bm: torch.Tensor, b_trans: bool = False, stream=None) -> torch.Tensor:
     """out = A B^T (B [N, K]) or, with b_trans, out = A B (B [K, N]); tcgen05 kernel."""
+    if A.dim() != 2 or Bm.dim() != 2 or Bm.shape[0 if b_trans else 1] != A.shape[1]:
+        raise ValueError(f"gemm_bf16: A {tuple(A.shape)} and B {tuple(Bm.shape)} (b_trans={b_trans}) do not match")
+    _need(A, "A", torch.bfloat16)
+    _need(Bm, "B", torch.bfloat16)
+    _need_cuda(A=A, B=Bm)
     M, K = A.shape
     N = Bm.shape[1] if b_trans else Bm.shape[0]
     out = torch.empty(M, N, dtype=torch.bfloat16, device=A.device)
@@ -224,6 +295,13 @@ def gemm_bf16(A: torch.Tensor, Bm: torch.Tensor, b_trans: bool = False, stream=N
 
 def gemm_nf4(A: torch.Tensor, q: dict, rows: int, cols: int, dgrad: bool = False, stream=None) -> torch.Tensor:
     """out = A W^T (forward) or A W (dgrad) with W [rows, cols] given as an NF4 tensor dict."""
+    K = rows if dgrad else cols
+    _need_rows(A, "A", A.shape[0] if A.dim() == 2 else 0, A.stride(0) if A.dim() == 2 else 0, K)
+    if A.shape[1] != K:
+        raise ValueError(f"gemm_nf4: A has {A.shape[1]} columns, the product needs {K}")
+    if q.get("n") != rows * cols:
+        raise ValueError(f"gemm_nf4: the NF4 tensor holds {q.get('n')} weights, not {rows} x {cols}")
+    _need_cuda(A=A, **{k: q[k] for k in ("packed", "q8", "nested", "offset")})
     M = A.shape[0]
     N = cols if dgrad else rows
     out = torch.empty(M, N, dtype=torch.bfloat16, device=A.device)
@@ -234,6 +312,10 @@ def gemm_nf4(A: torch.Tensor, q: dict, rows: int, cols: int, dgrad: bool = False
 
 def attention_fwd(cfg: B.LayerCfg, q, k, v, ld_q: int, ld_kv: int, stream=None):
     M = cfg.batch * cfg.seq
+    _need_rows(q, "q", M, ld_q, cfg.n_q * cfg.head_dim)
+    _need_rows(k, "k", M, ld_kv, cfg.n_kv * cfg.head_dim)
+    _need_rows(v, "v", M, ld_kv, cfg.n_kv * cfg.head_dim)
+    _need_cuda(q=q, k=k, v=v)
     o = torch.empty(M, cfg.n_q * cfg.head_dim, dtype=torch.bfloat16, device=q.device)
     lse = torch.empty(cfg.batch, cfg.n_q, cfg.seq, dtype=torch.float32, device=q.device)
     B.call("nf4ls_attention_fwd", ctypes.byref(cfg), _p(q), _p(k), _p(v), ld_q, ld_kv, _p(o), _p(lse), _s(stream))
