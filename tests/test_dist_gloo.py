@@ -1,4 +1,4 @@
-"""Host logic of the data-parallel step on two CPU ranks over gloo.
+"""Host logic of the data-parallel step on two and three CPU ranks over gloo.
 
 A stand-in model computes rank-dependent fp32 "gradients" from its token ids and
 applies the oracle's AdamW; the test checks that after a few DataParallelStep calls
@@ -66,8 +66,8 @@ def _worker(rank, world, port, q):
         dist.destroy_process_group()
 
 
-def test_data_parallel_step_two_ranks_gloo():
-    world = 2
+@pytest.mark.parametrize("world", [2, 3])
+def test_data_parallel_step_ranks_gloo(world):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
@@ -81,8 +81,9 @@ def test_data_parallel_step_two_ranks_gloo():
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    np.testing.assert_array_equal(res[0][0], res[1][0])
-    assert not np.array_equal(res[0][1][0], res[1][1][0])
+    for r in range(1, world):
+        np.testing.assert_array_equal(res[0][0], res[r][0])
+        assert not np.array_equal(res[0][1][0], res[r][1][0])
     # single-process replay on the averaged gradients
     ref = FakeModel()
     for s in range(3):
@@ -116,10 +117,11 @@ def _fetch_worker(rank, world, port, q):
         dist.destroy_process_group()
 
 
-def test_layer_sharded_fetch_two_ranks_gloo():
+@pytest.mark.parametrize("world", [2, 3])
+def test_layer_sharded_fetch_ranks_gloo(world):
     """Every rank ends with every layer's bytes while reading only the layers it owns
-    (l % world == rank) from its own store, and all ranks get the same NCCL id."""
-    world = 2
+    (l % world == rank) from its own store, and all ranks get the same NCCL id (three
+    ranks: 7 layers do not split evenly)."""
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
@@ -138,6 +140,6 @@ def test_layer_sharded_fetch_two_ranks_gloo():
         assert ok
         assert all(l % world == r for l in reads) and reads
         assert rr == r and w == world and len(nccl_id) == 128
-    assert res[0][2][2] == res[1][2][2]
+        assert nccl_id == res[0][2][2]
     # the fetch is split: together the ranks read each of the 12 fills exactly once
-    assert len(res[0][1]) + len(res[1][1]) == 7 + 5
+    assert sum(len(res[r][1]) for r in range(world)) == 7 + 5
