@@ -1,7 +1,9 @@
 """Pins of the oracle's layer, loss, optimiser and accounting (CPU only).
 
 Pins: library routines run independently of the oracle (torch rms_norm,
-scaled_dot_product_attention, torch.optim.AdamW, scipy logsumexp), float64
+scaled_dot_product_attention, torch.optim.AdamW, scipy logsumexp, and torch autograd
+through rms_norm, scaled_dot_product_attention and cross_entropy for the backward
+pieces), RoPE as a complex rotation with its adjoint as the backward, float64
 central finite differences on tiny shapes with bf16 rounding off, structural
 LoRA facts the gate record relies on (B = 0 gives an exactly zero adapter
 output and dA = 0; a random B makes every gradient nonzero), and the page's
@@ -206,3 +208,73 @@ def test_gflop_per_token_table_from_page():
     assert abs(qwen(896, 4864, 24, 14, 2, 64, 151936) - g["qwen25_05b"]) <= 0.01
     assert abs(qwen(1536, 8960, 28, 12, 2, 128, 151936) - g["qwen25_15b"]) <= 0.01
     assert abs(qwen(2048, 11008, 36, 16, 2, 128, 151936) - g["qwen25_3b"]) <= 0.01
+
+
+# ------------------------------------------------------------------ backward pieces vs torch autograd
+def test_attention_backward_matches_torch_autograd():
+    """dq, dk, dv of causal GQA attention (three query heads per kv head) against
+    torch autograd through scaled_dot_product_attention, float64."""
+    rng = np.random.default_rng(21)
+    B_, S, nq, nkv, d = 2, 9, 6, 2, 8
+    q, k, v = (rng.normal(size=(B_, S, n, d)) for n in (nq, nkv, nkv))
+    do = rng.normal(size=(B_, S, nq, d))
+    o, P = layer.attention(q, k, v)
+    dq, dk, dv = layer.attention_bwd(q, k, v, P, do)
+    tq, tk, tv = (torch.tensor(a, requires_grad=True) for a in (q, k, v))
+    grp = nq // nkv
+    out = torch.nn.functional.scaled_dot_product_attention(
+        tq.transpose(1, 2), tk.repeat_interleave(grp, dim=2).transpose(1, 2),
+        tv.repeat_interleave(grp, dim=2).transpose(1, 2), is_causal=True).transpose(1, 2)
+    out.backward(torch.tensor(do))
+    np.testing.assert_allclose(o, out.detach().numpy(), rtol=1e-10, atol=1e-12)
+    for mine, ref in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+        np.testing.assert_allclose(mine, ref.numpy(), rtol=1e-9, atol=1e-12)
+
+
+def test_rmsnorm_backward_matches_torch_autograd():
+    rng = np.random.default_rng(22)
+    x = rng.normal(size=(5, 48))
+    w = 1.0 + 0.1 * rng.normal(size=48)
+    dy = rng.normal(size=(5, 48))
+    y, r = layer.rmsnorm(x, w, 1e-5)
+    dx = layer.rmsnorm_bwd(x, w, r, dy)
+    tx = torch.tensor(x, requires_grad=True)
+    ty = torch.nn.functional.rms_norm(tx, (48,), torch.tensor(w), eps=1e-5)
+    ty.backward(torch.tensor(dy))
+    np.testing.assert_allclose(y, ty.detach().numpy(), rtol=1e-12)
+    np.testing.assert_allclose(dx, tx.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_rope_matches_complex_rotation_and_its_adjoint():
+    """Rotate-half RoPE is multiplication of (x_i + i x_{i+d/2}) by e^{i p theta_i};
+    its backward is the adjoint: <rope(x), y> = <x, rope_bwd(y)>."""
+    rng = np.random.default_rng(23)
+    S, d = 7, 16
+    cos, sin = layer.rope_tables(S, d, 500000.0)
+    x = rng.normal(size=(2, S, 3, d))
+    y = layer.rope(x, cos, sin)
+    z = (x[..., : d // 2] + 1j * x[..., d // 2:])
+    inv = 500000.0 ** (-(2.0 * np.arange(d // 2)) / d)
+    rot = np.exp(1j * np.arange(S)[:, None] * inv[None, :])[None, :, None, :]
+    zr = z * rot
+    np.testing.assert_allclose(y[..., : d // 2], zr.real, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(y[..., d // 2:], zr.imag, rtol=1e-12, atol=1e-14)
+    g = rng.normal(size=x.shape)
+    assert math.isclose(float(np.sum(y * g)), float(np.sum(x * layer.rope_bwd(g, cos, sin))), rel_tol=1e-12)
+
+
+def test_cross_entropy_gradient_matches_torch_autograd():
+    """Loss and dlogits of the shifted causal-LM cross-entropy (no target for the last
+    position of each sequence) against torch's cross_entropy with ignore_index."""
+    rng = np.random.default_rng(24)
+    batch, seq, V = 2, 6, 11
+    logits = rng.normal(size=(batch * seq, V)) * 3
+    ids = rng.integers(0, V, size=(batch, seq))
+    loss, d = model.cross_entropy(logits, ids, batch, seq, rnd=False)
+    tgt = np.full((batch, seq), -100)
+    tgt[:, :-1] = ids[:, 1:]
+    tl = torch.tensor(logits, requires_grad=True)
+    ref = torch.nn.functional.cross_entropy(tl, torch.tensor(tgt.reshape(-1)), ignore_index=-100)
+    ref.backward()
+    assert math.isclose(loss, float(ref.detach()), rel_tol=1e-12)
+    np.testing.assert_allclose(d, tl.grad.numpy(), rtol=1e-10, atol=1e-14)
