@@ -278,3 +278,54 @@ def test_cross_entropy_gradient_matches_torch_autograd():
     ref.backward()
     assert math.isclose(loss, float(ref.detach()), rel_tol=1e-12)
     np.testing.assert_allclose(d, tl.grad.numpy(), rtol=1e-10, atol=1e-14)
+
+
+def _hf_layer(shape, W, seq):
+    """A transformers LlamaDecoderLayer (float64, eager attention) holding W."""
+    from transformers import LlamaConfig
+    from transformers.models.llama.modeling_llama import LlamaDecoderLayer, LlamaRotaryEmbedding
+    cfg = LlamaConfig(hidden_size=shape.hidden, intermediate_size=shape.inter, num_attention_heads=shape.n_q,
+                      num_key_value_heads=shape.n_kv, head_dim=shape.head_dim, rms_norm_eps=shape.rms_eps,
+                      rope_theta=shape.rope_theta, attention_bias=False, mlp_bias=False, hidden_act="silu",
+                      max_position_embeddings=max(seq, 8))
+    cfg._attn_implementation = "eager"
+    hf = LlamaDecoderLayer(cfg, layer_idx=0).double()
+    with torch.no_grad():
+        for mod, key in ((hf.self_attn.q_proj, "q"), (hf.self_attn.k_proj, "k"), (hf.self_attn.v_proj, "v"),
+                         (hf.self_attn.o_proj, "o"), (hf.mlp.gate_proj, "gate"), (hf.mlp.up_proj, "up"),
+                         (hf.mlp.down_proj, "down")):
+            mod.weight.copy_(torch.tensor(W[key]))
+        hf.input_layernorm.weight.copy_(torch.tensor(W["norm_in"]))
+        hf.post_attention_layernorm.weight.copy_(torch.tensor(W["norm_post"]))
+    return hf, LlamaRotaryEmbedding(cfg)
+
+
+@pytest.mark.parametrize("with_lora", [False, True])
+def test_layer_forward_matches_transformers_llama_decoder_layer(with_lora):
+    """The oracle's decoder layer (float64, no bf16 rounding) against transformers'
+    LlamaDecoderLayer, the body the pages run: pre-norm residual blocks, GQA, rotate-half
+    RoPE, SiLU-gated MLP.  With the adapter on, the reference layer gets the merged
+    weights W_q + (alpha / r) B_q A_q and W_v + (alpha / r) B_v A_v, which is what the
+    LoRA update adds.  The reference computes its RoPE angles in fp32, hence a 1e-6
+    tolerance rather than float64 rounding (measured 1.5e-8)."""
+    shape = synth.TINY
+    batch, seq = 2, 8
+    W = _weights(shape, seed=31)
+    lo = _lora(shape, seed=32) if with_lora else None
+    x = np.random.default_rng(33).normal(size=(batch * seq, shape.hidden))
+    out, _ = layer.forward(x, W, lo, shape, batch, seq, rnd=False)
+    Wm = dict(W)
+    if lo is not None:
+        s = shape.lora_alpha / shape.lora_r
+        Wm["q"] = W["q"] + s * lo["B_q"] @ lo["A_q"]
+        Wm["v"] = W["v"] + s * lo["B_v"] @ lo["A_v"]
+    hf, rot = _hf_layer(shape, Wm, seq)
+    tx = torch.tensor(x.reshape(batch, seq, shape.hidden))
+    pos = torch.arange(seq)[None].expand(batch, seq)
+    cos, sin = rot(tx, pos)
+    mask = torch.triu(torch.full((seq, seq), float("-inf"), dtype=torch.float64), 1)[None, None]
+    with torch.no_grad():
+        ref = hf(tx, attention_mask=mask, position_ids=pos, position_embeddings=(cos, sin))
+    ref = (ref[0] if isinstance(ref, tuple) else ref).numpy().reshape(batch * seq, shape.hidden)
+    err = np.max(np.abs(out - ref))
+    assert err <= 1e-6 * np.max(np.abs(ref)), err
