@@ -329,3 +329,50 @@ def test_layer_forward_matches_transformers_llama_decoder_layer(with_lora):
     ref = (ref[0] if isinstance(ref, tuple) else ref).numpy().reshape(batch * seq, shape.hidden)
     err = np.max(np.abs(out - ref))
     assert err <= 1e-6 * np.max(np.abs(ref)), err
+
+
+def test_model_step_matches_transformers_llama_autograd():
+    """One training step of the oracle (a 2-layer tied model, float64, no rounding)
+    against transformers' LlamaForCausalLM with autograd: the loss of its labels path,
+    and the LoRA gradients from the gradient G of the merged weight W + s B A, which are
+    dA = s B^T G and dB = s G A^T exactly."""
+    from transformers import LlamaConfig, LlamaForCausalLM
+    shape = synth.TINY
+    n_layers, vocab, batch, seq = 2, 32, 2, 6
+    rng = np.random.default_rng(41)
+    layers = [_weights(shape, seed=42 + i) for i in range(n_layers)]
+    loras = [_lora(shape, seed=50 + i) for i in range(n_layers)]
+    emb = rng.normal(0, 0.5, (vocab, shape.hidden))
+    w_final = 1.0 + 0.1 * rng.normal(size=shape.hidden)
+    ids = rng.integers(0, vocab, (batch, seq))
+    loss, grads, _ = model.forward_backward(ids, layers, loras, emb, None, w_final, shape, batch, seq, rnd=False)
+
+    cfg = LlamaConfig(hidden_size=shape.hidden, intermediate_size=shape.inter, num_attention_heads=shape.n_q,
+                      num_key_value_heads=shape.n_kv, head_dim=shape.head_dim, rms_norm_eps=shape.rms_eps,
+                      rope_theta=shape.rope_theta, attention_bias=False, mlp_bias=False, hidden_act="silu",
+                      vocab_size=vocab, num_hidden_layers=n_layers, tie_word_embeddings=True,
+                      max_position_embeddings=seq)
+    cfg._attn_implementation = "eager"
+    hf = LlamaForCausalLM(cfg).double()
+    s = shape.lora_alpha / shape.lora_r
+    with torch.no_grad():
+        hf.model.embed_tokens.weight.copy_(torch.tensor(emb))
+        hf.model.norm.weight.copy_(torch.tensor(w_final))
+        for L, W, lo in zip(hf.model.layers, layers, loras):
+            merged = dict(W, q=W["q"] + s * lo["B_q"] @ lo["A_q"], v=W["v"] + s * lo["B_v"] @ lo["A_v"])
+            for mod, key in ((L.self_attn.q_proj, "q"), (L.self_attn.k_proj, "k"), (L.self_attn.v_proj, "v"),
+                             (L.self_attn.o_proj, "o"), (L.mlp.gate_proj, "gate"), (L.mlp.up_proj, "up"),
+                             (L.mlp.down_proj, "down")):
+                mod.weight.copy_(torch.tensor(merged[key]))
+            L.input_layernorm.weight.copy_(torch.tensor(W["norm_in"]))
+            L.post_attention_layernorm.weight.copy_(torch.tensor(W["norm_post"]))
+    tid = torch.tensor(ids)
+    ref = hf(input_ids=tid, labels=tid).loss
+    ref.backward()
+    assert math.isclose(loss, float(ref.detach()), rel_tol=1e-6)
+    for L, lo, g in zip(hf.model.layers, loras, grads):
+        Gq = L.self_attn.q_proj.weight.grad.numpy()
+        Gv = L.self_attn.v_proj.weight.grad.numpy()
+        for mine, want in ((g["dA_q"], s * lo["B_q"].T @ Gq), (g["dB_q"], s * Gq @ lo["A_q"].T),
+                           (g["dA_v"], s * lo["B_v"].T @ Gv), (g["dB_v"], s * Gv @ lo["A_v"].T)):
+            assert np.max(np.abs(mine - want)) <= 1e-5 * np.max(np.abs(want))
