@@ -231,3 +231,62 @@ def test_quantize_deterministic_and_roundtrip_through_bytes():
     assert np.array_equal(quant.dequantize_bits({**{k: r[k] for k in ("packed", "q8", "nested")},
                                                  "offset": r["offset"]}),
                           quant.dequantize_bits(q1))
+
+
+# ----------------------------------------------------------------------------- properties
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@st.composite
+def _weight_blocks(draw):
+    """1-9 blocks of 64 bf16 values: a per-block scale over 40 binades, some blocks all
+    zero, some holding a single nonzero, signs mixed."""
+    nb = draw(st.integers(1, 9))
+    rng = np.random.default_rng(draw(st.integers(0, 2 ** 31 - 1)))
+    w = np.empty(64 * nb, np.float32)
+    for b in range(nb):
+        kind = draw(st.sampled_from(["normal", "zero", "single", "uniform"]))
+        scale = np.float32(2.0 ** draw(st.integers(-30, 10)))
+        if kind == "zero":
+            blk = np.zeros(64, np.float32)
+        elif kind == "single":
+            blk = np.zeros(64, np.float32)
+            blk[draw(st.integers(0, 63))] = scale * draw(st.sampled_from([-1.0, 1.0, 0.37]))
+        elif kind == "uniform":
+            blk = (rng.uniform(-1, 1, 64) * scale).astype(np.float32)
+        else:
+            blk = (rng.normal(0, 1, 64) * scale).astype(np.float32)
+        w[b * 64:(b + 1) * 64] = blk
+    return bf16.round_f32(w)
+
+
+@settings(max_examples=60, deadline=None)
+@given(_weight_blocks())
+def test_quantizer_properties(w):
+    """What any correct blockwise NF4 quantiser with double-quantised absmax does,
+    on blocks spanning 40 binades: each code is a nearest NF4 entry to x / absmax
+    (up to the fp32 midpoint window); a block's largest magnitude maps to -1 or +1; an
+    all-zero block gives the zero code and dequantises to exact zeros; the nested scale
+    reproduces absmax within the 8-bit table's resolution."""
+    q = quant.quantize(w)
+    nf4 = codebooks.nf4_table().astype(np.float64)
+    codes = quant.unpack_codes(q["packed"]).reshape(-1, 64)
+    xb = w.astype(np.float64).reshape(-1, 64)
+    am = np.abs(xb).max(axis=1)
+    zero = codebooks.zero_index(nf4)
+    for b in range(xb.shape[0]):
+        if am[b] == 0.0:
+            assert np.all(codes[b] == zero)
+            continue
+        u = xb[b] / am[b]
+        dist = np.abs(u[:, None] - nf4[None, :])
+        chosen = dist[np.arange(64), codes[b]]
+        assert np.all(chosen <= dist.min(axis=1) + 1e-6)
+        i = int(np.argmax(np.abs(xb[b])))
+        assert nf4[codes[b][i]] == np.sign(xb[b][i])
+    wh = quant.dequantize(q).reshape(-1, 64)
+    assert np.all(wh[am == 0.0] == 0.0)
+    s = quant.block_scales(q).astype(np.float64)
+    c8 = codebooks.code8_table().astype(np.float64)
+    gap = np.max(np.diff(c8)) / 2 * float(np.max(q["nested"])) + 1e-6 * am.max()
+    assert np.all(np.abs(s - am) <= gap + 2.0 ** -20 * am)
