@@ -1,0 +1,78 @@
+"""The oracle's pins have teeth (CPU only): each case plants one plausible mistake in
+the oracle (a dropped term, a sign, a missing scale, a wrong index or a missing step,
+patched into the oracle module for the duration of the case) and checks that the pin
+meant to guard that step now fails.  Nothing here touches the product path."""
+import numpy as np
+import pytest
+
+from oracle import layer, model
+from tests import test_oracle_layer as P
+
+
+def _rmsnorm_bwd_dropped_term(x, w, r, dy):
+    return r * dy * w                         # the - x r^3 <w dy, x> / H term is gone
+
+
+def _rope_sign_flip(x, cos, sin):
+    h = x.shape[-1] // 2
+    x1, x2 = x[..., :h], x[..., h:]
+    c, s = cos[None, :, None, :], sin[None, :, None, :]
+    return np.concatenate([x1 * c + x2 * s, x2 * c - x1 * s], axis=-1)   # rotates the other way
+
+
+def _attention_no_scale(q, k, v):
+    return _orig_attention(q * np.sqrt(q.shape[-1]), k, v)               # forgets 1/sqrt(d)
+
+
+def _attention_bwd_dk_without_q(q, k, v, Pr, do):
+    dq, dk, dv = _orig_attention_bwd(q, k, v, Pr, do)
+    return dq, dk * 0.5, dv                                              # a halved dK
+
+
+def _silu_as_sigmoid(x):
+    return layer.sigmoid(x)                                              # x * sigmoid(x) lost its x
+
+
+def _ce_unshifted(logits, ids, batch, seq, rnd=True):
+    ids = np.asarray(ids).reshape(batch, seq)
+    shifted = np.concatenate([ids[:, :1], ids[:, :-1]], axis=1)         # targets one position late
+    return _orig_ce(logits, shifted, batch, seq, rnd)
+
+
+def _adamw_no_bias_correction(p, g, m, v, step, lr=2e-4, b1=0.9, b2=0.999, eps=1e-8, wd=0.0):
+    m = b1 * m + (1 - b1) * g
+    v = b2 * v + (1 - b2) * g * g
+    return p - lr * (m / (np.sqrt(v) + eps) + wd * p), m, v
+
+
+_orig_attention = layer.attention
+_orig_attention_bwd = layer.attention_bwd
+_orig_ce = model.cross_entropy
+
+CASES = [
+    ("rmsnorm_bwd", layer, "rmsnorm_bwd", _rmsnorm_bwd_dropped_term,
+     [P.test_rmsnorm_backward_matches_torch_autograd]),
+    ("rope sign", layer, "rope", _rope_sign_flip,
+     [P.test_rope_matches_complex_rotation_and_its_adjoint]),
+    ("attention scale", layer, "attention", _attention_no_scale,
+     [P.test_attention_matches_torch_sdpa,
+      lambda: P.test_layer_forward_matches_transformers_llama_decoder_layer(False)]),
+    ("attention dK", layer, "attention_bwd", _attention_bwd_dk_without_q,
+     [P.test_attention_backward_matches_torch_autograd,
+      lambda: P.test_layer_backward_finite_differences(1, 8)]),
+    ("SiLU", layer, "silu", _silu_as_sigmoid,
+     [lambda: P.test_layer_forward_matches_transformers_llama_decoder_layer(True)]),
+    ("cross-entropy shift", model, "cross_entropy", _ce_unshifted,
+     [P.test_cross_entropy_gradient_matches_torch_autograd, P.test_model_step_matches_transformers_llama_autograd]),
+    ("AdamW bias correction", model, "adamw", _adamw_no_bias_correction, [P.test_adamw_matches_torch]),
+]
+
+
+@pytest.mark.parametrize("name,mod,attr,bad,pins", CASES, ids=[c[0] for c in CASES])
+def test_pins_catch_planted_mistake(monkeypatch, name, mod, attr, bad, pins):
+    for pin in pins:
+        pin()                                        # holds on the oracle as it is
+    monkeypatch.setattr(mod, attr, bad)
+    for pin in pins:
+        with pytest.raises(AssertionError):
+            pin()
