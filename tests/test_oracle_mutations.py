@@ -5,8 +5,9 @@ meant to guard that step now fails.  Nothing here touches the product path."""
 import numpy as np
 import pytest
 
-from oracle import layer, model
+from oracle import codebooks, layer, model, quant
 from tests import test_oracle_layer as P
+from tests import test_oracle_quant as Q
 
 
 def _rmsnorm_bwd_dropped_term(x, w, r, dy):
@@ -45,6 +46,28 @@ def _adamw_no_bias_correction(p, g, m, v, step, lr=2e-4, b1=0.9, b2=0.999, eps=1
     return p - lr * (m / (np.sqrt(v) + eps) + wd * p), m, v
 
 
+def _nearest_off_by_one(u, table):
+    idx = _orig_nearest(u, table)
+    if len(table) == 16:                                                 # every 7th NF4 code one too high
+        idx = np.minimum(idx + (np.arange(idx.size).reshape(idx.shape) % 7 == 3), 15)
+    return idx
+
+
+def _quantize_swapped_nibbles(w):
+    q = dict(_orig_quantize(w))
+    p = q["packed"]
+    q["packed"] = (((p & 0x0F) << 4) | (p >> 4)).astype(np.uint8)   # element 2j in the low nibble
+    return q
+
+
+def _quantize_offset_off(w):
+    q = dict(_orig_quantize(w))
+    q["offset"] = np.float32(q["offset"] * 1.01)
+    return q
+
+
+_orig_nearest = codebooks.nearest_index
+_orig_quantize = quant.quantize
 _orig_attention = layer.attention
 _orig_attention_bwd = layer.attention_bwd
 _orig_ce = model.cross_entropy
@@ -65,6 +88,12 @@ CASES = [
     ("cross-entropy shift", model, "cross_entropy", _ce_unshifted,
      [P.test_cross_entropy_gradient_matches_torch_autograd, P.test_model_step_matches_transformers_llama_autograd]),
     ("AdamW bias correction", model, "adamw", _adamw_no_bias_correction, [P.test_adamw_matches_torch]),
+    ("NF4 code off by one", codebooks, "nearest_index", _nearest_off_by_one,
+     [Q.test_quantizer_properties, lambda: Q.test_quantizer_brute_force(64 * 4, 0)]),
+    ("nibble order", quant, "quantize", _quantize_swapped_nibbles,
+     [Q.test_quantizer_properties, Q.test_nibble_order_high_first]),
+    ("offset", quant, "quantize", _quantize_offset_off,
+     [Q.test_quantizer_properties, lambda: Q.test_quantizer_brute_force(64 * 4, 0)]),
 ]
 
 
