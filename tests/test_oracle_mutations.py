@@ -25,6 +25,15 @@ def _attention_no_scale(q, k, v):
     return _orig_attention(q * np.sqrt(q.shape[-1]), k, v)               # forgets 1/sqrt(d)
 
 
+def _attention_gqa_interleaved(q, k, v):
+    # query head h read kv head h % n_kv instead of h // (n_q / n_kv)
+    nq, nkv = q.shape[2], k.shape[2]
+    order = [(h % nkv) * (nq // nkv) + h // nkv for h in range(nq)]
+    o, Pr = _orig_attention(q[:, :, order], k, v)
+    inv = np.argsort(order)
+    return o[:, :, inv], Pr[:, inv]
+
+
 def _attention_bwd_dk_without_q(q, k, v, Pr, do):
     dq, dk, dv = _orig_attention_bwd(q, k, v, Pr, do)
     return dq, dk * 0.5, dv                                              # a halved dK
@@ -80,6 +89,8 @@ CASES = [
     ("attention scale", layer, "attention", _attention_no_scale,
      [P.test_attention_matches_torch_sdpa,
       lambda: P.test_layer_forward_matches_transformers_llama_decoder_layer(False)]),
+    ("attention GQA mapping", layer, "attention", _attention_gqa_interleaved,
+     [P.test_attention_matches_torch_sdpa]),
     ("attention dK", layer, "attention_bwd", _attention_bwd_dk_without_q,
      [P.test_attention_backward_matches_torch_autograd,
       lambda: P.test_layer_backward_finite_differences(1, 8)]),
