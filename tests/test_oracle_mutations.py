@@ -5,7 +5,8 @@ meant to guard that step now fails.  Nothing here touches the product path."""
 import numpy as np
 import pytest
 
-from oracle import codebooks, layer, model, quant
+from oracle import bf16, codebooks, layer, model, quant
+from tests import test_oracle_bf16 as F
 from tests import test_oracle_layer as P
 from tests import test_oracle_quant as Q
 
@@ -75,6 +76,30 @@ def _quantize_offset_off(w):
     return q
 
 
+def _bf16_truncating(x):
+    b = np.ascontiguousarray(np.asarray(x, dtype=np.float32)).view(np.uint32)
+    return (b >> np.uint32(16)).astype(np.uint16)                       # drops the low half: rounds toward 0
+
+
+def _bf16_ties_away(x):
+    b = np.ascontiguousarray(np.asarray(x, dtype=np.float32)).view(np.uint32).astype(np.uint64)
+    return ((b + np.uint64(0x8000)) >> np.uint64(16)).astype(np.uint16)  # halfway cases go up in magnitude
+
+
+def _round_f64_ties_away(x):
+    a = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+    b = a.view(np.uint64)
+    b = (b + np.uint64(1 << 44)) & ~np.uint64((1 << 45) - 1)
+    return b.view(np.float64)
+
+
+def _block_scales_group_of_64(q):
+    code8 = codebooks.code8_table()
+    gidx = np.minimum(np.arange(q["q8"].size) // 64, q["nested"].size - 1)   # groups of 64 blocks
+    prod = (code8[q["q8"].astype(np.int64)] * q["nested"][gidx]).astype(np.float32)
+    return (prod + np.float32(q["offset"])).astype(np.float32)
+
+
 _orig_nearest = codebooks.nearest_index
 _orig_quantize = quant.quantize
 _orig_attention = layer.attention
@@ -105,6 +130,15 @@ CASES = [
      [Q.test_quantizer_properties, Q.test_nibble_order_high_first]),
     ("offset", quant, "quantize", _quantize_offset_off,
      [Q.test_quantizer_properties, lambda: Q.test_quantizer_brute_force(64 * 4, 0)]),
+    ("bf16 truncation", bf16, "f32_to_bf16_bits", _bf16_truncating,
+     [F.test_f32_to_bf16_bits_matches_torch_on_constructed_patterns, F.test_f32_to_bf16_ties_go_to_even,
+      Q.test_dequant_across_nested_groups_with_different_scales]),
+    ("bf16 ties away", bf16, "f32_to_bf16_bits", _bf16_ties_away,
+     [F.test_f32_to_bf16_bits_matches_torch_on_constructed_patterns, F.test_f32_to_bf16_ties_go_to_even]),
+    ("float64 bf16 ties away", bf16, "round_f64", _round_f64_ties_away,
+     [F.test_round_f64_ties_and_near_ties]),
+    ("nested group of 64 blocks", quant, "block_scales", _block_scales_group_of_64,
+     [Q.test_dequant_across_nested_groups_with_different_scales]),
 ]
 
 

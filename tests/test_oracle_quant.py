@@ -9,9 +9,11 @@ import io
 import json
 import math
 import os
+from fractions import Fraction
 
 import numpy as np
 import pytest
+import torch
 
 from oracle import account, bf16, codebooks, quant
 from nf4_layer_streamed_b200 import synth
@@ -124,12 +126,13 @@ def test_bytes_per_param_and_store_sizes_from_pages():
 # ----------------------------------------------------------------------------- quantiser
 
 def _brute_quantize(w):
-    """Pure-Python loops over blocks, elements and all table entries."""
+    """Pure-Python loops over blocks, elements and all table entries.  Also returns the
+    fp32 ratios u = x / absmax and c / nested that each nearest-entry choice was made on."""
     nf4 = [float(v) for v in codebooks.nf4_table()]
     c8 = [float(v) for v in codebooks.code8_table()]
     x = [float(v) for v in np.asarray(w, np.float32)]
     nb = len(x) // 64
-    absmax, codes = [], []
+    absmax, codes, us = [], [], []
     for b in range(nb):
         blk = x[b * 64:(b + 1) * 64]
         am = max(abs(v) for v in blk)
@@ -137,16 +140,18 @@ def _brute_quantize(w):
         for v in blk:
             if am == 0.0:
                 codes.append(nf4.index(0.0))
+                us.append(None)
                 continue
             u = float(np.float32(v) / np.float32(am))
             best = min(range(16), key=lambda j: (abs(u - nf4[j]), j))
             codes.append(best)
+            us.append(u)
     tot = 0.0
     for am in absmax:
         tot += am
     offset = float(np.float32(tot / nb))
     cs = [float(np.float32(np.float32(am) - np.float32(offset))) for am in absmax]
-    nested, q8 = [], []
+    nested, q8, uus = [], [], []
     for g in range(0, nb, 256):
         grp = cs[g:g + 256]
         nm = max(abs(c) for c in grp)
@@ -154,11 +159,29 @@ def _brute_quantize(w):
         for c in grp:
             if nm == 0.0:
                 q8.append(c8.index(0.0))
+                uus.append(None)
                 continue
             u = float(np.float32(c) / np.float32(nm))
             q8.append(min(range(256), key=lambda j: (abs(u - c8[j]), j)))
+            uus.append(u)
     packed = [(codes[2 * j] << 4) | codes[2 * j + 1] for j in range(len(codes) // 2)]
-    return packed, q8, nested, offset
+    return packed, q8, nested, offset, codes, us, uus
+
+
+def _check_choices(got, want, ratios, table):
+    """Every choice equals the exact nearest entry, except where the ratio lies between
+    the exact midpoint of two neighbouring entries and that midpoint rounded to fp32
+    (the stated fp32-midpoint rule); there the two choices must be those neighbours."""
+    t = [Fraction(float(v)) for v in table]
+    got, want = np.asarray(got), np.asarray(want)
+    for i in np.nonzero(got != want)[0]:
+        a, b = sorted((int(got[i]), int(want[i])))
+        assert b == a + 1, (i, got[i], want[i])
+        exact_mid = (t[a] + t[b]) / 2
+        f32_mid = Fraction(float(np.float32(float(exact_mid))))
+        u = Fraction(ratios[i])
+        assert min(exact_mid, f32_mid) <= u <= max(exact_mid, f32_mid), (i, float(u), float(exact_mid))
+    return int(np.count_nonzero(got != want))
 
 
 @pytest.mark.parametrize("n,seed", [(64 * 4, 0), (64 * 300, 1), (64 * 513, 2)])
@@ -167,13 +190,29 @@ def test_quantizer_brute_force(n, seed):
     w = bf16.round_f32(rng.normal(0, 0.02, n).astype(np.float32))
     w[:64] = 0.0                       # a zero block
     q = quant.quantize(w)
-    packed, q8, nested, offset = _brute_quantize(w)
+    packed, q8, nested, offset, codes, us, uus = _brute_quantize(w)
     assert q["offset"] == np.float32(offset)
     np.testing.assert_array_equal(q["nested"], np.array(nested, np.float32))
-    # nearest-entry choices may differ only inside the fp32-midpoint window; check bytes
-    # where the brute force is unambiguous, and that all choices are near-optimal.
-    assert np.mean(q["packed"] == np.array(packed, np.uint8)) > 0.999
-    assert np.mean(q["q8"] == np.array(q8, np.uint8)) > 0.999
+    _check_choices(quant.unpack_codes(q["packed"]), codes, us, codebooks.nf4_table())
+    _check_choices(q["q8"], q8, uus, codebooks.code8_table())
+
+
+def test_quantizer_brute_force_at_midpoints():
+    """Ratios placed exactly on, and one fp32 ulp either side of, every fp32 midpoint
+    of the NF4 table: the oracle's choices differ from the exact nearest entry only
+    inside the fp32-midpoint window, and an exact fp32 tie goes to the lower index."""
+    nf4 = codebooks.nf4_table()
+    mids = codebooks.midpoints(nf4)
+    u = np.concatenate([mids, np.nextafter(mids, np.float32(2)), np.nextafter(mids, np.float32(-2))])
+    u = np.concatenate([u, np.zeros((-u.size) % 64 + 64, np.float32)])
+    u[63] = 1.0                                      # absmax 1 in the first block: x / absmax = x
+    w = u.astype(np.float32)
+    w[64:128] = np.where(np.arange(64) == 0, 1.0, w[64:128]).astype(np.float32)
+    q = quant.quantize(w)
+    _, _, _, _, codes, us, _ = _brute_quantize(w)
+    _check_choices(quant.unpack_codes(q["packed"]), codes, us, nf4)
+    got = quant.unpack_codes(q["packed"])[:mids.size]
+    np.testing.assert_array_equal(got, np.arange(mids.size))   # on the fp32 midpoint: lower index
 
 
 def test_nibble_order_high_first():
@@ -217,6 +256,71 @@ def test_dequant_error_bound_and_zero_block():
     bound = g4 * absmax[:, None] + g8 * nested_max + 2.0 ** -8 * np.abs(xb) + 1e-9
     assert np.all(np.abs(xb - wh.reshape(-1, 64)) <= bound)
     assert np.all(wh.reshape(-1, 64)[10] == 0.0)
+
+
+def _multi_group_tensor():
+    """3 full nested groups and a partial fourth (50 blocks) whose deviations of the
+    block absmax from the mean are scaled by 1, 2^-8, 2^6 and 2^-4 (|d| below 2^-7,
+    2^-15, 2^-1 and 2^-11).  Deviations come in +d / -d pairs of multiples of 2^-23
+    around 1, so the fp32 absmax values are exact, their mean (the offset) is exactly
+    1, and each group's nested absmax is exactly its largest |d|.  Each block holds
+    its absmax once (with a random sign) and NF4 table values times it elsewhere."""
+    rng = np.random.default_rng(21)
+    scales = [1.0, 2.0 ** -8, 2.0 ** 6, 2.0 ** -4]
+    sizes = [256, 256, 256, 50]
+    nf4 = codebooks.nf4_table()
+    absmax, nested = [], []
+    for sc, nb in zip(scales, sizes):
+        k = rng.integers(1, int(2 ** 16 * sc), nb // 2)  # |d| = k * 2^-23 < 2^-7 * scale
+        d = np.concatenate([k, -k]).astype(np.float64) * 2.0 ** -23
+        rng.shuffle(d)
+        absmax.append(1.0 + d)
+        nested.append(float(np.max(np.abs(d))))
+    absmax = np.concatenate(absmax)
+    assert np.all(absmax.astype(np.float32).astype(np.float64) == absmax)
+    nb = absmax.size
+    codes = rng.integers(0, 16, (nb, 64))
+    top = rng.integers(0, 64, nb)
+    codes[np.arange(nb), top] = np.where(rng.random(nb) < 0.5, 0, 15)     # the -1 or +1 entry
+    w = (nf4[codes].astype(np.float64) * absmax[:, None]).astype(np.float32)
+    # the fp32 product nf4[c] * absmax can round; the block's largest magnitude is exact
+    assert np.all(np.abs(w).max(axis=1).astype(np.float64) == absmax)
+    return w.reshape(-1), absmax, np.array(nested), np.array(sizes)
+
+
+def test_dequant_across_nested_groups_with_different_scales():
+    """Pins the nested-group indexing of the double quantisation and of the scale
+    decode: the offset is exactly 1, each group's nested absmax is its own largest
+    deviation (groups of 256 consecutive blocks, the last one partial), each decoded
+    block scale is within half an 8-bit table gap times its OWN group's nested absmax
+    of the true absmax (a wrong group would be off by up to 2^14 of that), and the
+    dequantised weights equal a pure-Python per-element decode."""
+    w, absmax, nested, sizes = _multi_group_tensor()
+    q = quant.quantize(w)
+    assert q["offset"] == np.float32(1.0)
+    np.testing.assert_array_equal(q["nested"].astype(np.float64), nested)
+    c8 = codebooks.code8_table().astype(np.float64)
+    halfgap = np.max(np.diff(c8)) / 2
+    group = np.repeat(np.arange(sizes.size), sizes)
+    s = quant.block_scales(q).astype(np.float64)
+    err = np.abs(s - absmax)
+    # two fp32 roundings (the product and the sum with 1) add at most 2^-23 + 2^-24 each
+    assert np.all(err <= halfgap * nested[group] + 2.0 ** -22), np.max(err / nested[group])
+    # the smallest groups resolve far below the largest group's table gap
+    assert np.max(err[group == 1]) < halfgap * nested[2] * 2.0 ** -10
+
+    nf4 = [float(v) for v in codebooks.nf4_table()]
+    c8f = [float(v) for v in codebooks.code8_table()]
+    bits = quant.dequantize_bits(q)
+    packed, q8, nst, off = list(q["packed"]), list(q["q8"]), list(q["nested"]), np.float32(q["offset"])
+    for i in range(0, w.size, 7):                   # every 7th element, across all four groups
+        b = i // 64
+        g = b // 256
+        c = (packed[i // 2] >> 4) if i % 2 == 0 else (packed[i // 2] & 15)
+        sc = np.float32(np.float32(np.float32(c8f[q8[b]]) * np.float32(nst[g])) + off)
+        val = np.float32(np.float32(nf4[c]) * sc)
+        ref = int(torch.from_numpy(np.array([val], np.float32)).to(torch.bfloat16).view(torch.int16)[0]) & 0xFFFF
+        assert int(bits[i]) == ref, (i, b, g)
 
 
 def test_quantize_deterministic_and_roundtrip_through_bytes():
