@@ -1,7 +1,7 @@
 // K10: causal grouped-query attention, forward and deterministic backward.
 //
 // The attention of the HF Llama decoder layer that the pages' system runs through
-// functional_call ("Soup layer-streamed NF4 gate record" §2.1): softmax(q k^T / sqrt(d)
+// functional_call ("Soup 层流式 NF4 训练实测：在 4 GB 显存上以位级一致标准完成 8B 模型 LoRA 微调" §2.1): softmax(q k^T / sqrt(d)
 // + causal mask) v, with key/value head h / (n_q / n_kv) serving query head h.
 // At seq 512 it is about 2% of the layer's FLOPs (the GEMM share table of §4.4 leaves
 // it out), so this round uses the warp-level bf16 tensor-core instruction

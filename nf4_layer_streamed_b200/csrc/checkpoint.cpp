@@ -1,7 +1,7 @@
 // Adapter checkpoint / resume.  The trainable state of the run is the LoRA adapter
 // (A and B of every adapted projection, fp32), the AdamW moments and the step count
 // that drives the bias correction; the NF4 base is frozen and comes back from its
-// own shards.  "Soup layer-streamed NF4 gate record" §3.2 records a release whose
+// own shards.  "Soup 层流式 NF4 训练实测：在 4 GB 显存上以位级一致标准完成 8B 模型 LoRA 微调" §3.2 records a release whose
 // adapters were written correctly during training but read back as empty, and no
 // test had saved an adapter and loaded it again: here the loader refuses any file
 // whose shapes, size or checksum do not match, before it touches the device, and

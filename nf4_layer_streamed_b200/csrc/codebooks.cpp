@@ -1,5 +1,5 @@
 // Code tables of the double-quantised NF4 format, built on the host from the
-// published constructions.  "Soup layer-streamed NF4 gate record" §2.4: the NF4
+// published constructions.  "Soup 层流式 NF4 训练实测：在 4 GB 显存上以位级一致标准完成 8B 模型 LoRA 微调" §2.4: the NF4
 // table (16 fp32) and the nested table (256 fp32) are constant for every weight,
 // so one resident copy is shared and the shard records their hash.
 //

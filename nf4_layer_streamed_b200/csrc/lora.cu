@@ -1,7 +1,8 @@
 // K6/K7: the LoRA products of the q_proj and v_proj adapters (r = 16).
 //
-// "Soup v0.72.4 技术解析" §4.2 (LoRA r=16, alpha=32 on q_proj and v_proj) and the
-// gate record §2.2 check 2 (LoRA gradients nonzero in every layer): the adapter
+// "Soup v0.72.4 技术解析" §4.2 (LoRA r=16, alpha=32 on q_proj and v_proj) and
+// "Soup 层流式 NF4 训练实测：在 4 GB 显存上以位级一致标准完成 8B 模型 LoRA 微调"
+// §2.2 check 2 (LoRA gradients nonzero in every layer): the adapter
 // adds s (x A^T) B^T to the q and v projections (s = alpha / r) and trains A and B.
 // The up-projection is folded into the q/k/v GEMM as an extra 64-wide reduction
 // block; this file holds the skinny products around it, all of them HBM-bound:

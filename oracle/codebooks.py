@@ -1,6 +1,6 @@
 """Code tables of the double-quantised NF4 format (oracle; test infrastructure only).
 
-Source for what the tables are: "Soup layer-streamed NF4 gate record"
+Source for what the tables are: "Soup 层流式 NF4 训练实测：在 4 GB 显存上以位级一致标准完成 8B 模型 LoRA 微调"
 (m.mzlw.cn), §2.4 -- the NF4 code table holds 16 fp32 values, the nested
 (absmax) code table 256 fp32 values, both constant for every weight, which is
 why one resident copy is shared.  The pages print neither table, so the

@@ -3,7 +3,7 @@
 
 Follows the training step of the pages' system: frozen NF4 decoder layers,
 resident unquantised bf16 embedding and lm_head ("4GB 显存微调 8B 模型是真的",
-layer-streaming mechanism section; "Soup layer-streamed NF4 gate record"
+layer-streaming mechanism section; "Soup 层流式 NF4 训练实测：在 4 GB 显存上以位级一致标准完成 8B 模型 LoRA 微调",
 §4.3), LoRA r=16 / alpha=32 on q_proj and v_proj trained with AdamW.
 
 Readings: cross-entropy of logits[t] against ids[t+1] for t = 0..S-2 of each

@@ -1,6 +1,6 @@
 """Blockwise NF4 with double-quantised absmax (oracle; test infrastructure only).
 
-What is computed follows "Soup layer-streamed NF4 gate record" (m.mzlw.cn)
+What is computed follows "Soup 层流式 NF4 训练实测：在 4 GB 显存上以位级一致标准完成 8B 模型 LoRA 微调" (m.mzlw.cn)
 §2.1 (offline per-tensor quantisation into packed bytes plus absmax, nested
 absmax and offset sidecars) and §2.4 (per-weight streamed bytes: N/2 packed +
 N/64 absmax + N/4096 nested absmax + 4 bytes offset, about 0.516 B/param;

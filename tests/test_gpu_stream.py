@@ -3,7 +3,7 @@ SmolLM2-shaped training run streamed at depth 2 and 3 against the HBM-resident r
 (25 AdamW steps, loss curves and adapters bit-equal; first step against the oracle),
 the poisoned-pool run, and the 32B-class layers above the 165 MiB aliasing threshold
 whose LoRA gradients after buffer reuse must equal the resident gradients exactly.
-These are the gate-record checks of "Soup layer-streamed NF4 gate record" §2.2 (streamed
+These are the gate-record checks of "Soup 层流式 NF4 训练实测：在 4 GB 显存上以位级一致标准完成 8B 模型 LoRA 微调" §2.2 (streamed
 = resident, n=2 = n=3, same-seed reruns, nonzero LoRA gradients in every layer) and the
 Issue #331 scenario of the layer-streaming review's bug history."""
 import ctypes
@@ -258,7 +258,7 @@ def test_32b_class_layers_over_165mib_gradients_after_reuse_equal_resident():
 def test_adapter_checkpoint_resume_is_bit_exact(tmp_path):
     """Six streamed steps in one run equal three steps, a save, a new model that
     loads the file and three more steps: losses, adapter and both AdamW moments
-    bit-equal ("Soup layer-streamed NF4 gate record" §3.2: an adapter that was
+    bit-equal ("Soup 层流式 NF4 训练实测：在 4 GB 显存上以位级一致标准完成 8B 模型 LoRA 微调" §3.2: an adapter that was
     saved must come back, not load as a no-op)."""
     wl = synth.WORKLOADS["smollm2_30L_tied_b1s512"]
     ids = [synth.token_ids(wl.vocab, wl.batch, wl.seq, wl.seed, step=s, device=DEV) for s in range(6)]
