@@ -84,6 +84,17 @@ int nf4ls_profile_reset(void);
  * Synchronises the device. */
 int nf4ls_device_error(int32_t out[4]);
 
+/* Exercises the expiry of a bounded wait, the path a kernel takes instead of
+ * hanging when an arrival it waits for never comes.  Launches one block of two warps
+ * on `stream` that wait on an mbarrier nothing arrives on: warp 0 gives up after
+ * limit_us microseconds and records code 1, kernel id 3, block 0, site 1 in the
+ * device error record; warp 1 (limit 1000x longer) leaves through the abort flag
+ * that warp 0 raised.  result_dev: 2 int32 (device), set to 0 for each warp whose
+ * wait did not complete.  The kernel ends by itself; the context stays usable.
+ * NF4LS_INVALID_ARG for limit_us outside [1, 1e6] or a NULL result.  No passage of
+ * the pages defines this: it is the library's own failure detection. */
+int nf4ls_wait_probe(int32_t limit_us, int32_t* result_dev, nf4ls_stream stream);
+
 /* ------------------------------------------------------------------ code tables
  * [gate] §2.4: the NF4 code table (16 fp32) and the nested absmax table (256 fp32)
  * are constant for every weight, so one resident copy is shared; the shard records
@@ -158,7 +169,10 @@ int nf4_dequantize_tensor(const uint8_t* packed_dev, const uint8_t* q8_dev, cons
  * nf4ls_quantize_noalloc_max_elems() weights (2^28, 16 MiB of device memory held by
  * every GPU that loads the library until the process exits).  Larger n returns
  * NF4LS_INVALID_ARG.  The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress); make it before any stream capture.  All calls share the
+ * (cudaGetSymbolAddress); make it before any stream capture.  The first call in a
+ * new CUDA context on that device (after a device reset, or under a context the
+ * caller created) looks it up again, since an address is valid only in the context
+ * it came from.  All calls share the
  * array, so calls that overlap on the GPU race; serialise them on one stream.  No
  * part of the array needs to start at zero.  Allocates nothing; results are the same
  * bytes nf4_quantize_tensor produces. */
@@ -342,6 +356,44 @@ int nf4ls_pool_destroy(nf4ls_pool* pool);
 int nf4ls_nccl_unique_id(uint8_t id_out[128]);
 int nf4ls_pool_share(nf4ls_pool* pool, int rank, int world, const uint8_t id[128]);
 
+/* ------------------------------------------------------------------ slot plan (host only)
+ * The slot decisions behind every pool call, with no device work, so that they can be
+ * checked without a GPU (for instance on several CPU ranks, for the sharded fetch):
+ * the pool takes each of its decisions through this same plan object.  A plan has the
+ * pool's depth and layer count; nf4ls_plan_share switches it to the sharded fetch
+ * (before it holds a layer, as nf4ls_pool_share).  nf4ls_plan_prefetch,
+ * nf4ls_plan_acquire and nf4ls_plan_release mirror nf4ls_pool_prefetch,
+ * stream_prefetch and nf4ls_pool_release, return the same statuses
+ * (NF4LS_BUFFER_BUSY when every slot is acquired or filled and not yet acquired, or
+ * when the layer is already acquired; the plan is then unchanged) and fill `out`
+ * (may be NULL) with what the pool does for that call. */
+typedef struct nf4ls_plan nf4ls_plan;
+
+typedef struct {
+    int32_t slot;           /* the slot that serves the layer                            */
+    int32_t hit;            /* 1: the layer already sat in that slot, nothing is copied  */
+    int32_t fill;           /* 1: this call fills the slot                               */
+    int32_t after_release;  /* 1: the fill waits for the slot's previous release event   */
+    int32_t owner;          /* the rank that reads the layer from its host store         */
+    int32_t host_read;      /* 1: this rank copies it from its own store                 */
+    int32_t broadcast;      /* 1: shared pool: the fill is a broadcast from the owner    */
+} nf4ls_plan_step;
+
+int nf4ls_plan_create(int n_layers, int depth, nf4ls_plan** out);
+int nf4ls_plan_share(nf4ls_plan* plan, int rank, int world);
+int nf4ls_plan_prefetch(nf4ls_plan* plan, int layer, nf4ls_plan_step* out);
+int nf4ls_plan_acquire(nf4ls_plan* plan, int layer, nf4ls_plan_step* out);
+int nf4ls_plan_release(nf4ls_plan* plan, int layer);
+int nf4ls_plan_destroy(nf4ls_plan* plan);
+
+/* The pool calls one pass of nf4ls_forward_backward makes (dir +1: the forward over
+ * layers 0..n-1; dir -1: the backward over n-1..0), in order: op 0 = acquire
+ * (stream_prefetch), 1 = prefetch (nf4ls_pool_prefetch; on NF4LS_BUFFER_BUSY the step
+ * skips the remaining prefetches for that layer), 2 = run the layer, 3 = release.
+ * ops[i], layers[i] for i < *n_out; NF4LS_INVALID_ARG (with *n_out set) when cap is
+ * too small. */
+int nf4ls_step_pass_ops(int n_layers, int dir, int32_t* ops, int32_t* layers, int cap, int32_t* n_out);
+
 /* ------------------------------------------------------------------ disk stream source
  * [review] mechanism section: the frozen base lives in (pinned) host memory and falls
  * back to an NVMe disk when memory is short; SATA and spinning disks are refused
@@ -453,17 +505,20 @@ int nf4ls_adamw_step(const nf4ls_model_cfg* cfg, const nf4ls_model* model, int32
  *
  * File: a 64-byte header (magic NF4LS_ADAPTER_MAGIC, version, H, I, n_q, n_kv,
  * head_dim, lora_r, n_layers, lora_alpha, step, floats per array, FNV-1a 64
- * checksum of the arrays) then the three fp32 arrays, little-endian, in the device
- * layout.  nf4ls_adapter_file_bytes gives its size (0 for a NULL or empty config).
+ * checksum over the header with that field zeroed and then the arrays) then the
+ * three fp32 arrays, little-endian, in the device layout.  nf4ls_adapter_file_bytes
+ * gives its size (0 for a NULL or empty config).
  *
  * nf4ls_adapter_save: copies the three arrays to the host on `stream` (ordered after
- * the steps already queued there), writes path + ".tmp", fsyncs it and renames it to
- * path, so an interrupted save leaves an older file at path intact.  step >= 0 is
- * stored as given: pass the count of AdamW steps applied so far.  NF4LS_IO on a
- * failed open / write / rename (the temporary file is removed).
+ * the steps already queued there), writes path + ".tmp", fsyncs it, renames it to
+ * path and fsyncs the directory, so an interrupted save leaves an older file at
+ * path intact and a completed one survives a crash.  step >= 0 is stored as given:
+ * pass the count of AdamW steps applied so far.  NF4LS_IO on a failed open / write /
+ * rename / directory flush (the temporary file is removed).
  *
  * nf4ls_adapter_load: reads and checks the whole file first; NF4LS_INVALID_ARG for a
- * wrong magic or version, NF4LS_SHAPE when H, I, heads, head_dim, lora_r, lora_alpha,
+ * wrong magic or version (files of version 1, whose checksum left the header out,
+ * are refused), NF4LS_SHAPE when H, I, heads, head_dim, lora_r, lora_alpha,
  * n_layers or the array size differ from cfg (batch and seq may differ), NF4LS_IO
  * for a short, over-long or checksum-failing file.  Only then are the three device
  * arrays overwritten (on `stream`, synchronised before return) and *step set; on any
@@ -471,7 +526,7 @@ int nf4ls_adamw_step(const nf4ls_model_cfg* cfg, const nf4ls_model* model, int32
  * the resumed run passes *step + 1.  The gradient buffer is not saved: every step
  * rewrites it. */
 #define NF4LS_ADAPTER_MAGIC   0x41344E46u /* "FN4A" little-endian */
-#define NF4LS_ADAPTER_VERSION 1u
+#define NF4LS_ADAPTER_VERSION 2u
 size_t nf4ls_adapter_file_bytes(const nf4ls_model_cfg* cfg);
 int nf4ls_adapter_save(const char* path, const nf4ls_model_cfg* cfg, const nf4ls_model* model, int32_t step,
                        nf4ls_stream stream);

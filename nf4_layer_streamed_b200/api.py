@@ -152,6 +152,14 @@ def device_error():
     return st, list(out)
 
 
+def wait_probe(limit_us: int, result: torch.Tensor, stream=None) -> None:
+    """Launches the bounded-wait expiry probe (a wait that nothing ends) on the
+    stream; result: int32 [2] on the device, 0 per warp whose wait gave up."""
+    _need(result, "result", torch.int32, 2)
+    _need_cuda(result=result)
+    B.call("nf4ls_wait_probe", int(limit_us), _p(result), _s(stream))
+
+
 # ----------------------------------------------------------------------------- NF4 tensors
 
 def nf4_quantize_tensor(w: torch.Tensor, stream=None) -> dict:
@@ -408,6 +416,65 @@ class Pool:
         """A uint8 view of the slot at device address ptr (for reading a streamed shard)."""
         off = ptr - self.slots.data_ptr()
         return self.slots[off: off + nbytes]
+
+
+class SlotPlan:
+    """The pool's slot decisions on the host (no device work): prefetch / acquire /
+    release return what the pool does for the same call (slot, hit, fill, wait for
+    the slot's release, owner rank, host read, broadcast) as a dict."""
+
+    def __init__(self, n_layers: int, depth: int):
+        h = ctypes.c_void_p()
+        B.call("nf4ls_plan_create", n_layers, depth, ctypes.byref(h))
+        self.handle = h
+
+    @staticmethod
+    def _dict(st: B.PlanStep) -> dict:
+        return {k: int(getattr(st, k)) for k, _ in B.PlanStep._fields_}
+
+    def share(self, rank: int, world: int) -> None:
+        B.call("nf4ls_plan_share", self.handle, rank, world)
+
+    def prefetch(self, layer: int):
+        """The step dict, or None when the pool would answer BUFFER_BUSY."""
+        st = B.PlanStep()
+        r = B.call_status("nf4ls_plan_prefetch", self.handle, layer, ctypes.byref(st))
+        if r == -6:
+            return None
+        B.check(r)
+        return self._dict(st)
+
+    def acquire(self, layer: int) -> dict:
+        st = B.PlanStep()
+        B.call("nf4ls_plan_acquire", self.handle, layer, ctypes.byref(st))
+        return self._dict(st)
+
+    def release(self, layer: int) -> None:
+        B.call("nf4ls_plan_release", self.handle, layer)
+
+    def close(self) -> None:
+        if self.handle:
+            B.lib().nf4ls_plan_destroy(self.handle)
+            self.handle = None
+
+    def __enter__(self) -> "SlotPlan":
+        return self
+
+    def __exit__(self, *exc) -> None:
+        self.close()
+
+
+PASS_OPS = ("acquire", "prefetch", "run", "release")
+
+
+def step_pass_ops(n_layers: int, direction: int) -> list:
+    """[(op name, layer)] of the pool calls one pass of the model step makes."""
+    n = ctypes.c_int32(0)
+    B.call_status("nf4ls_step_pass_ops", n_layers, direction, None, None, 0, ctypes.byref(n))
+    ops = (ctypes.c_int32 * n.value)()
+    layers = (ctypes.c_int32 * n.value)()
+    B.call("nf4ls_step_pass_ops", n_layers, direction, ops, layers, n.value, ctypes.byref(n))
+    return [(PASS_OPS[o], l) for o, l in zip(ops, layers)]
 
 
 def nccl_unique_id() -> bytes:

@@ -63,6 +63,12 @@ class PoolStats(ctypes.Structure):
                 ("acquisitions", ctypes.c_uint64), ("peer_bytes", ctypes.c_uint64)]
 
 
+class PlanStep(ctypes.Structure):
+    _fields_ = [("slot", ctypes.c_int32), ("hit", ctypes.c_int32), ("fill", ctypes.c_int32),
+                ("after_release", ctypes.c_int32), ("owner", ctypes.c_int32), ("host_read", ctypes.c_int32),
+                ("broadcast", ctypes.c_int32)]
+
+
 class DiskInfo(ctypes.Structure):
     _fields_ = [("read_gbs", ctypes.c_double), ("block_device", ctypes.c_int32), ("nvme", ctypes.c_int32),
                 ("rotational", ctypes.c_int32), ("direct_io", ctypes.c_int32)]
@@ -78,6 +84,7 @@ SIGNATURES = {
     "nf4ls_last_error": (ctypes.c_char_p, []),
     "nf4ls_version": (ctypes.c_int, []),
     "nf4ls_device_error": (ctypes.c_int, [P]),
+    "nf4ls_wait_probe": (ctypes.c_int, [ctypes.c_int32, P, P]),
     "nf4ls_launch_count": (U64, []),
     "nf4ls_profile": (ctypes.c_int, [ctypes.c_int]),
     "nf4ls_profile_read": (ctypes.c_int, [ctypes.c_int, P]),
@@ -112,6 +119,13 @@ SIGNATURES = {
     "nf4ls_pool_destroy": (ctypes.c_int, [P]),
     "nf4ls_nccl_unique_id": (ctypes.c_int, [P]),
     "nf4ls_pool_share": (ctypes.c_int, [P, ctypes.c_int, ctypes.c_int, P]),
+    "nf4ls_plan_create": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.POINTER(P)]),
+    "nf4ls_plan_share": (ctypes.c_int, [P, ctypes.c_int, ctypes.c_int]),
+    "nf4ls_plan_prefetch": (ctypes.c_int, [P, ctypes.c_int, ctypes.POINTER(PlanStep)]),
+    "nf4ls_plan_acquire": (ctypes.c_int, [P, ctypes.c_int, ctypes.POINTER(PlanStep)]),
+    "nf4ls_plan_release": (ctypes.c_int, [P, ctypes.c_int]),
+    "nf4ls_plan_destroy": (ctypes.c_int, [P]),
+    "nf4ls_step_pass_ops": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, P, P, ctypes.c_int, ctypes.POINTER(I32)]),
     "nf4ls_disk_probe": (ctypes.c_int, [ctypes.c_char_p, SZ, ctypes.POINTER(DiskInfo)]),
     "nf4ls_disk_accept": (ctypes.c_int, [ctypes.POINTER(DiskInfo), ctypes.c_double]),
     "nf4ls_choose_source": (ctypes.c_int, [SZ, SZ, ctypes.POINTER(ctypes.c_int32)]),

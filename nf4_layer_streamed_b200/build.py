@@ -21,7 +21,7 @@ BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libnf4ls.so")
 INCLUDE = os.path.join(ROOT, "include")
 
-SOURCES = ["abi.cpp", "codebooks.cpp", "pool.cpp", "device.cu", "quant.cu", "gemm.cu", "body.cu", "lora.cu", "noalloc.cu",
+SOURCES = ["abi.cpp", "codebooks.cpp", "plan.cpp", "pool.cpp", "device.cu", "quant.cu", "gemm.cu", "body.cu", "lora.cu", "noalloc.cu",
            "attention.cu", "attention_tc.cu", "layer.cu", "model.cu", "checkpoint.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",

@@ -11,7 +11,9 @@
 // n_floats fp32 each, in the order LoRA parameters, AdamW first moment, AdamW
 // second moment.  Each array is the device layout as is: n_layers blocks of
 // nf4ls_lora_stride floats, [A_q | B_q | A_v | B_v] per layer.  The header's
-// checksum is 64-bit FNV-1a over the three arrays' bytes in file order.
+// checksum is 64-bit FNV-1a over the header itself (with the checksum field set to
+// zero) and then the three arrays' bytes in file order, so a damaged step count or
+// alpha is refused like a damaged array.
 #include <errno.h>
 #include <fcntl.h>
 #include <stdio.h>
@@ -47,6 +49,25 @@ uint64_t fnv1a64(const void* data, size_t n, uint64_t h) {
   return h;
 }
 constexpr uint64_t kFnvBasis = 0xCBF29CE484222325ull;
+
+uint64_t file_checksum(const AdapterHeader& h, const float* arrays, size_t n_bytes) {
+  AdapterHeader z = h;
+  z.checksum = 0;
+  return fnv1a64(arrays, n_bytes, fnv1a64(&z, sizeof z, kFnvBasis));
+}
+
+// Makes a completed rename durable: the new directory entry is on disk once the
+// directory itself has been flushed.
+int fsync_parent_dir(const char* path) {
+  std::string dir(path);
+  const size_t slash = dir.find_last_of('/');
+  dir = slash == std::string::npos ? std::string(".") : (slash == 0 ? std::string("/") : dir.substr(0, slash));
+  const int fd = ::open(dir.c_str(), O_RDONLY | O_DIRECTORY | O_CLOEXEC);
+  if (fd < 0) return -1;
+  const int r = ::fsync(fd);
+  ::close(fd);
+  return r;
+}
 
 int check_args(const char* path, const nf4ls_model_cfg* c, const nf4ls_model* m, const char* who) {
   if (!path || !*path || !c || !m) return fail(NF4LS_INVALID_ARG, "%s: null path, config or model", who);
@@ -121,7 +142,7 @@ extern "C" int nf4ls_adapter_save(const char* path, const nf4ls_model_cfg* cfg, 
   h.lora_alpha = cfg->layer.lora_alpha;
   h.step = step;
   h.n_floats = n;
-  h.checksum = fnv1a64(host.data(), host.size() * sizeof(float), kFnvBasis);
+  h.checksum = file_checksum(h, host.data(), host.size() * sizeof(float));
 
   // Written under a temporary name and renamed into place, so a crash mid-write
   // leaves the previous checkpoint intact.
@@ -141,6 +162,8 @@ extern "C" int nf4ls_adapter_save(const char* path, const nf4ls_model_cfg* cfg, 
     ::unlink(tmp.c_str());
     return fail(NF4LS_IO, "nf4ls_adapter_save: rename to %s: %s", path, strerror(e));
   }
+  if (fsync_parent_dir(path) != 0)
+    return fail(NF4LS_IO, "nf4ls_adapter_save: flushing the directory of %s: %s", path, strerror(errno));
   return NF4LS_OK;
 }
 
@@ -184,7 +207,7 @@ extern "C" int nf4ls_adapter_load(const char* path, const nf4ls_model_cfg* cfg, 
   ::close(fd);
   if (rd != 0) return fail(NF4LS_IO, "nf4ls_adapter_load: %s is truncated", path);
   if (trailing) return fail(NF4LS_IO, "nf4ls_adapter_load: %s has bytes after the last array", path);
-  if (fnv1a64(host.data(), host.size() * sizeof(float), kFnvBasis) != h.checksum)
+  if (file_checksum(h, host.data(), host.size() * sizeof(float)) != h.checksum)
     return fail(NF4LS_IO, "nf4ls_adapter_load: %s fails its checksum", path);
 
   // Every check has passed: only now is the device state overwritten.

@@ -16,7 +16,7 @@ namespace nf4ls {
 // wait expired), [1] = kernel id, [2] = block, [3] = site.  The record lives in a
 // file-scope __device__ array of device.cu; its address is looked up per device.
 
-enum KernelId : int { KID_GEMM = 1, KID_ATTN = 2 };
+enum KernelId : int { KID_GEMM = 1, KID_ATTN = 2, KID_WAIT_PROBE = 3 };
 
 // A bounded wait gives up after this many nanoseconds of global time.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
@@ -89,17 +89,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Gives up when *abort is
-// set by another thread of the block, or after kWaitLimitNs, in which case it sets
+// set by another thread of the block, or after limit_ns, in which case it sets
 // *abort, records the site in the device error flag and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int* err, int kid, int site) {
+                                          int* err, int kid, int site,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const unsigned long long t0 = global_ns();
   while (true) {
     if (mbar_try_wait(a, parity)) return true;
     if (*abort_flag) return false;
-    if (global_ns() - t0 > kWaitLimitNs) {
+    if (global_ns() - t0 > limit_ns) {
       *abort_flag = 1;
       record_error(err, 1, kid, site);
       return false;

@@ -1,33 +1,82 @@
-// Device error record of libnf4ls.  Kernels with bounded waits (the tcgen05 GEMM)
-// write the site of an expired wait here instead of hanging; the host reads and
-// clears it through nf4ls_device_error().  The record is a file-scope __device__
-// array, so every device that loads the library holds its own copy; its address is
-// looked up once per device with cudaGetSymbolAddress.
+// Device error record of libnf4ls.  Kernels with bounded waits (the tcgen05 GEMM
+// and attention) write the site of an expired wait here instead of hanging; the host
+// reads and clears it through nf4ls_device_error().  The record is a file-scope
+// __device__ array, so every device that loads the library holds its own copy; its
+// address is looked up with cudaGetSymbolAddress once per CUDA context (again after a
+// device reset, which replaces the context).
 #include <atomic>
 #include <mutex>
 #include <vector>
 
+#include "common.cuh"
 #include "internal.h"
 
 namespace nf4ls {
 
 __device__ int g_dev_error[4];
 
+unsigned long long current_context_id() {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrent>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetId>(f);
+  });
+  CUcontext c = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&c) != CUDA_SUCCESS || !c || get_id(c, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
 int* device_error_ptr() {
   static int* ptrs[64] = {nullptr};
+  static unsigned long long ctx[64] = {0};
   static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  const unsigned long long id = current_context_id();
   std::lock_guard<std::mutex> g(mu);
-  if (!ptrs[dev]) {
+  if (!ptrs[dev] || id == 0 || id != ctx[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_dev_error) != cudaSuccess) return nullptr;
     ptrs[dev] = static_cast<int*>(p);
+    ctx[dev] = current_context_id();  // the lookup makes the device's primary context current
   }
   return ptrs[dev];
 }
 
 namespace {
+
+// The expiry path of the bounded mbarrier wait, on its own: one block of two warps
+// waits on an mbarrier that no thread ever arrives on.  Warp 0 waits limit_ns and
+// gives up (site 1), which records the error and raises the block's abort flag;
+// warp 1 waits on the same barrier with a limit a thousand times longer and must
+// leave through that flag without recording anything (site 2 never appears).  No
+// copy or tensor-core work is in flight, so giving up is safe here.
+__global__ void k_wait_probe(int* err, unsigned long long limit_ns, int32_t* result) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+  }
+  __syncthreads();
+  const int warp = threadIdx.x / 32;
+  const bool ok = warp == 0 ? mbar_wait(&bar, 0, &abort_flag, err, KID_WAIT_PROBE, 1, limit_ns)
+                            : mbar_wait(&bar, 0, &abort_flag, err, KID_WAIT_PROBE, 2, limit_ns * 1000ull);
+  if ((threadIdx.x & 31) == 0) result[warp] = ok ? 1 : 0;
+}
+
 std::atomic<uint64_t> g_launches{0};
 std::atomic<int> g_profile{0};
 struct Rec {
@@ -128,4 +177,18 @@ extern "C" int nf4ls_device_error(int32_t out[4]) {
   NF4_CUDA_TRY(cudaMemcpy(out, p, 4 * sizeof(int32_t), cudaMemcpyDeviceToHost));
   NF4_CUDA_TRY(cudaMemset(p, 0, 4 * sizeof(int32_t)));
   return out[0] ? NF4LS_DEVICE_FAULT : NF4LS_OK;
+}
+
+extern "C" int nf4ls_wait_probe(int32_t limit_us, int32_t* result_dev, nf4ls_stream stream) {
+  nf4ls::clear_error();
+  if (limit_us < 1 || limit_us > 1000000 || !result_dev)
+    return nf4ls::fail(NF4LS_INVALID_ARG, "nf4ls_wait_probe: limit_us %d outside [1, 1000000] or null result",
+                       limit_us);
+  int* err = nf4ls::device_error_ptr();
+  if (!err) return nf4ls::fail(NF4LS_CUDA, "nf4ls_wait_probe: no device record");
+  nf4ls::k_wait_probe<<<1, 64, 0, static_cast<cudaStream_t>(stream)>>>(err, 1000ull * (unsigned long long)limit_us,
+                                                                     result_dev);
+  nf4ls::note_launch();
+  NF4_CUDA_TRY(cudaGetLastError());
+  return NF4LS_OK;
 }

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <vector>
+
 #include "../../include/nf4ls.h"
 
 namespace nf4ls {
@@ -30,6 +32,87 @@ void clear_error();
 
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ----------------------------------------------------------------------------- slot plan
+// Host-only bookkeeping of a streaming pool's slots, with no CUDA state: which slot a
+// layer goes to, whether a request is served by a slot that already holds the layer
+// (a hit) or fills one, whether that fill must wait for the slot's previous reader,
+// and, under the layer-sharded fetch, which rank reads the layer from its host store.
+// The pool (pool.cpp) takes every slot decision here and adds only the CUDA work;
+// nf4ls_plan_* (plan.cpp) exports the same object so that the decisions can be driven
+// without a GPU.  Slots are reused least recently released first.
+struct PlanStep {
+  int slot = -1;
+  bool hit = false;            // the layer already sits in a slot: nothing is copied
+  bool fill = false;           // this request fills the slot
+  bool after_release = false;  // the slot was released before: the fill waits for that release
+  int owner = 0;               // the rank that reads the layer from its host store
+  bool host_read = false;      // fill and owner == this rank
+  bool broadcast = false;      // fill and the pool is shared: the owner's bytes go to every rank
+};
+
+class SlotPlan {
+ public:
+  void init(int n_layers, int depth);
+  void share(int rank, int world) {
+    rank_ = rank;
+    world_ = world;
+    shared_ = true;
+  }
+  int depth() const { return (int)s_.size(); }
+  int n_layers() const { return n_layers_; }
+  int find(int layer) const;         // the slot holding layer, or -1
+  bool holds_any() const;
+  bool acquired(int slot) const { return s_[slot].acquired; }
+  int layer_in(int slot) const { return s_[slot].layer; }
+  // What a request for layer would do, without changing anything (BUFFER_BUSY when it
+  // needs a slot and every slot is acquired or filled and not yet acquired).
+  int preview(int layer, PlanStep* st) const;
+  int issue(int layer, PlanStep* st);                  // preview, then take the slot
+  void mark_acquired(int slot);                        // the caller now reads the slot
+  int acquire(int layer, PlanStep* st);                // issue + BUFFER_BUSY if held + mark
+  int acquired_slot(int layer) const;                  // -1 unless layer is acquired
+  void release(int slot);                              // the caller's reads are ordered before reuse
+
+ private:
+  struct Slot {
+    int layer = -1;
+    bool acquired = false;
+    bool pending = false;   // filled and not yet acquired
+    bool released = false; // released at least once
+    uint64_t release_tick = 0;
+  };
+  int victim() const;
+  std::vector<Slot> s_;
+  uint64_t tick_ = 0;
+  int n_layers_ = 0, rank_ = 0, world_ = 1;
+  bool shared_ = false;
+};
+
+// The pool calls of one pass over the layers, in the order the model step makes them:
+// for each layer of the pass (dir +1: 0..n-1, dir -1: n-1..0) acquire it, prefetch the
+// next `lookahead` layers of the pass (stopping at the first BUFFER_BUSY, which is not
+// an error), run it, release it.  f(op, layer) returns a status.
+enum PassOp : int { PASS_ACQUIRE = 0, PASS_PREFETCH = 1, PASS_RUN = 2, PASS_RELEASE = 3 };
+template <typename F>
+int for_each_pass_op(int n_layers, int dir, int lookahead, F&& f) {
+  for (int t = 0; t < n_layers; ++t) {
+    const int i = dir > 0 ? t : n_layers - 1 - t;
+    NF4_TRY(f(PASS_ACQUIRE, i));
+    for (int k = 1; k <= lookahead; ++k) {
+      const int j = i + dir * k;
+      if (j < 0 || j >= n_layers) break;
+      const int st = f(PASS_PREFETCH, j);
+      if (st == NF4LS_BUFFER_BUSY) break;
+      NF4_TRY(st);
+    }
+    NF4_TRY(f(PASS_RUN, i));
+    NF4_TRY(f(PASS_RELEASE, i));
+  }
+  return NF4LS_OK;
+}
+// Layers the model step prefetches ahead of the one it runs.
+constexpr int kStepLookahead = 1;
 
 // ----------------------------------------------------------------------------- code tables
 struct Codebooks {
@@ -127,6 +210,11 @@ int gemm_half_mode();
 int attention_tc();
 int check_cfg(const nf4ls_layer_cfg* c);
 int* device_error_ptr();
+// Process-unique id of the CUDA context current on this thread, 0 when none is
+// current or the driver cannot say.  A symbol address looked up in one context is
+// valid only there: a device reset (a new primary context) or another context needs
+// a fresh lookup.
+unsigned long long current_context_id();
 
 // ----------------------------------------------------------------------------- accounting
 // Every kernel launch of the library bumps a process-wide counter.

@@ -94,30 +94,29 @@ struct Phase {
   }
 };
 
-int acquire(const nf4ls_model* m, int layer, int dir, cudaStream_t s, const void** shard) {
-  if (!m->pool) {
-    *shard = m->shards_dev[layer];
-    return NF4LS_OK;
-  }
-  NF4_TRY(stream_prefetch(m->pool, layer, s, shard));
-  return NF4LS_OK;
-}
-
-int lookahead(const nf4ls_model* m, const nf4ls_model_cfg* c, int layer, int dir, int depth) {
-  if (!m->pool) return NF4LS_OK;
-  for (int k = 1; k < depth; ++k) {
-    const int j = layer + dir * k;
-    if (j < 0 || j >= c->n_layers) break;
-    const int st = nf4ls_pool_prefetch(m->pool, j);
-    if (st == NF4LS_BUFFER_BUSY) break;  // no free slot yet: the next acquire copies it
-    NF4_TRY(st);
-  }
-  return NF4LS_OK;
-}
-
-int release(const nf4ls_model* m, int layer, cudaStream_t s) {
-  if (!m->pool) return NF4LS_OK;
-  return nf4ls_pool_release(m->pool, layer, s);
+// One pass over the layers (dir +1 forward, -1 backward) in the pool-call order of
+// for_each_pass_op: acquire layer i, prefetch the next layer of the pass (a busy pool
+// is not an error: the next acquire copies it), run(i, shard), release i.  With
+// resident shards the pool calls drop out.
+template <typename Run>
+int layer_pass(const nf4ls_model_cfg* c, const nf4ls_model* m, int dir, cudaStream_t s, Run&& run) {
+  const void* shard = nullptr;
+  return for_each_pass_op(c->n_layers, dir, kStepLookahead, [&](int op, int layer) -> int {
+    switch (op) {
+      case PASS_ACQUIRE:
+        if (!m->pool) {
+          shard = m->shards_dev[layer];
+          return NF4LS_OK;
+        }
+        return stream_prefetch(m->pool, layer, s, &shard);
+      case PASS_PREFETCH:
+        return m->pool ? nf4ls_pool_prefetch(m->pool, layer) : NF4LS_OK;
+      case PASS_RUN:
+        return run(layer, shard);
+      default:
+        return m->pool ? nf4ls_pool_release(m->pool, layer, s) : NF4LS_OK;
+    }
+  });
 }
 
 int check_model(const nf4ls_model_cfg* c, const nf4ls_model* m) {
@@ -138,11 +137,6 @@ int check_model(const nf4ls_model_cfg* c, const nf4ls_model* m) {
   if (!aligned(m->ws_dev, 256)) return fail(NF4LS_ALIGN, "model: workspace must be 256-byte aligned");
   if (m->ws_bytes < model_ws(c).total) return fail(NF4LS_INVALID_ARG, "model: workspace too small");
   return NF4LS_OK;
-}
-
-int pool_depth(const nf4ls_model* m) {
-  if (!m->pool) return 1;
-  return 2;  // prefetch one layer ahead, as the pages do
 }
 
 // The streamed head: logits, loss and (need_grad) dL/dhf in one pass over the vocab
@@ -212,19 +206,14 @@ int forward_to_loss(const nf4ls_model_cfg* c, const nf4ls_model* m, const int32_
     E = d;
   }
   NF4_TRY(embed(ids, static_cast<const __nv_bfloat16*>(E), xs, M, H, s));
-  const int depth = pool_depth(m);
   {
-  Phase fwd_phase(s, 2000);
-  for (int i = 0; i < c->n_layers; ++i) {
-    const void* shard;
-    NF4_TRY(acquire(m, i, +1, s, &shard));
-    NF4_TRY(lookahead(m, c, i, +1, depth));
-    nf4ls_lora l;
-    lora_views(lc, m->lora_dev + (size_t)i * stride, &l, nullptr, nullptr);
-    NF4_TRY(layer_fwd_impl(lc, shard, lora_on ? &l : nullptr, xs + (size_t)i * act, xs + (size_t)(i + 1) * act,
-                           at<void>(ws, L.layer), L.total - L.layer, s));
-    NF4_TRY(release(m, i, s));
-  }
+    Phase fwd_phase(s, 2000);
+    NF4_TRY(layer_pass(c, m, +1, s, [&](int i, const void* shard) {
+      nf4ls_lora l;
+      lora_views(lc, m->lora_dev + (size_t)i * stride, &l, nullptr, nullptr);
+      return layer_fwd_impl(lc, shard, lora_on ? &l : nullptr, xs + (size_t)i * act, xs + (size_t)(i + 1) * act,
+                            at<void>(ws, L.layer), L.total - L.layer, s);
+    }));
   }
   Phase head(s, 2001);
   auto* hf = at<__nv_bfloat16>(ws, L.hf);
@@ -294,19 +283,14 @@ extern "C" int nf4ls_forward_backward(const nf4ls_model_cfg* cfg, const nf4ls_mo
                         nullptr, dh, M, H, lc->rms_eps, s));
   }
   const size_t stride = stride_of(lc);
-  const int depth = pool_depth(m);
   Phase bwd_phase(s, 2003);
-  for (int i = cfg->n_layers - 1; i >= 0; --i) {
-    const void* shard;
-    NF4_TRY(acquire(m, i, -1, s, &shard));
-    NF4_TRY(lookahead(m, cfg, i, -1, depth));
+  return layer_pass(cfg, m, -1, s, [&](int i, const void* shard) {
     nf4ls_lora l;
     nf4ls_lora_grads g;
     lora_views(lc, m->lora_dev + (size_t)i * stride, &l, &g, m->grads_dev + (size_t)i * stride);
-    NF4_TRY(layer_bwd_impl(lc, shard, &l, xs + (size_t)i * act, dh, dh, &g, at<void>(ws, L.layer), L.total - L.layer, s));
-    NF4_TRY(release(m, i, s));
-  }
-  return NF4LS_OK;
+    return layer_bwd_impl(lc, shard, &l, xs + (size_t)i * act, dh, dh, &g, at<void>(ws, L.layer), L.total - L.layer,
+                          s);
+  });
 }
 
 extern "C" int nf4ls_adamw_step(const nf4ls_model_cfg* cfg, const nf4ls_model* m, int32_t step, nf4ls_stream stream) {

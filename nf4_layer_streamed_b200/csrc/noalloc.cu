@@ -11,10 +11,13 @@
 // passes its input and output buffers.
 //
 // The array holds the absmax values of tensors up to kMaxElems weights (16 MiB of
-// device memory, plus the offset pass's 8 KB), and every GPU that loads the library holds its own copy until the
-// process exits.  Host code cannot use the array's name as a device address; the
-// address is looked up once per device with cudaGetSymbolAddress, on the first call
-// made with that device current.  Make that first call before any stream capture.
+// device memory, plus the offset pass's 8 KB), and every GPU that loads the library
+// holds its own copy until the process exits.  Host code cannot use the array's name
+// as a device address; the address is looked up with cudaGetSymbolAddress on the
+// first call made with that device current, and again on the first call in a new
+// CUDA context (after a device reset, or under a context the caller created), since
+// an address from one context is not valid in another.  Make that first call before
+// any stream capture.
 // Every call shares the one array: calls whose kernels overlap on the GPU (on
 // different streams) race on it.  Nothing in it needs to start at zero: each call
 // writes every absmax value it later reads.
@@ -32,18 +35,21 @@ static __device__ __align__(256) float g_quant_scratch[kScratchFloats];
 
 std::mutex g_mu;
 float* g_ptr[64] = {nullptr};
+unsigned long long g_ctx[64] = {0};  // the context each cached address belongs to
 
 int scratch_address(float** out) {
   int dev = 0;
   NF4_CUDA_TRY(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64) return fail(NF4LS_INVALID_ARG, "nf4_quantize_tensor_noalloc: device %d out of range", dev);
+  const unsigned long long id = current_context_id();
   std::lock_guard<std::mutex> g(g_mu);
-  if (!g_ptr[dev]) {
+  if (!g_ptr[dev] || id == 0 || id != g_ctx[dev]) {
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_quant_scratch);
     if (e != cudaSuccess)
       return fail(NF4LS_CUDA, "nf4_quantize_tensor_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
     g_ptr[dev] = static_cast<float*>(p);
+    g_ctx[dev] = current_context_id();
   }
   *out = g_ptr[dev];
   return NF4LS_OK;

@@ -126,17 +126,14 @@ struct nf4ls_pool {
   uint8_t* slots = nullptr;
   size_t slot_bytes = 0;
   cudaStream_t copy = nullptr;
+  // Which layer each slot holds, hits, reuse order and ownership: the host-only plan.
+  // What the device sees of a slot: its events.
+  SlotPlan plan;
   struct Slot {
-    int layer = -1;
-    bool acquired = false;
-    bool pending = false;  // filled by a prefetch and not yet acquired
-    bool freed_recorded = false;
     bool filling = false;  // disk source: the reader has not enqueued this slot's copy yet
-    uint64_t release_tick = 0;
     cudaEvent_t ready = nullptr, freed = nullptr;
   };
   std::vector<Slot> slot;
-  uint64_t tick = 0;
   bool poison = false;
   nf4ls_pool_stats stats{};
   std::mutex mu;
@@ -145,63 +142,39 @@ struct nf4ls_pool {
   ncclComm_t comm = nullptr;
   int rank = 0, world = 1;
 
-  int find(int layer) const {
-    for (int i = 0; i < depth; ++i)
-      if (slot[i].layer == layer) return i;
-    return -1;
-  }
-
-  int victim() const {
-    int best = -1;
-    for (int i = 0; i < depth; ++i) {
-      const Slot& s = slot[i];
-      if (s.acquired || s.pending) continue;
-      if (s.layer < 0) return i;
-      if (best < 0 || s.release_tick < slot[best].release_tick) best = i;
-    }
-    return best;
-  }
+  int find(int layer) const { return plan.find(layer); }
 
   int issue(int layer, int* out_idx) {
-    int i = find(layer);
-    if (i >= 0) {
-      *out_idx = i;
-      return NF4LS_OK;
-    }
-    i = victim();
-    if (i < 0) return fail(NF4LS_BUFFER_BUSY, "pool: every slot is acquired or pending (depth %d)", depth);
-    Slot& s = slot[i];
-    uint8_t* dst = slots + (size_t)i * slot_bytes;
+    PlanStep st;
+    NF4_TRY(plan.preview(layer, &st));
+    *out_idx = st.slot;
+    if (!st.fill) return NF4LS_OK;
+    if (file && file->error) return fail(file->error, "pool: disk source failed earlier: %s", file->error_msg.c_str());
+    NF4_TRY(plan.issue(layer, &st));
+    Slot& s = slot[st.slot];
+    uint8_t* dst = slots + (size_t)st.slot * slot_bytes;
     if (file) {  // the reader thread reads the layer and enqueues the copy
-      if (file->error) return fail(file->error, "pool: disk source failed earlier: %s", file->error_msg.c_str());
-      file->jobs.push_back(FileSource::Job{layer, i, s.freed_recorded});
+      file->jobs.push_back(FileSource::Job{layer, st.slot, st.after_release});
       file->cv_job.notify_one();
-      s.layer = layer;
-      s.pending = true;
       s.filling = true;
       stats.bytes_copied += bytes[layer];
       stats.copies += 1;
-      *out_idx = i;
       return NF4LS_OK;
     }
-    if (s.freed_recorded) NF4_CUDA_TRY(cudaStreamWaitEvent(copy, s.freed, 0));
+    if (st.after_release) NF4_CUDA_TRY(cudaStreamWaitEvent(copy, s.freed, 0));
     if (poison) NF4_CUDA_TRY(cudaMemsetAsync(dst, 0xFF, slot_bytes, copy));
-    const int owner = layer % world;
-    if (owner == rank) {
+    if (st.host_read) {
       NF4_CUDA_TRY(cudaMemcpyAsync(dst, store + off[layer], bytes[layer], cudaMemcpyHostToDevice, copy));
       stats.bytes_copied += bytes[layer];
       stats.copies += 1;
     }
-    if (comm) {  // from the owner's slot into every other rank's slot, in place
-      const ncclResult_t r = nccl_api().broadcast(dst, dst, bytes[layer], ncclUint8, owner, comm, copy);
+    if (st.broadcast) {  // from the owner's slot into every other rank's slot, in place
+      const ncclResult_t r = nccl_api().broadcast(dst, dst, bytes[layer], ncclUint8, st.owner, comm, copy);
       if (r != ncclSuccess) return fail(NF4LS_CUDA, "pool: NCCL broadcast of layer %d: %s", layer,
                                         nccl_api().error_string(r));
-      if (owner != rank) stats.peer_bytes += bytes[layer];
+      if (!st.host_read) stats.peer_bytes += bytes[layer];
     }
     NF4_CUDA_TRY(cudaEventRecord(s.ready, copy));
-    s.layer = layer;
-    s.pending = true;
-    *out_idx = i;
     return NF4LS_OK;
   }
 
@@ -211,7 +184,7 @@ struct nf4ls_pool {
     const bool ok = file->cv_done.wait_for(lk, std::chrono::milliseconds(kFillWaitMs),
                                            [&] { return !slot[idx].filling || file->error != NF4LS_OK; });
     if (file->error) return fail(file->error, "pool: disk source: %s", file->error_msg.c_str());
-    if (!ok) return fail(NF4LS_TIMEOUT, "pool: layer %d not read from disk after %d ms", slot[idx].layer, kFillWaitMs);
+    if (!ok) return fail(NF4LS_TIMEOUT, "pool: layer %d not read from disk after %d ms", plan.layer_in(idx), kFillWaitMs);
     return NF4LS_OK;
   }
 
@@ -308,6 +281,7 @@ int make_pool(const size_t* layer_off, const size_t* layer_bytes, int n_layers, 
   p->slots = static_cast<uint8_t*>(slots_dev);
   p->slot_bytes = slot_bytes;
   p->slot.resize(depth);
+  p->plan.init(n_layers, depth);
   cudaError_t e = cudaGetDevice(&p->device);
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&p->copy, cudaStreamNonBlocking);
   for (int i = 0; i < depth && e == cudaSuccess; ++i) {
@@ -425,8 +399,7 @@ extern "C" int nf4ls_pool_share(nf4ls_pool* p, int rank, int world, const uint8_
   std::lock_guard<std::mutex> g(p->mu);
   if (p->file) return fail(NF4LS_INVALID_ARG, "nf4ls_pool_share: a pool with a file store cannot be shared");
   if (p->comm) return fail(NF4LS_INVALID_ARG, "nf4ls_pool_share: already shared");
-  for (const auto& s : p->slot)
-    if (s.layer >= 0) return fail(NF4LS_INVALID_ARG, "nf4ls_pool_share: the pool must not hold a layer yet");
+  if (p->plan.holds_any()) return fail(NF4LS_INVALID_ARG, "nf4ls_pool_share: the pool must not hold a layer yet");
   const NcclApi& n = nccl_api();
   if (!n.ok) return fail(NF4LS_CUDA, "nf4ls_pool_share: libnccl.so.2 not found");
   NF4_CUDA_TRY(cudaSetDevice(p->device));
@@ -438,6 +411,7 @@ extern "C" int nf4ls_pool_share(nf4ls_pool* p, int rank, int world, const uint8_
   p->comm = comm;
   p->rank = rank;
   p->world = world;
+  p->plan.share(rank, world);
   return NF4LS_OK;
 }
 
@@ -537,11 +511,10 @@ extern "C" int stream_prefetch(nf4ls_pool* p, int layer, nf4ls_stream compute, c
   int idx;
   NF4_TRY(p->issue(layer, &idx));
   nf4ls_pool::Slot& s = p->slot[idx];
-  if (s.acquired) return fail(NF4LS_BUFFER_BUSY, "stream_prefetch: layer %d is already acquired", layer);
+  if (p->plan.acquired(idx)) return fail(NF4LS_BUFFER_BUSY, "stream_prefetch: layer %d is already acquired", layer);
   NF4_TRY(p->wait_filled(lk, idx));
   NF4_CUDA_TRY(cudaStreamWaitEvent(static_cast<cudaStream_t>(compute), s.ready, 0));
-  s.acquired = true;
-  s.pending = false;
+  p->plan.mark_acquired(idx);
   p->stats.acquisitions += 1;
   if (hit) p->stats.hits += 1;
   *slot_dev = p->slots + (size_t)idx * p->slot_bytes;
@@ -552,13 +525,10 @@ extern "C" int nf4ls_pool_release(nf4ls_pool* p, int layer, nf4ls_stream compute
   clear_error();
   if (!p || layer < 0 || layer >= p->n_layers) return fail(NF4LS_INVALID_ARG, "nf4ls_pool_release: bad argument");
   std::lock_guard<std::mutex> g(p->mu);
-  const int idx = p->find(layer);
-  if (idx < 0 || !p->slot[idx].acquired) return fail(NF4LS_INVALID_ARG, "nf4ls_pool_release: layer %d not acquired", layer);
-  nf4ls_pool::Slot& s = p->slot[idx];
-  NF4_CUDA_TRY(cudaEventRecord(s.freed, static_cast<cudaStream_t>(compute)));
-  s.freed_recorded = true;
-  s.acquired = false;
-  s.release_tick = ++p->tick;
+  const int idx = p->plan.acquired_slot(layer);
+  if (idx < 0) return fail(NF4LS_INVALID_ARG, "nf4ls_pool_release: layer %d not acquired", layer);
+  NF4_CUDA_TRY(cudaEventRecord(p->slot[idx].freed, static_cast<cudaStream_t>(compute)));
+  p->plan.release(idx);
   return NF4LS_OK;
 }
 

@@ -14,8 +14,11 @@ GPU's host-to-device link, so the ranks can split the layer stream -- the owner 
 layer l (rank l % world) copies it from its host store and the library's pool
 broadcasts it from the owner's slot into the other ranks' slots with NCCL over
 NVLink.  Each rank then moves 1/world of the bytes over PCIe; the slot contents,
-hence the results, do not change.  ``emulate_sharded_fetch`` runs the same schedule
-on host byte arrays with any torch.distributed backend (the CPU tests use gloo).
+hence the results, do not change.  ``run_fetch_plan`` drives the library's own slot
+plan (the object the pool takes every slot decision through) with the pool calls
+of the model step and carries out each fill it decides on host byte arrays, with
+any torch.distributed backend (the CPU tests use gloo); ``emulate_sharded_fetch``
+is a plain restatement of the same schedule, kept as a second opinion.
 """
 from __future__ import annotations
 
@@ -86,3 +89,57 @@ def emulate_sharded_fetch(store: torch.Tensor, offsets, sizes, order, group=None
         dist.broadcast(buf, src=src, group=group)
         got[layer] = buf
     return got, own_reads
+
+
+def run_fetch_plan(stores, offsets, sizes, n_layers: int, depth: int, steps: int, slot_bytes: int,
+                   group=None, on_run=None, move_bytes: bool = True) -> dict:
+    """The sharded fetch of `steps` training steps on host arrays, every decision
+    taken by the library's slot plan (api.SlotPlan shared as this rank of the group),
+    in the pool-call order of the model step (api.step_pass_ops, forward then
+    backward).  A fill the plan decides is carried out as the pool does it: the owner
+    copies the layer from its store (``stores(layer)`` -> uint8 tensor) into the slot,
+    then the slot's bytes are broadcast from the owner.  ``on_run(layer, bytes)`` sees
+    the slot's bytes when the step runs a layer.  With move_bytes False only the
+    decisions are made (no collective).  Returns the fill log [(layer, slot, owner,
+    after_release)], the layers this rank read from its own store, and hit / run
+    counts."""
+    from . import api
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    slots = torch.zeros(depth, slot_bytes, dtype=torch.uint8)
+    fills, reads, hits, runs = [], [], 0, 0
+    ops = api.step_pass_ops(n_layers, +1) + api.step_pass_ops(n_layers, -1)
+    with api.SlotPlan(n_layers, depth) as plan:
+        plan.share(rank, world)
+
+        def carry(layer, st):
+            if not st["fill"]:
+                return
+            fills.append((layer, st["slot"], st["owner"], st["after_release"]))
+            if not move_bytes:
+                return
+            buf = slots[st["slot"], :sizes[layer]]
+            if st["host_read"]:
+                buf.copy_(stores(layer)[offsets[layer]:offsets[layer] + sizes[layer]])
+                reads.append(layer)
+            if st["broadcast"]:
+                dist.broadcast(buf, src=st["owner"], group=group)
+
+        for _ in range(steps):
+            for op, layer in ops:
+                if op == "acquire":
+                    st = plan.acquire(layer)
+                    hits += st["hit"]
+                    carry(layer, st)
+                    held = st["slot"]
+                elif op == "prefetch":
+                    st = plan.prefetch(layer)
+                    if st is not None:
+                        carry(layer, st)
+                elif op == "run":
+                    runs += 1
+                    if on_run is not None:
+                        on_run(layer, slots[held, :sizes[layer]])
+                else:
+                    plan.release(layer)
+    return {"fills": fills, "reads": reads, "hits": hits, "runs": runs}

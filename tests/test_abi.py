@@ -162,22 +162,26 @@ def test_adapter_load_refuses_bad_files_before_touching_the_device(tmp_path):
     assert B.lib().nf4ls_adapter_file_bytes(None) == 0
     m = B.Model(256, None, 256, 256, 256, 256, 256, 256, None, 256, 0, None, None)
     body = np.arange(3 * n, dtype=np.float32).tobytes()
-    csum = _fnv1a64(body)
 
     def header(**kw):
-        f = dict(magic=0x41344E46, version=1, hidden=lc.hidden, inter=lc.inter, n_q=lc.n_q, n_kv=lc.n_kv,
+        # the checksum covers the header (checksum field zero) and then the body
+        f = dict(magic=0x41344E46, version=2, hidden=lc.hidden, inter=lc.inter, n_q=lc.n_q, n_kv=lc.n_kv,
                  head_dim=lc.head_dim, r=lc.lora_r, layers=n_layers, alpha=lc.lora_alpha, step=7, n=n,
-                 csum=csum)
+                 csum=None)
         f.update(kw)
-        return struct.pack("<IIiiiiiiifiIQQ", f["magic"], f["version"], f["hidden"], f["inter"], f["n_q"],
-                           f["n_kv"], f["head_dim"], f["r"], f["layers"], f["alpha"], f["step"], 0, f["n"],
-                           f["csum"])
+
+        def pack(c):
+            return struct.pack("<IIiiiiiiifiIQQ", f["magic"], f["version"], f["hidden"], f["inter"], f["n_q"],
+                               f["n_kv"], f["head_dim"], f["r"], f["layers"], f["alpha"], f["step"], 0, f["n"], c)
+        return pack(_fnv1a64(pack(0) + body) if f["csum"] is None else f["csum"])
+
+    csum = _fnv1a64(header(csum=0) + body)
 
     assert len(header()) == 64
     step = ctypes.c_int32(-1)
     cases = [
         ("magic", header(magic=0x12345678) + body, -1),
-        ("version", header(version=2) + body, -1),
+        ("version", header(version=3) + body, -1),
         ("hidden", header(hidden=lc.hidden * 2) + body, -2),
         ("rank", header(r=lc.lora_r * 2) + body, -2),
         ("alpha", header(alpha=lc.lora_alpha + 1) + body, -2),
@@ -188,7 +192,11 @@ def test_adapter_load_refuses_bad_files_before_touching_the_device(tmp_path):
         ("trailing", header() + body + b"\0", -11),
         ("corrupt", header() + body[:-1] + bytes([body[-1] ^ 1]), -11),
         ("checksum", header(csum=csum ^ 1) + body, -11),
+        # a damaged step (still >= 0) or alpha with the checksum of the intact header
+        ("step", header(step=8, csum=csum) + body, -11),
+        ("version1", header(version=1) + body, -1),
     ]
+    assert header(csum=None) == header(csum=csum)
     for name, blob, want in cases:
         p = tmp_path / f"{name}.adapter"
         p.write_bytes(blob)
@@ -210,3 +218,11 @@ def test_adapter_load_refuses_bad_files_before_touching_the_device(tmp_path):
     assert B.call_status("nf4ls_adapter_load", g, ctypes.byref(cfg), ctypes.byref(no_moments), ctypes.byref(step),
                          None) == -1
     assert B.call_status("nf4ls_adapter_save", g, ctypes.byref(cfg), ctypes.byref(m), -1, None) == -1
+
+
+def test_wait_probe_refuses_bad_arguments_on_the_host():
+    # the limits are checked before any device work, so these run without a GPU
+    for limit in (0, -5, 1_000_001):
+        assert B.call_status("nf4ls_wait_probe", limit, ctypes.c_void_p(256), None) == -1, limit
+    assert B.call_status("nf4ls_wait_probe", 1000, None, None) == -1
+    assert "limit_us" in B.last_error()

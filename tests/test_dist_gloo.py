@@ -143,3 +143,82 @@ def test_layer_sharded_fetch_ranks_gloo(world):
         assert nccl_id == res[0][2][2]
     # the fetch is split: together the ranks read each of the 12 fills exactly once
     assert sum(len(res[r][1]) for r in range(world)) == 7 + 5
+
+
+def _plan_worker(rank, world, depth, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        n_layers, size, steps = 7, 4096, 2
+        g = torch.Generator().manual_seed(11)
+        truth = torch.randint(0, 256, (n_layers * size,), generator=g, dtype=torch.uint8)
+        offs = [i * size for i in range(n_layers)]
+        sizes = [size - 17 * i for i in range(n_layers)]
+        # this rank's store holds the true bytes only for the layers it owns: a layer
+        # read from the wrong rank's store shows up as 0xA0 + rank junk
+        mine = torch.full_like(truth, 0xA0 + rank)
+        for l in range(n_layers):
+            if l % world == rank:
+                mine[offs[l]:offs[l] + sizes[l]] = truth[offs[l]:offs[l] + sizes[l]]
+        # 1. decisions only: every rank's plan must decide the same fills in the same order
+        dry = dp.run_fetch_plan(lambda l: mine, offs, sizes, n_layers, depth, steps, size, move_bytes=False)
+        logs = [None] * world
+        dist.all_gather_object(logs, dry["fills"])
+        same = all(l == logs[0] for l in logs)
+        if not same:
+            q.put((rank, False, None, None, None))
+            return
+        # 2. the fills carried out: owner reads, broadcast to the others, and every
+        # layer the step runs finds its true bytes in its slot
+        bad = []
+
+        def on_run(layer, got):
+            if not torch.equal(got, truth[offs[layer]:offs[layer] + sizes[layer]]):
+                bad.append(layer)
+
+        res = dp.run_fetch_plan(lambda l: mine, offs, sizes, n_layers, depth, steps, size, on_run=on_run)
+        q.put((rank, same and res["fills"] == dry["fills"], res, bad, logs[0]))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,depth", [(2, 2), (3, 2), (2, 3), (3, 3)])
+def test_library_fetch_plan_on_gloo_ranks(world, depth):
+    """The library's own slot plan (the pool's decisions: slot reuse least recently
+    released first, hits across the forward-backward turn, fills after the slot's
+    release, owners) driven by each rank with the model step's pool-call order for
+    two steps: all ranks decide the same fills in the same order, so the broadcasts
+    pair up; each fill is read from the host store by its owner alone and every layer
+    the step runs finds its true bytes, although each rank's store holds only its own
+    layers.  At depth 2 a step refills every layer but the two the previous pass left
+    (2 L - 2 the first step, 2 L - 4 after)."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_plan_worker, args=(r, world, depth, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = {}
+    for _ in range(world):
+        r, same, out, bad, log = q.get(timeout=120)
+        res[r] = (same, out, bad, log)
+    for p in procs:
+        p.join(30)
+        assert p.exitcode == 0
+    n_layers = 7
+    log = res[0][3]
+    for r in range(world):
+        same, out, bad, _ = res[r]
+        assert same, r
+        assert bad == [], (r, bad)
+        assert out["runs"] == 2 * 2 * n_layers
+        assert all(l % world == r for l in out["reads"]) and out["reads"], r
+    # together the ranks read each fill exactly once
+    assert sorted(sum((res[r][1]["reads"] for r in range(world)), [])) == sorted(l for l, _, _, _ in log)
+    # past the first fill of each slot, every fill reuses a slot and waits for its previous reader
+    assert all(after for _, _, _, after in log[depth:])
+    if depth == 2:
+        assert len(log) == (2 * n_layers - 2) + (2 * n_layers - 4)
+    else:
+        assert len(log) < (2 * n_layers - 2) + (2 * n_layers - 4)

@@ -100,6 +100,14 @@ def test_llama8b_layer_matches_oracle():
     _check_against_oracle(shape, 1, 512, r)
 
 
+def test_llama8b_layer_b2s384_matches_oracle():
+    """The tcgen05 attention forward, dQ and dK/dV at three 128-key tiles per sequence
+    and two sequences, inside a full 8B layer forward and backward, against the oracle."""
+    shape = synth.LLAMA_8B
+    r = _run(shape, 2, 384, True, seed=4321)
+    _check_against_oracle(shape, 2, 384, r)
+
+
 def test_llama8b_batch4_rows_equal_batch1_rows():
     shape = synth.LLAMA_8B
     cfg4 = api.layer_cfg(shape, 4, 512)
