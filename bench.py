@@ -271,6 +271,52 @@ def time_steps(m, ids, warmup: int, steps: int) -> float:
     return a.elapsed_time(b) / steps
 
 
+def smollm2_layer_times(iters: int = 20) -> dict:
+    """One SmolLM2-135M-shaped layer at 1 x 512 tokens with random LoRA B: layer_forward
+    and layer_backward (recompute + dL/dx + LoRA gradients), CUDA events, after warm-up;
+    and the same with per-launch GEMM events (their time and FLOPs by kind)."""
+    import torch
+
+    from nf4_layer_streamed_b200 import api, synth
+    shape = synth.SMOLLM2_135M
+    cfg = api.layer_cfg(shape, 1, 512)
+    w = synth.layer_weights(shape, 0, 1234, device="cuda")
+    shard = api.nf4_quantize_shard(cfg, w, fingerprint=1)
+    lo = synth.lora_params(shape, 0, 1234, b_random=True, device="cuda")
+    x = synth.hidden_states(shape, 1, 512, 1234, device="cuda").view(512, shape.hidden)
+    dy = synth.tensor_values((512, shape.hidden), seed=5, scale=1e-3, device="cuda")
+    ws = api.LayerWorkspace(cfg)
+    res = {}
+    for name, f in (("forward", lambda: api.layer_forward(cfg, shard, lo, x, ws)),
+                    ("backward", lambda: api.layer_backward(cfg, shard, lo, x, dy, ws))):
+        for _ in range(3):
+            f()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n0 = api.launch_count()
+        a.record()
+        for _ in range(iters):
+            f()
+        b.record()
+        torch.cuda.synchronize()
+        res[name] = {"us": a.elapsed_time(b) / iters * 1000.0, "launches": (api.launch_count() - n0) / iters}
+    api.profile(True)
+    api.profile_reset()
+    api.layer_forward(cfg, shard, lo, x, ws)
+    api.layer_backward(cfg, shard, lo, x, dy, ws)
+    torch.cuda.synchronize()
+    api.profile(False)
+    gemms = {}
+    for code, name in api.GEMM_DETAILS.items():
+        r = api.profile_read(code)
+        if r["launches"]:
+            gemms[name] = {"launches": r["launches"], "us": r["ms"] * 1000.0}
+    api.profile_reset()
+    res["gemm_launches"] = gemms
+    res["note"] = "per-kernel times of every launch: profiles/launches_smollm2_layer_b1s512.md"
+    return res
+
+
 def extra_points(args, wl, ms_step: float, copy_ms: float) -> dict:
     """Single-GPU context for the headline: the same steps with every shard resident in
     HBM (compute only), the copy/compute overlap, and the batch-16 point where the step
@@ -326,6 +372,19 @@ def extra_points(args, wl, ms_step: float, copy_ms: float) -> dict:
         if os.path.exists(path):
             os.unlink(path)
         os.rmdir(d)
+    # the small configurations: one SmolLM2-shaped layer (1 x 512) forward and backward,
+    # and the 30-layer SmolLM2-shaped tied stack streamed at depth 2 and 3 and resident
+    out["smollm2_layer_b1s512"] = smollm2_layer_times()
+    wl2 = synth.WORKLOADS["smollm2_30L_tied_b1s512"]
+    ids2 = [dp.rank_token_ids(wl2, 0, s) for s in range(4)]
+    pts = {}
+    for name, kw in (("depth2", {"depth": 2}), ("depth3", {"depth": 3}), ("resident", {"resident": True})):
+        m = api.StreamedModel(wl2, **kw)
+        t2 = time_steps(m, ids2, 3, 10)
+        m.close()
+        del m
+        pts[name] = {"ms_per_step": t2, "tokens_per_s": wl2.tokens / (t2 / 1000.0)}
+    out["smollm2_30L_tied_b1s512"] = pts
     wl16 = synth.WORKLOADS["llama8b_32L_b16s512"]
     ids16 = [dp.rank_token_ids(wl16, 0, s) for s in range(3)]
     m = api.StreamedModel(wl16, depth=args.depth)

@@ -561,6 +561,16 @@ int nf4ls_attention_fwd(const nf4ls_layer_cfg* cfg, const void* q_dev, const voi
                         const void* v_dev, int ld_q, int ld_kv, void* o_dev, float* lse_dev,
                         nf4ls_stream stream);
 
+/* Its backward: from q, k, v (as above), o and do [M, n_q*d] (row stride n_q*d), lse
+ * [batch, n_q, seq] of the forward -> dq [M, n_q*d], dk, dv [M, n_kv*d] (bf16, row
+ * strides n_q*d and n_kv*d) and delta = rowsum(do * o) fp32 [batch, n_q, seq] (a
+ * by-product, written).  dq, dk, dv are the gradients with respect to the forward's
+ * q, k, v (before any RoPE transpose). */
+int nf4ls_attention_bwd(const nf4ls_layer_cfg* cfg, const void* q_dev, const void* k_dev,
+                        const void* v_dev, int ld_q, int ld_kv, const void* o_dev, const void* do_dev,
+                        const float* lse_dev, float* delta_dev, void* dq_dev, void* dk_dev, void* dv_dev,
+                        nf4ls_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -330,6 +330,26 @@ def attention_fwd(cfg: B.LayerCfg, q, k, v, ld_q: int, ld_kv: int, stream=None):
     return o, lse
 
 
+def attention_bwd(cfg: B.LayerCfg, q, k, v, ld_q: int, ld_kv: int, o, do, lse, stream=None):
+    """Gradients (dq, dk, dv) of the causal GQA attention and delta = rowsum(do * o)."""
+    M = cfg.batch * cfg.seq
+    qd, kvd = cfg.n_q * cfg.head_dim, cfg.n_kv * cfg.head_dim
+    _need_rows(q, "q", M, ld_q, qd)
+    _need_rows(k, "k", M, ld_kv, kvd)
+    _need_rows(v, "v", M, ld_kv, kvd)
+    _need(o, "o", torch.bfloat16, M * qd)
+    _need(do, "do", torch.bfloat16, M * qd)
+    _need(lse, "lse", torch.float32, cfg.batch * cfg.n_q * cfg.seq)
+    _need_cuda(q=q, k=k, v=v, o=o, do=do, lse=lse)
+    dq = torch.empty(M, qd, dtype=torch.bfloat16, device=q.device)
+    dk = torch.empty(M, kvd, dtype=torch.bfloat16, device=q.device)
+    dv = torch.empty(M, kvd, dtype=torch.bfloat16, device=q.device)
+    delta = torch.empty(cfg.batch, cfg.n_q, cfg.seq, dtype=torch.float32, device=q.device)
+    B.call("nf4ls_attention_bwd", ctypes.byref(cfg), _p(q), _p(k), _p(v), ld_q, ld_kv, _p(o), _p(do), _p(lse),
+           _p(delta), _p(dq), _p(dk), _p(dv), _s(stream))
+    return dq, dk, dv, delta
+
+
 # ----------------------------------------------------------------------------- streaming pool
 
 class Pool:

@@ -148,6 +148,8 @@ SIGNATURES = {
     "nf4ls_gemm_nf4": (ctypes.c_int, [P, ctypes.c_int, ctypes.c_int, P, P, P, P, ctypes.c_int, ctypes.c_int,
                                       ctypes.c_int, P, ctypes.c_int, P]),
     "nf4ls_attention_fwd": (ctypes.c_int, [ctypes.POINTER(LayerCfg), P, P, P, ctypes.c_int, ctypes.c_int, P, P, P]),
+    "nf4ls_attention_bwd": (ctypes.c_int, [ctypes.POINTER(LayerCfg), P, P, P, ctypes.c_int, ctypes.c_int, P, P, P, P,
+                                           P, P, P, P]),
 }
 
 _LIB = None

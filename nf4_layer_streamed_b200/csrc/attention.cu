@@ -519,12 +519,12 @@ int attention_bwd(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfl
   NF4_TRY(check_attn(seq, nq, nkv, d, ldq, ldkv));
   const int M = batch * seq;
   const float scale = 1.0f / sqrtf((float)d);
+  if (attention_tc() && attention_fwd_tc_supported(seq, d, nq, nkv, ldq, ldkv, ldo) && ld_dq % 8 == 0 &&
+      ld_dkv % 8 == 0)  // the tcgen05 query-side kernel forms delta itself
+    return attention_bwd_tc(q, k, v, ldq, ldkv, o, dout, ldo, lse, delta, dq, dk, dv, ld_dq, ld_dkv, batch, seq, nq,
+                            nkv, s);
   k_attn_delta<<<(M * nq + 7) / 8, 256, 0, s>>>(o, dout, ldo, M, seq, nq, d, delta);
   note_launch();
-  if (attention_tc() && attention_fwd_tc_supported(seq, d, nq, nkv, ldq, ldkv, ldo) && ld_dq % 8 == 0 &&
-      ld_dkv % 8 == 0)
-    return attention_bwd_tc(q, k, v, ldq, ldkv, dout, ldo, lse, delta, dq, dk, dv, ld_dq, ld_dkv, batch, seq, nq, nkv,
-                            s);
   dim3 gq(seq / TQ, nq, batch), gk(nkv, batch, seq / TK);
   if (d == 128) {
     const int sq = 6 * Tile<128>::BYTES, sk = 10 * Tile<128>::BYTES + 2048;
@@ -557,4 +557,21 @@ extern "C" int nf4ls_attention_fwd(const nf4ls_layer_cfg* cfg, const void* q_dev
                               static_cast<const __nv_bfloat16*>(v_dev), ld_q, ld_kv, static_cast<__nv_bfloat16*>(o_dev),
                               cfg->n_q * cfg->head_dim, lse_dev, cfg->batch, cfg->seq, cfg->n_q, cfg->n_kv,
                               cfg->head_dim, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int nf4ls_attention_bwd(const nf4ls_layer_cfg* cfg, const void* q_dev, const void* k_dev, const void* v_dev,
+                                   int ld_q, int ld_kv, const void* o_dev, const void* do_dev, const float* lse_dev,
+                                   float* delta_dev, void* dq_dev, void* dk_dev, void* dv_dev, nf4ls_stream stream) {
+  nf4ls::clear_error();
+  if (!cfg || !q_dev || !k_dev || !v_dev || !o_dev || !do_dev || !lse_dev || !delta_dev || !dq_dev || !dk_dev ||
+      !dv_dev)
+    return nf4ls::fail(NF4LS_INVALID_ARG, "null argument");
+  const int qd = cfg->n_q * cfg->head_dim, kvd = cfg->n_kv * cfg->head_dim;
+  return nf4ls::attention_bwd(static_cast<const __nv_bfloat16*>(q_dev), static_cast<const __nv_bfloat16*>(k_dev),
+                              static_cast<const __nv_bfloat16*>(v_dev), ld_q, ld_kv,
+                              static_cast<const __nv_bfloat16*>(o_dev), static_cast<const __nv_bfloat16*>(do_dev), qd,
+                              lse_dev, delta_dev, static_cast<__nv_bfloat16*>(dq_dev),
+                              static_cast<__nv_bfloat16*>(dk_dev), static_cast<__nv_bfloat16*>(dv_dev), qd, kvd,
+                              cfg->batch, cfg->seq, cfg->n_q, cfg->n_kv, cfg->head_dim,
+                              static_cast<cudaStream_t>(stream));
 }

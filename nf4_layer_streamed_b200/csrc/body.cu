@@ -1,6 +1,5 @@
 // Layer-body and model-end kernels around the tcgen05 GEMMs: RMSNorm forward and
-// backward (K8), RoPE tables and the RoPE transpose for dL/dq, dL/dk (K9), the LoRA
-// down-projection, its gradient products and the padded adapter operands (K6/K7),
+// backward (K8), RoPE tables and the RoPE transpose for dL/dq, dL/dk (K9),
 // embedding gather (K13), causal-LM cross-entropy with its gradient (K12), the
 // single-layer mean-square loss, and AdamW (K14).
 //
@@ -121,6 +120,109 @@ __global__ void k_rmsnorm_bwd(const __nv_bfloat16* __restrict__ x, const __nv_bf
   }
 }
 
+// The same two kernels with the row held in registers (MAXV 16-byte vectors per lane
+// at most): one read of each input row instead of two, and every load of a row issued
+// before the first use.  Same arithmetic, in the same order, as the kernels above.
+template <int MAXV>
+__global__ void __launch_bounds__(256) k_rmsnorm_fwd_reg(const __nv_bfloat16* __restrict__ x,
+                                                         const __nv_bfloat16* __restrict__ w,
+                                                         __nv_bfloat16* __restrict__ y, int M, int H, float eps) {
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)row * H);
+  const uint4* wr = reinterpret_cast<const uint4*>(w);
+  uint4* yr = reinterpret_cast<uint4*>(y + (size_t)row * H);
+  const int nv = H / 8;
+  uint4 v[MAXV];
+#pragma unroll
+  for (int j = 0; j < MAXV; ++j)
+    if (lane + 32 * j < nv) v[j] = xr[lane + 32 * j];
+  float ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < MAXV; ++j)
+    if (lane + 32 * j < nv) {
+      float f[8];
+      unpack8(v[j], f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ss += f[e] * f[e];
+    }
+  ss = warp_sum(ss);
+  const float r = 1.0f / sqrtf(ss / (float)H + eps);
+#pragma unroll
+  for (int j = 0; j < MAXV; ++j) {
+    const int i = lane + 32 * j;
+    if (i < nv) {
+      float f[8], g[8];
+      unpack8(v[j], f);
+      unpack8(wr[i], g);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) f[e] = f[e] * r * g[e];
+      yr[i] = pack8(f);
+    }
+  }
+}
+
+template <int MAXV>
+__global__ void __launch_bounds__(256) k_rmsnorm_bwd_reg(const __nv_bfloat16* __restrict__ x,
+                                                         const __nv_bfloat16* __restrict__ w,
+                                                         const __nv_bfloat16* __restrict__ dy,
+                                                         const __nv_bfloat16* __restrict__ resid,
+                                                         __nv_bfloat16* __restrict__ dx, int M, int H, float eps) {
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)row * H);
+  const uint4* wr = reinterpret_cast<const uint4*>(w);
+  const uint4* dr = reinterpret_cast<const uint4*>(dy + (size_t)row * H);
+  const uint4* rr = resid ? reinterpret_cast<const uint4*>(resid + (size_t)row * H) : nullptr;
+  uint4* out = reinterpret_cast<uint4*>(dx + (size_t)row * H);
+  const int nv = H / 8;
+  uint4 xv[MAXV], dv[MAXV];
+#pragma unroll
+  for (int j = 0; j < MAXV; ++j)
+    if (lane + 32 * j < nv) {
+      xv[j] = xr[lane + 32 * j];
+      dv[j] = dr[lane + 32 * j];
+    }
+  float ss = 0.f, dot = 0.f;
+#pragma unroll
+  for (int j = 0; j < MAXV; ++j)
+    if (lane + 32 * j < nv) {
+      float a[8], b[8], c[8];
+      unpack8(xv[j], a);
+      unpack8(wr[lane + 32 * j], b);
+      unpack8(dv[j], c);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        ss += a[e] * a[e];
+        dot += b[e] * c[e] * a[e];
+      }
+    }
+  ss = warp_sum(ss);
+  dot = warp_sum(dot);
+  const float r = 1.0f / sqrtf(ss / (float)H + eps);
+  const float k = r * r * r * dot / (float)H;
+#pragma unroll
+  for (int j = 0; j < MAXV; ++j) {
+    const int i = lane + 32 * j;
+    if (i < nv) {
+      float a[8], b[8], c[8], e[8];
+      unpack8(xv[j], a);
+      unpack8(wr[i], b);
+      unpack8(dv[j], c);
+      if (rr)
+        unpack8(rr[i], e);
+      else
+#pragma unroll
+        for (int q = 0; q < 8; ++q) e[q] = 0.f;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) e[q] += r * b[q] * c[q] - a[q] * k;
+      out[i] = pack8(e);
+    }
+  }
+}
+
 // ------------------------------------------------------------------ RoPE
 // cos/sin of position p and frequency j, twice: [seq, d/2] (row per position) for
 // k_rope_bwd and [d/2, seq] (row per frequency) for the GEMM epilogue, whose lanes hold
@@ -185,13 +287,6 @@ __global__ void k_rope_bwd8(__nv_bfloat16* __restrict__ x, int ld, int cols, int
   }
   *reinterpret_cast<uint4*>(p) = pack8(o1);
   *reinterpret_cast<uint4*>(p + half) = pack8(o2);
-}
-
-__global__ void k_zero_cols(__nv_bfloat16* __restrict__ x, int ld, int M, int c0, int c1) {
-  const int w = c1 - c0;
-  const size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
-  if (i >= (size_t)M * w) return;
-  x[(i / w) * ld + c0 + (i % w)] = __float2bfloat16_rn(0.f);
 }
 
 // ------------------------------------------------------------------ embedding, CE, losses, AdamW
@@ -474,10 +569,21 @@ inline unsigned blocks_for(size_t n, int threads) { return (unsigned)((n + threa
 
 }  // namespace
 
+// Rows of up to 32 * 24 16-byte vectors (H <= 6144) are held in registers; an instance
+// per register budget: 4 vectors per lane (H <= 1024: the SmolLM2 shapes), 16 (the 8B
+// hidden size 4096), 24 (the 32B-class 5120).
 int rmsnorm_fwd(const __nv_bfloat16* x, const __nv_bfloat16* w, __nv_bfloat16* y, int M, int H, float eps,
                 cudaStream_t s) {
   if (H % 8) return fail(NF4LS_SHAPE, "rmsnorm: H %% 8");
-  k_rmsnorm_fwd<<<(M + 7) / 8, 256, 0, s>>>(x, w, y, M, H, eps);
+  const int per_lane = (H / 8 + 31) / 32;
+  if (per_lane <= 4)
+    k_rmsnorm_fwd_reg<4><<<(M + 7) / 8, 256, 0, s>>>(x, w, y, M, H, eps);
+  else if (per_lane <= 16)
+    k_rmsnorm_fwd_reg<16><<<(M + 7) / 8, 256, 0, s>>>(x, w, y, M, H, eps);
+  else if (per_lane <= 24)
+    k_rmsnorm_fwd_reg<24><<<(M + 7) / 8, 256, 0, s>>>(x, w, y, M, H, eps);
+  else
+    k_rmsnorm_fwd<<<(M + 7) / 8, 256, 0, s>>>(x, w, y, M, H, eps);
   note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;
@@ -485,7 +591,15 @@ int rmsnorm_fwd(const __nv_bfloat16* x, const __nv_bfloat16* w, __nv_bfloat16* y
 
 int rmsnorm_bwd(const __nv_bfloat16* x, const __nv_bfloat16* w, const __nv_bfloat16* dy, const __nv_bfloat16* resid,
                 __nv_bfloat16* dx, int M, int H, float eps, cudaStream_t s) {
-  k_rmsnorm_bwd<<<(M + 7) / 8, 256, 0, s>>>(x, w, dy, resid, dx, M, H, eps);
+  const int per_lane = (H / 8 + 31) / 32;
+  if (H % 8)
+    return fail(NF4LS_SHAPE, "rmsnorm_bwd: H %% 8");
+  else if (per_lane <= 4)
+    k_rmsnorm_bwd_reg<4><<<(M + 7) / 8, 256, 0, s>>>(x, w, dy, resid, dx, M, H, eps);
+  else if (per_lane <= 16)
+    k_rmsnorm_bwd_reg<16><<<(M + 7) / 8, 256, 0, s>>>(x, w, dy, resid, dx, M, H, eps);
+  else
+    k_rmsnorm_bwd<<<(M + 7) / 8, 256, 0, s>>>(x, w, dy, resid, dx, M, H, eps);
   note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;
@@ -512,12 +626,6 @@ int rope_bwd(__nv_bfloat16* x, int ld, int M, int cols, int seq, int d, const fl
   return NF4LS_OK;
 }
 
-int zero_cols(__nv_bfloat16* x, int ld, int M, int c0, int c1, cudaStream_t s) {
-  k_zero_cols<<<blocks_for((size_t)M * (c1 - c0), 256), 256, 0, s>>>(x, ld, M, c0, c1);
-  note_launch();
-  NF4_CUDA_TRY(cudaGetLastError());
-  return NF4LS_OK;
-}
 
 int embed(const int32_t* ids, const __nv_bfloat16* E, __nv_bfloat16* h, int M, int H, cudaStream_t s) {
   k_embed<<<M, 128, 0, s>>>(ids, E, h, M, H);

@@ -4,8 +4,9 @@
 //
 // The products come from the layer-streaming pages: the frozen base linears run
 // for the forward, for the checkpoint recompute and for dL/dx = W^T dL/dy
-// ("4GB 显存微调 8B 模型是真的", mechanism section; "Soup layer-streamed NF4 gate
-// record" §4.4: C = 6, no dL/dW), on NF4 weights with double-quantised absmax
+// ("4GB 显存微调 8B 模型是真的", mechanism section;
+// "Soup 层流式 NF4 训练实测：在 4 GB 显存上以位级一致标准完成 8B 模型 LoRA 微调"
+// §4.4: C = 6, no dL/dW), on NF4 weights with double-quantised absmax
 // (§2.1, §2.4).  The decode is the dequantisation of §2.4 exactly:
 // w^ = bf16_rne(fp32(nf4[code] * fp32(fp32(code8[q8] * nested) + offset))).
 //

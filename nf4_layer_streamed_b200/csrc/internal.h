@@ -241,10 +241,12 @@ int tma_map_bf16(CUtensorMap* map, const void* ptr, uint64_t cols, uint64_t rows
 bool attention_fwd_tc_supported(int seq, int d, int nq, int nkv, int ldq, int ldkv, int ldo);
 int attention_fwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, int ldq, int ldkv,
                      __nv_bfloat16* o, int ldo, float* lse, int batch, int seq, int nq, int nkv, cudaStream_t s);
+// The tcgen05 backward: the query-side kernel also forms delta = rowsum(dO * O) (into
+// `delta`, [batch, nq, seq]) for the key-side kernel that follows it.
 int attention_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, int ldq, int ldkv,
-                     const __nv_bfloat16* dout, int ldo, const float* lse, const float* delta, __nv_bfloat16* dq,
-                     __nv_bfloat16* dk, __nv_bfloat16* dv, int ld_dq, int ld_dkv, int batch, int seq, int nq, int nkv,
-                     cudaStream_t s);
+                     const __nv_bfloat16* o, const __nv_bfloat16* dout, int ldo, const float* lse, float* delta,
+                     __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv, int ld_dq, int ld_dkv, int batch, int seq,
+                     int nq, int nkv, cudaStream_t s);
 int attention_fwd(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, int ldq, int ldkv,
                   __nv_bfloat16* o, int ldo, float* lse, int batch, int seq, int nq, int nkv, int d,
                   cudaStream_t s);
@@ -253,15 +255,19 @@ int attention_bwd(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfl
                   __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv, int ld_dq, int ld_dkv, int batch,
                   int seq, int nq, int nkv, int d, cudaStream_t s);
 
-size_t lora_partial_bytes(int M, int Nmax);
-int lora_pack2(const nf4ls_lora* l, int H, int qd, int kvd, float scale, __nv_bfloat16* bup, __nv_bfloat16* adn,
-               __nv_bfloat16* bqt, __nv_bfloat16* bvt, cudaStream_t s);
-int lora_rows(const __nv_bfloat16* X, int ldx, int M, int nseg, const int* xcol, const int* K,
-              const __nv_bfloat16* const* W, const int* ldw, float scale, float* part, __nv_bfloat16* out_b, int ldb,
-              int oc, cudaStream_t s);
-int lora_cols(const __nv_bfloat16* X, int ldx, int xcol, int N, int M, const __nv_bfloat16* Y, int ldy, int ycol,
-              int NR, float scale, float* part, float* out0, float* out1, int so_n, int so_r, cudaStream_t s);
-int zero_cols(__nv_bfloat16* x, int ld, int M, int c0, int c1, cudaStream_t s);
+// LoRA (lora.cu).  Forward: h1 = rmsnorm(x) w, t = [h1 A_q^T | h1 A_v^T] into tpad
+// [M, 64] (bf16, zeros in columns 32-63) and the bf16 adapter operands bup [Nqkv, 64],
+// adn [64, H], bqt [16, qd], bvt [16, kvd] from the fp32 masters, in one launch.
+int norm_lora_fwd(const __nv_bfloat16* x, const __nv_bfloat16* w, __nv_bfloat16* h1, int M, int H, float eps,
+                  const nf4ls_lora* l, int qd, int kvd, float scale, __nv_bfloat16* tpad, __nv_bfloat16* bup,
+                  __nv_bfloat16* adn, __nv_bfloat16* bqt, __nv_bfloat16* bvt, cudaStream_t s);
+// Backward, two launches: dB_q, dB_v, dA_q, dA_v (fp32, written) and dt into dtpad
+// [M, 64] (bf16, zeros in columns 32-63) from dq (columns [0, qd) of dqkv) and dv
+// (columns [vcol, vcol + kvd)); part: lora_partial_bytes of scratch.
+size_t lora_partial_bytes(int M, int H, int qd, int kvd);
+int lora_bwd(const __nv_bfloat16* dqkv, int ld, int vcol, int M, int H, int qd, int kvd, const __nv_bfloat16* tpad,
+             const __nv_bfloat16* bqt, const __nv_bfloat16* bvt, const __nv_bfloat16* h1, float scale,
+             __nv_bfloat16* dtpad, const nf4ls_lora_grads* g, void* part, cudaStream_t s);
 int embed(const int32_t* ids, const __nv_bfloat16* E, __nv_bfloat16* h, int M, int H, cudaStream_t s);
 // Streamed head, per vocab chunk [v0, v0 + n) of the output matrix (rows Wc in HBM):
 // logits [M, n] (bf16, from the GEMM) are folded into the per-row running max mx, sum

@@ -71,7 +71,7 @@ WsLayout ws_layout(const nf4ls_layer_cfg* c) {
   L.delta = take((size_t)c->batch * c->n_q * c->seq * 4);
   L.bqt = take(16 * qd * 2);
   L.bvt = take(16 * kvd * 2);
-  L.part = take(lora_partial_bytes((int)M, (int)std::max(H, qd)));
+  L.part = take(lora_partial_bytes((int)M, (int)H, (int)qd, (int)kvd));
   L.dtpad = take(M * 64 * 2);
   L.dh1 = take(M * H * 2);
   // bf16 copy of the layer's seven linears for the dequantise-then-multiply path
@@ -161,20 +161,18 @@ int forward_body(LayerCtx& x, const nf4ls_lora* lora, const __nv_bfloat16* X, __
   auto* h2 = at<__nv_bfloat16>(ws, x.L.h2);
   auto* act = at<__nv_bfloat16>(ws, x.L.act);
   auto* tpad = at<__nv_bfloat16>(ws, x.L.tpad);
-  NF4_TRY(rmsnorm_fwd(X, x.v.norm_in, h1, M, H, c->rms_eps, s));
   GemmExtra ex;
   if (lora) {
+    // h1 and t = [h1 A_q^T | h1 A_v^T] (columns 0-31 of the padded extra operand) in one
+    // pass, with the bf16 adapter operands
     auto* bup = at<__nv_bfloat16>(ws, x.L.bup);
-    auto* adn = at<__nv_bfloat16>(ws, x.L.adn);
-    NF4_TRY(lora_pack2(lora, H, x.qd, x.kvd, x.scale, bup, adn, at<__nv_bfloat16>(ws, x.L.bqt),
-                       at<__nv_bfloat16>(ws, x.L.bvt), s));
-    NF4_TRY(zero_cols(tpad, 64, M, 32, 64, s));
-    // t = [h1 A_q^T | h1 A_v^T] into columns 0-31 of the padded extra operand
-    const int xcol[2] = {0, 0}, K[2] = {H, H}, ldw[2] = {H, H};
-    const __nv_bfloat16* Wd[2] = {adn, adn + (size_t)16 * H};
-    NF4_TRY(lora_rows(h1, H, M, 2, xcol, K, Wd, ldw, 1.0f, at<float>(ws, x.L.part), tpad, 64, 0, s));
+    NF4_TRY(norm_lora_fwd(X, x.v.norm_in, h1, M, H, c->rms_eps, lora, x.qd, x.kvd, x.scale, tpad, bup,
+                          at<__nv_bfloat16>(ws, x.L.adn), at<__nv_bfloat16>(ws, x.L.bqt),
+                          at<__nv_bfloat16>(ws, x.L.bvt), s));
     ex.a = tpad;
     ex.b = bup;
+  } else {
+    NF4_TRY(rmsnorm_fwd(X, x.v.norm_in, h1, M, H, c->rms_eps, s));
   }
   GemmEpilogue e;
   e.kind = EPI_ROPE;
@@ -278,20 +276,12 @@ int layer_bwd_impl(const nf4ls_layer_cfg* c, const void* shard, const nf4ls_lora
   NF4_TRY(rope_bwd(dqkv, x.nqkv, M, x.qd + x.kvd, c->seq, c->head_dim, at<float>(ws, x.L.cos), at<float>(ws, x.L.sin), s));
   GemmExtra ex;
   if (lora) {
-    auto* tpad = at<__nv_bfloat16>(ws, x.L.tpad);
+    // dB = s [dq^T t_q | dv^T t_v], dt = s [dq B_q | dv B_v] (bf16, the extra operand of
+    // the dL/dx GEMM), dA = dt^T h1
     auto* dtpad = at<__nv_bfloat16>(ws, x.L.dtpad);
-    float* part = at<float>(ws, x.L.part);
-    const int vcol = x.qd + x.kvd;
-    // dB = s dq^T t_q, s dv^T t_v
-    NF4_TRY(lora_cols(dqkv, x.nqkv, 0, x.qd, M, tpad, 64, 0, 16, x.scale, part, g->dB_q, nullptr, 16, 1, s));
-    NF4_TRY(lora_cols(dqkv, x.nqkv, vcol, x.kvd, M, tpad, 64, 16, 16, x.scale, part, g->dB_v, nullptr, 16, 1, s));
-    // dt = s [dq B_q | dv B_v] (bf16, the extra operand of the dL/dx GEMM)
-    NF4_TRY(zero_cols(dtpad, 64, M, 32, 64, s));
-    const int xcol[2] = {0, vcol}, K[2] = {x.qd, x.kvd}, ldw[2] = {x.qd, x.kvd};
-    const __nv_bfloat16* Wt[2] = {at<__nv_bfloat16>(ws, x.L.bqt), at<__nv_bfloat16>(ws, x.L.bvt)};
-    NF4_TRY(lora_rows(dqkv, x.nqkv, M, 2, xcol, K, Wt, ldw, x.scale, part, dtpad, 64, 0, s));
-    // dA = dt^T h1 for q (dt columns 0-15) and v (16-31)
-    NF4_TRY(lora_cols(h1, H, 0, H, M, dtpad, 64, 0, 32, 1.0f, part, g->dA_q, g->dA_v, 1, H, s));
+    NF4_TRY(lora_bwd(dqkv, x.nqkv, x.qd + x.kvd, M, H, x.qd, x.kvd, at<__nv_bfloat16>(ws, x.L.tpad),
+                     at<__nv_bfloat16>(ws, x.L.bqt), at<__nv_bfloat16>(ws, x.L.bvt), h1, x.scale, dtpad, g,
+                     at<void>(ws, x.L.part), s));
     ex.a = dtpad;
     ex.b = at<__nv_bfloat16>(ws, x.L.adn);
   }

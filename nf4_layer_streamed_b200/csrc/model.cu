@@ -6,8 +6,9 @@
 // From the layer-streaming review ("4GB 显存微调 8B 模型是真的", mechanism section):
 // only the adapter, its gradients and its optimiser state stay resident, together with
 // the unquantised embedding and lm_head; the frozen layers are prefetched one step
-// ahead on a side stream, i+1 in the forward and i-1 in the backward.  From the gate
-// record §4.4: lm_head sits outside the checkpointed layers (2 forward + 2 dL/dx FLOP
+// ahead on a side stream, i+1 in the forward and i-1 in the backward.  From
+// "Soup 层流式 NF4 训练实测：在 4 GB 显存上以位级一致标准完成 8B 模型 LoRA 微调"
+// §4.4: lm_head sits outside the checkpointed layers (2 forward + 2 dL/dx FLOP
 // per parameter and token).  The DPO/KTO write-up ("Soup v0.72.4 技术解析" §3.1) reuses
 // the same streamed base with the adapter switched off as the reference model, which
 // nf4ls_forward_loss(lora_on = 0) provides.

@@ -9,7 +9,7 @@ product out = x W^T and the dL/dx product out = dy W.
 
     python -m nf4_layer_streamed_b200.gemm_bench [--M 2048] [--shapes gateup,down] [--iters 20]
     python -m nf4_layer_streamed_b200.gemm_bench --once --shapes gateup   (one launch each: for ncu)
-    python -m nf4_layer_streamed_b200.gemm_bench --attention 4 [--once]      (attention forward, batch 4)
+    python -m nf4_layer_streamed_b200.gemm_bench --attention 4 [--once]      (attention fwd / bwd, batch 4)
     python -m nf4_layer_streamed_b200.gemm_bench --layer 4 [--once]   (quantise + one 8B layer fwd/bwd)
 
 Prints one JSON object per (shape, direction, kernel) with the mean launch time
@@ -101,38 +101,37 @@ def run_quant(iters: int = 10):
 
 
 def run_attention(batch: int, once: bool, iters: int = 20):
-    """Causal GQA attention forward of the Llama-8B layer (32 query heads, 8 kv heads,
-    d 128) at seq 512: the tcgen05 kernel and the mma.sync kernel."""
+    """Causal GQA attention of the Llama-8B layer (32 query heads, 8 kv heads, d 128) at
+    seq 512: forward and backward (query side with delta, then key side), the tcgen05
+    kernels and the mma.sync kernels.  Algorithmic FLOPs: forward 4 S^2 d n_q B / 2
+    (causal half), backward 2.5 times that (five products against two)."""
     shape = synth.LLAMA_8B
     seq = 512
     cfg = api.layer_cfg(shape, batch, seq)
     qd, kvd = shape.q_dim, shape.kv_dim
     ld = qd + 2 * kvd
     qkv = synth.tensor_values((batch * seq, ld), seed=3, scale=1.0, device="cuda")
+    do = synth.tensor_values((batch * seq, qd), seed=4, scale=1.0, device="cuda")
+    args = (cfg, qkv, qkv[:, qd:], qkv[:, qd + kvd:], ld, ld)
     out = []
+    flops = 4.0 * seq * seq * shape.head_dim * shape.n_q * batch / 2
     for tc in ((True,) if once else (True, False)):
         api.set_attention_path(tc)
-        f = lambda: api.attention_fwd(cfg, qkv, qkv[:, qd:], qkv[:, qd + kvd:], ld, ld)
+        o, lse = api.attention_fwd(*args)
+        fwd = lambda: api.attention_fwd(*args)
+        bwd = lambda: api.attention_bwd(*args, o, do, lse)
         if once:
-            f()
-            f()
+            for f in (fwd, fwd, bwd, bwd):
+                f()
             torch.cuda.synchronize()
             continue
-        for _ in range(3):
-            f()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(iters):
-            f()
-        e1.record()
-        torch.cuda.synchronize()
-        us = e0.elapsed_time(e1) / iters * 1000.0
-        flops = 4.0 * seq * seq * shape.head_dim * shape.n_q * batch / 2
-        rec = {"kernel": "attention_fwd_tcgen05" if tc else "attention_fwd_mma_sync", "batch": batch, "seq": seq,
-               "us": us, "tflops": flops / us / 1e6}
-        out.append(rec)
-        print(json.dumps(rec), flush=True)
+        name = "tcgen05" if tc else "mma_sync"
+        for part, f, fl in (("forward", fwd, flops), ("backward", bwd, 2.5 * flops)):
+            us = _time(f, iters) * 1000.0
+            rec = {"kernel": f"attention_{part}_{name}", "batch": batch, "seq": seq, "us": us,
+                   "tflops": fl / us / 1e6}
+            out.append(rec)
+            print(json.dumps(rec), flush=True)
     api.set_attention_path(True)
     return out
 

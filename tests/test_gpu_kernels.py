@@ -233,3 +233,38 @@ def test_tcgen05_attention_matches_mma_sync_attention(seq):
     close(lse1, f64(lse_ref), tol=1e-4, what="log-sum-exp")
     st, err = api.device_error()
     assert st == 0, err
+
+
+@pytest.mark.parametrize("batch,seq", [(2, 128), (2, 384), (1, 512)])
+def test_tcgen05_attention_backward_against_oracle(batch, seq):
+    """The tcgen05 attention backward (query side: dQ and delta; key side: dK, dV over
+    the query heads of each kv group) on the Llama-8B head layout, against the oracle's
+    float64 backward on the same bf16 q, k, v, o and dO: dq, dk, dv within 2e-2 max|ref|,
+    delta = rowsum(dO * O) within 1e-4 (fp32 sums of bf16 products), and bit-exact
+    across reruns."""
+    shape = synth.LLAMA_8B
+    cfg = api.layer_cfg(shape, batch, seq)
+    M, qd, kvd = batch * seq, shape.q_dim, shape.kv_dim
+    ld = qd + 2 * kvd
+    qkv = synth.tensor_values((M, ld), seed=seq + 11, scale=1.0).to(DEV)
+    args = (cfg, qkv, qkv[:, qd:], qkv[:, qd + kvd:], ld, ld)
+    o, lse = api.attention_fwd(*args)
+    do = synth.tensor_values((M, qd), seed=seq + 12, scale=1.0).to(DEV)
+    dq, dk, dv, delta = api.attention_bwd(*args, o, do, lse)
+    dq2, dk2, dv2, delta2 = api.attention_bwd(*args, o, do, lse)
+    torch.cuda.synchronize()
+    assert torch.equal(dq, dq2) and torch.equal(dk, dk2) and torch.equal(dv, dv2) and torch.equal(delta, delta2)
+    x = f64(qkv)
+    q = x[:, :qd].reshape(batch, seq, shape.n_q, shape.head_dim)
+    k = x[:, qd:qd + kvd].reshape(batch, seq, shape.n_kv, shape.head_dim)
+    v = x[:, qd + kvd:].reshape(batch, seq, shape.n_kv, shape.head_dim)
+    _, P = olayer.attention(q, k, v)
+    d_o = f64(do).reshape(batch, seq, shape.n_q, shape.head_dim)
+    rq, rk, rv = olayer.attention_bwd(q, k, v, P, d_o)
+    close(dq, rq.reshape(M, qd), what="dq")
+    close(dk, rk.reshape(M, kvd), what="dk")
+    close(dv, rv.reshape(M, kvd), what="dv")
+    ref_delta = (f64(o) * f64(do)).reshape(batch, seq, shape.n_q, shape.head_dim).sum(-1).transpose(0, 2, 1)
+    close(delta, ref_delta, tol=1e-4, what="delta")
+    st, err = api.device_error()
+    assert st == 0, err
