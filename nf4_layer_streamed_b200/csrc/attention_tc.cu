@@ -69,6 +69,14 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// 2^x by the hardware approximation (ex2.approx, flush-to-zero): its relative error is
+// far below the bf16 rounding that every probability gets next.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // D[tmem] (+)= A[tmem] * B[smem desc]: A of M = 128 lanes x 16 bf16 (8 columns).
 __device__ __forceinline__ void umma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
                                              uint32_t accumulate) {
@@ -199,23 +207,28 @@ __global__ void __launch_bounds__(F_THREADS, 2) k_attn_fwd_tc(const __grid_const
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(s_full, kt & 1, abort_flag, p.err, KID_ATTN, 27)))) break;
       tc_fence_after();
       const bool diag = kt == qt;
+      // row maximum of the raw scores (the scale is positive), two TMEM loads per wait
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tmem_ld32(trow + c * 32, v);
+      for (int c = 0; c < 4; c += 2) {
+        uint32_t v[2][32];
+        tmem_ld32(trow + c * 32, v[0]);
+        tmem_ld32(trow + c * 32 + 32, v[1]);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (!diag || c * 32 + i <= r) mx = fmaxf(mx, __uint_as_float(v[i]) * sl);
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (!diag || (c + h) * 32 + i <= r) mx = fmaxf(mx, __uint_as_float(v[h][i]));
       }
+      mx *= sl;
       const float m_new = (kt == 0 || mx > m_run + kRescaleLog2) ? fmaxf(mx, m_run) : m_run;
       const bool resc = kt > 0 && m_new != m_run;
       if (__any_sync(0xffffffffu, resc)) {
         // the previous tile's P V product must be in O before O is scaled
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(o_full, (kt - 1) & 1, abort_flag, p.err, KID_ATTN, 28)))) break;
         tc_fence_after();
-        const float alpha = resc ? exp2f(m_run - m_new) : 1.0f;
+        const float alpha = resc ? fast_exp2(m_run - m_new) : 1.0f;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t v[32];
@@ -231,20 +244,28 @@ __global__ void __launch_bounds__(F_THREADS, 2) k_attn_fwd_tc(const __grid_const
       m_run = m_new;
       float sum = 0.f;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        // keys 32 c .. 32 c + 31; their P goes to columns 16 c .., scores already read
-        uint32_t v[32], pk[16];
-        tmem_ld32(trow + c * 32, v);
+      for (int c = 0; c < 4; c += 2) {
+        // keys 32 c .. 32 c + 63; their P goes to columns 16 c .., scores already read
+        uint32_t v[2][32], pk[2][16];
+        tmem_ld32(trow + c * 32, v[0]);
+        tmem_ld32(trow + c * 32 + 32, v[1]);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int k0 = c * 32 + 2 * j;
-          const float p0 = (!diag || k0 <= r) ? exp2f(__uint_as_float(v[2 * j]) * sl - m_run) : 0.f;
-          const float p1 = (!diag || k0 + 1 <= r) ? exp2f(__uint_as_float(v[2 * j + 1]) * sl - m_run) : 0.f;
-          sum += p0 + p1;
-          pk[j] = pack_bf16x2(p0, p1);
-        }
-        tmem_st16(trow + c * 16, pk);
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int k0 = (c + h) * 32 + 2 * j;
+            float p0 = fast_exp2(fmaf(__uint_as_float(v[h][2 * j]), sl, -m_run));
+            float p1 = fast_exp2(fmaf(__uint_as_float(v[h][2 * j + 1]), sl, -m_run));
+            if (diag) {
+              p0 = k0 <= r ? p0 : 0.f;
+              p1 = k0 + 1 <= r ? p1 : 0.f;
+            }
+            sum += p0 + p1;
+            pk[h][j] = pack_bf16x2(p0, p1);
+          }
+        tmem_st16(trow + c * 16, pk[0]);
+        tmem_st16(trow + c * 16 + 16, pk[1]);
       }
       tmem_wait_st();
       l_run += sum;
@@ -314,10 +335,7 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 }
 
 struct AttnBwdParams {
-  CUtensorMap tq, tk, tv, tdo;  // box 64 cols x 128 rows, 128-byte swizzle
-  const __nv_bfloat16* o;       // attention output (query side: delta)
-  const __nv_bfloat16* dout;
-  int ldo;
+  CUtensorMap tq, tk, tv, tdo, to;  // box 64 cols x 128 rows, 128-byte swizzle (to: the output O)
   const float* lse;
   float* delta;                 // written by the query side, read by the key side
   __nv_bfloat16* dq;
@@ -333,9 +351,9 @@ struct AttnBwdParams {
 constexpr int B_THREADS = 320, B_PROD = 8, B_MMA = 9, B_EW = 256;
 constexpr int B_OFF_A = 0;                              // Q, dO (query side) or K, V (key side)
 constexpr int B_OFF_RING = 2 * TILE_BYTES;              // 2 stages x (two 32 KB tiles)
-constexpr int B_OFF_LD = B_OFF_RING + 4 * TILE_BYTES;   // key side: 2 stages x (128 lse + 128 delta floats)
-constexpr int B_OFF_RED = B_OFF_LD + 2 * 1024;          // query side: delta halves [2][128]
-constexpr int B_OFF_BAR = B_OFF_RED + 1024;
+constexpr int B_OFF_X = B_OFF_RING + 4 * TILE_BYTES;    // query side: O tile and delta halves [2][128];
+                                                        // key side: 2 stages x (128 lse + 128 delta floats)
+constexpr int B_OFF_BAR = B_OFF_X + TILE_BYTES + 1024;
 constexpr int SMEM_BWD = 1024 + B_OFF_BAR + 256;
 
 __device__ __forceinline__ void bar_ew() { asm volatile("bar.sync 1, %0;" ::"n"(B_EW) : "memory"); }
@@ -393,10 +411,12 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
       tma_prefetch_desc(&p.tk);
       tma_prefetch_desc(&p.tv);
       tma_prefetch_desc(&p.tdo);
-      mbar_arrive_expect_tx(q_full, 2 * TILE_BYTES);
+      tma_prefetch_desc(&p.to);
+      mbar_arrive_expect_tx(q_full, 3 * TILE_BYTES);
       for (int j = 0; j < 2; ++j) {
         tma_load_2d(base + B_OFF_A + j * ATOM, &p.tq, q_full, h * 128 + 64 * j, row0 + qt * TT);
         tma_load_2d(base + B_OFF_A + TILE_BYTES + j * ATOM, &p.tdo, q_full, h * 128 + 64 * j, row0 + qt * TT);
+        tma_load_2d(base + B_OFF_X + j * ATOM, &p.to, q_full, h * 128 + 64 * j, row0 + qt * TT);
       }
       int issued = 0;
       for (int kt = 0; kt < n_kt; ++kt) {
@@ -471,28 +491,31 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
     const int qpos = qt * TT + r;
     const uint32_t trow = tmem + ((uint32_t)(wq * 32) << 16);
     const size_t li = ((size_t)b * p.nq + h) * p.seq + qpos;
-    // delta = rowsum(dO * O) over this thread's 64 dims, the two halves added through smem
-    float* red = reinterpret_cast<float*>(base + B_OFF_RED);
-    {
-      const uint4* o4 = reinterpret_cast<const uint4*>(p.o + (size_t)(row0 + qpos) * p.ldo + h * 128 + g * 64);
-      const uint4* d4 = reinterpret_cast<const uint4*>(p.dout + (size_t)(row0 + qpos) * p.ldo + h * 128 + g * 64);
+    // delta = rowsum(dO * O) over this thread's 64 dims (its row in swizzle atom g of the
+    // dO and O tiles), the two halves added through smem
+    float* red = reinterpret_cast<float*>(base + B_OFF_X + TILE_BYTES);
+    bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort_flag, p.err, KID_ATTN, 45));
+    if (ok) {
+      const uint8_t* dO_row = base + B_OFF_A + TILE_BYTES + g * ATOM + r * 128;
+      const uint8_t* o_row = base + B_OFF_X + g * ATOM + r * 128;
       float s = 0.f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const uint4 a = o4[i], c = d4[i];
-        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, cw[4] = {c.x, c.y, c.z, c.w};
+      for (int c = 0; c < 8; ++c) {
+        const uint32_t off = (uint32_t)((c ^ (r & 7)) << 4);
+        const uint4 a = *reinterpret_cast<const uint4*>(o_row + off);
+        const uint4 d = *reinterpret_cast<const uint4*>(dO_row + off);
+        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, dw[4] = {d.x, d.y, d.z, d.w};
 #pragma unroll
-        for (int j = 0; j < 4; ++j) s += bf16_lo(aw[j]) * bf16_lo(cw[j]) + bf16_hi(aw[j]) * bf16_hi(cw[j]);
+        for (int j = 0; j < 4; ++j) s += bf16_lo(aw[j]) * bf16_lo(dw[j]) + bf16_hi(aw[j]) * bf16_hi(dw[j]);
       }
       red[g * 128 + r] = s;
     }
     bar_ew();
-    const float dl = red[r] + red[128 + r];
-    if (g == 0) p.delta[li] = dl;
+    const float dl = ok ? red[r] + red[128 + r] : 0.f;
+    if (ok && g == 0) p.delta[li] = dl;
     const float lse2 = p.lse[li] * 1.4426950408889634f;
     const float sl = p.scale_log2;
-    bool ok = true;
-    for (int it = 0; it < n_it; ++it) {
+    for (int it = 0; ok && it < n_it; ++it) {
       const int bf = it & 1;
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sd_full[bf], (it >> 1) & 1, abort_flag, p.err, KID_ATTN, 46))))
         break;
@@ -508,7 +531,7 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int kj = key0 + 2 * j + e;
-          const float pe = kj <= qpos ? exp2f(__uint_as_float(sv[2 * j + e]) * sl - lse2) : 0.f;
+          const float pe = kj <= qpos ? fast_exp2(fmaf(__uint_as_float(sv[2 * j + e]), sl, -lse2)) : 0.f;
           ds[e] = pe * (__uint_as_float(dpv[2 * j + e]) - dl);
         }
         dd[j] = pack_bf16x2(ds[0], ds[1]);
@@ -552,8 +575,21 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
   }
 }
 
-// KEY side: dK, dV of one 128-key tile of one kv head.
-__global__ void __launch_bounds__(B_THREADS, 1) k_attn_dkv_tc(const __grid_constant__ AttnBwdParams p) {
+// st.shared::cluster of four floats at a shared::cluster address (another CTA's smem).
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
+// KEY side: dK, dV of one 128-key tile of one kv head, by a cluster of two CTAs that split
+// the group's query heads (the first ceil(group / 2) heads and the rest): the second CTA
+// sends its fp32 partial sums through distributed shared memory and the first adds them to
+// its own in that fixed order.  Halving the longest CTAs' work balances the grid (two CTAs
+// per key tile instead of one, the first key tiles holding the most query tiles).
+constexpr int PEER_LD = 132;  // row stride (floats) of the partial sums in the first CTA's smem
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
+    k_attn_dkv_tc(const __grid_constant__ AttnBwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + B_OFF_BAR);
@@ -568,9 +604,12 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dkv_tc(const __grid_const
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kvh = blockIdx.x, b = blockIdx.y, kt = gridDim.z - 1 - blockIdx.z;  // the longest key tiles first
+  const int kvh = blockIdx.x >> 1, b = blockIdx.y, kt = blockIdx.z;  // z slowest: the longest key tiles first
+  const uint32_t crank = cluster_ctarank();
   const int grp = p.nq / p.nkv, n_qt = p.seq / TT;
-  const int per_head = n_qt - kt, n_st = grp * per_head, n_it = 2 * n_st;  // (head, query tile) stages, halves
+  const int hpc = (grp + 1) / 2, h_begin = (int)crank * hpc, h_count = min(grp, h_begin + hpc) - h_begin;
+  // (head, query tile) stages of this CTA, halves
+  const int per_head = n_qt - kt, n_st = h_count * per_head, n_it = 2 * n_st;
   const int row0 = b * p.seq;
 
   if (threadIdx.x == 0) {
@@ -610,9 +649,9 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dkv_tc(const __grid_const
       for (int sti = 0; sti < n_st; ++sti) {
         const int bf = sti & 1;
         if (sti >= 2 && !mbar_wait(&qd_empty[bf], ((sti >> 1) - 1) & 1, abort_flag, p.err, KID_ATTN, 31)) break;
-        const int h = kvh * grp + sti / per_head, qt = kt + sti % per_head;
+        const int h = kvh * grp + h_begin + sti / per_head, qt = kt + sti % per_head;
         uint8_t* buf = base + B_OFF_RING + bf * 2 * TILE_BYTES;
-        float* ld = reinterpret_cast<float*>(base + B_OFF_LD + bf * 1024);
+        float* ld = reinterpret_cast<float*>(base + B_OFF_X + bf * 1024);
         mbar_arrive_expect_tx(&qd_full[bf], 2 * TILE_BYTES + 1024);
         for (int j = 0; j < 2; ++j) {
           tma_load_2d(buf + j * ATOM, &p.tq, &qd_full[bf], h * 128 + 64 * j, row0 + qt * TT);
@@ -632,7 +671,7 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dkv_tc(const __grid_const
     constexpr uint32_t idesc_s = idesc_bf16(128, 64, false);   // S^T, dP^T: N = 64 queries
     constexpr uint32_t idesc_a = idesc_bf16(128, 128, true);   // dV, dK: dO, Q N-major
     const uint32_t sK = smem_u32(base + B_OFF_A), sV = sK + TILE_BYTES;
-    bool ok = __all_sync(0xffffffffu, mbar_wait(kv_full, 0, abort_flag, p.err, KID_ATTN, 32));
+    bool ok = n_it > 0 && __all_sync(0xffffffffu, mbar_wait(kv_full, 0, abort_flag, p.err, KID_ATTN, 32));
     // item it: stage it / 2 (a (head, query tile) pair), half it % 2, TMEM buffer it % 2
     auto second = [&](int it) -> bool {  // dV += P^T dO_half, dK += dS^T Q_half
       if (!__all_sync(0xffffffffu, mbar_wait(&p_full[it & 1], (it >> 1) & 1, abort_flag, p.err, KID_ATTN, 34)))
@@ -691,7 +730,7 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dkv_tc(const __grid_const
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sd_full[bf], (it >> 1) & 1, abort_flag, p.err, KID_ATTN, 35))))
         break;
       tc_fence_after();
-      const float* ld = reinterpret_cast<const float*>(base + B_OFF_LD + (sti & 1) * 1024);
+      const float* ld = reinterpret_cast<const float*>(base + B_OFF_X + (sti & 1) * 1024);
       uint32_t sv[32], dpv[32], pp[16], dd[16];
       tmem_ld32(trow + bf * 128 + g * 32, sv);
       tmem_ld32(trow + bf * 128 + 64 + g * 32, dpv);
@@ -704,7 +743,7 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dkv_tc(const __grid_const
         for (int e = 0; e < 2; ++e) {
           const int qi = qi0 + 2 * j + e;
           const float pe =
-              key <= qt * TT + qi ? exp2f(__uint_as_float(sv[2 * j + e]) * sl - ld[qi] * 1.4426950408889634f) : 0.f;
+              key <= qt * TT + qi ? fast_exp2(fmaf(__uint_as_float(sv[2 * j + e]), sl, -ld[qi] * 1.4426950408889634f)) : 0.f;
           pv[e] = pe;
           ds[e] = pe * (__uint_as_float(dpv[2 * j + e]) - ld[128 + qi]);
         }
@@ -718,31 +757,73 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dkv_tc(const __grid_const
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[bf]);
     }
-    if (ok && __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, p.err, KID_ATTN, 36))) {
-      tc_fence_after();
+    const bool have = n_it > 0 && ok && __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, p.err, KID_ATTN, 36));
+    if (have) tc_fence_after();
+    // both CTAs have finished their products: the first CTA's ring is free for the partials
+    cluster_sync_all();
+    float* peer = reinterpret_cast<float*>(base + B_OFF_RING);  // dV [128][PEER_LD], then dK
+    if (crank == 1) {
+      const uint32_t dst = mapa_shared(smem_u32(peer), 0);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t v[32], k[32];
+        if (have) {
+          tmem_ld32(trow + 256 + g * 64 + c * 32, v);
+          tmem_ld32(trow + 384 + g * 64 + c * 32, k);
+          tmem_wait_ld();
+        }
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const uint32_t o = (uint32_t)((r * PEER_LD + g * 64 + c * 32 + 4 * q4) * 4);
+          if (have) {
+            st_cluster_v4(dst + o, __uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1]),
+                          __uint_as_float(v[4 * q4 + 2]), __uint_as_float(v[4 * q4 + 3]));
+            st_cluster_v4(dst + 128 * PEER_LD * 4 + o, __uint_as_float(k[4 * q4]), __uint_as_float(k[4 * q4 + 1]),
+                          __uint_as_float(k[4 * q4 + 2]), __uint_as_float(k[4 * q4 + 3]));
+          } else {
+            st_cluster_v4(dst + o, 0.f, 0.f, 0.f, 0.f);
+            st_cluster_v4(dst + 128 * PEER_LD * 4 + o, 0.f, 0.f, 0.f, 0.f);
+          }
+        }
+      }
+    }
+    cluster_sync_all();
+    if (crank == 0) {
       uint4* dv = reinterpret_cast<uint4*>(p.dv + (size_t)(row0 + key) * p.ld_dkv + kvh * 128 + g * 64);
       uint4* dk = reinterpret_cast<uint4*>(p.dk + (size_t)(row0 + key) * p.ld_dkv + kvh * 128 + g * 64);
       const float sc = p.scale;
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        uint32_t v[32], k[32];
-        tmem_ld32(trow + 256 + g * 64 + c * 32, v);
-        tmem_ld32(trow + 384 + g * 64 + c * 32, k);
-        tmem_wait_ld();
+        float v[32], k[32];
+        {
+          uint32_t vr[32], kr[32];
+          if (have) {
+            tmem_ld32(trow + 256 + g * 64 + c * 32, vr);
+            tmem_ld32(trow + 384 + g * 64 + c * 32, kr);
+            tmem_wait_ld();
+          }
+          const float* pv = peer + r * PEER_LD + g * 64 + c * 32;
+          const float* pk = pv + 128 * PEER_LD;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            v[i] = (have ? __uint_as_float(vr[i]) : 0.f) + pv[i];
+            k[i] = ((have ? __uint_as_float(kr[i]) : 0.f) + pk[i]) * sc;
+          }
+        }
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
-          dv[c * 4 + q4] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * q4]), __uint_as_float(v[8 * q4 + 1])),
-                                      pack_bf16x2(__uint_as_float(v[8 * q4 + 2]), __uint_as_float(v[8 * q4 + 3])),
-                                      pack_bf16x2(__uint_as_float(v[8 * q4 + 4]), __uint_as_float(v[8 * q4 + 5])),
-                                      pack_bf16x2(__uint_as_float(v[8 * q4 + 6]), __uint_as_float(v[8 * q4 + 7])));
-          dk[c * 4 + q4] =
-              make_uint4(pack_bf16x2(__uint_as_float(k[8 * q4]) * sc, __uint_as_float(k[8 * q4 + 1]) * sc),
-                         pack_bf16x2(__uint_as_float(k[8 * q4 + 2]) * sc, __uint_as_float(k[8 * q4 + 3]) * sc),
-                         pack_bf16x2(__uint_as_float(k[8 * q4 + 4]) * sc, __uint_as_float(k[8 * q4 + 5]) * sc),
-                         pack_bf16x2(__uint_as_float(k[8 * q4 + 6]) * sc, __uint_as_float(k[8 * q4 + 7]) * sc));
+          dv[c * 4 + q4] = make_uint4(pack_bf16x2(v[8 * q4], v[8 * q4 + 1]), pack_bf16x2(v[8 * q4 + 2], v[8 * q4 + 3]),
+                                      pack_bf16x2(v[8 * q4 + 4], v[8 * q4 + 5]), pack_bf16x2(v[8 * q4 + 6], v[8 * q4 + 7]));
+          dk[c * 4 + q4] = make_uint4(pack_bf16x2(k[8 * q4], k[8 * q4 + 1]), pack_bf16x2(k[8 * q4 + 2], k[8 * q4 + 3]),
+                                      pack_bf16x2(k[8 * q4 + 4], k[8 * q4 + 5]), pack_bf16x2(k[8 * q4 + 6], k[8 * q4 + 7]));
         }
       }
     }
+  }
+  if (warp >= B_EW / 32) {  // the TMA and MMA warps join the two cluster barriers too
+    __syncwarp();
+    cluster_sync_all();
+    cluster_sync_all();
   }
   __syncthreads();
   if (warp == B_MMA && *abort_flag) {  // products already issued finish before TMEM is freed
@@ -810,10 +891,7 @@ int attention_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_
   NF4_TRY(tma_map_bf16(&p.tv, v, (uint64_t)nkv * 128, rows, (uint64_t)ldkv * 2, 64, TT));
   NF4_TRY(tma_map_bf16(&p.tdo, dout, (uint64_t)nq * 128, rows, (uint64_t)ldo * 2, 64, TT));
   if (!aligned(lse, 16) || !aligned(delta, 16)) return fail(NF4LS_ALIGN, "attention backward: lse / delta alignment");
-  if (!aligned(o, 16) || !aligned(dout, 16) || ldo % 8) return fail(NF4LS_ALIGN, "attention backward: O / dO rows");
-  p.o = o;
-  p.dout = dout;
-  p.ldo = ldo;
+  NF4_TRY(tma_map_bf16(&p.to, o, (uint64_t)nq * 128, rows, (uint64_t)ldo * 2, 64, TT));
   p.lse = lse;
   p.delta = delta;
   p.dq = dq;
@@ -838,7 +916,7 @@ int attention_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_
   // the query side writes delta, which the key side reads
   k_attn_dq_tc<<<dim3(seq / TT, nq, batch), B_THREADS, SMEM_BWD, s>>>(p);
   note_launch();
-  k_attn_dkv_tc<<<dim3(nkv, batch, seq / TT), B_THREADS, SMEM_BWD, s>>>(p);
+  k_attn_dkv_tc<<<dim3(2 * nkv, batch, seq / TT), B_THREADS, SMEM_BWD, s>>>(p);
   note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;

@@ -42,116 +42,98 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
                     pack_bf16x2(f[6], f[7]));
 }
 
-// ------------------------------------------------------------------ RMSNorm (one warp per row)
-__global__ void k_rmsnorm_fwd(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ w,
-                              __nv_bfloat16* __restrict__ y, int M, int H, float eps) {
-  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= M) return;
+// ------------------------------------------------------------------ RMSNorm
+// y = bf16(x r w) with r = 1 / sqrt(mean(x^2) + eps);
+// dx = resid + r w dy - x r^3 sum(w dy x) / H.
+// One block per row: VPT 16-byte vectors per thread, every
+// load of the row issued at once and the row kept in registers (one read of x and dy),
+// the block's sums added through shared memory in warp order.  Many small blocks keep
+// enough loads in flight for HBM.
+__device__ __forceinline__ float block_sum(float v, float* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  v = warp_sum(v);
+  __syncthreads();  // red may still be read from a previous sum
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float a = 0.f;
+  for (int i = 0; i < nw; ++i) a += red[i];
+  return a;
+}
+
+__device__ void pack_element(const LoraPack& a, size_t i) {
+  const int H = a.H, qd = a.qd, kvd = a.kvd, nq = qd + 2 * kvd;
+  const size_t n1 = (size_t)nq * 64, n2 = (size_t)64 * H, n3 = (size_t)16 * qd;
+  if (i < n1) {
+    const int n = (int)(i / 64), c = (int)(i % 64);
+    float v = 0.f;
+    if (n < qd && c < 16)
+      v = a.scale * __bfloat162float(__float2bfloat16_rn(a.Bq[(size_t)n * 16 + c]));
+    else if (n >= qd + kvd && c >= 16 && c < 32)
+      v = a.scale * __bfloat162float(__float2bfloat16_rn(a.Bv[(size_t)(n - qd - kvd) * 16 + c - 16]));
+    a.bup[i] = __float2bfloat16_rn(v);
+    return;
+  }
+  i -= n1;
+  if (i < n2) {
+    const int r = (int)(i / H), k = (int)(i % H);
+    float v = 0.f;
+    if (r < 16)
+      v = a.Aq[(size_t)r * H + k];
+    else if (r < 32)
+      v = a.Av[(size_t)(r - 16) * H + k];
+    a.adn[i] = __float2bfloat16_rn(v);
+    return;
+  }
+  i -= n2;
+  if (i < n3) {
+    const int r = (int)(i / qd), n = (int)(i % qd);
+    a.bqt[i] = __float2bfloat16_rn(a.Bq[(size_t)n * 16 + r]);
+    return;
+  }
+  i -= n3;
+  const int r = (int)(i / kvd), n = (int)(i % kvd);
+  a.bvt[i] = __float2bfloat16_rn(a.Bv[(size_t)n * 16 + r]);
+}
+
+__host__ __device__ inline size_t pack_elements(const LoraPack& a) {
+  return (size_t)(a.qd + 2 * a.kvd) * 64 + (size_t)64 * a.H + 16ull * a.qd + 16ull * a.kvd;
+}
+
+// Blocks [0, M): one row each.  Blocks from M on (when pack.bup is set): the adapter
+// operand conversion, grid-stride.
+template <int VPT>
+__global__ void __launch_bounds__(1024) k_rmsnorm_fwd_row(const __nv_bfloat16* __restrict__ x,
+                                                          const __nv_bfloat16* __restrict__ w,
+                                                          __nv_bfloat16* __restrict__ y, int M, int H, float eps,
+                                                          const LoraPack pack) {
+  __shared__ float red[32];
+  if ((int)blockIdx.x >= M) {
+    const size_t n = pack_elements(pack), stride = (size_t)(gridDim.x - M) * blockDim.x;
+    for (size_t i = (size_t)(blockIdx.x - M) * blockDim.x + threadIdx.x; i < n; i += stride) pack_element(pack, i);
+    return;
+  }
+  const int row = blockIdx.x, t = threadIdx.x, T = blockDim.x, nv = H / 8;
   const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)row * H);
   const uint4* wr = reinterpret_cast<const uint4*>(w);
   uint4* yr = reinterpret_cast<uint4*>(y + (size_t)row * H);
-  const int nv = H / 8;
-  float ss = 0.f;
-#pragma unroll 4
-  for (int i = lane; i < nv; i += 32) {
-    float f[8];
-    unpack8(xr[i], f);
+  uint4 v[VPT];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) ss += f[j] * f[j];
-  }
-  ss = warp_sum(ss);
-  const float r = 1.0f / sqrtf(ss / (float)H + eps);
-#pragma unroll 4
-  for (int i = lane; i < nv; i += 32) {
-    float f[8], g[8];
-    unpack8(xr[i], f);
-    unpack8(wr[i], g);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) f[j] = f[j] * r * g[j];
-    yr[i] = pack8(f);
-  }
-}
-
-// dx = resid + r w dy - x r^3 sum(w dy x) / H
-__global__ void k_rmsnorm_bwd(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ w,
-                              const __nv_bfloat16* __restrict__ dy, const __nv_bfloat16* __restrict__ resid,
-                              __nv_bfloat16* __restrict__ dx, int M, int H, float eps) {
-  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= M) return;
-  const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)row * H);
-  const uint4* wr = reinterpret_cast<const uint4*>(w);
-  const uint4* dr = reinterpret_cast<const uint4*>(dy + (size_t)row * H);
-  const uint4* rr = resid ? reinterpret_cast<const uint4*>(resid + (size_t)row * H) : nullptr;
-  uint4* out = reinterpret_cast<uint4*>(dx + (size_t)row * H);
-  const int nv = H / 8;
-  float ss = 0.f, dot = 0.f;
-#pragma unroll 4
-  for (int i = lane; i < nv; i += 32) {
-    float a[8], b[8], c[8];
-    unpack8(xr[i], a);
-    unpack8(wr[i], b);
-    unpack8(dr[i], c);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      ss += a[j] * a[j];
-      dot += b[j] * c[j] * a[j];
-    }
-  }
-  ss = warp_sum(ss);
-  dot = warp_sum(dot);
-  const float r = 1.0f / sqrtf(ss / (float)H + eps);
-  const float k = r * r * r * dot / (float)H;
-#pragma unroll 4
-  for (int i = lane; i < nv; i += 32) {
-    float a[8], b[8], c[8], e[8];
-    unpack8(xr[i], a);
-    unpack8(wr[i], b);
-    unpack8(dr[i], c);
-    if (rr)
-      unpack8(rr[i], e);
-    else
-#pragma unroll
-      for (int j = 0; j < 8; ++j) e[j] = 0.f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) e[j] += r * b[j] * c[j] - a[j] * k;
-    out[i] = pack8(e);
-  }
-}
-
-// The same two kernels with the row held in registers (MAXV 16-byte vectors per lane
-// at most): one read of each input row instead of two, and every load of a row issued
-// before the first use.  Same arithmetic, in the same order, as the kernels above.
-template <int MAXV>
-__global__ void __launch_bounds__(256) k_rmsnorm_fwd_reg(const __nv_bfloat16* __restrict__ x,
-                                                         const __nv_bfloat16* __restrict__ w,
-                                                         __nv_bfloat16* __restrict__ y, int M, int H, float eps) {
-  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= M) return;
-  const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)row * H);
-  const uint4* wr = reinterpret_cast<const uint4*>(w);
-  uint4* yr = reinterpret_cast<uint4*>(y + (size_t)row * H);
-  const int nv = H / 8;
-  uint4 v[MAXV];
-#pragma unroll
-  for (int j = 0; j < MAXV; ++j)
-    if (lane + 32 * j < nv) v[j] = xr[lane + 32 * j];
+  for (int j = 0; j < VPT; ++j)
+    if (t + j * T < nv) v[j] = xr[t + j * T];
   float ss = 0.f;
 #pragma unroll
-  for (int j = 0; j < MAXV; ++j)
-    if (lane + 32 * j < nv) {
+  for (int j = 0; j < VPT; ++j)
+    if (t + j * T < nv) {
       float f[8];
       unpack8(v[j], f);
 #pragma unroll
       for (int e = 0; e < 8; ++e) ss += f[e] * f[e];
     }
-  ss = warp_sum(ss);
+  ss = block_sum(ss, red);
   const float r = 1.0f / sqrtf(ss / (float)H + eps);
 #pragma unroll
-  for (int j = 0; j < MAXV; ++j) {
-    const int i = lane + 32 * j;
+  for (int j = 0; j < VPT; ++j) {
+    const int i = t + j * T;
     if (i < nv) {
       float f[8], g[8];
       unpack8(v[j], f);
@@ -163,35 +145,34 @@ __global__ void __launch_bounds__(256) k_rmsnorm_fwd_reg(const __nv_bfloat16* __
   }
 }
 
-template <int MAXV>
-__global__ void __launch_bounds__(256) k_rmsnorm_bwd_reg(const __nv_bfloat16* __restrict__ x,
-                                                         const __nv_bfloat16* __restrict__ w,
-                                                         const __nv_bfloat16* __restrict__ dy,
-                                                         const __nv_bfloat16* __restrict__ resid,
-                                                         __nv_bfloat16* __restrict__ dx, int M, int H, float eps) {
-  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= M) return;
+template <int VPT>
+__global__ void __launch_bounds__(1024) k_rmsnorm_bwd_row(const __nv_bfloat16* __restrict__ x,
+                                                          const __nv_bfloat16* __restrict__ w,
+                                                          const __nv_bfloat16* __restrict__ dy,
+                                                          const __nv_bfloat16* __restrict__ resid,
+                                                          __nv_bfloat16* __restrict__ dx, int H, float eps) {
+  __shared__ float red[32];
+  const int row = blockIdx.x, t = threadIdx.x, T = blockDim.x, nv = H / 8;
   const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)row * H);
   const uint4* wr = reinterpret_cast<const uint4*>(w);
   const uint4* dr = reinterpret_cast<const uint4*>(dy + (size_t)row * H);
   const uint4* rr = resid ? reinterpret_cast<const uint4*>(resid + (size_t)row * H) : nullptr;
   uint4* out = reinterpret_cast<uint4*>(dx + (size_t)row * H);
-  const int nv = H / 8;
-  uint4 xv[MAXV], dv[MAXV];
+  uint4 xv[VPT], dv[VPT], rv[VPT];
 #pragma unroll
-  for (int j = 0; j < MAXV; ++j)
-    if (lane + 32 * j < nv) {
-      xv[j] = xr[lane + 32 * j];
-      dv[j] = dr[lane + 32 * j];
+  for (int j = 0; j < VPT; ++j)
+    if (t + j * T < nv) {
+      xv[j] = xr[t + j * T];
+      dv[j] = dr[t + j * T];
+      rv[j] = rr ? rr[t + j * T] : make_uint4(0u, 0u, 0u, 0u);
     }
   float ss = 0.f, dot = 0.f;
 #pragma unroll
-  for (int j = 0; j < MAXV; ++j)
-    if (lane + 32 * j < nv) {
+  for (int j = 0; j < VPT; ++j)
+    if (t + j * T < nv) {
       float a[8], b[8], c[8];
       unpack8(xv[j], a);
-      unpack8(wr[lane + 32 * j], b);
+      unpack8(wr[t + j * T], b);
       unpack8(dv[j], c);
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
@@ -199,29 +180,28 @@ __global__ void __launch_bounds__(256) k_rmsnorm_bwd_reg(const __nv_bfloat16* __
         dot += b[e] * c[e] * a[e];
       }
     }
-  ss = warp_sum(ss);
-  dot = warp_sum(dot);
+  ss = block_sum(ss, red);
+  dot = block_sum(dot, red);
   const float r = 1.0f / sqrtf(ss / (float)H + eps);
   const float k = r * r * r * dot / (float)H;
 #pragma unroll
-  for (int j = 0; j < MAXV; ++j) {
-    const int i = lane + 32 * j;
+  for (int j = 0; j < VPT; ++j) {
+    const int i = t + j * T;
     if (i < nv) {
       float a[8], b[8], c[8], e[8];
       unpack8(xv[j], a);
       unpack8(wr[i], b);
       unpack8(dv[j], c);
-      if (rr)
-        unpack8(rr[i], e);
-      else
-#pragma unroll
-        for (int q = 0; q < 8; ++q) e[q] = 0.f;
+      unpack8(rv[j], e);
 #pragma unroll
       for (int q = 0; q < 8; ++q) e[q] += r * b[q] * c[q] - a[q] * k;
       out[i] = pack8(e);
     }
   }
 }
+
+// threads per row block: VPT vectors each, rounded up to whole warps
+inline int row_threads(int H, int vpt) { return ((H / 8 + vpt - 1) / vpt + 31) / 32 * 32; }
 
 // ------------------------------------------------------------------ RoPE
 // cos/sin of position p and frequency j, twice: [seq, d/2] (row per position) for
@@ -569,21 +549,23 @@ inline unsigned blocks_for(size_t n, int threads) { return (unsigned)((n + threa
 
 }  // namespace
 
-// Rows of up to 32 * 24 16-byte vectors (H <= 6144) are held in registers; an instance
-// per register budget: 4 vectors per lane (H <= 1024: the SmolLM2 shapes), 16 (the 8B
-// hidden size 4096), 24 (the 32B-class 5120).
+// One block per row, the row in registers: 4 vectors (32 values) per thread up to
+// H = 32768 (128 threads at H = 4096), 2 below H = 1024 (SmolLM2: 576 -> 64 threads).
 int rmsnorm_fwd(const __nv_bfloat16* x, const __nv_bfloat16* w, __nv_bfloat16* y, int M, int H, float eps,
-                cudaStream_t s) {
-  if (H % 8) return fail(NF4LS_SHAPE, "rmsnorm: H %% 8");
-  const int per_lane = (H / 8 + 31) / 32;
-  if (per_lane <= 4)
-    k_rmsnorm_fwd_reg<4><<<(M + 7) / 8, 256, 0, s>>>(x, w, y, M, H, eps);
-  else if (per_lane <= 16)
-    k_rmsnorm_fwd_reg<16><<<(M + 7) / 8, 256, 0, s>>>(x, w, y, M, H, eps);
-  else if (per_lane <= 24)
-    k_rmsnorm_fwd_reg<24><<<(M + 7) / 8, 256, 0, s>>>(x, w, y, M, H, eps);
+                cudaStream_t s, const LoraPack* pack) {
+  if (H % 8 || H > 32768) return fail(NF4LS_SHAPE, "rmsnorm: H %% 8, H <= 32768");
+  if (M <= 0) return NF4LS_OK;
+  LoraPack pk{};
+  const int threads = row_threads(H, H < 1024 ? 2 : 4);
+  int grid = M;
+  if (pack) {  // about 16 operand elements per thread of the extra blocks
+    pk = *pack;
+    grid += (int)std::min<size_t>(1024, (pack_elements(pk) + 16ull * threads - 1) / (16ull * threads));
+  }
+  if (H < 1024)
+    k_rmsnorm_fwd_row<2><<<grid, threads, 0, s>>>(x, w, y, M, H, eps, pk);
   else
-    k_rmsnorm_fwd<<<(M + 7) / 8, 256, 0, s>>>(x, w, y, M, H, eps);
+    k_rmsnorm_fwd_row<4><<<grid, threads, 0, s>>>(x, w, y, M, H, eps, pk);
   note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;
@@ -591,15 +573,12 @@ int rmsnorm_fwd(const __nv_bfloat16* x, const __nv_bfloat16* w, __nv_bfloat16* y
 
 int rmsnorm_bwd(const __nv_bfloat16* x, const __nv_bfloat16* w, const __nv_bfloat16* dy, const __nv_bfloat16* resid,
                 __nv_bfloat16* dx, int M, int H, float eps, cudaStream_t s) {
-  const int per_lane = (H / 8 + 31) / 32;
-  if (H % 8)
-    return fail(NF4LS_SHAPE, "rmsnorm_bwd: H %% 8");
-  else if (per_lane <= 4)
-    k_rmsnorm_bwd_reg<4><<<(M + 7) / 8, 256, 0, s>>>(x, w, dy, resid, dx, M, H, eps);
-  else if (per_lane <= 16)
-    k_rmsnorm_bwd_reg<16><<<(M + 7) / 8, 256, 0, s>>>(x, w, dy, resid, dx, M, H, eps);
+  if (H % 8 || H > 32768) return fail(NF4LS_SHAPE, "rmsnorm_bwd: H %% 8, H <= 32768");
+  if (M <= 0) return NF4LS_OK;
+  if (H < 1024)
+    k_rmsnorm_bwd_row<2><<<M, row_threads(H, 2), 0, s>>>(x, w, dy, resid, dx, H, eps);
   else
-    k_rmsnorm_bwd<<<(M + 7) / 8, 256, 0, s>>>(x, w, dy, resid, dx, M, H, eps);
+    k_rmsnorm_bwd_row<4><<<M, row_threads(H, 4), 0, s>>>(x, w, dy, resid, dx, H, eps);
   note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;

@@ -225,8 +225,25 @@ void profile_begin(cudaStream_t s, cudaEvent_t* e0);
 void profile_end(cudaStream_t s, cudaEvent_t e0, int kind, int detail, double flops);
 
 // ----------------------------------------------------------------------------- body kernels
+// The bf16 operands of the LoRA adapter, converted from the fp32 masters (q_proj and
+// v_proj, r = 16): bup [Nqkv, 64] (q rows: s B_q in columns 0-15; v rows: s B_v in columns
+// 16-31; else 0), adn [64, H] (rows 0-15 A_q, rows 16-31 A_v, else 0), bqt [16, qd] = B_q^T,
+// bvt [16, kvd] = B_v^T.
+struct LoraPack {
+  const float* Aq;
+  const float* Av;
+  const float* Bq;
+  const float* Bv;
+  int H, qd, kvd;
+  float scale;
+  __nv_bfloat16* bup;
+  __nv_bfloat16* adn;
+  __nv_bfloat16* bqt;
+  __nv_bfloat16* bvt;
+};
+// y = rmsnorm(x) w; with pack, the same launch also fills the adapter operands.
 int rmsnorm_fwd(const __nv_bfloat16* x, const __nv_bfloat16* w, __nv_bfloat16* y, int M, int H, float eps,
-                cudaStream_t s);
+                cudaStream_t s, const LoraPack* pack = nullptr);
 // dx = resid + rmsnorm_bwd(x, w, dy); resid may be null.
 int rmsnorm_bwd(const __nv_bfloat16* x, const __nv_bfloat16* w, const __nv_bfloat16* dy,
                 const __nv_bfloat16* resid, __nv_bfloat16* dx, int M, int H, float eps, cudaStream_t s);
@@ -255,13 +272,10 @@ int attention_bwd(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfl
                   __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv, int ld_dq, int ld_dkv, int batch,
                   int seq, int nq, int nkv, int d, cudaStream_t s);
 
-// LoRA (lora.cu).  Forward: h1 = rmsnorm(x) w, t = [h1 A_q^T | h1 A_v^T] into tpad
-// [M, 64] (bf16, zeros in columns 32-63) and the bf16 adapter operands bup [Nqkv, 64],
-// adn [64, H], bqt [16, qd], bvt [16, kvd] from the fp32 masters, in one launch.
-int norm_lora_fwd(const __nv_bfloat16* x, const __nv_bfloat16* w, __nv_bfloat16* h1, int M, int H, float eps,
-                  const nf4ls_lora* l, int qd, int kvd, float scale, __nv_bfloat16* tpad, __nv_bfloat16* bup,
-                  __nv_bfloat16* adn, __nv_bfloat16* bqt, __nv_bfloat16* bvt, cudaStream_t s);
-// Backward, two launches: dB_q, dB_v, dA_q, dA_v (fp32, written) and dt into dtpad
+// LoRA (lora.cu).  Forward: t = [h1 A_q^T | h1 A_v^T] into tpad [M, 64] (bf16, zeros in
+// columns 32-63) from h1 and adn (the bf16 A_q, A_v rows of LoraPack).
+int lora_down(const __nv_bfloat16* h1, int M, int H, const __nv_bfloat16* adn, __nv_bfloat16* tpad, cudaStream_t s);
+// Backward, three launches: dB_q, dB_v, dA_q, dA_v (fp32, written) and dt into dtpad
 // [M, 64] (bf16, zeros in columns 32-63) from dq (columns [0, qd) of dqkv) and dv
 // (columns [vcol, vcol + kvd)); part: lora_partial_bytes of scratch.
 size_t lora_partial_bytes(int M, int H, int qd, int kvd);

@@ -163,14 +163,25 @@ int forward_body(LayerCtx& x, const nf4ls_lora* lora, const __nv_bfloat16* X, __
   auto* tpad = at<__nv_bfloat16>(ws, x.L.tpad);
   GemmExtra ex;
   if (lora) {
-    // h1 and t = [h1 A_q^T | h1 A_v^T] (columns 0-31 of the padded extra operand) in one
-    // pass, with the bf16 adapter operands
-    auto* bup = at<__nv_bfloat16>(ws, x.L.bup);
-    NF4_TRY(norm_lora_fwd(X, x.v.norm_in, h1, M, H, c->rms_eps, lora, x.qd, x.kvd, x.scale, tpad, bup,
-                          at<__nv_bfloat16>(ws, x.L.adn), at<__nv_bfloat16>(ws, x.L.bqt),
-                          at<__nv_bfloat16>(ws, x.L.bvt), s));
+    // the input RMSNorm's launch also converts the adapter to its bf16 operands; then
+    // t = [h1 A_q^T | h1 A_v^T] (columns 0-31 of the padded extra operand)
+    LoraPack pk;
+    pk.Aq = lora->A_q;
+    pk.Av = lora->A_v;
+    pk.Bq = lora->B_q;
+    pk.Bv = lora->B_v;
+    pk.H = H;
+    pk.qd = x.qd;
+    pk.kvd = x.kvd;
+    pk.scale = x.scale;
+    pk.bup = at<__nv_bfloat16>(ws, x.L.bup);
+    pk.adn = at<__nv_bfloat16>(ws, x.L.adn);
+    pk.bqt = at<__nv_bfloat16>(ws, x.L.bqt);
+    pk.bvt = at<__nv_bfloat16>(ws, x.L.bvt);
+    NF4_TRY(rmsnorm_fwd(X, x.v.norm_in, h1, M, H, c->rms_eps, s, &pk));
+    NF4_TRY(lora_down(h1, M, H, pk.adn, tpad, s));
     ex.a = tpad;
-    ex.b = bup;
+    ex.b = pk.bup;
   } else {
     NF4_TRY(rmsnorm_fwd(X, x.v.norm_in, h1, M, H, c->rms_eps, s));
   }

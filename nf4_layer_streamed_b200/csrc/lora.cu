@@ -5,25 +5,22 @@
 // §2.2 check 2 (LoRA gradients nonzero in every layer): the adapter adds
 // s (x A^T) B^T to the q and v projections (s = alpha / r) and trains A and B.  The
 // up-projection is folded into the q/k/v GEMM as an extra 64-wide reduction block;
-// this file holds the skinny products around it, all of them HBM-bound, in three
-// launches per layer and step direction:
+// this file holds the skinny products around it, all of them HBM-bound, in one launch
+// per forward and three per backward:
 //
-//   forward (k_norm_lora_fwd, one launch):
-//     h1 = rmsnorm(x) w_in and t = [h1 A_q^T | h1 A_v^T] in one pass over x, plus the
-//     bf16 operands of the adapter (s B_q, s B_v for the up-projection block, A_q, A_v
-//     for the dL/dx block, B_q^T, B_v^T for dt) converted from the fp32 masters;
-//   backward (two launches):
-//     k_lora_bwd_partial: per (128-row block, column chunk of dq or dv) the partial
-//       sums of dB = s dX^T t (over the rows) and of dt = s dX B (over the columns),
-//       from one read of dX;
-//     k_lora_bwd_final: dB (partials added in row-block order); dt (partials added in
-//       column-chunk order, rounded to bf16: the extra operand of the dL/dx GEMM); the
-//       partial sums of dA = dt^T h1 per (128-row group, column chunk of h1), which the
-//       last block of each column chunk to finish adds in row-group order.
+//   k_lora_down: t = [h1 A_q^T | h1 A_v^T] (bf16, the extra operand of the q/k/v GEMM)
+//     from h1 and the bf16 adapter rows, which the input RMSNorm's launch converts
+//     from the fp32 masters together with the other adapter operands (body.cu);
+//   k_lora_bwd_partial: per (128-row block, column chunk of dq or dv) the partial sums
+//     of dB = s dX^T t (over the rows) and of dt = s dX B (over the columns), from one
+//     read of dX;
+//   k_lora_bwd_reduce: dB (partials added in row-block order) and dt (partials added
+//     in column-chunk order, rounded to bf16: the extra operand of the dL/dx GEMM);
+//   k_lora_bwd_da: dA = dt^T h1, one block per 32 columns of h1 over all rows.
 //
 // The products run on the warp-level bf16 tensor-core instruction (mma.sync m16n8k16);
 // every reduction is in a fixed order, so each result is bit-reproducible and a
-// token's row results (h1, t, dt) do not depend on how many tokens share the launch.
+// token's row results (t, dt) do not depend on how many tokens share the launch.
 #include <algorithm>
 #include <mutex>
 #include <utility>
@@ -58,141 +55,74 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
 __device__ __forceinline__ void zero16(uint32_t addr) { st_shared_v4(addr, 0u, 0u, 0u, 0u); }
 
 // ============================================================================ forward
-constexpr int NL_ROWS = 16, NL_THREADS = 256, NL_WARPS = 8;
+constexpr int LD_ROWS = 16, LD_THREADS = 256, LD_WARPS = 8, LD_KC = 128;  // rows per block, k-chunk
+constexpr int LD_LS = LD_KC + 8;                                         // smem row stride (elements)
+constexpr int LD_STAGES = 4;
+constexpr int LD_STAGE_BYTES = (LD_ROWS + 32) * LD_LS * 2;
+constexpr int LD_SMEM = LD_STAGES * LD_STAGE_BYTES;
 
-struct NormLoraArgs {
-  const __nv_bfloat16* x;
-  const __nv_bfloat16* w;
-  __nv_bfloat16* h1;
-  int M, H;
-  float eps;
-  const float* Aq;  // [16, H] fp32 masters
-  const float* Av;
-  const float* Bq;  // [qd, 16]
-  const float* Bv;  // [kvd, 16]
-  __nv_bfloat16* tpad;  // [M, 64]: t_q in columns 0-15, t_v in 16-31, zeros in 32-63
-  int qd, kvd;
-  float scale;
-  // bf16 adapter operands:
-  //   bup [Nqkv, 64]: q rows: s B_q in columns 0-15; v rows: s B_v in columns 16-31; else 0
-  //   adn [64, H]   : rows 0-15 A_q, rows 16-31 A_v, else 0
-  //   bqt [16, qd] = B_q^T, bvt [16, kvd] = B_v^T
-  __nv_bfloat16* bup;
-  __nv_bfloat16* adn;
-  __nv_bfloat16* bqt;
-  __nv_bfloat16* bvt;
-};
-
-__device__ void pack_element(const NormLoraArgs& a, size_t i) {
-  const int H = a.H, qd = a.qd, kvd = a.kvd, nq = qd + 2 * kvd;
-  const size_t n1 = (size_t)nq * 64, n2 = (size_t)64 * H, n3 = (size_t)16 * qd;
-  if (i < n1) {
-    const int n = (int)(i / 64), c = (int)(i % 64);
-    float v = 0.f;
-    if (n < qd && c < 16)
-      v = a.scale * __bfloat162float(__float2bfloat16_rn(a.Bq[(size_t)n * 16 + c]));
-    else if (n >= qd + kvd && c >= 16 && c < 32)
-      v = a.scale * __bfloat162float(__float2bfloat16_rn(a.Bv[(size_t)(n - qd - kvd) * 16 + c - 16]));
-    a.bup[i] = __float2bfloat16_rn(v);
-    return;
-  }
-  i -= n1;
-  if (i < n2) {
-    const int r = (int)(i / H), k = (int)(i % H);
-    float v = 0.f;
-    if (r < 16)
-      v = a.Aq[(size_t)r * H + k];
-    else if (r < 32)
-      v = a.Av[(size_t)(r - 16) * H + k];
-    a.adn[i] = __float2bfloat16_rn(v);
-    return;
-  }
-  i -= n2;
-  if (i < n3) {
-    const int r = (int)(i / qd), n = (int)(i % qd);
-    a.bqt[i] = __float2bfloat16_rn(a.Bq[(size_t)n * 16 + r]);
-    return;
-  }
-  i -= n3;
-  const int r = (int)(i / kvd), n = (int)(i % kvd);
-  a.bvt[i] = __float2bfloat16_rn(a.Bv[(size_t)n * 16 + r]);
-}
-
-// One block: 16 token rows.  Warp w normalises rows 2w and 2w + 1 (the row held in
-// registers, MAXV 16-byte vectors per lane at most), writes h1 and keeps the bf16 row in
-// shared memory; then each warp multiplies the 16 rows by the 32 adapter rows over the
-// 16-wide k-steps w, w + 8, ... (A fragments by ldmatrix, B fragments converted from the
-// fp32 masters), and the eight partial products are added in warp order.  The block's
-// share of the operand conversion follows.
-template <int MAXV>
-__global__ void __launch_bounds__(NL_THREADS) k_norm_lora_fwd(const __grid_constant__ NormLoraArgs a) {
+// One block: 16 token rows.  The reduction over H runs in chunks of 128 columns through a
+// ring of LD_STAGES shared-memory stages filled by cp.async: the h1 rows and the 32 bf16
+// adapter rows (A_q, A_v of adn).  Warp w takes the chunk's k-step w, so it accumulates
+// the global k-steps w, w + 8, ...; the eight partial products are then added in warp
+// order.
+__global__ void __launch_bounds__(LD_THREADS) k_lora_down(const __nv_bfloat16* __restrict__ h1, int M, int H,
+                                                          const __nv_bfloat16* __restrict__ adn,
+                                                          __nv_bfloat16* __restrict__ tpad) {
   extern __shared__ __align__(16) uint8_t smem[];
-  const int H = a.H, ld = H + 8, nv = H / 8;
-  __nv_bfloat16* tile = reinterpret_cast<__nv_bfloat16*>(smem);
-  float* red = reinterpret_cast<float*>(smem + (size_t)NL_ROWS * ld * 2);  // [8][16][32]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * NL_ROWS;
-
-  for (int rr = 0; rr < 2; ++rr) {
-    const int r = warp * 2 + rr, m = m0 + r;
-    uint4* trow = reinterpret_cast<uint4*>(tile + (size_t)r * ld);
-    if (m >= a.M) {
-      for (int i = lane; i < nv; i += 32) trow[i] = make_uint4(0u, 0u, 0u, 0u);
-      continue;
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31, g4 = lane >> 2, t4 = lane & 3;
+  const int m0 = blockIdx.x * LD_ROWS;
+  const int n_chunks = (H + LD_KC - 1) / LD_KC;
+  auto tile = [&](int b) { return reinterpret_cast<__nv_bfloat16*>(smem + (size_t)b * LD_STAGE_BYTES); };
+  // chunk c into stage b: rows 0-15 h1, rows 16-47 adapter rows 0-31 (16 pieces each)
+  auto stage = [&](int c, int b) {
+    for (int e = t; e < (LD_ROWS + 32) * 16; e += LD_THREADS) {
+      const int r = e >> 4, q = e & 15, col = c * LD_KC + q * 8;
+      const uint32_t dst = smem_u32(tile(b) + r * LD_LS + q * 8);
+      const int m = m0 + r;
+      if (col >= H || (r < LD_ROWS && m >= M))
+        zero16(dst);
+      else if (r < LD_ROWS)
+        cp_async16(dst, h1 + (size_t)m * H + col);
+      else
+        cp_async16(dst, adn + (size_t)(r - LD_ROWS) * H + col);
     }
-    const uint4* xr = reinterpret_cast<const uint4*>(a.x + (size_t)m * H);
-    uint4 v[MAXV];
-#pragma unroll
-    for (int j = 0; j < MAXV; ++j)
-      if (lane + 32 * j < nv) v[j] = xr[lane + 32 * j];
-    float ss = 0.f;
-#pragma unroll
-    for (int j = 0; j < MAXV; ++j)
-      if (lane + 32 * j < nv) {
-        float f[8];
-        unpack8(v[j], f);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) ss += f[e] * f[e];
-      }
-    ss = warp_sum(ss);
-    const float rs = 1.0f / sqrtf(ss / (float)H + a.eps);
-    const uint4* wr = reinterpret_cast<const uint4*>(a.w);
-    uint4* yr = reinterpret_cast<uint4*>(a.h1 + (size_t)m * H);
-#pragma unroll
-    for (int j = 0; j < MAXV; ++j) {
-      const int i = lane + 32 * j;
-      if (i < nv) {
-        float f[8], g[8];
-        unpack8(v[j], f);
-        unpack8(wr[i], g);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] = f[e] * rs * g[e];
-        const uint4 o = pack8(f);
-        yr[i] = o;
-        trow[i] = o;
-      }
-    }
-  }
-  __syncthreads();
-
-  // t = h1 [A_q; A_v]^T: 16 rows x 32 outputs
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
   float acc[4][4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-  const uint32_t st = smem_u32(tile);
-  const int g4 = lane >> 2, t4 = lane & 3;
-  for (int ks = warp; ks < H / 16; ks += NL_WARPS) {
-    uint32_t a0, a1, a2, a3;
-    ldsm4(st + ((lane & 15) * ld + ks * 16 + (lane >> 4) * 8) * 2, a0, a1, a2, a3);
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
-      const float* A = (nt < 2 ? a.Aq : a.Av) + (size_t)((nt & 1) * 8 + g4) * H + ks * 16 + 2 * t4;
-      const float2 lo = *reinterpret_cast<const float2*>(A);
-      const float2 hi = *reinterpret_cast<const float2*>(A + 8);
-      mma16816(acc[nt], a0, a1, a2, a3, pack_bf16x2(lo.x, lo.y), pack_bf16x2(hi.x, hi.y));
+  for (int c = 0; c < LD_STAGES - 1; ++c) {
+    if (c < n_chunks)
+      stage(c, c);
+    else
+      asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+  for (int c = 0; c < n_chunks; ++c) {
+    const int b = c % LD_STAGES;
+    asm volatile("cp.async.wait_group %0;" ::"n"(LD_STAGES - 2) : "memory");
+    __syncthreads();  // chunk c has landed for every thread; the stage of chunk c - 1 is free
+    if (c + LD_STAGES - 1 < n_chunks)
+      stage(c + LD_STAGES - 1, (c + LD_STAGES - 1) % LD_STAGES);
+    else
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    if (c * LD_KC + warp * 16 < H) {
+      const __nv_bfloat16* T = tile(b);
+      uint32_t a0, a1, a2, a3, b0, b1, b2, b3, b4, b5, b6, b7;
+      ldsm4(smem_u32(T + (lane & 15) * LD_LS + warp * 16 + (lane >> 4) * 8), a0, a1, a2, a3);
+      const int br = (lane & 7) + (lane >> 4) * 8, bc = warp * 16 + ((lane >> 3) & 1) * 8;
+      ldsm4(smem_u32(T + (LD_ROWS + br) * LD_LS + bc), b0, b1, b2, b3);
+      ldsm4(smem_u32(T + (LD_ROWS + 16 + br) * LD_LS + bc), b4, b5, b6, b7);
+      mma16816(acc[0], a0, a1, a2, a3, b0, b1);
+      mma16816(acc[1], a0, a1, a2, a3, b2, b3);
+      mma16816(acc[2], a0, a1, a2, a3, b4, b5);
+      mma16816(acc[3], a0, a1, a2, a3, b6, b7);
     }
   }
-  float* R = red + warp * (NL_ROWS * 32);
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  __syncthreads();
+  float* red = reinterpret_cast<float*>(smem);  // the stages are free now
+  float* R = red + warp * (LD_ROWS * 32);
 #pragma unroll
   for (int nt = 0; nt < 4; ++nt) {
     R[g4 * 32 + nt * 8 + 2 * t4] = acc[nt][0];
@@ -201,20 +131,14 @@ __global__ void __launch_bounds__(NL_THREADS) k_norm_lora_fwd(const __grid_const
     R[(g4 + 8) * 32 + nt * 8 + 2 * t4 + 1] = acc[nt][3];
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < NL_ROWS * 64; e += NL_THREADS) {
-    const int r = e >> 6, c = e & 63, m = m0 + r;
-    if (m >= a.M) continue;
+  for (int e = t; e < LD_ROWS * 64; e += LD_THREADS) {
+    const int r = e >> 6, cc = e & 63, m = m0 + r;
+    if (m >= M) continue;
     float v = 0.f;
-    if (c < 32)
-      for (int w = 0; w < NL_WARPS; ++w) v += red[w * (NL_ROWS * 32) + r * 32 + c];
-    a.tpad[(size_t)m * 64 + c] = __float2bfloat16_rn(v);
+    if (cc < 32)
+      for (int w = 0; w < LD_WARPS; ++w) v += red[w * (LD_ROWS * 32) + r * 32 + cc];
+    tpad[(size_t)m * 64 + cc] = __float2bfloat16_rn(v);
   }
-
-  // this block's share of the bf16 adapter operands
-  const size_t total = (size_t)(a.qd + 2 * a.kvd) * 64 + (size_t)64 * H + 16ull * a.qd + 16ull * a.kvd;
-  const size_t per = (total + gridDim.x - 1) / gridDim.x;
-  const size_t b0 = (size_t)blockIdx.x * per, b1 = min(total, b0 + per);
-  for (size_t i = b0 + threadIdx.x; i < b1; i += NL_THREADS) pack_element(a, i);
 }
 
 // ============================================================================ backward
@@ -229,11 +153,9 @@ struct LoraBwdArgs {
   const __nv_bfloat16* bvt;   // [16, kvd] = B_v^T
   float* part_dB;             // [n_rb][qd + kvd][16]
   float* part_dt;             // [n_cc][M][16]
-  int* counters;              // [n_hc]
-  int n_rb, n_rg, HC, n_hc, n_db_blocks;
+  int n_rb, n_db_blocks;
   const __nv_bfloat16* h1;    // [M, H]
   __nv_bfloat16* dtpad;       // [M, 64]: dt_q in 0-15, dt_v in 16-31, zeros in 32-63
-  float* part_dA;             // [n_rg][32][H]
   float scale;
   float* dA_q;                // [16, H]
   float* dB_q;                // [qd, 16]
@@ -252,8 +174,6 @@ __global__ void __launch_bounds__(LB_THREADS) k_lora_bwd_partial(const __grid_co
   __nv_bfloat16* bs = ts + LB_ROWS * 24;                             // [16][CW + 8]
   const int rb = blockIdx.x, cc = blockIdx.y;
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31, g4 = lane >> 2, t4 = lane & 3;
-  if (rb == 0 && cc == 0)
-    for (int i = t; i < a.n_hc; i += LB_THREADS) a.counters[i] = 0;  // for k_lora_bwd_final
   const bool is_v = cc >= a.n_cc_q;
   const int c0 = cc * CW;                                   // column in [dq | dv]
   const int seg_col = is_v ? c0 - a.qd : c0;                // column within dq or dv
@@ -346,13 +266,9 @@ __global__ void __launch_bounds__(LB_THREADS) k_lora_bwd_partial(const __grid_co
 }
 
 // Blocks [0, n_db_blocks): dB, one element per thread, the row-block partials added in
-// order.  The others, per (row group rg of 128 rows, column chunk hc of HC columns of
-// h1): dt of the group's rows (column-chunk partials added in order, times s, rounded
-// to bf16; the hc = 0 blocks also store it as the dL/dx GEMM's extra operand), then the
-// partial dA = dt^T h1 over the group's rows; the last of the n_rg blocks of a chunk to
-// finish adds the partials in row-group order.
-__global__ void __launch_bounds__(LB_THREADS) k_lora_bwd_final(const __grid_constant__ LoraBwdArgs a) {
-  extern __shared__ __align__(16) uint8_t smem[];
+// order.  The others: dt of 8 rows per block (one row per warp, column-chunk partials
+// added in order, times s, rounded to bf16) into dtpad, zeros in its columns 32-63.
+__global__ void __launch_bounds__(LB_THREADS) k_lora_bwd_reduce(const __grid_constant__ LoraBwdArgs a) {
   const int t = threadIdx.x;
   const int NB = a.qd + a.kvd;
   if ((int)blockIdx.x < a.n_db_blocks) {
@@ -368,101 +284,122 @@ __global__ void __launch_bounds__(LB_THREADS) k_lora_bwd_final(const __grid_cons
       a.dB_v[(size_t)(col - a.qd) * 16 + r] = v;
     return;
   }
-  const int b = blockIdx.x - a.n_db_blocks;
-  const int rg = b / a.n_hc, hc = b % a.n_hc;
-  const int HC = a.HC, lh = HC + 8, m0 = rg * LB_ROWS;
-  __nv_bfloat16* dts = reinterpret_cast<__nv_bfloat16*>(smem);  // [128][40]
-  __nv_bfloat16* hs = dts + LB_ROWS * 40;                        // [128][HC + 8]
-  __shared__ int last;
-  const uint32_t sd = smem_u32(dts), sh = smem_u32(hs);
-  const int cpr = HC / 8;
-  for (int i = t; i < LB_ROWS * cpr; i += LB_THREADS) {
-    const int r = i / cpr, c = i % cpr, m = m0 + r;
-    const uint32_t dst = sh + (r * lh + c * 8) * 2;
-    if (m < a.M)
-      cp_async16(dst, a.h1 + (size_t)m * a.H + hc * HC + c * 8);
-    else
-      zero16(dst);
-  }
-  for (int e = t; e < LB_ROWS * 64; e += LB_THREADS) {
-    const int r = e >> 6, c = e & 63, m = m0 + r;
-    float v = 0.f;
-    if (m < a.M && c < 32) {
-      const int cb = c < 16 ? 0 : a.n_cc_q, ce = c < 16 ? a.n_cc_q : a.n_cc;
-      for (int k = cb; k < ce; ++k) v += a.part_dt[((size_t)k * a.M + m) * 16 + (c & 15)];
-      v *= a.scale;
-    }
-    const __nv_bfloat16 bv = __float2bfloat16_rn(v);
-    if (c < 32) dts[r * 40 + c] = bv;
-    if (hc == 0 && m < a.M) a.dtpad[(size_t)m * 64 + c] = bv;
-  }
-  cp_async_wait_all();
-  __syncthreads();
+  const int m = ((int)blockIdx.x - a.n_db_blocks) * 8 + (t >> 5), c = t & 31;
+  if (m >= a.M) return;
+  const int cb = c < 16 ? 0 : a.n_cc_q, ce = c < 16 ? a.n_cc_q : a.n_cc;
+  float v = 0.f;
+  for (int k = cb; k < ce; ++k) v += a.part_dt[((size_t)k * a.M + m) * 16 + (c & 15)];
+  a.dtpad[(size_t)m * 64 + c] = __float2bfloat16_rn(v * a.scale);
+  a.dtpad[(size_t)m * 64 + 32 + c] = __float2bfloat16_rn(0.f);
+}
 
-  // partial dA: D[32 x HC] = dt^T [32 x 128] h1 [128 x HC]; warp w takes the 16-column
-  // groups w, w + 8, ... for both 16-row halves (q, v)
-  const int warp = t >> 5, lane = t & 31, g4 = lane >> 2, t4 = lane & 3;
-  for (int grp = warp; grp < HC / 16; grp += 8) {
-    float acc[2][2][4];
+// dA = dt^T h1: one block per 64 columns of h1, over all M rows in chunks of 128 through
+// a ring of DA_STAGES cp.async stages.  Warp w takes the chunk's k-step w (16 rows), so it
+// accumulates the rows 16 w .. of every chunk; the eight partial products are added in
+// warp order.
+constexpr int DA_COLS = 64, DA_ROWS = 128, DA_DS = 40, DA_HS = DA_COLS + 8, DA_STAGES = 4;
+constexpr int DA_PIECES = 4 + DA_COLS / 8;  // 16-byte pieces per row: dt (32 columns), h1
+constexpr int DA_STAGE_BYTES = DA_ROWS * (DA_DS + DA_HS) * 2;
+constexpr int DA_SMEM = DA_STAGES * DA_STAGE_BYTES;
+
+__global__ void __launch_bounds__(LB_THREADS) k_lora_bwd_da(const __grid_constant__ LoraBwdArgs a) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31, g4 = lane >> 2, t4 = lane & 3;
+  const int c0 = blockIdx.x * DA_COLS;
+  const int n_chunks = (a.M + DA_ROWS - 1) / DA_ROWS;
+  auto ds = [&](int b) { return reinterpret_cast<__nv_bfloat16*>(smem + (size_t)b * DA_STAGE_BYTES); };
+  auto hs = [&](int b) {
+    return reinterpret_cast<__nv_bfloat16*>(smem + (size_t)b * DA_STAGE_BYTES + DA_ROWS * DA_DS * 2);
+  };
+  auto stage = [&](int ch, int b) {  // 128 rows x (4 pieces of dt + DA_COLS / 8 pieces of h1)
+    for (int i = t; i < DA_ROWS * DA_PIECES; i += LB_THREADS) {
+      const int r = i / DA_PIECES, q = i % DA_PIECES, m = ch * DA_ROWS + r;
+      const uint32_t dst = q < 4 ? smem_u32(ds(b) + r * DA_DS + q * 8) : smem_u32(hs(b) + r * DA_HS + (q - 4) * 8);
+      if (m >= a.M)
+        zero16(dst);
+      else if (q < 4)
+        cp_async16(dst, a.dtpad + (size_t)m * 64 + q * 8);
+      else
+        cp_async16(dst, a.h1 + (size_t)m * a.H + c0 + (q - 4) * 8);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  constexpr int NT = DA_COLS / 8;  // n8 tiles of the block's columns
+  float acc[2][NT][4];
 #pragma unroll
-    for (int i = 0; i < 2; ++i)
+  for (int i = 0; i < 2; ++i)
 #pragma unroll
-      for (int j = 0; j < 2; ++j) acc[i][j][0] = acc[i][j][1] = acc[i][j][2] = acc[i][j][3] = 0.f;
+    for (int j = 0; j < NT; ++j) acc[i][j][0] = acc[i][j][1] = acc[i][j][2] = acc[i][j][3] = 0.f;
+  for (int ch = 0; ch < DA_STAGES - 1; ++ch) {
+    if (ch < n_chunks)
+      stage(ch, ch);
+    else
+      asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+  for (int ch = 0; ch < n_chunks; ++ch) {
+    const int b = ch % DA_STAGES;
+    asm volatile("cp.async.wait_group %0;" ::"n"(DA_STAGES - 2) : "memory");
+    __syncthreads();  // chunk ch has landed; the stage of chunk ch - 1 is free
+    if (ch + DA_STAGES - 1 < n_chunks)
+      stage(ch + DA_STAGES - 1, (ch + DA_STAGES - 1) % DA_STAGES);
+    else
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    const int kr = warp * 16;  // this warp's 16 rows of the chunk
+    uint32_t af[2][4];
 #pragma unroll
-    for (int kk = 0; kk < LB_ROWS / 16; ++kk) {
+    for (int mt = 0; mt < 2; ++mt) {  // dA rows 16 mt ..: A = dt^T from the dt rows
+      const int m = kr + (lane & 7) + (lane >> 4) * 8, n = mt * 16 + ((lane >> 3) & 1) * 8;
+      ldsm4t(smem_u32(ds(b) + m * DA_DS + n), af[mt][0], af[mt][1], af[mt][2], af[mt][3]);
+    }
+#pragma unroll
+    for (int h = 0; h < NT / 2; ++h) {  // h1 columns 16 h ..: B fragments of two n8 tiles
       uint32_t b0, b1, b2, b3;
-      {
-        const int m = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8, n = grp * 16 + (lane >> 4) * 8;
-        ldsm4t(sh + (m * lh + n) * 2, b0, b1, b2, b3);
-      }
+      const int m = kr + (lane & 7) + ((lane >> 3) & 1) * 8, n = h * 16 + (lane >> 4) * 8;
+      ldsm4t(smem_u32(hs(b) + m * DA_HS + n), b0, b1, b2, b3);
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt) {
-        uint32_t a0, a1, a2, a3;
-        const int m = kk * 16 + (lane & 7) + (lane >> 4) * 8, n = mt * 16 + ((lane >> 3) & 1) * 8;
-        ldsm4t(sd + (m * 40 + n) * 2, a0, a1, a2, a3);
-        mma16816(acc[mt][0], a0, a1, a2, a3, b0, b1);
-        mma16816(acc[mt][1], a0, a1, a2, a3, b2, b3);
+        mma16816(acc[mt][2 * h], af[mt][0], af[mt][1], af[mt][2], af[mt][3], b0, b1);
+        mma16816(acc[mt][2 * h + 1], af[mt][0], af[mt][1], af[mt][2], af[mt][3], b2, b3);
       }
     }
-    float* P = a.part_dA + (size_t)rg * 32 * a.H + hc * HC + grp * 16;
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        const int row = mt * 16 + g4, col = nt * 8 + 2 * t4;
-        P[(size_t)row * a.H + col] = acc[mt][nt][0];
-        P[(size_t)row * a.H + col + 1] = acc[mt][nt][1];
-        P[(size_t)(row + 8) * a.H + col] = acc[mt][nt][2];
-        P[(size_t)(row + 8) * a.H + col + 1] = acc[mt][nt][3];
-      }
   }
-  __threadfence();
+  asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
-  if (t == 0) last = atomicAdd(&a.counters[hc], 1) == a.n_rg - 1;
+  float* red = reinterpret_cast<float*>(smem);  // the stages are free now
+  float* R = red + warp * (32 * DA_COLS);
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int row = mt * 16 + g4, col = nt * 8 + 2 * t4;
+      R[row * DA_COLS + col] = acc[mt][nt][0];
+      R[row * DA_COLS + col + 1] = acc[mt][nt][1];
+      R[(row + 8) * DA_COLS + col] = acc[mt][nt][2];
+      R[(row + 8) * DA_COLS + col + 1] = acc[mt][nt][3];
+    }
   __syncthreads();
-  if (!last) return;
-  __threadfence();
-  for (int e = t; e < 32 * HC; e += LB_THREADS) {
-    const int row = e / HC, col = hc * HC + e % HC;
+  for (int e = t; e < 32 * DA_COLS; e += LB_THREADS) {
+    const int row = e / DA_COLS, col = c0 + e % DA_COLS;
     float v = 0.f;
-    for (int g = 0; g < a.n_rg; ++g) v += __ldcg(a.part_dA + ((size_t)g * 32 + row) * a.H + col);
+    for (int w = 0; w < 8; ++w) v += red[w * (32 * DA_COLS) + e];
     if (row < 16)
       a.dA_q[(size_t)row * a.H + col] = v;
     else
       a.dA_v[(size_t)(row - 16) * a.H + col] = v;
   }
-  if (t == 0) a.counters[hc] = 0;
 }
 
+// Column chunk of k_lora_bwd_partial: 128 where it divides both widths (so that a
+// 2048-token batch of the 8B layer runs 16 x 40 blocks, several per SM), else 64.
 int chunk_width(int a, int b) {
-  for (int w : {256, 192, 128, 64})
+  for (int w : {128, 64})
     if (a % w == 0 && b % w == 0) return w;
   return 0;
 }
 
 struct BwdShape {
-  int CW, n_cc_q, n_cc, n_rb, n_rg, HC, n_hc, n_db_blocks;
-  size_t part_dB, part_dt, part_dA, counters, total;
+  int CW, n_cc_q, n_cc, n_rb, n_db_blocks;
+  size_t part_dB, part_dt, total;
 };
 
 BwdShape bwd_shape(int M, int H, int qd, int kvd) {
@@ -471,9 +408,6 @@ BwdShape bwd_shape(int M, int H, int qd, int kvd) {
   b.n_cc_q = b.CW ? qd / b.CW : 0;
   b.n_cc = b.CW ? (qd + kvd) / b.CW : 0;
   b.n_rb = (M + LB_ROWS - 1) / LB_ROWS;
-  b.n_rg = b.n_rb;
-  b.HC = chunk_width(H, H);
-  b.n_hc = b.HC ? H / b.HC : 0;
   b.n_db_blocks = ((qd + kvd) * 16 + LB_THREADS - 1) / LB_THREADS;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -483,8 +417,6 @@ BwdShape bwd_shape(int M, int H, int qd, int kvd) {
   };
   b.part_dB = take((size_t)b.n_rb * (qd + kvd) * 16 * 4);
   b.part_dt = take((size_t)b.n_cc * M * 16 * 4);
-  b.part_dA = take((size_t)b.n_rg * 32 * H * 4);
-  b.counters = take((size_t)std::max(b.n_hc, 1) * 4);
   b.total = off;
   return b;
 }
@@ -514,43 +446,12 @@ int allow_smem(const void* kernel, size_t bytes) {
 
 size_t lora_partial_bytes(int M, int H, int qd, int kvd) { return bwd_shape(M, H, qd, kvd).total; }
 
-int norm_lora_fwd(const __nv_bfloat16* x, const __nv_bfloat16* w, __nv_bfloat16* h1, int M, int H, float eps,
-                  const nf4ls_lora* l, int qd, int kvd, float scale, __nv_bfloat16* tpad, __nv_bfloat16* bup,
-                  __nv_bfloat16* adn, __nv_bfloat16* bqt, __nv_bfloat16* bvt, cudaStream_t s) {
-  if (H % 16 || H > 32 * 24 * 8 || qd % 8 || kvd % 8) return fail(NF4LS_SHAPE, "norm_lora_fwd: H %d", H);
-  NormLoraArgs a;
-  a.x = x;
-  a.w = w;
-  a.h1 = h1;
-  a.M = M;
-  a.H = H;
-  a.eps = eps;
-  a.Aq = l->A_q;
-  a.Av = l->A_v;
-  a.Bq = l->B_q;
-  a.Bv = l->B_v;
-  a.tpad = tpad;
-  a.qd = qd;
-  a.kvd = kvd;
-  a.scale = scale;
-  a.bup = bup;
-  a.adn = adn;
-  a.bqt = bqt;
-  a.bvt = bvt;
-  const size_t smem = (size_t)NL_ROWS * (H + 8) * 2 + (size_t)NL_WARPS * NL_ROWS * 32 * 4;
-  const int grid = (M + NL_ROWS - 1) / NL_ROWS;
-  const int per_lane = (H / 8 + 31) / 32;
-  // one instance per register budget of the row: SmolLM2 (576: 3), 8B (4096: 16), 32B (5120: 20)
-  if (per_lane <= 4) {
-    NF4_TRY(allow_smem((const void*)k_norm_lora_fwd<4>, smem));
-    k_norm_lora_fwd<4><<<grid, NL_THREADS, smem, s>>>(a);
-  } else if (per_lane <= 16) {
-    NF4_TRY(allow_smem((const void*)k_norm_lora_fwd<16>, smem));
-    k_norm_lora_fwd<16><<<grid, NL_THREADS, smem, s>>>(a);
-  } else {
-    NF4_TRY(allow_smem((const void*)k_norm_lora_fwd<24>, smem));
-    k_norm_lora_fwd<24><<<grid, NL_THREADS, smem, s>>>(a);
-  }
+int lora_down(const __nv_bfloat16* h1, int M, int H, const __nv_bfloat16* adn, __nv_bfloat16* tpad, cudaStream_t s) {
+  if (H % 16) return fail(NF4LS_SHAPE, "lora_down: H %d", H);
+  if (M <= 0) return NF4LS_OK;
+  static_assert(LD_WARPS * LD_ROWS * 32 * 4 <= LD_SMEM, "partials fit in the stages");
+  NF4_TRY(allow_smem((const void*)k_lora_down, LD_SMEM));
+  k_lora_down<<<(M + LD_ROWS - 1) / LD_ROWS, LD_THREADS, LD_SMEM, s>>>(h1, M, H, adn, tpad);
   note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;
@@ -560,7 +461,9 @@ int lora_bwd(const __nv_bfloat16* dqkv, int ld, int vcol, int M, int H, int qd, 
              const __nv_bfloat16* bqt, const __nv_bfloat16* bvt, const __nv_bfloat16* h1, float scale,
              __nv_bfloat16* dtpad, const nf4ls_lora_grads* g, void* part, cudaStream_t s) {
   const BwdShape sh = bwd_shape(M, H, qd, kvd);
-  if (!sh.CW || !sh.HC || ld % 8 || vcol % 8) return fail(NF4LS_SHAPE, "lora_bwd: qd %d, kvd %d, H %d", qd, kvd, H);
+  if (!sh.CW || H % DA_COLS || ld % 8 || vcol % 8)
+    return fail(NF4LS_SHAPE, "lora_bwd: qd %d, kvd %d, H %d", qd, kvd, H);
+  if (M <= 0) return NF4LS_OK;
   LoraBwdArgs a;
   a.dqkv = dqkv;
   a.ld = ld;
@@ -578,12 +481,7 @@ int lora_bwd(const __nv_bfloat16* dqkv, int ld, int vcol, int M, int H, int qd, 
   uint8_t* pb = static_cast<uint8_t*>(part);
   a.part_dB = reinterpret_cast<float*>(pb + sh.part_dB);
   a.part_dt = reinterpret_cast<float*>(pb + sh.part_dt);
-  a.part_dA = reinterpret_cast<float*>(pb + sh.part_dA);
-  a.counters = reinterpret_cast<int*>(pb + sh.counters);
   a.n_rb = sh.n_rb;
-  a.n_rg = sh.n_rg;
-  a.HC = sh.HC;
-  a.n_hc = sh.n_hc;
   a.n_db_blocks = sh.n_db_blocks;
   a.h1 = h1;
   a.dtpad = dtpad;
@@ -596,10 +494,11 @@ int lora_bwd(const __nv_bfloat16* dqkv, int ld, int vcol, int M, int H, int qd, 
   NF4_TRY(allow_smem((const void*)k_lora_bwd_partial, smem1));
   k_lora_bwd_partial<<<dim3(sh.n_rb, sh.n_cc), LB_THREADS, smem1, s>>>(a);
   note_launch();
-  NF4_CUDA_TRY(cudaGetLastError());
-  const size_t smem2 = (size_t)LB_ROWS * 40 * 2 + (size_t)LB_ROWS * (sh.HC + 8) * 2;
-  NF4_TRY(allow_smem((const void*)k_lora_bwd_final, smem2));
-  k_lora_bwd_final<<<sh.n_db_blocks + sh.n_rg * sh.n_hc, LB_THREADS, smem2, s>>>(a);
+  k_lora_bwd_reduce<<<sh.n_db_blocks + (M + 7) / 8, LB_THREADS, 0, s>>>(a);
+  note_launch();
+  static_assert(8 * 32 * DA_COLS * 4 <= DA_SMEM, "partials fit in the stages");
+  NF4_TRY(allow_smem((const void*)k_lora_bwd_da, DA_SMEM));
+  k_lora_bwd_da<<<H / DA_COLS, LB_THREADS, DA_SMEM, s>>>(a);
   note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;

@@ -10,7 +10,8 @@ product out = x W^T and the dL/dx product out = dy W.
     python -m nf4_layer_streamed_b200.gemm_bench [--M 2048] [--shapes gateup,down] [--iters 20]
     python -m nf4_layer_streamed_b200.gemm_bench --once --shapes gateup   (one launch each: for ncu)
     python -m nf4_layer_streamed_b200.gemm_bench --attention 4 [--once]      (attention fwd / bwd, batch 4)
-    python -m nf4_layer_streamed_b200.gemm_bench --layer 4 [--once]   (quantise + one 8B layer fwd/bwd)
+    python -m nf4_layer_streamed_b200.gemm_bench --layer 4 [--once] [--layer-shape smollm2]
+                                                   (quantise + one layer fwd/bwd)
 
 Prints one JSON object per (shape, direction, kernel) with the mean launch time
 (CUDA events on the launching stream, after warm-up) and TFLOP/s = 2 M N K / time.
@@ -136,11 +137,12 @@ def run_attention(batch: int, once: bool, iters: int = 20):
     return out
 
 
-def run_layer(batch: int, once: bool, iters: int = 10):
-    """One Llama-8B-shaped layer at batch x 512: the shard quantiser, then layer_forward
-    and layer_backward (recompute + dL/dx + LoRA gradients) with random LoRA B.  With
-    --once each runs once (a small case for ncu: every kernel of the layer appears)."""
-    shape = synth.LLAMA_8B
+def run_layer(batch: int, once: bool, iters: int = 10, shape_name: str = "llama8b"):
+    """One Llama-8B-shaped (or SmolLM2-135M-shaped) layer at batch x 512: the shard
+    quantiser, then layer_forward and layer_backward (recompute + dL/dx + LoRA gradients)
+    with random LoRA B.  With --once each runs once (a small case for ncu: every kernel
+    of the layer appears)."""
+    shape = {"llama8b": synth.LLAMA_8B, "smollm2": synth.SMOLLM2_135M}[shape_name]
     seq = 512
     cfg = api.layer_cfg(shape, batch, seq)
     w = synth.layer_weights(shape, 0, 1234, device="cuda")
@@ -191,6 +193,8 @@ def main(argv=None):
                     help="pair tile height: 0 auto, 1 512 tokens, 2 256 tokens, 3 last partial wave as 256")
     ap.add_argument("--layer", type=int, default=0, metavar="BATCH",
                     help="time the shard quantiser and one 8B layer forward / backward at this batch instead")
+    ap.add_argument("--layer-shape", default="llama8b", choices=["llama8b", "smollm2"],
+                    help="the layer shape of --layer")
     ap.add_argument("--attention", type=int, default=0, metavar="BATCH",
                     help="time the attention forward of the 8B layer at this batch (seq 512) instead")
     a = ap.parse_args(argv)
@@ -200,7 +204,7 @@ def main(argv=None):
         run_attention(a.attention, a.once)
         return
     if a.layer:
-        run_layer(a.layer, a.once)
+        run_layer(a.layer, a.once, shape_name=a.layer_shape)
         st, err = api.device_error()
         if st != 0:
             raise RuntimeError(f"device error record {err}")
