@@ -362,7 +362,11 @@ __device__ __forceinline__ void bar_ew() { asm volatile("bar.sync 1, %0;" ::"n"(
 // column is c0: warp half g wrote its 32 rows' packed values to columns c0 + 32 g ..
 __device__ __forceinline__ uint32_t packed_col(uint32_t c0, int ks) { return c0 + (ks >> 1) * 32 + (ks & 1) * 8; }
 
-// QUERY side: dQ of one 128-query tile of one query head.
+// QUERY side: dQ of one 128-query tile of one query head.  The Q and dO tiles are
+// copied once into TMEM (bf16 pairs, one query row per lane), so that S = Q K^T and
+// dP = dO V^T take their A operand from TMEM and read only the 64-key halves of K and V
+// from shared memory: an N = 64 product with both operands in shared memory would read
+// 6 KB per 32 tensor-core cycles, more than shared memory delivers.
 __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_constant__ AttnBwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -374,7 +378,8 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
   uint64_t* p_full = bars + 7;      // 2
   uint64_t* acc_full = bars + 9;
   uint64_t* drain = bars + 10;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+  uint64_t* qa_full = bars + 11;    // Q and dO are in TMEM (one arrival per elementwise warp)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -393,6 +398,7 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
     }
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
+    mbar_init(qa_full, B_EW / 32);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -403,7 +409,9 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;  // item buffers [0,128) and [128,256) (S | dP), dQ [256,384)
+  // item buffers [0,128) and [128,256) (S | dP), dQ [256,384), Q [384,448), dO [448,512)
+  const uint32_t tmem = *tmem_slot;
+  constexpr uint32_t T_Q = 384, T_DO = 448;
 
   if (warp == B_PROD) {
     if (lane == 0) {
@@ -438,8 +446,7 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
   } else if (warp == B_MMA) {
     constexpr uint32_t idesc_s = idesc_bf16(128, 64, false);   // S, dP: N = 64 keys
     constexpr uint32_t idesc_a = idesc_bf16(128, 128, true);   // dQ += dS K: K N-major
-    const uint32_t sQ = smem_u32(base + B_OFF_A), sO = sQ + TILE_BYTES;
-    bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort_flag, p.err, KID_ATTN, 42));
+    bool ok = __all_sync(0xffffffffu, mbar_wait(qa_full, 0, abort_flag, p.err, KID_ATTN, 42)) && !*abort_flag;
     // item it: key tile it / 2, half it % 2, TMEM buffer it % 2
     auto second = [&](int it) -> bool {  // dQ += dS_it K_half(it)
       if (!__all_sync(0xffffffffu, mbar_wait(&p_full[it & 1], (it >> 1) & 1, abort_flag, p.err, KID_ATTN, 44)))
@@ -469,12 +476,12 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
         // tcgen05.mma of one thread run in issue order: these may overwrite the dS of
         // item it - 2, whose product was issued before
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {  // over the head dim
+        for (int ks = 0; ks < 8; ++ks) {  // over the head dim: Q, dO columns 8 ks .. in TMEM
           const uint32_t off = (ks >> 2) * ATOM + (ks & 3) * 32;
-          umma_bf16(tmem + bf * 128, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sK + hh * 8192 + off, 16, 1024),
-                    idesc_s, ks ? 1u : 0u);
-          umma_bf16(tmem + bf * 128 + 64, sdesc_sw128(sO + off, 16, 1024),
-                    sdesc_sw128(sV + hh * 8192 + off, 16, 1024), idesc_s, ks ? 1u : 0u);
+          umma_bf16_ta(tmem + bf * 128, tmem + T_Q + ks * 8, sdesc_sw128(sK + hh * 8192 + off, 16, 1024), idesc_s,
+                       ks ? 1u : 0u);
+          umma_bf16_ta(tmem + bf * 128 + 64, tmem + T_DO + ks * 8, sdesc_sw128(sV + hh * 8192 + off, 16, 1024),
+                       idesc_s, ks ? 1u : 0u);
         }
         umma_commit(&sd_full[bf]);
       }
@@ -496,20 +503,35 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
     float* red = reinterpret_cast<float*>(base + B_OFF_X + TILE_BYTES);
     bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort_flag, p.err, KID_ATTN, 45));
     if (ok) {
+      // this thread's row of swizzle atom g (dims 64 g ..): chunk c holds dims 8 c .. 8 c + 7,
+      // TMEM column 32 g + 4 c + i their pair i
+      const uint8_t* q_row = base + B_OFF_A + g * ATOM + r * 128;
       const uint8_t* dO_row = base + B_OFF_A + TILE_BYTES + g * ATOM + r * 128;
       const uint8_t* o_row = base + B_OFF_X + g * ATOM + r * 128;
+      uint32_t qv[32], dv[32];
       float s = 0.f;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         const uint32_t off = (uint32_t)((c ^ (r & 7)) << 4);
         const uint4 a = *reinterpret_cast<const uint4*>(o_row + off);
         const uint4 d = *reinterpret_cast<const uint4*>(dO_row + off);
-        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, dw[4] = {d.x, d.y, d.z, d.w};
+        const uint4 q = *reinterpret_cast<const uint4*>(q_row + off);
+        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, dw[4] = {d.x, d.y, d.z, d.w}, qw[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-        for (int j = 0; j < 4; ++j) s += bf16_lo(aw[j]) * bf16_lo(dw[j]) + bf16_hi(aw[j]) * bf16_hi(dw[j]);
+        for (int j = 0; j < 4; ++j) {
+          s += bf16_lo(aw[j]) * bf16_lo(dw[j]) + bf16_hi(aw[j]) * bf16_hi(dw[j]);
+          qv[4 * c + j] = qw[j];
+          dv[4 * c + j] = dw[j];
+        }
       }
       red[g * 128 + r] = s;
+      tmem_st32(trow + T_Q + g * 32, qv);
+      tmem_st32(trow + T_DO + g * 32, dv);
+      tmem_wait_st();
     }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(qa_full);  // also on failure: the MMA warp then sees the abort
     bar_ew();
     const float dl = ok ? red[r] + red[128 + r] : 0.f;
     if (ok && g == 0) p.delta[li] = dl;
@@ -736,19 +758,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
       tmem_ld32(trow + bf * 128 + 64 + g * 32, dpv);
       tmem_wait_ld();
       const int qi0 = hh * 64 + g * 32;  // query within the tile
+      const int lim = key - qt * TT - qi0;  // columns c < lim are masked (only on the diagonal tile)
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        float pv[2], ds[2];
+      for (int j4 = 0; j4 < 8; ++j4) {  // four columns: their lse and delta in one vector load each
+        const float4 l4 = *reinterpret_cast<const float4*>(ld + qi0 + 4 * j4);
+        const float4 d4 = *reinterpret_cast<const float4*>(ld + 128 + qi0 + 4 * j4);
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dl[4] = {d4.x, d4.y, d4.z, d4.w};
+        float pv[4], ds[4];
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int qi = qi0 + 2 * j + e;
+        for (int e = 0; e < 4; ++e) {
+          const int c = 4 * j4 + e;
           const float pe =
-              key <= qt * TT + qi ? fast_exp2(fmaf(__uint_as_float(sv[2 * j + e]), sl, -ld[qi] * 1.4426950408889634f)) : 0.f;
+              c >= lim ? fast_exp2(fmaf(__uint_as_float(sv[c]), sl, -lv[e] * 1.4426950408889634f)) : 0.f;
           pv[e] = pe;
-          ds[e] = pe * (__uint_as_float(dpv[2 * j + e]) - ld[128 + qi]);
+          ds[e] = pe * (__uint_as_float(dpv[c]) - dl[e]);
         }
-        pp[j] = pack_bf16x2(pv[0], pv[1]);
-        dd[j] = pack_bf16x2(ds[0], ds[1]);
+        pp[2 * j4] = pack_bf16x2(pv[0], pv[1]);
+        pp[2 * j4 + 1] = pack_bf16x2(pv[2], pv[3]);
+        dd[2 * j4] = pack_bf16x2(ds[0], ds[1]);
+        dd[2 * j4 + 1] = pack_bf16x2(ds[2], ds[3]);
       }
       tmem_st16(trow + bf * 128 + g * 32, pp);        // over the scores this warp has read
       tmem_st16(trow + bf * 128 + 64 + g * 32, dd);

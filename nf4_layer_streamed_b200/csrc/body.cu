@@ -60,59 +60,67 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   return a;
 }
 
-__device__ void pack_element(const LoraPack& a, size_t i) {
+// The adapter operands in 16-byte pieces (8 bf16 outputs each), 32-bit indices:
+//   bup [qd + 2 kvd, 64]: s B_q in columns 0-15 of the q rows, s B_v in 16-31 of the v rows
+//   adn [64, H]:          A_q in rows 0-15, A_v in 16-31, zero rows 32-63
+//   bqt [16, qd], bvt [16, kvd]: B_q^T, B_v^T
+__device__ void pack_piece(const LoraPack& a, int i) {
   const int H = a.H, qd = a.qd, kvd = a.kvd, nq = qd + 2 * kvd;
-  const size_t n1 = (size_t)nq * 64, n2 = (size_t)64 * H, n3 = (size_t)16 * qd;
-  if (i < n1) {
-    const int n = (int)(i / 64), c = (int)(i % 64);
-    float v = 0.f;
+  float f[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) f[e] = 0.f;
+  __nv_bfloat16* dst;
+  if (i < nq * 8) {
+    const int n = i >> 3, c = (i & 7) * 8;
+    const float* src = nullptr;
     if (n < qd && c < 16)
-      v = a.scale * __bfloat162float(__float2bfloat16_rn(a.Bq[(size_t)n * 16 + c]));
+      src = a.Bq + (size_t)n * 16 + c;
     else if (n >= qd + kvd && c >= 16 && c < 32)
-      v = a.scale * __bfloat162float(__float2bfloat16_rn(a.Bv[(size_t)(n - qd - kvd) * 16 + c - 16]));
-    a.bup[i] = __float2bfloat16_rn(v);
-    return;
+      src = a.Bv + (size_t)(n - qd - kvd) * 16 + (c - 16);
+    if (src)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) f[e] = a.scale * __bfloat162float(__float2bfloat16_rn(src[e]));
+    dst = a.bup + (size_t)n * 64 + c;
+  } else if ((i -= nq * 8) < 8 * H) {
+    const int per = H / 8, r = i / per, k = (i - r * per) * 8;
+    const float* src = r < 16 ? a.Aq + (size_t)r * H + k : r < 32 ? a.Av + (size_t)(r - 16) * H + k : nullptr;
+    if (src)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) f[e] = src[e];
+    dst = a.adn + (size_t)r * H + k;
+  } else if ((i -= 8 * H) < 2 * qd) {
+    const int per = qd / 8, r = i / per, n = (i - r * per) * 8;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) f[e] = a.Bq[(size_t)(n + e) * 16 + r];
+    dst = a.bqt + (size_t)r * qd + n;
+  } else {
+    i -= 2 * qd;
+    const int per = kvd / 8, r = i / per, n = (i - r * per) * 8;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) f[e] = a.Bv[(size_t)(n + e) * 16 + r];
+    dst = a.bvt + (size_t)r * kvd + n;
   }
-  i -= n1;
-  if (i < n2) {
-    const int r = (int)(i / H), k = (int)(i % H);
-    float v = 0.f;
-    if (r < 16)
-      v = a.Aq[(size_t)r * H + k];
-    else if (r < 32)
-      v = a.Av[(size_t)(r - 16) * H + k];
-    a.adn[i] = __float2bfloat16_rn(v);
-    return;
-  }
-  i -= n2;
-  if (i < n3) {
-    const int r = (int)(i / qd), n = (int)(i % qd);
-    a.bqt[i] = __float2bfloat16_rn(a.Bq[(size_t)n * 16 + r]);
-    return;
-  }
-  i -= n3;
-  const int r = (int)(i / kvd), n = (int)(i % kvd);
-  a.bvt[i] = __float2bfloat16_rn(a.Bv[(size_t)n * 16 + r]);
+  *reinterpret_cast<uint4*>(dst) = pack8(f);
 }
 
-__host__ __device__ inline size_t pack_elements(const LoraPack& a) {
-  return (size_t)(a.qd + 2 * a.kvd) * 64 + (size_t)64 * a.H + 16ull * a.qd + 16ull * a.kvd;
+__host__ __device__ inline int pack_pieces(const LoraPack& a) {
+  return (a.qd + 2 * a.kvd) * 8 + 8 * a.H + 2 * a.qd + 2 * a.kvd;
 }
 
-// Blocks [0, M): one row each.  Blocks from M on (when pack.bup is set): the adapter
-// operand conversion, grid-stride.
+// Blocks [0, n_pack): the adapter operand conversion, grid-stride (first, so that it
+// runs beside the rows rather than after them); the blocks after: one row each.
 template <int VPT>
 __global__ void __launch_bounds__(1024) k_rmsnorm_fwd_row(const __nv_bfloat16* __restrict__ x,
                                                           const __nv_bfloat16* __restrict__ w,
                                                           __nv_bfloat16* __restrict__ y, int M, int H, float eps,
-                                                          const LoraPack pack) {
+                                                          const LoraPack pack, int n_pack) {
   __shared__ float red[32];
-  if ((int)blockIdx.x >= M) {
-    const size_t n = pack_elements(pack), stride = (size_t)(gridDim.x - M) * blockDim.x;
-    for (size_t i = (size_t)(blockIdx.x - M) * blockDim.x + threadIdx.x; i < n; i += stride) pack_element(pack, i);
+  if ((int)blockIdx.x < n_pack) {
+    const int n = pack_pieces(pack), stride = n_pack * blockDim.x;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) pack_piece(pack, i);
     return;
   }
-  const int row = blockIdx.x, t = threadIdx.x, T = blockDim.x, nv = H / 8;
+  const int row = blockIdx.x - n_pack, t = threadIdx.x, T = blockDim.x, nv = H / 8;
   const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)row * H);
   const uint4* wr = reinterpret_cast<const uint4*>(w);
   uint4* yr = reinterpret_cast<uint4*>(y + (size_t)row * H);
@@ -143,6 +151,175 @@ __global__ void __launch_bounds__(1024) k_rmsnorm_fwd_row(const __nv_bfloat16* _
       yr[i] = pack8(f);
     }
   }
+}
+
+// The input RMSNorm with the LoRA down-projection as its second output:
+//   h1 = bf16(x r w),  t = [h1 A_q^T | h1 A_v^T] (bf16, columns 0-31 of the 64-wide extra
+//   operand of the q/k/v GEMM, zeros in 32-63),
+// so that h1 is not read back for t.  A cluster of C CTAs takes 64 rows; CTA c of the
+// cluster holds the column slice [c S, (c + 1) S) of those rows (S = H / C) in registers
+// (four threads per row) and the same slice of the 32 adapter rows, rounded to bf16, in
+// shared memory.  The rows' sums of squares are partial per CTA and added in CTA order
+// through distributed shared memory; each CTA then writes its slice of h1 and forms the
+// partial t of its slice on mma.sync m16n8k16 (warp w: row tile w % 4, k-steps
+// w / 4, w / 4 + 2, ..); the warp partials are added in k order, and the cluster's C
+// partials in CTA order, CTA c writing rows 64 c / C ...  The same launch converts the
+// adapter to its bf16 operands (every thread a share of pack_piece).
+constexpr int ND_R = 64, ND_THREADS = 256, ND_TPR = ND_THREADS / ND_R;  // threads per row
+
+struct NormDownShape {
+  int C, S;  // cluster size, slice width
+  size_t smem;
+};
+inline NormDownShape norm_down_shape(int H) {
+  NormDownShape sh{0, 0, 0};
+  for (int c : {8, 4, 2, 1})
+    if (H % (16 * c) == 0 && H / c <= 1024) {
+      sh.C = c;
+      sh.S = H / c;
+      break;
+    }
+  if (sh.C) {
+    const size_t hs = (size_t)ND_R * (sh.S + 8) * 2, as = (size_t)32 * (sh.S + 8) * 2;
+    sh.smem = hs + std::max(as, (size_t)ND_THREADS / 32 * 16 * 32 * 4) + (size_t)ND_R * 32 * 4 + ND_R * 4;
+  }
+  return sh;
+}
+
+template <int VPT>
+__global__ void __launch_bounds__(ND_THREADS) k_rmsnorm_down(const __nv_bfloat16* __restrict__ x,
+                                                             const __nv_bfloat16* __restrict__ w,
+                                                             __nv_bfloat16* __restrict__ y, int M, int H, int S,
+                                                             float eps, const LoraPack pack,
+                                                             __nv_bfloat16* __restrict__ tpad) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31, ls = S + 8, nv = S / 8;
+  const int C = (int)(gridDim.y), c = (int)cluster_ctarank(), m0 = blockIdx.x * ND_R, col0 = c * S;
+  __nv_bfloat16* hs = reinterpret_cast<__nv_bfloat16*>(smem);                 // [64][S + 8] h1 slice
+  __nv_bfloat16* as = hs + (size_t)ND_R * ls;                                  // [32][S + 8] adapter slice
+  float* red = reinterpret_cast<float*>(as);                                   // after the products: [8][16][32]
+  const size_t as_bytes = std::max((size_t)32 * ls * 2, (size_t)ND_THREADS / 32 * 16 * 32 * 4);
+  float* P = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(as) + as_bytes);  // [64][32] this slice's t
+  float* ssp = P + ND_R * 32;                                                  // [64] partial sums of squares
+  const int row = t / ND_TPR, sub = t % ND_TPR, m = m0 + row;
+  const bool live = m < M;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)m * H + col0);
+  uint4 v[VPT];
+#pragma unroll
+  for (int j = 0; j < VPT; ++j)
+    if (live && sub + ND_TPR * j < nv) v[j] = xr[sub + ND_TPR * j];
+  // the adapter slice: rows 0-15 A_q, 16-31 A_v, bf16 (the values of the packed adn);
+  // eight 16-byte loads in flight per thread
+  {
+    const int n4 = 32 * (S / 4);
+    for (int i0 = 0; i0 < n4; i0 += 8 * ND_THREADS) {
+      float4 f[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * ND_THREADS + t;
+        if (i < n4) {
+          const int r = i / (S / 4), k = (i - r * (S / 4)) * 4;
+          f[u] = __ldg(reinterpret_cast<const float4*>(
+              (r < 16 ? pack.Aq + (size_t)r * H : pack.Av + (size_t)(r - 16) * H) + col0 + k));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * ND_THREADS + t;
+        if (i < n4) {
+          const int r = i / (S / 4), k = (i - r * (S / 4)) * 4;
+          *reinterpret_cast<uint2*>(as + r * ls + k) =
+              make_uint2(pack_bf16x2(f[u].x, f[u].y), pack_bf16x2(f[u].z, f[u].w));
+        }
+      }
+    }
+  }
+  float ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < VPT; ++j)
+    if (live && sub + ND_TPR * j < nv) {
+      float f[8];
+      unpack8(v[j], f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ss += f[e] * f[e];
+    }
+#pragma unroll
+  for (int o = 1; o < ND_TPR; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if (sub == 0) ssp[row] = ss;
+  cluster_sync_all();  // every slice's partial sums are in its CTA's shared memory
+  float tot = 0.f;
+  for (int q = 0; q < C; ++q) tot += ld_cluster_f32(mapa_shared(smem_u32(ssp + row), (uint32_t)q));
+  const float r = 1.0f / sqrtf(tot / (float)H + eps);
+  const uint4* wr = reinterpret_cast<const uint4*>(w + col0);
+  uint4* yr = reinterpret_cast<uint4*>(y + (size_t)m * H + col0);
+  uint4* hrow = reinterpret_cast<uint4*>(hs + row * ls);
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+    const int i = sub + ND_TPR * j;
+    if (i < nv) {
+      uint4 h = make_uint4(0u, 0u, 0u, 0u);
+      if (live) {
+        float f[8], g[8];
+        unpack8(v[j], f);
+        unpack8(wr[i], g);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = f[e] * r * g[e];
+        h = pack8(f);
+        yr[i] = h;
+      }
+      hrow[i] = h;
+    }
+  }
+  __syncthreads();
+  // partial t of the slice: row tile mt = warp % 4 (16 rows), k-steps kq, kq + 2, ..
+  const int mt = warp & 3, kq = warp >> 2;
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+  for (int ks = kq; ks < S / 16; ks += 2) {
+    uint32_t a0, a1, a2, a3, b0, b1, b2, b3, b4, b5, b6, b7;
+    ldsm4(smem_u32(hs + (mt * 16 + (lane & 15)) * ls + ks * 16 + (lane >> 4) * 8), a0, a1, a2, a3);
+    const int br = (lane & 7) + (lane >> 4) * 8, bc = ks * 16 + ((lane >> 3) & 1) * 8;
+    ldsm4(smem_u32(as + br * ls + bc), b0, b1, b2, b3);
+    ldsm4(smem_u32(as + (16 + br) * ls + bc), b4, b5, b6, b7);
+    mma16816(acc[0], a0, a1, a2, a3, b0, b1);
+    mma16816(acc[1], a0, a1, a2, a3, b2, b3);
+    mma16816(acc[2], a0, a1, a2, a3, b4, b5);
+    mma16816(acc[3], a0, a1, a2, a3, b6, b7);
+  }
+  __syncthreads();  // every warp is done with the adapter slice: red may overwrite it
+  {
+    const int g4 = lane >> 2, t4 = lane & 3;
+    float* R = red + warp * (16 * 32);
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+      R[g4 * 32 + nt * 8 + 2 * t4] = acc[nt][0];
+      R[g4 * 32 + nt * 8 + 2 * t4 + 1] = acc[nt][1];
+      R[(g4 + 8) * 32 + nt * 8 + 2 * t4] = acc[nt][2];
+      R[(g4 + 8) * 32 + nt * 8 + 2 * t4 + 1] = acc[nt][3];
+    }
+  }
+  __syncthreads();
+  for (int e = t; e < ND_R * 32; e += ND_THREADS) {  // the slice's t: the two k halves in order
+    const int rr = e >> 5, cc = e & 31, tile = rr >> 4, ri = rr & 15;
+    P[e] = red[tile * (16 * 32) + ri * 32 + cc] + red[(4 + tile) * (16 * 32) + ri * 32 + cc];
+  }
+  cluster_sync_all();  // every slice's t is in its CTA's shared memory
+  const int rows_per = ND_R / C;
+  for (int e = t; e < rows_per * 64; e += ND_THREADS) {
+    const int rr = c * rows_per + (e >> 6), cc = e & 63, mm = m0 + rr;
+    if (mm >= M) continue;
+    float v2 = 0.f;
+    if (cc < 32)
+      for (int q = 0; q < C; ++q) v2 += ld_cluster_f32(mapa_shared(smem_u32(P + rr * 32 + cc), (uint32_t)q));
+    tpad[(size_t)mm * 64 + cc] = __float2bfloat16_rn(v2);
+  }
+  // the adapter's bf16 operands, a share per thread of the whole grid
+  {
+    const int n = pack_pieces(pack), stride = gridDim.x * gridDim.y * ND_THREADS;
+    for (int i = (blockIdx.y * gridDim.x + blockIdx.x) * ND_THREADS + t; i < n; i += stride) pack_piece(pack, i);
+  }
+  cluster_sync_all();  // no CTA leaves while another still reads its shared memory
 }
 
 template <int VPT>
@@ -549,25 +726,74 @@ inline unsigned blocks_for(size_t n, int threads) { return (unsigned)((n + threa
 
 }  // namespace
 
-// One block per row, the row in registers: 4 vectors (32 values) per thread up to
-// H = 32768 (128 threads at H = 4096), 2 below H = 1024 (SmolLM2: 576 -> 64 threads).
+// One block per row, the row in registers: 2 vectors (16 values) per thread up to
+// H = 16384 (256 threads at H = 4096, 64 at SmolLM2's 576), 4 up to H = 32768.
 int rmsnorm_fwd(const __nv_bfloat16* x, const __nv_bfloat16* w, __nv_bfloat16* y, int M, int H, float eps,
                 cudaStream_t s, const LoraPack* pack) {
   if (H % 8 || H > 32768) return fail(NF4LS_SHAPE, "rmsnorm: H %% 8, H <= 32768");
   if (M <= 0) return NF4LS_OK;
   LoraPack pk{};
-  const int threads = row_threads(H, H < 1024 ? 2 : 4);
-  int grid = M;
-  if (pack) {  // about 16 operand elements per thread of the extra blocks
+  const int vpt = H <= 16384 ? 2 : 4;
+  const int threads = row_threads(H, vpt);
+  int n_pack = 0;
+  if (pack) {  // about four 16-byte pieces per thread of the extra blocks
     pk = *pack;
-    grid += (int)std::min<size_t>(1024, (pack_elements(pk) + 16ull * threads - 1) / (16ull * threads));
+    if (pk.qd % 8 || pk.kvd % 8) return fail(NF4LS_SHAPE, "rmsnorm: adapter widths %% 8");
+    n_pack = std::min(1024, (pack_pieces(pk) + 4 * threads - 1) / (4 * threads));
   }
-  if (H < 1024)
-    k_rmsnorm_fwd_row<2><<<grid, threads, 0, s>>>(x, w, y, M, H, eps, pk);
+  if (vpt == 2)
+    k_rmsnorm_fwd_row<2><<<M + n_pack, threads, 0, s>>>(x, w, y, M, H, eps, pk, n_pack);
   else
-    k_rmsnorm_fwd_row<4><<<grid, threads, 0, s>>>(x, w, y, M, H, eps, pk);
+    k_rmsnorm_fwd_row<4><<<M + n_pack, threads, 0, s>>>(x, w, y, M, H, eps, pk, n_pack);
   note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
+  return NF4LS_OK;
+}
+
+// Input RMSNorm + adapter operand conversion + t = h1 [A_q; A_v]^T in one launch.
+int rmsnorm_lora_fwd(const __nv_bfloat16* x, const __nv_bfloat16* w, __nv_bfloat16* y, int M, int H, float eps,
+                     const LoraPack& pack, __nv_bfloat16* tpad, cudaStream_t s) {
+  const NormDownShape sh = norm_down_shape(H);
+  if (!sh.C) return fail(NF4LS_SHAPE, "rmsnorm_lora_fwd: H %d (a multiple of 16 up to 8192)", H);
+  if (pack.qd % 8 || pack.kvd % 8) return fail(NF4LS_SHAPE, "rmsnorm_lora_fwd: adapter widths %% 8");
+  if (!aligned(pack.Aq, 16) || !aligned(pack.Av, 16) || !aligned(x, 16) || !aligned(y, 16) || !aligned(w, 16))
+    return fail(NF4LS_ALIGN, "rmsnorm_lora_fwd: 16-byte aligned operands");
+  if (M <= 0) return NF4LS_OK;
+  const int vpt = (sh.S / 8 + ND_TPR - 1) / ND_TPR;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((M + ND_R - 1) / ND_R, sh.C, 1);
+  cfg.blockDim = dim3(ND_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = sh.smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = sh.C;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  auto go = [&](auto kernel, int slot) -> int {
+    static int configured[16][4] = {};
+    int dev = 0;
+    NF4_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 16 && configured[dev][slot] < (int)sh.smem) {
+      NF4_CUDA_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sh.smem));
+      configured[dev][slot] = (int)sh.smem;
+    }
+    NF4_CUDA_TRY(cudaLaunchKernelEx(&cfg, kernel, x, w, y, M, H, sh.S, eps, pack, tpad));
+    return NF4LS_OK;
+  };
+  int st;
+  if (vpt <= 8)
+    st = go(k_rmsnorm_down<8>, 0);
+  else if (vpt <= 16)
+    st = go(k_rmsnorm_down<16>, 1);
+  else if (vpt <= 24)
+    st = go(k_rmsnorm_down<24>, 2);
+  else
+    st = go(k_rmsnorm_down<32>, 3);
+  if (st != NF4LS_OK) return st;
+  note_launch();
   return NF4LS_OK;
 }
 
@@ -575,7 +801,7 @@ int rmsnorm_bwd(const __nv_bfloat16* x, const __nv_bfloat16* w, const __nv_bfloa
                 __nv_bfloat16* dx, int M, int H, float eps, cudaStream_t s) {
   if (H % 8 || H > 32768) return fail(NF4LS_SHAPE, "rmsnorm_bwd: H %% 8, H <= 32768");
   if (M <= 0) return NF4LS_OK;
-  if (H < 1024)
+  if (H <= 16384)
     k_rmsnorm_bwd_row<2><<<M, row_threads(H, 2), 0, s>>>(x, w, dy, resid, dx, H, eps);
   else
     k_rmsnorm_bwd_row<4><<<M, row_threads(H, 4), 0, s>>>(x, w, dy, resid, dx, H, eps);

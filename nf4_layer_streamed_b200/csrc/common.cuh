@@ -282,6 +282,13 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t a, uint32_t rank) {
   return r;
 }
 
+// ld.shared::cluster of one float at a shared::cluster address (possibly another CTA's).
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+
 // Arrive on an mbarrier given by its shared::cluster address (possibly the other CTA's).
 // Release at CTA scope: what the arrival publishes is this thread's own CTA's shared
 // memory, already handed to the async proxy by fence.proxy.async, and CTA scope orders

@@ -244,6 +244,10 @@ struct LoraPack {
 // y = rmsnorm(x) w; with pack, the same launch also fills the adapter operands.
 int rmsnorm_fwd(const __nv_bfloat16* x, const __nv_bfloat16* w, __nv_bfloat16* y, int M, int H, float eps,
                 cudaStream_t s, const LoraPack* pack = nullptr);
+// y = rmsnorm(x) w (the input norm) with the adapter operands filled and
+// t = [y A_q^T | y A_v^T] written to columns 0-31 of tpad [M, 64] (32-63 zero).
+int rmsnorm_lora_fwd(const __nv_bfloat16* x, const __nv_bfloat16* w, __nv_bfloat16* y, int M, int H, float eps,
+                     const LoraPack& pack, __nv_bfloat16* tpad, cudaStream_t s);
 // dx = resid + rmsnorm_bwd(x, w, dy); resid may be null.
 int rmsnorm_bwd(const __nv_bfloat16* x, const __nv_bfloat16* w, const __nv_bfloat16* dy,
                 const __nv_bfloat16* resid, __nv_bfloat16* dx, int M, int H, float eps, cudaStream_t s);
@@ -272,9 +276,7 @@ int attention_bwd(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfl
                   __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv, int ld_dq, int ld_dkv, int batch,
                   int seq, int nq, int nkv, int d, cudaStream_t s);
 
-// LoRA (lora.cu).  Forward: t = [h1 A_q^T | h1 A_v^T] into tpad [M, 64] (bf16, zeros in
-// columns 32-63) from h1 and adn (the bf16 A_q, A_v rows of LoraPack).
-int lora_down(const __nv_bfloat16* h1, int M, int H, const __nv_bfloat16* adn, __nv_bfloat16* tpad, cudaStream_t s);
+// LoRA backward (lora.cu); the forward's t comes from rmsnorm_lora_fwd (body.cu).
 // Backward, three launches: dB_q, dB_v, dA_q, dA_v (fp32, written) and dt into dtpad
 // [M, 64] (bf16, zeros in columns 32-63) from dq (columns [0, qd) of dqkv) and dv
 // (columns [vcol, vcol + kvd)); part: lora_partial_bytes of scratch.
@@ -303,11 +305,13 @@ int adamw(float* p, const float* g, float* m, float* v, size_t n, int step, floa
           float wd, cudaStream_t s);
 
 // ----------------------------------------------------------------------------- layer
+// tables_ready: the RoPE tables of the workspace are already those of cfg (a model pass
+// writes them at its first layer and the other layers of the pass reuse them).
 int layer_fwd_impl(const nf4ls_layer_cfg* cfg, const void* shard, const nf4ls_lora* lora, const __nv_bfloat16* x,
-                   __nv_bfloat16* y, void* ws, size_t ws_bytes, cudaStream_t s);
+                   __nv_bfloat16* y, void* ws, size_t ws_bytes, cudaStream_t s, bool tables_ready = false);
 int layer_bwd_impl(const nf4ls_layer_cfg* cfg, const void* shard, const nf4ls_lora* lora, const __nv_bfloat16* x,
                    const __nv_bfloat16* dy, __nv_bfloat16* dx, const nf4ls_lora_grads* g, void* ws, size_t ws_bytes,
-                   cudaStream_t s);
+                   cudaStream_t s, bool tables_ready = false);
 size_t layer_ws_bytes(const nf4ls_layer_cfg* cfg);
 
 }  // namespace nf4ls

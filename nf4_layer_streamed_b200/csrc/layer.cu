@@ -96,7 +96,8 @@ struct LayerCtx {
   GemmWeights w_qkv, w_o, w_gu, w_down;
 };
 
-int prepare(LayerCtx& x, const nf4ls_layer_cfg* c, const void* shard, void* ws, size_t ws_bytes, cudaStream_t s) {
+int prepare(LayerCtx& x, const nf4ls_layer_cfg* c, const void* shard, void* ws, size_t ws_bytes, cudaStream_t s,
+            bool tables_ready) {
   NF4_TRY(check_cfg(c));
   if (!shard || !ws) return fail(NF4LS_INVALID_ARG, "layer: null shard or workspace");
   if (!aligned(shard, 256) || !aligned(ws, 256)) return fail(NF4LS_ALIGN, "layer: shard and workspace must be 256-byte aligned");
@@ -144,6 +145,7 @@ int prepare(LayerCtx& x, const nf4ls_layer_cfg* c, const void* shard, void* ws, 
     x.w_down.n_seg = 1;
     x.w_down.seg[0] = x.v.t[6];
   }
+  if (tables_ready) return NF4LS_OK;
   return rope_tables(at<float>(ws, x.L.cos), at<float>(ws, x.L.sin), at<float>(ws, x.L.cos_t),
                      at<float>(ws, x.L.sin_t), c->seq, c->head_dim, c->rope_theta, s);
 }
@@ -163,7 +165,7 @@ int forward_body(LayerCtx& x, const nf4ls_lora* lora, const __nv_bfloat16* X, __
   auto* tpad = at<__nv_bfloat16>(ws, x.L.tpad);
   GemmExtra ex;
   if (lora) {
-    // the input RMSNorm's launch also converts the adapter to its bf16 operands; then
+    // one launch: the input RMSNorm, the adapter's bf16 operands and
     // t = [h1 A_q^T | h1 A_v^T] (columns 0-31 of the padded extra operand)
     LoraPack pk;
     pk.Aq = lora->A_q;
@@ -178,8 +180,7 @@ int forward_body(LayerCtx& x, const nf4ls_lora* lora, const __nv_bfloat16* X, __
     pk.adn = at<__nv_bfloat16>(ws, x.L.adn);
     pk.bqt = at<__nv_bfloat16>(ws, x.L.bqt);
     pk.bvt = at<__nv_bfloat16>(ws, x.L.bvt);
-    NF4_TRY(rmsnorm_fwd(X, x.v.norm_in, h1, M, H, c->rms_eps, s, &pk));
-    NF4_TRY(lora_down(h1, M, H, pk.adn, tpad, s));
+    NF4_TRY(rmsnorm_lora_fwd(X, x.v.norm_in, h1, M, H, c->rms_eps, pk, tpad, s));
     ex.a = tpad;
     ex.b = pk.bup;
   } else {
@@ -232,21 +233,21 @@ int forward_body(LayerCtx& x, const nf4ls_lora* lora, const __nv_bfloat16* X, __
 size_t layer_ws_bytes(const nf4ls_layer_cfg* cfg) { return ws_layout(cfg).total; }
 
 int layer_fwd_impl(const nf4ls_layer_cfg* c, const void* shard, const nf4ls_lora* lora, const __nv_bfloat16* X,
-                   __nv_bfloat16* y, void* ws, size_t ws_bytes, cudaStream_t s) {
+                   __nv_bfloat16* y, void* ws, size_t ws_bytes, cudaStream_t s, bool tables_ready) {
   if (!X || !y) return fail(NF4LS_INVALID_ARG, "layer_forward: null activation");
   LayerCtx x;
-  NF4_TRY(prepare(x, c, shard, ws, ws_bytes, s));
+  NF4_TRY(prepare(x, c, shard, ws, ws_bytes, s, tables_ready));
   return forward_body(x, lora, X, y, false, s);
 }
 
 int layer_bwd_impl(const nf4ls_layer_cfg* c, const void* shard, const nf4ls_lora* lora, const __nv_bfloat16* X,
                    const __nv_bfloat16* dy, __nv_bfloat16* dx, const nf4ls_lora_grads* g, void* ws, size_t ws_bytes,
-                   cudaStream_t s) {
+                   cudaStream_t s, bool tables_ready) {
   if (!X || !dy || !dx) return fail(NF4LS_INVALID_ARG, "layer_backward: null activation");
   if (lora && (!g || !g->dA_q || !g->dB_q || !g->dA_v || !g->dB_v))
     return fail(NF4LS_INVALID_ARG, "layer_backward: LoRA gradients needed when the adapter is on");
   LayerCtx x;
-  NF4_TRY(prepare(x, c, shard, ws, ws_bytes, s));
+  NF4_TRY(prepare(x, c, shard, ws, ws_bytes, s, tables_ready));
   // checkpoint recompute (keeps g and u for the SwiGLU backward)
   NF4_TRY(forward_body(x, lora, X, nullptr, true, s));
   const int M = x.M, H = x.H, I = x.I;

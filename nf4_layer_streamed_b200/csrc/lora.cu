@@ -5,18 +5,17 @@
 // §2.2 check 2 (LoRA gradients nonzero in every layer): the adapter adds
 // s (x A^T) B^T to the q and v projections (s = alpha / r) and trains A and B.  The
 // up-projection is folded into the q/k/v GEMM as an extra 64-wide reduction block;
-// this file holds the skinny products around it, all of them HBM-bound, in one launch
-// per forward and three per backward:
+// this file holds the skinny products of the backward, all of them HBM-bound, in three
+// launches (the down-projection t = [h1 A_q^T | h1 A_v^T] of the forward is a second
+// output of the input RMSNorm's launch, body.cu):
 //
-//   k_lora_down: t = [h1 A_q^T | h1 A_v^T] (bf16, the extra operand of the q/k/v GEMM)
-//     from h1 and the bf16 adapter rows, which the input RMSNorm's launch converts
-//     from the fp32 masters together with the other adapter operands (body.cu);
 //   k_lora_bwd_partial: per (128-row block, column chunk of dq or dv) the partial sums
 //     of dB = s dX^T t (over the rows) and of dt = s dX B (over the columns), from one
 //     read of dX;
 //   k_lora_bwd_reduce: dB (partials added in row-block order) and dt (partials added
 //     in column-chunk order, rounded to bf16: the extra operand of the dL/dx GEMM);
-//   k_lora_bwd_da: dA = dt^T h1, one block per 32 columns of h1 over all rows.
+//   k_lora_bwd_da: dA = dt^T h1, a cluster of eight blocks per 64 columns of h1, each
+//     over an eighth of the rows, the partials added across the cluster in shared memory.
 //
 // The products run on the warp-level bf16 tensor-core instruction (mma.sync m16n8k16);
 // every reduction is in a fixed order, so each result is bit-reproducible and a
@@ -54,92 +53,6 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
 
 __device__ __forceinline__ void zero16(uint32_t addr) { st_shared_v4(addr, 0u, 0u, 0u, 0u); }
 
-// ============================================================================ forward
-constexpr int LD_ROWS = 16, LD_THREADS = 256, LD_WARPS = 8, LD_KC = 128;  // rows per block, k-chunk
-constexpr int LD_LS = LD_KC + 8;                                         // smem row stride (elements)
-constexpr int LD_STAGES = 4;
-constexpr int LD_STAGE_BYTES = (LD_ROWS + 32) * LD_LS * 2;
-constexpr int LD_SMEM = LD_STAGES * LD_STAGE_BYTES;
-
-// One block: 16 token rows.  The reduction over H runs in chunks of 128 columns through a
-// ring of LD_STAGES shared-memory stages filled by cp.async: the h1 rows and the 32 bf16
-// adapter rows (A_q, A_v of adn).  Warp w takes the chunk's k-step w, so it accumulates
-// the global k-steps w, w + 8, ...; the eight partial products are then added in warp
-// order.
-__global__ void __launch_bounds__(LD_THREADS) k_lora_down(const __nv_bfloat16* __restrict__ h1, int M, int H,
-                                                          const __nv_bfloat16* __restrict__ adn,
-                                                          __nv_bfloat16* __restrict__ tpad) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  const int t = threadIdx.x, warp = t >> 5, lane = t & 31, g4 = lane >> 2, t4 = lane & 3;
-  const int m0 = blockIdx.x * LD_ROWS;
-  const int n_chunks = (H + LD_KC - 1) / LD_KC;
-  auto tile = [&](int b) { return reinterpret_cast<__nv_bfloat16*>(smem + (size_t)b * LD_STAGE_BYTES); };
-  // chunk c into stage b: rows 0-15 h1, rows 16-47 adapter rows 0-31 (16 pieces each)
-  auto stage = [&](int c, int b) {
-    for (int e = t; e < (LD_ROWS + 32) * 16; e += LD_THREADS) {
-      const int r = e >> 4, q = e & 15, col = c * LD_KC + q * 8;
-      const uint32_t dst = smem_u32(tile(b) + r * LD_LS + q * 8);
-      const int m = m0 + r;
-      if (col >= H || (r < LD_ROWS && m >= M))
-        zero16(dst);
-      else if (r < LD_ROWS)
-        cp_async16(dst, h1 + (size_t)m * H + col);
-      else
-        cp_async16(dst, adn + (size_t)(r - LD_ROWS) * H + col);
-    }
-    asm volatile("cp.async.commit_group;" ::: "memory");
-  };
-  float acc[4][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-  for (int c = 0; c < LD_STAGES - 1; ++c) {
-    if (c < n_chunks)
-      stage(c, c);
-    else
-      asm volatile("cp.async.commit_group;" ::: "memory");
-  }
-  for (int c = 0; c < n_chunks; ++c) {
-    const int b = c % LD_STAGES;
-    asm volatile("cp.async.wait_group %0;" ::"n"(LD_STAGES - 2) : "memory");
-    __syncthreads();  // chunk c has landed for every thread; the stage of chunk c - 1 is free
-    if (c + LD_STAGES - 1 < n_chunks)
-      stage(c + LD_STAGES - 1, (c + LD_STAGES - 1) % LD_STAGES);
-    else
-      asm volatile("cp.async.commit_group;" ::: "memory");
-    if (c * LD_KC + warp * 16 < H) {
-      const __nv_bfloat16* T = tile(b);
-      uint32_t a0, a1, a2, a3, b0, b1, b2, b3, b4, b5, b6, b7;
-      ldsm4(smem_u32(T + (lane & 15) * LD_LS + warp * 16 + (lane >> 4) * 8), a0, a1, a2, a3);
-      const int br = (lane & 7) + (lane >> 4) * 8, bc = warp * 16 + ((lane >> 3) & 1) * 8;
-      ldsm4(smem_u32(T + (LD_ROWS + br) * LD_LS + bc), b0, b1, b2, b3);
-      ldsm4(smem_u32(T + (LD_ROWS + 16 + br) * LD_LS + bc), b4, b5, b6, b7);
-      mma16816(acc[0], a0, a1, a2, a3, b0, b1);
-      mma16816(acc[1], a0, a1, a2, a3, b2, b3);
-      mma16816(acc[2], a0, a1, a2, a3, b4, b5);
-      mma16816(acc[3], a0, a1, a2, a3, b6, b7);
-    }
-  }
-  asm volatile("cp.async.wait_all;" ::: "memory");
-  __syncthreads();
-  float* red = reinterpret_cast<float*>(smem);  // the stages are free now
-  float* R = red + warp * (LD_ROWS * 32);
-#pragma unroll
-  for (int nt = 0; nt < 4; ++nt) {
-    R[g4 * 32 + nt * 8 + 2 * t4] = acc[nt][0];
-    R[g4 * 32 + nt * 8 + 2 * t4 + 1] = acc[nt][1];
-    R[(g4 + 8) * 32 + nt * 8 + 2 * t4] = acc[nt][2];
-    R[(g4 + 8) * 32 + nt * 8 + 2 * t4 + 1] = acc[nt][3];
-  }
-  __syncthreads();
-  for (int e = t; e < LD_ROWS * 64; e += LD_THREADS) {
-    const int r = e >> 6, cc = e & 63, m = m0 + r;
-    if (m >= M) continue;
-    float v = 0.f;
-    if (cc < 32)
-      for (int w = 0; w < LD_WARPS; ++w) v += red[w * (LD_ROWS * 32) + r * 32 + cc];
-    tpad[(size_t)m * 64 + cc] = __float2bfloat16_rn(v);
-  }
-}
 
 // ============================================================================ backward
 constexpr int LB_ROWS = 128, LB_THREADS = 256;
@@ -293,29 +206,40 @@ __global__ void __launch_bounds__(LB_THREADS) k_lora_bwd_reduce(const __grid_con
   a.dtpad[(size_t)m * 64 + 32 + c] = __float2bfloat16_rn(0.f);
 }
 
-// dA = dt^T h1: one block per 64 columns of h1, over all M rows in chunks of 128 through
-// a ring of DA_STAGES cp.async stages.  Warp w takes the chunk's k-step w (16 rows), so it
-// accumulates the rows 16 w .. of every chunk; the eight partial products are added in
-// warp order.
-constexpr int DA_COLS = 64, DA_ROWS = 128, DA_DS = 40, DA_HS = DA_COLS + 8, DA_STAGES = 4;
+// dA = dt^T h1.  A cluster of DA_SPLIT CTAs per 64 columns of h1: CTA y of the cluster
+// takes the row range [y R, (y + 1) R) (R = M / DA_SPLIT rounded up to whole 64-row
+// chunks), streamed through three cp.async stages.  Warp w takes rows 16 w .. 16 w + 15 of
+// every chunk, the four warp partials are added in warp order, and the
+// cluster's eight partials are added in CTA order through distributed shared memory,
+// CTA y producing output rows 4 y .. 4 y + 3.  The sum order is fixed by M alone.
+constexpr int DA_COLS = 64, DA_ROWS = 64, DA_DS = 40, DA_HS = DA_COLS + 8, DA_STAGES = 3;
+constexpr int DA_SPLIT = 8, DA_THREADS = 128, DA_WARPS = DA_THREADS / 32;
+constexpr int DA_KSTEPS = DA_ROWS / (16 * DA_WARPS);  // k-steps of 16 rows per warp and chunk
 constexpr int DA_PIECES = 4 + DA_COLS / 8;  // 16-byte pieces per row: dt (32 columns), h1
 constexpr int DA_STAGE_BYTES = DA_ROWS * (DA_DS + DA_HS) * 2;
-constexpr int DA_SMEM = DA_STAGES * DA_STAGE_BYTES;
+constexpr int DA_RED_BYTES = DA_WARPS * 32 * DA_COLS * 4;  // warp partials
+constexpr int DA_SMEM = DA_STAGES * DA_STAGE_BYTES;  // 42 KB: five CTAs per SM
+static_assert(DA_RED_BYTES + 32 * DA_COLS * 4 <= DA_SMEM, "partials fit in the stages");
+static_assert(32 % DA_SPLIT == 0, "output rows split evenly over the cluster");
 
-__global__ void __launch_bounds__(LB_THREADS) k_lora_bwd_da(const __grid_constant__ LoraBwdArgs a) {
+__global__ void __cluster_dims__(1, DA_SPLIT, 1) __launch_bounds__(DA_THREADS)
+    k_lora_bwd_da(const __grid_constant__ LoraBwdArgs a) {
   extern __shared__ __align__(16) uint8_t smem[];
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31, g4 = lane >> 2, t4 = lane & 3;
   const int c0 = blockIdx.x * DA_COLS;
-  const int n_chunks = (a.M + DA_ROWS - 1) / DA_ROWS;
+  const int y = (int)cluster_ctarank();
+  const int R = ((a.M + DA_SPLIT - 1) / DA_SPLIT + DA_ROWS - 1) / DA_ROWS * DA_ROWS;
+  const int r0 = y * R, r1 = min(a.M, r0 + R);
+  const int n_chunks = r1 > r0 ? (r1 - r0 + DA_ROWS - 1) / DA_ROWS : 0;
   auto ds = [&](int b) { return reinterpret_cast<__nv_bfloat16*>(smem + (size_t)b * DA_STAGE_BYTES); };
   auto hs = [&](int b) {
     return reinterpret_cast<__nv_bfloat16*>(smem + (size_t)b * DA_STAGE_BYTES + DA_ROWS * DA_DS * 2);
   };
   auto stage = [&](int ch, int b) {  // 128 rows x (4 pieces of dt + DA_COLS / 8 pieces of h1)
-    for (int i = t; i < DA_ROWS * DA_PIECES; i += LB_THREADS) {
-      const int r = i / DA_PIECES, q = i % DA_PIECES, m = ch * DA_ROWS + r;
+    for (int i = t; i < DA_ROWS * DA_PIECES; i += DA_THREADS) {
+      const int r = i / DA_PIECES, q = i % DA_PIECES, m = r0 + ch * DA_ROWS + r;
       const uint32_t dst = q < 4 ? smem_u32(ds(b) + r * DA_DS + q * 8) : smem_u32(hs(b) + r * DA_HS + (q - 4) * 8);
-      if (m >= a.M)
+      if (m >= r1)
         zero16(dst);
       else if (q < 4)
         cp_async16(dst, a.dtpad + (size_t)m * 64 + q * 8);
@@ -338,55 +262,70 @@ __global__ void __launch_bounds__(LB_THREADS) k_lora_bwd_da(const __grid_constan
   }
   for (int ch = 0; ch < n_chunks; ++ch) {
     const int b = ch % DA_STAGES;
-    asm volatile("cp.async.wait_group %0;" ::"n"(DA_STAGES - 2) : "memory");
-    __syncthreads();  // chunk ch has landed; the stage of chunk ch - 1 is free
+    // the stage chunk ch + DA_STAGES - 1 goes to was last read for chunk ch - 1
+    __syncthreads();
     if (ch + DA_STAGES - 1 < n_chunks)
       stage(ch + DA_STAGES - 1, (ch + DA_STAGES - 1) % DA_STAGES);
     else
       asm volatile("cp.async.commit_group;" ::: "memory");
-    const int kr = warp * 16;  // this warp's 16 rows of the chunk
-    uint32_t af[2][4];
+    asm volatile("cp.async.wait_group %0;" ::"n"(DA_STAGES - 1) : "memory");
+    __syncthreads();  // chunk ch has landed for every thread
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {  // dA rows 16 mt ..: A = dt^T from the dt rows
-      const int m = kr + (lane & 7) + (lane >> 4) * 8, n = mt * 16 + ((lane >> 3) & 1) * 8;
-      ldsm4t(smem_u32(ds(b) + m * DA_DS + n), af[mt][0], af[mt][1], af[mt][2], af[mt][3]);
-    }
+    for (int kk = 0; kk < DA_KSTEPS; ++kk) {
+      const int kr = (warp * DA_KSTEPS + kk) * 16;  // 16 rows of the chunk
+      uint32_t af[2][4];
 #pragma unroll
-    for (int h = 0; h < NT / 2; ++h) {  // h1 columns 16 h ..: B fragments of two n8 tiles
-      uint32_t b0, b1, b2, b3;
-      const int m = kr + (lane & 7) + ((lane >> 3) & 1) * 8, n = h * 16 + (lane >> 4) * 8;
-      ldsm4t(smem_u32(hs(b) + m * DA_HS + n), b0, b1, b2, b3);
+      for (int mt = 0; mt < 2; ++mt) {  // dA rows 16 mt ..: A = dt^T from the dt rows
+        const int m = kr + (lane & 7) + (lane >> 4) * 8, n = mt * 16 + ((lane >> 3) & 1) * 8;
+        ldsm4t(smem_u32(ds(b) + m * DA_DS + n), af[mt][0], af[mt][1], af[mt][2], af[mt][3]);
+      }
 #pragma unroll
-      for (int mt = 0; mt < 2; ++mt) {
-        mma16816(acc[mt][2 * h], af[mt][0], af[mt][1], af[mt][2], af[mt][3], b0, b1);
-        mma16816(acc[mt][2 * h + 1], af[mt][0], af[mt][1], af[mt][2], af[mt][3], b2, b3);
+      for (int h = 0; h < NT / 2; ++h) {  // h1 columns 16 h ..: B fragments of two n8 tiles
+        uint32_t b0, b1, b2, b3;
+        const int m = kr + (lane & 7) + ((lane >> 3) & 1) * 8, n = h * 16 + (lane >> 4) * 8;
+        ldsm4t(smem_u32(hs(b) + m * DA_HS + n), b0, b1, b2, b3);
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+          mma16816(acc[mt][2 * h], af[mt][0], af[mt][1], af[mt][2], af[mt][3], b0, b1);
+          mma16816(acc[mt][2 * h + 1], af[mt][0], af[mt][1], af[mt][2], af[mt][3], b2, b3);
+        }
       }
     }
   }
   asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
   float* red = reinterpret_cast<float*>(smem);  // the stages are free now
-  float* R = red + warp * (32 * DA_COLS);
+  float* P = reinterpret_cast<float*>(smem + DA_RED_BYTES);  // this CTA's [32][DA_COLS] partial
+  float* R_ = red + warp * (32 * DA_COLS);
 #pragma unroll
   for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const int row = mt * 16 + g4, col = nt * 8 + 2 * t4;
-      R[row * DA_COLS + col] = acc[mt][nt][0];
-      R[row * DA_COLS + col + 1] = acc[mt][nt][1];
-      R[(row + 8) * DA_COLS + col] = acc[mt][nt][2];
-      R[(row + 8) * DA_COLS + col + 1] = acc[mt][nt][3];
+      R_[row * DA_COLS + col] = acc[mt][nt][0];
+      R_[row * DA_COLS + col + 1] = acc[mt][nt][1];
+      R_[(row + 8) * DA_COLS + col] = acc[mt][nt][2];
+      R_[(row + 8) * DA_COLS + col + 1] = acc[mt][nt][3];
     }
   __syncthreads();
-  for (int e = t; e < 32 * DA_COLS; e += LB_THREADS) {
-    const int row = e / DA_COLS, col = c0 + e % DA_COLS;
+  for (int e = t; e < 32 * DA_COLS; e += DA_THREADS) {
     float v = 0.f;
-    for (int w = 0; w < 8; ++w) v += red[w * (32 * DA_COLS) + e];
-    if (row < 16)
-      a.dA_q[(size_t)row * a.H + col] = v;
-    else
-      a.dA_v[(size_t)(row - 16) * a.H + col] = v;
+    for (int w = 0; w < DA_WARPS; ++w) v += red[w * (32 * DA_COLS) + e];
+    P[e] = v;
   }
+  cluster_sync_all();  // every CTA's partial is in its shared memory
+  constexpr int ROWS_PER_CTA = 32 / DA_SPLIT;
+  for (int e = t; e < ROWS_PER_CTA * DA_COLS; e += DA_THREADS) {
+    const int row = y * ROWS_PER_CTA + e / DA_COLS, col = e % DA_COLS;
+    const uint32_t local = smem_u32(P + row * DA_COLS + col);
+    float v = 0.f;
+    for (int c = 0; c < DA_SPLIT; ++c) v += ld_cluster_f32(mapa_shared(local, (uint32_t)c));
+    if (row < 16)
+      a.dA_q[(size_t)row * a.H + c0 + col] = v;
+    else
+      a.dA_v[(size_t)(row - 16) * a.H + c0 + col] = v;
+  }
+  cluster_sync_all();  // no CTA leaves while another still reads its partial
 }
 
 // Column chunk of k_lora_bwd_partial: 128 where it divides both widths (so that a
@@ -446,17 +385,6 @@ int allow_smem(const void* kernel, size_t bytes) {
 
 size_t lora_partial_bytes(int M, int H, int qd, int kvd) { return bwd_shape(M, H, qd, kvd).total; }
 
-int lora_down(const __nv_bfloat16* h1, int M, int H, const __nv_bfloat16* adn, __nv_bfloat16* tpad, cudaStream_t s) {
-  if (H % 16) return fail(NF4LS_SHAPE, "lora_down: H %d", H);
-  if (M <= 0) return NF4LS_OK;
-  static_assert(LD_WARPS * LD_ROWS * 32 * 4 <= LD_SMEM, "partials fit in the stages");
-  NF4_TRY(allow_smem((const void*)k_lora_down, LD_SMEM));
-  k_lora_down<<<(M + LD_ROWS - 1) / LD_ROWS, LD_THREADS, LD_SMEM, s>>>(h1, M, H, adn, tpad);
-  note_launch();
-  NF4_CUDA_TRY(cudaGetLastError());
-  return NF4LS_OK;
-}
-
 int lora_bwd(const __nv_bfloat16* dqkv, int ld, int vcol, int M, int H, int qd, int kvd, const __nv_bfloat16* tpad,
              const __nv_bfloat16* bqt, const __nv_bfloat16* bvt, const __nv_bfloat16* h1, float scale,
              __nv_bfloat16* dtpad, const nf4ls_lora_grads* g, void* part, cudaStream_t s) {
@@ -496,9 +424,8 @@ int lora_bwd(const __nv_bfloat16* dqkv, int ld, int vcol, int M, int H, int qd, 
   note_launch();
   k_lora_bwd_reduce<<<sh.n_db_blocks + (M + 7) / 8, LB_THREADS, 0, s>>>(a);
   note_launch();
-  static_assert(8 * 32 * DA_COLS * 4 <= DA_SMEM, "partials fit in the stages");
   NF4_TRY(allow_smem((const void*)k_lora_bwd_da, DA_SMEM));
-  k_lora_bwd_da<<<H / DA_COLS, LB_THREADS, DA_SMEM, s>>>(a);
+  k_lora_bwd_da<<<dim3(H / DA_COLS, DA_SPLIT), DA_THREADS, DA_SMEM, s>>>(a);
   note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;

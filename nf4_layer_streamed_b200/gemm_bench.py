@@ -189,6 +189,7 @@ def main(argv=None):
     ap.add_argument("--once", action="store_true")
     ap.add_argument("--single", action="store_true", help="one CTA per tile instead of CTA pairs")
     ap.add_argument("--quant", action="store_true", help="also time the quantiser and dequantiser")
+    ap.add_argument("--quant-only", action="store_true", help="time only the quantiser and dequantiser")
     ap.add_argument("--half", type=int, default=0,
                     help="pair tile height: 0 auto, 1 512 tokens, 2 256 tokens, 3 last partial wave as 256")
     ap.add_argument("--layer", type=int, default=0, metavar="BATCH",
@@ -202,6 +203,9 @@ def main(argv=None):
     api.set_gemm_half(a.half)
     if a.attention:
         run_attention(a.attention, a.once)
+        return
+    if a.quant_only:
+        run_quant(1 if a.once else 10)
         return
     if a.layer:
         run_layer(a.layer, a.once, shape_name=a.layer_shape)

@@ -11,12 +11,14 @@ GPU-to-GPU comparisons.
   Llama-8B-shaped model at batch 1 x 128 with random LoRA B, first step, with the
   head resident and with the head streamed in vocab chunks (16384 rows, a ragged
   last chunk of 13568): loss within 1e-3 relative, dA / dB of both layers within
-  2e-2 max|ref| or, where larger, within the oracle's own bf16 noise floor: the
-  largest change that the oracle's bf16 roundings make to that gradient (the oracle
-  run with and without them).  At this configuration (a random-init model, uniform
-  targets, 128 tokens) the last layer's LoRA gradients are ill-conditioned: the
-  roundings alone move them by about 3% of max|ref|, so any bf16 implementation
-  differs from the rounded oracle by that much.  This stands in for the first step
+  2e-2 max|ref| or, where larger, within twice the oracle's own bf16 noise floor:
+  the largest change that the oracle's bf16 roundings make to that gradient (the
+  oracle run with and without them).  At this configuration (a random-init model,
+  uniform targets, 128 tokens) the last layer's LoRA gradients are ill-conditioned:
+  the roundings alone move them by about 3% of max|ref|.  The kernels round at the
+  same points, not always to the same neighbour, so they sit about as far from the
+  unrounded result as the rounded oracle does; the two differ by at most the sum of
+  those distances, twice the floor.  This stands in for the first step
   of the 32-layer 8B workload, whose oracle run would take far longer than a test
   should.
 """
@@ -122,6 +124,6 @@ def test_llama8b_untied_two_layers_first_step_against_oracle(head_chunk_rows):
     for i in range(wl.n_layers):
         for k in ("dA_q", "dB_q", "dA_v", "dB_v"):
             ref = og[i][k]
-            tol = max(TOL, floor[i][k] / np.max(np.abs(ref)))
+            tol = max(TOL, 2.0 * floor[i][k] / np.max(np.abs(ref)))
             close(grads[i][k], ref, tol, f"layer {i} {k} (noise floor {floor[i][k]:.3e})")
             assert torch.count_nonzero(grads[i][k]) > 0
