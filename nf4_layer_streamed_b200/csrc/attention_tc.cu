@@ -31,8 +31,41 @@ constexpr int TT = 128;                   // query / key tile
 constexpr int TILE_BYTES = TT * 128 * 2;  // 128 rows x 128 dims bf16 = 32 KB
 constexpr int ATOM = TILE_BYTES / 2;      // one 64-dim (or 64-key) swizzle atom: 16 KB
 
+// Tiled 2D store of a box from shared memory (the map's 128-byte swizzled layout) to
+// global memory, in this thread's bulk async-group.  c0 * 2 bytes is a multiple of 16.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map), "r"(src),
+               "r"(c0), "r"(c1)
+               : "memory");
+}
+// Closes this thread's bulk async-group and waits until its stores have read shared memory.
+__device__ __forceinline__ void tma_store_drain() {
+  asm volatile("cp.async.bulk.commit_group;\ncp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// One thread's 32 fp32 values (columns 32 c .. 32 c + 31 of its row r of a 128 x 128 tile),
+// times sc, as bf16 into the tile's two 128-byte swizzled 64-column atoms at tile.
+__device__ __forceinline__ void stage_row32(uint32_t tile, int r, int c, const uint32_t (&v)[32], float sc) {
+  const uint32_t row = tile + (uint32_t)(c >> 1) * (TT * 128) + (uint32_t)r * 128;
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) {
+    const int chunk = (c & 1) * 4 + q4;  // 16-byte chunk of the 128-byte row
+    st_shared_v4(row + ((uint32_t)(chunk ^ (r & 7)) << 4),
+                 pack_bf16x2(__uint_as_float(v[8 * q4]) * sc, __uint_as_float(v[8 * q4 + 1]) * sc),
+                 pack_bf16x2(__uint_as_float(v[8 * q4 + 2]) * sc, __uint_as_float(v[8 * q4 + 3]) * sc),
+                 pack_bf16x2(__uint_as_float(v[8 * q4 + 4]) * sc, __uint_as_float(v[8 * q4 + 5]) * sc),
+                 pack_bf16x2(__uint_as_float(v[8 * q4 + 6]) * sc, __uint_as_float(v[8 * q4 + 7]) * sc));
+  }
+}
+
+__device__ __forceinline__ void stage_row32(uint32_t tile, int r, int c, const float (&v)[32]) {
+  uint32_t u[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(v[i]);
+  stage_row32(tile, r, c, u, 1.0f);
+}
+
 struct AttnTcParams {
-  CUtensorMap tq, tk, tv;  // [rows, cols] bf16, box 64 cols x 128 rows, 128-byte swizzle
+  CUtensorMap tq, tk, tv, to;  // [rows, cols] bf16, box 64 cols x 128 rows, 128-byte swizzle (to: output)
   __nv_bfloat16* o;
   float* lse;
   int ldo, seq, nq, nkv;
@@ -273,24 +306,28 @@ __global__ void __launch_bounds__(F_THREADS, 2) k_attn_fwd_tc(const __grid_const
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
     }
+    // O / sum through the freed Q tile's shared memory and two TMA stores (coalesced rows);
+    // all four warps reach the barrier, the store is issued only when no wait failed
     if (ok && __all_sync(0xffffffffu, mbar_wait(o_full, (nk - 1) & 1, abort_flag, p.err, KID_ATTN, 29))) {
       tc_fence_after();
       const float inv = 1.0f / l_run;
-      uint4* dst = reinterpret_cast<uint4*>(p.o + (size_t)(row0 + qpos) * p.ldo + h * 128);
+      const uint32_t tile = smem_u32(base + F_OFF_Q);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tmem_ld32(trow + 128 + c * 32, v);
+      for (int c = 0; c < 4; c += 2) {
+        uint32_t v[2][32];
+        tmem_ld32(trow + 128 + c * 32, v[0]);
+        tmem_ld32(trow + 128 + c * 32 + 32, v[1]);
         tmem_wait_ld();
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4)
-          dst[c * 4 + q4] =
-              make_uint4(pack_bf16x2(__uint_as_float(v[8 * q4]) * inv, __uint_as_float(v[8 * q4 + 1]) * inv),
-                         pack_bf16x2(__uint_as_float(v[8 * q4 + 2]) * inv, __uint_as_float(v[8 * q4 + 3]) * inv),
-                         pack_bf16x2(__uint_as_float(v[8 * q4 + 4]) * inv, __uint_as_float(v[8 * q4 + 5]) * inv),
-                         pack_bf16x2(__uint_as_float(v[8 * q4 + 6]) * inv, __uint_as_float(v[8 * q4 + 7]) * inv));
+        stage_row32(tile, r, c, v[0], inv);
+        stage_row32(tile, r, c + 1, v[1], inv);
       }
       p.lse[((size_t)b * p.nq + h) * p.seq + qpos] = (m_run + log2f(l_run)) * 0.6931471805599453f;
+    }
+    fence_proxy_async_smem();
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (threadIdx.x == 0 && !*abort_flag) {
+      for (int j = 0; j < 2; ++j) tma_store_2d(&p.to, smem_u32(base + F_OFF_Q + j * ATOM), h * 128 + 64 * j, row0 + qt * TT);
+      tma_store_drain();
     }
   }
 
@@ -310,21 +347,25 @@ __global__ void __launch_bounds__(F_THREADS, 2) k_attn_fwd_tc(const __grid_const
 }
 
 // ------------------------------------------------------------------------------ backward
-// dQ (per query tile and head) and dK, dV (per key tile and kv head) on tcgen05, in
-// blocks of 128 rows by 64 columns ("items"), two items in flight: while eight warps
-// turn item i's scores into P and dS, the tensor core already computes item i + 1's.
-//   query side, item = 64 keys:    S = Q K^T, dP = dO V^T (N = 64); after the
-//     elementwise step dQ += dS K (dS from TMEM as the A operand, K = 64).
-//   key side, item = 64 queries:   S^T = K Q^T, dP^T = V dO^T; then dV += P^T dO and
+// dQ (per query tile and head) and dK, dV (per key tile and kv head) on tcgen05, one
+// 128 x 128 block ("item") at a time:
+//   query side, item = one key tile:   S = Q K^T, dP = dO V^T (N = 128); after the
+//     elementwise step dQ += dS K (dS from TMEM as the A operand, K = 128).
+//   key side, item = one query tile:   S^T = K Q^T, dP^T = V dO^T; then dV += P^T dO and
 //     dK += dS^T Q.
-// P = 2^(S log2e / sqrt(d) - lse log2e) (causal mask), dS = P (dP - delta).  TMEM holds
-// two item buffers (S and dP, 64 columns each) and the accumulators; P / dS are written
-// back as bf16 (two per 32-bit column) over the scores that the same warp has read,
-// warp g of a lane quarter taking the item's columns [32 g, 32 g + 32).  The query-side
-// kernel also forms delta = rowsum(dO * O) for its rows and writes it for the key side,
-// which runs after it.  Accumulation runs in a fixed order (query side: key tiles in
-// order; key side: query heads of the group, then query tiles), so results are
-// bit-reproducible.
+// Every product is M = 128, N = 128: a tcgen05.mma of N = 64 runs at about 60% of the
+// tensor core's rate (measured), one of N >= 128 at its full rate, so a whole tile per
+// item and one item buffer (the S and dP blocks and the two accumulators fill the 512
+// TMEM columns) beat half tiles with two buffers in flight.
+// P = 2^(S log2e / sqrt(d) - lse log2e) (causal mask), dS = P (dP - delta).  The eight
+// elementwise warps take a lane quarter and 64 columns each, in two 32-column chunks;
+// P / dS are written back as bf16 (two per 32-bit column) over scores that the same
+// warp has already read: chunk h of warp half g packs into columns 64 g + 16 h ..
+// of its block, so the A operand of k-step ks (16 rows of the reduction) sits at
+// column 64 (ks / 4) + 8 (ks % 4).  The query-side kernel also forms
+// delta = rowsum(dO * O) for its rows and writes it for the key side, which runs after
+// it.  Accumulation runs in a fixed order (query side: key tiles in order; key side:
+// query heads of the group, then query tiles), so results are bit-reproducible.
 
 // 1D bulk copy global -> shared completing transaction bytes on bar (16-byte multiples).
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -336,6 +377,7 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 
 struct AttnBwdParams {
   CUtensorMap tq, tk, tv, tdo, to;  // box 64 cols x 128 rows, 128-byte swizzle (to: the output O)
+  CUtensorMap tdq, tdk, tdv;        // the gradients, same boxes (TMA stores)
   const float* lse;
   float* delta;                 // written by the query side, read by the key side
   __nv_bfloat16* dq;
@@ -358,15 +400,15 @@ constexpr int SMEM_BWD = 1024 + B_OFF_BAR + 256;
 
 __device__ __forceinline__ void bar_ew() { asm volatile("bar.sync 1, %0;" ::"n"(B_EW) : "memory"); }
 
-// TMEM column of the A operand of 16-row step ks (0-3) of an item buffer whose first
-// column is c0: warp half g wrote its 32 rows' packed values to columns c0 + 32 g ..
-__device__ __forceinline__ uint32_t packed_col(uint32_t c0, int ks) { return c0 + (ks >> 1) * 32 + (ks & 1) * 8; }
+// TMEM column of the A operand of 16-row step ks (0-7) of a block whose first column is
+// c0: warp half g packed its 64 rows' values to columns c0 + 64 g .. c0 + 64 g + 31.
+__device__ __forceinline__ uint32_t packed_col(uint32_t c0, int ks) { return c0 + (ks >> 2) * 64 + (ks & 3) * 8; }
 
 // QUERY side: dQ of one 128-query tile of one query head.  The Q and dO tiles are
 // copied once into TMEM (bf16 pairs, one query row per lane), so that S = Q K^T and
-// dP = dO V^T take their A operand from TMEM and read only the 64-key halves of K and V
-// from shared memory: an N = 64 product with both operands in shared memory would read
-// 6 KB per 32 tensor-core cycles, more than shared memory delivers.
+// dP = dO V^T take their A operand from TMEM and read only K and V from shared memory
+// (4 KB per 64 tensor-core cycles instead of 8 KB, which is all that shared memory
+// delivers, while the next K and V tiles land in it).
 __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_constant__ AttnBwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -374,8 +416,8 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
   uint64_t* q_full = bars;          // Q, dO
   uint64_t* kv_full = bars + 1;     // 2 stages
   uint64_t* kv_empty = bars + 3;    // 2
-  uint64_t* sd_full = bars + 5;     // 2 item buffers
-  uint64_t* p_full = bars + 7;      // 2
+  uint64_t* sd_full = bars + 5;     // S and dP of the item are in TMEM
+  uint64_t* p_full = bars + 6;      // dS of the item is in TMEM (one arrival per elementwise warp)
   uint64_t* acc_full = bars + 9;
   uint64_t* drain = bars + 10;
   uint64_t* qa_full = bars + 11;    // Q and dO are in TMEM (one arrival per elementwise warp)
@@ -385,7 +427,7 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = gridDim.x - 1 - blockIdx.x, h = blockIdx.y, b = blockIdx.z;  // longest rows first
   const int kvh = h / (p.nq / p.nkv);
-  const int n_kt = qt + 1, n_it = 2 * n_kt;  // key tiles at or before the diagonal, halves
+  const int n_kt = qt + 1;  // key tiles at or before the diagonal
   const int row0 = b * p.seq;
 
   if (threadIdx.x == 0) {
@@ -393,9 +435,9 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
     for (int i = 0; i < 2; ++i) {
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
-      mbar_init(&sd_full[i], 1);
-      mbar_init(&p_full[i], 8);
     }
+    mbar_init(sd_full, 1);
+    mbar_init(p_full, B_EW / 32);
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
     mbar_init(qa_full, B_EW / 32);
@@ -409,7 +451,7 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  // item buffers [0,128) and [128,256) (S | dP), dQ [256,384), Q [384,448), dO [448,512)
+  // S [0,128), dP [128,256) (dS packed over it), dQ [256,384), Q [384,448), dO [448,512)
   const uint32_t tmem = *tmem_slot;
   constexpr uint32_t T_Q = 384, T_DO = 448;
 
@@ -444,51 +486,43 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
       }
     }
   } else if (warp == B_MMA) {
-    constexpr uint32_t idesc_s = idesc_bf16(128, 64, false);   // S, dP: N = 64 keys
+    constexpr uint32_t idesc_s = idesc_bf16(128, 128, false);  // S, dP: N = 128 keys
     constexpr uint32_t idesc_a = idesc_bf16(128, 128, true);   // dQ += dS K: K N-major
     bool ok = __all_sync(0xffffffffu, mbar_wait(qa_full, 0, abort_flag, p.err, KID_ATTN, 42)) && !*abort_flag;
-    // item it: key tile it / 2, half it % 2, TMEM buffer it % 2
-    auto second = [&](int it) -> bool {  // dQ += dS_it K_half(it)
-      if (!__all_sync(0xffffffffu, mbar_wait(&p_full[it & 1], (it >> 1) & 1, abort_flag, p.err, KID_ATTN, 44)))
-        return false;
+    auto dq_product = [&](int kt) -> bool {  // dQ += dS_kt K_kt, then the K/V stage is free
+      if (!__all_sync(0xffffffffu, mbar_wait(p_full, kt & 1, abort_flag, p.err, KID_ATTN, 44))) return false;
       tc_fence_after();
       if (lane == 0) {
-        const int kt = it >> 1, hh = it & 1;
         const uint32_t sK = smem_u32(base + B_OFF_RING + (kt & 1) * 2 * TILE_BYTES);
-        const uint32_t c0 = (uint32_t)(it & 1) * 128 + 64;  // dS over the dP columns
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          umma_bf16_ta(tmem + 256, tmem + packed_col(c0, ks), sdesc_sw128(sK + hh * 8192 + ks * 2048, ATOM, 1024),
-                       idesc_a, (it | ks) ? 1u : 0u);
-        if (hh == 1) umma_commit(&kv_empty[kt & 1]);
+        for (int ks = 0; ks < 8; ++ks)  // 16 keys per step
+          umma_bf16_ta(tmem + 256, tmem + packed_col(128, ks), sdesc_sw128(sK + ks * 2048, ATOM, 1024), idesc_a,
+                       (kt | ks) ? 1u : 0u);
+        umma_commit(&kv_empty[kt & 1]);
       }
       __syncwarp();
       return true;
     };
-    for (int it = 0; ok && it < n_it; ++it) {
-      const int kt = it >> 1, hh = it & 1, bf = it & 1;
-      if (hh == 0 && !(ok = __all_sync(0xffffffffu, mbar_wait(&kv_full[kt & 1], (kt >> 1) & 1, abort_flag, p.err,
-                                                               KID_ATTN, 43))))
+    for (int kt = 0; ok && kt < n_kt; ++kt) {
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&kv_full[kt & 1], (kt >> 1) & 1, abort_flag, p.err, KID_ATTN,
+                                                   43))))
         break;
+      // the previous item's dS is read (issue order) before S and dP overwrite it
+      if (kt >= 1 && !(ok = dq_product(kt - 1))) break;
       tc_fence_after();
       if (lane == 0) {
         const uint32_t sK = smem_u32(base + B_OFF_RING + (kt & 1) * 2 * TILE_BYTES), sV = sK + TILE_BYTES;
-        // tcgen05.mma of one thread run in issue order: these may overwrite the dS of
-        // item it - 2, whose product was issued before
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {  // over the head dim: Q, dO columns 8 ks .. in TMEM
           const uint32_t off = (ks >> 2) * ATOM + (ks & 3) * 32;
-          umma_bf16_ta(tmem + bf * 128, tmem + T_Q + ks * 8, sdesc_sw128(sK + hh * 8192 + off, 16, 1024), idesc_s,
-                       ks ? 1u : 0u);
-          umma_bf16_ta(tmem + bf * 128 + 64, tmem + T_DO + ks * 8, sdesc_sw128(sV + hh * 8192 + off, 16, 1024),
-                       idesc_s, ks ? 1u : 0u);
+          umma_bf16_ta(tmem, tmem + T_Q + ks * 8, sdesc_sw128(sK + off, 16, 1024), idesc_s, ks ? 1u : 0u);
+          umma_bf16_ta(tmem + 128, tmem + T_DO + ks * 8, sdesc_sw128(sV + off, 16, 1024), idesc_s, ks ? 1u : 0u);
         }
-        umma_commit(&sd_full[bf]);
+        umma_commit(sd_full);
       }
       __syncwarp();
-      if (it >= 1 && !(ok = second(it - 1))) break;
     }
-    if (ok) ok = second(n_it - 1);
+    if (ok) ok = dq_product(n_kt - 1);
     if (ok && lane == 0) umma_commit(acc_full);
     __syncwarp();
   } else {
@@ -537,50 +571,52 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
     if (ok && g == 0) p.delta[li] = dl;
     const float lse2 = p.lse[li] * 1.4426950408889634f;
     const float sl = p.scale_log2;
-    for (int it = 0; ok && it < n_it; ++it) {
-      const int bf = it & 1;
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sd_full[bf], (it >> 1) & 1, abort_flag, p.err, KID_ATTN, 46))))
-        break;
+    for (int kt = 0; ok && kt < n_kt; ++kt) {
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(sd_full, kt & 1, abort_flag, p.err, KID_ATTN, 46)))) break;
       tc_fence_after();
-      uint32_t sv[32], dpv[32], dd[16];
-      tmem_ld32(trow + bf * 128 + g * 32, sv);
-      tmem_ld32(trow + bf * 128 + 64 + g * 32, dpv);
-      tmem_wait_ld();
-      const int key0 = (it >> 1) * TT + (it & 1) * 64 + g * 32;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        float ds[2];
+      for (int hc = 0; hc < 2; ++hc) {  // keys 64 g + 32 hc .. of the tile
+        uint32_t sv[32], dpv[32], dd[16];
+        tmem_ld32(trow + g * 64 + hc * 32, sv);
+        tmem_ld32(trow + 128 + g * 64 + hc * 32, dpv);
+        tmem_wait_ld();
+        const int key0 = kt * TT + g * 64 + hc * 32;
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int kj = key0 + 2 * j + e;
-          const float pe = kj <= qpos ? fast_exp2(fmaf(__uint_as_float(sv[2 * j + e]), sl, -lse2)) : 0.f;
-          ds[e] = pe * (__uint_as_float(dpv[2 * j + e]) - dl);
+        for (int j = 0; j < 16; ++j) {
+          float ds[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int kj = key0 + 2 * j + e;
+            const float pe = kj <= qpos ? fast_exp2(fmaf(__uint_as_float(sv[2 * j + e]), sl, -lse2)) : 0.f;
+            ds[e] = pe * (__uint_as_float(dpv[2 * j + e]) - dl);
+          }
+          dd[j] = pack_bf16x2(ds[0], ds[1]);
         }
-        dd[j] = pack_bf16x2(ds[0], ds[1]);
+        tmem_st16(trow + 128 + g * 64 + hc * 16, dd);  // over dP values this warp has read
       }
-      tmem_st16(trow + bf * 128 + 64 + g * 32, dd);  // over the dP values this warp has read
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[bf]);
+      if (lane == 0) mbar_arrive(p_full);
     }
+    // dQ through the freed ring's shared memory and two TMA stores (coalesced rows); every
+    // elementwise warp reaches the barrier, the store is issued only when no wait failed
     if (ok && __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, p.err, KID_ATTN, 47))) {
       tc_fence_after();
-      uint4* dst = reinterpret_cast<uint4*>(p.dq + (size_t)(row0 + qpos) * p.ld_dq + h * 128 + g * 64);
-      const float sc = p.scale;
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t v[32];
-        tmem_ld32(trow + 256 + g * 64 + c * 32, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4)
-          dst[c * 4 + q4] =
-              make_uint4(pack_bf16x2(__uint_as_float(v[8 * q4]) * sc, __uint_as_float(v[8 * q4 + 1]) * sc),
-                         pack_bf16x2(__uint_as_float(v[8 * q4 + 2]) * sc, __uint_as_float(v[8 * q4 + 3]) * sc),
-                         pack_bf16x2(__uint_as_float(v[8 * q4 + 4]) * sc, __uint_as_float(v[8 * q4 + 5]) * sc),
-                         pack_bf16x2(__uint_as_float(v[8 * q4 + 6]) * sc, __uint_as_float(v[8 * q4 + 7]) * sc));
-      }
+      uint32_t v[2][32];
+      tmem_ld32(trow + 256 + g * 64, v[0]);
+      tmem_ld32(trow + 256 + g * 64 + 32, v[1]);
+      tmem_wait_ld();
+      const uint32_t tile = smem_u32(base + B_OFF_RING);
+      stage_row32(tile, r, 2 * g, v[0], p.scale);
+      stage_row32(tile, r, 2 * g + 1, v[1], p.scale);
+    }
+    fence_proxy_async_smem();
+    bar_ew();
+    if (threadIdx.x == 0 && !*abort_flag) {
+      for (int j = 0; j < 2; ++j)
+        tma_store_2d(&p.tdq, smem_u32(base + B_OFF_RING + j * ATOM), h * 128 + 64 * j, row0 + qt * TT);
+      tma_store_drain();
     }
   }
   __syncthreads();
@@ -618,8 +654,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
   uint64_t* kv_full = bars;         // K, V
   uint64_t* qd_full = bars + 1;     // 2 stages (Q, dO, lse, delta of one (head, query tile))
   uint64_t* qd_empty = bars + 3;    // 2
-  uint64_t* sd_full = bars + 5;     // 2 item buffers
-  uint64_t* p_full = bars + 7;      // 2
+  uint64_t* sd_full = bars + 5;     // S^T and dP^T of the item are in TMEM
+  uint64_t* p_full = bars + 6;      // P^T and dS^T of the item are in TMEM (one arrival per warp)
   uint64_t* acc_full = bars + 9;
   uint64_t* drain = bars + 10;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
@@ -630,8 +666,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
   const uint32_t crank = cluster_ctarank();
   const int grp = p.nq / p.nkv, n_qt = p.seq / TT;
   const int hpc = (grp + 1) / 2, h_begin = (int)crank * hpc, h_count = min(grp, h_begin + hpc) - h_begin;
-  // (head, query tile) stages of this CTA, halves
-  const int per_head = n_qt - kt, n_st = h_count * per_head, n_it = 2 * n_st;
+  // (head, query tile) items of this CTA
+  const int per_head = n_qt - kt, n_st = h_count * per_head;
   const int row0 = b * p.seq;
 
   if (threadIdx.x == 0) {
@@ -639,9 +675,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&qd_full[i], 1);
       mbar_init(&qd_empty[i], 1);
-      mbar_init(&sd_full[i], 1);
-      mbar_init(&p_full[i], 8);
     }
+    mbar_init(sd_full, 1);
+    mbar_init(p_full, B_EW / 32);
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -654,7 +690,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;  // item buffers [0,128), [128,256) (S^T | dP^T), dV [256,384), dK [384,512)
+  const uint32_t tmem = *tmem_slot;  // S^T [0,128), dP^T [128,256) (P^T, dS^T packed over them), dV, dK
 
   if (warp == B_PROD) {
     if (lane == 0) {
@@ -690,53 +726,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
       }
     }
   } else if (warp == B_MMA) {
-    constexpr uint32_t idesc_s = idesc_bf16(128, 64, false);   // S^T, dP^T: N = 64 queries
+    constexpr uint32_t idesc_s = idesc_bf16(128, 128, false);  // S^T, dP^T: N = 128 queries
     constexpr uint32_t idesc_a = idesc_bf16(128, 128, true);   // dV, dK: dO, Q N-major
     const uint32_t sK = smem_u32(base + B_OFF_A), sV = sK + TILE_BYTES;
-    bool ok = n_it > 0 && __all_sync(0xffffffffu, mbar_wait(kv_full, 0, abort_flag, p.err, KID_ATTN, 32));
-    // item it: stage it / 2 (a (head, query tile) pair), half it % 2, TMEM buffer it % 2
-    auto second = [&](int it) -> bool {  // dV += P^T dO_half, dK += dS^T Q_half
-      if (!__all_sync(0xffffffffu, mbar_wait(&p_full[it & 1], (it >> 1) & 1, abort_flag, p.err, KID_ATTN, 34)))
-        return false;
+    bool ok = n_st > 0 && __all_sync(0xffffffffu, mbar_wait(kv_full, 0, abort_flag, p.err, KID_ATTN, 32));
+    auto kv_products = [&](int sti) -> bool {  // dV += P^T dO, dK += dS^T Q; then the stage is free
+      if (!__all_sync(0xffffffffu, mbar_wait(p_full, sti & 1, abort_flag, p.err, KID_ATTN, 34))) return false;
       tc_fence_after();
       if (lane == 0) {
-        const int sti = it >> 1, hh = it & 1;
         const uint32_t sQ = smem_u32(base + B_OFF_RING + (sti & 1) * 2 * TILE_BYTES), sO = sQ + TILE_BYTES;
-        const uint32_t c0 = (uint32_t)(it & 1) * 128;
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {  // 16 queries per step
-          const uint32_t acc = (it | ks) ? 1u : 0u;
-          const uint32_t row = (uint32_t)(hh * 8192 + ks * 2048);
-          umma_bf16_ta(tmem + 256, tmem + packed_col(c0, ks), sdesc_sw128(sO + row, ATOM, 1024), idesc_a, acc);
-          umma_bf16_ta(tmem + 384, tmem + packed_col(c0 + 64, ks), sdesc_sw128(sQ + row, ATOM, 1024), idesc_a, acc);
+        for (int ks = 0; ks < 8; ++ks) {  // 16 queries per step
+          const uint32_t acc = (sti | ks) ? 1u : 0u;
+          umma_bf16_ta(tmem + 256, tmem + packed_col(0, ks), sdesc_sw128(sO + ks * 2048, ATOM, 1024), idesc_a, acc);
+          umma_bf16_ta(tmem + 384, tmem + packed_col(128, ks), sdesc_sw128(sQ + ks * 2048, ATOM, 1024), idesc_a, acc);
         }
-        if (hh == 1) umma_commit(&qd_empty[sti & 1]);
+        umma_commit(&qd_empty[sti & 1]);
       }
       __syncwarp();
       return true;
     };
-    for (int it = 0; ok && it < n_it; ++it) {
-      const int sti = it >> 1, hh = it & 1, bf = it & 1;
-      if (hh == 0 && !(ok = __all_sync(0xffffffffu, mbar_wait(&qd_full[sti & 1], (sti >> 1) & 1, abort_flag, p.err,
-                                                               KID_ATTN, 33))))
+    for (int sti = 0; ok && sti < n_st; ++sti) {
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&qd_full[sti & 1], (sti >> 1) & 1, abort_flag, p.err, KID_ATTN,
+                                                   33))))
         break;
+      // the previous item's P^T and dS^T are read (issue order) before S^T, dP^T overwrite them
+      if (sti >= 1 && !(ok = kv_products(sti - 1))) break;
       tc_fence_after();
       if (lane == 0) {
         const uint32_t sQ = smem_u32(base + B_OFF_RING + (sti & 1) * 2 * TILE_BYTES), sO = sQ + TILE_BYTES;
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {  // S^T = K Q^T, dP^T = V dO^T over the head dim
           const uint32_t off = (ks >> 2) * ATOM + (ks & 3) * 32;
-          umma_bf16(tmem + bf * 128, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + hh * 8192 + off, 16, 1024),
-                    idesc_s, ks ? 1u : 0u);
-          umma_bf16(tmem + bf * 128 + 64, sdesc_sw128(sV + off, 16, 1024),
-                    sdesc_sw128(sO + hh * 8192 + off, 16, 1024), idesc_s, ks ? 1u : 0u);
+          umma_bf16(tmem, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024), idesc_s, ks ? 1u : 0u);
+          umma_bf16(tmem + 128, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sO + off, 16, 1024), idesc_s,
+                    ks ? 1u : 0u);
         }
-        umma_commit(&sd_full[bf]);
+        umma_commit(sd_full);
       }
       __syncwarp();
-      if (it >= 1 && !(ok = second(it - 1))) break;
     }
-    if (ok) ok = second(n_it - 1);
+    if (ok) ok = kv_products(n_st - 1);
     if (ok && lane == 0) umma_commit(acc_full);
     __syncwarp();
   } else {
@@ -746,46 +776,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
     const uint32_t trow = tmem + ((uint32_t)(wq * 32) << 16);
     const float sl = p.scale_log2;
     bool ok = true;
-    for (int it = 0; it < n_it; ++it) {
-      const int sti = it >> 1, hh = it & 1, bf = it & 1;
+    for (int sti = 0; sti < n_st; ++sti) {
       const int qt = kt + sti % per_head;
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sd_full[bf], (it >> 1) & 1, abort_flag, p.err, KID_ATTN, 35))))
-        break;
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(sd_full, sti & 1, abort_flag, p.err, KID_ATTN, 35)))) break;
       tc_fence_after();
       const float* ld = reinterpret_cast<const float*>(base + B_OFF_X + (sti & 1) * 1024);
-      uint32_t sv[32], dpv[32], pp[16], dd[16];
-      tmem_ld32(trow + bf * 128 + g * 32, sv);
-      tmem_ld32(trow + bf * 128 + 64 + g * 32, dpv);
-      tmem_wait_ld();
-      const int qi0 = hh * 64 + g * 32;  // query within the tile
-      const int lim = key - qt * TT - qi0;  // columns c < lim are masked (only on the diagonal tile)
 #pragma unroll
-      for (int j4 = 0; j4 < 8; ++j4) {  // four columns: their lse and delta in one vector load each
-        const float4 l4 = *reinterpret_cast<const float4*>(ld + qi0 + 4 * j4);
-        const float4 d4 = *reinterpret_cast<const float4*>(ld + 128 + qi0 + 4 * j4);
-        const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dl[4] = {d4.x, d4.y, d4.z, d4.w};
-        float pv[4], ds[4];
+      for (int hc = 0; hc < 2; ++hc) {  // queries 64 g + 32 hc .. of the tile
+        uint32_t sv[32], dpv[32], pp[16], dd[16];
+        tmem_ld32(trow + g * 64 + hc * 32, sv);
+        tmem_ld32(trow + 128 + g * 64 + hc * 32, dpv);
+        tmem_wait_ld();
+        const int qi0 = g * 64 + hc * 32;     // query within the tile
+        const int lim = key - qt * TT - qi0;  // columns c < lim are masked (only on the diagonal tile)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c = 4 * j4 + e;
-          const float pe =
-              c >= lim ? fast_exp2(fmaf(__uint_as_float(sv[c]), sl, -lv[e] * 1.4426950408889634f)) : 0.f;
-          pv[e] = pe;
-          ds[e] = pe * (__uint_as_float(dpv[c]) - dl[e]);
+        for (int j4 = 0; j4 < 8; ++j4) {  // four columns: their lse and delta in one vector load each
+          const float4 l4 = *reinterpret_cast<const float4*>(ld + qi0 + 4 * j4);
+          const float4 d4 = *reinterpret_cast<const float4*>(ld + 128 + qi0 + 4 * j4);
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dl[4] = {d4.x, d4.y, d4.z, d4.w};
+          float pv[4], ds[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = 4 * j4 + e;
+            const float pe =
+                c >= lim ? fast_exp2(fmaf(__uint_as_float(sv[c]), sl, -lv[e] * 1.4426950408889634f)) : 0.f;
+            pv[e] = pe;
+            ds[e] = pe * (__uint_as_float(dpv[c]) - dl[e]);
+          }
+          pp[2 * j4] = pack_bf16x2(pv[0], pv[1]);
+          pp[2 * j4 + 1] = pack_bf16x2(pv[2], pv[3]);
+          dd[2 * j4] = pack_bf16x2(ds[0], ds[1]);
+          dd[2 * j4 + 1] = pack_bf16x2(ds[2], ds[3]);
         }
-        pp[2 * j4] = pack_bf16x2(pv[0], pv[1]);
-        pp[2 * j4 + 1] = pack_bf16x2(pv[2], pv[3]);
-        dd[2 * j4] = pack_bf16x2(ds[0], ds[1]);
-        dd[2 * j4 + 1] = pack_bf16x2(ds[2], ds[3]);
+        tmem_st16(trow + g * 64 + hc * 16, pp);  // over scores this warp has read
+        tmem_st16(trow + 128 + g * 64 + hc * 16, dd);
       }
-      tmem_st16(trow + bf * 128 + g * 32, pp);        // over the scores this warp has read
-      tmem_st16(trow + bf * 128 + 64 + g * 32, dd);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[bf]);
+      if (lane == 0) mbar_arrive(p_full);
     }
-    const bool have = n_it > 0 && ok && __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, p.err, KID_ATTN, 36));
+    const bool have = n_st > 0 && ok && __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, p.err, KID_ATTN, 36));
     if (have) tc_fence_after();
     // both CTAs have finished their products: the first CTA's ring is free for the partials
     cluster_sync_all();
@@ -817,34 +848,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
     }
     cluster_sync_all();
     if (crank == 0) {
-      uint4* dv = reinterpret_cast<uint4*>(p.dv + (size_t)(row0 + key) * p.ld_dkv + kvh * 128 + g * 64);
-      uint4* dk = reinterpret_cast<uint4*>(p.dk + (size_t)(row0 + key) * p.ld_dkv + kvh * 128 + g * 64);
+      // dV, dK through the freed K / V tiles' shared memory and four TMA stores
+      const uint32_t tv = smem_u32(base + B_OFF_A), tk = tv + TILE_BYTES;
       const float sc = p.scale;
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         float v[32], k[32];
-        {
-          uint32_t vr[32], kr[32];
-          if (have) {
-            tmem_ld32(trow + 256 + g * 64 + c * 32, vr);
-            tmem_ld32(trow + 384 + g * 64 + c * 32, kr);
-            tmem_wait_ld();
-          }
-          const float* pv = peer + r * PEER_LD + g * 64 + c * 32;
-          const float* pk = pv + 128 * PEER_LD;
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            v[i] = (have ? __uint_as_float(vr[i]) : 0.f) + pv[i];
-            k[i] = ((have ? __uint_as_float(kr[i]) : 0.f) + pk[i]) * sc;
-          }
+        uint32_t vr[32], kr[32];
+        if (have) {
+          tmem_ld32(trow + 256 + g * 64 + c * 32, vr);
+          tmem_ld32(trow + 384 + g * 64 + c * 32, kr);
+          tmem_wait_ld();
         }
+        const float* pv = peer + r * PEER_LD + g * 64 + c * 32;
+        const float* pk = pv + 128 * PEER_LD;
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          dv[c * 4 + q4] = make_uint4(pack_bf16x2(v[8 * q4], v[8 * q4 + 1]), pack_bf16x2(v[8 * q4 + 2], v[8 * q4 + 3]),
-                                      pack_bf16x2(v[8 * q4 + 4], v[8 * q4 + 5]), pack_bf16x2(v[8 * q4 + 6], v[8 * q4 + 7]));
-          dk[c * 4 + q4] = make_uint4(pack_bf16x2(k[8 * q4], k[8 * q4 + 1]), pack_bf16x2(k[8 * q4 + 2], k[8 * q4 + 3]),
-                                      pack_bf16x2(k[8 * q4 + 4], k[8 * q4 + 5]), pack_bf16x2(k[8 * q4 + 6], k[8 * q4 + 7]));
+        for (int i = 0; i < 32; ++i) {
+          v[i] = (have ? __uint_as_float(vr[i]) : 0.f) + pv[i];
+          k[i] = ((have ? __uint_as_float(kr[i]) : 0.f) + pk[i]) * sc;
         }
+        stage_row32(tv, r, 2 * g + c, v);
+        stage_row32(tk, r, 2 * g + c, k);
+      }
+      fence_proxy_async_smem();
+      bar_ew();
+      if (threadIdx.x == 0 && !*abort_flag) {
+        for (int j = 0; j < 2; ++j) {
+          tma_store_2d(&p.tdv, tv + j * ATOM, kvh * 128 + 64 * j, row0 + kt * TT);
+          tma_store_2d(&p.tdk, tk + j * ATOM, kvh * 128 + 64 * j, row0 + kt * TT);
+        }
+        tma_store_drain();
       }
     }
   }
@@ -882,6 +915,7 @@ int attention_fwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_
   NF4_TRY(tma_map_bf16(&p.tq, q, (uint64_t)nq * 128, rows, (uint64_t)ldq * 2, 64, TT));
   NF4_TRY(tma_map_bf16(&p.tk, k, (uint64_t)nkv * 128, rows, (uint64_t)ldkv * 2, 64, TT));
   NF4_TRY(tma_map_bf16(&p.tv, v, (uint64_t)nkv * 128, rows, (uint64_t)ldkv * 2, 64, TT));
+  NF4_TRY(tma_map_bf16(&p.to, o, (uint64_t)nq * 128, rows, (uint64_t)ldo * 2, 64, TT));
   p.o = o;
   p.lse = lse;
   p.ldo = ldo;
@@ -920,6 +954,9 @@ int attention_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_
   NF4_TRY(tma_map_bf16(&p.tdo, dout, (uint64_t)nq * 128, rows, (uint64_t)ldo * 2, 64, TT));
   if (!aligned(lse, 16) || !aligned(delta, 16)) return fail(NF4LS_ALIGN, "attention backward: lse / delta alignment");
   NF4_TRY(tma_map_bf16(&p.to, o, (uint64_t)nq * 128, rows, (uint64_t)ldo * 2, 64, TT));
+  NF4_TRY(tma_map_bf16(&p.tdq, dq, (uint64_t)nq * 128, rows, (uint64_t)ld_dq * 2, 64, TT));
+  NF4_TRY(tma_map_bf16(&p.tdk, dk, (uint64_t)nkv * 128, rows, (uint64_t)ld_dkv * 2, 64, TT));
+  NF4_TRY(tma_map_bf16(&p.tdv, dv, (uint64_t)nkv * 128, rows, (uint64_t)ld_dkv * 2, 64, TT));
   p.lse = lse;
   p.delta = delta;
   p.dq = dq;
