@@ -633,16 +633,23 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
   }
 }
 
-// st.shared::cluster of four floats at a shared::cluster address (another CTA's smem).
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+// Bulk copy of bytes (a multiple of 16) from this CTA's shared memory to another CTA's of
+// the cluster, completing transaction bytes on that CTA's mbarrier (both given by their
+// shared::cluster addresses).
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src, uint32_t bytes,
+                                                  uint32_t bar_cluster) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   dst_cluster),
+               "r"(src), "r"(bytes), "r"(bar_cluster)
                : "memory");
 }
 
 // KEY side: dK, dV of one 128-key tile of one kv head, by a cluster of two CTAs that split
 // the group's query heads (the first ceil(group / 2) heads and the rest): the second CTA
-// sends its fp32 partial sums through distributed shared memory and the first adds them to
-// its own in that fixed order.  Halving the longest CTAs' work balances the grid (two CTAs
+// stages its fp32 partial sums in its own shared memory and sends them in two bulk copies
+// into the first CTA's (distributed shared memory; per-thread remote stores of the same
+// 132 KB measured about 13 000 cycles), and the first adds them to its own in that fixed
+// order.  Halving the longest CTAs' work balances the grid (two CTAs
 // per key tile instead of one, the first key tiles holding the most query tiles).
 constexpr int PEER_LD = 132;  // row stride (floats) of the partial sums in the first CTA's smem
 
@@ -660,6 +667,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
   uint64_t* drain = bars + 10;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint64_t* peer_full = bars + 12;  // (first CTA) the second CTA's partial sums have landed
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kvh = blockIdx.x >> 1, b = blockIdx.y, kt = blockIdx.z;  // z slowest: the longest key tiles first
@@ -680,6 +688,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
     mbar_init(p_full, B_EW / 32);
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
+    mbar_init(peer_full, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -818,11 +827,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
     }
     const bool have = n_st > 0 && ok && __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, p.err, KID_ATTN, 36));
     if (have) tc_fence_after();
-    // both CTAs have finished their products: the first CTA's ring is free for the partials
-    cluster_sync_all();
     float* peer = reinterpret_cast<float*>(base + B_OFF_RING);  // dV [128][PEER_LD], then dK
-    if (crank == 1) {
-      const uint32_t dst = mapa_shared(smem_u32(peer), 0);
+    constexpr uint32_t PEER_BYTES = 128 * PEER_LD * 4;              // one tensor's partial sums
+    if (crank == 1) {  // this CTA's ring is free: stage the partial sums there (zeros if none)
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t v[32], k[32];
@@ -833,19 +840,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
         }
 #pragma unroll
         for (int q4 = 0; q4 < 8; ++q4) {
-          const uint32_t o = (uint32_t)((r * PEER_LD + g * 64 + c * 32 + 4 * q4) * 4);
+          const uint32_t o = smem_u32(peer + r * PEER_LD + g * 64 + c * 32 + 4 * q4);
           if (have) {
-            st_cluster_v4(dst + o, __uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1]),
-                          __uint_as_float(v[4 * q4 + 2]), __uint_as_float(v[4 * q4 + 3]));
-            st_cluster_v4(dst + 128 * PEER_LD * 4 + o, __uint_as_float(k[4 * q4]), __uint_as_float(k[4 * q4 + 1]),
-                          __uint_as_float(k[4 * q4 + 2]), __uint_as_float(k[4 * q4 + 3]));
+            st_shared_v4(o, v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+            st_shared_v4(o + PEER_BYTES, k[4 * q4], k[4 * q4 + 1], k[4 * q4 + 2], k[4 * q4 + 3]);
           } else {
-            st_cluster_v4(dst + o, 0.f, 0.f, 0.f, 0.f);
-            st_cluster_v4(dst + 128 * PEER_LD * 4 + o, 0.f, 0.f, 0.f, 0.f);
+            st_shared_v4(o, 0u, 0u, 0u, 0u);
+            st_shared_v4(o + PEER_BYTES, 0u, 0u, 0u, 0u);
           }
         }
       }
+      fence_proxy_async_smem();
+      bar_ew();
+    } else if (threadIdx.x == 0) {
+      mbar_arrive_expect_tx(peer_full, 2 * PEER_BYTES);
     }
+    // both CTAs have finished their products: the first CTA's ring is free for the partials
+    cluster_sync_all();
+    if (crank == 1 && threadIdx.x == 0) {
+      const uint32_t dst = mapa_shared(smem_u32(peer), 0), bar = mapa_shared(smem_u32(peer_full), 0);
+      bulk_copy_to_peer(dst, smem_u32(peer), PEER_BYTES, bar);
+      bulk_copy_to_peer(dst + PEER_BYTES, smem_u32(peer) + PEER_BYTES, PEER_BYTES, bar);
+    }
+    bool got = true;
+    if (crank == 0) got = __all_sync(0xffffffffu, mbar_wait(peer_full, 0, abort_flag, p.err, KID_ATTN, 37));
+    // the second CTA's shared memory stays until the first has its copy
     cluster_sync_all();
     if (crank == 0) {
       // dV, dK through the freed K / V tiles' shared memory and four TMA stores
@@ -872,6 +891,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
       }
       fence_proxy_async_smem();
       bar_ew();
+      (void)got;
       if (threadIdx.x == 0 && !*abort_flag) {
         for (int j = 0; j < 2; ++j) {
           tma_store_2d(&p.tdv, tv + j * ATOM, kvh * 128 + 64 * j, row0 + kt * TT);
