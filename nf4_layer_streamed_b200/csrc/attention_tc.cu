@@ -574,12 +574,17 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
     for (int kt = 0; ok && kt < n_kt; ++kt) {
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(sd_full, kt & 1, abort_flag, p.err, KID_ATTN, 46)))) break;
       tc_fence_after();
+      // both 32-key chunks in one TMEM round trip
+      uint32_t sv[2][32], dpv[2][32];
+#pragma unroll
+      for (int hc = 0; hc < 2; ++hc) {
+        tmem_ld32(trow + g * 64 + hc * 32, sv[hc]);
+        tmem_ld32(trow + 128 + g * 64 + hc * 32, dpv[hc]);
+      }
+      tmem_wait_ld();
 #pragma unroll
       for (int hc = 0; hc < 2; ++hc) {  // keys 64 g + 32 hc .. of the tile
-        uint32_t sv[32], dpv[32], dd[16];
-        tmem_ld32(trow + g * 64 + hc * 32, sv);
-        tmem_ld32(trow + 128 + g * 64 + hc * 32, dpv);
-        tmem_wait_ld();
+        uint32_t dd[16];
         const int key0 = kt * TT + g * 64 + hc * 32;
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
@@ -587,8 +592,8 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int kj = key0 + 2 * j + e;
-            const float pe = kj <= qpos ? fast_exp2(fmaf(__uint_as_float(sv[2 * j + e]), sl, -lse2)) : 0.f;
-            ds[e] = pe * (__uint_as_float(dpv[2 * j + e]) - dl);
+            const float pe = kj <= qpos ? fast_exp2(fmaf(__uint_as_float(sv[hc][2 * j + e]), sl, -lse2)) : 0.f;
+            ds[e] = pe * (__uint_as_float(dpv[hc][2 * j + e]) - dl);
           }
           dd[j] = pack_bf16x2(ds[0], ds[1]);
         }
