@@ -417,7 +417,7 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
   uint64_t* kv_full = bars + 1;     // 2 stages
   uint64_t* kv_empty = bars + 3;    // 2
   uint64_t* sd_full = bars + 5;     // S and dP of the item are in TMEM
-  uint64_t* p_full = bars + 6;      // dS of the item is in TMEM (one arrival per elementwise warp)
+  uint64_t* p_half = bars + 6;      // 2: dS chunk hc of the item is in TMEM (one arrival per warp)
   uint64_t* acc_full = bars + 9;
   uint64_t* drain = bars + 10;
   uint64_t* qa_full = bars + 11;    // Q and dO are in TMEM (one arrival per elementwise warp)
@@ -437,7 +437,8 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
       mbar_init(&kv_empty[i], 1);
     }
     mbar_init(sd_full, 1);
-    mbar_init(p_full, B_EW / 32);
+    mbar_init(&p_half[0], B_EW / 32);
+    mbar_init(&p_half[1], B_EW / 32);
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
     mbar_init(qa_full, B_EW / 32);
@@ -489,18 +490,24 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
     constexpr uint32_t idesc_s = idesc_bf16(128, 128, false);  // S, dP: N = 128 keys
     constexpr uint32_t idesc_a = idesc_bf16(128, 128, true);   // dQ += dS K: K N-major
     bool ok = __all_sync(0xffffffffu, mbar_wait(qa_full, 0, abort_flag, p.err, KID_ATTN, 42)) && !*abort_flag;
-    auto dq_product = [&](int kt) -> bool {  // dQ += dS_kt K_kt, then the K/V stage is free
-      if (!__all_sync(0xffffffffu, mbar_wait(p_full, kt & 1, abort_flag, p.err, KID_ATTN, 44))) return false;
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t sK = smem_u32(base + B_OFF_RING + (kt & 1) * 2 * TILE_BYTES);
+    // dQ += dS_kt K_kt, each half as soon as its dS chunks are in TMEM (chunk hc holds the
+    // k-steps with ks & 2 == 2 hc); then the K/V stage is free
+    auto dq_product = [&](int kt) -> bool {
+      const uint32_t sK = smem_u32(base + B_OFF_RING + (kt & 1) * 2 * TILE_BYTES);
+      for (int hc = 0; hc < 2; ++hc) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&p_half[hc], kt & 1, abort_flag, p.err, KID_ATTN, 44))) return false;
+        tc_fence_after();
+        if (lane == 0) {
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks)  // 16 keys per step
-          umma_bf16_ta(tmem + 256, tmem + packed_col(128, ks), sdesc_sw128(sK + ks * 2048, ATOM, 1024), idesc_a,
-                       (kt | ks) ? 1u : 0u);
-        umma_commit(&kv_empty[kt & 1]);
+          for (int i = 0; i < 4; ++i) {  // 16 keys per step
+            const int ks = (i >> 1) * 4 + hc * 2 + (i & 1);
+            umma_bf16_ta(tmem + 256, tmem + packed_col(128, ks), sdesc_sw128(sK + ks * 2048, ATOM, 1024), idesc_a,
+                         (kt | hc | i) ? 1u : 0u);
+          }
+          if (hc == 1) umma_commit(&kv_empty[kt & 1]);
+        }
+        __syncwarp();
       }
-      __syncwarp();
       return true;
     };
     for (int kt = 0; ok && kt < n_kt; ++kt) {
@@ -598,11 +605,11 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
           dd[j] = pack_bf16x2(ds[0], ds[1]);
         }
         tmem_st16(trow + 128 + g * 64 + hc * 16, dd);  // over dP values this warp has read
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_half[hc]);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
     }
     // dQ through the freed ring's shared memory and two TMA stores (coalesced rows); every
     // elementwise warp reaches the barrier, the store is issued only when no wait failed
@@ -667,7 +674,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
   uint64_t* qd_full = bars + 1;     // 2 stages (Q, dO, lse, delta of one (head, query tile))
   uint64_t* qd_empty = bars + 3;    // 2
   uint64_t* sd_full = bars + 5;     // S^T and dP^T of the item are in TMEM
-  uint64_t* p_full = bars + 6;      // P^T and dS^T of the item are in TMEM (one arrival per warp)
+  uint64_t* p_half = bars + 6;      // 2: P^T, dS^T chunk hc of the item are in TMEM (one arrival per warp)
   uint64_t* acc_full = bars + 9;
   uint64_t* drain = bars + 10;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
@@ -690,7 +697,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
       mbar_init(&qd_empty[i], 1);
     }
     mbar_init(sd_full, 1);
-    mbar_init(p_full, B_EW / 32);
+    mbar_init(&p_half[0], B_EW / 32);
+    mbar_init(&p_half[1], B_EW / 32);
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
     mbar_init(peer_full, 1);
@@ -744,20 +752,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
     constexpr uint32_t idesc_a = idesc_bf16(128, 128, true);   // dV, dK: dO, Q N-major
     const uint32_t sK = smem_u32(base + B_OFF_A), sV = sK + TILE_BYTES;
     bool ok = n_st > 0 && __all_sync(0xffffffffu, mbar_wait(kv_full, 0, abort_flag, p.err, KID_ATTN, 32));
-    auto kv_products = [&](int sti) -> bool {  // dV += P^T dO, dK += dS^T Q; then the stage is free
-      if (!__all_sync(0xffffffffu, mbar_wait(p_full, sti & 1, abort_flag, p.err, KID_ATTN, 34))) return false;
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t sQ = smem_u32(base + B_OFF_RING + (sti & 1) * 2 * TILE_BYTES), sO = sQ + TILE_BYTES;
+    // dV += P^T dO, dK += dS^T Q, each half as soon as its chunks are in TMEM (chunk hc holds
+    // the k-steps with ks & 2 == 2 hc); then the stage is free
+    auto kv_products = [&](int sti) -> bool {
+      const uint32_t sQ = smem_u32(base + B_OFF_RING + (sti & 1) * 2 * TILE_BYTES), sO = sQ + TILE_BYTES;
+      for (int hc = 0; hc < 2; ++hc) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&p_half[hc], sti & 1, abort_flag, p.err, KID_ATTN, 34))) return false;
+        tc_fence_after();
+        if (lane == 0) {
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {  // 16 queries per step
-          const uint32_t acc = (sti | ks) ? 1u : 0u;
-          umma_bf16_ta(tmem + 256, tmem + packed_col(0, ks), sdesc_sw128(sO + ks * 2048, ATOM, 1024), idesc_a, acc);
-          umma_bf16_ta(tmem + 384, tmem + packed_col(128, ks), sdesc_sw128(sQ + ks * 2048, ATOM, 1024), idesc_a, acc);
+          for (int i = 0; i < 4; ++i) {  // 16 queries per step
+            const int ks = (i >> 1) * 4 + hc * 2 + (i & 1);
+            const uint32_t acc = (sti | hc | i) ? 1u : 0u;
+            umma_bf16_ta(tmem + 256, tmem + packed_col(0, ks), sdesc_sw128(sO + ks * 2048, ATOM, 1024), idesc_a, acc);
+            umma_bf16_ta(tmem + 384, tmem + packed_col(128, ks), sdesc_sw128(sQ + ks * 2048, ATOM, 1024), idesc_a,
+                         acc);
+          }
+          if (hc == 1) umma_commit(&qd_empty[sti & 1]);
         }
-        umma_commit(&qd_empty[sti & 1]);
+        __syncwarp();
       }
-      __syncwarp();
       return true;
     };
     for (int sti = 0; ok && sti < n_st; ++sti) {
@@ -824,11 +838,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
         }
         tmem_st16(trow + g * 64 + hc * 16, pp);  // over scores this warp has read
         tmem_st16(trow + 128 + g * 64 + hc * 16, dd);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_half[hc]);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
     }
     const bool have = n_st > 0 && ok && __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, p.err, KID_ATTN, 36));
     if (have) tc_fence_after();
