@@ -33,8 +33,9 @@ sys.path.insert(0, ROOT)
 METRIC = "trained tok/s per step (8B-shaped NF4+LoRA, streamed); GEMM % bf16 TC peak"
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # dram__bytes_read.sum + dram__bytes_write.sum per NF4-decode GEMM launch, averaged over
-# the 352 launches of one step of this workload (one ncu capture of the current kernel)
-NF4_GEMM_DRAM_BYTES_PER_LAUNCH = 102.3e6
+# the 11 launches of one layer of this workload (one ncu capture of the current kernel;
+# every layer of the step runs the same 11 launches)
+NF4_GEMM_DRAM_BYTES_PER_LAUNCH = 101.7e6
 
 
 def peaks():
@@ -583,7 +584,7 @@ def main():
                          "launches_per_step": nf4["launches"] / args.steps,
                          "ms_per_step": nf4["ms"] / args.steps,
                          "traffic": NF4_GEMM_DRAM_BYTES_PER_LAUNCH if wl.name == "llama8b_32L_b4s512" else None,
-                         "traffic_unit": "bytes per launch (DRAM read + write, ncu)",
+                         "traffic_unit": "bytes per launch (DRAM read + write, ncu, one layer's 11 launches)",
                          "timing": "CUDA events on the launching stream around every launch, in a second "
                                    "timed pass over the same steps"},
             "dense_gemm": {"launches_per_step": dense["launches"] / args.steps, "ms_per_step": dense["ms"] / args.steps,
