@@ -413,7 +413,7 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + B_OFF_BAR);
-  uint64_t* q_full = bars;          // Q, dO
+  uint64_t* q_full = bars;          // Q, dO (copied into TMEM first)
   uint64_t* kv_full = bars + 1;     // 2 stages
   uint64_t* kv_empty = bars + 3;    // 2
   uint64_t* sd_full = bars + 5;     // S and dP of the item are in TMEM
@@ -423,6 +423,7 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
   uint64_t* qa_full = bars + 11;    // Q and dO are in TMEM (one arrival per elementwise warp)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint64_t* o_full = bars + 13;     // the O tile (for delta)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = gridDim.x - 1 - blockIdx.x, h = blockIdx.y, b = blockIdx.z;  // longest rows first
@@ -432,6 +433,7 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(o_full, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
@@ -463,12 +465,14 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
       tma_prefetch_desc(&p.tv);
       tma_prefetch_desc(&p.tdo);
       tma_prefetch_desc(&p.to);
-      mbar_arrive_expect_tx(q_full, 3 * TILE_BYTES);
+      mbar_arrive_expect_tx(q_full, 2 * TILE_BYTES);
       for (int j = 0; j < 2; ++j) {
         tma_load_2d(base + B_OFF_A + j * ATOM, &p.tq, q_full, h * 128 + 64 * j, row0 + qt * TT);
         tma_load_2d(base + B_OFF_A + TILE_BYTES + j * ATOM, &p.tdo, q_full, h * 128 + 64 * j, row0 + qt * TT);
-        tma_load_2d(base + B_OFF_X + j * ATOM, &p.to, q_full, h * 128 + 64 * j, row0 + qt * TT);
       }
+      mbar_arrive_expect_tx(o_full, TILE_BYTES);
+      for (int j = 0; j < 2; ++j)
+        tma_load_2d(base + B_OFF_X + j * ATOM, &p.to, o_full, h * 128 + 64 * j, row0 + qt * TT);
       int issued = 0;
       for (int kt = 0; kt < n_kt; ++kt) {
         const int st = kt & 1;
@@ -483,6 +487,7 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
       }
       if (*abort_flag) {  // let the copies already issued land before the CTA exits
         mbar_wait_drain(q_full, 0);
+        mbar_wait_drain(o_full, 0);
         for (int kt = (issued > 2 ? issued - 2 : 0); kt < issued; ++kt) mbar_wait_drain(&kv_full[kt & 1], (kt >> 1) & 1);
       }
     }
@@ -539,33 +544,25 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
     const int qpos = qt * TT + r;
     const uint32_t trow = tmem + ((uint32_t)(wq * 32) << 16);
     const size_t li = ((size_t)b * p.nq + h) * p.seq + qpos;
-    // delta = rowsum(dO * O) over this thread's 64 dims (its row in swizzle atom g of the
-    // dO and O tiles), the two halves added through smem
+    // First Q and dO into TMEM (the MMA warp starts on them), then delta = rowsum(dO * O)
+    // over this thread's 64 dims (its row in swizzle atom g of the dO and O tiles), the two
+    // halves added through smem.  Chunk c of the row holds dims 8 c .. 8 c + 7 of the atom,
+    // TMEM column 32 g + 4 c + i their pair i.
     float* red = reinterpret_cast<float*>(base + B_OFF_X + TILE_BYTES);
+    const uint8_t* q_row = base + B_OFF_A + g * ATOM + r * 128;
+    const uint8_t* dO_row = base + B_OFF_A + TILE_BYTES + g * ATOM + r * 128;
+    const uint8_t* o_row = base + B_OFF_X + g * ATOM + r * 128;
     bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort_flag, p.err, KID_ATTN, 45));
     if (ok) {
-      // this thread's row of swizzle atom g (dims 64 g ..): chunk c holds dims 8 c .. 8 c + 7,
-      // TMEM column 32 g + 4 c + i their pair i
-      const uint8_t* q_row = base + B_OFF_A + g * ATOM + r * 128;
-      const uint8_t* dO_row = base + B_OFF_A + TILE_BYTES + g * ATOM + r * 128;
-      const uint8_t* o_row = base + B_OFF_X + g * ATOM + r * 128;
       uint32_t qv[32], dv[32];
-      float s = 0.f;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         const uint32_t off = (uint32_t)((c ^ (r & 7)) << 4);
-        const uint4 a = *reinterpret_cast<const uint4*>(o_row + off);
         const uint4 d = *reinterpret_cast<const uint4*>(dO_row + off);
         const uint4 q = *reinterpret_cast<const uint4*>(q_row + off);
-        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, dw[4] = {d.x, d.y, d.z, d.w}, qw[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          s += bf16_lo(aw[j]) * bf16_lo(dw[j]) + bf16_hi(aw[j]) * bf16_hi(dw[j]);
-          qv[4 * c + j] = qw[j];
-          dv[4 * c + j] = dw[j];
-        }
+        qv[4 * c] = q.x, qv[4 * c + 1] = q.y, qv[4 * c + 2] = q.z, qv[4 * c + 3] = q.w;
+        dv[4 * c] = d.x, dv[4 * c + 1] = d.y, dv[4 * c + 2] = d.z, dv[4 * c + 3] = d.w;
       }
-      red[g * 128 + r] = s;
       tmem_st32(trow + T_Q + g * 32, qv);
       tmem_st32(trow + T_DO + g * 32, dv);
       tmem_wait_st();
@@ -573,6 +570,20 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(qa_full);  // also on failure: the MMA warp then sees the abort
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_full, 0, abort_flag, p.err, KID_ATTN, 48));
+    if (ok) {
+      float s = 0.f;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint32_t off = (uint32_t)((c ^ (r & 7)) << 4);
+        const uint4 a = *reinterpret_cast<const uint4*>(o_row + off);
+        const uint4 d = *reinterpret_cast<const uint4*>(dO_row + off);
+        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, dw[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) s += bf16_lo(aw[j]) * bf16_lo(dw[j]) + bf16_hi(aw[j]) * bf16_hi(dw[j]);
+      }
+      red[g * 128 + r] = s;
+    }
     bar_ew();
     const float dl = ok ? red[r] + red[128 + r] : 0.f;
     if (ok && g == 0) p.delta[li] = dl;
