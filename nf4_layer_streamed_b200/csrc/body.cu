@@ -158,14 +158,15 @@ __global__ void __launch_bounds__(1024) k_rmsnorm_fwd_row(const __nv_bfloat16* _
 //   operand of the q/k/v GEMM, zeros in 32-63),
 // so that h1 is not read back for t.  A cluster of C CTAs takes 64 rows; CTA c of the
 // cluster holds the column slice [c S, (c + 1) S) of those rows (S = H / C) in registers
-// (four threads per row) and the same slice of the 32 adapter rows, rounded to bf16, in
+// (a warp per eight rows, 512 contiguous bytes per load) and the same slice of the 32
+// adapter rows, rounded to bf16, in
 // shared memory.  The rows' sums of squares are partial per CTA and added in CTA order
 // through distributed shared memory; each CTA then writes its slice of h1 and forms the
 // partial t of its slice on mma.sync m16n8k16 (warp w: row tile w % 4, k-steps
 // w / 4, w / 4 + 2, ..); the warp partials are added in k order, and the cluster's C
 // partials in CTA order, CTA c writing rows 64 c / C ...  The same launch converts the
 // adapter to its bf16 operands (every thread a share of pack_piece).
-constexpr int ND_R = 64, ND_THREADS = 256, ND_TPR = ND_THREADS / ND_R;  // threads per row
+constexpr int ND_R = 64, ND_THREADS = 256;  // rows per cluster, threads per CTA (eight rows per warp)
 
 struct NormDownShape {
   int C, S;  // cluster size, slice width
@@ -186,8 +187,8 @@ inline NormDownShape norm_down_shape(int H) {
   return sh;
 }
 
-template <int VPT>
-__global__ void __launch_bounds__(ND_THREADS) k_rmsnorm_down(const __nv_bfloat16* __restrict__ x,
+template <int NH>
+__global__ void __launch_bounds__(ND_THREADS, 2) k_rmsnorm_down(const __nv_bfloat16* __restrict__ x,
                                                              const __nv_bfloat16* __restrict__ w,
                                                              __nv_bfloat16* __restrict__ y, int M, int H, int S,
                                                              float eps, const LoraPack pack,
@@ -201,13 +202,17 @@ __global__ void __launch_bounds__(ND_THREADS) k_rmsnorm_down(const __nv_bfloat16
   const size_t as_bytes = std::max((size_t)32 * ls * 2, (size_t)ND_THREADS / 32 * 16 * 32 * 4);
   float* P = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(as) + as_bytes);  // [64][32] this slice's t
   float* ssp = P + ND_R * 32;                                                  // [64] partial sums of squares
-  const int row = t / ND_TPR, sub = t % ND_TPR, m = m0 + row;
-  const bool live = m < M;
-  const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)m * H + col0);
-  uint4 v[VPT];
+  // warp w holds rows 8 w .. 8 w + 7 of the block; lane l the 16-byte vectors 32 h + l of
+  // each row slice (h < NH): one warp instruction reads 512 contiguous bytes of a row
+  uint4 v[8][NH];
 #pragma unroll
-  for (int j = 0; j < VPT; ++j)
-    if (live && sub + ND_TPR * j < nv) v[j] = xr[sub + ND_TPR * j];
+  for (int rr = 0; rr < 8; ++rr) {
+    const int m = m0 + warp * 8 + rr;
+    const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)m * H + col0);
+#pragma unroll
+    for (int hh = 0; hh < NH; ++hh)
+      if (m < M && hh * 32 + lane < nv) v[rr][hh] = xr[hh * 32 + lane];
+  }
   // the adapter slice: rows 0-15 A_q, 16-31 A_v, bf16 (the values of the packed adn);
   // eight 16-byte loads in flight per thread
   {
@@ -234,40 +239,51 @@ __global__ void __launch_bounds__(ND_THREADS) k_rmsnorm_down(const __nv_bfloat16
       }
     }
   }
-  float ss = 0.f;
 #pragma unroll
-  for (int j = 0; j < VPT; ++j)
-    if (live && sub + ND_TPR * j < nv) {
-      float f[8];
-      unpack8(v[j], f);
+  for (int rr = 0; rr < 8; ++rr) {
+    const int m = m0 + warp * 8 + rr;
+    float ss = 0.f;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) ss += f[e] * f[e];
-    }
+    for (int hh = 0; hh < NH; ++hh)
+      if (m < M && hh * 32 + lane < nv) {
+        float f[8];
+        unpack8(v[rr][hh], f);
 #pragma unroll
-  for (int o = 1; o < ND_TPR; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  if (sub == 0) ssp[row] = ss;
-  cluster_sync_all();  // every slice's partial sums are in its CTA's shared memory
-  float tot = 0.f;
-  for (int q = 0; q < C; ++q) tot += ld_cluster_f32(mapa_shared(smem_u32(ssp + row), (uint32_t)q));
-  const float r = 1.0f / sqrtf(tot / (float)H + eps);
-  const uint4* wr = reinterpret_cast<const uint4*>(w + col0);
-  uint4* yr = reinterpret_cast<uint4*>(y + (size_t)m * H + col0);
-  uint4* hrow = reinterpret_cast<uint4*>(hs + row * ls);
-#pragma unroll
-  for (int j = 0; j < VPT; ++j) {
-    const int i = sub + ND_TPR * j;
-    if (i < nv) {
-      uint4 h = make_uint4(0u, 0u, 0u, 0u);
-      if (live) {
-        float f[8], g[8];
-        unpack8(v[j], f);
-        unpack8(wr[i], g);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] = f[e] * r * g[e];
-        h = pack8(f);
-        yr[i] = h;
+        for (int e = 0; e < 8; ++e) ss += f[e] * f[e];
       }
-      hrow[i] = h;
+    ss = warp_sum(ss);
+    if (lane == 0) ssp[warp * 8 + rr] = ss;
+  }
+  cluster_sync_all();  // every slice's partial sums are in its CTA's shared memory
+  const uint4* wr = reinterpret_cast<const uint4*>(w + col0);
+  uint4 wv[NH];
+#pragma unroll
+  for (int hh = 0; hh < NH; ++hh)
+    if (hh * 32 + lane < nv) wv[hh] = wr[hh * 32 + lane];
+#pragma unroll
+  for (int rr = 0; rr < 8; ++rr) {
+    const int row = warp * 8 + rr, m = m0 + row;
+    float tot = 0.f;
+    for (int q = 0; q < C; ++q) tot += ld_cluster_f32(mapa_shared(smem_u32(ssp + row), (uint32_t)q));
+    const float r = 1.0f / sqrtf(tot / (float)H + eps);
+    uint4* yr = reinterpret_cast<uint4*>(y + (size_t)m * H + col0);
+    uint4* hrow = reinterpret_cast<uint4*>(hs + row * ls);
+#pragma unroll
+    for (int hh = 0; hh < NH; ++hh) {
+      const int i = hh * 32 + lane;
+      if (i < nv) {
+        uint4 h = make_uint4(0u, 0u, 0u, 0u);
+        if (m < M) {
+          float f[8], g[8];
+          unpack8(v[rr][hh], f);
+          unpack8(wv[hh], g);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f[e] = f[e] * r * g[e];
+          h = pack8(f);
+          yr[i] = h;
+        }
+        hrow[i] = h;
+      }
     }
   }
   __syncthreads();
@@ -759,7 +775,7 @@ int rmsnorm_lora_fwd(const __nv_bfloat16* x, const __nv_bfloat16* w, __nv_bfloat
   if (!aligned(pack.Aq, 16) || !aligned(pack.Av, 16) || !aligned(x, 16) || !aligned(y, 16) || !aligned(w, 16))
     return fail(NF4LS_ALIGN, "rmsnorm_lora_fwd: 16-byte aligned operands");
   if (M <= 0) return NF4LS_OK;
-  const int vpt = (sh.S / 8 + ND_TPR - 1) / ND_TPR;
+  const int nh = (sh.S / 8 + 31) / 32;  // 512-byte pieces per row slice
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((M + ND_R - 1) / ND_R, sh.C, 1);
   cfg.blockDim = dim3(ND_THREADS, 1, 1);
@@ -784,14 +800,14 @@ int rmsnorm_lora_fwd(const __nv_bfloat16* x, const __nv_bfloat16* w, __nv_bfloat
     return NF4LS_OK;
   };
   int st;
-  if (vpt <= 8)
-    st = go(k_rmsnorm_down<8>, 0);
-  else if (vpt <= 16)
-    st = go(k_rmsnorm_down<16>, 1);
-  else if (vpt <= 24)
-    st = go(k_rmsnorm_down<24>, 2);
+  if (nh <= 1)
+    st = go(k_rmsnorm_down<1>, 0);
+  else if (nh <= 2)
+    st = go(k_rmsnorm_down<2>, 1);
+  else if (nh <= 3)
+    st = go(k_rmsnorm_down<3>, 2);
   else
-    st = go(k_rmsnorm_down<32>, 3);
+    st = go(k_rmsnorm_down<4>, 3);
   if (st != NF4LS_OK) return st;
   note_launch();
   return NF4LS_OK;
