@@ -1,7 +1,7 @@
 """Parity of layer_forward / layer_backward against the oracle (GPU).
 
 One SmolLM2-135M-shaped layer at batch 1, seq 512 (the single-layer workload with
-B = 0, and a random-B variant so that dA is exercised), a ragged small case, and one
+B = 0, and a random-B variant so that dA is exercised), two ragged small cases, and one
 Llama-8B-shaped layer at batch 1, seq 512 in full.  Outputs and gradients within
 2e-2 * max|ref|, loss within 1e-3 relative.  The two GEMM paths (decode in the
 mainloop, dequantise then multiply) must agree bit for bit, and the batch-4 run must
@@ -73,6 +73,15 @@ def test_ragged_small_layer_matches_oracle():
     shape = synth.SMOLLM2_135M
     r = _run(shape, 3, 64, True, seed=7)
     _check_against_oracle(shape, 3, 64, r)
+
+
+def test_ragged_pair_tiles_layer_matches_oracle():
+    """320 tokens (5 x 64): the CTA-pair GEMMs end on a partial tile, the fused input
+    RMSNorm / LoRA-down runs five clusters of 64 rows, and the dA kernel's eight row
+    slices of 64 leave three of them empty."""
+    shape = synth.SMOLLM2_135M
+    r = _run(shape, 5, 64, True, seed=11)
+    _check_against_oracle(shape, 5, 64, r)
 
 
 def test_gemm_paths_bit_identical():
