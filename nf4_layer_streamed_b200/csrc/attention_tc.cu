@@ -1,6 +1,6 @@
 // K10 forward on the 5th-generation tensor cores: causal grouped-query attention
-// softmax(q k^T / sqrt(d) + causal mask) v for head_dim 128 and seq a multiple of 128,
-// the shapes of the Llama-8B layer
+// softmax(q k^T / sqrt(d) + causal mask) v for head_dim 128 and seq a multiple of 128
+// (up to 8192), the shapes of the Llama-8B and 32B-class layers
 // ("Soup 层流式 NF4 训练实测：在 4 GB 显存上以位级一致标准完成 8B 模型 LoRA 微调"
 // §2.1: the HF Llama layer body; the workloads' seq 512).
 //
@@ -953,7 +953,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
 }  // namespace
 
 bool attention_fwd_tc_supported(int seq, int d, int nq, int nkv, int ldq, int ldkv, int ldo) {
-  return d == 128 && seq % TT == 0 && seq <= 4 * TT && nq % nkv == 0 && ldq % 8 == 0 && ldkv % 8 == 0 &&
+  return d == 128 && seq % TT == 0 && seq <= 64 * TT && nq % nkv == 0 && ldq % 8 == 0 && ldkv % 8 == 0 &&
          ldo % 8 == 0;
 }
 

@@ -192,7 +192,8 @@ def test_pair_tile_heights_give_identical_results(M, rows, cols):
 
 
 @pytest.mark.parametrize("shape,batch,seq", [(synth.SMOLLM2_135M, 1, 512), (synth.LLAMA_8B, 2, 128),
-                                             (synth.LLAMA_8B, 2, 384), (synth.LLAMA_8B, 1, 512)])
+                                             (synth.LLAMA_8B, 2, 384), (synth.LLAMA_8B, 1, 512),
+                                             (synth.QWEN_32B_CLASS, 1, 1024)])
 def test_attention_forward_against_oracle(shape, batch, seq):
     cfg = api.layer_cfg(shape, batch, seq)
     M = batch * seq
@@ -207,9 +208,9 @@ def test_attention_forward_against_oracle(shape, batch, seq):
     close(o, ref.reshape(M, qd), what="attention out")
 
 
-@pytest.mark.parametrize("seq", [128, 384, 512])
+@pytest.mark.parametrize("seq", [128, 384, 512, 1024])
 def test_tcgen05_attention_matches_mma_sync_attention(seq):
-    """The tcgen05 forward (head_dim 128, whole-row softmax in TMEM) against the
+    """The tcgen05 forward (head_dim 128, online softmax over key tiles in TMEM) against the
     mma.sync forward on the same GQA inputs: outputs within 1e-2 max|ref|, the
     log-sum-exp within 1e-4, and bit-exact across reruns."""
     shape = synth.LLAMA_8B
@@ -235,7 +236,7 @@ def test_tcgen05_attention_matches_mma_sync_attention(seq):
     assert st == 0, err
 
 
-@pytest.mark.parametrize("batch,seq", [(2, 128), (2, 384), (1, 512)])
+@pytest.mark.parametrize("batch,seq", [(2, 128), (2, 384), (1, 512), (1, 1024)])
 def test_tcgen05_attention_backward_against_oracle(batch, seq):
     """The tcgen05 attention backward (query side: dQ and delta; key side: dK, dV over
     the query heads of each kv group) on the Llama-8B head layout, against the oracle's

@@ -15,7 +15,7 @@ import torch
 
 from nf4_layer_streamed_b200 import api, binding as B, synth
 from oracle import model as omodel
-from tests.helpers import LOSS_RTOL, close, f64, oracle_lora, oracle_weights
+from tests.helpers import LOSS_RTOL, TOL, close, f64, oracle_lora, oracle_weights
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -141,9 +141,16 @@ def test_smollm2_30_layers_first_step_against_oracle():
         loss, og, _ = omodel.forward_backward(ids.cpu().numpy(), layers, loras, emb, None,
                                               np.ones(shape.hidden), shape, wl.batch, wl.seq, rnd=True)
         assert abs(loss_gpu - loss) <= LOSS_RTOL * abs(loss), (loss_gpu, loss)
+        # through 30 layers the oracle's own bf16 roundings move the first layer's dB by
+        # about 1.6% of max|ref| (its run with and without them); where twice that exceeds
+        # 2e-2 it is the bound, as for the 8B two-layer model (tests/test_gpu_oracle_parity.py)
+        _, ex, _ = omodel.forward_backward(ids.cpu().numpy(), layers, loras, emb, None,
+                                           np.ones(shape.hidden), shape, wl.batch, wl.seq, rnd=False)
         for i in (0, wl.n_layers - 1):
-            close(grads[i]["dB_q"], og[i]["dB_q"], what=f"layer {i} dB_q")
-            close(grads[i]["dB_v"], og[i]["dB_v"], what=f"layer {i} dB_v")
+            for k in ("dB_q", "dB_v"):
+                floor = float(np.max(np.abs(og[i][k] - ex[i][k])))
+                tol = max(TOL, 2.0 * floor / float(np.max(np.abs(og[i][k]))))
+                close(grads[i][k], og[i][k], tol, what=f"layer {i} {k} (noise floor {floor:.3e})")
         # second step: B is now nonzero, so dA is nonzero in every layer
         m.adamw_step()
         ids2 = synth.token_ids(wl.vocab, wl.batch, wl.seq, wl.seed, step=1, device=DEV)
