@@ -494,7 +494,7 @@ int attention_fwd(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfl
                   __nv_bfloat16* o, int ldo, float* lse, int batch, int seq, int nq, int nkv, int d, cudaStream_t s) {
   NF4_TRY(check_attn(seq, nq, nkv, d, ldq, ldkv));
   if (attention_tc() && attention_fwd_tc_supported(seq, d, nq, nkv, ldq, ldkv, ldo))
-    return attention_fwd_tc(q, k, v, ldq, ldkv, o, ldo, lse, batch, seq, nq, nkv, s);
+    return attention_fwd_tc(q, k, v, ldq, ldkv, o, ldo, lse, batch, seq, nq, nkv, d, s);
   const float scale_log2 = (1.0f / sqrtf((float)d)) * kLog2e;
   dim3 grid(seq / TQ, nq, batch);
   if (d == 128) {
@@ -519,8 +519,8 @@ int attention_bwd(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfl
   NF4_TRY(check_attn(seq, nq, nkv, d, ldq, ldkv));
   const int M = batch * seq;
   const float scale = 1.0f / sqrtf((float)d);
-  if (attention_tc() && attention_fwd_tc_supported(seq, d, nq, nkv, ldq, ldkv, ldo) && ld_dq % 8 == 0 &&
-      ld_dkv % 8 == 0)  // the tcgen05 query-side kernel forms delta itself
+  if (attention_tc() && attention_bwd_tc_supported(seq, d, nq, nkv, ldq, ldkv, ldo, ld_dq, ld_dkv))
+    // the tcgen05 query-side kernel forms delta itself
     return attention_bwd_tc(q, k, v, ldq, ldkv, o, dout, ldo, lse, delta, dq, dk, dv, ld_dq, ld_dkv, batch, seq, nq,
                             nkv, s);
   k_attn_delta<<<(M * nq + 7) / 8, 256, 0, s>>>(o, dout, ldo, M, seq, nq, d, delta);

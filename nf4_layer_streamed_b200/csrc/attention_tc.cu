@@ -121,7 +121,9 @@ __device__ __forceinline__ void umma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, u
       : "memory");
 }
 
+template <int D>
 __global__ void __launch_bounds__(F_THREADS, 2) k_attn_fwd_tc(const __grid_constant__ AttnTcParams p) {
+  constexpr int NA = D / 64, KS = D / 16, TB = NA * ATOM;  // swizzle atoms, k-steps and bytes of a tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + F_OFF_BAR);
@@ -172,19 +174,19 @@ __global__ void __launch_bounds__(F_THREADS, 2) k_attn_fwd_tc(const __grid_const
       tma_prefetch_desc(&p.tq);
       tma_prefetch_desc(&p.tk);
       tma_prefetch_desc(&p.tv);
-      mbar_arrive_expect_tx(q_full, TILE_BYTES);
-      for (int j = 0; j < 2; ++j) tma_load_2d(base + F_OFF_Q + j * ATOM, &p.tq, q_full, h * 128 + 64 * j, row0 + qt * TT);
+      mbar_arrive_expect_tx(q_full, TB);
+      for (int j = 0; j < NA; ++j) tma_load_2d(base + F_OFF_Q + j * ATOM, &p.tq, q_full, h * D + 64 * j, row0 + qt * TT);
       int issued_k = 0, issued_v = 0;
       for (int kt = 0; kt < nk; ++kt) {
         if (kt > 0 && !mbar_wait(k_empty, (kt - 1) & 1, abort_flag, p.err, KID_ATTN, 21)) break;
-        mbar_arrive_expect_tx(k_full, TILE_BYTES);
-        for (int j = 0; j < 2; ++j)
-          tma_load_2d(base + F_OFF_K + j * ATOM, &p.tk, k_full, kvh * 128 + 64 * j, row0 + kt * TT);
+        mbar_arrive_expect_tx(k_full, TB);
+        for (int j = 0; j < NA; ++j)
+          tma_load_2d(base + F_OFF_K + j * ATOM, &p.tk, k_full, kvh * D + 64 * j, row0 + kt * TT);
         issued_k = kt + 1;
         if (kt > 0 && !mbar_wait(v_empty, (kt - 1) & 1, abort_flag, p.err, KID_ATTN, 22)) break;
-        mbar_arrive_expect_tx(v_full, TILE_BYTES);
-        for (int j = 0; j < 2; ++j)
-          tma_load_2d(base + F_OFF_V + j * ATOM, &p.tv, v_full, kvh * 128 + 64 * j, row0 + kt * TT);
+        mbar_arrive_expect_tx(v_full, TB);
+        for (int j = 0; j < NA; ++j)
+          tma_load_2d(base + F_OFF_V + j * ATOM, &p.tv, v_full, kvh * D + 64 * j, row0 + kt * TT);
         issued_v = kt + 1;
       }
       if (*abort_flag) {  // let the copies already issued land before the CTA exits
@@ -196,7 +198,7 @@ __global__ void __launch_bounds__(F_THREADS, 2) k_attn_fwd_tc(const __grid_const
   } else if (warp == F_MMA) {
     // ------------------------------------------------------------------ MMA issuer
     constexpr uint32_t idesc_s = idesc_bf16(128, 128, false);  // Q K^T: both K-major
-    constexpr uint32_t idesc_o = idesc_bf16(128, 128, true);   // P V: V N-major
+    constexpr uint32_t idesc_o = idesc_bf16(128, D, true);     // P V: V N-major
     const uint32_t sQ = smem_u32(base + F_OFF_Q), sK = smem_u32(base + F_OFF_K), sV = smem_u32(base + F_OFF_V);
     // every wait is agreed on by the whole warp (__all_sync), so that no lane goes on alone
     bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort_flag, p.err, KID_ATTN, 23));
@@ -207,7 +209,7 @@ __global__ void __launch_bounds__(F_THREADS, 2) k_attn_fwd_tc(const __grid_const
         // tcgen05.mma of one thread run in issue order, so S may overwrite the P that
         // the previous tile's P V product reads
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
+        for (int ks = 0; ks < KS; ++ks) {
           const uint32_t off = (ks >> 2) * ATOM + (ks & 3) * 32;
           umma_bf16(tmem, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024), idesc_s, ks ? 1u : 0u);
         }
@@ -263,7 +265,7 @@ __global__ void __launch_bounds__(F_THREADS, 2) k_attn_fwd_tc(const __grid_const
         tc_fence_after();
         const float alpha = resc ? fast_exp2(m_run - m_new) : 1.0f;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < D / 32; ++c) {
           uint32_t v[32];
           tmem_ld32(trow + 128 + c * 32, v);
           tmem_wait_ld();
@@ -313,7 +315,7 @@ __global__ void __launch_bounds__(F_THREADS, 2) k_attn_fwd_tc(const __grid_const
       const float inv = 1.0f / l_run;
       const uint32_t tile = smem_u32(base + F_OFF_Q);
 #pragma unroll
-      for (int c = 0; c < 4; c += 2) {
+      for (int c = 0; c < D / 32; c += 2) {
         uint32_t v[2][32];
         tmem_ld32(trow + 128 + c * 32, v[0]);
         tmem_ld32(trow + 128 + c * 32 + 32, v[1]);
@@ -326,7 +328,7 @@ __global__ void __launch_bounds__(F_THREADS, 2) k_attn_fwd_tc(const __grid_const
     fence_proxy_async_smem();
     asm volatile("bar.sync 1, 128;" ::: "memory");
     if (threadIdx.x == 0 && !*abort_flag) {
-      for (int j = 0; j < 2; ++j) tma_store_2d(&p.to, smem_u32(base + F_OFF_Q + j * ATOM), h * 128 + 64 * j, row0 + qt * TT);
+      for (int j = 0; j < NA; ++j) tma_store_2d(&p.to, smem_u32(base + F_OFF_Q + j * ATOM), h * D + 64 * j, row0 + qt * TT);
       tma_store_drain();
     }
   }
@@ -953,38 +955,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
 }  // namespace
 
 bool attention_fwd_tc_supported(int seq, int d, int nq, int nkv, int ldq, int ldkv, int ldo) {
-  return d == 128 && seq % TT == 0 && seq <= 64 * TT && nq % nkv == 0 && ldq % 8 == 0 && ldkv % 8 == 0 &&
-         ldo % 8 == 0;
+  return (d == 64 || d == 128) && seq % TT == 0 && seq <= 64 * TT && nq % nkv == 0 && ldq % 8 == 0 &&
+         ldkv % 8 == 0 && ldo % 8 == 0;
 }
 
+bool attention_bwd_tc_supported(int seq, int d, int nq, int nkv, int ldq, int ldkv, int ldo, int ld_dq, int ld_dkv) {
+  return d == 128 && attention_fwd_tc_supported(seq, d, nq, nkv, ldq, ldkv, ldo) && ld_dq % 8 == 0 && ld_dkv % 8 == 0;
+}
+
+namespace {
+template <int D>
+int launch_fwd_tc(const AttnTcParams& p, int batch, int seq, int nq, cudaStream_t s) {
+  static int configured[16] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 16 && !configured[dev]) {
+    NF4_CUDA_TRY(cudaFuncSetAttribute(k_attn_fwd_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_TC));
+    configured[dev] = 1;
+  }
+  k_attn_fwd_tc<D><<<dim3(seq / TT, nq, batch), F_THREADS, SMEM_TC, s>>>(p);
+  note_launch();
+  NF4_CUDA_TRY(cudaGetLastError());
+  return NF4LS_OK;
+}
+}  // namespace
+
 int attention_fwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, int ldq, int ldkv,
-                     __nv_bfloat16* o, int ldo, float* lse, int batch, int seq, int nq, int nkv, cudaStream_t s) {
+                     __nv_bfloat16* o, int ldo, float* lse, int batch, int seq, int nq, int nkv, int d, cudaStream_t s) {
   static_assert(SMEM_TC <= 232448, "shared memory of the tcgen05 attention");
   AttnTcParams p;
   const uint64_t rows = (uint64_t)batch * seq;
-  NF4_TRY(tma_map_bf16(&p.tq, q, (uint64_t)nq * 128, rows, (uint64_t)ldq * 2, 64, TT));
-  NF4_TRY(tma_map_bf16(&p.tk, k, (uint64_t)nkv * 128, rows, (uint64_t)ldkv * 2, 64, TT));
-  NF4_TRY(tma_map_bf16(&p.tv, v, (uint64_t)nkv * 128, rows, (uint64_t)ldkv * 2, 64, TT));
-  NF4_TRY(tma_map_bf16(&p.to, o, (uint64_t)nq * 128, rows, (uint64_t)ldo * 2, 64, TT));
+  NF4_TRY(tma_map_bf16(&p.tq, q, (uint64_t)nq * d, rows, (uint64_t)ldq * 2, 64, TT));
+  NF4_TRY(tma_map_bf16(&p.tk, k, (uint64_t)nkv * d, rows, (uint64_t)ldkv * 2, 64, TT));
+  NF4_TRY(tma_map_bf16(&p.tv, v, (uint64_t)nkv * d, rows, (uint64_t)ldkv * 2, 64, TT));
+  NF4_TRY(tma_map_bf16(&p.to, o, (uint64_t)nq * d, rows, (uint64_t)ldo * 2, 64, TT));
   p.o = o;
   p.lse = lse;
   p.ldo = ldo;
   p.seq = seq;
   p.nq = nq;
   p.nkv = nkv;
-  p.scale_log2 = (1.0f / sqrtf(128.0f)) * 1.4426950408889634f;
+  p.scale_log2 = (1.0f / sqrtf((float)d)) * 1.4426950408889634f;
   p.err = device_error_ptr();
-  static int configured[16] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 16 && !configured[dev]) {
-    NF4_CUDA_TRY(cudaFuncSetAttribute(k_attn_fwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_TC));
-    configured[dev] = 1;
-  }
-  k_attn_fwd_tc<<<dim3(seq / TT, nq, batch), F_THREADS, SMEM_TC, s>>>(p);
-  note_launch();
-  NF4_CUDA_TRY(cudaGetLastError());
-  return NF4LS_OK;
+  return d == 64 ? launch_fwd_tc<64>(p, batch, seq, nq, s) : launch_fwd_tc<128>(p, batch, seq, nq, s);
 }
 
 }  // namespace nf4ls
