@@ -522,7 +522,7 @@ int attention_bwd(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfl
   if (attention_tc() && attention_bwd_tc_supported(seq, d, nq, nkv, ldq, ldkv, ldo, ld_dq, ld_dkv))
     // the tcgen05 query-side kernel forms delta itself
     return attention_bwd_tc(q, k, v, ldq, ldkv, o, dout, ldo, lse, delta, dq, dk, dv, ld_dq, ld_dkv, batch, seq, nq,
-                            nkv, s);
+                            nkv, d, s);
   k_attn_delta<<<(M * nq + 7) / 8, 256, 0, s>>>(o, dout, ldo, M, seq, nq, d, delta);
   note_launch();
   dim3 gq(seq / TQ, nq, batch), gk(nkv, batch, seq / TK);

@@ -101,6 +101,8 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)[32]) { tmem_st32(taddr, r); }
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)[16]) { tmem_st16(taddr, r); }
 
 // 2^x by the hardware approximation (ex2.approx, flush-to-zero): its relative error is
 // far below the bf16 rounding that every probability gets next.
@@ -411,7 +413,10 @@ __device__ __forceinline__ uint32_t packed_col(uint32_t c0, int ks) { return c0 
 // dP = dO V^T take their A operand from TMEM and read only K and V from shared memory
 // (4 KB per 64 tensor-core cycles instead of 8 KB, which is all that shared memory
 // delivers, while the next K and V tiles land in it).
+template <int D>
 __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_constant__ AttnBwdParams p) {
+  // swizzle atoms, k-steps and bytes of a Q / dO / O / K / V tile; dims per column half
+  constexpr int NA = D / 64, KS = D / 16, TB = NA * ATOM, DH = D / 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + B_OFF_BAR);
@@ -467,23 +472,23 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
       tma_prefetch_desc(&p.tv);
       tma_prefetch_desc(&p.tdo);
       tma_prefetch_desc(&p.to);
-      mbar_arrive_expect_tx(q_full, 2 * TILE_BYTES);
-      for (int j = 0; j < 2; ++j) {
-        tma_load_2d(base + B_OFF_A + j * ATOM, &p.tq, q_full, h * 128 + 64 * j, row0 + qt * TT);
-        tma_load_2d(base + B_OFF_A + TILE_BYTES + j * ATOM, &p.tdo, q_full, h * 128 + 64 * j, row0 + qt * TT);
+      mbar_arrive_expect_tx(q_full, 2 * TB);
+      for (int j = 0; j < NA; ++j) {
+        tma_load_2d(base + B_OFF_A + j * ATOM, &p.tq, q_full, h * D + 64 * j, row0 + qt * TT);
+        tma_load_2d(base + B_OFF_A + TILE_BYTES + j * ATOM, &p.tdo, q_full, h * D + 64 * j, row0 + qt * TT);
       }
-      mbar_arrive_expect_tx(o_full, TILE_BYTES);
-      for (int j = 0; j < 2; ++j)
-        tma_load_2d(base + B_OFF_X + j * ATOM, &p.to, o_full, h * 128 + 64 * j, row0 + qt * TT);
+      mbar_arrive_expect_tx(o_full, TB);
+      for (int j = 0; j < NA; ++j)
+        tma_load_2d(base + B_OFF_X + j * ATOM, &p.to, o_full, h * D + 64 * j, row0 + qt * TT);
       int issued = 0;
       for (int kt = 0; kt < n_kt; ++kt) {
         const int st = kt & 1;
         if (kt >= 2 && !mbar_wait(&kv_empty[st], ((kt >> 1) - 1) & 1, abort_flag, p.err, KID_ATTN, 41)) break;
         uint8_t* buf = base + B_OFF_RING + st * 2 * TILE_BYTES;
-        mbar_arrive_expect_tx(&kv_full[st], 2 * TILE_BYTES);
-        for (int j = 0; j < 2; ++j) {
-          tma_load_2d(buf + j * ATOM, &p.tk, &kv_full[st], kvh * 128 + 64 * j, row0 + kt * TT);
-          tma_load_2d(buf + TILE_BYTES + j * ATOM, &p.tv, &kv_full[st], kvh * 128 + 64 * j, row0 + kt * TT);
+        mbar_arrive_expect_tx(&kv_full[st], 2 * TB);
+        for (int j = 0; j < NA; ++j) {
+          tma_load_2d(buf + j * ATOM, &p.tk, &kv_full[st], kvh * D + 64 * j, row0 + kt * TT);
+          tma_load_2d(buf + TILE_BYTES + j * ATOM, &p.tv, &kv_full[st], kvh * D + 64 * j, row0 + kt * TT);
         }
         issued = kt + 1;
       }
@@ -495,7 +500,7 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
     }
   } else if (warp == B_MMA) {
     constexpr uint32_t idesc_s = idesc_bf16(128, 128, false);  // S, dP: N = 128 keys
-    constexpr uint32_t idesc_a = idesc_bf16(128, 128, true);   // dQ += dS K: K N-major
+    constexpr uint32_t idesc_a = idesc_bf16(128, D, true);     // dQ += dS K: K N-major
     bool ok = __all_sync(0xffffffffu, mbar_wait(qa_full, 0, abort_flag, p.err, KID_ATTN, 42)) && !*abort_flag;
     // dQ += dS_kt K_kt, each half as soon as its dS chunks are in TMEM (chunk hc holds the
     // k-steps with ks & 2 == 2 hc); then the K/V stage is free
@@ -527,7 +532,7 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
       if (lane == 0) {
         const uint32_t sK = smem_u32(base + B_OFF_RING + (kt & 1) * 2 * TILE_BYTES), sV = sK + TILE_BYTES;
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {  // over the head dim: Q, dO columns 8 ks .. in TMEM
+        for (int ks = 0; ks < KS; ++ks) {  // over the head dim: Q, dO columns 8 ks .. in TMEM
           const uint32_t off = (ks >> 2) * ATOM + (ks & 3) * 32;
           umma_bf16_ta(tmem, tmem + T_Q + ks * 8, sdesc_sw128(sK + off, 16, 1024), idesc_s, ks ? 1u : 0u);
           umma_bf16_ta(tmem + 128, tmem + T_DO + ks * 8, sdesc_sw128(sV + off, 16, 1024), idesc_s, ks ? 1u : 0u);
@@ -547,26 +552,27 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
     const uint32_t trow = tmem + ((uint32_t)(wq * 32) << 16);
     const size_t li = ((size_t)b * p.nq + h) * p.seq + qpos;
     // First Q and dO into TMEM (the MMA warp starts on them), then delta = rowsum(dO * O)
-    // over this thread's 64 dims (its row in swizzle atom g of the dO and O tiles), the two
-    // halves added through smem.  Chunk c of the row holds dims 8 c .. 8 c + 7 of the atom,
-    // TMEM column 32 g + 4 c + i their pair i.
+    // over this thread's DH dims (dims g DH .. of its row: 16-byte chunks c0 + c of swizzle
+    // atom g DH / 64 of the dO and O tiles), the two halves added through smem.  TMEM
+    // column g DH / 2 + 4 c + i holds the pair i of chunk c.
     float* red = reinterpret_cast<float*>(base + B_OFF_X + TILE_BYTES);
-    const uint8_t* q_row = base + B_OFF_A + g * ATOM + r * 128;
-    const uint8_t* dO_row = base + B_OFF_A + TILE_BYTES + g * ATOM + r * 128;
-    const uint8_t* o_row = base + B_OFF_X + g * ATOM + r * 128;
+    const int atom = (g * DH) / 64, c0 = ((g * DH) % 64) / 8;
+    const uint8_t* q_row = base + B_OFF_A + atom * ATOM + r * 128;
+    const uint8_t* dO_row = base + B_OFF_A + TILE_BYTES + atom * ATOM + r * 128;
+    const uint8_t* o_row = base + B_OFF_X + atom * ATOM + r * 128;
     bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort_flag, p.err, KID_ATTN, 45));
     if (ok) {
-      uint32_t qv[32], dv[32];
+      uint32_t qv[DH / 2], dv[DH / 2];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint32_t off = (uint32_t)((c ^ (r & 7)) << 4);
+      for (int c = 0; c < DH / 8; ++c) {
+        const uint32_t off = (uint32_t)(((c0 + c) ^ (r & 7)) << 4);
         const uint4 d = *reinterpret_cast<const uint4*>(dO_row + off);
         const uint4 q = *reinterpret_cast<const uint4*>(q_row + off);
         qv[4 * c] = q.x, qv[4 * c + 1] = q.y, qv[4 * c + 2] = q.z, qv[4 * c + 3] = q.w;
         dv[4 * c] = d.x, dv[4 * c + 1] = d.y, dv[4 * c + 2] = d.z, dv[4 * c + 3] = d.w;
       }
-      tmem_st32(trow + T_Q + g * 32, qv);
-      tmem_st32(trow + T_DO + g * 32, dv);
+      tmem_st_cols(trow + T_Q + g * (DH / 2), qv);
+      tmem_st_cols(trow + T_DO + g * (DH / 2), dv);
       tmem_wait_st();
     }
     tc_fence_before();
@@ -576,8 +582,8 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
     if (ok) {
       float s = 0.f;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint32_t off = (uint32_t)((c ^ (r & 7)) << 4);
+      for (int c = 0; c < DH / 8; ++c) {
+        const uint32_t off = (uint32_t)(((c0 + c) ^ (r & 7)) << 4);
         const uint4 a = *reinterpret_cast<const uint4*>(o_row + off);
         const uint4 d = *reinterpret_cast<const uint4*>(dO_row + off);
         const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, dw[4] = {d.x, d.y, d.z, d.w};
@@ -628,19 +634,19 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
     // elementwise warp reaches the barrier, the store is issued only when no wait failed
     if (ok && __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, p.err, KID_ATTN, 47))) {
       tc_fence_after();
-      uint32_t v[2][32];
-      tmem_ld32(trow + 256 + g * 64, v[0]);
-      tmem_ld32(trow + 256 + g * 64 + 32, v[1]);
+      uint32_t v[DH / 32][32];
+#pragma unroll
+      for (int i = 0; i < DH / 32; ++i) tmem_ld32(trow + 256 + g * DH + 32 * i, v[i]);
       tmem_wait_ld();
       const uint32_t tile = smem_u32(base + B_OFF_RING);
-      stage_row32(tile, r, 2 * g, v[0], p.scale);
-      stage_row32(tile, r, 2 * g + 1, v[1], p.scale);
+#pragma unroll
+      for (int i = 0; i < DH / 32; ++i) stage_row32(tile, r, g * (DH / 32) + i, v[i], p.scale);
     }
     fence_proxy_async_smem();
     bar_ew();
     if (threadIdx.x == 0 && !*abort_flag) {
-      for (int j = 0; j < 2; ++j)
-        tma_store_2d(&p.tdq, smem_u32(base + B_OFF_RING + j * ATOM), h * 128 + 64 * j, row0 + qt * TT);
+      for (int j = 0; j < NA; ++j)
+        tma_store_2d(&p.tdq, smem_u32(base + B_OFF_RING + j * ATOM), h * D + 64 * j, row0 + qt * TT);
       tma_store_drain();
     }
   }
@@ -678,8 +684,11 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t
 // per key tile instead of one, the first key tiles holding the most query tiles).
 constexpr int PEER_LD = 132;  // row stride (floats) of the partial sums in the first CTA's smem
 
+template <int D>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
     k_attn_dkv_tc(const __grid_constant__ AttnBwdParams p) {
+  // swizzle atoms, k-steps and bytes of a K / V / Q / dO tile; dims per column half
+  constexpr int NA = D / 64, KS = D / 16, TB = NA * ATOM, DH = D / 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + B_OFF_BAR);
@@ -733,10 +742,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
       tma_prefetch_desc(&p.tk);
       tma_prefetch_desc(&p.tv);
       tma_prefetch_desc(&p.tdo);
-      mbar_arrive_expect_tx(kv_full, 2 * TILE_BYTES);
-      for (int j = 0; j < 2; ++j) {
-        tma_load_2d(base + B_OFF_A + j * ATOM, &p.tk, kv_full, kvh * 128 + 64 * j, row0 + kt * TT);
-        tma_load_2d(base + B_OFF_A + TILE_BYTES + j * ATOM, &p.tv, kv_full, kvh * 128 + 64 * j, row0 + kt * TT);
+      mbar_arrive_expect_tx(kv_full, 2 * TB);
+      for (int j = 0; j < NA; ++j) {
+        tma_load_2d(base + B_OFF_A + j * ATOM, &p.tk, kv_full, kvh * D + 64 * j, row0 + kt * TT);
+        tma_load_2d(base + B_OFF_A + TILE_BYTES + j * ATOM, &p.tv, kv_full, kvh * D + 64 * j, row0 + kt * TT);
       }
       int issued = 0;
       for (int sti = 0; sti < n_st; ++sti) {
@@ -745,10 +754,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
         const int h = kvh * grp + h_begin + sti / per_head, qt = kt + sti % per_head;
         uint8_t* buf = base + B_OFF_RING + bf * 2 * TILE_BYTES;
         float* ld = reinterpret_cast<float*>(base + B_OFF_X + bf * 1024);
-        mbar_arrive_expect_tx(&qd_full[bf], 2 * TILE_BYTES + 1024);
-        for (int j = 0; j < 2; ++j) {
-          tma_load_2d(buf + j * ATOM, &p.tq, &qd_full[bf], h * 128 + 64 * j, row0 + qt * TT);
-          tma_load_2d(buf + TILE_BYTES + j * ATOM, &p.tdo, &qd_full[bf], h * 128 + 64 * j, row0 + qt * TT);
+        mbar_arrive_expect_tx(&qd_full[bf], 2 * TB + 1024);
+        for (int j = 0; j < NA; ++j) {
+          tma_load_2d(buf + j * ATOM, &p.tq, &qd_full[bf], h * D + 64 * j, row0 + qt * TT);
+          tma_load_2d(buf + TILE_BYTES + j * ATOM, &p.tdo, &qd_full[bf], h * D + 64 * j, row0 + qt * TT);
         }
         const size_t lo = ((size_t)b * p.nq + h) * p.seq + qt * TT;
         bulk_load(ld, p.lse + lo, 512, &qd_full[bf]);
@@ -762,7 +771,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
     }
   } else if (warp == B_MMA) {
     constexpr uint32_t idesc_s = idesc_bf16(128, 128, false);  // S^T, dP^T: N = 128 queries
-    constexpr uint32_t idesc_a = idesc_bf16(128, 128, true);   // dV, dK: dO, Q N-major
+    constexpr uint32_t idesc_a = idesc_bf16(128, D, true);     // dV, dK: dO, Q N-major
     const uint32_t sK = smem_u32(base + B_OFF_A), sV = sK + TILE_BYTES;
     bool ok = n_st > 0 && __all_sync(0xffffffffu, mbar_wait(kv_full, 0, abort_flag, p.err, KID_ATTN, 32));
     // dV += P^T dO, dK += dS^T Q, each half as soon as its chunks are in TMEM (chunk hc holds
@@ -797,7 +806,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
       if (lane == 0) {
         const uint32_t sQ = smem_u32(base + B_OFF_RING + (sti & 1) * 2 * TILE_BYTES), sO = sQ + TILE_BYTES;
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {  // S^T = K Q^T, dP^T = V dO^T over the head dim
+        for (int ks = 0; ks < KS; ++ks) {  // S^T = K Q^T, dP^T = V dO^T over the head dim
           const uint32_t off = (ks >> 2) * ATOM + (ks & 3) * 32;
           umma_bf16(tmem, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024), idesc_s, ks ? 1u : 0u);
           umma_bf16(tmem + 128, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sO + off, 16, 1024), idesc_s,
@@ -863,16 +872,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
     constexpr uint32_t PEER_BYTES = 128 * PEER_LD * 4;              // one tensor's partial sums
     if (crank == 1) {  // this CTA's ring is free: stage the partial sums there (zeros if none)
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < DH / 32; ++c) {
         uint32_t v[32], k[32];
         if (have) {
-          tmem_ld32(trow + 256 + g * 64 + c * 32, v);
-          tmem_ld32(trow + 384 + g * 64 + c * 32, k);
+          tmem_ld32(trow + 256 + g * DH + c * 32, v);
+          tmem_ld32(trow + 384 + g * DH + c * 32, k);
           tmem_wait_ld();
         }
 #pragma unroll
         for (int q4 = 0; q4 < 8; ++q4) {
-          const uint32_t o = smem_u32(peer + r * PEER_LD + g * 64 + c * 32 + 4 * q4);
+          const uint32_t o = smem_u32(peer + r * PEER_LD + g * DH + c * 32 + 4 * q4);
           if (have) {
             st_shared_v4(o, v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
             st_shared_v4(o + PEER_BYTES, k[4 * q4], k[4 * q4 + 1], k[4 * q4 + 2], k[4 * q4 + 3]);
@@ -903,31 +912,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
       const uint32_t tv = smem_u32(base + B_OFF_A), tk = tv + TILE_BYTES;
       const float sc = p.scale;
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < DH / 32; ++c) {
         float v[32], k[32];
         uint32_t vr[32], kr[32];
         if (have) {
-          tmem_ld32(trow + 256 + g * 64 + c * 32, vr);
-          tmem_ld32(trow + 384 + g * 64 + c * 32, kr);
+          tmem_ld32(trow + 256 + g * DH + c * 32, vr);
+          tmem_ld32(trow + 384 + g * DH + c * 32, kr);
           tmem_wait_ld();
         }
-        const float* pv = peer + r * PEER_LD + g * 64 + c * 32;
+        const float* pv = peer + r * PEER_LD + g * DH + c * 32;
         const float* pk = pv + 128 * PEER_LD;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           v[i] = (have ? __uint_as_float(vr[i]) : 0.f) + pv[i];
           k[i] = ((have ? __uint_as_float(kr[i]) : 0.f) + pk[i]) * sc;
         }
-        stage_row32(tv, r, 2 * g + c, v);
-        stage_row32(tk, r, 2 * g + c, k);
+        stage_row32(tv, r, g * (DH / 32) + c, v);
+        stage_row32(tk, r, g * (DH / 32) + c, k);
       }
       fence_proxy_async_smem();
       bar_ew();
       (void)got;
       if (threadIdx.x == 0 && !*abort_flag) {
-        for (int j = 0; j < 2; ++j) {
-          tma_store_2d(&p.tdv, tv + j * ATOM, kvh * 128 + 64 * j, row0 + kt * TT);
-          tma_store_2d(&p.tdk, tk + j * ATOM, kvh * 128 + 64 * j, row0 + kt * TT);
+        for (int j = 0; j < NA; ++j) {
+          tma_store_2d(&p.tdv, tv + j * ATOM, kvh * D + 64 * j, row0 + kt * TT);
+          tma_store_2d(&p.tdk, tk + j * ATOM, kvh * D + 64 * j, row0 + kt * TT);
         }
         tma_store_drain();
       }
@@ -960,7 +969,7 @@ bool attention_fwd_tc_supported(int seq, int d, int nq, int nkv, int ldq, int ld
 }
 
 bool attention_bwd_tc_supported(int seq, int d, int nq, int nkv, int ldq, int ldkv, int ldo, int ld_dq, int ld_dkv) {
-  return d == 128 && attention_fwd_tc_supported(seq, d, nq, nkv, ldq, ldkv, ldo) && ld_dq % 8 == 0 && ld_dkv % 8 == 0;
+  return attention_fwd_tc_supported(seq, d, nq, nkv, ldq, ldkv, ldo) && ld_dq % 8 == 0 && ld_dkv % 8 == 0;
 }
 
 namespace {
@@ -1004,22 +1013,43 @@ int attention_fwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_
 
 namespace nf4ls {
 
+namespace {
+template <int D>
+int launch_bwd_tc(const AttnBwdParams& p, int batch, int seq, int nq, int nkv, cudaStream_t s) {
+  static int configured[16] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 16 && !configured[dev]) {
+    NF4_CUDA_TRY(cudaFuncSetAttribute(k_attn_dq_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BWD));
+    NF4_CUDA_TRY(cudaFuncSetAttribute(k_attn_dkv_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BWD));
+    configured[dev] = 1;
+  }
+  // the query side writes delta, which the key side reads
+  k_attn_dq_tc<D><<<dim3(seq / TT, nq, batch), B_THREADS, SMEM_BWD, s>>>(p);
+  note_launch();
+  k_attn_dkv_tc<D><<<dim3(2 * nkv, batch, seq / TT), B_THREADS, SMEM_BWD, s>>>(p);
+  note_launch();
+  NF4_CUDA_TRY(cudaGetLastError());
+  return NF4LS_OK;
+}
+}  // namespace
+
 int attention_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, int ldq, int ldkv,
                      const __nv_bfloat16* o, const __nv_bfloat16* dout, int ldo, const float* lse, float* delta,
                      __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv, int ld_dq, int ld_dkv, int batch, int seq,
-                     int nq, int nkv, cudaStream_t s) {
+                     int nq, int nkv, int d, cudaStream_t s) {
   static_assert(SMEM_BWD <= 232448, "shared memory of the tcgen05 attention backward");
   AttnBwdParams p;
   const uint64_t rows = (uint64_t)batch * seq;
-  NF4_TRY(tma_map_bf16(&p.tq, q, (uint64_t)nq * 128, rows, (uint64_t)ldq * 2, 64, TT));
-  NF4_TRY(tma_map_bf16(&p.tk, k, (uint64_t)nkv * 128, rows, (uint64_t)ldkv * 2, 64, TT));
-  NF4_TRY(tma_map_bf16(&p.tv, v, (uint64_t)nkv * 128, rows, (uint64_t)ldkv * 2, 64, TT));
-  NF4_TRY(tma_map_bf16(&p.tdo, dout, (uint64_t)nq * 128, rows, (uint64_t)ldo * 2, 64, TT));
+  NF4_TRY(tma_map_bf16(&p.tq, q, (uint64_t)nq * d, rows, (uint64_t)ldq * 2, 64, TT));
+  NF4_TRY(tma_map_bf16(&p.tk, k, (uint64_t)nkv * d, rows, (uint64_t)ldkv * 2, 64, TT));
+  NF4_TRY(tma_map_bf16(&p.tv, v, (uint64_t)nkv * d, rows, (uint64_t)ldkv * 2, 64, TT));
+  NF4_TRY(tma_map_bf16(&p.tdo, dout, (uint64_t)nq * d, rows, (uint64_t)ldo * 2, 64, TT));
   if (!aligned(lse, 16) || !aligned(delta, 16)) return fail(NF4LS_ALIGN, "attention backward: lse / delta alignment");
-  NF4_TRY(tma_map_bf16(&p.to, o, (uint64_t)nq * 128, rows, (uint64_t)ldo * 2, 64, TT));
-  NF4_TRY(tma_map_bf16(&p.tdq, dq, (uint64_t)nq * 128, rows, (uint64_t)ld_dq * 2, 64, TT));
-  NF4_TRY(tma_map_bf16(&p.tdk, dk, (uint64_t)nkv * 128, rows, (uint64_t)ld_dkv * 2, 64, TT));
-  NF4_TRY(tma_map_bf16(&p.tdv, dv, (uint64_t)nkv * 128, rows, (uint64_t)ld_dkv * 2, 64, TT));
+  NF4_TRY(tma_map_bf16(&p.to, o, (uint64_t)nq * d, rows, (uint64_t)ldo * 2, 64, TT));
+  NF4_TRY(tma_map_bf16(&p.tdq, dq, (uint64_t)nq * d, rows, (uint64_t)ld_dq * 2, 64, TT));
+  NF4_TRY(tma_map_bf16(&p.tdk, dk, (uint64_t)nkv * d, rows, (uint64_t)ld_dkv * 2, 64, TT));
+  NF4_TRY(tma_map_bf16(&p.tdv, dv, (uint64_t)nkv * d, rows, (uint64_t)ld_dkv * 2, 64, TT));
   p.lse = lse;
   p.delta = delta;
   p.dq = dq;
@@ -1030,24 +1060,10 @@ int attention_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_
   p.seq = seq;
   p.nq = nq;
   p.nkv = nkv;
-  p.scale = 1.0f / sqrtf(128.0f);
+  p.scale = 1.0f / sqrtf((float)d);
   p.scale_log2 = p.scale * 1.4426950408889634f;
   p.err = device_error_ptr();
-  static int configured[16] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 16 && !configured[dev]) {
-    NF4_CUDA_TRY(cudaFuncSetAttribute(k_attn_dq_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BWD));
-    NF4_CUDA_TRY(cudaFuncSetAttribute(k_attn_dkv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BWD));
-    configured[dev] = 1;
-  }
-  // the query side writes delta, which the key side reads
-  k_attn_dq_tc<<<dim3(seq / TT, nq, batch), B_THREADS, SMEM_BWD, s>>>(p);
-  note_launch();
-  k_attn_dkv_tc<<<dim3(2 * nkv, batch, seq / TT), B_THREADS, SMEM_BWD, s>>>(p);
-  note_launch();
-  NF4_CUDA_TRY(cudaGetLastError());
-  return NF4LS_OK;
+  return d == 64 ? launch_bwd_tc<64>(p, batch, seq, nq, nkv, s) : launch_bwd_tc<128>(p, batch, seq, nq, nkv, s);
 }
 
 }  // namespace nf4ls

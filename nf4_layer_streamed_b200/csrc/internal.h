@@ -258,8 +258,7 @@ int rope_bwd(__nv_bfloat16* x, int ld, int M, int cols, int seq, int d, const fl
 // box_cols x box_rows.
 int tma_map_bf16(CUtensorMap* map, const void* ptr, uint64_t cols, uint64_t rows, uint64_t row_bytes,
                  uint32_t box_cols, uint32_t box_rows);
-// The tcgen05 attention (head_dim 64 or 128 forward, 128 backward; seq a multiple of 128
-// up to 8192).
+// The tcgen05 attention (head_dim 64 or 128; seq a multiple of 128 up to 8192).
 bool attention_fwd_tc_supported(int seq, int d, int nq, int nkv, int ldq, int ldkv, int ldo);
 bool attention_bwd_tc_supported(int seq, int d, int nq, int nkv, int ldq, int ldkv, int ldo, int ld_dq, int ld_dkv);
 int attention_fwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, int ldq, int ldkv,
@@ -269,7 +268,7 @@ int attention_fwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_
 int attention_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, int ldq, int ldkv,
                      const __nv_bfloat16* o, const __nv_bfloat16* dout, int ldo, const float* lse, float* delta,
                      __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv, int ld_dq, int ld_dkv, int batch, int seq,
-                     int nq, int nkv, cudaStream_t s);
+                     int nq, int nkv, int d, cudaStream_t s);
 int attention_fwd(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, int ldq, int ldkv,
                   __nv_bfloat16* o, int ldo, float* lse, int batch, int seq, int nq, int nkv, int d,
                   cudaStream_t s);
