@@ -1,11 +1,13 @@
 // K10 forward on the 5th-generation tensor cores: causal grouped-query attention
-// softmax(q k^T / sqrt(d) + causal mask) v for head_dim 128 and seq a multiple of 128
-// (up to 8192), the shapes of the Llama-8B and 32B-class layers
+// softmax(q k^T / sqrt(d) + causal mask) v for head_dim 64 or 128 (a template parameter)
+// and seq a multiple of 128 (up to 8192): the shapes of the SmolLM2-shaped, Llama-8B and
+// 32B-class layers
 // ("Soup 层流式 NF4 训练实测：在 4 GB 显存上以位级一致标准完成 8B 模型 LoRA 微调"
 // §2.1: the HF Llama layer body; the workloads' seq 512).
 //
 // One CTA per (128-query tile, query head, sequence), two CTAs per SM: 96 KB of shared
-// memory (the Q tile and one K and one V tile) and 256 TMEM columns each, so that one
+// memory (the Q tile and one K and one V tile, a 32 KB slot each, the first half of which
+// a head_dim-64 tile uses) and 256 TMEM columns each, so that one
 // CTA's softmax runs while the other's products keep the tensor core busy.  Per key
 // tile kt = 0 .. qt (online softmax, one query row per thread of four warps):
 //   1. S = Q K_kt^T (tcgen05.mma, M = N = 128, K = 16 steps) into TMEM columns [0, 128).
