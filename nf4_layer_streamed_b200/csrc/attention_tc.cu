@@ -144,8 +144,10 @@ __global__ void __launch_bounds__(F_THREADS, 2) k_attn_fwd_tc(const __grid_const
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = gridDim.x - 1 - blockIdx.x;  // longest rows first
-  const int h = blockIdx.y, b = blockIdx.z;
+  // z slowest: every head's longest query rows first, then the next tile height, so the
+  // shortest CTAs fill the last wave
+  const int qt = gridDim.z - 1 - blockIdx.z;
+  const int h = blockIdx.x, b = blockIdx.y;
   const int kvh = h / (p.nq / p.nkv);
   const int nk = qt + 1;                      // key tiles at or before the diagonal
   const int row0 = b * p.seq;
@@ -435,7 +437,7 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
   uint64_t* o_full = bars + 13;     // the O tile (for delta)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = gridDim.x - 1 - blockIdx.x, h = blockIdx.y, b = blockIdx.z;  // longest rows first
+  const int qt = gridDim.z - 1 - blockIdx.z, h = blockIdx.x, b = blockIdx.y;  // z slowest: longest rows first
   const int kvh = h / (p.nq / p.nkv);
   const int n_kt = qt + 1;  // key tiles at or before the diagonal
   const int row0 = b * p.seq;
@@ -678,13 +680,14 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t
 }
 
 // KEY side: dK, dV of one 128-key tile of one kv head, by a cluster of two CTAs that split
-// the group's query heads (the first ceil(group / 2) heads and the rest): the second CTA
-// stages its fp32 partial sums in its own shared memory and sends them in two bulk copies
-// into the first CTA's (distributed shared memory; per-thread remote stores of the same
-// 132 KB measured about 13 000 cycles), and the first adds them to its own in that fixed
-// order.  Halving the longest CTAs' work balances the grid (two CTAs
-// per key tile instead of one, the first key tiles holding the most query tiles).
-constexpr int PEER_LD = 132;  // row stride (floats) of the partial sums in the first CTA's smem
+// the group's query heads (the first ceil(group / 2) heads and the rest).  Each CTA then
+// finishes one of the two tensors: it stages the other tensor's fp32 partial sums in its own
+// shared memory and sends them in one bulk copy into the peer's (distributed shared memory),
+// and adds the peer's to its own in the order first CTA + second CTA.  Halving the longest
+// CTAs' work balances the grid (two CTAs per key tile instead of one, the first key tiles
+// holding the most query tiles); splitting the exchange halves the copy and the final pass
+// of each CTA (per-thread remote stores of both tensors, 132 KB, from one CTA measured
+// about 13 000 cycles).
 
 template <int D>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
@@ -870,79 +873,69 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
     }
     const bool have = n_st > 0 && ok && __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, p.err, KID_ATTN, 36));
     if (have) tc_fence_after();
-    float* peer = reinterpret_cast<float*>(base + B_OFF_RING);  // dV [128][PEER_LD], then dK
-    constexpr uint32_t PEER_BYTES = 128 * PEER_LD * 4;              // one tensor's partial sums
-    if (crank == 1) {  // this CTA's ring is free: stage the partial sums there (zeros if none)
+    // The partial sums cross over: the first CTA finishes dV and the second dK, so each sends
+    // the other tensor (fp32 rows of D floats, 16-byte chunks swizzled by row) from the start
+    // of its freed ring into the back half of the peer's ring.
+    constexpr uint32_t PB = 128u * D * 4u;  // one tensor's partial sums
+    const uint32_t ring = smem_u32(base + B_OFF_RING);
+    const uint32_t t_send = trow + (crank == 0 ? 384u : 256u), t_keep = trow + (crank == 0 ? 256u : 384u);
+    const uint32_t prow = (uint32_t)r * (D * 4);
 #pragma unroll
-      for (int c = 0; c < DH / 32; ++c) {
-        uint32_t v[32], k[32];
-        if (have) {
-          tmem_ld32(trow + 256 + g * DH + c * 32, v);
-          tmem_ld32(trow + 384 + g * DH + c * 32, k);
-          tmem_wait_ld();
-        }
-#pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-          const uint32_t o = smem_u32(peer + r * PEER_LD + g * DH + c * 32 + 4 * q4);
-          if (have) {
-            st_shared_v4(o, v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
-            st_shared_v4(o + PEER_BYTES, k[4 * q4], k[4 * q4 + 1], k[4 * q4 + 2], k[4 * q4 + 3]);
-          } else {
-            st_shared_v4(o, 0u, 0u, 0u, 0u);
-            st_shared_v4(o + PEER_BYTES, 0u, 0u, 0u, 0u);
-          }
-        }
+    for (int c = 0; c < DH / 32; ++c) {
+      uint32_t v[32];
+      if (have) {
+        tmem_ld32(t_send + g * DH + c * 32, v);
+        tmem_wait_ld();
       }
-      fence_proxy_async_smem();
-      bar_ew();
-    } else if (threadIdx.x == 0) {
-      mbar_arrive_expect_tx(peer_full, 2 * PEER_BYTES);
+#pragma unroll
+      for (int q4 = 0; q4 < 8; ++q4) {
+        const uint32_t o = ring + prow + ((uint32_t)(((g * DH + c * 32) / 4 + q4) ^ (r & 7)) << 4);
+        if (have)
+          st_shared_v4(o, v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+        else
+          st_shared_v4(o, 0u, 0u, 0u, 0u);
+      }
     }
-    // both CTAs have finished their products: the first CTA's ring is free for the partials
+    fence_proxy_async_smem();
+    if (threadIdx.x == 0) mbar_arrive_expect_tx(peer_full, PB);
+    bar_ew();
+    // both CTAs have finished their products: both rings are free
     cluster_sync_all();
-    if (crank == 1 && threadIdx.x == 0) {
-      const uint32_t dst = mapa_shared(smem_u32(peer), 0), bar = mapa_shared(smem_u32(peer_full), 0);
-      bulk_copy_to_peer(dst, smem_u32(peer), PEER_BYTES, bar);
-      bulk_copy_to_peer(dst + PEER_BYTES, smem_u32(peer) + PEER_BYTES, PEER_BYTES, bar);
+    if (threadIdx.x == 0) {
+      const uint32_t other = crank ^ 1u;
+      bulk_copy_to_peer(mapa_shared(ring + PB, other), ring, PB, mapa_shared(smem_u32(peer_full), other));
     }
-    bool got = true;
-    if (crank == 0) got = __all_sync(0xffffffffu, mbar_wait(peer_full, 0, abort_flag, p.err, KID_ATTN, 37));
-    // the second CTA's shared memory stays until the first has its copy
+    (void)__all_sync(0xffffffffu, mbar_wait(peer_full, 0, abort_flag, p.err, KID_ATTN, 37));
+    // this CTA's tensor (its sums plus the peer's) through the freed K tile's shared memory
+    // and NA TMA stores; dK takes the softmax scale
+    const uint32_t tile = smem_u32(base + B_OFF_A);
+    const float sc = crank == 0 ? 1.0f : p.scale;
+#pragma unroll
+    for (int c = 0; c < DH / 32; ++c) {
+      float v[32];
+      uint32_t vr[32];
+      if (have) {
+        tmem_ld32(t_keep + g * DH + c * 32, vr);
+        tmem_wait_ld();
+      }
+#pragma unroll
+      for (int q4 = 0; q4 < 8; ++q4) {
+        const uint4 in = ld_shared_v4(ring + PB + prow + ((uint32_t)(((g * DH + c * 32) / 4 + q4) ^ (r & 7)) << 4));
+        const float iv[4] = {__uint_as_float(in.x), __uint_as_float(in.y), __uint_as_float(in.z), __uint_as_float(in.w)};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[4 * q4 + e] = ((have ? __uint_as_float(vr[4 * q4 + e]) : 0.f) + iv[e]) * sc;
+      }
+      stage_row32(tile, r, g * (DH / 32) + c, v);
+    }
+    fence_proxy_async_smem();
+    bar_ew();
+    if (threadIdx.x == 0 && !*abort_flag) {
+      const CUtensorMap* map = crank == 0 ? &p.tdv : &p.tdk;
+      for (int j = 0; j < NA; ++j) tma_store_2d(map, tile + j * ATOM, kvh * D + 64 * j, row0 + kt * TT);
+      tma_store_drain();
+    }
+    // the peer has its copy of this CTA's partial sums before this shared memory goes
     cluster_sync_all();
-    if (crank == 0) {
-      // dV, dK through the freed K / V tiles' shared memory and four TMA stores
-      const uint32_t tv = smem_u32(base + B_OFF_A), tk = tv + TILE_BYTES;
-      const float sc = p.scale;
-#pragma unroll
-      for (int c = 0; c < DH / 32; ++c) {
-        float v[32], k[32];
-        uint32_t vr[32], kr[32];
-        if (have) {
-          tmem_ld32(trow + 256 + g * DH + c * 32, vr);
-          tmem_ld32(trow + 384 + g * DH + c * 32, kr);
-          tmem_wait_ld();
-        }
-        const float* pv = peer + r * PEER_LD + g * DH + c * 32;
-        const float* pk = pv + 128 * PEER_LD;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          v[i] = (have ? __uint_as_float(vr[i]) : 0.f) + pv[i];
-          k[i] = ((have ? __uint_as_float(kr[i]) : 0.f) + pk[i]) * sc;
-        }
-        stage_row32(tv, r, g * (DH / 32) + c, v);
-        stage_row32(tk, r, g * (DH / 32) + c, k);
-      }
-      fence_proxy_async_smem();
-      bar_ew();
-      (void)got;
-      if (threadIdx.x == 0 && !*abort_flag) {
-        for (int j = 0; j < NA; ++j) {
-          tma_store_2d(&p.tdv, tv + j * ATOM, kvh * D + 64 * j, row0 + kt * TT);
-          tma_store_2d(&p.tdk, tk + j * ATOM, kvh * D + 64 * j, row0 + kt * TT);
-        }
-        tma_store_drain();
-      }
-    }
   }
   if (warp >= B_EW / 32) {  // the TMA and MMA warps join the two cluster barriers too
     __syncwarp();
@@ -984,7 +977,7 @@ int launch_fwd_tc(const AttnTcParams& p, int batch, int seq, int nq, cudaStream_
     NF4_CUDA_TRY(cudaFuncSetAttribute(k_attn_fwd_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_TC));
     configured[dev] = 1;
   }
-  k_attn_fwd_tc<D><<<dim3(seq / TT, nq, batch), F_THREADS, SMEM_TC, s>>>(p);
+  k_attn_fwd_tc<D><<<dim3(nq, batch, seq / TT), F_THREADS, SMEM_TC, s>>>(p);
   note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;
@@ -1027,7 +1020,7 @@ int launch_bwd_tc(const AttnBwdParams& p, int batch, int seq, int nq, int nkv, c
     configured[dev] = 1;
   }
   // the query side writes delta, which the key side reads
-  k_attn_dq_tc<D><<<dim3(seq / TT, nq, batch), B_THREADS, SMEM_BWD, s>>>(p);
+  k_attn_dq_tc<D><<<dim3(nq, batch, seq / TT), B_THREADS, SMEM_BWD, s>>>(p);
   note_launch();
   k_attn_dkv_tc<D><<<dim3(2 * nkv, batch, seq / TT), B_THREADS, SMEM_BWD, s>>>(p);
   note_launch();
