@@ -375,14 +375,6 @@ __global__ void __launch_bounds__(F_THREADS, 2) k_attn_fwd_tc(const __grid_const
 // it.  Accumulation runs in a fixed order (query side: key tiles in order; key side:
 // query heads of the group, then query tiles), so results are bit-reproducible.
 
-// 1D bulk copy global -> shared completing transaction bytes on bar (16-byte multiples).
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   smem_u32(dst)),
-               "l"(src), "r"(bytes), "r"(smem_u32(bar))
-               : "memory");
-}
-
 struct AttnBwdParams {
   CUtensorMap tq, tk, tv, tdo, to;  // box 64 cols x 128 rows, 128-byte swizzle (to: the output O)
   CUtensorMap tdq, tdk, tdv;        // the gradients, same boxes (TMA stores)

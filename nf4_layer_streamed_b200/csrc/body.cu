@@ -60,12 +60,13 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   return a;
 }
 
-// The adapter operands in 16-byte pieces (8 bf16 outputs each), 32-bit indices:
+// The adapter's B operands in 16-byte pieces (8 bf16 outputs each), 32-bit indices:
 //   bup [qd + 2 kvd, 64]: s B_q in columns 0-15 of the q rows, s B_v in 16-31 of the v rows
-//   adn [64, H]:          A_q in rows 0-15, A_v in 16-31, zero rows 32-63
 //   bqt [16, qd], bvt [16, kvd]: B_q^T, B_v^T
+// (the A operand, adn [64, H] = A_q in rows 0-15, A_v in 16-31, zero rows 32-63, is
+// written by k_rmsnorm_down from its shared-memory copy of the adapter).
 __device__ void pack_piece(const LoraPack& a, int i) {
-  const int H = a.H, qd = a.qd, kvd = a.kvd, nq = qd + 2 * kvd;
+  const int qd = a.qd, kvd = a.kvd, nq = qd + 2 * kvd;
   float f[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) f[e] = 0.f;
@@ -81,14 +82,7 @@ __device__ void pack_piece(const LoraPack& a, int i) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) f[e] = a.scale * __bfloat162float(__float2bfloat16_rn(src[e]));
     dst = a.bup + (size_t)n * 64 + c;
-  } else if ((i -= nq * 8) < 8 * H) {
-    const int per = H / 8, r = i / per, k = (i - r * per) * 8;
-    const float* src = r < 16 ? a.Aq + (size_t)r * H + k : r < 32 ? a.Av + (size_t)(r - 16) * H + k : nullptr;
-    if (src)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) f[e] = src[e];
-    dst = a.adn + (size_t)r * H + k;
-  } else if ((i -= 8 * H) < 2 * qd) {
+  } else if ((i -= nq * 8) < 2 * qd) {
     const int per = qd / 8, r = i / per, n = (i - r * per) * 8;
 #pragma unroll
     for (int e = 0; e < 8; ++e) f[e] = a.Bq[(size_t)(n + e) * 16 + r];
@@ -103,24 +97,15 @@ __device__ void pack_piece(const LoraPack& a, int i) {
   *reinterpret_cast<uint4*>(dst) = pack8(f);
 }
 
-__host__ __device__ inline int pack_pieces(const LoraPack& a) {
-  return (a.qd + 2 * a.kvd) * 8 + 8 * a.H + 2 * a.qd + 2 * a.kvd;
-}
+__host__ __device__ inline int pack_pieces(const LoraPack& a) { return (a.qd + 2 * a.kvd) * 8 + 2 * a.qd + 2 * a.kvd; }
 
-// Blocks [0, n_pack): the adapter operand conversion, grid-stride (first, so that it
-// runs beside the rows rather than after them); the blocks after: one row each.
+// One block per row.
 template <int VPT>
 __global__ void __launch_bounds__(1024) k_rmsnorm_fwd_row(const __nv_bfloat16* __restrict__ x,
                                                           const __nv_bfloat16* __restrict__ w,
-                                                          __nv_bfloat16* __restrict__ y, int M, int H, float eps,
-                                                          const LoraPack pack, int n_pack) {
+                                                          __nv_bfloat16* __restrict__ y, int H, float eps) {
   __shared__ float red[32];
-  if ((int)blockIdx.x < n_pack) {
-    const int n = pack_pieces(pack), stride = n_pack * blockDim.x;
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) pack_piece(pack, i);
-    return;
-  }
-  const int row = blockIdx.x - n_pack, t = threadIdx.x, T = blockDim.x, nv = H / 8;
+  const int row = blockIdx.x, t = threadIdx.x, T = blockDim.x, nv = H / 8;
   const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)row * H);
   const uint4* wr = reinterpret_cast<const uint4*>(w);
   uint4* yr = reinterpret_cast<uint4*>(y + (size_t)row * H);
@@ -159,13 +144,14 @@ __global__ void __launch_bounds__(1024) k_rmsnorm_fwd_row(const __nv_bfloat16* _
 // so that h1 is not read back for t.  A cluster of C CTAs takes 64 rows; CTA c of the
 // cluster holds the column slice [c S, (c + 1) S) of those rows (S = H / C) in registers
 // (a warp per eight rows, 512 contiguous bytes per load) and the same slice of the 32
-// adapter rows, rounded to bf16, in
-// shared memory.  The rows' sums of squares are partial per CTA and added in CTA order
-// through distributed shared memory; each CTA then writes its slice of h1 and forms the
-// partial t of its slice on mma.sync m16n8k16 (warp w: row tile w % 4, k-steps
-// w / 4, w / 4 + 2, ..); the warp partials are added in k order, and the cluster's C
-// partials in CTA order, CTA c writing rows 64 c / C ...  The same launch converts the
-// adapter to its bf16 operands (every thread a share of pack_piece).
+// adapter rows, rounded to bf16, in shared memory.  The fp32 adapter slice arrives by 32
+// bulk copies into the h1 buffer (free until h1 is written) while the rows load; the
+// launch's share of the adapter's bf16 operands (every thread some pack_piece) runs
+// beside the same loads.  The rows' sums of squares are partial per CTA and added in
+// CTA order through distributed shared memory; each CTA then writes its slice of h1 and
+// forms the partial t of its slice on mma.sync m16n8k16 (warp w: row tile w % 4,
+// k-steps w / 4, w / 4 + 2, ..); the warp partials are added in k order, and the
+// cluster's C partials in CTA order, CTA c writing rows 64 c / C ...
 constexpr int ND_R = 64, ND_THREADS = 256;  // rows per cluster, threads per CTA (eight rows per warp)
 
 struct NormDownShape {
@@ -182,7 +168,8 @@ inline NormDownShape norm_down_shape(int H) {
     }
   if (sh.C) {
     const size_t hs = (size_t)ND_R * (sh.S + 8) * 2, as = (size_t)32 * (sh.S + 8) * 2;
-    sh.smem = hs + std::max(as, (size_t)ND_THREADS / 32 * 16 * 32 * 4) + (size_t)ND_R * 32 * 4 + ND_R * 4;
+    // + the mbarrier of the adapter copies and the abort flag of its wait
+    sh.smem = hs + std::max(as, (size_t)ND_THREADS / 32 * 16 * 32 * 4) + (size_t)ND_R * 32 * 4 + ND_R * 4 + 16;
   }
   return sh;
 }
@@ -192,16 +179,32 @@ __global__ void __launch_bounds__(ND_THREADS, 2) k_rmsnorm_down(const __nv_bfloa
                                                              const __nv_bfloat16* __restrict__ w,
                                                              __nv_bfloat16* __restrict__ y, int M, int H, int S,
                                                              float eps, const LoraPack pack,
-                                                             __nv_bfloat16* __restrict__ tpad) {
+                                                             __nv_bfloat16* __restrict__ tpad, int* err) {
   extern __shared__ __align__(16) uint8_t smem[];
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31, ls = S + 8, nv = S / 8;
   const int C = (int)(gridDim.y), c = (int)cluster_ctarank(), m0 = blockIdx.x * ND_R, col0 = c * S;
   __nv_bfloat16* hs = reinterpret_cast<__nv_bfloat16*>(smem);                 // [64][S + 8] h1 slice
+  float* stage = reinterpret_cast<float*>(smem);                              // before h1: [32][S] fp32 adapter slice
   __nv_bfloat16* as = hs + (size_t)ND_R * ls;                                  // [32][S + 8] adapter slice
   float* red = reinterpret_cast<float*>(as);                                   // after the products: [8][16][32]
   const size_t as_bytes = std::max((size_t)32 * ls * 2, (size_t)ND_THREADS / 32 * 16 * 32 * 4);
   float* P = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(as) + as_bytes);  // [64][32] this slice's t
   float* ssp = P + ND_R * 32;                                                  // [64] partial sums of squares
+  uint64_t* abar = reinterpret_cast<uint64_t*>(ssp + ND_R);                    // the adapter slice has landed
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(abar + 1);
+  if (t == 0) {
+    mbar_init(abar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (warp == 0) {  // lane r: adapter row r (0-15 A_q, 16-31 A_v), S floats, 16-byte aligned (S % 16 == 0)
+    if (lane == 0) mbar_arrive_expect_tx(abar, 32u * (uint32_t)S * 4u);
+    __syncwarp();
+    bulk_load(stage + (size_t)lane * S,
+              (lane < 16 ? pack.Aq + (size_t)lane * H : pack.Av + (size_t)(lane - 16) * H) + col0, (uint32_t)S * 4u,
+              abar);
+  }
   // warp w holds rows 8 w .. 8 w + 7 of the block; lane l the 16-byte vectors 32 h + l of
   // each row slice (h < NH): one warp instruction reads 512 contiguous bytes of a row
   uint4 v[8][NH];
@@ -213,31 +216,15 @@ __global__ void __launch_bounds__(ND_THREADS, 2) k_rmsnorm_down(const __nv_bfloa
     for (int hh = 0; hh < NH; ++hh)
       if (m < M && hh * 32 + lane < nv) v[rr][hh] = xr[hh * 32 + lane];
   }
-  // the adapter slice: rows 0-15 A_q, 16-31 A_v, bf16 (the values of the packed adn);
-  // eight 16-byte loads in flight per thread
+  const uint4* wr = reinterpret_cast<const uint4*>(w + col0);
+  uint4 wv[NH];
+#pragma unroll
+  for (int hh = 0; hh < NH; ++hh)
+    if (hh * 32 + lane < nv) wv[hh] = wr[hh * 32 + lane];
+  // the adapter's B operands, a share per thread of the whole grid, while the rows load
   {
-    const int n4 = 32 * (S / 4);
-    for (int i0 = 0; i0 < n4; i0 += 8 * ND_THREADS) {
-      float4 f[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i = i0 + u * ND_THREADS + t;
-        if (i < n4) {
-          const int r = i / (S / 4), k = (i - r * (S / 4)) * 4;
-          f[u] = __ldg(reinterpret_cast<const float4*>(
-              (r < 16 ? pack.Aq + (size_t)r * H : pack.Av + (size_t)(r - 16) * H) + col0 + k));
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i = i0 + u * ND_THREADS + t;
-        if (i < n4) {
-          const int r = i / (S / 4), k = (i - r * (S / 4)) * 4;
-          *reinterpret_cast<uint2*>(as + r * ls + k) =
-              make_uint2(pack_bf16x2(f[u].x, f[u].y), pack_bf16x2(f[u].z, f[u].w));
-        }
-      }
-    }
+    const int n = pack_pieces(pack), stride = gridDim.x * gridDim.y * ND_THREADS;
+    for (int i = (blockIdx.y * gridDim.x + blockIdx.x) * ND_THREADS + t; i < n; i += stride) pack_piece(pack, i);
   }
 #pragma unroll
   for (int rr = 0; rr < 8; ++rr) {
@@ -254,17 +241,47 @@ __global__ void __launch_bounds__(ND_THREADS, 2) k_rmsnorm_down(const __nv_bfloa
     ss = warp_sum(ss);
     if (lane == 0) ssp[warp * 8 + rr] = ss;
   }
-  cluster_sync_all();  // every slice's partial sums are in its CTA's shared memory
-  const uint4* wr = reinterpret_cast<const uint4*>(w + col0);
-  uint4 wv[NH];
+  // the adapter slice to bf16 (the values of the packed adn), next to the h1 buffer.  A
+  // wait that runs out records the site and leaves through the same barriers.
+  (void)mbar_wait(abar, 0, abort_flag, err, KID_NORM, 1);
+  {
+    const int n4 = 32 * (S / 4);
+    for (int i = t; i < n4; i += ND_THREADS) {
+      const int r = i / (S / 4), k = (i - r * (S / 4)) * 4;
+      const float4 f = *reinterpret_cast<const float4*>(stage + (size_t)r * S + k);
+      *reinterpret_cast<uint2*>(as + r * ls + k) = make_uint2(pack_bf16x2(f.x, f.y), pack_bf16x2(f.z, f.w));
+    }
+  }
+  if (blockIdx.x == 0) {  // the first cluster writes the adapter's A operand adn: its slice of rows 0-31, zero rows 32-63
+    __syncthreads();
+    for (int i = t; i < ND_R * nv; i += ND_THREADS) {
+      const int r = i / nv, k = (i - r * nv) * 8;
+      *reinterpret_cast<uint4*>(pack.adn + (size_t)r * H + col0 + k) =
+          r < 32 ? *reinterpret_cast<const uint4*>(as + r * ls + k) : make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+  // every slice's partial sums are in its CTA's shared memory, and this CTA is done with
+  // the staged adapter slice
+  cluster_sync_all();
+  // the warp's eight row totals, each the sum of the C partials in CTA order: lane l fetches
+  // row l % 8's partials of CTAs l / 8 and l / 8 + 4 (all in flight at once) and gathers
+  // its row's eight by shuffles
+  float tot8 = 0.f;
+  {
+    const int rq = lane & 7, q0 = lane >> 3;
+    const uint32_t a = smem_u32(ssp + warp * 8 + rq);
+    const float p0 = q0 < C ? ld_cluster_f32(mapa_shared(a, (uint32_t)q0)) : 0.f;
+    const float p1 = q0 + 4 < C ? ld_cluster_f32(mapa_shared(a, (uint32_t)(q0 + 4))) : 0.f;
 #pragma unroll
-  for (int hh = 0; hh < NH; ++hh)
-    if (hh * 32 + lane < nv) wv[hh] = wr[hh * 32 + lane];
+    for (int q = 0; q < 8; ++q) {
+      const float pq = __shfl_sync(0xffffffffu, q < 4 ? p0 : p1, (q & 3) * 8 + rq);
+      if (q < C) tot8 += pq;
+    }
+  }
 #pragma unroll
   for (int rr = 0; rr < 8; ++rr) {
     const int row = warp * 8 + rr, m = m0 + row;
-    float tot = 0.f;
-    for (int q = 0; q < C; ++q) tot += ld_cluster_f32(mapa_shared(smem_u32(ssp + row), (uint32_t)q));
+    const float tot = __shfl_sync(0xffffffffu, tot8, rr);
     const float r = 1.0f / sqrtf(tot / (float)H + eps);
     uint4* yr = reinterpret_cast<uint4*>(y + (size_t)m * H + col0);
     uint4* hrow = reinterpret_cast<uint4*>(hs + row * ls);
@@ -292,6 +309,7 @@ __global__ void __launch_bounds__(ND_THREADS, 2) k_rmsnorm_down(const __nv_bfloa
   float acc[4][4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+#pragma unroll 4
   for (int ks = kq; ks < S / 16; ks += 2) {
     uint32_t a0, a1, a2, a3, b0, b1, b2, b3, b4, b5, b6, b7;
     ldsm4(smem_u32(hs + (mt * 16 + (lane & 15)) * ls + ks * 16 + (lane >> 4) * 8), a0, a1, a2, a3);
@@ -325,15 +343,14 @@ __global__ void __launch_bounds__(ND_THREADS, 2) k_rmsnorm_down(const __nv_bfloa
   for (int e = t; e < rows_per * 64; e += ND_THREADS) {
     const int rr = c * rows_per + (e >> 6), cc = e & 63, mm = m0 + rr;
     if (mm >= M) continue;
-    float v2 = 0.f;
-    if (cc < 32)
-      for (int q = 0; q < C; ++q) v2 += ld_cluster_f32(mapa_shared(smem_u32(P + rr * 32 + cc), (uint32_t)q));
+    float part[8], v2 = 0.f;  // the C partials fetched together, then added in CTA order
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      part[q] = cc < 32 && q < C ? ld_cluster_f32(mapa_shared(smem_u32(P + rr * 32 + cc), (uint32_t)q)) : 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      if (q < C) v2 += part[q];
     tpad[(size_t)mm * 64 + cc] = __float2bfloat16_rn(v2);
-  }
-  // the adapter's bf16 operands, a share per thread of the whole grid
-  {
-    const int n = pack_pieces(pack), stride = gridDim.x * gridDim.y * ND_THREADS;
-    for (int i = (blockIdx.y * gridDim.x + blockIdx.x) * ND_THREADS + t; i < n; i += stride) pack_piece(pack, i);
   }
   cluster_sync_all();  // no CTA leaves while another still reads its shared memory
 }
@@ -745,22 +762,15 @@ inline unsigned blocks_for(size_t n, int threads) { return (unsigned)((n + threa
 // One block per row, the row in registers: 2 vectors (16 values) per thread up to
 // H = 16384 (256 threads at H = 4096, 64 at SmolLM2's 576), 4 up to H = 32768.
 int rmsnorm_fwd(const __nv_bfloat16* x, const __nv_bfloat16* w, __nv_bfloat16* y, int M, int H, float eps,
-                cudaStream_t s, const LoraPack* pack) {
+                cudaStream_t s) {
   if (H % 8 || H > 32768) return fail(NF4LS_SHAPE, "rmsnorm: H %% 8, H <= 32768");
   if (M <= 0) return NF4LS_OK;
-  LoraPack pk{};
   const int vpt = H <= 16384 ? 2 : 4;
   const int threads = row_threads(H, vpt);
-  int n_pack = 0;
-  if (pack) {  // about four 16-byte pieces per thread of the extra blocks
-    pk = *pack;
-    if (pk.qd % 8 || pk.kvd % 8) return fail(NF4LS_SHAPE, "rmsnorm: adapter widths %% 8");
-    n_pack = std::min(1024, (pack_pieces(pk) + 4 * threads - 1) / (4 * threads));
-  }
   if (vpt == 2)
-    k_rmsnorm_fwd_row<2><<<M + n_pack, threads, 0, s>>>(x, w, y, M, H, eps, pk, n_pack);
+    k_rmsnorm_fwd_row<2><<<M, threads, 0, s>>>(x, w, y, H, eps);
   else
-    k_rmsnorm_fwd_row<4><<<M + n_pack, threads, 0, s>>>(x, w, y, M, H, eps, pk, n_pack);
+    k_rmsnorm_fwd_row<4><<<M, threads, 0, s>>>(x, w, y, H, eps);
   note_launch();
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;
@@ -796,7 +806,7 @@ int rmsnorm_lora_fwd(const __nv_bfloat16* x, const __nv_bfloat16* w, __nv_bfloat
       NF4_CUDA_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sh.smem));
       configured[dev][slot] = (int)sh.smem;
     }
-    NF4_CUDA_TRY(cudaLaunchKernelEx(&cfg, kernel, x, w, y, M, H, sh.S, eps, pack, tpad));
+    NF4_CUDA_TRY(cudaLaunchKernelEx(&cfg, kernel, x, w, y, M, H, sh.S, eps, pack, tpad, device_error_ptr()));
     return NF4LS_OK;
   };
   int st;

@@ -16,7 +16,7 @@ namespace nf4ls {
 // wait expired), [1] = kernel id, [2] = block, [3] = site.  The record lives in a
 // file-scope __device__ array of device.cu; its address is looked up per device.
 
-enum KernelId : int { KID_GEMM = 1, KID_ATTN = 2, KID_WAIT_PROBE = 3 };
+enum KernelId : int { KID_GEMM = 1, KID_ATTN = 2, KID_WAIT_PROBE = 3, KID_NORM = 4 };
 
 // A bounded wait gives up after this many nanoseconds of global time.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
@@ -128,6 +128,15 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       "[%2];" ::"r"(smem_u32(dst)),
       "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
       : "memory");
+}
+
+// 1D bulk copy global -> this CTA's shared memory, completing transaction bytes on bar
+// (addresses 16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
 }
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {

@@ -241,9 +241,9 @@ struct LoraPack {
   __nv_bfloat16* bqt;
   __nv_bfloat16* bvt;
 };
-// y = rmsnorm(x) w; with pack, the same launch also fills the adapter operands.
+// y = rmsnorm(x) w.
 int rmsnorm_fwd(const __nv_bfloat16* x, const __nv_bfloat16* w, __nv_bfloat16* y, int M, int H, float eps,
-                cudaStream_t s, const LoraPack* pack = nullptr);
+                cudaStream_t s);
 // y = rmsnorm(x) w (the input norm) with the adapter operands filled and
 // t = [y A_q^T | y A_v^T] written to columns 0-31 of tpad [M, 64] (32-63 zero).
 int rmsnorm_lora_fwd(const __nv_bfloat16* x, const __nv_bfloat16* w, __nv_bfloat16* y, int M, int H, float eps,

@@ -318,8 +318,11 @@ __global__ void __cluster_dims__(1, DA_SPLIT, 1) __launch_bounds__(DA_THREADS)
   for (int e = t; e < ROWS_PER_CTA * DA_COLS; e += DA_THREADS) {
     const int row = y * ROWS_PER_CTA + e / DA_COLS, col = e % DA_COLS;
     const uint32_t local = smem_u32(P + row * DA_COLS + col);
-    float v = 0.f;
-    for (int c = 0; c < DA_SPLIT; ++c) v += ld_cluster_f32(mapa_shared(local, (uint32_t)c));
+    float part[DA_SPLIT], v = 0.f;  // the partials fetched together, then added in CTA order
+#pragma unroll
+    for (int c = 0; c < DA_SPLIT; ++c) part[c] = ld_cluster_f32(mapa_shared(local, (uint32_t)c));
+#pragma unroll
+    for (int c = 0; c < DA_SPLIT; ++c) v += part[c];
     if (row < 16)
       a.dA_q[(size_t)row * a.H + c0 + col] = v;
     else
