@@ -147,11 +147,14 @@ __global__ void __launch_bounds__(1024) k_rmsnorm_fwd_row(const __nv_bfloat16* _
 // adapter rows, rounded to bf16, in shared memory.  The fp32 adapter slice arrives by 32
 // bulk copies into the h1 buffer (free until h1 is written) while the rows load; the
 // launch's share of the adapter's bf16 operands (every thread some pack_piece) runs
-// beside the same loads.  The rows' sums of squares are partial per CTA and added in
-// CTA order through distributed shared memory; each CTA then writes its slice of h1 and
-// forms the partial t of its slice on mma.sync m16n8k16 (warp w: row tile w % 4,
-// k-steps w / 4, w / 4 + 2, ..); the warp partials are added in k order, and the
-// cluster's C partials in CTA order, CTA c writing rows 64 c / C ...
+// beside the same loads.  The rows' sums of squares are partial per CTA; every CTA
+// stores its partials into every CTA's shared memory (distributed shared memory) and
+// adds the C partials of each row in CTA order.  Each CTA then writes its slice of h1
+// and forms the partial t of its slice on mma.sync m16n8k16 (warp w: row tile w % 4,
+// k-steps w / 4, w / 4 + 2, ..); the warp partials are added in k order and stored into
+// the CTA that owns the rows (CTA c: rows 64 c / C ...), which adds the cluster's C
+// partials in CTA order.  Only stores cross CTAs, each before a cluster barrier, so no
+// CTA waits for another at the end.
 constexpr int ND_R = 64, ND_THREADS = 256;  // rows per cluster, threads per CTA (eight rows per warp)
 
 struct NormDownShape {
@@ -168,8 +171,9 @@ inline NormDownShape norm_down_shape(int H) {
     }
   if (sh.C) {
     const size_t hs = (size_t)ND_R * (sh.S + 8) * 2, as = (size_t)32 * (sh.S + 8) * 2;
-    // + the mbarrier of the adapter copies and the abort flag of its wait
-    sh.smem = hs + std::max(as, (size_t)ND_THREADS / 32 * 16 * 32 * 4) + (size_t)ND_R * 32 * 4 + ND_R * 4 + 16;
+    // + every CTA's partial sums of squares [8][64], the mbarrier of the adapter copies and
+    // the abort flag of its wait
+    sh.smem = hs + std::max(as, (size_t)ND_THREADS / 32 * 16 * 32 * 4) + (size_t)ND_R * 32 * 4 + 8 * ND_R * 4 + 16;
   }
   return sh;
 }
@@ -188,15 +192,16 @@ __global__ void __launch_bounds__(ND_THREADS, 2) k_rmsnorm_down(const __nv_bfloa
   __nv_bfloat16* as = hs + (size_t)ND_R * ls;                                  // [32][S + 8] adapter slice
   float* red = reinterpret_cast<float*>(as);                                   // after the products: [8][16][32]
   const size_t as_bytes = std::max((size_t)32 * ls * 2, (size_t)ND_THREADS / 32 * 16 * 32 * 4);
-  float* P = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(as) + as_bytes);  // [64][32] this slice's t
-  float* ssp = P + ND_R * 32;                                                  // [64] partial sums of squares
-  uint64_t* abar = reinterpret_cast<uint64_t*>(ssp + ND_R);                    // the adapter slice has landed
+  float* Pin = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(as) + as_bytes);  // [C][64 / C][32] t partials
+  float* ssall = Pin + ND_R * 32;                                              // [C][64] partial sums of squares
+  uint64_t* abar = reinterpret_cast<uint64_t*>(ssall + 8 * ND_R);              // the adapter slice has landed
   volatile int* abort_flag = reinterpret_cast<volatile int*>(abar + 1);
   if (t == 0) {
     mbar_init(abar, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
+  cluster_arrive_relaxed();  // this CTA has started: the others may store into its shared memory
   __syncthreads();
   if (warp == 0) {  // lane r: adapter row r (0-15 A_q, 16-31 A_v), S floats, 16-byte aligned (S % 16 == 0)
     if (lane == 0) mbar_arrive_expect_tx(abar, 32u * (uint32_t)S * 4u);
@@ -226,6 +231,7 @@ __global__ void __launch_bounds__(ND_THREADS, 2) k_rmsnorm_down(const __nv_bfloa
     const int n = pack_pieces(pack), stride = gridDim.x * gridDim.y * ND_THREADS;
     for (int i = (blockIdx.y * gridDim.x + blockIdx.x) * ND_THREADS + t; i < n; i += stride) pack_piece(pack, i);
   }
+  float mine = 0.f;  // lane l: the partial of the warp's row l % 8
 #pragma unroll
   for (int rr = 0; rr < 8; ++rr) {
     const int m = m0 + warp * 8 + rr;
@@ -239,7 +245,14 @@ __global__ void __launch_bounds__(ND_THREADS, 2) k_rmsnorm_down(const __nv_bfloa
         for (int e = 0; e < 8; ++e) ss += f[e] * f[e];
       }
     ss = warp_sum(ss);
-    if (lane == 0) ssp[warp * 8 + rr] = ss;
+    if ((lane & 7) == rr) mine = ss;
+  }
+  cluster_wait();  // every CTA of the cluster has started
+  {  // into slot c of every CTA: lane l to CTAs l / 8 and l / 8 + 4
+    const uint32_t a = smem_u32(ssall + c * ND_R + warp * 8 + (lane & 7));
+    const int q0 = lane >> 3;
+    if (q0 < C) st_cluster_f32(mapa_shared(a, (uint32_t)q0), mine);
+    if (q0 + 4 < C) st_cluster_f32(mapa_shared(a, (uint32_t)(q0 + 4)), mine);
   }
   // the adapter slice to bf16 (the values of the packed adn), next to the h1 buffer.  A
   // wait that runs out records the site and leaves through the same barriers.
@@ -260,24 +273,14 @@ __global__ void __launch_bounds__(ND_THREADS, 2) k_rmsnorm_down(const __nv_bfloa
           r < 32 ? *reinterpret_cast<const uint4*>(as + r * ls + k) : make_uint4(0u, 0u, 0u, 0u);
     }
   }
-  // every slice's partial sums are in its CTA's shared memory, and this CTA is done with
+  // every CTA's partial sums are in every CTA's shared memory, and this CTA is done with
   // the staged adapter slice
   cluster_sync_all();
-  // the warp's eight row totals, each the sum of the C partials in CTA order: lane l fetches
-  // row l % 8's partials of CTAs l / 8 and l / 8 + 4 (all in flight at once) and gathers
-  // its row's eight by shuffles
+  // lane l: the total of the warp's row l % 8, the C partials added in CTA order
   float tot8 = 0.f;
-  {
-    const int rq = lane & 7, q0 = lane >> 3;
-    const uint32_t a = smem_u32(ssp + warp * 8 + rq);
-    const float p0 = q0 < C ? ld_cluster_f32(mapa_shared(a, (uint32_t)q0)) : 0.f;
-    const float p1 = q0 + 4 < C ? ld_cluster_f32(mapa_shared(a, (uint32_t)(q0 + 4))) : 0.f;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const float pq = __shfl_sync(0xffffffffu, q < 4 ? p0 : p1, (q & 3) * 8 + rq);
-      if (q < C) tot8 += pq;
-    }
-  }
+  for (int q = 0; q < 8; ++q)
+    if (q < C) tot8 += ssall[q * ND_R + warp * 8 + (lane & 7)];
 #pragma unroll
   for (int rr = 0; rr < 8; ++rr) {
     const int row = warp * 8 + rr, m = m0 + row;
@@ -334,25 +337,23 @@ __global__ void __launch_bounds__(ND_THREADS, 2) k_rmsnorm_down(const __nv_bfloa
     }
   }
   __syncthreads();
-  for (int e = t; e < ND_R * 32; e += ND_THREADS) {  // the slice's t: the two k halves in order
-    const int rr = e >> 5, cc = e & 31, tile = rr >> 4, ri = rr & 15;
-    P[e] = red[tile * (16 * 32) + ri * 32 + cc] + red[(4 + tile) * (16 * 32) + ri * 32 + cc];
-  }
-  cluster_sync_all();  // every slice's t is in its CTA's shared memory
   const int rows_per = ND_R / C;
+  for (int e = t; e < ND_R * 32; e += ND_THREADS) {  // the slice's t (the two k halves in order) to slot c of its owner
+    const int rr = e >> 5, cc = e & 31, tile = rr >> 4, ri = rr & 15, q = rr / rows_per;
+    const float v2 = red[tile * (16 * 32) + ri * 32 + cc] + red[(4 + tile) * (16 * 32) + ri * 32 + cc];
+    st_cluster_f32(mapa_shared(smem_u32(Pin + (c * rows_per + rr - q * rows_per) * 32 + cc), (uint32_t)q), v2);
+  }
+  cluster_sync_all();  // every CTA's partial t of this CTA's rows is here
   for (int e = t; e < rows_per * 64; e += ND_THREADS) {
-    const int rr = c * rows_per + (e >> 6), cc = e & 63, mm = m0 + rr;
+    const int rl = e >> 6, cc = e & 63, mm = m0 + c * rows_per + rl;
     if (mm >= M) continue;
-    float part[8], v2 = 0.f;  // the C partials fetched together, then added in CTA order
+    float v2 = 0.f;  // the C partials in CTA order
+    if (cc < 32)
 #pragma unroll
-    for (int q = 0; q < 8; ++q)
-      part[q] = cc < 32 && q < C ? ld_cluster_f32(mapa_shared(smem_u32(P + rr * 32 + cc), (uint32_t)q)) : 0.f;
-#pragma unroll
-    for (int q = 0; q < 8; ++q)
-      if (q < C) v2 += part[q];
+      for (int q = 0; q < 8; ++q)
+        if (q < C) v2 += Pin[(q * rows_per + rl) * 32 + cc];
     tpad[(size_t)mm * 64 + cc] = __float2bfloat16_rn(v2);
   }
-  cluster_sync_all();  // no CTA leaves while another still reads its shared memory
 }
 
 template <int VPT>

@@ -284,11 +284,24 @@ __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// The two halves of cluster_sync_all, for work between them: arrive (relaxed, no memory
+// ordering) and wait.  A CTA's shared memory may take stores from the others once every
+// CTA of the cluster has arrived at least once.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+
 // shared::cluster address of the object at local address `a` in CTA `rank` of the cluster.
 __device__ __forceinline__ uint32_t mapa_shared(uint32_t a, uint32_t rank) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
   return r;
+}
+
+// st.shared::cluster of one float at a shared::cluster address (possibly another CTA's).
+__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
 
 // ld.shared::cluster of one float at a shared::cluster address (possibly another CTA's).
