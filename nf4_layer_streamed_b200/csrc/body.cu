@@ -145,16 +145,16 @@ __global__ void __launch_bounds__(1024) k_rmsnorm_fwd_row(const __nv_bfloat16* _
 // cluster holds the column slice [c S, (c + 1) S) of those rows (S = H / C) in registers
 // (a warp per eight rows, 512 contiguous bytes per load) and the same slice of the 32
 // adapter rows, rounded to bf16, in shared memory.  The fp32 adapter slice arrives by 32
-// bulk copies into the h1 buffer (free until h1 is written) while the rows load; the
-// launch's share of the adapter's bf16 operands (every thread some pack_piece) runs
-// beside the same loads.  The rows' sums of squares are partial per CTA; every CTA
-// stores its partials into every CTA's shared memory (distributed shared memory) and
-// adds the C partials of each row in CTA order.  Each CTA then writes its slice of h1
-// and forms the partial t of its slice on mma.sync m16n8k16 (warp w: row tile w % 4,
-// k-steps w / 4, w / 4 + 2, ..); the warp partials are added in k order and stored into
-// the CTA that owns the rows (CTA c: rows 64 c / C ...), which adds the cluster's C
-// partials in CTA order.  Only stores cross CTAs, each before a cluster barrier, so no
-// CTA waits for another at the end.
+// bulk copies into the h1 buffer (free until h1 is written) while the rows load.  The
+// rows' sums of squares are partial per CTA; every CTA stores its partials into every
+// CTA's shared memory (distributed shared memory) and adds the C partials of each row in
+// CTA order.  Between the two halves of that cluster barrier each CTA converts its
+// adapter slice and does its share of the adapter's B operands (pack_piece).  Each CTA
+// then writes its slice of h1 and forms the partial t of its slice on mma.sync m16n8k16
+// (warp w: row tile w % 4, k-steps w / 4, w / 4 + 2, ..); the warp partials are added in
+// k order and stored into the CTA that owns the rows (CTA c: rows 64 c / C ...), which
+// adds the cluster's C partials in CTA order.  Only stores cross CTAs, each before a
+// cluster barrier, so no CTA waits for another at the end.
 constexpr int ND_R = 64, ND_THREADS = 256;  // rows per cluster, threads per CTA (eight rows per warp)
 
 struct NormDownShape {
@@ -210,6 +210,13 @@ __global__ void __launch_bounds__(ND_THREADS, 2) k_rmsnorm_down(const __nv_bfloa
               (lane < 16 ? pack.Aq + (size_t)lane * H : pack.Av + (size_t)(lane - 16) * H) + col0, (uint32_t)S * 4u,
               abar);
   }
+  if (warp == 1 && lane < 2) {  // this CTA's share of B_q (lane 0) or B_v (lane 1) into L2 for pack_piece
+    const size_t bytes = (size_t)(lane ? pack.kvd : pack.qd) * 64, n_cta = (size_t)gridDim.x * gridDim.y;
+    const size_t chunk = (bytes / n_cta + 255) / 256 * 256, b0 = (size_t)(blockIdx.y * gridDim.x + blockIdx.x) * chunk;
+    if (b0 < bytes)
+      bulk_prefetch_l2(reinterpret_cast<const uint8_t*>(lane ? pack.Bv : pack.Bq) + b0,
+                       (uint32_t)std::min(chunk, bytes - b0));
+  }
   // warp w holds rows 8 w .. 8 w + 7 of the block; lane l the 16-byte vectors 32 h + l of
   // each row slice (h < NH): one warp instruction reads 512 contiguous bytes of a row
   uint4 v[8][NH];
@@ -226,11 +233,6 @@ __global__ void __launch_bounds__(ND_THREADS, 2) k_rmsnorm_down(const __nv_bfloa
 #pragma unroll
   for (int hh = 0; hh < NH; ++hh)
     if (hh * 32 + lane < nv) wv[hh] = wr[hh * 32 + lane];
-  // the adapter's B operands, a share per thread of the whole grid, while the rows load
-  {
-    const int n = pack_pieces(pack), stride = gridDim.x * gridDim.y * ND_THREADS;
-    for (int i = (blockIdx.y * gridDim.x + blockIdx.x) * ND_THREADS + t; i < n; i += stride) pack_piece(pack, i);
-  }
   float mine = 0.f;  // lane l: the partial of the warp's row l % 8
 #pragma unroll
   for (int rr = 0; rr < 8; ++rr) {
@@ -254,6 +256,12 @@ __global__ void __launch_bounds__(ND_THREADS, 2) k_rmsnorm_down(const __nv_bfloa
     if (q0 < C) st_cluster_f32(mapa_shared(a, (uint32_t)q0), mine);
     if (q0 + 4 < C) st_cluster_f32(mapa_shared(a, (uint32_t)(q0 + 4)), mine);
   }
+  cluster_arrive();  // this CTA's partial sums are out; the work below runs while the others finish theirs
+  // the adapter's B operands, a share per thread of the whole grid
+  {
+    const int n = pack_pieces(pack), stride = gridDim.x * gridDim.y * ND_THREADS;
+    for (int i = (blockIdx.y * gridDim.x + blockIdx.x) * ND_THREADS + t; i < n; i += stride) pack_piece(pack, i);
+  }
   // the adapter slice to bf16 (the values of the packed adn), next to the h1 buffer.  A
   // wait that runs out records the site and leaves through the same barriers.
   (void)mbar_wait(abar, 0, abort_flag, err, KID_NORM, 1);
@@ -273,9 +281,10 @@ __global__ void __launch_bounds__(ND_THREADS, 2) k_rmsnorm_down(const __nv_bfloa
           r < 32 ? *reinterpret_cast<const uint4*>(as + r * ls + k) : make_uint4(0u, 0u, 0u, 0u);
     }
   }
-  // every CTA's partial sums are in every CTA's shared memory, and this CTA is done with
-  // the staged adapter slice
-  cluster_sync_all();
+  // every thread of this CTA is done with the staged adapter slice before h1 overwrites
+  // it (the cluster barrier's arrivals came before the conversion, so it does not order it)
+  __syncthreads();
+  cluster_wait();  // every CTA's partial sums are in every CTA's shared memory
   // lane l: the total of the warp's row l % 8, the C partials added in CTA order
   float tot8 = 0.f;
 #pragma unroll
@@ -783,7 +792,8 @@ int rmsnorm_lora_fwd(const __nv_bfloat16* x, const __nv_bfloat16* w, __nv_bfloat
   const NormDownShape sh = norm_down_shape(H);
   if (!sh.C) return fail(NF4LS_SHAPE, "rmsnorm_lora_fwd: H %d (a multiple of 16 up to 8192)", H);
   if (pack.qd % 8 || pack.kvd % 8) return fail(NF4LS_SHAPE, "rmsnorm_lora_fwd: adapter widths %% 8");
-  if (!aligned(pack.Aq, 16) || !aligned(pack.Av, 16) || !aligned(x, 16) || !aligned(y, 16) || !aligned(w, 16))
+  if (!aligned(pack.Aq, 16) || !aligned(pack.Av, 16) || !aligned(pack.Bq, 16) || !aligned(pack.Bv, 16) ||
+      !aligned(x, 16) || !aligned(y, 16) || !aligned(w, 16))
     return fail(NF4LS_ALIGN, "rmsnorm_lora_fwd: 16-byte aligned operands");
   if (M <= 0) return NF4LS_OK;
   const int nh = (sh.S / 8 + 31) / 32;  // 512-byte pieces per row slice

@@ -139,6 +139,11 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                : "memory");
 }
 
+// Bulk prefetch of bytes (a multiple of 16, 16-byte aligned) from global memory into L2.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
@@ -284,13 +289,16 @@ __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// The two halves of cluster_sync_all, for work between them: arrive (relaxed, no memory
-// ordering) and wait.  A CTA's shared memory may take stores from the others once every
-// CTA of the cluster has arrived at least once.
+// The two halves of cluster_sync_all, for work between them: arrive (release, or relaxed
+// with no memory ordering) and wait (acquire).  A CTA's shared memory may take stores
+// from the others once every CTA of the cluster has arrived at least once.
 __device__ __forceinline__ void cluster_arrive_relaxed() {
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
-__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 
 // shared::cluster address of the object at local address `a` in CTA `rank` of the cluster.
 __device__ __forceinline__ uint32_t mapa_shared(uint32_t a, uint32_t rank) {

@@ -57,6 +57,61 @@ int* device_error_ptr() {
 
 namespace {
 
+// Per device: the side stream (least priority, non-blocking) and its two events, made
+// on first use and again when the device's context has changed.
+struct SideSlot {
+  std::mutex mu;
+  unsigned long long ctx = 0;
+  cudaStream_t side = nullptr;
+  cudaEvent_t ready = nullptr, done = nullptr;
+};
+SideSlot g_side[64];
+
+}  // namespace
+
+SideStream::SideStream() = default;
+
+SideStream::~SideStream() {
+  if (forked_) g_side[dev_].mu.unlock();
+}
+
+int SideStream::fork(cudaStream_t s) {
+  if (forked_) return fail(NF4LS_INVALID_ARG, "side stream: forked twice");
+  int dev = 0;
+  NF4_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(NF4LS_CUDA, "side stream: device %d", dev);
+  SideSlot& sl = g_side[dev];
+  sl.mu.lock();
+  dev_ = dev;
+  forked_ = true;
+  const unsigned long long id = current_context_id();
+  if (!sl.side || id == 0 || id != sl.ctx) {  // handles of an earlier context are gone with it
+    int least = 0, greatest = 0;
+    NF4_CUDA_TRY(cudaDeviceGetStreamPriorityRange(&least, &greatest));
+    NF4_CUDA_TRY(cudaStreamCreateWithPriority(&sl.side, cudaStreamNonBlocking, least));
+    NF4_CUDA_TRY(cudaEventCreateWithFlags(&sl.ready, cudaEventDisableTiming));
+    NF4_CUDA_TRY(cudaEventCreateWithFlags(&sl.done, cudaEventDisableTiming));
+    sl.ctx = id;
+  }
+  side_ = sl.side;
+  ready_ = sl.ready;
+  done_ = sl.done;
+  NF4_CUDA_TRY(cudaEventRecord(ready_, s));
+  NF4_CUDA_TRY(cudaStreamWaitEvent(side_, ready_, 0));
+  return NF4LS_OK;
+}
+
+int SideStream::join(cudaStream_t s) {
+  if (!forked_) return NF4LS_OK;
+  NF4_CUDA_TRY(cudaEventRecord(done_, side_));
+  NF4_CUDA_TRY(cudaStreamWaitEvent(s, done_, 0));
+  forked_ = false;
+  g_side[dev_].mu.unlock();
+  return NF4LS_OK;
+}
+
+namespace {
+
 // The expiry path of the bounded mbarrier wait, on its own: one block of two warps
 // waits on an mbarrier that no thread ever arrives on.  Warp 0 waits limit_ns and
 // gives up (site 1), which records the error and raises the block's abort flag;

@@ -278,13 +278,35 @@ int attention_bwd(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfl
                   int seq, int nq, int nkv, int d, cudaStream_t s);
 
 // LoRA backward (lora.cu); the forward's t comes from rmsnorm_lora_fwd (body.cu).
-// Backward, three launches: dB_q, dB_v, dA_q, dA_v (fp32, written) and dt into dtpad
-// [M, 64] (bf16, zeros in columns 32-63) from dq (columns [0, qd) of dqkv) and dv
-// (columns [vcol, vcol + kvd)); part: lora_partial_bytes of scratch.
+// dB_q, dB_v, dA_q, dA_v (fp32, written) and dt into dtpad [M, 64] (bf16, zeros in
+// columns 32-63) from dq (columns [0, qd) of dqkv) and dv (columns [vcol, vcol + kvd));
+// part: lora_partial_bytes of scratch.  phases: LORA_BWD_DT = the partial sums and dt
+// (two launches; the dL/dx GEMM needs dt), LORA_BWD_DB_DA = dB from the same partial
+// sums and dA = dt^T h1 (two launches; nothing in the layer's backward waits for them),
+// on stream s, the second after the first in stream order.
+constexpr int LORA_BWD_DT = 1, LORA_BWD_DB_DA = 2;
 size_t lora_partial_bytes(int M, int H, int qd, int kvd);
 int lora_bwd(const __nv_bfloat16* dqkv, int ld, int vcol, int M, int H, int qd, int kvd, const __nv_bfloat16* tpad,
              const __nv_bfloat16* bqt, const __nv_bfloat16* bvt, const __nv_bfloat16* h1, float scale,
-             __nv_bfloat16* dtpad, const nf4ls_lora_grads* g, void* part, cudaStream_t s);
+             __nv_bfloat16* dtpad, const nf4ls_lora_grads* g, void* part, int phases, cudaStream_t s);
+// A second stream on the current device for work that can run beside the caller's:
+// fork records an event on s, launches made on side() after it wait for it, and join
+// makes s wait for everything launched on side() since.  The fork-join sequence holds
+// a per-device lock (one sequence at a time per device and process).
+class SideStream {
+ public:
+  SideStream();
+  ~SideStream();
+  int fork(cudaStream_t s);
+  cudaStream_t side() const { return side_; }
+  int join(cudaStream_t s);
+
+ private:
+  int dev_ = -1;
+  bool forked_ = false;
+  cudaStream_t side_ = nullptr;
+  cudaEvent_t ready_ = nullptr, done_ = nullptr;
+};
 int embed(const int32_t* ids, const __nv_bfloat16* E, __nv_bfloat16* h, int M, int H, cudaStream_t s);
 // Streamed head, per vocab chunk [v0, v0 + n) of the output matrix (rows Wc in HBM):
 // logits [M, n] (bf16, from the GEMM) are folded into the per-row running max mx, sum

@@ -181,11 +181,14 @@ __global__ void __launch_bounds__(LB_THREADS) k_lora_bwd_partial(const __grid_co
 // Blocks [0, n_db_blocks): dB, one element per thread, the row-block partials added in
 // order.  The others: dt of 8 rows per block (one row per warp, column-chunk partials
 // added in order, times s, rounded to bf16) into dtpad, zeros in its columns 32-63.
-__global__ void __launch_bounds__(LB_THREADS) k_lora_bwd_reduce(const __grid_constant__ LoraBwdArgs a) {
-  const int t = threadIdx.x;
+// A launch runs blocks first_block, first_block + 1, .. (dt and dB go to different
+// streams).
+__global__ void __launch_bounds__(LB_THREADS) k_lora_bwd_reduce(const __grid_constant__ LoraBwdArgs a,
+                                                                int first_block) {
+  const int t = threadIdx.x, blk = first_block + (int)blockIdx.x;
   const int NB = a.qd + a.kvd;
-  if ((int)blockIdx.x < a.n_db_blocks) {
-    const int e = blockIdx.x * LB_THREADS + t;
+  if (blk < a.n_db_blocks) {
+    const int e = blk * LB_THREADS + t;
     if (e >= NB * 16) return;
     const int col = e >> 4, r = e & 15;
     float v = 0.f;
@@ -197,7 +200,7 @@ __global__ void __launch_bounds__(LB_THREADS) k_lora_bwd_reduce(const __grid_con
       a.dB_v[(size_t)(col - a.qd) * 16 + r] = v;
     return;
   }
-  const int m = ((int)blockIdx.x - a.n_db_blocks) * 8 + (t >> 5), c = t & 31;
+  const int m = (blk - a.n_db_blocks) * 8 + (t >> 5), c = t & 31;
   if (m >= a.M) return;
   const int cb = c < 16 ? 0 : a.n_cc_q, ce = c < 16 ? a.n_cc_q : a.n_cc;
   float v = 0.f;
@@ -390,7 +393,7 @@ size_t lora_partial_bytes(int M, int H, int qd, int kvd) { return bwd_shape(M, H
 
 int lora_bwd(const __nv_bfloat16* dqkv, int ld, int vcol, int M, int H, int qd, int kvd, const __nv_bfloat16* tpad,
              const __nv_bfloat16* bqt, const __nv_bfloat16* bvt, const __nv_bfloat16* h1, float scale,
-             __nv_bfloat16* dtpad, const nf4ls_lora_grads* g, void* part, cudaStream_t s) {
+             __nv_bfloat16* dtpad, const nf4ls_lora_grads* g, void* part, int phases, cudaStream_t s) {
   const BwdShape sh = bwd_shape(M, H, qd, kvd);
   if (!sh.CW || H % DA_COLS || ld % 8 || vcol % 8)
     return fail(NF4LS_SHAPE, "lora_bwd: qd %d, kvd %d, H %d", qd, kvd, H);
@@ -421,15 +424,21 @@ int lora_bwd(const __nv_bfloat16* dqkv, int ld, int vcol, int M, int H, int qd, 
   a.dB_q = g->dB_q;
   a.dA_v = g->dA_v;
   a.dB_v = g->dB_v;
-  const size_t smem1 = (size_t)LB_ROWS * (sh.CW + 8) * 2 + (size_t)LB_ROWS * 24 * 2 + 16ull * (sh.CW + 8) * 2;
-  NF4_TRY(allow_smem((const void*)k_lora_bwd_partial, smem1));
-  k_lora_bwd_partial<<<dim3(sh.n_rb, sh.n_cc), LB_THREADS, smem1, s>>>(a);
-  note_launch();
-  k_lora_bwd_reduce<<<sh.n_db_blocks + (M + 7) / 8, LB_THREADS, 0, s>>>(a);
-  note_launch();
-  NF4_TRY(allow_smem((const void*)k_lora_bwd_da, DA_SMEM));
-  k_lora_bwd_da<<<dim3(H / DA_COLS, DA_SPLIT), DA_THREADS, DA_SMEM, s>>>(a);
-  note_launch();
+  if (phases & LORA_BWD_DT) {
+    const size_t smem1 = (size_t)LB_ROWS * (sh.CW + 8) * 2 + (size_t)LB_ROWS * 24 * 2 + 16ull * (sh.CW + 8) * 2;
+    NF4_TRY(allow_smem((const void*)k_lora_bwd_partial, smem1));
+    k_lora_bwd_partial<<<dim3(sh.n_rb, sh.n_cc), LB_THREADS, smem1, s>>>(a);
+    note_launch();
+    k_lora_bwd_reduce<<<(M + 7) / 8, LB_THREADS, 0, s>>>(a, sh.n_db_blocks);
+    note_launch();
+  }
+  if (phases & LORA_BWD_DB_DA) {
+    k_lora_bwd_reduce<<<sh.n_db_blocks, LB_THREADS, 0, s>>>(a, 0);
+    note_launch();
+    NF4_TRY(allow_smem((const void*)k_lora_bwd_da, DA_SMEM));
+    k_lora_bwd_da<<<dim3(H / DA_COLS, DA_SPLIT), DA_THREADS, DA_SMEM, s>>>(a);
+    note_launch();
+  }
   NF4_CUDA_TRY(cudaGetLastError());
   return NF4LS_OK;
 }
