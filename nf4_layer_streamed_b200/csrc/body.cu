@@ -265,12 +265,16 @@ __global__ void __launch_bounds__(ND_THREADS, 2) k_rmsnorm_down(const __nv_bfloa
   // the adapter slice to bf16 (the values of the packed adn), next to the h1 buffer.  A
   // wait that runs out records the site and leaves through the same barriers.
   (void)mbar_wait(abar, 0, abort_flag, err, KID_NORM, 1);
-  {
-    const int n4 = 32 * (S / 4);
-    for (int i = t; i < n4; i += ND_THREADS) {
-      const int r = i / (S / 4), k = (i - r * (S / 4)) * 4;
-      const float4 f = *reinterpret_cast<const float4*>(stage + (size_t)r * S + k);
-      *reinterpret_cast<uint2*>(as + r * ls + k) = make_uint2(pack_bf16x2(f.x, f.y), pack_bf16x2(f.z, f.w));
+  {  // thread t: 4-float pieces t, t + 256, ..: (row r, piece k) stepped without a division per piece
+    const int q4 = S / 4, dr = ND_THREADS / q4, dk = ND_THREADS - dr * q4;
+    int r = t / q4, k = t - r * q4;
+    for (; r < 32; r += dr, k += dk) {
+      if (k >= q4) {
+        k -= q4;
+        if (++r >= 32) break;
+      }
+      const float4 f = *reinterpret_cast<const float4*>(stage + (size_t)r * S + 4 * k);
+      *reinterpret_cast<uint2*>(as + r * ls + 4 * k) = make_uint2(pack_bf16x2(f.x, f.y), pack_bf16x2(f.z, f.w));
     }
   }
   if (blockIdx.x == 0) {  // the first cluster writes the adapter's A operand adn: its slice of rows 0-31, zero rows 32-63
