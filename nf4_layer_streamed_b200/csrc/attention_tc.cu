@@ -5,7 +5,8 @@
 // ("Soup 层流式 NF4 训练实测：在 4 GB 显存上以位级一致标准完成 8B 模型 LoRA 微调"
 // §2.1: the HF Llama layer body; the workloads' seq 512).
 //
-// One CTA per (128-query tile, query head, sequence), two CTAs per SM: 96 KB of shared
+// One CTA per (128-query tile, query head, sequence; the query tile is the grid's slowest
+// dimension, longest rows first), two CTAs per SM: 96 KB of shared
 // memory (the Q tile and one K and one V tile, a 32 KB slot each, the first half of which
 // a head_dim-64 tile uses) and 256 TMEM columns each, so that one
 // CTA's softmax runs while the other's products keep the tensor core busy.  Per key
@@ -698,7 +699,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
   uint64_t* drain = bars + 10;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  uint64_t* peer_full = bars + 12;  // (first CTA) the second CTA's partial sums have landed
+  uint64_t* peer_full = bars + 12;  // the peer CTA's partial sums of this CTA's tensor have landed
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kvh = blockIdx.x >> 1, b = blockIdx.y, kt = blockIdx.z;  // z slowest: the longest key tiles first
