@@ -54,6 +54,7 @@ constexpr int NUM_DECODERS = 256;
 struct GemmParams {
   CUtensorMap tmA, tmAx, tmB, tmBx;
   CUtensorMap tmC[4];
+  CUtensorMap tmAux;  // CTA-pair residual / dSwiGLU side input (x, or [g | u]), box 64 cols x 128 rows
   int M, N, K, num_kb, has_extra, n_mt;
   int n_seg, swiglu, dense_swiglu_rows;
   int seg_start[5];
@@ -75,6 +76,7 @@ struct GemmParams {
   float* out_f32;
   const float* alpha;
   int accumulate;
+  int aux_tma;  // CTA-pair residual / dSwiGLU epilogue: the side input arrives by TMA in the freed stage memory
   int half;   // CTA-pair kernel: 256-token pair tiles (one 128-row accumulator per CTA)
   int tile0;  // CTA-pair kernel: tile index of the launch's first pair (mt fastest)
   float nf4[16];
@@ -386,6 +388,76 @@ __device__ __forceinline__ void epilogue_rows(const GemmParams& p, uint32_t tmem
   }
 }
 
+// The CTA-pair kernel's residual and dSwiGLU epilogues with their side input staged by
+// TMA: once the accumulators are complete the pipeline's shared memory is free, and per
+// 128-row accumulator one thread loads that accumulator's rows of the tile's side input
+// (the residual x, or g and u: 4 or 4 + 4 boxes of 128 rows x 64 columns, 64 or 128 KB)
+// into it; the epilogue warps then read their rows' 16-column chunks from there instead
+// of one global load per chunk in flight.  Before the second accumulator's loads reuse
+// the memory, every epilogue warp has arrived on aux_free after its last read of the
+// first.  Same items, order and arithmetic as epilogue_rows' residual and dSwiGLU
+// branches, so the results are identical.  issuer: the thread that issues the loads.
+template <int n_acc>
+__device__ __forceinline__ void epilogue_side_tma(const GemmParams& p, uint32_t tmem, int m0, int nt, int q, int lane,
+                                                  int part, int nparts, uint8_t* stage_mem, uint64_t* aux_full,
+                                                  uint64_t* aux_free, volatile int* abort_flag, bool issuer) {
+  constexpr int CW = 16, BOX = 128 * 64 * 2;  // one box: 16 KB
+  const bool dsw = p.epi == EPI_DSWIGLU;
+  const int nch = min(BN, p.N - nt * BN) / CW;
+  const uint32_t sm = smem_u32(stage_mem);
+  int issued = 0;
+  for (int a = 0; a < n_acc; ++a) {
+    if (issuer) {
+      // the first accumulator's rows are read by every epilogue warp before the memory is reused
+      bool ok = a == 0 || mbar_wait(aux_free, (uint32_t)(a - 1) & 1, abort_flag, p.err, KID_GEMM, 16);
+      if (ok) {
+        mbar_arrive_expect_tx(&aux_full[a], (dsw ? 8 : 4) * BOX);
+        for (int j = 0; j < 4; ++j) {
+          tma_load_2d(stage_mem + j * BOX, &p.tmAux, &aux_full[a], nt * BN + 64 * j, m0 + a * 128);
+          if (dsw)
+            tma_load_2d(stage_mem + (4 + j) * BOX, &p.tmAux, &aux_full[a], p.inter + nt * BN + 64 * j, m0 + a * 128);
+        }
+        issued = a + 1;
+      }
+    }
+    const bool have = __all_sync(0xffffffffu, mbar_wait(&aux_full[a], 0, abort_flag, p.err, KID_GEMM, 17));
+    const int r = q * 32 + lane, m = m0 + a * 128 + r;
+    for (int c = 0; c < nch; ++c) {
+      if (((a * nch + c) % nparts) != part) continue;
+      float v[CW];
+      ld_acc16(tmem + ((uint32_t)(q * 32) << 16) + a * 256 + c * CW, v);
+      if (!have || m >= p.M) continue;
+      const uint32_t row = sm + (uint32_t)(c >> 2) * BOX + (uint32_t)r * 128;
+      const uint32_t o0 = (uint32_t)(((c & 3) * 2) ^ (r & 7)) << 4, o1 = (uint32_t)(((c & 3) * 2 + 1) ^ (r & 7)) << 4;
+      float g[CW];
+      unpack16(ld_shared_v4(row + o0), ld_shared_v4(row + o1), g);
+      const int col = nt * BN + c * CW;
+      if (!dsw) {
+#pragma unroll
+        for (int i = 0; i < CW; ++i) v[i] += g[i];
+        store16(p.out + (size_t)m * p.ldo + col, v);
+      } else {
+        float u[CW], du[CW];
+        unpack16(ld_shared_v4(row + 4 * BOX + o0), ld_shared_v4(row + 4 * BOX + o1), u);
+#pragma unroll
+        for (int i = 0; i < CW; ++i) {
+          const float sg = sigmoid_f(g[i]);
+          du[i] = v[i] * g[i] * sg;
+          v[i] = v[i] * u[i] * sg * (1.0f + g[i] * (1.0f - sg));
+        }
+        store16(p.out + (size_t)m * p.ldo + col, v);
+        store16(p.out + (size_t)m * p.ldo + p.inter + col, du);
+      }
+    }
+    if (a + 1 < n_acc) {  // this warp is done with the staged rows
+      __syncwarp();
+      if (lane == 0) mbar_arrive(aux_free);
+    }
+  }
+  if (issuer && *abort_flag)  // let the loads already issued land before the CTA exits
+    for (int a = 0; a < issued; ++a) mbar_wait_drain(&aux_full[a], 0);
+}
+
 // ------------------------------------------------------------------------------ kernel
 template <bool DECODE, bool BMN>
 __global__ void __launch_bounds__(DECODE ? 448 : 192, 1) k_gemm(const __grid_constant__ GemmParams p) {
@@ -665,6 +737,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DECODE ? 448 : 192, 
   uint64_t* accum_full = codes_full + P_STAGES;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint64_t* aux_full = reinterpret_cast<uint64_t*>(misc + 112);  // 2: a side-input stage has landed
+  uint64_t* aux_free = reinterpret_cast<uint64_t*>(misc + 128);  // the epilogue warps are done with it
   float* code8_s = reinterpret_cast<float*>(misc + 256);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -681,6 +755,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DECODE ? 448 : 192, 
       mbar_init(&codes_full[s], 1);
     }
     mbar_init(accum_full, 1);
+    mbar_init(&aux_full[0], 1);
+    mbar_init(&aux_full[1], 1);
+    mbar_init(aux_free, DECODE ? 12 : 4);  // the epilogue warps
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -692,6 +769,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DECODE ? 448 : 192, 
       tma_prefetch_desc(&p.tmBx);
     }
     if (!DECODE) tma_prefetch_desc(&p.tmB);
+    if (p.aux_tma) tma_prefetch_desc(&p.tmAux);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, 512);
@@ -804,7 +882,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DECODE ? 448 : 192, 
     prefetch_aux(p, m0, nt, threadIdx.x - 64, 128, 128 * NACC);
     if (mbar_wait(accum_full, 0, abort_flag, p.err, KID_GEMM, 13)) {
       tc_fence_after();
-      epilogue_rows<NACC, !DECODE>(p, tmem, m0, nt, q, lane, 0, DECODE ? 3 : 1);
+      if (p.aux_tma)
+        epilogue_side_tma<NACC>(p, tmem, m0, nt, q, lane, 0, DECODE ? 3 : 1, base, aux_full, aux_free, abort_flag,
+                                   threadIdx.x == 64);
+      else
+        epilogue_rows<NACC, !DECODE>(p, tmem, m0, nt, q, lane, 0, DECODE ? 3 : 1);
     }
   } else if (DECODE) {
     // ---------------------------------------------------------------- NF4 decoders (both CTAs)
@@ -890,7 +972,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DECODE ? 448 : 192, 
     // then share the epilogue: 3 warps per TMEM lane quarter
     if (mbar_wait(accum_full, 0, abort_flag, p.err, KID_GEMM, 15)) {
       tc_fence_after();
-      epilogue_rows<NACC, !DECODE>(p, tmem, m0, nt, warp & 3, lane, (warp - 2) / 4, 3);
+      if (p.aux_tma)
+        epilogue_side_tma<NACC>(p, tmem, m0, nt, warp & 3, lane, (warp - 2) / 4, 3, base, aux_full, aux_free,
+                                   abort_flag, false);
+      else
+        epilogue_rows<NACC, !DECODE>(p, tmem, m0, nt, warp & 3, lane, (warp - 2) / 4, 3);
     }
   }
 
@@ -1141,6 +1227,17 @@ int gemm(const __nv_bfloat16* A, int lda, int M, int N, int K, const GemmWeights
   p.out_f32 = epi.out_f32;
   p.alpha = epi.alpha;
   p.accumulate = epi.accumulate;
+  // CTA pairs: the residual x or the dSwiGLU side input [g | u] by TMA (16-byte rows and
+  // column offsets)
+  p.aux_tma = 0;
+  const bool dsw = epi.kind == EPI_DSWIGLU;
+  const int64_t side_cols = dsw ? (int64_t)2 * epi.inter : N;
+  if (pair && (dsw || epi.kind == EPI_RESID) && epi.aux0 && aligned(epi.aux0, 16) && epi.ld_aux0 % 8 == 0 &&
+      (!dsw || epi.inter % 8 == 0) && epi.ld_aux0 >= side_cols) {
+    NF4_TRY(make_map(&p.tmAux, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, epi.aux0, (uint64_t)side_cols, M,
+                     (uint64_t)epi.ld_aux0 * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B));
+    p.aux_tma = 1;
+  }
   if (epi.kind == EPI_ACC_F32 && (epi.ldo % 4 || !aligned(epi.out_f32, 16)))
     return fail(NF4LS_ALIGN, "gemm: fp32 output needs 16-byte rows");
   p.err = device_error_ptr();
