@@ -54,7 +54,8 @@ constexpr int NUM_DECODERS = 256;
 struct GemmParams {
   CUtensorMap tmA, tmAx, tmB, tmBx;
   CUtensorMap tmC[4];
-  CUtensorMap tmAux;  // CTA-pair residual / dSwiGLU side input (x, or [g | u]), box 64 cols x 128 rows
+  CUtensorMap tmAux;   // CTA-pair residual / dSwiGLU side input (x, or [g | u]), box 64 cols x 128 rows;
+  CUtensorMap tmAux2;  //   RoPE: the cos (tmAux) and sin (tmAux2) tables [d/2, seq], box 128 positions
   int M, N, K, num_kb, has_extra, n_mt;
   int n_seg, swiglu, dense_swiglu_rows;
   int seg_start[5];
@@ -76,7 +77,7 @@ struct GemmParams {
   float* out_f32;
   const float* alpha;
   int accumulate;
-  int aux_tma;  // CTA-pair residual / dSwiGLU epilogue: the side input arrives by TMA in the freed stage memory
+  int aux_tma;  // CTA-pair epilogue: 1 = residual / dSwiGLU side input, 2 = RoPE tables, by TMA into the freed stage memory
   int half;   // CTA-pair kernel: 256-token pair tiles (one 128-row accumulator per CTA)
   int tile0;  // CTA-pair kernel: tile index of the launch's first pair (mt fastest)
   float nf4[16];
@@ -458,6 +459,80 @@ __device__ __forceinline__ void epilogue_side_tma(const GemmParams& p, uint32_t 
     for (int a = 0; a < issued; ++a) mbar_wait_drain(&aux_full[a], 0);
 }
 
+// The CTA-pair kernel's RoPE epilogue with the cos and sin of its rows staged by TMA: per
+// 128-row accumulator (128 consecutive positions, seq a multiple of 128) one thread loads
+// both tables' [d/2 frequencies x 128 positions] blocks into the freed pipeline memory,
+// and each thread reads its row's angles from there (consecutive lanes, consecutive
+// words) instead of 32 global loads per 16-column chunk.  Same items, order and
+// arithmetic as epilogue_rows' RoPE branch, so the results are identical.
+template <int n_acc>
+__device__ __forceinline__ void epilogue_rope_tma(const GemmParams& p, uint32_t tmem, int m0, int nt, int q, int lane,
+                                                  int part, int nparts, uint8_t* stage_mem, uint64_t* aux_full,
+                                                  uint64_t* aux_free, volatile int* abort_flag, bool issuer) {
+  constexpr int CW = 16;
+  const int d = p.head_dim, half = d / 2;
+  const uint32_t tab_bytes = (uint32_t)half * 128 * 4;
+  const float* cos_s = reinterpret_cast<const float*>(stage_mem);
+  const float* sin_s = cos_s + half * 128;
+  int issued = 0, item = 0;
+  for (int a = 0; a < n_acc; ++a) {
+    if (issuer) {
+      // the first accumulator's angles are read by every epilogue warp before the memory is reused
+      bool ok = a == 0 || mbar_wait(aux_free, (uint32_t)(a - 1) & 1, abort_flag, p.err, KID_GEMM, 18);
+      if (ok) {
+        const int pos0 = (m0 + a * 128) % p.seq;
+        mbar_arrive_expect_tx(&aux_full[a], 2 * tab_bytes);
+        tma_load_2d(stage_mem, &p.tmAux, &aux_full[a], pos0, 0);
+        tma_load_2d(stage_mem + tab_bytes, &p.tmAux2, &aux_full[a], pos0, 0);
+        issued = a + 1;
+      }
+    }
+    const bool have = __all_sync(0xffffffffu, mbar_wait(&aux_full[a], 0, abort_flag, p.err, KID_GEMM, 19));
+    const int r = q * 32 + lane, m = m0 + a * 128 + r;
+    const bool mv = m < p.M;
+    const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + a * 256;
+    float v[CW], w[CW];
+    for (int h = 0; h < BN / d; ++h) {
+      const int hc = nt * BN + h * d;
+      if (hc >= p.N) break;
+      if (hc < p.rope_cols) {
+        for (int i = 0; i < half / CW; ++i) {
+          if ((item++ % nparts) != part) continue;
+          ld_acc16(tb + h * d + i * CW, v);
+          ld_acc16(tb + h * d + half + i * CW, w);
+          if (!mv || !have) continue;
+          float c_[CW], s_[CW];
+#pragma unroll
+          for (int j = 0; j < CW; ++j) {
+            c_[j] = cos_s[(i * CW + j) * 128 + r];
+            s_[j] = sin_s[(i * CW + j) * 128 + r];
+          }
+          float o1[CW], o2[CW];
+#pragma unroll
+          for (int j = 0; j < CW; ++j) {
+            o1[j] = v[j] * c_[j] - w[j] * s_[j];
+            o2[j] = w[j] * c_[j] + v[j] * s_[j];
+          }
+          store16(p.out + (size_t)m * p.ldo + hc + i * CW, o1);
+          store16(p.out + (size_t)m * p.ldo + hc + half + i * CW, o2);
+        }
+      } else {
+        for (int c = 0; c < d / CW; ++c) {
+          if ((item++ % nparts) != part) continue;
+          ld_acc16(tb + h * d + c * CW, v);
+          if (mv) store16(p.out + (size_t)m * p.ldo + hc + c * CW, v);
+        }
+      }
+    }
+    if (a + 1 < n_acc) {  // this warp is done with the staged angles
+      __syncwarp();
+      if (lane == 0) mbar_arrive(aux_free);
+    }
+  }
+  if (issuer && *abort_flag)  // let the loads already issued land before the CTA exits
+    for (int a = 0; a < issued; ++a) mbar_wait_drain(&aux_full[a], 0);
+}
+
 // ------------------------------------------------------------------------------ kernel
 template <bool DECODE, bool BMN>
 __global__ void __launch_bounds__(DECODE ? 448 : 192, 1) k_gemm(const __grid_constant__ GemmParams p) {
@@ -770,6 +845,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DECODE ? 448 : 192, 
     }
     if (!DECODE) tma_prefetch_desc(&p.tmB);
     if (p.aux_tma) tma_prefetch_desc(&p.tmAux);
+    if (p.aux_tma == 2) tma_prefetch_desc(&p.tmAux2);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, 512);
@@ -882,9 +958,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DECODE ? 448 : 192, 
     prefetch_aux(p, m0, nt, threadIdx.x - 64, 128, 128 * NACC);
     if (mbar_wait(accum_full, 0, abort_flag, p.err, KID_GEMM, 13)) {
       tc_fence_after();
-      if (p.aux_tma)
+      if (p.aux_tma == 1)
         epilogue_side_tma<NACC>(p, tmem, m0, nt, q, lane, 0, DECODE ? 3 : 1, base, aux_full, aux_free, abort_flag,
                                    threadIdx.x == 64);
+      else if (p.aux_tma == 2)
+        epilogue_rope_tma<NACC>(p, tmem, m0, nt, q, lane, 0, DECODE ? 3 : 1, base, aux_full, aux_free, abort_flag,
+                                threadIdx.x == 64);
       else
         epilogue_rows<NACC, !DECODE>(p, tmem, m0, nt, q, lane, 0, DECODE ? 3 : 1);
     }
@@ -972,9 +1051,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DECODE ? 448 : 192, 
     // then share the epilogue: 3 warps per TMEM lane quarter
     if (mbar_wait(accum_full, 0, abort_flag, p.err, KID_GEMM, 15)) {
       tc_fence_after();
-      if (p.aux_tma)
+      if (p.aux_tma == 1)
         epilogue_side_tma<NACC>(p, tmem, m0, nt, warp & 3, lane, (warp - 2) / 4, 3, base, aux_full, aux_free,
                                    abort_flag, false);
+      else if (p.aux_tma == 2)
+        epilogue_rope_tma<NACC>(p, tmem, m0, nt, warp & 3, lane, (warp - 2) / 4, 3, base, aux_full, aux_free,
+                                abort_flag, false);
       else
         epilogue_rows<NACC, !DECODE>(p, tmem, m0, nt, warp & 3, lane, (warp - 2) / 4, 3);
     }
@@ -1237,6 +1319,17 @@ int gemm(const __nv_bfloat16* A, int lda, int M, int N, int K, const GemmWeights
     NF4_TRY(make_map(&p.tmAux, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, epi.aux0, (uint64_t)side_cols, M,
                      (uint64_t)epi.ld_aux0 * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B));
     p.aux_tma = 1;
+  }
+  // CTA pairs, RoPE: the angle tables [d/2, seq] by TMA, 128 positions per box (an
+  // accumulator's rows are 128 consecutive positions when seq is a multiple of 128)
+  if (pair && epi.kind == EPI_ROPE && epi.seq % 128 == 0 && epi.head_dim % 32 == 0 && aligned(epi.rope_cos, 16) &&
+      aligned(epi.rope_sin, 16)) {
+    const int half = epi.head_dim / 2;
+    NF4_TRY(make_map(&p.tmAux, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, epi.rope_cos, epi.seq, half, (uint64_t)epi.seq * 4,
+                     128, half, CU_TENSOR_MAP_SWIZZLE_NONE));
+    NF4_TRY(make_map(&p.tmAux2, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, epi.rope_sin, epi.seq, half, (uint64_t)epi.seq * 4,
+                     128, half, CU_TENSOR_MAP_SWIZZLE_NONE));
+    p.aux_tma = 2;
   }
   if (epi.kind == EPI_ACC_F32 && (epi.ldo % 4 || !aligned(epi.out_f32, 16)))
     return fail(NF4LS_ALIGN, "gemm: fp32 output needs 16-byte rows");
