@@ -35,7 +35,7 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 # dram__bytes_read.sum + dram__bytes_write.sum per NF4-decode GEMM launch, averaged over
 # the 11 launches of one layer of this workload (one ncu capture of the current kernel;
 # every layer of the step runs the same 11 launches)
-NF4_GEMM_DRAM_BYTES_PER_LAUNCH = 101.7e6
+NF4_GEMM_DRAM_BYTES_PER_LAUNCH = 101.4e6
 
 
 def peaks():
