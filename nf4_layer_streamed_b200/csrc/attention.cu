@@ -515,15 +515,14 @@ int attention_fwd(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfl
 int attention_bwd(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, int ldq, int ldkv,
                   const __nv_bfloat16* o, const __nv_bfloat16* dout, int ldo, const float* lse, float* delta,
                   __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv, int ld_dq, int ld_dkv, int batch, int seq,
-                  int nq, int nkv, int d, const float* rope_cos, const float* rope_sin, cudaStream_t s) {
+                  int nq, int nkv, int d, cudaStream_t s) {
   NF4_TRY(check_attn(seq, nq, nkv, d, ldq, ldkv));
   const int M = batch * seq;
   const float scale = 1.0f / sqrtf((float)d);
   if (attention_tc() && attention_bwd_tc_supported(seq, d, nq, nkv, ldq, ldkv, ldo, ld_dq, ld_dkv))
-    // the tcgen05 query-side kernel forms delta itself; the RoPE transpose is applied in
-    // the dQ and dK epilogues
+    // the tcgen05 query-side kernel forms delta itself
     return attention_bwd_tc(q, k, v, ldq, ldkv, o, dout, ldo, lse, delta, dq, dk, dv, ld_dq, ld_dkv, batch, seq, nq,
-                            nkv, d, rope_cos, rope_sin, s);
+                            nkv, d, s);
   k_attn_delta<<<(M * nq + 7) / 8, 256, 0, s>>>(o, dout, ldo, M, seq, nq, d, delta);
   note_launch();
   dim3 gq(seq / TQ, nq, batch), gk(nkv, batch, seq / TK);
@@ -545,10 +544,6 @@ int attention_bwd(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfl
     note_launch();
   }
   NF4_CUDA_TRY(cudaGetLastError());
-  if (rope_cos) {  // the RoPE transpose as separate passes over dQ and dK
-    NF4_TRY(rope_bwd(dq, ld_dq, M, nq * d, seq, d, rope_cos, rope_sin, s));
-    NF4_TRY(rope_bwd(dk, ld_dkv, M, nkv * d, seq, d, rope_cos, rope_sin, s));
-  }
   return NF4LS_OK;
 }
 
@@ -577,6 +572,6 @@ extern "C" int nf4ls_attention_bwd(const nf4ls_layer_cfg* cfg, const void* q_dev
                               static_cast<const __nv_bfloat16*>(o_dev), static_cast<const __nv_bfloat16*>(do_dev), qd,
                               lse_dev, delta_dev, static_cast<__nv_bfloat16*>(dq_dev),
                               static_cast<__nv_bfloat16*>(dk_dev), static_cast<__nv_bfloat16*>(dv_dev), qd, kvd,
-                              cfg->batch, cfg->seq, cfg->n_q, cfg->n_kv, cfg->head_dim, nullptr, nullptr,
+                              cfg->batch, cfg->seq, cfg->n_q, cfg->n_kv, cfg->head_dim,
                               static_cast<cudaStream_t>(stream));
 }

@@ -67,41 +67,6 @@ __device__ __forceinline__ void stage_row32(uint32_t tile, int r, int c, const f
   stage_row32(tile, r, c, u, 1.0f);
 }
 
-// The transpose of the RoPE rotation, in place on row r of a staged bf16 tile (D columns
-// in 64-column atoms as stage_row32 writes them; the row's position pos): column j pairs
-// with j + D/2 (rope_bwd_pair, then bf16 again, as the standalone RoPE backward kernel
-// does).  The row's D/16 chunks of eight pairs are split over the two threads that share
-// the row: thread half g takes chunks g, g + 2, ...
-template <int D>
-__device__ __forceinline__ void rope_bwd_row(uint32_t tile, int r, int g, int pos, const float* __restrict__ cos_t,
-                                             const float* __restrict__ sin_t) {
-  constexpr int HALF = D / 2;
-#pragma unroll
-  for (int k = g; k < HALF / 8; k += 2) {
-    const int j0 = 8 * k, j1 = j0 + HALF;
-    const uint32_t aa = tile + (uint32_t)(j0 >> 6) * ATOM + (uint32_t)r * 128 + ((uint32_t)(((j0 & 63) >> 3) ^ (r & 7)) << 4);
-    const uint32_t ab = tile + (uint32_t)(j1 >> 6) * ATOM + (uint32_t)r * 128 + ((uint32_t)(((j1 & 63) >> 3) ^ (r & 7)) << 4);
-    const uint4 ua = ld_shared_v4(aa), ub = ld_shared_v4(ab);
-    const float4* cp = reinterpret_cast<const float4*>(cos_t + (size_t)pos * HALF + j0);
-    const float4* sp = reinterpret_cast<const float4*>(sin_t + (size_t)pos * HALF + j0);
-    const float4 c0 = __ldg(cp), c1 = __ldg(cp + 1), s0 = __ldg(sp), s1 = __ldg(sp + 1);
-    const float c[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-    const float sn[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-    const uint32_t wa[4] = {ua.x, ua.y, ua.z, ua.w}, wb[4] = {ub.x, ub.y, ub.z, ub.w};
-    uint32_t oa[4], ob[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      float a0, a1, b0, b1;
-      rope_bwd_pair(bf16_lo(wa[q]), bf16_lo(wb[q]), c[2 * q], sn[2 * q], a0, b0);
-      rope_bwd_pair(bf16_hi(wa[q]), bf16_hi(wb[q]), c[2 * q + 1], sn[2 * q + 1], a1, b1);
-      oa[q] = pack_bf16x2(a0, a1);
-      ob[q] = pack_bf16x2(b0, b1);
-    }
-    st_shared_v4(aa, oa[0], oa[1], oa[2], oa[3]);
-    st_shared_v4(ab, ob[0], ob[1], ob[2], ob[3]);
-  }
-}
-
 struct AttnTcParams {
   CUtensorMap tq, tk, tv, to;  // [rows, cols] bf16, box 64 cols x 128 rows, 128-byte swizzle (to: output)
   __nv_bfloat16* o;
@@ -414,8 +379,6 @@ __global__ void __launch_bounds__(F_THREADS, 2) k_attn_fwd_tc(const __grid_const
 struct AttnBwdParams {
   CUtensorMap tq, tk, tv, tdo, to;  // box 64 cols x 128 rows, 128-byte swizzle (to: the output O)
   CUtensorMap tdq, tdk, tdv;        // the gradients, same boxes (TMA stores)
-  const float* rope_cos;            // [seq, d/2] cos, sin of the RoPE angles: dQ and dK leave
-  const float* rope_sin;            //   through the rotation's transpose (null: as they are)
   const float* lse;
   float* delta;                 // written by the query side, read by the key side
   __nv_bfloat16* dq;
@@ -675,10 +638,6 @@ __global__ void __launch_bounds__(B_THREADS, 1) k_attn_dq_tc(const __grid_consta
       const uint32_t tile = smem_u32(base + B_OFF_RING);
 #pragma unroll
       for (int i = 0; i < DH / 32; ++i) stage_row32(tile, r, g * (DH / 32) + i, v[i], p.scale);
-    }
-    if (p.rope_cos) {  // the pair's other half was staged by the row's other thread
-      bar_ew();
-      rope_bwd_row<D>(smem_u32(base + B_OFF_RING), r, g, qt * TT + r, p.rope_cos, p.rope_sin);
     }
     fence_proxy_async_smem();
     bar_ew();
@@ -961,10 +920,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(B_THREADS, 1)
       }
       stage_row32(tile, r, g * (DH / 32) + c, v);
     }
-    if (crank == 1 && p.rope_cos) {  // dK: the pair's other half was staged by the row's other thread
-      bar_ew();
-      rope_bwd_row<D>(tile, r, g, kt * TT + r, p.rope_cos, p.rope_sin);
-    }
     fence_proxy_async_smem();
     bar_ew();
     if (threadIdx.x == 0 && !*abort_flag) {
@@ -1070,7 +1025,7 @@ int launch_bwd_tc(const AttnBwdParams& p, int batch, int seq, int nq, int nkv, c
 int attention_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, int ldq, int ldkv,
                      const __nv_bfloat16* o, const __nv_bfloat16* dout, int ldo, const float* lse, float* delta,
                      __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv, int ld_dq, int ld_dkv, int batch, int seq,
-                     int nq, int nkv, int d, const float* rope_cos, const float* rope_sin, cudaStream_t s) {
+                     int nq, int nkv, int d, cudaStream_t s) {
   static_assert(SMEM_BWD <= 232448, "shared memory of the tcgen05 attention backward");
   AttnBwdParams p;
   const uint64_t rows = (uint64_t)batch * seq;
@@ -1083,10 +1038,6 @@ int attention_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_
   NF4_TRY(tma_map_bf16(&p.tdq, dq, (uint64_t)nq * d, rows, (uint64_t)ld_dq * 2, 64, TT));
   NF4_TRY(tma_map_bf16(&p.tdk, dk, (uint64_t)nkv * d, rows, (uint64_t)ld_dkv * 2, 64, TT));
   NF4_TRY(tma_map_bf16(&p.tdv, dv, (uint64_t)nkv * d, rows, (uint64_t)ld_dkv * 2, 64, TT));
-  if ((rope_cos || rope_sin) && (!rope_cos || !rope_sin || !aligned(rope_cos, 16) || !aligned(rope_sin, 16)))
-    return fail(NF4LS_ALIGN, "attention backward: RoPE tables (both, 16-byte aligned)");
-  p.rope_cos = rope_cos;
-  p.rope_sin = rope_sin;
   p.lse = lse;
   p.delta = delta;
   p.dq = dq;

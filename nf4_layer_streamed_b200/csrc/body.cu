@@ -460,10 +460,8 @@ __global__ void k_rope_bwd(__nv_bfloat16* __restrict__ x, int ld, int M, int col
   __nv_bfloat16* p = x + (size_t)m * ld + head * d;
   const float c = cos_t[pos * half + j], s = sin_t[pos * half + j];
   const float a = __bfloat162float(p[j]), b = __bfloat162float(p[j + half]);
-  float o1, o2;
-  rope_bwd_pair(a, b, c, s, o1, o2);
-  p[j] = __float2bfloat16_rn(o1);
-  p[j + half] = __float2bfloat16_rn(o2);
+  p[j] = __float2bfloat16_rn(a * c + b * s);
+  p[j + half] = __float2bfloat16_rn(b * c - a * s);
 }
 
 // The same, eight frequencies per thread: one 16-byte load and store of each half and
@@ -487,7 +485,10 @@ __global__ void k_rope_bwd8(__nv_bfloat16* __restrict__ x, int ld, int cols, int
   unpack8(*reinterpret_cast<const uint4*>(p), a);
   unpack8(*reinterpret_cast<const uint4*>(p + half), b);
 #pragma unroll
-  for (int j = 0; j < 8; ++j) rope_bwd_pair(a[j], b[j], c[j], sn[j], o1[j], o2[j]);
+  for (int j = 0; j < 8; ++j) {
+    o1[j] = a[j] * c[j] + b[j] * sn[j];
+    o2[j] = b[j] * c[j] - a[j] * sn[j];
+  }
   *reinterpret_cast<uint4*>(p) = pack8(o1);
   *reinterpret_cast<uint4*>(p + half) = pack8(o2);
 }

@@ -118,15 +118,6 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) 
   return true;
 }
 
-// The transpose of the RoPE rotation of the pair (a, b) (columns j and j + d/2 of a head)
-// at the angle with cosine c and sine s: (a c + b s, b c - a s), each product and each
-// sum rounded on its own (no contraction), so that every kernel applying it gives the
-// same bits.
-__device__ __forceinline__ void rope_bwd_pair(float a, float b, float c, float s, float& o1, float& o2) {
-  o1 = __fadd_rn(__fmul_rn(a, c), __fmul_rn(b, s));
-  o2 = __fsub_rn(__fmul_rn(b, c), __fmul_rn(a, s));
-}
-
 // ----------------------------------------------------------------------------- TMA
 // Tiled 2D load of a box into shared memory, completing transaction bytes on bar.
 // c0 is the innermost coordinate (elements); c0 * element size must be a multiple of 16.

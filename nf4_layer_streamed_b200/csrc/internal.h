@@ -268,17 +268,14 @@ int attention_fwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_
 int attention_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, int ldq, int ldkv,
                      const __nv_bfloat16* o, const __nv_bfloat16* dout, int ldo, const float* lse, float* delta,
                      __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv, int ld_dq, int ld_dkv, int batch, int seq,
-                     int nq, int nkv, int d, const float* rope_cos, const float* rope_sin, cudaStream_t s);
+                     int nq, int nkv, int d, cudaStream_t s);
 int attention_fwd(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, int ldq, int ldkv,
                   __nv_bfloat16* o, int ldo, float* lse, int batch, int seq, int nq, int nkv, int d,
                   cudaStream_t s);
-// rope_cos, rope_sin ([seq, d/2] RoPE angle tables, or both null): dq and dk come out
-// through the transpose of the RoPE rotation (the gradients of the q and k before the
-// rotation), bit-equal to rope_bwd applied after the attention backward.
 int attention_bwd(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, int ldq, int ldkv,
                   const __nv_bfloat16* o, const __nv_bfloat16* dout, int ldo, const float* lse, float* delta,
                   __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv, int ld_dq, int ld_dkv, int batch,
-                  int seq, int nq, int nkv, int d, const float* rope_cos, const float* rope_sin, cudaStream_t s);
+                  int seq, int nq, int nkv, int d, cudaStream_t s);
 
 // LoRA backward (lora.cu); the forward's t comes from rmsnorm_lora_fwd (body.cu).
 // dB_q, dB_v, dA_q, dA_v (fp32, written) and dt into dtpad [M, 64] (bf16, zeros in

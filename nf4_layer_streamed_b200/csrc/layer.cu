@@ -282,10 +282,10 @@ int layer_bwd_impl(const nf4ls_layer_cfg* c, const void* shard, const nf4ls_lora
   e3.out = dO;
   e3.ldo = x.qd;
   NF4_TRY(gemm(dh, H, M, x.qd, H, x.w_o, true, GemmExtra(), e3, s));
-  // dq, dk with the RoPE transpose applied (in the tcgen05 kernels' epilogues)
   NF4_TRY(attention_bwd(qkv, qkv + x.qd, qkv + x.qd + x.kvd, x.nqkv, x.nqkv, o, dO, x.qd, at<float>(ws, x.L.lse),
                         at<float>(ws, x.L.delta), dqkv, dqkv + x.qd, dqkv + x.qd + x.kvd, x.nqkv, x.nqkv, c->batch, c->seq,
-                        c->n_q, c->n_kv, c->head_dim, at<float>(ws, x.L.cos), at<float>(ws, x.L.sin), s));
+                        c->n_q, c->n_kv, c->head_dim, s));
+  NF4_TRY(rope_bwd(dqkv, x.nqkv, M, x.qd + x.kvd, c->seq, c->head_dim, at<float>(ws, x.L.cos), at<float>(ws, x.L.sin), s));
   GemmExtra ex;
   SideStream side;
   auto lora_phases = [&](int phases, cudaStream_t st) {
