@@ -34,17 +34,6 @@ constexpr int TT = 128;                   // query / key tile
 constexpr int TILE_BYTES = TT * 128 * 2;  // 128 rows x 128 dims bf16 = 32 KB
 constexpr int ATOM = TILE_BYTES / 2;      // one 64-dim (or 64-key) swizzle atom: 16 KB
 
-// Tiled 2D store of a box from shared memory (the map's 128-byte swizzled layout) to
-// global memory, in this thread's bulk async-group.  c0 * 2 bytes is a multiple of 16.
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) {
-  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map), "r"(src),
-               "r"(c0), "r"(c1)
-               : "memory");
-}
-// Closes this thread's bulk async-group and waits until its stores have read shared memory.
-__device__ __forceinline__ void tma_store_drain() {
-  asm volatile("cp.async.bulk.commit_group;\ncp.async.bulk.wait_group.read 0;" ::: "memory");
-}
 // One thread's 32 fp32 values (columns 32 c .. 32 c + 31 of its row r of a 128 x 128 tile),
 // times sc, as bf16 into the tile's two 128-byte swizzled 64-column atoms at tile.
 __device__ __forceinline__ void stage_row32(uint32_t tile, int r, int c, const uint32_t (&v)[32], float sc) {
