@@ -330,11 +330,16 @@ int adamw(float* p, const float* g, float* m, float* v, size_t n, int step, floa
 // ----------------------------------------------------------------------------- layer
 // tables_ready: the RoPE tables of the workspace are already those of cfg (a model pass
 // writes them at its first layer and the other layers of the pass reuse them).
+// keep (forward): also keep g and u, so that the workspace holds everything the layer's
+// backward would recompute.  recompute (backward): false when the workspace still holds
+// this layer's forward with keep (the last layer of a model step, whose backward follows
+// its forward with nothing else in the workspace between); the results are the same.
 int layer_fwd_impl(const nf4ls_layer_cfg* cfg, const void* shard, const nf4ls_lora* lora, const __nv_bfloat16* x,
-                   __nv_bfloat16* y, void* ws, size_t ws_bytes, cudaStream_t s, bool tables_ready = false);
+                   __nv_bfloat16* y, void* ws, size_t ws_bytes, cudaStream_t s, bool tables_ready = false,
+                   bool keep = false);
 int layer_bwd_impl(const nf4ls_layer_cfg* cfg, const void* shard, const nf4ls_lora* lora, const __nv_bfloat16* x,
                    const __nv_bfloat16* dy, __nv_bfloat16* dx, const nf4ls_lora_grads* g, void* ws, size_t ws_bytes,
-                   cudaStream_t s, bool tables_ready = false);
+                   cudaStream_t s, bool tables_ready = false, bool recompute = true);
 size_t layer_ws_bytes(const nf4ls_layer_cfg* cfg);
 
 }  // namespace nf4ls

@@ -233,23 +233,24 @@ int forward_body(LayerCtx& x, const nf4ls_lora* lora, const __nv_bfloat16* X, __
 size_t layer_ws_bytes(const nf4ls_layer_cfg* cfg) { return ws_layout(cfg).total; }
 
 int layer_fwd_impl(const nf4ls_layer_cfg* c, const void* shard, const nf4ls_lora* lora, const __nv_bfloat16* X,
-                   __nv_bfloat16* y, void* ws, size_t ws_bytes, cudaStream_t s, bool tables_ready) {
+                   __nv_bfloat16* y, void* ws, size_t ws_bytes, cudaStream_t s, bool tables_ready, bool keep) {
   if (!X || !y) return fail(NF4LS_INVALID_ARG, "layer_forward: null activation");
   LayerCtx x;
   NF4_TRY(prepare(x, c, shard, ws, ws_bytes, s, tables_ready));
-  return forward_body(x, lora, X, y, false, s);
+  return forward_body(x, lora, X, y, keep, s);
 }
 
 int layer_bwd_impl(const nf4ls_layer_cfg* c, const void* shard, const nf4ls_lora* lora, const __nv_bfloat16* X,
                    const __nv_bfloat16* dy, __nv_bfloat16* dx, const nf4ls_lora_grads* g, void* ws, size_t ws_bytes,
-                   cudaStream_t s, bool tables_ready) {
+                   cudaStream_t s, bool tables_ready, bool recompute) {
   if (!X || !dy || !dx) return fail(NF4LS_INVALID_ARG, "layer_backward: null activation");
   if (lora && (!g || !g->dA_q || !g->dB_q || !g->dA_v || !g->dB_v))
     return fail(NF4LS_INVALID_ARG, "layer_backward: LoRA gradients needed when the adapter is on");
   LayerCtx x;
   NF4_TRY(prepare(x, c, shard, ws, ws_bytes, s, tables_ready));
-  // checkpoint recompute (keeps g and u for the SwiGLU backward)
-  NF4_TRY(forward_body(x, lora, X, nullptr, true, s));
+  // checkpoint recompute (keeps g and u for the SwiGLU backward), unless the workspace
+  // still holds this layer's forward with g and u kept
+  if (recompute) NF4_TRY(forward_body(x, lora, X, nullptr, true, s));
   const int M = x.M, H = x.H, I = x.I;
   auto* gu = at<__nv_bfloat16>(ws, x.L.gu);
   auto* dgu = at<__nv_bfloat16>(ws, x.L.dgu);

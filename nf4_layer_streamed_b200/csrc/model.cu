@@ -212,8 +212,10 @@ int forward_to_loss(const nf4ls_model_cfg* c, const nf4ls_model* m, const int32_
     NF4_TRY(layer_pass(c, m, +1, s, [&](int i, const void* shard) {
       nf4ls_lora l;
       lora_views(lc, m->lora_dev + (size_t)i * stride, &l, nullptr, nullptr);
+      // the last layer of a training step keeps its activations: its backward, next in
+      // the workspace after the head, skips the checkpoint recompute
       return layer_fwd_impl(lc, shard, lora_on ? &l : nullptr, xs + (size_t)i * act, xs + (size_t)(i + 1) * act,
-                            at<void>(ws, L.layer), L.total - L.layer, s, i != 0);
+                            at<void>(ws, L.layer), L.total - L.layer, s, i != 0, need_grad && i == c->n_layers - 1);
     }));
   }
   Phase head(s, 2001);
@@ -290,7 +292,7 @@ extern "C" int nf4ls_forward_backward(const nf4ls_model_cfg* cfg, const nf4ls_mo
     nf4ls_lora_grads g;
     lora_views(lc, m->lora_dev + (size_t)i * stride, &l, &g, m->grads_dev + (size_t)i * stride);
     return layer_bwd_impl(lc, shard, &l, xs + (size_t)i * act, dh, dh, &g, at<void>(ws, L.layer), L.total - L.layer,
-                          s, i != cfg->n_layers - 1);
+                          s, i != cfg->n_layers - 1, i != cfg->n_layers - 1);
   });
 }
 
