@@ -5,17 +5,20 @@
 // §2.2 check 2 (LoRA gradients nonzero in every layer): the adapter adds
 // s (x A^T) B^T to the q and v projections (s = alpha / r) and trains A and B.  The
 // up-projection is folded into the q/k/v GEMM as an extra 64-wide reduction block;
-// this file holds the skinny products of the backward, all of them HBM-bound, in three
+// this file holds the skinny products of the backward, all of them HBM-bound, in four
 // launches (the down-projection t = [h1 A_q^T | h1 A_v^T] of the forward is a second
 // output of the input RMSNorm's launch, body.cu):
 //
 //   k_lora_bwd_partial: per (128-row block, column chunk of dq or dv) the partial sums
 //     of dB = s dX^T t (over the rows) and of dt = s dX B (over the columns), from one
 //     read of dX;
-//   k_lora_bwd_reduce: dB (partials added in row-block order) and dt (partials added
-//     in column-chunk order, rounded to bf16: the extra operand of the dL/dx GEMM);
+//   k_lora_bwd_reduce, launched twice: dt (partials added in column-chunk order,
+//     rounded to bf16: the extra operand of the dL/dx GEMM), then dB (partials added in
+//     row-block order);
 //   k_lora_bwd_da: dA = dt^T h1, a cluster of eight blocks per 64 columns of h1, each
 //     over an eighth of the rows, the partials added across the cluster in shared memory.
+// The layer's backward runs the last two (dB and dA, which nothing in the layer waits
+// for) on a side stream beside the q/k/v dL/dx GEMM.
 //
 // The products run on the warp-level bf16 tensor-core instruction (mma.sync m16n8k16);
 // every reduction is in a fixed order, so each result is bit-reproducible and a
